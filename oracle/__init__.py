@@ -1,0 +1,177 @@
+"""CPU oracle for the int8 dynamic-quantization linear layer (numpy front end).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference leg of ``bench.py`` may import this package.  The
+product path (``quantized_gemm_token_b200``) never does, and this package
+never imports the product.
+
+The arithmetic lives in ``dq_oracle.c`` (plain single-threaded C); this
+module only marshals numpy arrays.  bf16 tensors are carried as their uint16
+bit patterns.
+
+What each routine follows (page titles and parts):
+  * quantize_rows_bf16 / quantize_rows_f32 -- per-token (per-row) absmax int8
+    dynamic quantization: "int8 dynamic quant + bsr support" (pytorch/ao PR
+    821, description); absmax/127 symmetric scale: "sparse_fc supported"
+    (PaddlePaddle PR 41770, SpmmPluginDynamic constructor).  Scale
+    s = max(absmax, 1e-8f)/127 in fp32, q = clamp(rint(x/s), -127, 127), ties
+    to even.
+  * gemm_s32 / gemm_s64 -- int8 x int8 -> int32 (PR 821 review: the dot
+    accumulator is int32; overflow bound 2^31/2^14).
+  * epilogue_bf16 -- out = bf16(acc * s_row * s_col + bias) (PR 821: i8i8->bf16
+    keeps accuracy).
+  * bsr_gemm_s32 / bsr_pack / bsr_densify -- 64x64 BSR weight given as
+    crow_indices / col_indices / values (PR 821 description; --bsr 64).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I = ctypes.c_int64
+        lib.oracle_quantize_rows_bf16.argtypes = [P, I, I, I, P, I, P]
+        lib.oracle_quantize_rows_bf16.restype = ctypes.c_int
+        lib.oracle_quantize_rows_f32.argtypes = [P, I, I, I, P, I, P]
+        lib.oracle_quantize_rows_f32.restype = ctypes.c_int
+        lib.oracle_gemm_s32.argtypes = [P, I, I, I, P, I, I, P]
+        lib.oracle_gemm_s64.argtypes = [P, I, I, I, P, I, I, P]
+        lib.oracle_epilogue_bf16.argtypes = [P, I, I, P, P, P, P]
+        lib.oracle_bsr_gemm_s32.argtypes = [P, I, I, I, I, P, P, P, I, P]
+        lib.oracle_bsr_pack.argtypes = [P, I, I, P, P, I, P]
+        lib.oracle_bsr_densify.argtypes = [I, I, P, P, P, I, P]
+        lib.oracle_float_to_bf16.argtypes = [ctypes.c_float]
+        lib.oracle_float_to_bf16.restype = ctypes.c_uint16
+        lib.oracle_bf16_to_float.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_float.restype = ctypes.c_float
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def quantize_rows_bf16(x_bits: np.ndarray):
+    """x_bits: uint16 [M, K] (bf16 patterns) -> (q int8 [M, K], scales fp32 [M])."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), np.int8)
+    s = np.empty((M,), np.float32)
+    rc = _load().oracle_quantize_rows_bf16(_ptr(x), M, K, K, _ptr(q), K, _ptr(s))
+    if rc != 0:
+        raise ValueError("row too long for the oracle")
+    return q, s
+
+
+def quantize_rows_f32(w: np.ndarray):
+    """w: fp32 [N, K] -> (q int8 [N, K], per-row scales fp32 [N])."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    q = np.empty((N, K), np.int8)
+    s = np.empty((N,), np.float32)
+    _load().oracle_quantize_rows_f32(_ptr(w), N, K, K, _ptr(q), K, _ptr(s))
+    return q, s
+
+
+def gemm_s32(A: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """A int8 [M, K], W int8 [N, K] -> int32 [M, N] = A @ W^T (exact)."""
+    A = _c(A, np.int8)
+    W = _c(W, np.int8)
+    M, K = A.shape
+    N = W.shape[0]
+    assert W.shape[1] == K
+    out = np.empty((M, N), np.int32)
+    _load().oracle_gemm_s32(_ptr(A), M, K, K, _ptr(W), N, K, _ptr(out))
+    return out
+
+
+def gemm_s64(A: np.ndarray, W: np.ndarray) -> np.ndarray:
+    A = _c(A, np.int8)
+    W = _c(W, np.int8)
+    M, K = A.shape
+    N = W.shape[0]
+    out = np.empty((M, N), np.int64)
+    _load().oracle_gemm_s64(_ptr(A), M, K, K, _ptr(W), N, K, _ptr(out))
+    return out
+
+
+def epilogue_bf16(acc, s_row, s_col, bias_bits=None) -> np.ndarray:
+    """acc int32 [M, N] -> bf16 bits uint16 [M, N]."""
+    acc = _c(acc, np.int32)
+    M, N = acc.shape
+    s_row = _c(s_row, np.float32)
+    s_col = _c(s_col, np.float32)
+    out = np.empty((M, N), np.uint16)
+    if bias_bits is not None:
+        bias_bits = _c(bias_bits, np.uint16)
+        bp = _ptr(bias_bits)
+    else:
+        bp = None
+    _load().oracle_epilogue_bf16(_ptr(acc), M, N, _ptr(s_row), _ptr(s_col), bp, _ptr(out))
+    return out
+
+
+def bsr_gemm_s32(A, N, crow, col, values, bs=64) -> np.ndarray:
+    A = _c(A, np.int8)
+    M, K = A.shape
+    crow = _c(crow, np.int32)
+    col = _c(col, np.int32)
+    values = _c(values, np.int8)
+    out = np.empty((M, N), np.int32)
+    _load().oracle_bsr_gemm_s32(_ptr(A), M, K, K, N, _ptr(crow), _ptr(col), _ptr(values),
+                                bs, _ptr(out))
+    return out
+
+
+def bsr_pack(W, crow, col, bs=64) -> np.ndarray:
+    W = _c(W, np.int8)
+    N, K = W.shape
+    crow = _c(crow, np.int32)
+    col = _c(col, np.int32)
+    nnzb = int(crow[-1])
+    values = np.empty((nnzb, bs, bs), np.int8)
+    _load().oracle_bsr_pack(_ptr(W), N, K, _ptr(crow), _ptr(col), bs, _ptr(values))
+    return values
+
+
+def bsr_densify(N, K, crow, col, values, bs=64) -> np.ndarray:
+    crow = _c(crow, np.int32)
+    col = _c(col, np.int32)
+    values = _c(values, np.int8)
+    out = np.empty((N, K), np.int32)
+    _load().oracle_bsr_densify(N, K, _ptr(crow), _ptr(col), _ptr(values), bs, _ptr(out))
+    return out
+
+
+def linear_bf16(q, s_row, Wq, s_col, bias_bits=None):
+    """Composition: exact GEMM then the fp32/bf16 epilogue."""
+    return epilogue_bf16(gemm_s32(q, Wq), s_row, s_col, bias_bits)
+
+
+def dynamic_linear_bf16(x_bits, Wq, s_col, bias_bits=None):
+    """The full layer: per-token quantize, int8 GEMM, fused-epilogue math."""
+    q, s_row = quantize_rows_bf16(x_bits)
+    return linear_bf16(q, s_row, Wq, s_col, bias_bits), q, s_row
+
+
+def float_to_bf16(f: float) -> int:
+    return int(_load().oracle_float_to_bf16(float(f)))
+
+
+def bf16_to_float(h: int) -> float:
+    return float(_load().oracle_bf16_to_float(int(h)))

@@ -1,0 +1,214 @@
+/*
+ * dq_oracle.c -- plain, slow, single-threaded CPU oracle for the int8
+ * dynamic-quantization linear layer (dense and 64x64 block-sparse weight).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the test suite, the smoke check and the CPU-baseline
+ * leg of the benchmark use it.  It shares no code, header, table or helper
+ * with the CUDA library.
+ *
+ * Every routine is the method's definition written out with scalar loops,
+ * in the order the sources state it:
+ *
+ *  - Per-token ("per-row") dynamic absmax quantization of activations to
+ *    int8 ("int8 dynamic quant + bsr support", pytorch/ao PR 821, title and
+ *    description), with the absmax/127 symmetric scale that the Paddle
+ *    "sparse_fc supported" PR (PaddlePaddle PR 41770, SpmmPluginDynamic
+ *    constructor) computes for its int8 weight.  Scale and rounding are
+ *    fixed as: s = fp32( max(absmax, 1e-8f) / 127 ), q = clamp(rint(x/s),
+ *    -127, 127), round half to even, every operation one IEEE fp32 op.
+ *  - The same formula per output channel for the weight (Paddle PR 41770,
+ *    review of the plugin: a per-channel scale turns the GEMM alpha into a
+ *    vector).
+ *  - int8 x int8 -> int32 GEMM, exact integer accumulation ("triton dot
+ *    accumulator uses int32", PR 821 review by pearu; overflow bound
+ *    2^31 / 2^14 stated there).
+ *  - The bf16 output epilogue out = bf16( acc * s_row * s_col + bias ),
+ *    evaluated left to right in fp32 with round-to-nearest-even and no
+ *    fused multiply-add; bf16 output is what keeps accuracy (PR 821,
+ *    i8i8->bf16 eval vs i8i8->i8/32 eval).
+ *  - The BSR (crow_indices / col_indices / values of 64x64 blocks) weight
+ *    product (PR 821 description and the vit_h_14 --bsr 64 benchmark
+ *    command), plus the pack / densify conversions between a dense int8
+ *    weight and its BSR form.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fwrapv -fPIC
+ * -shared (see oracle/build.py).  -ffp-contract=off forbids FMA contraction
+ * so each fp32 multiply and add rounds on its own; -fwrapv makes an int32
+ * overflow (which the int64 twin of the GEMM would expose) well defined.
+ */
+#include <fenv.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+/* bf16 is carried as its 16-bit pattern: the top half of an IEEE fp32. */
+static float bf16_bits_to_float(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* fp32 -> bf16, round to nearest, ties to even, on the bit pattern.
+ * NaN stays a (quiet) NaN; +-inf stays +-inf; an overflow rounds to inf. */
+static uint16_t float_to_bf16_bits_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u) {           /* inf or NaN */
+        if (u & 0x007fffffu) return (uint16_t)((u >> 16) | 0x0040u);
+        return (uint16_t)(u >> 16);
+    }
+    uint32_t keep_lsb = (u >> 16) & 1u;                /* ties go to even */
+    u += 0x7fffu + keep_lsb;
+    return (uint16_t)(u >> 16);
+}
+
+uint16_t oracle_float_to_bf16(float f) { return float_to_bf16_bits_rne(f); }
+float oracle_bf16_to_float(uint16_t h) { return bf16_bits_to_float(h); }
+
+/* ---- per-row symmetric absmax quantization (activations and weight) --- */
+
+/* One row: absmax -> scale -> int8 codes.  `vals` already holds the row as
+ * fp32 values (exact for bf16 input). */
+static float quantize_one_row(const float* vals, int64_t K, int8_t* q) {
+    float absmax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        float a = fabsf(vals[k]);
+        if (a > absmax) absmax = a;
+    }
+    const float eps = 1e-8f;
+    float clipped = absmax > eps ? absmax : eps;       /* max(absmax, 1e-8) */
+    float scale = clipped / 127.0f;                    /* one IEEE division */
+    for (int64_t k = 0; k < K; ++k) {
+        float ratio = vals[k] / scale;                 /* true division, RN */
+        float r = nearbyintf(ratio);                   /* ties to even */
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        q[k] = (int8_t)r;
+    }
+    return scale;
+}
+
+/* x: bf16 bits [M, K], row stride ldx elements.  q: int8 [M, K], row
+ * stride ldq.  scales: fp32 [M].  Returns 0, or -1 if a row is too long for
+ * the scratch row (K > 1<<20). */
+int oracle_quantize_rows_bf16(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                              int8_t* q, int64_t ldq, float* scales) {
+    static float row[1 << 20];
+    if (K > (1 << 20)) return -1;
+    fesetround(FE_TONEAREST);
+    for (int64_t i = 0; i < M; ++i) {
+        for (int64_t k = 0; k < K; ++k) row[k] = bf16_bits_to_float(x[i * ldx + k]);
+        scales[i] = quantize_one_row(row, K, q + i * ldq);
+    }
+    return 0;
+}
+
+/* Weight preparation: fp32 [N, K] (nn.Linear layout, row n = output
+ * channel n), per-output-channel symmetric int8.  Same formula per row. */
+int oracle_quantize_rows_f32(const float* w, int64_t N, int64_t K, int64_t ldw,
+                             int8_t* q, int64_t ldq, float* scales) {
+    fesetround(FE_TONEAREST);
+    for (int64_t n = 0; n < N; ++n)
+        scales[n] = quantize_one_row(w + n * ldw, K, q + n * ldq);
+    return 0;
+}
+
+/* ---- int8 GEMM, exact integer accumulation ----------------------------- */
+
+/* acc[m, n] = sum_k A[m, k] * W[n, k]; A [M, K] ld lda, W [N, K] ld ldw,
+ * acc int32 [M, N] row-major. */
+void oracle_gemm_s32(const int8_t* A, int64_t M, int64_t K, int64_t lda,
+                     const int8_t* W, int64_t N, int64_t ldw, int32_t* acc) {
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int32_t s = 0;
+            for (int64_t k = 0; k < K; ++k)
+                s += (int32_t)A[m * lda + k] * (int32_t)W[n * ldw + k];
+            acc[m * N + n] = s;
+        }
+}
+
+/* Twin with int64 accumulation, for the brute-force overflow check. */
+void oracle_gemm_s64(const int8_t* A, int64_t M, int64_t K, int64_t lda,
+                     const int8_t* W, int64_t N, int64_t ldw, int64_t* acc) {
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t s = 0;
+            for (int64_t k = 0; k < K; ++k)
+                s += (int64_t)A[m * lda + k] * (int64_t)W[n * ldw + k];
+            acc[m * N + n] = s;
+        }
+}
+
+/* ---- epilogue: dequantize, bias, bf16 ----------------------------------- */
+
+/* out[m, n] = bf16_rne( ((float)acc[m, n] * s_row[m]) * s_col[n] + bias[n] )
+ * Left to right, each op one fp32 rounding.  bias == NULL means no addition
+ * at all (not even +0.0). */
+void oracle_epilogue_bf16(const int32_t* acc, int64_t M, int64_t N,
+                          const float* s_row, const float* s_col,
+                          const uint16_t* bias, uint16_t* out) {
+    fesetround(FE_TONEAREST);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float f = (float)acc[m * N + n];
+            f = f * s_row[m];
+            f = f * s_col[n];
+            if (bias) f = f + bf16_bits_to_float(bias[n]);
+            out[m * N + n] = float_to_bf16_bits_rne(f);
+        }
+}
+
+/* ---- block-sparse (BSR) weight ------------------------------------------ */
+
+/* W in BSR form with bs x bs blocks over an [N, K] weight: block row b holds
+ * output channels bs*b .. bs*b+bs-1; its blocks are p = crow[b] .. crow[b+1]-1,
+ * block p sits at block column col[p] and its values are values[p][j][t]
+ * (row j = channel, t = k offset, t contiguous).  Duplicate blocks add.
+ * acc int32 [M, N] row-major. */
+void oracle_bsr_gemm_s32(const int8_t* A, int64_t M, int64_t K, int64_t lda, int64_t N,
+                         const int32_t* crow, const int32_t* col, const int8_t* values,
+                         int64_t bs, int32_t* acc) {
+    (void)K;
+    memset(acc, 0, (size_t)(M * N) * sizeof(int32_t));
+    const int64_t nbr = N / bs;
+    for (int64_t b = 0; b < nbr; ++b)
+        for (int64_t p = crow[b]; p < crow[b + 1]; ++p) {
+            const int64_t c = col[p];
+            const int8_t* blk = values + p * bs * bs;
+            for (int64_t m = 0; m < M; ++m)
+                for (int64_t j = 0; j < bs; ++j) {
+                    int32_t s = 0;
+                    for (int64_t t = 0; t < bs; ++t)
+                        s += (int32_t)A[m * lda + c * bs + t] * (int32_t)blk[j * bs + t];
+                    acc[m * N + b * bs + j] += s;
+                }
+        }
+}
+
+/* Dense int8 [N, K] -> BSR values for the given (crow, col) pattern:
+ * values[p][j][t] = W[bs*b + j][bs*col[p] + t]. */
+void oracle_bsr_pack(const int8_t* W, int64_t N, int64_t K, const int32_t* crow,
+                     const int32_t* col, int64_t bs, int8_t* values) {
+    const int64_t nbr = N / bs;
+    for (int64_t b = 0; b < nbr; ++b)
+        for (int64_t p = crow[b]; p < crow[b + 1]; ++p)
+            for (int64_t j = 0; j < bs; ++j)
+                for (int64_t t = 0; t < bs; ++t)
+                    values[(p * bs + j) * bs + t] = W[(b * bs + j) * K + col[p] * bs + t];
+}
+
+/* BSR -> dense int32 [N, K] (int32 so that duplicate blocks can add
+ * without wrapping); entries outside every block are 0. */
+void oracle_bsr_densify(int64_t N, int64_t K, const int32_t* crow, const int32_t* col,
+                        const int8_t* values, int64_t bs, int32_t* W) {
+    memset(W, 0, (size_t)(N * K) * sizeof(int32_t));
+    const int64_t nbr = N / bs;
+    for (int64_t b = 0; b < nbr; ++b)
+        for (int64_t p = crow[b]; p < crow[b + 1]; ++p)
+            for (int64_t j = 0; j < bs; ++j)
+                for (int64_t t = 0; t < bs; ++t)
+                    W[(b * bs + j) * K + col[p] * bs + t] += values[(p * bs + j) * bs + t];
+}
