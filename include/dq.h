@@ -1,0 +1,205 @@
+/*
+ * dq.h -- C ABI of libdq: the int8 dynamic-quantization linear layer on
+ * NVIDIA B200 (sm_100a), dense and 64x64 block-sparse (BSR) weight.
+ *
+ * The layer (pytorch/ao PR 821, "int8 dynamic quant + bsr support",
+ * description and review) is
+ *
+ *     q, s_row = per-token absmax int8 quantization of x        (bf16 -> int8)
+ *     acc      = q . W_q^T                                        (int8 x int8 -> int32)
+ *     out      = bf16( acc * s_row * s_col + bias )              (fused epilogue)
+ *
+ * with W_q an int8 weight quantized per output channel (absmax / 127, as the
+ * Paddle "sparse_fc supported" PR 41770 computes its int8 weight scale, made
+ * per channel as asked in its review).  The int32 accumulator never reaches
+ * global memory in bf16 mode: the dequantization is fused into the GEMM,
+ * which the PR 821 description names as the fix for its slowdown.
+ *
+ * Conventions for every entry point:
+ *  - Tensor pointers are DEVICE pointers (unless stated), owned by the caller;
+ *    libdq never frees or keeps them.  Calls are asynchronous on `stream`
+ *    (a cudaStream_t; NULL = legacy default stream).
+ *  - No entry point allocates device memory or synchronises, except where
+ *    stated (dq_sync_status, dq_bsr_validate).  The first call on a device
+ *    resolves the driver's tensor-map encoder and queries the device.
+ *  - Arguments are validated on the host before any launch; a violation
+ *    returns DQ_ERR_INVALID_ARG or DQ_ERR_UNSUPPORTED and launches nothing.
+ *    Nothing aborts, throws or prints.
+ *  - Matrices are row-major.  "ld" arguments are row strides in ELEMENTS.
+ *  - Every wait inside a kernel is bounded (default 2 s, see
+ *    dq_set_wait_timeout_ns).  A wait that runs out makes the kernel record
+ *    DQ_ERR_TIMEOUT in a per-device error word and return; the error surfaces
+ *    through dq_sync_status().
+ *  - Only sm_100 devices (B200) are supported: anything else returns
+ *    DQ_ERR_UNSUPPORTED.  There is no CPU or other fallback.
+ */
+#ifndef DQ_H_
+#define DQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DQ_API __attribute__((visibility("default")))
+#else
+#define DQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the runtime's stream handle) passed as a plain pointer. */
+typedef struct CUstream_st* dq_stream_t;
+
+typedef enum {
+    DQ_OK = 0,
+    DQ_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad stride, bad enum */
+    DQ_ERR_UNSUPPORTED = 2,   /* shape / alignment / device outside what libdq handles */
+    DQ_ERR_CUDA = 3,          /* a CUDA runtime or driver call failed: dq_last_cuda_error() */
+    DQ_ERR_TIMEOUT = 4        /* a bounded device wait ran out (reported by dq_sync_status) */
+} dq_status;
+
+typedef enum {
+    DQ_OUT_BF16 = 0,          /* out = bf16(acc * s_row * s_col + bias): the layer */
+    DQ_OUT_S32 = 1            /* out = acc as int32 (scales and bias ignored) */
+} dq_out_dtype;
+
+/* Static description of a status code. Never NULL. */
+DQ_API const char* dq_status_string(dq_status s);
+
+/* The cudaError_t value behind the most recent DQ_ERR_CUDA on this host
+ * thread (0 if none). */
+DQ_API int dq_last_cuda_error(void);
+
+/* Library version: major*10000 + minor*100 + patch. */
+DQ_API int dq_version(void);
+
+/* Synchronises `stream`, then reads and clears the current device's error
+ * word.  Returns DQ_ERR_TIMEOUT if any kernel since the last call ran out a
+ * bounded wait, DQ_ERR_CUDA if the synchronisation failed, DQ_OK otherwise.
+ * Blocking. */
+DQ_API dq_status dq_sync_status(dq_stream_t stream);
+
+/* Limit, in nanoseconds of %globaltimer, for every bounded wait in kernels
+ * launched after this call from any host thread (default 2e9).  0 restores
+ * the default.  Host-side setting; takes effect at the next launch. */
+DQ_API void dq_set_wait_timeout_ns(uint64_t ns);
+
+/* Launches a one-CTA kernel that waits on an mbarrier nothing ever arrives
+ * on, through the same bounded wait the GEMM kernels use, and so records
+ * DQ_ERR_TIMEOUT after the configured limit.  For testing the failure path
+ * without faulting the GPU.  Asynchronous. */
+DQ_API dq_status dq_selftest_wait_timeout(dq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Quantization (first stage of the layer; pytorch/ao PR 821 "int8 dynamic
+ * quant", Paddle PR 41770 absmax / 127 scale).
+ *
+ * For each row i:  a = max_k |x[i,k]|,  s[i] = fp32( max(a, 1e-8f) / 127 ),
+ *                  q[i,k] = clamp( rint_half_even( fp32(x[i,k] / s[i]) ), -127, 127 ).
+ * Every fp32 operation is one IEEE operation rounded to nearest even (true
+ * division, no reciprocal), so results are bit-identical to a scalar IEEE
+ * evaluation.  Non-finite inputs give unspecified (but in-bounds) results.
+ *
+ * x: bf16 [M, K] (as 16-bit patterns), row stride ldx >= K.
+ * q: int8 [M, K], row stride ldq >= K.   scales: fp32 [M].
+ * M >= 0, K >= 1 (M == 0 is a no-op).  Any alignment is accepted; rows
+ * with K % 8 == 0, ldx % 8 == 0, ldq % 8 == 0 and 16-byte-aligned x and
+ * 8-byte-aligned q take the vectorised single-pass kernel.
+ * ------------------------------------------------------------------------ */
+DQ_API dq_status dq_quantize_rows(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                           int8_t* q, int64_t ldq, float* scales, dq_stream_t stream);
+
+/* Weight preparation with the same formula per output channel: w fp32
+ * [N, K] (nn.Linear layout: row n is output channel n), row stride ldw.
+ * wq int8 [N, K] (row stride ldwq), s_col fp32 [N].  Offline step, not part
+ * of the per-token hot path, but run on the GPU by the same kernel family. */
+DQ_API dq_status dq_quantize_weight(const float* w, int64_t N, int64_t K, int64_t ldw,
+                             int8_t* wq, int64_t ldwq, float* s_col, dq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Dense int8 linear (second and third stages fused).
+ *
+ *   acc[m,n] = sum_k A[m,k] * W[n,k]            exact int32 (|acc| <= K*127^2)
+ *   DQ_OUT_BF16: out[m,n] = bf16_rne( ((float)acc * s_row[m]) * s_col[n] (+ bias[n]) )
+ *                each step one fp32 op, round to nearest even, no FMA;
+ *                bias == NULL means no addition at all.
+ *   DQ_OUT_S32:  out[m,n] = acc (s_row, s_col, bias ignored, may be NULL).
+ *
+ * A: int8 [M, K], row-major, contiguous (K-major).   s_row: fp32 [M].
+ * W: int8 [N, K], row-major, contiguous (K-major).   s_col: fp32 [N].
+ * bias: bf16 [N] or NULL.   out: [M, N] row-major contiguous, bf16 or int32.
+ * Requirements: M >= 0; 1 <= K <= 133144 (the int32 bound: 133144 * 127^2 <
+ * 2^31) and K % 16 == 0; N >= 1 with N % 8 == 0; A, W, out 16-byte aligned.
+ *
+ * workspace / workspace_bytes: optional caller-owned device scratch for the
+ * split-K (stream-K) schedules that keep all SMs busy when the output has
+ * few tiles.  Pass NULL/0 to disable splitting (always correct, possibly
+ * slower).  The size the library can use is dq_int8_linear_workspace_size();
+ * a smaller buffer disables splitting.  The workspace must be ZERO-FILLED
+ * before its first use; every call that completes leaves it zero-filled
+ * again (after DQ_ERR_TIMEOUT, zero it again).  Two calls in flight at the
+ * same time must not share a workspace.
+ * ------------------------------------------------------------------------ */
+DQ_API dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K,
+                         const int8_t* W, const float* s_col, int64_t N,
+                         const void* bias_bf16, void* out, dq_out_dtype out_dtype,
+                         void* workspace, size_t workspace_bytes, dq_stream_t stream);
+
+/* Bytes of workspace dq_int8_linear can use for this shape on the current
+ * device (0 when the schedule never splits). */
+DQ_API size_t dq_int8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* ------------------------------------------------------------------------
+ * Block-sparse (BSR) int8 linear, 64x64 blocks (pytorch/ao PR 821: the
+ * kernel takes crow_indices / col_indices / values directly; vit_h_14
+ * benchmark with --bsr 64).
+ *
+ * W [N, K] in BSR form: block row b (output channels 64b .. 64b+63) holds
+ * blocks p = crow[b] .. crow[b+1]-1; block p covers input channels
+ * 64*col[p] .. 64*col[p]+63 and values[p] is its 64x64 int8 tile, row j =
+ * channel 64b+j, 64 contiguous k values.  Duplicate blocks add.
+ *   acc[m, 64b+j] = sum_p sum_t A[m, 64 col[p] + t] * values[p][j][t]
+ * then the same epilogue as dq_int8_linear.  Block rows with no block give
+ * bias (or 0) in bf16 mode and 0 in int32 mode.
+ *
+ * crow: int32 [N/64 + 1], col: int32 [nnzb], values: int8 [nnzb, 64, 64].
+ * Requirements: K % 64 == 0, N % 64 == 0, K <= 133120, nnzb >= 0, pointers
+ * 16-byte aligned.  Indices must be canonical (crow[0] == 0, non-decreasing,
+ * crow[N/64] == nnzb, 0 <= col < K/64; order inside a row is free).  The
+ * kernel clamps block ranges to [0, nnzb] and a column outside [0, K/64)
+ * reads zeros, so malformed indices give wrong numbers but never an
+ * out-of-bounds access; dq_bsr_validate checks them on the host.
+ * ------------------------------------------------------------------------ */
+DQ_API dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K, int64_t N,
+                             const int32_t* crow, const int32_t* col, const int8_t* values,
+                             int64_t nnzb, const float* s_col, const void* bias_bf16,
+                             void* out, dq_out_dtype out_dtype, dq_stream_t stream);
+
+/* Gathers the 64x64 blocks named by (crow, col) out of a dense int8 weight
+ * wq [N, K] (row stride K) into values [nnzb, 64, 64].  Offline weight
+ * preparation (mask, quantize per channel, pack).  Same index requirements
+ * as dq_bsr_int8_linear. */
+DQ_API dq_status dq_bsr_pack(const int8_t* wq, int64_t N, int64_t K, const int32_t* crow,
+                      const int32_t* col, int64_t nnzb, int8_t* values, dq_stream_t stream);
+
+/* Host-side, synchronous: copies crow and col to the host and checks the
+ * canonical form above.  DQ_OK or DQ_ERR_INVALID_ARG. */
+DQ_API dq_status dq_bsr_validate(const int32_t* crow, const int32_t* col, int64_t N, int64_t K,
+                          int64_t nnzb);
+
+/* ------------------------------------------------------------------------
+ * Measurement helper: a kernel that only issues tcgen05.mma.kind::i8
+ * (128x256x32, operands resident in shared memory, accumulator in TMEM) on
+ * every SM, `iters` times per CTA, with no global-memory traffic.  Used to
+ * state the measured dense INT8 tensor-pipe peak: ops = grid * iters *
+ * 2*128*256*32.  grid <= 0 means one CTA per SM.
+ * ------------------------------------------------------------------------ */
+DQ_API dq_status dq_mma_peak_probe(int grid, int iters, dq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DQ_H_ */

@@ -1,0 +1,313 @@
+"""Python binding of libdq: the int8 dynamic-quantization linear layer on B200.
+
+Argument marshalling only.  Every step of the layer runs in libdq's CUDA
+kernels (``csrc/``); PyTorch supplies device memory and streams.  There is no
+CPU or eager fallback: if ``libdq.so`` is missing, importing this package
+raises, and every call on a non-sm_100 device returns an error.
+
+Function names match the C ABI in ``include/dq.h``.  Tensors are torch CUDA
+tensors; bf16 tensors are passed by pointer as 16-bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdq.so")
+
+DQ_OK, DQ_ERR_INVALID_ARG, DQ_ERR_UNSUPPORTED, DQ_ERR_CUDA, DQ_ERR_TIMEOUT = range(5)
+DQ_OUT_BF16, DQ_OUT_S32 = 0, 1
+
+# C prototypes: (name, restype, argtypes)
+_P, _I64, _I32, _SZ, _U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
+_PROTOS = {
+    "dq_status_string": (ctypes.c_char_p, [_I32]),
+    "dq_last_cuda_error": (_I32, []),
+    "dq_version": (_I32, []),
+    "dq_sync_status": (_I32, [_P]),
+    "dq_set_wait_timeout_ns": (None, [_U64]),
+    "dq_selftest_wait_timeout": (_I32, [_P]),
+    "dq_quantize_rows": (_I32, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
+    "dq_quantize_weight": (_I32, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
+    "dq_int8_linear": (_I32, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P, _I32, _P, _SZ, _P]),
+    "dq_int8_linear_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "dq_bsr_int8_linear": (_I32, [_P, _P, _I64, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _I32, _P]),
+    "dq_bsr_pack": (_I32, [_P, _I64, _I64, _P, _P, _I64, _P, _P]),
+    "dq_bsr_validate": (_I32, [_P, _P, _I64, _I64, _I64]),
+    "dq_mma_peak_probe": (_I32, [_I32, _I32, _P]),
+    "dq_debug_set_schedule": (None, [_I32]),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libdq.so not found at {LIB_PATH}: build it with "
+            "`python -m quantized_gemm_token_b200.build` (nvcc, sm_100a). "
+            "There is no fallback implementation.")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _PROTOS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+class DQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.dq_status_string(status).decode()
+        if status == DQ_ERR_CUDA:
+            msg += f" (cudaError {lib.dq_last_cuda_error()})"
+        super().__init__(f"{where}: {msg}")
+
+
+def _check(status: int, where: str):
+    if status != DQ_OK:
+        raise DQError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t: torch.Tensor, dtype, name: str, ndim: int = None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name}: expected a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dims, got {t.dim()}")
+
+
+def _contig(t: torch.Tensor, name: str):
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+# ---------------------------------------------------------------- status
+
+def dq_status_string(status: int) -> str:
+    return lib.dq_status_string(status).decode()
+
+
+def dq_version() -> int:
+    return lib.dq_version()
+
+
+def dq_sync_status(stream=None) -> int:
+    """Synchronise `stream` and return (and clear) the device error status."""
+    return lib.dq_sync_status(_stream(stream))
+
+
+def dq_set_wait_timeout_ns(ns: int) -> None:
+    lib.dq_set_wait_timeout_ns(int(ns))
+
+
+def dq_selftest_wait_timeout(stream=None) -> None:
+    _check(lib.dq_selftest_wait_timeout(_stream(stream)), "dq_selftest_wait_timeout")
+
+
+def dq_debug_set_schedule(mode: int) -> None:
+    lib.dq_debug_set_schedule(int(mode))
+
+
+# ---------------------------------------------------------------- quantize
+
+def dq_quantize_rows(x: torch.Tensor, q: torch.Tensor = None, scales: torch.Tensor = None, stream=None):
+    """Per-token int8 quantization: x bf16 [M, K] (row stride x.stride(0))
+    -> (q int8 [M, K], scales fp32 [M])."""
+    _need(x, torch.bfloat16, "x", 2)
+    if x.stride(1) != 1:
+        raise ValueError("x: rows must be contiguous")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _need(q, torch.int8, "q", 2)
+    _need(scales, torch.float32, "scales", 1)
+    if q.stride(1) != 1 or tuple(q.shape) != (M, K) or scales.numel() != M:
+        raise ValueError("q / scales: shape or layout mismatch")
+    _check(lib.dq_quantize_rows(_ptr(x), M, K, x.stride(0), _ptr(q), q.stride(0), _ptr(scales),
+                                _stream(stream)), "dq_quantize_rows")
+    return q, scales
+
+
+def dq_quantize_weight(w: torch.Tensor, wq: torch.Tensor = None, s_col: torch.Tensor = None, stream=None):
+    """Per-output-channel int8 weight: w fp32 [N, K] -> (wq int8 [N, K], s_col fp32 [N])."""
+    _need(w, torch.float32, "w", 2)
+    if w.stride(1) != 1:
+        raise ValueError("w: rows must be contiguous")
+    N, K = w.shape
+    if wq is None:
+        wq = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    if s_col is None:
+        s_col = torch.empty((N,), dtype=torch.float32, device=w.device)
+    _check(lib.dq_quantize_weight(_ptr(w), N, K, w.stride(0), _ptr(wq), wq.stride(0), _ptr(s_col),
+                                  _stream(stream)), "dq_quantize_weight")
+    return wq, s_col
+
+
+# ---------------------------------------------------------------- linear
+
+def _out_code(out_dtype) -> int:
+    if out_dtype in ("bf16", torch.bfloat16, DQ_OUT_BF16):
+        return DQ_OUT_BF16
+    if out_dtype in ("s32", "int32", torch.int32, DQ_OUT_S32):
+        return DQ_OUT_S32
+    raise ValueError(f"out_dtype {out_dtype!r}")
+
+
+def dq_int8_linear_workspace_size(M: int, N: int, K: int) -> int:
+    return int(lib.dq_int8_linear_workspace_size(M, N, K))
+
+
+def dq_int8_linear(A, s_row, W, s_col, bias=None, out=None, out_dtype="bf16", workspace=None, stream=None):
+    """out[M, N] = bf16(acc * s_row * s_col + bias), acc = A @ W^T exactly
+    (or acc itself as int32 with out_dtype="s32").  `workspace` is an
+    optional zero-filled uint8 CUDA tensor (see dq_int8_linear_workspace_size)."""
+    code = _out_code(out_dtype)
+    _need(A, torch.int8, "A", 2)
+    _need(W, torch.int8, "W", 2)
+    _contig(A, "A")
+    _contig(W, "W")
+    M, K = A.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("A and W disagree on K")
+    if code == DQ_OUT_BF16:
+        _need(s_row, torch.float32, "s_row", 1)
+        _need(s_col, torch.float32, "s_col", 1)
+        if s_row.numel() != M or s_col.numel() != N:
+            raise ValueError("scale length mismatch")
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias", 1)
+        if bias.numel() != N:
+            raise ValueError("bias length mismatch")
+    odt = torch.bfloat16 if code == DQ_OUT_BF16 else torch.int32
+    if out is None:
+        out = torch.empty((M, N), dtype=odt, device=A.device)
+    _need(out, odt, "out", 2)
+    _contig(out, "out")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _need(workspace, torch.uint8, "workspace")
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()
+    _check(lib.dq_int8_linear(_ptr(A), _ptr(s_row), M, K, _ptr(W), _ptr(s_col), N, _ptr(bias), _ptr(out),
+                              code, ws_ptr, ws_bytes, _stream(stream)), "dq_int8_linear")
+    return out
+
+
+def dq_bsr_int8_linear(A, s_row, N, crow, col, values, s_col, bias=None, out=None, out_dtype="bf16",
+                       stream=None):
+    """BSR (64x64 int8 blocks) variant of dq_int8_linear; W given as
+    crow int32 [N/64+1], col int32 [nnzb], values int8 [nnzb, 64, 64]."""
+    code = _out_code(out_dtype)
+    _need(A, torch.int8, "A", 2)
+    _contig(A, "A")
+    M, K = A.shape
+    _need(crow, torch.int32, "crow", 1)
+    _need(col, torch.int32, "col", 1)
+    _need(values, torch.int8, "values", 3)
+    _contig(values, "values")
+    nnzb = values.shape[0]
+    if crow.numel() != N // 64 + 1 or col.numel() != nnzb or tuple(values.shape[1:]) != (64, 64):
+        raise ValueError("BSR arrays do not match N / nnzb")
+    if code == DQ_OUT_BF16:
+        _need(s_row, torch.float32, "s_row", 1)
+        _need(s_col, torch.float32, "s_col", 1)
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias", 1)
+    odt = torch.bfloat16 if code == DQ_OUT_BF16 else torch.int32
+    if out is None:
+        out = torch.empty((M, N), dtype=odt, device=A.device)
+    _need(out, odt, "out", 2)
+    _contig(out, "out")
+    _check(lib.dq_bsr_int8_linear(_ptr(A), _ptr(s_row), M, K, N, _ptr(crow), _ptr(col),
+                                  _ptr(values) if nnzb else None, nnzb, _ptr(s_col), _ptr(bias), _ptr(out),
+                                  code, _stream(stream)), "dq_bsr_int8_linear")
+    return out
+
+
+def dq_bsr_pack(wq, crow, col, values=None, stream=None):
+    """Gather the 64x64 blocks of a dense int8 weight [N, K] named by (crow, col)."""
+    _need(wq, torch.int8, "wq", 2)
+    _contig(wq, "wq")
+    N, K = wq.shape
+    nnzb = col.numel()
+    if values is None:
+        values = torch.empty((nnzb, 64, 64), dtype=torch.int8, device=wq.device)
+    _check(lib.dq_bsr_pack(_ptr(wq), N, K, _ptr(crow), _ptr(col), nnzb, _ptr(values) if nnzb else None,
+                           _stream(stream)), "dq_bsr_pack")
+    return values
+
+
+def dq_bsr_validate(crow, col, N: int, K: int) -> int:
+    return lib.dq_bsr_validate(_ptr(crow), _ptr(col) if col.numel() else None, N, K, col.numel())
+
+
+def dq_mma_peak_probe(grid: int, iters: int, stream=None) -> None:
+    _check(lib.dq_mma_peak_probe(grid, iters, _stream(stream)), "dq_mma_peak_probe")
+
+
+# ---------------------------------------------------------------- layer
+
+class Int8DynamicLinear:
+    """The layer: per-token dynamic int8 quantization of bf16 activations,
+    then the fused i8i8->bf16 GEMM against a per-channel int8 weight (dense,
+    or 64x64 BSR when built with from_bsr).  Holds the quantized weight, the
+    activation scratch and the stream-K workspace; call it on bf16 [M, K]."""
+
+    def __init__(self, wq, s_col, bias=None, bsr=None):
+        self.wq, self.s_col, self.bias, self.bsr = wq, s_col, bias, bsr
+        self.N = s_col.numel()
+        self.K = wq.shape[1] if bsr is None else bsr["K"]
+        self._q = self._s = self._ws = None
+
+    @classmethod
+    def from_float(cls, w: torch.Tensor, bias: torch.Tensor = None):
+        wq, s_col = dq_quantize_weight(w)
+        return cls(wq, s_col, bias)
+
+    @classmethod
+    def from_bsr(cls, w_masked: torch.Tensor, crow: torch.Tensor, col: torch.Tensor, bias=None):
+        """w_masked: fp32 [N, K] already zero outside the kept 64x64 blocks."""
+        wq, s_col = dq_quantize_weight(w_masked)
+        values = dq_bsr_pack(wq, crow, col)
+        return cls(None, s_col, bias, dict(crow=crow, col=col, values=values, K=w_masked.shape[1]))
+
+    def _buffers(self, M, device):
+        if self._q is None or self._q.shape[0] < M:
+            self._q = torch.empty((M, self.K), dtype=torch.int8, device=device)
+            self._s = torch.empty((M,), dtype=torch.float32, device=device)
+            if self.bsr is None:
+                n = dq_int8_linear_workspace_size(M, self.N, self.K)
+                self._ws = torch.zeros((n,), dtype=torch.uint8, device=device) if n else None
+        return self._q[:M], self._s[:M]
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor = None, stream=None):
+        M = x.shape[0]
+        q, s = self._buffers(M, x.device)
+        dq_quantize_rows(x, q, s, stream=stream)
+        if self.bsr is None:
+            ws = self._ws
+            if ws is not None and ws.numel() < dq_int8_linear_workspace_size(M, self.N, self.K):
+                ws = None
+            return dq_int8_linear(q, s, self.wq, self.s_col, self.bias, out=out, workspace=ws, stream=stream)
+        b = self.bsr
+        return dq_bsr_int8_linear(q, s, self.N, b["crow"], b["col"], b["values"], self.s_col, self.bias,
+                                  out=out, stream=stream)

@@ -1,0 +1,742 @@
+// gemm.cu -- the int8 x int8 -> int32 GEMM with the dequantization epilogue
+// fused (pytorch/ao PR 821, "int8 dynamic quant + bsr support": i8i8->bf16,
+// no int32 intermediate in global memory), dense and 64x64 BSR weight.
+//
+// One persistent, warp-specialised kernel template for sm_100a:
+//   warp 0      TMA producer: streams K slices of both operands into a ring
+//               of shared-memory stages (mbarrier full/empty pairs).
+//   warp 1      MMA issuer: one thread issues tcgen05.mma.kind::i8 (M = 128)
+//               into an int32 accumulator in TMEM; tcgen05.commit releases the
+//               stage and, at the end of a tile, hands the accumulator over.
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (thread = TMEM lane =
+//               output row), dequantize in fp32 (acc * s_row * s_col + bias,
+//               each op rounded to nearest even, no FMA), convert to bf16 and
+//               store.  Accumulators are multi-buffered in TMEM so the
+//               epilogue of tile i overlaps the MMAs of tile i+1.
+//
+// Three operand arrangements share it:
+//   Dense  A slot = 128 activation rows, B slot = BN weight channels.
+//   Swap   A slot = 128 weight channels, B slot = BN (16..128) tokens: for
+//          few tokens the weight stream, not the token count, fills MMA M.
+//   Bsr    A slot = 128 activation rows x one 64-wide k slice, B slot = one
+//          nonzero 64x64 weight block; the producer walks crow/col of one
+//          block row (PR 821: the kernel takes crow_indices / col_indices /
+//          values directly).
+//
+// Schedules: whole tiles round-robin over one CTA per SM, or (when the tile
+// count would leave SMs idle) stream-K: the tile x k-block iteration space is
+// cut into equal contiguous ranges, one per CTA; partial tiles meet in an
+// int32 workspace through red.add, and the last arriving CTA (an arrival
+// counter) runs the epilogue and zeroes the workspace again.  Integer adds
+// are exact and associative, so every schedule gives identical bits.
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace dq {
+
+enum class Kind : int { Dense = 0, Swap = 1, Bsr = 2 };
+
+struct GemmArgs {
+  int M, N, K;
+  int a_tiles, b_tiles;   // tiles along the A slot (128 rows) and the B slot (BN rows)
+  int kb_total;           // k blocks per tile (Dense / Swap)
+  int num_tiles;
+  int stream_k;           // 0: whole tiles round-robin; 1: stream-K ranges
+  long long iters_total;  // num_tiles * kb_total (stream-K)
+  const float* s_row;
+  const float* s_col;
+  const uint16_t* bias;   // bf16 bits or null
+  void* out;
+  int out_s32;
+  int32_t* ws;            // stream-K partial tiles: [tile][BN][128] int32
+  uint32_t* ws_cnt;       // stream-K arrival counters: [tile]
+  const int32_t* crow;    // Bsr
+  const int32_t* col;
+  int nnzb;
+  WaitCtl wait;
+};
+
+template <Kind KIND, int BN>
+struct Cfg {
+  static constexpr int BM = 128;
+  static constexpr int KB = KIND == Kind::Bsr ? 64 : 128;     // k bytes per stage
+  static constexpr int A_BYTES = BM * KB;
+  static constexpr int B_BYTES = BN * KB;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+  static constexpr int ACC_RAW = 512 / BN;
+  static constexpr int ACC_BUFS = ACC_RAW > 8 ? 8 : ACC_RAW;
+  static constexpr int ACC_COLS = ACC_BUFS * BN;
+  static constexpr int TMEM_COLS = ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128
+                                   : ACC_COLS <= 256 ? 256 : 512;
+  static constexpr int K_STEPS = KB / 32;                     // MMA K = 32 bytes
+  static constexpr int CW = BN >= 32 ? 32 : 16;               // epilogue chunk (columns)
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int THREADS = 192;
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(STAGES >= 2, "stages");
+};
+
+struct Seg {
+  int tile;
+  int kb0, kb1;
+};
+
+// Enumerates the (tile, k range) segments of one CTA; every role walks the
+// same sequence.
+struct SegIter {
+  const GemmArgs* g;
+  long long it, it_end;   // stream-K
+  int next_tile;          // round-robin
+  __device__ SegIter(const GemmArgs& args) : g(&args) {
+    const long long G = gridDim.x, c = blockIdx.x;
+    if (args.stream_k) {
+      it = c * args.iters_total / G;
+      it_end = (c + 1) * args.iters_total / G;
+    }
+    next_tile = blockIdx.x;
+  }
+  __device__ bool next(Seg& s) {
+    if (g->stream_k) {
+      if (it >= it_end) return false;
+      s.tile = static_cast<int>(it / g->kb_total);
+      s.kb0 = static_cast<int>(it - static_cast<long long>(s.tile) * g->kb_total);
+      const long long left = it_end - it;
+      s.kb1 = static_cast<int>(min(static_cast<long long>(g->kb_total), s.kb0 + left));
+      it += s.kb1 - s.kb0;
+      return true;
+    }
+    if (next_tile >= g->num_tiles) return false;
+    s.tile = next_tile;
+    next_tile += gridDim.x;
+    s.kb0 = 0;
+    s.kb1 = g->kb_total;
+    return true;
+  }
+};
+
+// Stream-K: number of CTAs whose ranges touch `tile`.
+__device__ __forceinline__ int sk_contributors(const GemmArgs& g, int tile) {
+  const long long G = gridDim.x, T = g.iters_total;
+  const long long first = static_cast<long long>(tile) * g.kb_total;
+  const long long last = first + g.kb_total - 1;
+  const long long c0 = ((first + 1) * G - 1) / T;
+  const long long c1 = ((last + 1) * G - 1) / T;
+  return static_cast<int>(c1 - c0 + 1);
+}
+
+// Block range of one BSR block row, clamped to [0, nnzb].
+__device__ __forceinline__ void bsr_range(const GemmArgs& g, int br, int& p0, int& p1) {
+  int a = __ldg(g.crow + br), b = __ldg(g.crow + br + 1);
+  a = min(max(a, 0), g.nnzb);
+  b = min(max(b, a), g.nnzb);
+  p0 = a;
+  p1 = b;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Epilogue for one chunk of CW columns of one row in the Dense/Bsr layout
+// (thread = output row m, columns n0 .. n0+CW-1).  r = raw int32 accumulator.
+template <int CW>
+__device__ __forceinline__ void store_row_chunk(const GemmArgs& g, int m, int n0, const uint32_t* r,
+                                                float srow) {
+  if (g.out_s32) {
+    int32_t* o = static_cast<int32_t*>(g.out) + static_cast<int64_t>(m) * g.N + n0;
+#pragma unroll
+    for (int v = 0; v < CW / 4; ++v)
+      if (n0 + 4 * v < g.N)
+        *reinterpret_cast<int4*>(o + 4 * v) =
+            make_int4(static_cast<int>(r[4 * v]), static_cast<int>(r[4 * v + 1]),
+                      static_cast<int>(r[4 * v + 2]), static_cast<int>(r[4 * v + 3]));
+    return;
+  }
+  uint16_t* o = static_cast<uint16_t*>(g.out) + static_cast<int64_t>(m) * g.N + n0;
+#pragma unroll
+  for (int v = 0; v < CW / 8; ++v) {
+    const int n = n0 + 8 * v;
+    if (n < g.N) {
+      const float4 c0 = __ldg(reinterpret_cast<const float4*>(g.s_col + n));
+      const float4 c1 = __ldg(reinterpret_cast<const float4*>(g.s_col + n + 4));
+      const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      float f[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        f[j] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[8 * v + j])), srow), sc[j]);
+      if (g.bias) {
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(g.bias + n));
+        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          f[2 * j] = __fadd_rn(f[2 * j], __uint_as_float(bw[j] << 16));
+          f[2 * j + 1] = __fadd_rn(f[2 * j + 1], __uint_as_float(bw[j] & 0xffff0000u));
+        }
+      }
+      *reinterpret_cast<uint4*>(o + 8 * v) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                        pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+    }
+  }
+}
+
+// Epilogue for the Swap layout: thread = output channel n, columns are
+// tokens m0 .. m0+CW-1.
+template <int CW>
+__device__ __forceinline__ void store_col_chunk(const GemmArgs& g, int n, int m0, const uint32_t* r) {
+  if (n >= g.N) return;
+  if (g.out_s32) {
+    int32_t* o = static_cast<int32_t*>(g.out) + n;
+#pragma unroll
+    for (int j = 0; j < CW; ++j)
+      if (m0 + j < g.M) o[static_cast<int64_t>(m0 + j) * g.N] = static_cast<int>(r[j]);
+    return;
+  }
+  const float sc = __ldg(g.s_col + n);
+  const bool has_bias = g.bias != nullptr;
+  const float b = has_bias ? __uint_as_float(static_cast<uint32_t>(__ldg(g.bias + n)) << 16) : 0.0f;
+  uint16_t* o = static_cast<uint16_t*>(g.out) + n;
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    const int m = m0 + j;
+    if (m < g.M) {
+      float f = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), __ldg(g.s_row + m)), sc);
+      if (has_bias) f = __fadd_rn(f, b);
+      __nv_bfloat16 h = __float2bfloat16_rn(f);
+      o[static_cast<int64_t>(m) * g.N] = *reinterpret_cast<uint16_t*>(&h);
+    }
+  }
+}
+
+template <Kind KIND, int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                const __grid_constant__ GemmArgs g) {
+  using C = Cfg<KIND, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + C::STAGES;
+  uint64_t* accf_bar = bars + 2 * C::STAGES;
+  uint64_t* acce_bar = accf_bar + C::ACC_BUFS;
+  uint64_t* drain_bar = acce_bar + C::ACC_BUFS;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* sk_last = const_cast<int*>(abort_flag + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(full_bar + s), 1);
+      mbar_init(smem_u32(empty_bar + s), 1);
+    }
+    for (int a = 0; a < C::ACC_BUFS; ++a) {
+      mbar_init(smem_u32(accf_bar + a), 1);
+      mbar_init(smem_u32(acce_bar + a), 128);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      SegIter iter(g);
+      Seg s;
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      while (ok && iter.next(s)) {
+        const int ta = s.tile / g.b_tiles, tb = s.tile % g.b_tiles;
+        int k0 = s.kb0, k1 = s.kb1;
+        if constexpr (KIND == Kind::Bsr) bsr_range(g, tb, k0, k1);
+        for (int kb = k0; kb < k1; ++kb) {
+          if (!mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, g.wait, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(full_bar + stage);
+          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          const uint32_t da = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t db = smem_u32(sB + stage * C::B_BYTES);
+          if constexpr (KIND == Kind::Bsr) {
+            const int c = __ldg(g.col + kb);
+            tma_load_2d(da, &tm_a, fb, c * 64, ta * 128);
+            tma_load_2d(db, &tm_b, fb, 0, kb * 64);
+          } else {
+            tma_load_2d(da, &tm_a, fb, kb * C::KB, ta * 128);
+            tma_load_2d(db, &tm_b, fb, kb * C::KB, tb * BN);
+          }
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the (at most STAGES) most recent loads land before the CTA
+        // leaves; each wait is bounded by a short limit.
+        WaitCtl quick = g.wait;
+        quick.timeout_ns = quick.timeout_ns < 50000000ull ? quick.timeout_ns : 50000000ull;
+        volatile int never = 0;
+        for (long long i = 0; i < issued && i < C::STAGES; ++i) {
+          if (--stage < 0) {
+            stage = C::STAGES - 1;
+            phase ^= 1;
+          }
+          mbar_wait(smem_u32(full_bar + stage), phase, quick, &never);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(128, BN);
+      SegIter iter(g);
+      Seg s;
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      while (ok && iter.next(s)) {
+        int k0 = s.kb0, k1 = s.kb1;
+        if constexpr (KIND == Kind::Bsr) {
+          bsr_range(g, s.tile % g.b_tiles, k0, k1);
+          if (k0 == k1) continue;    // empty block row: no accumulator
+        }
+        if (!mbar_wait(smem_u32(acce_bar + acc), acc_phase ^ 1, g.wait, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = k0; kb < k1; ++kb) {
+          if (!mbar_wait(smem_u32(full_bar + stage), phase, g.wait, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = smem_desc_kmajor<C::KB>(smem_u32(sA + stage * C::A_BYTES));
+          const uint64_t bd = smem_desc_kmajor<C::KB>(smem_u32(sB + stage * C::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < C::K_STEPS; ++k)
+            mma_i8(d, ad + 2 * k, bd + 2 * k, idesc, (kb > k0 || k > 0) ? 1u : 0u);
+          mma_commit(smem_u32(empty_bar + stage));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(accf_bar + acc));
+        if (++acc == C::ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      // Every MMA issued by this thread has completed once drain_bar flips.
+      mma_commit(smem_u32(drain_bar));
+      volatile int never = 0;
+      mbar_wait(smem_u32(drain_bar), 0, g.wait, &never);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    constexpr int CW = C::CW;
+    const int sp = warp & 3;                 // TMEM sub-partition of this warp
+    const int row = sp * 32 + lane;          // TMEM lane = accumulator row
+    const int ep_tid = threadIdx.x - 64;
+    SegIter iter(g);
+    Seg s;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    while (iter.next(s)) {
+      const int ta = s.tile / g.b_tiles, tb = s.tile % g.b_tiles;
+      if constexpr (KIND == Kind::Bsr) {
+        int p0, p1;
+        bsr_range(g, tb, p0, p1);
+        if (p0 == p1) {
+          // Block row without blocks: the epilogue of acc = 0.
+          const int m = ta * 128 + row;
+          if (m < g.M) {
+            const float srow = g.out_s32 ? 0.0f : __ldg(g.s_row + m);
+            uint32_t z[CW];
+#pragma unroll
+            for (int j = 0; j < CW; ++j) z[j] = 0;
+#pragma unroll 1
+            for (int c = 0; c < BN / CW; ++c) store_row_chunk<CW>(g, m, tb * BN + c * CW, z, srow);
+          }
+          continue;
+        }
+      }
+      if (!mbar_wait(smem_u32(accf_bar + acc), acc_phase, g.wait, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const bool whole = !g.stream_k || (s.kb0 == 0 && s.kb1 == g.kb_total);
+
+      if (whole) {
+        float srow = 0.0f;
+        int m = 0;
+        if constexpr (KIND != Kind::Swap) {
+          m = ta * 128 + row;
+          if (!g.out_s32 && m < g.M) srow = __ldg(g.s_row + m);
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN / CW; ++c) {
+          uint32_t r[CW];
+          if constexpr (CW == 32) tmem_ld_32x32b_x32(tbase + c * CW, r);
+          else tmem_ld_32x32b_x16(tbase + c * CW, r);
+          tmem_ld_wait();
+          if (c == BN / CW - 1) {
+            tc_fence_before();
+            mbar_arrive(smem_u32(acce_bar + acc));
+          }
+          if constexpr (KIND == Kind::Swap) store_col_chunk<CW>(g, ta * 128 + row, tb * BN + c * CW, r);
+          else if (m < g.M) store_row_chunk<CW>(g, m, tb * BN + c * CW, r, srow);
+        }
+      } else {
+        // Stream-K partial tile: add into the workspace (coalesced: one
+        // column of 128 rows is 512 contiguous bytes), then the last of the
+        // contributing CTAs finishes the tile.
+        int32_t* wt = g.ws + static_cast<int64_t>(s.tile) * BN * 128;
+#pragma unroll 1
+        for (int c = 0; c < BN / CW; ++c) {
+          uint32_t r[CW];
+          if constexpr (CW == 32) tmem_ld_32x32b_x32(tbase + c * CW, r);
+          else tmem_ld_32x32b_x16(tbase + c * CW, r);
+          tmem_ld_wait();
+          if (c == BN / CW - 1) {
+            tc_fence_before();
+            mbar_arrive(smem_u32(acce_bar + acc));
+          }
+#pragma unroll
+          for (int j = 0; j < CW; ++j) atomicAdd(wt + (c * CW + j) * 128 + row, static_cast<int>(r[j]));
+        }
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (ep_tid == 0) {
+          const uint32_t prev = atomicAdd(g.ws_cnt + s.tile, 1u);
+          *sk_last = (static_cast<int>(prev) == sk_contributors(g, s.tile) - 1) ? 1 : 0;
+        }
+        named_bar_sync(1, 128);
+        if (*sk_last) {
+          __threadfence();
+          float srow = 0.0f;
+          int m = 0;
+          if constexpr (KIND != Kind::Swap) {
+            m = ta * 128 + row;
+            if (!g.out_s32 && m < g.M) srow = __ldg(g.s_row + m);
+          }
+#pragma unroll 1
+          for (int c = 0; c < BN / CW; ++c) {
+            uint32_t r[CW];
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+              int32_t* p = wt + (c * CW + j) * 128 + row;
+              r[j] = static_cast<uint32_t>(__ldcg(p));
+              __stcg(p, 0);
+            }
+            if constexpr (KIND == Kind::Swap) store_col_chunk<CW>(g, ta * 128 + row, tb * BN + c * CW, r);
+            else if (m < g.M) store_row_chunk<CW>(g, m, tb * BN + c * CW, r, srow);
+          }
+          if (ep_tid == 0) g.ws_cnt[s.tile] = 0;
+        }
+        named_bar_sync(1, 128);   // sk_last is reused by the next partial tile
+      }
+      if (++acc == C::ACC_BUFS) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------- BSR pack
+
+__global__ void __launch_bounds__(256) bsr_pack_kernel(const int8_t* __restrict__ wq, int64_t K,
+                                                       const int32_t* __restrict__ crow,
+                                                       const int32_t* __restrict__ col, int nnzb,
+                                                       int nbc, int8_t* __restrict__ values) {
+  const int br = blockIdx.x;
+  int p0 = min(max(__ldg(crow + br), 0), nnzb);
+  int p1 = min(max(__ldg(crow + br + 1), p0), nnzb);
+  const int j = threadIdx.x >> 2;          // row inside the block (64 rows)
+  const int part = threadIdx.x & 3;        // 16-byte quarter of the 64-byte row
+  for (int p = p0; p < p1; ++p) {
+    const int c = __ldg(col + p);
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (c >= 0 && c < nbc)
+      v = __ldg(reinterpret_cast<const uint4*>(wq + (static_cast<int64_t>(br) * 64 + j) * K +
+                                               static_cast<int64_t>(c) * 64) + part);
+    reinterpret_cast<uint4*>(values + (static_cast<int64_t>(p) * 64 + j) * 64)[part] = v;
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+namespace {
+
+template <Kind KIND, int BN>
+dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, int grid,
+                 cudaStream_t stream) {
+  using C = Cfg<KIND, BN>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err);
+  gemm_kernel<KIND, BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ta, tb, args);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+constexpr int64_t kMaxK = 133144;   // floor((2^31 - 1) / 127^2): int32 accumulation is exact
+
+// Schedule override for measurements: 0 = automatic, 1 = whole tiles, 2 = stream-K.
+int g_schedule_override = 0;
+
+struct Plan {
+  Kind kind;
+  int bn;
+  int a_tiles, b_tiles, kb_total, num_tiles;
+  bool stream_k;
+  size_t ws_bytes;   // bytes needed for stream-K (0 if it never splits)
+};
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count) {
+  Plan p{};
+  if (M <= 128) {
+    p.kind = Kind::Swap;
+    p.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    p.a_tiles = static_cast<int>((N + 127) / 128);
+    p.b_tiles = static_cast<int>((M + p.bn - 1) / p.bn);
+  } else {
+    p.kind = Kind::Dense;
+    p.bn = N <= 128 ? 128 : 256;
+    p.a_tiles = static_cast<int>((M + 127) / 128);
+    p.b_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
+  }
+  p.kb_total = static_cast<int>((K + 127) / 128);
+  p.num_tiles = p.a_tiles * p.b_tiles;
+  const long long iters = static_cast<long long>(p.num_tiles) * p.kb_total;
+  // Stream-K pays when whole tiles would leave a large share of the SMs idle
+  // in the last wave, and every CTA still gets a few k blocks.
+  const int waves = (p.num_tiles + sm_count - 1) / sm_count;
+  const double eff = static_cast<double>(p.num_tiles) / (static_cast<double>(waves) * sm_count);
+  const bool worth = eff < 0.9 && iters >= 4LL * sm_count;
+  p.ws_bytes = worth ? static_cast<size_t>(p.num_tiles) * (static_cast<size_t>(p.bn) * 128 * 4 + 4) : 0;
+  p.stream_k = worth;
+  return p;
+}
+
+}  // namespace
+}  // namespace dq
+
+using namespace dq;
+
+extern "C" {
+
+size_t dq_int8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 1) return 0;
+  DeviceInfo* d = nullptr;
+  if (current_device(&d) != DQ_OK) return 0;
+  return make_plan(M, N, K, d->sm_count).ws_bytes;
+}
+
+// Measurement knob (not in the public header): force a schedule.
+void dq_debug_set_schedule(int mode) { g_schedule_override = mode; }
+
+dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K, const int8_t* W,
+                         const float* s_col, int64_t N, const void* bias_bf16, void* out,
+                         dq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                         dq_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (out_dtype != DQ_OUT_BF16 && out_dtype != DQ_OUT_S32) return DQ_ERR_INVALID_ARG;
+  if (M < 0 || K < 1 || N < 1) return DQ_ERR_INVALID_ARG;
+  if (M > 0 && (A == nullptr || W == nullptr || out == nullptr)) return DQ_ERR_INVALID_ARG;
+  if (M > 0 && out_dtype == DQ_OUT_BF16 && (s_row == nullptr || s_col == nullptr))
+    return DQ_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > kMaxK || N % 8 != 0) return DQ_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 128 || N > (int64_t(1) << 31) - 256) return DQ_ERR_UNSUPPORTED;
+  if (!aligned(A, 16) || !aligned(W, 16) || !aligned(out, 16)) return DQ_ERR_UNSUPPORTED;
+  if (out_dtype == DQ_OUT_BF16 && (!aligned(s_col, 16) || (bias_bf16 && !aligned(bias_bf16, 16))))
+    return DQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  dq_status st = current_device(&d);
+  if (st != DQ_OK) return st;
+  if (M == 0) return DQ_OK;
+
+  Plan p = make_plan(M, N, K, d->sm_count);
+  bool sk = p.stream_k && workspace != nullptr && workspace_bytes >= p.ws_bytes &&
+            aligned(workspace, 16);
+  if (g_schedule_override == 1) sk = false;
+  if (g_schedule_override == 2 && workspace != nullptr &&
+      workspace_bytes >= static_cast<size_t>(p.num_tiles) * (static_cast<size_t>(p.bn) * 128 * 4 + 4))
+    sk = static_cast<long long>(p.num_tiles) * p.kb_total >= d->sm_count;
+
+  CUtensorMap ta, tb;
+  const int8_t* a_src = p.kind == Kind::Swap ? W : A;
+  const int8_t* b_src = p.kind == Kind::Swap ? A : W;
+  const int64_t a_rows = p.kind == Kind::Swap ? N : M;
+  const int64_t b_rows = p.kind == Kind::Swap ? M : N;
+  if ((st = make_tmap_u8_2d(&ta, a_src, K, a_rows, K, 128, 128, 128)) != DQ_OK) return st;
+  if ((st = make_tmap_u8_2d(&tb, b_src, K, b_rows, K, 128, p.bn, 128)) != DQ_OK) return st;
+
+  GemmArgs g{};
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.a_tiles = p.a_tiles;
+  g.b_tiles = p.b_tiles;
+  g.kb_total = p.kb_total;
+  g.num_tiles = p.num_tiles;
+  g.stream_k = sk ? 1 : 0;
+  g.iters_total = static_cast<long long>(p.num_tiles) * p.kb_total;
+  g.s_row = s_row;
+  g.s_col = s_col;
+  g.bias = static_cast<const uint16_t*>(bias_bf16);
+  g.out = out;
+  g.out_s32 = out_dtype == DQ_OUT_S32 ? 1 : 0;
+  if (sk) {
+    g.ws = static_cast<int32_t*>(workspace);
+    g.ws_cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) +
+                                           static_cast<size_t>(p.num_tiles) * p.bn * 128 * 4);
+  }
+  g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
+  const int grid = sk ? d->sm_count : (p.num_tiles < d->sm_count ? p.num_tiles : d->sm_count);
+
+  if (p.kind == Kind::Dense) {
+    if (p.bn == 256) return launch<Kind::Dense, 256>(ta, tb, g, grid, stream);
+    return launch<Kind::Dense, 128>(ta, tb, g, grid, stream);
+  }
+  switch (p.bn) {
+    case 16: return launch<Kind::Swap, 16>(ta, tb, g, grid, stream);
+    case 32: return launch<Kind::Swap, 32>(ta, tb, g, grid, stream);
+    case 64: return launch<Kind::Swap, 64>(ta, tb, g, grid, stream);
+    default: return launch<Kind::Swap, 128>(ta, tb, g, grid, stream);
+  }
+}
+
+dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K, int64_t N,
+                             const int32_t* crow, const int32_t* col, const int8_t* values,
+                             int64_t nnzb, const float* s_col, const void* bias_bf16, void* out,
+                             dq_out_dtype out_dtype, dq_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (out_dtype != DQ_OUT_BF16 && out_dtype != DQ_OUT_S32) return DQ_ERR_INVALID_ARG;
+  if (M < 0 || K < 1 || N < 1 || nnzb < 0) return DQ_ERR_INVALID_ARG;
+  if (M > 0 && (A == nullptr || crow == nullptr || out == nullptr)) return DQ_ERR_INVALID_ARG;
+  if (M > 0 && nnzb > 0 && (col == nullptr || values == nullptr)) return DQ_ERR_INVALID_ARG;
+  if (M > 0 && out_dtype == DQ_OUT_BF16 && (s_row == nullptr || s_col == nullptr))
+    return DQ_ERR_INVALID_ARG;
+  if (K % 64 != 0 || N % 64 != 0 || K > 133120) return DQ_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 128 || N > (int64_t(1) << 31) - 256 || nnzb > (int64_t(1) << 24))
+    return DQ_ERR_UNSUPPORTED;
+  if (!aligned(A, 16) || !aligned(out, 16) || (values && !aligned(values, 16))) return DQ_ERR_UNSUPPORTED;
+  if (out_dtype == DQ_OUT_BF16 && (!aligned(s_col, 16) || (bias_bf16 && !aligned(bias_bf16, 16))))
+    return DQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  dq_status st = current_device(&d);
+  if (st != DQ_OK) return st;
+  if (M == 0) return DQ_OK;
+
+  CUtensorMap ta, tb;
+  if ((st = make_tmap_u8_2d(&ta, A, K, M, K, 64, 128, 64)) != DQ_OK) return st;
+  // With no blocks the B map is never read; describe A again to keep it valid.
+  if (nnzb > 0) st = make_tmap_u8_2d(&tb, values, 64, static_cast<uint64_t>(nnzb) * 64, 64, 64, 64, 64);
+  else st = make_tmap_u8_2d(&tb, A, K, M, K, 64, 64, 64);
+  if (st != DQ_OK) return st;
+
+  GemmArgs g{};
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.a_tiles = static_cast<int>((M + 127) / 128);
+  g.b_tiles = static_cast<int>(N / 64);
+  g.kb_total = 0;
+  const int64_t tiles = static_cast<int64_t>(g.a_tiles) * g.b_tiles;
+  if (tiles > 0x7fffffff) return DQ_ERR_UNSUPPORTED;
+  g.num_tiles = static_cast<int>(tiles);
+  g.stream_k = 0;
+  g.s_row = s_row;
+  g.s_col = s_col;
+  g.bias = static_cast<const uint16_t*>(bias_bf16);
+  g.out = out;
+  g.out_s32 = out_dtype == DQ_OUT_S32 ? 1 : 0;
+  g.crow = crow;
+  g.col = col;
+  g.nnzb = static_cast<int>(nnzb);
+  g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
+  const int grid = g.num_tiles < d->sm_count ? g.num_tiles : d->sm_count;
+  return launch<Kind::Bsr, 64>(ta, tb, g, grid, stream);
+}
+
+dq_status dq_bsr_pack(const int8_t* wq, int64_t N, int64_t K, const int32_t* crow, const int32_t* col,
+                      int64_t nnzb, int8_t* values, dq_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (N < 1 || K < 1 || nnzb < 0 || wq == nullptr || crow == nullptr) return DQ_ERR_INVALID_ARG;
+  if (nnzb > 0 && (col == nullptr || values == nullptr)) return DQ_ERR_INVALID_ARG;
+  if (K % 64 != 0 || N % 64 != 0 || nnzb > (int64_t(1) << 24)) return DQ_ERR_UNSUPPORTED;
+  if (!aligned(wq, 16) || (values && !aligned(values, 16))) return DQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  dq_status st = current_device(&d);
+  if (st != DQ_OK) return st;
+  if (nnzb == 0) return DQ_OK;
+  bsr_pack_kernel<<<static_cast<unsigned>(N / 64), 256, 0, stream>>>(wq, K, crow, col,
+                                                                     static_cast<int>(nnzb),
+                                                                     static_cast<int>(K / 64), values);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+dq_status dq_bsr_validate(const int32_t* crow, const int32_t* col, int64_t N, int64_t K, int64_t nnzb) {
+  if (crow == nullptr || N < 1 || K < 1 || nnzb < 0 || N % 64 != 0 || K % 64 != 0)
+    return DQ_ERR_INVALID_ARG;
+  if (nnzb > 0 && col == nullptr) return DQ_ERR_INVALID_ARG;
+  const int64_t nbr = N / 64;
+  int32_t* hc = new int32_t[nbr + 1];
+  int32_t* hk = nnzb > 0 ? new int32_t[nnzb] : nullptr;
+  dq_status st = DQ_OK;
+  cudaError_t e = cudaMemcpy(hc, crow, (nbr + 1) * sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && nnzb > 0) e = cudaMemcpy(hk, col, nnzb * sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) {
+    st = cuda_fail(e);
+  } else {
+    if (hc[0] != 0 || hc[nbr] != nnzb) st = DQ_ERR_INVALID_ARG;
+    for (int64_t b = 0; st == DQ_OK && b < nbr; ++b)
+      if (hc[b + 1] < hc[b]) st = DQ_ERR_INVALID_ARG;
+    for (int64_t p = 0; st == DQ_OK && p < nnzb; ++p)
+      if (hk[p] < 0 || hk[p] >= K / 64) st = DQ_ERR_INVALID_ARG;
+  }
+  delete[] hc;
+  delete[] hk;
+  return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,46 @@
+// internal.h -- host-side helpers shared by the libdq translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/dq.h"
+
+namespace dq {
+
+// Per-device facts, filled on the first call that touches a device.
+struct DeviceInfo {
+  int device = -1;
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+  size_t max_smem_optin = 0;
+  uint32_t* err_word = nullptr;   // device address of the per-device error word
+};
+
+// Resolves the current device's info; DQ_ERR_UNSUPPORTED if it is not sm_100.
+dq_status current_device(DeviceInfo** out);
+
+// Records a CUDA error for dq_last_cuda_error() and returns DQ_ERR_CUDA.
+dq_status cuda_fail(cudaError_t e);
+
+// Launch-time wait limit (ns) for bounded waits.
+unsigned long long wait_timeout_ns();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+// 2-D, uint8 elements: dims {inner, outer}, outer stride in bytes, box
+// {box_inner, box_outer}, swizzle = 128 or 64 (bytes), zero fill out of bounds.
+dq_status make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                          uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                          int swizzle_bytes);
+
+inline bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+}  // namespace dq
+
+// Measurement knob, not part of the public header: 0 = automatic schedule,
+// 1 = whole tiles only, 2 = stream-K whenever a workspace allows it.
+extern "C" DQ_API void dq_debug_set_schedule(int mode);

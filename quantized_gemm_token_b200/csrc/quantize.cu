@@ -1,0 +1,232 @@
+// quantize.cu -- per-row symmetric absmax int8 quantization.
+//
+// Per-token dynamic quantization of activations ("int8 dynamic quant + bsr
+// support", pytorch/ao PR 821) with the absmax/127 symmetric scale (Paddle
+// "sparse_fc supported", PR 41770, SpmmPluginDynamic), and the same formula
+// per output channel for the weight:
+//     s = fp32( max(absmax, 1e-8f) / 127 ),  q = clamp(rint(x / s), -127, 127)
+// with IEEE round-to-nearest-even division (no reciprocal): the result is
+// bit-identical to a scalar IEEE evaluation.
+//
+// The hot kernel keeps a whole row in registers: each row is owned by a
+// power-of-two group of 32..256 threads, each thread loads up to 8 16-byte
+// vectors (one HBM pass), the group reduces |x| with integer max on the bit
+// patterns (exact for finite values: a non-negative IEEE value orders like its
+// bits), and the codes are written straight from registers.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace dq {
+namespace {
+
+template <typename T>
+struct Elem;
+template <>
+struct Elem<uint16_t> {          // bf16 bit patterns
+  static constexpr int kPerVec = 8;
+  __device__ static float to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+};
+template <>
+struct Elem<float> {
+  static constexpr int kPerVec = 4;
+};
+
+__device__ __forceinline__ int8_t quant_one(float v, float s) {
+  int r = __float2int_rn(__fdiv_rn(v, s));     // rint(fp32(v / s)), ties to even
+  r = r > 127 ? 127 : (r < -127 ? -127 : r);
+  return static_cast<int8_t>(r);
+}
+
+__device__ __forceinline__ float scale_from_absmax(float a) {
+  return __fdiv_rn(fmaxf(a, 1e-8f), 127.0f);
+}
+
+__device__ __forceinline__ uint32_t pack4(int8_t a, int8_t b, int8_t c, int8_t d) {
+  return (static_cast<uint32_t>(static_cast<uint8_t>(a))) |
+         (static_cast<uint32_t>(static_cast<uint8_t>(b)) << 8) |
+         (static_cast<uint32_t>(static_cast<uint8_t>(c)) << 16) |
+         (static_cast<uint32_t>(static_cast<uint8_t>(d)) << 24);
+}
+
+// Register-resident single-pass kernel.  256 threads; a row is owned by
+// 2^tpr_log2 consecutive threads (32..256); VPT = max 16-byte vectors per
+// thread.
+template <typename T, int VPT>
+__global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict__ x, int64_t M,
+                                                             int64_t K, int64_t ldx,
+                                                             int8_t* __restrict__ q, int64_t ldq,
+                                                             float* __restrict__ scales,
+                                                             int tpr_log2) {
+  constexpr int E = Elem<T>::kPerVec;
+  const int tpr = 1 << tpr_log2;
+  const int t = threadIdx.x & (tpr - 1);
+  const int r_local = threadIdx.x >> tpr_log2;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (256 >> tpr_log2) + r_local;
+  const int nv = static_cast<int>(K / E);
+  __shared__ uint32_t warp_max[8];
+
+  uint4 v[VPT];
+  uint32_t amax = 0;
+  if (row < M) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int vi = t + i * tpr;
+      if (vi < nv) v[i] = __ldcs(xr + vi);
+    }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int vi = t + i * tpr;
+      if (vi < nv) {
+        if constexpr (E == 8) {
+          amax = __vmaxu2(amax, v[i].x & 0x7fff7fffu);
+          amax = __vmaxu2(amax, v[i].y & 0x7fff7fffu);
+          amax = __vmaxu2(amax, v[i].z & 0x7fff7fffu);
+          amax = __vmaxu2(amax, v[i].w & 0x7fff7fffu);
+        } else {
+          amax = max(amax, v[i].x & 0x7fffffffu);
+          amax = max(amax, v[i].y & 0x7fffffffu);
+          amax = max(amax, v[i].z & 0x7fffffffu);
+          amax = max(amax, v[i].w & 0x7fffffffu);
+        }
+      }
+    }
+    if constexpr (E == 8) amax = max(amax & 0xffffu, amax >> 16) << 16;   // to fp32 bits
+  }
+  amax = __reduce_max_sync(0xffffffffu, amax);
+  if (tpr > 32) {
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) warp_max[warp] = amax;
+    __syncthreads();
+    const int wpr = tpr >> 5;
+    const int w0 = r_local * wpr;
+    amax = 0;
+    for (int w = 0; w < wpr; ++w) amax = max(amax, warp_max[w0 + w]);
+  }
+  if (row >= M) return;
+  const float s = scale_from_absmax(__uint_as_float(amax));
+  if (t == 0) scales[row] = s;
+
+  int8_t* qr = q + row * ldq;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int vi = t + i * tpr;
+    if (vi < nv) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      if constexpr (E == 8) {
+        uint32_t out[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t a = w[2 * h], b = w[2 * h + 1];
+          out[h] = pack4(quant_one(__uint_as_float(a << 16), s),
+                         quant_one(__uint_as_float(a & 0xffff0000u), s),
+                         quant_one(__uint_as_float(b << 16), s),
+                         quant_one(__uint_as_float(b & 0xffff0000u), s));
+        }
+        *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(vi) * 8) = make_uint2(out[0], out[1]);
+      } else {
+        *reinterpret_cast<uint32_t*>(qr + static_cast<int64_t>(vi) * 4) =
+            pack4(quant_one(__uint_as_float(w[0]), s), quant_one(__uint_as_float(w[1]), s),
+                  quant_one(__uint_as_float(w[2]), s), quant_one(__uint_as_float(w[3]), s));
+      }
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float load_as_float(const T* p);
+template <>
+__device__ __forceinline__ float load_as_float<uint16_t>(const uint16_t* p) {
+  return __uint_as_float(static_cast<uint32_t>(*p) << 16);
+}
+template <>
+__device__ __forceinline__ float load_as_float<float>(const float* p) {
+  return *p;
+}
+
+// Any shape, stride or alignment: one CTA of 256 threads per row, two passes
+// over the row (the second mostly from L2).
+template <typename T>
+__global__ void __launch_bounds__(256) quant_rows_generic_kernel(const T* __restrict__ x, int64_t M,
+                                                                 int64_t K, int64_t ldx,
+                                                                 int8_t* __restrict__ q,
+                                                                 int64_t ldq,
+                                                                 float* __restrict__ scales) {
+  __shared__ float warp_max[8];
+  for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+    const T* xr = x + row * ldx;
+    float a = 0.0f;
+    for (int64_t k = threadIdx.x; k < K; k += 256) a = fmaxf(a, fabsf(load_as_float<T>(xr + k)));
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = a;
+    __syncthreads();
+    a = warp_max[0];
+    for (int w = 1; w < 8; ++w) a = fmaxf(a, warp_max[w]);
+    __syncthreads();
+    const float s = scale_from_absmax(a);
+    if (threadIdx.x == 0) scales[row] = s;
+    int8_t* qr = q + row * ldq;
+    for (int64_t k = threadIdx.x; k < K; k += 256) qr[k] = quant_one(load_as_float<T>(xr + k), s);
+  }
+}
+
+template <typename T>
+dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
+                          float* scales, cudaStream_t stream) {
+  if (M < 0 || K < 1 || ldx < K || ldq < K) return DQ_ERR_INVALID_ARG;
+  if (M > 0 && (x == nullptr || q == nullptr || scales == nullptr)) return DQ_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 31) - 1) return DQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  dq_status st = current_device(&d);
+  if (st != DQ_OK) return st;
+  if (M == 0) return DQ_OK;
+
+  constexpr int E = Elem<T>::kPerVec;
+  const int64_t nv = K / E;
+  const bool vec_ok = (K % E == 0) && (ldx % E == 0) && aligned(x, 16) && (ldq % E == 0) &&
+                      aligned(q, E) && nv <= 256 * 8;
+  if (vec_ok) {
+    int tpr_log2 = 5;
+    while ((int64_t(1) << tpr_log2) * 8 < nv) ++tpr_log2;     // tpr * 8 >= nv, tpr <= 256
+    const int64_t tpr = int64_t(1) << tpr_log2;
+    const int64_t vpt = (nv + tpr - 1) / tpr;
+    const int64_t rows_per_cta = 256 / tpr;
+    const int64_t grid = (M + rows_per_cta - 1) / rows_per_cta;
+    if (grid > 0x7fffffff) return DQ_ERR_UNSUPPORTED;
+    dim3 g(static_cast<unsigned>(grid));
+    if (vpt <= 1)
+      quant_rows_vec_kernel<T, 1><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+    else if (vpt <= 2)
+      quant_rows_vec_kernel<T, 2><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+    else if (vpt <= 4)
+      quant_rows_vec_kernel<T, 4><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+    else
+      quant_rows_vec_kernel<T, 8><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+  } else {
+    const int64_t grid = M < int64_t(d->sm_count) * 16 ? M : int64_t(d->sm_count) * 16;
+    quant_rows_generic_kernel<T><<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, M, K, ldx, q,
+                                                                                 ldq, scales);
+  }
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+}  // namespace
+}  // namespace dq
+
+extern "C" {
+
+dq_status dq_quantize_rows(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q,
+                           int64_t ldq, float* scales, dq_stream_t stream) {
+  return dq::launch_quantize<uint16_t>(static_cast<const uint16_t*>(x_bf16), M, K, ldx, q, ldq,
+                                       scales, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dq_status dq_quantize_weight(const float* w, int64_t N, int64_t K, int64_t ldw, int8_t* wq,
+                             int64_t ldwq, float* s_col, dq_stream_t stream) {
+  return dq::launch_quantize<float>(w, N, K, ldw, wq, ldwq, s_col,
+                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,346 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bit-exact for int8 codes, fp32 scales and int32 accumulators; bf16 outputs
+within 1 bf16 ulp (they are expected to be identical: both sides evaluate
+acc * s_row * s_col + bias left to right with one IEEE rounding per op).
+Sizes span several tiles with ragged tails; the five workloads run at full
+size with the oracle checked on sampled rows / channels.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import assert_bf16_close, bf16_bits, sample_rows, to_dev, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+dq = pytest.importorskip("quantized_gemm_token_b200") if torch.cuda.is_available() else None
+
+
+@pytest.fixture(autouse=True)
+def _sync_and_check():
+    yield
+    if torch.cuda.is_available():
+        assert dq.dq_sync_status() == dq.DQ_OK
+        dq.dq_debug_set_schedule(0)
+
+
+def _bits(a):
+    return synth.f32_to_bf16_bits(np.asarray(a, np.float32))
+
+
+# ---------------------------------------------------------------- quantize
+
+QSHAPES = [(1, 8, 8), (3, 16, 16), (64, 256, 256), (7, 1280, 1280), (5, 4096, 4096), (9, 5120, 5120),
+           (2, 8192, 8192), (3, 16384, 16384), (2, 16392, 16392), (4, 1000, 1000), (3, 8, 24),
+           (5, 64, 72), (300, 136, 136), (0, 64, 64)]
+
+
+@pytest.mark.parametrize("M,K,ldx", QSHAPES)
+def test_quantize_rows_parity(M, K, ldx):
+    x = synth.normal_bf16((max(M, 1), ldx), 1.0, 100 + K)[:M]
+    if M >= 3:
+        x[0, :K] = 0                                     # all-zero row
+        x[1, :K] = synth.normal_bf16((K,), 1e-9, 7)      # below eps
+        x[2, :K] = _bits(np.arange(K) % 7 - 3.5)         # exact ties at scale 1/..
+    xd = to_dev_bf16(x)
+    xv = xd.as_strided((M, K), (ldx, 1)) if M else xd[:, :K]
+    q, s = dq.dq_quantize_rows(xv)
+    qo, so = oracle.quantize_rows_bf16(np.ascontiguousarray(x[:, :K]))
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+def test_quantize_full_size_16384x8192():
+    d = synth.quant_sweep(0)
+    q, s = dq.dq_quantize_rows(to_dev_bf16(d["x"]))
+    qo, so = oracle.quantize_rows_bf16(d["x"])
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+@pytest.mark.parametrize("N,K", [(256, 256), (5120, 1280), (64, 100), (33, 4096)])
+def test_quantize_weight_parity(N, K):
+    w = synth.normal_f32((N, K), 0.02, 200 + K)
+    w[0] = 0
+    wq, sc = dq.dq_quantize_weight(to_dev(w))
+    wo, so = oracle.quantize_rows_f32(w)
+    assert np.array_equal(wq.cpu().numpy(), wo)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+def test_worked_example_through_the_abi():
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_4x4.json")))
+    # pad K to 16 (the GEMM needs K % 16 == 0); zeros change neither absmax nor sums
+    x = np.zeros((4, 16), np.float32)
+    x[:, :4] = g["x"]
+    w = np.zeros((8, 16), np.float32)
+    w[:4, :4] = g["w"]
+    bias = np.zeros(8, np.float32)
+    bias[:4] = g["bias"]
+    q, s = dq.dq_quantize_rows(to_dev_bf16(_bits(x)))
+    wq, sc = dq.dq_quantize_weight(to_dev(w))
+    assert q.cpu().numpy()[:, :4].tolist() == g["q"]
+    assert wq.cpu().numpy()[:4, :4].tolist() == g["w_q"]
+    acc = dq.dq_int8_linear(q, s, wq, sc, out_dtype="s32")
+    assert acc.cpu().numpy()[:, :4].tolist() == g["acc"]
+    out = dq.dq_int8_linear(q, s, wq, sc, bias=to_dev_bf16(_bits(bias)))
+    assert synth.bf16_bits_to_f32(bf16_bits(out))[:, :4].tolist() == g["out"]
+
+
+# ---------------------------------------------------------------- dense GEMM
+
+GSHAPES = [(1, 8, 16), (16, 64, 64), (17, 136, 144), (63, 256, 128), (64, 256, 256), (65, 264, 384),
+           (127, 520, 256), (128, 128, 1024), (129, 8, 128), (200, 256, 128), (255, 264, 640),
+           (300, 520, 384), (513, 1032, 256), (1000, 256, 4096), (200, 520, 8192), (33, 1032, 8192)]
+
+
+def _gemm_inputs(M, N, K, seed):
+    A = synth.uniform_int8((M, K), -127, 127, seed)
+    W = synth.uniform_int8((N, K), -127, 127, seed + 1)
+    s_row = synth.uniform_f32((M,), 0.001, 0.05, seed + 5)
+    s_col = synth.uniform_f32((N,), 0.001, 0.05, seed + 6)
+    bias = synth.normal_bf16((N,), 0.1, seed + 2)
+    return A, W, s_row, s_col, bias
+
+
+@pytest.mark.parametrize("schedule", [1, 2])
+@pytest.mark.parametrize("M,N,K", GSHAPES)
+def test_dense_parity(M, N, K, schedule):
+    A, W, s_row, s_col, bias = _gemm_inputs(M, N, K, 300 + M + N + K)
+    dq.dq_debug_set_schedule(schedule)
+    Ad, Wd = to_dev(A), to_dev(W)
+    ws = torch.zeros(64 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    acc = dq.dq_int8_linear(Ad, None, Wd, None, out_dtype="s32", workspace=ws)
+    want = oracle.gemm_s32(A, W)
+    assert np.array_equal(acc.cpu().numpy(), want)
+    for b in (None, bias):
+        out = dq.dq_int8_linear(Ad, to_dev(s_row), Wd, to_dev(s_col),
+                                bias=None if b is None else to_dev_bf16(b), workspace=ws)
+        assert_bf16_close(bf16_bits(out), oracle.epilogue_bf16(want, s_row, s_col, b))
+    # the workspace is left zeroed by every completed call
+    assert int(ws.count_nonzero()) == 0
+
+
+def test_stream_k_and_whole_tiles_agree():
+    for (M, N, K) in ((2048, 4096, 4096), (16, 28672, 2048), (128, 4096, 1024)):
+        A, W, s_row, s_col, _ = _gemm_inputs(M, N, K, 7)
+        Ad, Wd = to_dev(A), to_dev(W)
+        ws = torch.zeros(dq.dq_int8_linear_workspace_size(M, N, K) or 1 << 20, dtype=torch.uint8, device="cuda")
+        outs = []
+        for mode in (1, 2):
+            dq.dq_debug_set_schedule(mode)
+            outs.append(dq.dq_int8_linear(Ad, None, Wd, None, out_dtype="s32", workspace=ws).cpu().numpy())
+        assert np.array_equal(outs[0], outs[1])
+        rows = sample_rows(M, 24)
+        assert np.array_equal(outs[0][rows], oracle.gemm_s32(A[rows], W))
+
+
+def test_identity_weight_returns_quantized_activations():
+    K = 256
+    x = synth.normal_bf16((300, K), 1.0, 9)
+    q, _ = dq.dq_quantize_rows(to_dev_bf16(x))
+    wq, sc = dq.dq_quantize_weight(torch.eye(K, dtype=torch.float32, device="cuda"))
+    assert torch.equal(wq, 127 * torch.eye(K, dtype=torch.int8, device="cuda"))
+    acc = dq.dq_int8_linear(q, None, wq, None, out_dtype="s32")
+    assert torch.equal(acc, 127 * q.to(torch.int32))
+
+
+def test_output_canaries_untouched():
+    M, N, K = 129, 264, 128
+    A, W, s_row, s_col, bias = _gemm_inputs(M, N, K, 11)
+    big = torch.full((M * N + 2 * 4096,), 0x5A5A, dtype=torch.int16, device="cuda")
+    out = big[4096:4096 + M * N].view(torch.bfloat16).view(M, N)
+    dq.dq_int8_linear(to_dev(A), to_dev(s_row), to_dev(W), to_dev(s_col), bias=to_dev_bf16(bias), out=out)
+    assert int((big[:4096] != 0x5A5A).sum()) == 0 and int((big[-4096:] != 0x5A5A).sum()) == 0
+    assert_bf16_close(bf16_bits(out), oracle.linear_bf16(A, s_row, W, s_col, bias))
+
+
+# ---------------------------------------------------------------- layer configs
+
+def _frob(x_bits, w, out_bits, bias_bits=None):
+    ref = synth.bf16_bits_to_f32(x_bits).astype(np.float64) @ w.astype(np.float64).T
+    if bias_bits is not None:
+        ref += synth.bf16_bits_to_f32(bias_bits).astype(np.float64)
+    got = synth.bf16_bits_to_f32(out_bits).astype(np.float64)
+    return float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+
+
+def _layer_gpu(x, w, bias=None):
+    wq, sc = dq.dq_quantize_weight(to_dev(w))
+    q, s = dq.dq_quantize_rows(to_dev_bf16(x))
+    M, N, K = x.shape[0], w.shape[0], w.shape[1]
+    n = dq.dq_int8_linear_workspace_size(M, N, K)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda") if n else None
+    out = dq.dq_int8_linear(q, s, wq, sc, bias=None if bias is None else to_dev_bf16(bias), workspace=ws)
+    return q, s, wq, sc, out
+
+
+def test_config_tiny_layer():
+    d = synth.tiny(0)
+    q, s, wq, sc, out = _layer_gpu(d["x"], d["w"], d["bias"])
+    want, qo, so = oracle.dynamic_linear_bf16(d["x"], *oracle.quantize_rows_f32(d["w"]), d["bias"])
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(wq.cpu().numpy(), oracle.quantize_rows_f32(d["w"])[0])
+    assert_bf16_close(bf16_bits(out), want)
+    assert _frob(d["x"], d["w"], bf16_bits(out), d["bias"]) <= 2e-2
+
+
+def test_config_llm_layer_2048x4096x4096():
+    d = synth.llm(0)
+    q, s, wq, sc, out = _layer_gpu(d["x"], d["w"])
+    qo, so = oracle.quantize_rows_bf16(d["x"])
+    wo, sco = oracle.quantize_rows_f32(d["w"])
+    assert np.array_equal(q.cpu().numpy(), qo) and np.array_equal(wq.cpu().numpy(), wo)
+    assert np.array_equal(s.cpu().numpy(), so) and np.array_equal(sc.cpu().numpy(), sco)
+    rows = sample_rows(2048, 48)
+    want = oracle.linear_bf16(qo[rows], so[rows], wo, sco)
+    got = bf16_bits(out)
+    assert_bf16_close(got[rows], want)
+    # accuracy vs the unquantized fp32 product: reported, not gated (outliers)
+    e = _frob(d["x"][rows], d["w"], got[rows])
+    assert 3e-2 < e < 8e-2
+
+
+def test_config_large_m_38400x1024x4096():
+    d = synth.large_m(0)
+    A, B = to_dev(d["a"]), to_dev(d["b"])
+    acc = dq.dq_int8_linear(A, None, B, None, out_dtype="s32")
+    out = dq.dq_int8_linear(A, to_dev(d["s_row"]), B, to_dev(d["s_col"]))
+    rows = sample_rows(38400, 40)
+    want = oracle.gemm_s32(d["a"][rows], d["b"])
+    assert np.array_equal(acc.cpu().numpy()[rows], want)
+    assert_bf16_close(bf16_bits(out)[rows], oracle.epilogue_bf16(want, d["s_row"][rows], d["s_col"]))
+    # int32 and bf16 modes agree everywhere through the epilogue definition on GPU data
+    acc_np = acc.cpu().numpy()
+    rows2 = sample_rows(38400, 200, seed=3)
+    assert_bf16_close(bf16_bits(out)[rows2], oracle.epilogue_bf16(acc_np[rows2], d["s_row"][rows2], d["s_col"]))
+
+
+@pytest.mark.parametrize("M", [1, 16, 128])
+def test_config_small_m(M):
+    d = synth.small_m(0, M=M)
+    q, s, wq, sc, out = _layer_gpu(d["x"], d["w"])
+    qo, so = oracle.quantize_rows_bf16(d["x"])
+    assert np.array_equal(q.cpu().numpy(), qo)
+    wq_np = wq.cpu().numpy()
+    ch = np.unique(np.concatenate([np.arange(0, 28672, 97), [0, 127, 128, 28543, 28671]]))
+    wo, sco = oracle.quantize_rows_f32(d["w"][ch])
+    assert np.array_equal(wq_np[ch], wo)
+    want = oracle.linear_bf16(qo, so, wo, sco)
+    got = bf16_bits(out)[:, ch]
+    assert_bf16_close(got, want)
+    assert _frob(d["x"], d["w"][ch], got) <= 2e-2
+
+
+# ---------------------------------------------------------------- BSR
+
+def _bsr_gpu(d):
+    wq, sc = dq.dq_quantize_weight(to_dev(d["w"]))
+    crow, col = to_dev(d["crow"]), to_dev(d["col"])
+    values = dq.dq_bsr_pack(wq, crow, col)
+    return wq, sc, crow, col, values
+
+
+@pytest.mark.parametrize("layer", ["fc1", "fc2"])
+def test_config_vit_h_bsr(layer):
+    d = synth.vit_h_bsr(0, layer)
+    M, N, K = d["M"], d["N"], d["K"]
+    wq, sc, crow, col, values = _bsr_gpu(d)
+    wo, sco = oracle.quantize_rows_f32(d["w"])
+    assert np.array_equal(wq.cpu().numpy(), wo)
+    vo = oracle.bsr_pack(wo, d["crow"], d["col"])
+    assert np.array_equal(values.cpu().numpy(), vo)
+    assert dq.dq_bsr_validate(crow, col, N, K) == dq.DQ_OK
+    q, s = dq.dq_quantize_rows(to_dev_bf16(d["x"]))
+    out = dq.dq_bsr_int8_linear(q, s, N, crow, col, values, sc)
+    acc = dq.dq_bsr_int8_linear(q, s, N, crow, col, values, sc, out_dtype="s32")
+    rows = sample_rows(M, 48)
+    qo, so = oracle.quantize_rows_bf16(d["x"][rows])
+    assert np.array_equal(q.cpu().numpy()[rows], qo)
+    acc_o = oracle.bsr_gemm_s32(qo, N, d["crow"], d["col"], vo)
+    assert np.array_equal(acc.cpu().numpy()[rows], acc_o)
+    got = bf16_bits(out)
+    assert_bf16_close(got[rows], oracle.epilogue_bf16(acc_o, so, sco))
+    # BSR == dense GEMM on the densified (masked) weight, everywhere, bit for bit
+    dense = dq.dq_int8_linear(q, s, wq, sc)
+    assert torch.equal(dense.view(torch.int16), out.view(torch.int16))
+    # accuracy vs the masked fp32 weight
+    assert _frob(d["x"][rows], d["w"], got[rows]) <= 2e-2
+
+
+def _random_bsr(N, K, keep, seed, empty_rows=(), dup=False):
+    crow, col = synth.bsr_pattern(N // 64, K // 64, keep, seed)
+    counts = np.diff(crow)
+    cols = [list(col[crow[b]:crow[b + 1]]) for b in range(N // 64)]
+    for b in empty_rows:
+        cols[b] = []
+    if dup and cols[0]:
+        cols[0].append(cols[0][0])
+    counts = [len(c) for c in cols]
+    crow = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    col = np.array([c for cs in cols for c in cs], np.int32)
+    values = synth.uniform_int8((len(col), 64, 64), -127, 127, seed + 1)
+    return crow, col, values
+
+
+@pytest.mark.parametrize("case", ["empty_rows", "no_blocks", "dense", "duplicates", "ragged_m"])
+def test_bsr_edge_cases(case):
+    M, N, K = {"ragged_m": (1, 256, 192)}.get(case, (300, 320, 256))
+    keep = {"dense": 1.0, "no_blocks": 0.0}.get(case, 0.3)
+    crow, col, values = _random_bsr(N, K, keep, 500, empty_rows=(1, 3) if case == "empty_rows" else (),
+                                    dup=case == "duplicates")
+    A = synth.uniform_int8((M, K), -127, 127, 501)
+    s_row = synth.uniform_f32((M,), 0.001, 0.05, 505)
+    s_col = synth.uniform_f32((N,), 0.001, 0.05, 506)
+    bias = synth.normal_bf16((N,), 0.1, 502)
+    vd = to_dev(values) if len(col) else torch.empty((0, 64, 64), dtype=torch.int8, device="cuda")
+    cd = to_dev(col) if len(col) else torch.empty((0,), dtype=torch.int32, device="cuda")
+    acc = dq.dq_bsr_int8_linear(to_dev(A), None, N, to_dev(crow), cd, vd, None, out_dtype="s32")
+    want = oracle.bsr_gemm_s32(A, N, crow, col, values)
+    assert np.array_equal(acc.cpu().numpy(), want)
+    out = dq.dq_bsr_int8_linear(to_dev(A), to_dev(s_row), N, to_dev(crow), cd, vd, to_dev(s_col),
+                                bias=to_dev_bf16(bias))
+    assert_bf16_close(bf16_bits(out), oracle.epilogue_bf16(want, s_row, s_col, bias))
+    if case == "duplicates":
+        assert dq.dq_bsr_validate(to_dev(crow), cd, N, K) == dq.DQ_OK
+
+
+def test_bsr_validate_rejects_malformed():
+    crow = to_dev(np.array([0, 2, 1, 3], np.int32))
+    col = to_dev(np.array([0, 1, 2], np.int32))
+    assert dq.dq_bsr_validate(crow, col, 192, 192) == dq.DQ_ERR_INVALID_ARG
+    crow = to_dev(np.array([0, 1, 2, 3], np.int32))
+    col = to_dev(np.array([0, 1, 5], np.int32))
+    assert dq.dq_bsr_validate(crow, col, 192, 192) == dq.DQ_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- failure path
+
+def test_bounded_wait_times_out_and_context_survives():
+    dq.dq_set_wait_timeout_ns(20_000_000)          # 20 ms
+    try:
+        dq.dq_selftest_wait_timeout()
+        assert dq.dq_sync_status() == dq.DQ_ERR_TIMEOUT
+        assert dq.dq_sync_status() == dq.DQ_OK       # cleared
+    finally:
+        dq.dq_set_wait_timeout_ns(0)
+    # the context is still usable
+    A, W, s_row, s_col, bias = _gemm_inputs(64, 64, 64, 13)
+    acc = dq.dq_int8_linear(to_dev(A), None, to_dev(W), None, out_dtype="s32")
+    assert np.array_equal(acc.cpu().numpy(), oracle.gemm_s32(A, W))
+
+
+def test_non_contiguous_and_misaligned_rejected():
+    A = torch.zeros((64, 80), dtype=torch.int8, device="cuda")[:, 8:72]
+    W = torch.zeros((64, 64), dtype=torch.int8, device="cuda")
+    with pytest.raises(ValueError):
+        dq.dq_int8_linear(A, None, W, None, out_dtype="s32")
+    base = torch.zeros((64 * 64 + 1,), dtype=torch.int8, device="cuda")
+    A2 = base[1:].view(64, 64)
+    with pytest.raises(dq.DQError):
+        dq.dq_int8_linear(A2, None, W, None, out_dtype="s32")
