@@ -152,6 +152,41 @@ DQ_API dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, 
 DQ_API size_t dq_int8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* ------------------------------------------------------------------------
+ * Allocation-free variant of dq_int8_linear (the pages have no counterpart;
+ * this is an interface convenience of libdq).
+ *
+ * Some callers cannot call cudaMalloc or own any device buffer to lend: a
+ * plugin running inside an inference engine whose memory planner owns all
+ * device memory, code that runs while another component is capturing a CUDA
+ * graph (where an allocation would break the capture), or a latency-bound
+ * caller that cannot afford the device-wide synchronisation cudaMalloc and
+ * cudaFree can cause.  For them this entry point takes the same arguments as
+ * dq_int8_linear minus the workspace: the stream-K scratch it needs lives in
+ * a file-scope static device array of DQ_NOALLOC_SCRATCH_BYTES (32 MiB) that
+ * every GPU which loads libdq holds until the process exits.  The caller still
+ * passes inputs and outputs.  Nothing here calls cudaMalloc, cudaFree or any
+ * allocating library routine.
+ *
+ *  - If the chosen schedule needs more scratch than DQ_NOALLOC_SCRATCH_BYTES
+ *    (dq_int8_linear_workspace_size(M, N, K) > DQ_NOALLOC_SCRATCH_BYTES), the
+ *    call launches nothing and returns DQ_ERR_UNSUPPORTED.
+ *  - The first call on a device looks up the array's device address for that
+ *    device (cudaGetSymbolAddress, with that device current); make that first
+ *    call before any stream capture.
+ *  - Each call clears the part of the array it uses (cudaMemsetAsync on
+ *    `stream`) before the GEMM, because the array keeps the previous call's
+ *    contents.  All calls on a device share the one array: two calls whose
+ *    work overlaps on the GPU (different streams, no ordering between them)
+ *    race on it and may produce wrong results.  Serialise them.
+ *  - Everything else (requirements, results, errors) is as dq_int8_linear.
+ * ------------------------------------------------------------------------ */
+#define DQ_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+DQ_API dq_status dq_int8_linear_noalloc(const int8_t* A, const float* s_row, int64_t M, int64_t K,
+                                        const int8_t* W, const float* s_col, int64_t N,
+                                        const void* bias_bf16, void* out, dq_out_dtype out_dtype,
+                                        dq_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Block-sparse (BSR) int8 linear, 64x64 blocks (pytorch/ao PR 821: the
  * kernel takes crow_indices / col_indices / values directly; vit_h_14
  * benchmark with --bsr 64).

@@ -35,6 +35,7 @@ _PROTOS = {
     "dq_quantize_weight": (_I32, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "dq_int8_linear": (_I32, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P, _I32, _P, _SZ, _P]),
     "dq_int8_linear_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "dq_int8_linear_noalloc": (_I32, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P, _I32, _P]),
     "dq_bsr_int8_linear": (_I32, [_P, _P, _I64, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _I32, _P]),
     "dq_bsr_pack": (_I32, [_P, _I64, _I64, _P, _P, _I64, _P, _P]),
     "dq_bsr_validate": (_I32, [_P, _P, _I64, _I64, _I64]),
@@ -209,6 +210,22 @@ def dq_int8_linear(A, s_row, W, s_col, bias=None, out=None, out_dtype="bf16", wo
         ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()
     _check(lib.dq_int8_linear(_ptr(A), _ptr(s_row), M, K, _ptr(W), _ptr(s_col), N, _ptr(bias), _ptr(out),
                               code, ws_ptr, ws_bytes, _stream(stream)), "dq_int8_linear")
+    return out
+
+
+DQ_NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def dq_int8_linear_noalloc(A, s_row, W, s_col, out, bias=None, out_dtype="bf16", stream=None):
+    """dq_int8_linear for callers that cannot allocate: the split-K scratch
+    comes from libdq's static 32 MiB device array (see include/dq.h), and the
+    caller passes a preallocated `out`.  Calls that overlap on the GPU race on
+    that array; the first call on a device must precede any stream capture."""
+    code = _out_code(out_dtype)
+    M, K = A.shape
+    N = W.shape[0]
+    _check(lib.dq_int8_linear_noalloc(_ptr(A), _ptr(s_row), M, K, _ptr(W), _ptr(s_col), N, _ptr(bias),
+                                      _ptr(out), code, _stream(stream)), "dq_int8_linear_noalloc")
     return out
 
 

@@ -740,3 +740,59 @@ dq_status dq_bsr_validate(const int32_t* crow, const int32_t* col, int64_t N, in
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-alloc variant
+//
+// Scratch for dq_int8_linear_noalloc: callers that cannot allocate device
+// memory get the stream-K workspace from this file-scope array instead.  In
+// host code `g_noalloc_scratch` names a host-side stand-in, not the device
+// array, so its device address is looked up once per device.
+namespace dq {
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[DQ_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoallocMaxDevices = 64;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array on the current device (set-up on the
+// first call per device, with that device current).
+dq_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kNoallocMaxDevices) return DQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DQ_OK;
+}
+
+}  // namespace
+}  // namespace dq
+
+extern "C" dq_status dq_int8_linear_noalloc(const int8_t* A, const float* s_row, int64_t M, int64_t K,
+                                            const int8_t* W, const float* s_col, int64_t N,
+                                            const void* bias_bf16, void* out, dq_out_dtype out_dtype,
+                                            dq_stream_t stream) {
+  if (M < 1 || K < 1 || N < 1)   // M == 0 and bad sizes: the plain entry point decides, no scratch
+    return dq_int8_linear(A, s_row, M, K, W, s_col, N, bias_bf16, out, out_dtype, nullptr, 0, stream);
+  DeviceInfo* d = nullptr;
+  dq_status st = current_device(&d);
+  if (st != DQ_OK) return st;
+  const size_t need = dq_int8_linear_workspace_size(M, N, K);
+  if (need > DQ_NOALLOC_SCRATCH_BYTES) return DQ_ERR_UNSUPPORTED;
+  if (need == 0)
+    return dq_int8_linear(A, s_row, M, K, W, s_col, N, bias_bf16, out, out_dtype, nullptr, 0, stream);
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != DQ_OK) return st;
+  cudaError_t e = cudaMemsetAsync(scratch, 0, need, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return dq_int8_linear(A, s_row, M, K, W, s_col, N, bias_bf16, out, out_dtype, scratch, need, stream);
+}

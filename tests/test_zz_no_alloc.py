@@ -1,0 +1,72 @@
+"""The allocation-free entry point dq_int8_linear_noalloc, called through the
+C ABI, against dq_int8_linear with a caller-owned workspace.
+
+It exists for callers that cannot allocate device memory (an engine whose
+memory planner owns all device memory, code running during another
+component's CUDA-graph capture, latency-bound callers that cannot afford the
+synchronisation of cudaMalloc/cudaFree): its split-K scratch is a static
+32 MiB device array inside libdq.  This file is collected last on purpose;
+it needs nothing from the other tests and passes alone in a fresh process.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(M, N, K, seed):
+    A = synth.uniform_int8((M, K), -127, 127, seed)
+    W = synth.uniform_int8((N, K), -127, 127, seed + 1)
+    s_row = synth.uniform_f32((M,), 0.001, 0.05, seed + 5)
+    s_col = synth.uniform_f32((N,), 0.001, 0.05, seed + 6)
+    bias = synth.normal_bf16((N,), 0.1, seed + 2)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    b = torch.from_numpy(bias.view(np.int16)).view(torch.bfloat16).cuda()
+    return dev(A), dev(W), dev(s_row), dev(s_col), b
+
+
+def _call_noalloc(lib, A, s_row, W, s_col, bias, out, code):
+    M, K = A.shape
+    N = W.shape[0]
+    P = ctypes.c_void_p
+    ptr = lambda t: None if t is None else P(t.data_ptr())  # noqa: E731
+    stream = P(torch.cuda.current_stream().cuda_stream)
+    return lib.dq_int8_linear_noalloc(ptr(A), ptr(s_row), ctypes.c_int64(M), ctypes.c_int64(K), ptr(W),
+                                      ptr(s_col), ctypes.c_int64(N), ptr(bias), ptr(out), ctypes.c_int(code),
+                                      stream)
+
+
+# (M, N, K): swap-AB stream-K (1.8 MB of scratch), dense stream-K (8.4 MB)
+@pytest.mark.parametrize("M,N,K", [(16, 28672, 8192), (2000, 1024, 2048)])
+def test_noalloc_matches_workspace_entry_two_calls(M, N, K):
+    import quantized_gemm_token_b200 as dq
+    from gpu_util import assert_bf16_close, bf16_bits
+    lib = dq.lib
+    need = dq.dq_int8_linear_workspace_size(M, N, K)
+    assert 0 < need <= dq.DQ_NOALLOC_SCRATCH_BYTES      # these shapes do use the scratch
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for call, seed in enumerate((900, 950)):             # two calls in a row, different data
+        A, W, s_row, s_col, bias = _inputs(M, N, K, seed)
+        ref32 = dq.dq_int8_linear(A, None, W, None, out_dtype="s32", workspace=ws)
+        ref16 = dq.dq_int8_linear(A, s_row, W, s_col, bias=bias, workspace=ws)
+        out32 = torch.empty((M, N), dtype=torch.int32, device="cuda")
+        out16 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        assert _call_noalloc(lib, A, None, W, None, None, out32, dq.DQ_OUT_S32) == dq.DQ_OK
+        assert _call_noalloc(lib, A, s_row, W, s_col, bias, out16, dq.DQ_OUT_BF16) == dq.DQ_OK
+        assert dq.dq_sync_status() == dq.DQ_OK
+        assert torch.equal(out32, ref32), f"call {call}: int32 differs"
+        assert_bf16_close(bf16_bits(out16), bf16_bits(ref16))
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    import quantized_gemm_token_b200 as dq
+    M, N, K = 2048, 4096, 4096                            # stream-K here needs ~33.5 MB
+    assert dq.dq_int8_linear_workspace_size(M, N, K) > dq.DQ_NOALLOC_SCRATCH_BYTES
+    A, W, s_row, s_col, bias = _inputs(M, N, K, 990)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    assert _call_noalloc(dq.lib, A, s_row, W, s_col, None, out, dq.DQ_OUT_BF16) == dq.DQ_ERR_UNSUPPORTED
