@@ -58,7 +58,21 @@ def _load():
     return lib
 
 
-lib = _load()
+class _MissingLibrary:
+    """Stands in for libdq.so when it has not been built yet, so that the
+    build module stays importable; every use raises."""
+
+    def __init__(self, err: ImportError):
+        self._err = err
+
+    def __getattr__(self, name):
+        raise ImportError(str(self._err))
+
+
+try:
+    lib = _load()
+except ImportError as _e:
+    lib = _MissingLibrary(_e)
 
 
 class DQError(RuntimeError):

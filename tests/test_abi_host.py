@@ -81,10 +81,17 @@ def test_argument_validation_without_device(libdq):
 
 
 def test_binding_refuses_to_run_without_library(tmp_path, monkeypatch):
-    # The binding has no fallback: pointing it at a missing library must raise.
-    import importlib
+    # The binding has no fallback: with the library missing every call raises.
     import quantized_gemm_token_b200 as pkg
     monkeypatch.setattr(pkg, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         pkg._load()
-    importlib.reload(pkg)
+    try:
+        pkg._load()
+    except ImportError as e:
+        missing = pkg._MissingLibrary(e)
+    monkeypatch.setattr(pkg, "lib", missing)
+    with pytest.raises(ImportError):
+        pkg.dq_version()
+    with pytest.raises(ImportError):
+        pkg.dq_sync_status(0)
