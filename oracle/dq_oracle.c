@@ -20,9 +20,9 @@
  *  - The same formula per output channel for the weight (Paddle PR 41770,
  *    review of the plugin: a per-channel scale turns the GEMM alpha into a
  *    vector).
- *  - int8 x int8 -> int32 GEMM, exact integer accumulation ("triton dot
- *    accumulator uses int32", PR 821 review by pearu; overflow bound
- *    2^31 / 2^14 stated there).
+ *  - int8 x int8 -> int32 GEMM, exact integer accumulation (PR 821 review:
+ *    the Triton dot product accumulates in int32, and its overflow bound of
+ *    about 2^31 / 2^14 on K is worked out there).
  *  - The bf16 output epilogue out = bf16( acc * s_row * s_col + bias ),
  *    evaluated left to right in fp32 with round-to-nearest-even and no
  *    fused multiply-add; bf16 output is what keeps accuracy (PR 821,

@@ -67,7 +67,12 @@ struct Cfg {
   static constexpr int A_BYTES = BM * KB;
   static constexpr int B_BYTES = BN * KB;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  // Row-layout epilogues (Dense, Bsr) stage each warp's 32x32 output block in
+  // shared memory for a TMA store: 2 buffers x 4 warps x 4 KB (int32 worst case).
+  static constexpr bool STAGED_OUT = KIND != Kind::Swap;
+  static constexpr int OUT_BUF_BYTES = 32 * 32 * 4;
+  static constexpr int OUT_BYTES = STAGED_OUT ? 2 * 4 * OUT_BUF_BYTES : 0;
+  static constexpr int STAGES_RAW = (224 * 1024 - OUT_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
   static constexpr int ACC_RAW = 512 / BN;
   static constexpr int ACC_BUFS = ACC_RAW > 8 ? 8 : ACC_RAW;
@@ -76,7 +81,7 @@ struct Cfg {
                                    : ACC_COLS <= 256 ? 256 : 512;
   static constexpr int K_STEPS = KB / 32;                     // MMA K = 32 bytes
   static constexpr int CW = BN >= 32 ? 32 : 16;               // epilogue chunk (columns)
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_BYTES + 1024 /*align*/ + 512 /*barriers*/;
   static constexpr int THREADS = 192;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(STAGES >= 2, "stages");
@@ -144,45 +149,60 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Epilogue for one chunk of CW columns of one row in the Dense/Bsr layout
-// (thread = output row m, columns n0 .. n0+CW-1).  r = raw int32 accumulator.
-template <int CW>
-__device__ __forceinline__ void store_row_chunk(const GemmArgs& g, int m, int n0, const uint32_t* r,
-                                                float srow) {
+// Epilogue for one chunk of 32 columns of the Dense/Bsr layout: thread = row
+// `row` (0..31 inside its warp's 32-row slab), output columns n0 .. n0+31.
+// The 32x32 block is written into the warp's staging buffer with the tensor
+// map's swizzle (64 B rows for bf16, 128 B rows for int32) and stored by one
+// TMA bulk store, which also clips rows >= M and columns >= N.  Scales and
+// bias are only read for columns < N (N % 8 == 0).
+__device__ __forceinline__ void store_row_chunk_tma(const GemmArgs& g, const CUtensorMap* tm_c,
+                                                    uint8_t* buf, int lane, int m0, int n0,
+                                                    const uint32_t* r, float srow) {
+  const uint32_t base = smem_u32(buf);
   if (g.out_s32) {
-    int32_t* o = static_cast<int32_t*>(g.out) + static_cast<int64_t>(m) * g.N + n0;
 #pragma unroll
-    for (int v = 0; v < CW / 4; ++v)
-      if (n0 + 4 * v < g.N)
-        *reinterpret_cast<int4*>(o + 4 * v) =
-            make_int4(static_cast<int>(r[4 * v]), static_cast<int>(r[4 * v + 1]),
-                      static_cast<int>(r[4 * v + 2]), static_cast<int>(r[4 * v + 3]));
-    return;
-  }
-  uint16_t* o = static_cast<uint16_t*>(g.out) + static_cast<int64_t>(m) * g.N + n0;
-#pragma unroll
-  for (int v = 0; v < CW / 8; ++v) {
-    const int n = n0 + 8 * v;
-    if (n < g.N) {
-      const float4 c0 = __ldg(reinterpret_cast<const float4*>(g.s_col + n));
-      const float4 c1 = __ldg(reinterpret_cast<const float4*>(g.s_col + n + 4));
-      const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-      float f[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        f[j] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[8 * v + j])), srow), sc[j]);
-      if (g.bias) {
-        const uint4 b = __ldg(reinterpret_cast<const uint4*>(g.bias + n));
-        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          f[2 * j] = __fadd_rn(f[2 * j], __uint_as_float(bw[j] << 16));
-          f[2 * j + 1] = __fadd_rn(f[2 * j + 1], __uint_as_float(bw[j] & 0xffff0000u));
-        }
-      }
-      *reinterpret_cast<uint4*>(o + 8 * v) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                                        pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t off = static_cast<uint32_t>(lane * 128 + ((j ^ (lane & 7)) << 4));
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(r[4 * j]),
+                   "r"(r[4 * j + 1]), "r"(r[4 * j + 2]), "r"(r[4 * j + 3])
+                   : "memory");
     }
+  } else {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int n = n0 + 8 * v;
+      uint32_t w[4] = {0, 0, 0, 0};
+      if (n < g.N) {
+        const float4 c0 = __ldg(reinterpret_cast<const float4*>(g.s_col + n));
+        const float4 c1 = __ldg(reinterpret_cast<const float4*>(g.s_col + n + 4));
+        const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          f[j] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[8 * v + j])), srow), sc[j]);
+        if (g.bias) {
+          const uint4 b = __ldg(reinterpret_cast<const uint4*>(g.bias + n));
+          const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            f[2 * j] = __fadd_rn(f[2 * j], __uint_as_float(bw[j] << 16));
+            f[2 * j + 1] = __fadd_rn(f[2 * j + 1], __uint_as_float(bw[j] & 0xffff0000u));
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
+      }
+      const uint32_t off = static_cast<uint32_t>(lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4));
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(w[0]), "r"(w[1]),
+                   "r"(w[2]), "r"(w[3])
+                   : "memory");
+    }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && n0 < g.N && m0 < g.M) {   // boxes wholly past the matrix are not issued
+    tma_store_2d(tm_c, base, n0, m0);
+    bulk_commit_group();
   }
 }
 
@@ -217,14 +237,15 @@ __device__ __forceinline__ void store_col_chunk(const GemmArgs& g, int n, int m0
 template <Kind KIND, int BN>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                const __grid_constant__ GemmArgs g) {
+                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ GemmArgs g) {
   using C = Cfg<KIND, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* sOut = smem + C::STAGES * C::STAGE_BYTES;          // 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + C::OUT_BYTES);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + C::STAGES;
   uint64_t* accf_bar = bars + 2 * C::STAGES;
@@ -251,6 +272,7 @@ __global__ void __launch_bounds__(192, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    if constexpr (C::STAGED_OUT) tma_prefetch_desc(&tm_c);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -366,6 +388,16 @@ __global__ void __launch_bounds__(192, 1)
     const int sp = warp & 3;                 // TMEM sub-partition of this warp
     const int row = sp * 32 + lane;          // TMEM lane = accumulator row
     const int ep_tid = threadIdx.x - 64;
+    uint8_t* my_out = sOut + (warp - 2) * 2 * C::OUT_BUF_BYTES;   // this warp's two buffers
+    int out_flip = 0;
+    // Next staging buffer, once the TMA store that last read it is done.
+    auto next_buf = [&]() -> uint8_t* {
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+      uint8_t* b = my_out + out_flip * C::OUT_BUF_BYTES;
+      out_flip ^= 1;
+      return b;
+    };
     SegIter iter(g);
     Seg s;
     int acc = 0;
@@ -378,14 +410,13 @@ __global__ void __launch_bounds__(192, 1)
         if (p0 == p1) {
           // Block row without blocks: the epilogue of acc = 0.
           const int m = ta * 128 + row;
-          if (m < g.M) {
-            const float srow = g.out_s32 ? 0.0f : __ldg(g.s_row + m);
-            uint32_t z[CW];
+          const float srow = (g.out_s32 || m >= g.M) ? 0.0f : __ldg(g.s_row + m);
+          uint32_t z[CW];
 #pragma unroll
-            for (int j = 0; j < CW; ++j) z[j] = 0;
+          for (int j = 0; j < CW; ++j) z[j] = 0;
 #pragma unroll 1
-            for (int c = 0; c < BN / CW; ++c) store_row_chunk<CW>(g, m, tb * BN + c * CW, z, srow);
-          }
+          for (int c = 0; c < BN / CW; ++c)
+            store_row_chunk_tma(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, tb * BN + c * CW, z, srow);
           continue;
         }
       }
@@ -412,7 +443,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_arrive(smem_u32(acce_bar + acc));
           }
           if constexpr (KIND == Kind::Swap) store_col_chunk<CW>(g, ta * 128 + row, tb * BN + c * CW, r);
-          else if (m < g.M) store_row_chunk<CW>(g, m, tb * BN + c * CW, r, srow);
+          else store_row_chunk_tma(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, tb * BN + c * CW, r, srow);
         }
       } else {
         // Stream-K partial tile: add into the workspace (coalesced: one
@@ -457,7 +488,7 @@ __global__ void __launch_bounds__(192, 1)
               __stcg(p, 0);
             }
             if constexpr (KIND == Kind::Swap) store_col_chunk<CW>(g, ta * 128 + row, tb * BN + c * CW, r);
-            else if (m < g.M) store_row_chunk<CW>(g, m, tb * BN + c * CW, r, srow);
+            else store_row_chunk_tma(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, tb * BN + c * CW, r, srow);
           }
           if (ep_tid == 0) g.ws_cnt[s.tile] = 0;
         }
@@ -467,6 +498,10 @@ __global__ void __launch_bounds__(192, 1)
         acc = 0;
         acc_phase ^= 1;
       }
+    }
+    if constexpr (C::STAGED_OUT) {
+      if (lane == 0) bulk_wait_group<0>();     // all output stores complete
+      __syncwarp();
     }
   }
 
@@ -502,8 +537,8 @@ __global__ void __launch_bounds__(256) bsr_pack_kernel(const int8_t* __restrict_
 namespace {
 
 template <Kind KIND, int BN>
-dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, int grid,
-                 cudaStream_t stream) {
+dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
+                 int grid, cudaStream_t stream) {
   using C = Cfg<KIND, BN>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -512,7 +547,7 @@ dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a
                                     C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err);
-  gemm_kernel<KIND, BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ta, tb, args);
+  gemm_kernel<KIND, BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ta, tb, tc, args);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
@@ -550,7 +585,10 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count) {
   // in the last wave, and every CTA still gets a few k blocks.
   const int waves = (p.num_tiles + sm_count - 1) / sm_count;
   const double eff = static_cast<double>(p.num_tiles) / (static_cast<double>(waves) * sm_count);
-  const bool worth = eff < 0.9 && iters >= 4LL * sm_count;
+  // Measured on B200: for the dense arrangement the partial-tile reduction
+  // costs more than the idle SMs it saves, so only swap-AB (few tokens,
+  // weight streaming) splits.
+  const bool worth = p.kind == Kind::Swap && eff < 0.9 && iters >= 4LL * sm_count;
   p.ws_bytes = worth ? static_cast<size_t>(p.num_tiles) * (static_cast<size_t>(p.bn) * 128 * 4 + 4) : 0;
   p.stream_k = worth;
   return p;
@@ -608,6 +646,8 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   const int64_t b_rows = p.kind == Kind::Swap ? M : N;
   if ((st = make_tmap_u8_2d(&ta, a_src, K, a_rows, K, 128, 128, 128)) != DQ_OK) return st;
   if ((st = make_tmap_u8_2d(&tb, b_src, K, b_rows, K, 128, p.bn, 128)) != DQ_OK) return st;
+  CUtensorMap tc;
+  if ((st = make_tmap_out_2d(&tc, out, N, M, out_dtype == DQ_OUT_S32 ? 4 : 2)) != DQ_OK) return st;
 
   GemmArgs g{};
   g.M = static_cast<int>(M);
@@ -633,14 +673,14 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   const int grid = sk ? d->sm_count : (p.num_tiles < d->sm_count ? p.num_tiles : d->sm_count);
 
   if (p.kind == Kind::Dense) {
-    if (p.bn == 256) return launch<Kind::Dense, 256>(ta, tb, g, grid, stream);
-    return launch<Kind::Dense, 128>(ta, tb, g, grid, stream);
+    if (p.bn == 256) return launch<Kind::Dense, 256>(ta, tb, tc, g, grid, stream);
+    return launch<Kind::Dense, 128>(ta, tb, tc, g, grid, stream);
   }
   switch (p.bn) {
-    case 16: return launch<Kind::Swap, 16>(ta, tb, g, grid, stream);
-    case 32: return launch<Kind::Swap, 32>(ta, tb, g, grid, stream);
-    case 64: return launch<Kind::Swap, 64>(ta, tb, g, grid, stream);
-    default: return launch<Kind::Swap, 128>(ta, tb, g, grid, stream);
+    case 16: return launch<Kind::Swap, 16>(ta, tb, tc, g, grid, stream);
+    case 32: return launch<Kind::Swap, 32>(ta, tb, tc, g, grid, stream);
+    case 64: return launch<Kind::Swap, 64>(ta, tb, tc, g, grid, stream);
+    default: return launch<Kind::Swap, 128>(ta, tb, tc, g, grid, stream);
   }
 }
 
@@ -672,6 +712,8 @@ dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int
   if (nnzb > 0) st = make_tmap_u8_2d(&tb, values, 64, static_cast<uint64_t>(nnzb) * 64, 64, 64, 64, 64);
   else st = make_tmap_u8_2d(&tb, A, K, M, K, 64, 64, 64);
   if (st != DQ_OK) return st;
+  CUtensorMap tc;
+  if ((st = make_tmap_out_2d(&tc, out, N, M, out_dtype == DQ_OUT_S32 ? 4 : 2)) != DQ_OK) return st;
 
   GemmArgs g{};
   g.M = static_cast<int>(M);
@@ -694,7 +736,7 @@ dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int
   g.nnzb = static_cast<int>(nnzb);
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
   const int grid = g.num_tiles < d->sm_count ? g.num_tiles : d->sm_count;
-  return launch<Kind::Bsr, 64>(ta, tb, g, grid, stream);
+  return launch<Kind::Bsr, 64>(ta, tb, tc, g, grid, stream);
 }
 
 dq_status dq_bsr_pack(const int8_t* wq, int64_t N, int64_t K, const int32_t* crow, const int32_t* col,

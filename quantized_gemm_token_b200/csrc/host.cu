@@ -101,6 +101,26 @@ dq_status make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, ui
   return DQ_OK;
 }
 
+dq_status make_tmap_out_2d(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows,
+                           int elem_bytes) {
+  std::call_once(g_encode_once, resolve_encoder);
+  if (g_encode == nullptr) return cuda_fail(g_encode_err);
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  const bool four = elem_bytes == 4;
+  CUresult r = g_encode(map, four ? CU_TENSOR_MAP_DATA_TYPE_INT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base,
+                        dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        four ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda_error = static_cast<int>(r);
+    return DQ_ERR_CUDA;
+  }
+  return DQ_OK;
+}
+
 // ------------------------------------------------------------ self test
 
 __global__ void selftest_wait_kernel(WaitCtl ctl) {

@@ -35,6 +35,12 @@ dq_status make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, ui
                           uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer,
                           int swizzle_bytes);
 
+// 2-D tensor map for an output matrix [rows, cols] of 2- or 4-byte elements
+// (row stride in bytes), box {32 cols, 32 rows}, swizzle matching a 32-column
+// row: 64 B (2-byte elements) or 128 B (4-byte elements).
+dq_status make_tmap_out_2d(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows,
+                           int elem_bytes);
+
 inline bool aligned(const void* p, size_t a) {
   return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }

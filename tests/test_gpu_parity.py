@@ -344,3 +344,53 @@ def test_non_contiguous_and_misaligned_rejected():
     A2 = base[1:].view(64, 64)
     with pytest.raises(dq.DQError):
         dq.dq_int8_linear(A2, None, W, None, out_dtype="s32")
+
+
+# ---------------------------------------------------------------- exhaustive quantize
+
+@pytest.mark.parametrize("a", [1.0, 127.0, 3.5, 0.0123, 3e-6, 1e-9, 300.0, 65504.0, 1.5e30])
+def test_quantize_every_bf16_pattern_below_absmax(a):
+    """Every finite bf16 value v with |v| <= a, in rows whose absmax is a:
+    the kernel's multiply-then-check rounding must agree with the oracle's
+    IEEE division on every one of them (near ties included)."""
+    ab = int(_bits([a])[0])
+    av = float(synth.bf16_bits_to_f32(np.array([ab], np.uint16))[0])
+    allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = synth.bf16_bits_to_f32(allb)
+    cand = allb[np.isfinite(vals) & (np.abs(vals) <= av)]
+    K = 8192
+    rows = -(-len(cand) // (K - 1))
+    x = np.zeros((rows, K), np.uint16)
+    x[:, 0] = ab
+    flat = x[:, 1:].reshape(-1)
+    flat[:len(cand)] = cand
+    x[:, 1:] = flat.reshape(rows, K - 1)
+    q, s = dq.dq_quantize_rows(to_dev_bf16(x))
+    qo, so = oracle.quantize_rows_bf16(x)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), qo)
+
+
+def test_quantize_weight_near_ties_fp32():
+    """fp32 weights placed within a few ulps of (k + 1/2) * s on both sides."""
+    r = synth.rng(77)
+    rows = []
+    for absmax in (1.0, 0.02, 0.37, 5.0):
+        s = np.float32(np.float32(absmax) / np.float32(127.0))
+        ks = r.integers(-126, 126, size=1024)
+        base = ((ks.astype(np.float64) + 0.5) * float(s)).astype(np.float32)
+        row = base.copy()
+        steps = r.integers(-4, 5, size=base.size)
+        for i in range(base.size):
+            v = base[i]
+            for _ in range(abs(int(steps[i]))):
+                v = np.nextafter(v, np.float32(np.inf if steps[i] > 0 else -np.inf))
+            row[i] = v
+        row = np.clip(row, -absmax, absmax).astype(np.float32)
+        row[0] = np.float32(absmax)
+        rows.append(row)
+    w = np.stack(rows)
+    wq, sc = dq.dq_quantize_weight(to_dev(w))
+    wo, so = oracle.quantize_rows_f32(w)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    assert np.array_equal(wq.cpu().numpy(), wo)
