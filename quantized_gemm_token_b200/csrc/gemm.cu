@@ -19,9 +19,10 @@
 //   Swap   A slot = 128 weight channels, B slot = BN (16..128) tokens: for
 //          few tokens the weight stream, not the token count, fills MMA M.
 //   Bsr    A slot = 128 activation rows x one 64-wide k slice, B slot = one
-//          nonzero 64x64 weight block; the producer walks crow/col of one
-//          block row (PR 821: the kernel takes crow_indices / col_indices /
-//          values directly).
+//          nonzero 64x64 weight block; a tile spans 4 block rows (256
+//          channels) and each block accumulates into its block row's 64-column
+//          slice of the TMEM tile; the producer walks crow/col (PR 821: the
+//          kernel takes crow_indices / col_indices / values directly).
 //
 // Schedules: whole tiles round-robin over one CTA per SM, or (when the tile
 // count would leave SMs idle) stream-K: the tile x k-block iteration space is
@@ -57,6 +58,8 @@ struct GemmArgs {
   const int32_t* crow;    // Bsr
   const int32_t* col;
   int nnzb;
+  int nbr;                // Bsr: block rows (N / 64)
+  int idx_smem;           // Bsr: crow and col staged in shared memory (they fit)
   WaitCtl wait;
 };
 
@@ -65,13 +68,21 @@ struct Cfg {
   static constexpr int BM = 128;
   static constexpr int KB = KIND == Kind::Bsr ? 64 : 128;     // k bytes per stage
   static constexpr int A_BYTES = BM * KB;
-  static constexpr int B_BYTES = BN * KB;
+  // Bsr: a tile spans BN/64 block rows; each stage holds one 64x64 block
+  // that accumulates into its block row's 64-column slice of the tile.
+  static constexpr int B_ROWS = KIND == Kind::Bsr ? 64 : BN;
+  static constexpr int MMA_N = B_ROWS;
+  static constexpr int NSUB = KIND == Kind::Bsr ? BN / 64 : 1;
+  static constexpr int B_BYTES = B_ROWS * KB;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   // Row-layout epilogues (Dense, Bsr) stage each warp's 32x32 output block in
   // shared memory for a TMA store: 2 buffers x 4 warps x 4 KB (int32 worst case).
+  // Epilogue warps: two per TMEM sub-partition when a tile has at least two
+  // 32-column chunks, so one warp's latency hides behind the other's work.
+  static constexpr int EPI_WARPS = BN >= 64 ? 8 : 4;
   static constexpr bool STAGED_OUT = KIND != Kind::Swap;
-  static constexpr int OUT_BUF_BYTES = 32 * 32 * 4;
-  static constexpr int OUT_BYTES = STAGED_OUT ? 2 * 4 * OUT_BUF_BYTES : 0;
+  static constexpr int OUT_BUF_BYTES = 32 * 32 * 4;           // per epilogue warp
+  static constexpr int OUT_BYTES = STAGED_OUT ? EPI_WARPS * OUT_BUF_BYTES : 0;
   static constexpr int STAGES_RAW = (224 * 1024 - OUT_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
   static constexpr int ACC_RAW = 512 / BN;
@@ -81,8 +92,14 @@ struct Cfg {
                                    : ACC_COLS <= 256 ? 256 : 512;
   static constexpr int K_STEPS = KB / 32;                     // MMA K = 32 bytes
   static constexpr int CW = BN >= 32 ? 32 : 16;               // epilogue chunk (columns)
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_BYTES + 1024 /*align*/ + 512 /*barriers*/;
-  static constexpr int THREADS = 192;
+  // Bsr: crow and col are copied to shared memory when nbr + 1 + nnzb fits
+  // (every tile and every block needs them; a global load per block would put
+  // a dependent L2 round trip in front of each TMA issue).
+  static constexpr int IDX_INTS = KIND == Kind::Bsr ? 4096 : 0;
+  static constexpr int IDX_BYTES = IDX_INTS * 4;
+  static constexpr int SMEM_BYTES =
+      STAGES * STAGE_BYTES + OUT_BYTES + IDX_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(STAGES >= 2, "stages");
 };
@@ -135,9 +152,11 @@ __device__ __forceinline__ int sk_contributors(const GemmArgs& g, int tile) {
   return static_cast<int>(c1 - c0 + 1);
 }
 
-// Block range of one BSR block row, clamped to [0, nnzb].
-__device__ __forceinline__ void bsr_range(const GemmArgs& g, int br, int& p0, int& p1) {
-  int a = __ldg(g.crow + br), b = __ldg(g.crow + br + 1);
+// Block range of one BSR block row, clamped to [0, nnzb].  `sidx` holds crow
+// then col in shared memory, or is null (read global memory).
+__device__ __forceinline__ void bsr_range(const GemmArgs& g, const int* sidx, int br, int& p0, int& p1) {
+  int a = sidx ? sidx[br] : __ldg(g.crow + br);
+  int b = sidx ? sidx[br + 1] : __ldg(g.crow + br + 1);
   a = min(max(a, 0), g.nnzb);
   b = min(max(b, a), g.nnzb);
   p0 = a;
@@ -235,7 +254,7 @@ __device__ __forceinline__ void store_col_chunk(const GemmArgs& g, int n, int m0
 }
 
 template <Kind KIND, int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ GemmArgs g) {
   using C = Cfg<KIND, BN>;
@@ -245,7 +264,8 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
   uint8_t* sOut = smem + C::STAGES * C::STAGE_BYTES;          // 1024-aligned
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + C::OUT_BYTES);
+  int* sIdx = reinterpret_cast<int*>(sOut + C::OUT_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + C::OUT_BYTES + C::IDX_BYTES);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + C::STAGES;
   uint64_t* accf_bar = bars + 2 * C::STAGES;
@@ -266,7 +286,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < C::ACC_BUFS; ++a) {
       mbar_init(smem_u32(accf_bar + a), 1);
-      mbar_init(smem_u32(acce_bar + a), 128);
+      mbar_init(smem_u32(acce_bar + a), 32 * C::EPI_WARPS);
     }
     mbar_init(smem_u32(drain_bar), 1);
     fence_barrier_init();
@@ -277,6 +297,15 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
+  }
+  const int* idx = nullptr;      // Bsr: crow at idx[0..nbr], col at idx[nbr+1..]
+  if constexpr (KIND == Kind::Bsr) {
+    if (g.idx_smem) {
+      const int nbr = g.nbr;
+      for (int i = threadIdx.x; i <= nbr; i += blockDim.x) sIdx[i] = __ldg(g.crow + i);
+      for (int i = threadIdx.x; i < g.nnzb; i += blockDim.x) sIdx[nbr + 1 + i] = __ldg(g.col + i);
+      idx = sIdx;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -294,8 +323,13 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = true;
       while (ok && iter.next(s)) {
         const int ta = s.tile / g.b_tiles, tb = s.tile % g.b_tiles;
+        for (int j = 0; ok && j < C::NSUB; ++j) {
         int k0 = s.kb0, k1 = s.kb1;
-        if constexpr (KIND == Kind::Bsr) bsr_range(g, tb, k0, k1);
+        if constexpr (KIND == Kind::Bsr) {
+          const int br = tb * C::NSUB + j;
+          if (br >= g.nbr) break;
+          bsr_range(g, idx, br, k0, k1);
+        }
         for (int kb = k0; kb < k1; ++kb) {
           if (!mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, g.wait, abort_flag)) {
             ok = false;
@@ -306,7 +340,7 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t da = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t db = smem_u32(sB + stage * C::B_BYTES);
           if constexpr (KIND == Kind::Bsr) {
-            const int c = __ldg(g.col + kb);
+            const int c = idx ? idx[g.nbr + 1 + kb] : __ldg(g.col + kb);
             tma_load_2d(da, &tm_a, fb, c * 64, ta * 128);
             tma_load_2d(db, &tm_b, fb, 0, kb * 64);
           } else {
@@ -318,6 +352,7 @@ __global__ void __launch_bounds__(192, 1)
             stage = 0;
             phase ^= 1;
           }
+        }
         }
       }
       if (!ok) {
@@ -338,21 +373,24 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(128, BN);
+      constexpr uint32_t idesc = idesc_i8(128, C::MMA_N);
       SegIter iter(g);
       Seg s;
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       while (ok && iter.next(s)) {
-        int k0 = s.kb0, k1 = s.kb1;
-        if constexpr (KIND == Kind::Bsr) {
-          bsr_range(g, s.tile % g.b_tiles, k0, k1);
-          if (k0 == k1) continue;    // empty block row: no accumulator
-        }
         if (!mbar_wait(smem_u32(acce_bar + acc), acc_phase ^ 1, g.wait, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int j = 0; ok && j < C::NSUB; ++j) {
+        int k0 = s.kb0, k1 = s.kb1;
+        if constexpr (KIND == Kind::Bsr) {
+          const int br = (s.tile % g.b_tiles) * C::NSUB + j;
+          if (br >= g.nbr) break;
+          bsr_range(g, idx, br, k0, k1);
+        }
+        // an empty block row leaves its slice untouched; the epilogue writes zeros there
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN + j * C::MMA_N);
         for (int kb = k0; kb < k1; ++kb) {
           if (!mbar_wait(smem_u32(full_bar + stage), phase, g.wait, abort_flag)) {
             ok = false;
@@ -370,6 +408,7 @@ __global__ void __launch_bounds__(192, 1)
             phase ^= 1;
           }
         }
+        }
         if (!ok) break;
         mma_commit(smem_u32(accf_bar + acc));
         if (++acc == C::ACC_BUFS) {
@@ -384,17 +423,31 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // EPI_WARPS warps; warp w reads TMEM sub-partition w % 4 (rows 32*(w%4) ..
+    // +31) and, with EPI_WARPS == 8, the two warps of a sub-partition take
+    // alternate 32-column chunks of each tile.
     constexpr int CW = C::CW;
+    constexpr int NCH = BN / CW;
+    constexpr int GROUPS = C::EPI_WARPS / 4;
+    constexpr int EPI_THREADS = 32 * C::EPI_WARPS;
+    const int ew = warp - 2;
     const int sp = warp & 3;                 // TMEM sub-partition of this warp
+    const int grp = ew / 4;                  // which chunks: c % GROUPS == grp
     const int row = sp * 32 + lane;          // TMEM lane = accumulator row
     const int ep_tid = threadIdx.x - 64;
-    uint8_t* my_out = sOut + (warp - 2) * 2 * C::OUT_BUF_BYTES;   // this warp's two buffers
+    uint8_t* my_out = sOut + ew * C::OUT_BUF_BYTES;
     int out_flip = 0;
-    // Next staging buffer, once the TMA store that last read it is done.
+    // Staging buffer for the next 32x32 block, once the TMA store that last
+    // read it is done: two 2 KB slots for bf16, one 4 KB slot for int32.
     auto next_buf = [&]() -> uint8_t* {
+      if (g.out_s32) {
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        return my_out;
+      }
       if (lane == 0) bulk_wait_group_read<1>();
       __syncwarp();
-      uint8_t* b = my_out + out_flip * C::OUT_BUF_BYTES;
+      uint8_t* b = my_out + out_flip * (C::OUT_BUF_BYTES / 2);
       out_flip ^= 1;
       return b;
     };
@@ -404,41 +457,38 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t acc_phase = 0;
     while (iter.next(s)) {
       const int ta = s.tile / g.b_tiles, tb = s.tile % g.b_tiles;
-      if constexpr (KIND == Kind::Bsr) {
-        int p0, p1;
-        bsr_range(g, tb, p0, p1);
-        if (p0 == p1) {
-          // Block row without blocks: the epilogue of acc = 0.
-          const int m = ta * 128 + row;
-          const float srow = (g.out_s32 || m >= g.M) ? 0.0f : __ldg(g.s_row + m);
-          uint32_t z[CW];
-#pragma unroll
-          for (int j = 0; j < CW; ++j) z[j] = 0;
-#pragma unroll 1
-          for (int c = 0; c < BN / CW; ++c)
-            store_row_chunk_tma(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, tb * BN + c * CW, z, srow);
-          continue;
-        }
-      }
       if (!mbar_wait(smem_u32(accf_bar + acc), acc_phase, g.wait, abort_flag)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const bool whole = !g.stream_k || (s.kb0 == 0 && s.kb1 == g.kb_total);
+      // this warp's last chunk; after reading it the warp releases the accumulator
+      const int last_c = grp + ((NCH - 1 - grp) / GROUPS) * GROUPS;
 
       if (whole) {
         float srow = 0.0f;
-        int m = 0;
         if constexpr (KIND != Kind::Swap) {
-          m = ta * 128 + row;
+          const int m = ta * 128 + row;
           if (!g.out_s32 && m < g.M) srow = __ldg(g.s_row + m);
         }
 #pragma unroll 1
-        for (int c = 0; c < BN / CW; ++c) {
+        for (int c = grp; c < NCH; c += GROUPS) {
           uint32_t r[CW];
-          if constexpr (CW == 32) tmem_ld_32x32b_x32(tbase + c * CW, r);
-          else tmem_ld_32x32b_x16(tbase + c * CW, r);
-          tmem_ld_wait();
-          if (c == BN / CW - 1) {
+          bool empty_slice = false;     // Bsr: this chunk's block row has no block
+          if constexpr (KIND == Kind::Bsr) {
+            int p0, p1;
+            const int br = tb * C::NSUB + (c * CW) / 64;
+            if (br < g.nbr) bsr_range(g, idx, br, p0, p1);
+            empty_slice = br >= g.nbr || p0 == p1;
+          }
+          if (empty_slice) {
+#pragma unroll
+            for (int j = 0; j < CW; ++j) r[j] = 0;
+          } else {
+            if constexpr (CW == 32) tmem_ld_32x32b_x32(tbase + c * CW, r);
+            else tmem_ld_32x32b_x16(tbase + c * CW, r);
+            tmem_ld_wait();
+          }
+          if (c == last_c) {
             tc_fence_before();
             mbar_arrive(smem_u32(acce_bar + acc));
           }
@@ -451,12 +501,12 @@ __global__ void __launch_bounds__(192, 1)
         // contributing CTAs finishes the tile.
         int32_t* wt = g.ws + static_cast<int64_t>(s.tile) * BN * 128;
 #pragma unroll 1
-        for (int c = 0; c < BN / CW; ++c) {
+        for (int c = grp; c < NCH; c += GROUPS) {
           uint32_t r[CW];
           if constexpr (CW == 32) tmem_ld_32x32b_x32(tbase + c * CW, r);
           else tmem_ld_32x32b_x16(tbase + c * CW, r);
           tmem_ld_wait();
-          if (c == BN / CW - 1) {
+          if (c == last_c) {
             tc_fence_before();
             mbar_arrive(smem_u32(acce_bar + acc));
           }
@@ -464,22 +514,21 @@ __global__ void __launch_bounds__(192, 1)
           for (int j = 0; j < CW; ++j) atomicAdd(wt + (c * CW + j) * 128 + row, static_cast<int>(r[j]));
         }
         __threadfence();
-        named_bar_sync(1, 128);
+        named_bar_sync(1, EPI_THREADS);
         if (ep_tid == 0) {
           const uint32_t prev = atomicAdd(g.ws_cnt + s.tile, 1u);
           *sk_last = (static_cast<int>(prev) == sk_contributors(g, s.tile) - 1) ? 1 : 0;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, EPI_THREADS);
         if (*sk_last) {
           __threadfence();
           float srow = 0.0f;
-          int m = 0;
           if constexpr (KIND != Kind::Swap) {
-            m = ta * 128 + row;
+            const int m = ta * 128 + row;
             if (!g.out_s32 && m < g.M) srow = __ldg(g.s_row + m);
           }
 #pragma unroll 1
-          for (int c = 0; c < BN / CW; ++c) {
+          for (int c = grp; c < NCH; c += GROUPS) {
             uint32_t r[CW];
 #pragma unroll
             for (int j = 0; j < CW; ++j) {
@@ -492,7 +541,7 @@ __global__ void __launch_bounds__(192, 1)
           }
           if (ep_tid == 0) g.ws_cnt[s.tile] = 0;
         }
-        named_bar_sync(1, 128);   // sk_last is reused by the next partial tile
+        named_bar_sync(1, EPI_THREADS);   // sk_last is reused by the next partial tile
       }
       if (++acc == C::ACC_BUFS) {
         acc = 0;
@@ -720,7 +769,8 @@ dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int
   g.N = static_cast<int>(N);
   g.K = static_cast<int>(K);
   g.a_tiles = static_cast<int>((M + 127) / 128);
-  g.b_tiles = static_cast<int>(N / 64);
+  g.nbr = static_cast<int>(N / 64);
+  g.b_tiles = (g.nbr + 3) / 4;            // tiles of 4 block rows = 256 channels
   g.kb_total = 0;
   const int64_t tiles = static_cast<int64_t>(g.a_tiles) * g.b_tiles;
   if (tiles > 0x7fffffff) return DQ_ERR_UNSUPPORTED;
@@ -734,9 +784,10 @@ dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int
   g.crow = crow;
   g.col = col;
   g.nnzb = static_cast<int>(nnzb);
+  g.idx_smem = (N / 64 + 1 + nnzb) <= Cfg<Kind::Bsr, 256>::IDX_INTS ? 1 : 0;
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
   const int grid = g.num_tiles < d->sm_count ? g.num_tiles : d->sm_count;
-  return launch<Kind::Bsr, 64>(ta, tb, tc, g, grid, stream);
+  return launch<Kind::Bsr, 256>(ta, tb, tc, g, grid, stream);
 }
 
 dq_status dq_bsr_pack(const int8_t* wq, int64_t N, int64_t K, const int32_t* crow, const int32_t* col,

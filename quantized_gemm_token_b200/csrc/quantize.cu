@@ -38,7 +38,7 @@ __device__ __forceinline__ int8_t quant_one(float v, float s) {
   return static_cast<int8_t>(r);
 }
 
-// The same result as quant_one, mostly without a division.
+// Codes without a division, the same result as quant_one.
 //
 // Let y = fp32(v * inv) with inv = fp32(1 / s).  Each of the two roundings
 // has relative error at most 2^-24, and |v / s| <= 127 * (1 + 2^-23) because
@@ -46,18 +46,62 @@ __device__ __forceinline__ int8_t quant_one(float v, float s) {
 // rounded quotient q* = fp32(v / s) is within half an fp32 ulp of v/s, at
 // most 2^-18 below 128, so |y - q*| < 2^-15.  rint() can only tell y and q*
 // apart if a half-integer lies between them (or q* is one); so when y is
-// farther than 2^-14 from every half-integer, rint(y) == rint(q*).  Otherwise
-// (rare) the exact IEEE division decides.
-__device__ __forceinline__ int8_t quant_one_fast(float v, float s, float inv) {
-  const float y = __fmul_rn(v, inv);
-  const float frac = y - floorf(y);               // exact for |y| < 2^23
-  int r;
-  if (fabsf(frac - 0.5f) > 6.103515625e-05f)      // 2^-14
-    r = __float2int_rn(y);
-  else
-    r = __float2int_rn(__fdiv_rn(v, s));
-  r = r > 127 ? 127 : (r < -127 ? -127 : r);
-  return static_cast<int8_t>(r);
+// farther than 2^-14 from every half-integer, rint(y) == rint(q*) (and it
+// lies in [-127, 127], so no clamp is needed).  Otherwise the caller redoes
+// the vector with the exact IEEE division.
+//
+// rint(y) comes from t = fp32(y + 1.5 * 2^23): for |y| < 2^22 the sum lies in
+// [2^23, 2^24) where the fp32 spacing is 1, so round-to-nearest-even of the
+// sum is 1.5 * 2^23 + rint_half_even(y) (1.5 * 2^23 is even), the low byte of
+// t's bit pattern is rint(y) as a two's-complement int8, and r = t - 1.5 * 2^23
+// is exact.  |y - r| (exact by Sterbenz) is the distance to the nearest
+// integer; y is near a half-integer when it is >= 1/2 - 2^-14.
+//
+// The fp32 work runs as packed pairs (sm_100 f32x2 add/sub/mul, each lane of
+// the pair rounded like the scalar instruction).
+constexpr float kMagic = 12582912.0f;            // 1.5 * 2^23
+constexpr float kNear = 0.49993896484375f;       // 1/2 - 2^-14
+
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack_f2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul_f2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t add_f2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub_f2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Two codes (low bytes of the two t's) for the pair v; tracks max |y - r|.
+__device__ __forceinline__ void quant_pair(uint64_t v, uint64_t inv2, uint64_t magic2, float& emax,
+                                           uint32_t& t0, uint32_t& t1) {
+  const uint64_t y = mul_f2(v, inv2);
+  const uint64_t t = add_f2(y, magic2);
+  const uint64_t e = sub_f2(y, sub_f2(t, magic2));
+  float e0, e1, f0, f1;
+  unpack_f2(e, e0, e1);
+  emax = fmaxf(emax, fmaxf(fabsf(e0), fabsf(e1)));
+  unpack_f2(t, f0, f1);
+  t0 = __float_as_uint(f0);
+  t1 = __float_as_uint(f1);
+}
+
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
 
 __device__ __forceinline__ float scale_from_absmax(float a) {
@@ -102,6 +146,7 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict
       const int vi = t + i * tpr;
       if (vi < nv) {
         if constexpr (E == 8) {
+          // |x| of both halves, max per half: exact for finite bf16
           amax = __vmaxu2(amax, v[i].x & 0x7fff7fffu);
           amax = __vmaxu2(amax, v[i].y & 0x7fff7fffu);
           amax = __vmaxu2(amax, v[i].z & 0x7fff7fffu);
@@ -131,27 +176,44 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict
   const float inv = __frcp_rn(s);
   if (t == 0) scales[row] = s;
 
+  const float inv1 = inv;
+  const uint64_t inv2 = pack_f2(inv1, inv1);
+  const uint64_t magic2 = pack_f2(kMagic, kMagic);
   int8_t* qr = q + row * ldq;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int vi = t + i * tpr;
     if (vi < nv) {
       const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      float emax = 0.0f;
       if constexpr (E == 8) {
-        uint32_t out[2];
+        uint32_t b[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t a = w[2 * h], b = w[2 * h + 1];
-          out[h] = pack4(quant_one_fast(__uint_as_float(a << 16), s, inv),
-                         quant_one_fast(__uint_as_float(a & 0xffff0000u), s, inv),
-                         quant_one_fast(__uint_as_float(b << 16), s, inv),
-                         quant_one_fast(__uint_as_float(b & 0xffff0000u), s, inv));
+        for (int h = 0; h < 4; ++h)
+          quant_pair(pack_f2(__uint_as_float(w[h] << 16), __uint_as_float(w[h] & 0xffff0000u)), inv2, magic2,
+                     emax, b[2 * h], b[2 * h + 1]);
+        uint32_t out0 = pack_low_bytes(b[0], b[1], b[2], b[3]);
+        uint32_t out1 = pack_low_bytes(b[4], b[5], b[6], b[7]);
+        if (emax >= kNear) {   // rare: a code within 2^-14 of a tie, decide by IEEE division
+          float f[8];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            f[2 * h] = __uint_as_float(w[h] << 16);
+            f[2 * h + 1] = __uint_as_float(w[h] & 0xffff0000u);
+          }
+          out0 = pack4(quant_one(f[0], s), quant_one(f[1], s), quant_one(f[2], s), quant_one(f[3], s));
+          out1 = pack4(quant_one(f[4], s), quant_one(f[5], s), quant_one(f[6], s), quant_one(f[7], s));
         }
-        *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(vi) * 8) = make_uint2(out[0], out[1]);
+        *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(vi) * 8) = make_uint2(out0, out1);
       } else {
-        *reinterpret_cast<uint32_t*>(qr + static_cast<int64_t>(vi) * 4) =
-            pack4(quant_one_fast(__uint_as_float(w[0]), s, inv), quant_one_fast(__uint_as_float(w[1]), s, inv),
-                  quant_one_fast(__uint_as_float(w[2]), s, inv), quant_one_fast(__uint_as_float(w[3]), s, inv));
+        uint32_t b[4];
+        quant_pair(pack_f2(__uint_as_float(w[0]), __uint_as_float(w[1])), inv2, magic2, emax, b[0], b[1]);
+        quant_pair(pack_f2(__uint_as_float(w[2]), __uint_as_float(w[3])), inv2, magic2, emax, b[2], b[3]);
+        uint32_t out = pack_low_bytes(b[0], b[1], b[2], b[3]);
+        if (emax >= kNear)
+          out = pack4(quant_one(__uint_as_float(w[0]), s), quant_one(__uint_as_float(w[1]), s),
+                      quant_one(__uint_as_float(w[2]), s), quant_one(__uint_as_float(w[3]), s));
+        *reinterpret_cast<uint32_t*>(qr + static_cast<int64_t>(vi) * 4) = out;
       }
     }
   }
@@ -212,6 +274,11 @@ dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t*
   if (vec_ok) {
     int tpr_log2 = 5;
     while ((int64_t(1) << tpr_log2) * 8 < nv) ++tpr_log2;     // tpr * 8 >= nv, tpr <= 256
+    // Few rows: spread each row over more threads (fewer vectors each) so the
+    // grid fills the SMs several times over and per-thread chains are short.
+    while (tpr_log2 < 8 && ((int64_t(1) << tpr_log2) * 2 <= nv) &&
+           (M * (int64_t(1) << tpr_log2)) / 256 < int64_t(d->sm_count) * 8)
+      ++tpr_log2;
     const int64_t tpr = int64_t(1) << tpr_log2;
     const int64_t vpt = (nv + tpr - 1) / tpr;
     const int64_t rows_per_cta = 256 / tpr;

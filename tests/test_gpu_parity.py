@@ -288,10 +288,12 @@ def _random_bsr(N, K, keep, seed, empty_rows=(), dup=False):
     return crow, col, values
 
 
-@pytest.mark.parametrize("case", ["empty_rows", "no_blocks", "dense", "duplicates", "ragged_m"])
+@pytest.mark.parametrize("case", ["empty_rows", "no_blocks", "dense", "duplicates", "ragged_m", "many_blocks"])
 def test_bsr_edge_cases(case):
-    M, N, K = {"ragged_m": (1, 256, 192)}.get(case, (300, 320, 256))
-    keep = {"dense": 1.0, "no_blocks": 0.0}.get(case, 0.3)
+    # many_blocks: 4480 blocks, more indices than the kernel stages in shared
+    # memory, so crow/col are read from global memory
+    M, N, K = {"ragged_m": (1, 256, 192), "many_blocks": (130, 6400, 4096)}.get(case, (300, 320, 256))
+    keep = {"dense": 1.0, "no_blocks": 0.0, "many_blocks": 0.7}.get(case, 0.3)
     crow, col, values = _random_bsr(N, K, keep, 500, empty_rows=(1, 3) if case == "empty_rows" else (),
                                     dup=case == "duplicates")
     A = synth.uniform_int8((M, K), -127, 127, 501)
