@@ -41,6 +41,8 @@ _PROTOS = {
     "dq_bsr_validate": (_I32, [_P, _P, _I64, _I64, _I64]),
     "dq_mma_peak_probe": (_I32, [_I32, _I32, _P]),
     "dq_debug_set_schedule": (None, [_I32]),
+    "dq_debug_set_tile_n": (None, [_I32]),
+    "dq_debug_set_quant_kernel": (None, [_I32]),
 }
 
 
@@ -52,7 +54,11 @@ def _load():
             "There is no fallback implementation.")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in _PROTOS.items():
-        fn = getattr(lib, name)
+        try:
+            fn = getattr(lib, name)
+        except AttributeError:
+            raise ImportError(f"{LIB_PATH} is stale (no {name}): rebuild it with "
+                              "`python -m quantized_gemm_token_b200.build`") from None
         fn.restype = res
         fn.argtypes = args
     return lib
@@ -138,6 +144,14 @@ def dq_selftest_wait_timeout(stream=None) -> None:
 
 def dq_debug_set_schedule(mode: int) -> None:
     lib.dq_debug_set_schedule(int(mode))
+
+
+def dq_debug_set_tile_n(n: int) -> None:
+    lib.dq_debug_set_tile_n(int(n))
+
+
+def dq_debug_set_quant_kernel(mode: int) -> None:
+    lib.dq_debug_set_quant_kernel(int(mode))
 
 
 # ---------------------------------------------------------------- quantize

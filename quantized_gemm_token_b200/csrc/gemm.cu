@@ -30,38 +30,11 @@
 // int32 workspace through red.add, and the last arriving CTA (an arrival
 // counter) runs the epilogue and zeroes the workspace again.  Integer adds
 // are exact and associative, so every schedule gives identical bits.
-#include <cuda_bf16.h>
-
 #include <mutex>
 
-#include "internal.h"
-#include "sm100.cuh"
+#include "gemm_common.cuh"
 
 namespace dq {
-
-enum class Kind : int { Dense = 0, Swap = 1, Bsr = 2 };
-
-struct GemmArgs {
-  int M, N, K;
-  int a_tiles, b_tiles;   // tiles along the A slot (128 rows) and the B slot (BN rows)
-  int kb_total;           // k blocks per tile (Dense / Swap)
-  int num_tiles;
-  int stream_k;           // 0: whole tiles round-robin; 1: stream-K ranges
-  long long iters_total;  // num_tiles * kb_total (stream-K)
-  const float* s_row;
-  const float* s_col;
-  const uint16_t* bias;   // bf16 bits or null
-  void* out;
-  int out_s32;
-  int32_t* ws;            // stream-K partial tiles: [tile][BN][128] int32
-  uint32_t* ws_cnt;       // stream-K arrival counters: [tile]
-  const int32_t* crow;    // Bsr
-  const int32_t* col;
-  int nnzb;
-  int nbr;                // Bsr: block rows (N / 64)
-  int idx_smem;           // Bsr: crow and col staged in shared memory (they fit)
-  WaitCtl wait;
-};
 
 template <Kind KIND, int BN>
 struct Cfg {
@@ -103,155 +76,6 @@ struct Cfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(STAGES >= 2, "stages");
 };
-
-struct Seg {
-  int tile;
-  int kb0, kb1;
-};
-
-// Enumerates the (tile, k range) segments of one CTA; every role walks the
-// same sequence.
-struct SegIter {
-  const GemmArgs* g;
-  long long it, it_end;   // stream-K
-  int next_tile;          // round-robin
-  __device__ SegIter(const GemmArgs& args) : g(&args) {
-    const long long G = gridDim.x, c = blockIdx.x;
-    if (args.stream_k) {
-      it = c * args.iters_total / G;
-      it_end = (c + 1) * args.iters_total / G;
-    }
-    next_tile = blockIdx.x;
-  }
-  __device__ bool next(Seg& s) {
-    if (g->stream_k) {
-      if (it >= it_end) return false;
-      s.tile = static_cast<int>(it / g->kb_total);
-      s.kb0 = static_cast<int>(it - static_cast<long long>(s.tile) * g->kb_total);
-      const long long left = it_end - it;
-      s.kb1 = static_cast<int>(min(static_cast<long long>(g->kb_total), s.kb0 + left));
-      it += s.kb1 - s.kb0;
-      return true;
-    }
-    if (next_tile >= g->num_tiles) return false;
-    s.tile = next_tile;
-    next_tile += gridDim.x;
-    s.kb0 = 0;
-    s.kb1 = g->kb_total;
-    return true;
-  }
-};
-
-// Stream-K: number of CTAs whose ranges touch `tile`.
-__device__ __forceinline__ int sk_contributors(const GemmArgs& g, int tile) {
-  const long long G = gridDim.x, T = g.iters_total;
-  const long long first = static_cast<long long>(tile) * g.kb_total;
-  const long long last = first + g.kb_total - 1;
-  const long long c0 = ((first + 1) * G - 1) / T;
-  const long long c1 = ((last + 1) * G - 1) / T;
-  return static_cast<int>(c1 - c0 + 1);
-}
-
-// Block range of one BSR block row, clamped to [0, nnzb].  `sidx` holds crow
-// then col in shared memory, or is null (read global memory).
-__device__ __forceinline__ void bsr_range(const GemmArgs& g, const int* sidx, int br, int& p0, int& p1) {
-  int a = sidx ? sidx[br] : __ldg(g.crow + br);
-  int b = sidx ? sidx[br + 1] : __ldg(g.crow + br + 1);
-  a = min(max(a, 0), g.nnzb);
-  b = min(max(b, a), g.nnzb);
-  p0 = a;
-  p1 = b;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Epilogue for one chunk of 32 columns of the Dense/Bsr layout: thread = row
-// `row` (0..31 inside its warp's 32-row slab), output columns n0 .. n0+31.
-// The 32x32 block is written into the warp's staging buffer with the tensor
-// map's swizzle (64 B rows for bf16, 128 B rows for int32) and stored by one
-// TMA bulk store, which also clips rows >= M and columns >= N.  Scales and
-// bias are only read for columns < N (N % 8 == 0).
-__device__ __forceinline__ void store_row_chunk_tma(const GemmArgs& g, const CUtensorMap* tm_c,
-                                                    uint8_t* buf, int lane, int m0, int n0,
-                                                    const uint32_t* r, float srow) {
-  const uint32_t base = smem_u32(buf);
-  if (g.out_s32) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t off = static_cast<uint32_t>(lane * 128 + ((j ^ (lane & 7)) << 4));
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(r[4 * j]),
-                   "r"(r[4 * j + 1]), "r"(r[4 * j + 2]), "r"(r[4 * j + 3])
-                   : "memory");
-    }
-  } else {
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int n = n0 + 8 * v;
-      uint32_t w[4] = {0, 0, 0, 0};
-      if (n < g.N) {
-        const float4 c0 = __ldg(reinterpret_cast<const float4*>(g.s_col + n));
-        const float4 c1 = __ldg(reinterpret_cast<const float4*>(g.s_col + n + 4));
-        const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        float f[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          f[j] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[8 * v + j])), srow), sc[j]);
-        if (g.bias) {
-          const uint4 b = __ldg(reinterpret_cast<const uint4*>(g.bias + n));
-          const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            f[2 * j] = __fadd_rn(f[2 * j], __uint_as_float(bw[j] << 16));
-            f[2 * j + 1] = __fadd_rn(f[2 * j + 1], __uint_as_float(bw[j] & 0xffff0000u));
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) w[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
-      }
-      const uint32_t off = static_cast<uint32_t>(lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4));
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(w[0]), "r"(w[1]),
-                   "r"(w[2]), "r"(w[3])
-                   : "memory");
-    }
-  }
-  fence_proxy_async_smem();
-  __syncwarp();
-  if (lane == 0 && n0 < g.N && m0 < g.M) {   // boxes wholly past the matrix are not issued
-    tma_store_2d(tm_c, base, n0, m0);
-    bulk_commit_group();
-  }
-}
-
-// Epilogue for the Swap layout: thread = output channel n, columns are
-// tokens m0 .. m0+CW-1.
-template <int CW>
-__device__ __forceinline__ void store_col_chunk(const GemmArgs& g, int n, int m0, const uint32_t* r) {
-  if (n >= g.N) return;
-  if (g.out_s32) {
-    int32_t* o = static_cast<int32_t*>(g.out) + n;
-#pragma unroll
-    for (int j = 0; j < CW; ++j)
-      if (m0 + j < g.M) o[static_cast<int64_t>(m0 + j) * g.N] = static_cast<int>(r[j]);
-    return;
-  }
-  const float sc = __ldg(g.s_col + n);
-  const bool has_bias = g.bias != nullptr;
-  const float b = has_bias ? __uint_as_float(static_cast<uint32_t>(__ldg(g.bias + n)) << 16) : 0.0f;
-  uint16_t* o = static_cast<uint16_t*>(g.out) + n;
-#pragma unroll
-  for (int j = 0; j < CW; ++j) {
-    const int m = m0 + j;
-    if (m < g.M) {
-      float f = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), __ldg(g.s_row + m)), sc);
-      if (has_bias) f = __fadd_rn(f, b);
-      __nv_bfloat16 h = __float2bfloat16_rn(f);
-      o[static_cast<int64_t>(m) * g.N] = *reinterpret_cast<uint16_t*>(&h);
-    }
-  }
-}
 
 template <Kind KIND, int BN>
 __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
@@ -542,7 +366,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
           if (ep_tid == 0) g.ws_cnt[s.tile] = 0;
         }
         named_bar_sync(1, EPI_THREADS);   // sk_last is reused by the next partial tile
-      }
+            }
       if (++acc == C::ACC_BUFS) {
         acc = 0;
         acc_phase ^= 1;
@@ -603,8 +427,15 @@ dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap
 
 constexpr int64_t kMaxK = 133144;   // floor((2^31 - 1) / 127^2): int32 accumulation is exact
 
-// Schedule override for measurements: 0 = automatic, 1 = whole tiles, 2 = stream-K.
+// Measured on B200: the pair kernel only pays off when K is very large; for
+// K up to 8192 the 1-SM kernel is as fast or faster.
+constexpr int64_t kPairMinK = 16384;
+
+// Schedule override for measurements: 0 = automatic, 1 = 1-SM whole tiles,
+// 2 = 1-SM stream-K, 3 = pair (2-SM) kernel for every M.
 int g_schedule_override = 0;
+// Tile-width override for measurements (0 = automatic).
+int g_tile_n_override = 0;
 
 struct Plan {
   Kind kind;
@@ -613,6 +444,13 @@ struct Plan {
   bool stream_k;
   size_t ws_bytes;   // bytes needed for stream-K (0 if it never splits)
 };
+
+// Stream-K workspace: one int32 partial per tile ([BN][128], column-major so
+// that red.add of one column by a warp is one 512-byte line) plus an arrival
+// counter per tile.
+size_t sk_workspace_bytes(const Plan& p, int /*ctas*/) {
+  return static_cast<size_t>(p.num_tiles) * (static_cast<size_t>(p.bn) * 128 * 4 + 4);
+}
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count) {
   Plan p{};
@@ -624,6 +462,9 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count) {
   } else {
     p.kind = Kind::Dense;
     p.bn = N <= 128 ? 128 : 256;
+    if (g_tile_n_override == 128 || g_tile_n_override == 160 || g_tile_n_override == 192 ||
+        g_tile_n_override == 256)
+      p.bn = g_tile_n_override;
     p.a_tiles = static_cast<int>((M + 127) / 128);
     p.b_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
   }
@@ -637,8 +478,12 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count) {
   // Measured on B200: for the dense arrangement the partial-tile reduction
   // costs more than the idle SMs it saves, so only swap-AB (few tokens,
   // weight streaming) splits.
+  // Measured on B200: for the dense arrangement splitting costs more than the
+  // idle SMs of the last wave (both with red.add partials and with per-CTA
+  // partial slots plus ready flags), so only swap-AB (few tokens, weight
+  // streaming) splits.
   const bool worth = p.kind == Kind::Swap && eff < 0.9 && iters >= 4LL * sm_count;
-  p.ws_bytes = worth ? static_cast<size_t>(p.num_tiles) * (static_cast<size_t>(p.bn) * 128 * 4 + 4) : 0;
+  p.ws_bytes = worth ? sk_workspace_bytes(p, sm_count) : 0;
   p.stream_k = worth;
   return p;
 }
@@ -659,6 +504,7 @@ size_t dq_int8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
 
 // Measurement knob (not in the public header): force a schedule.
 void dq_debug_set_schedule(int mode) { g_schedule_override = mode; }
+void dq_debug_set_tile_n(int n) { g_tile_n_override = n; }
 
 dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K, const int8_t* W,
                          const float* s_col, int64_t N, const void* bias_bf16, void* out,
@@ -680,12 +526,42 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   if (st != DQ_OK) return st;
   if (M == 0) return DQ_OK;
 
+  // Dense arrangement: each 256x256 tile runs on a pair of SMs (gemm2sm.cu)
+  // unless a 1-SM schedule is forced for measurement (1 = whole tiles,
+  // 2 = stream-K); 3 forces the pair kernel for any M.
+  if ((M > 128 && K >= kPairMinK && g_schedule_override != 1 && g_schedule_override != 2) ||
+      g_schedule_override == 3) {
+    CUtensorMap ta, tb, tc;
+    if ((st = make_tmap_u8_2d(&ta, A, K, M, K, 128, 128, 128)) != DQ_OK) return st;
+    const int bn_pair = (g_tile_n_override == 160 || g_tile_n_override == 192) ? g_tile_n_override : 256;
+    if ((st = make_tmap_u8_2d(&tb, W, K, N, K, 128, bn_pair / 2, 128)) != DQ_OK) return st;
+    if ((st = make_tmap_out_2d(&tc, out, N, M, out_dtype == DQ_OUT_S32 ? 4 : 2)) != DQ_OK) return st;
+    GemmArgs g{};
+    g.M = static_cast<int>(M);
+    g.N = static_cast<int>(N);
+    g.K = static_cast<int>(K);
+    const int bn = (g_tile_n_override == 160 || g_tile_n_override == 192) ? g_tile_n_override : 256;
+    g.a_tiles = static_cast<int>((M + 255) / 256);
+    g.b_tiles = static_cast<int>((N + bn - 1) / bn);
+    g.kb_total = static_cast<int>((K + 127) / 128);
+    const int64_t tiles = static_cast<int64_t>(g.a_tiles) * g.b_tiles;
+    if (tiles > 0x7fffffff) return DQ_ERR_UNSUPPORTED;
+    g.num_tiles = static_cast<int>(tiles);
+    g.s_row = s_row;
+    g.s_col = s_col;
+    g.bias = static_cast<const uint16_t*>(bias_bf16);
+    g.out = out;
+    g.out_s32 = out_dtype == DQ_OUT_S32 ? 1 : 0;
+    g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
+    return launch_pair_gemm(ta, tb, tc, g, bn, *d, stream);
+  }
+
   Plan p = make_plan(M, N, K, d->sm_count);
   bool sk = p.stream_k && workspace != nullptr && workspace_bytes >= p.ws_bytes &&
             aligned(workspace, 16);
   if (g_schedule_override == 1) sk = false;
-  if (g_schedule_override == 2 && workspace != nullptr &&
-      workspace_bytes >= static_cast<size_t>(p.num_tiles) * (static_cast<size_t>(p.bn) * 128 * 4 + 4))
+  if (g_schedule_override == 2 && workspace != nullptr && aligned(workspace, 16) &&
+      workspace_bytes >= sk_workspace_bytes(p, d->sm_count))
     sk = static_cast<long long>(p.num_tiles) * p.kb_total >= d->sm_count;
 
   CUtensorMap ta, tb;
@@ -697,6 +573,7 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   if ((st = make_tmap_u8_2d(&tb, b_src, K, b_rows, K, 128, p.bn, 128)) != DQ_OK) return st;
   CUtensorMap tc;
   if ((st = make_tmap_out_2d(&tc, out, N, M, out_dtype == DQ_OUT_S32 ? 4 : 2)) != DQ_OK) return st;
+  const size_t slots_bytes = static_cast<size_t>(p.num_tiles) * p.bn * 128 * 4;
 
   GemmArgs g{};
   g.M = static_cast<int>(M);
@@ -715,15 +592,18 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   g.out_s32 = out_dtype == DQ_OUT_S32 ? 1 : 0;
   if (sk) {
     g.ws = static_cast<int32_t*>(workspace);
-    g.ws_cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) +
-                                           static_cast<size_t>(p.num_tiles) * p.bn * 128 * 4);
+    g.ws_cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + slots_bytes);
   }
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
   const int grid = sk ? d->sm_count : (p.num_tiles < d->sm_count ? p.num_tiles : d->sm_count);
 
   if (p.kind == Kind::Dense) {
-    if (p.bn == 256) return launch<Kind::Dense, 256>(ta, tb, tc, g, grid, stream);
-    return launch<Kind::Dense, 128>(ta, tb, tc, g, grid, stream);
+    switch (p.bn) {
+      case 256: return launch<Kind::Dense, 256>(ta, tb, tc, g, grid, stream);
+      case 192: return launch<Kind::Dense, 192>(ta, tb, tc, g, grid, stream);
+      case 160: return launch<Kind::Dense, 160>(ta, tb, tc, g, grid, stream);
+      default: return launch<Kind::Dense, 128>(ta, tb, tc, g, grid, stream);
+    }
   }
   switch (p.bn) {
     case 16: return launch<Kind::Swap, 16>(ta, tb, tc, g, grid, stream);

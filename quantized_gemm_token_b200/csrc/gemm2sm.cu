@@ -1,0 +1,309 @@
+// gemm2sm.cu -- the dense int8 x int8 -> int32 GEMM with the fused
+// dequantization epilogue (pytorch/ao PR 821, "int8 dynamic quant + bsr
+// support": i8i8->bf16 with no int32 intermediate in global memory), with
+// each MMA spread over a pair of SMs (a thread-block cluster of 2 CTAs and
+// tcgen05.mma.cta_group::2).
+//
+// Why a pair: with one SM per 128x256 tile, every 128-clock MMA step needs
+// 12 KB of operands written into shared memory by TMA and read back by the
+// tensor core, which the SM cannot sustain.  A pair computes a 256x256 tile:
+// each CTA loads 128 rows of A and 128 rows (half) of B per k step, and the
+// pair MMA reads each CTA's halves once for both SMs' tensor cores, so the
+// per-SM shared-memory traffic per step drops by a third.
+//
+// Roles (both CTAs run the same code; rank 0 of the cluster leads):
+//   warp 0      TMA producer in each CTA: its A and B halves into its own
+//               stage ring; the loads complete on the LEADER's full barrier,
+//               which expects the bytes of both CTAs.
+//   warp 1      MMA issuer, leader only: tcgen05.mma.cta_group::2.kind::i8
+//               (M = 256, N = 256, K = 32); tcgen05.commit frees the stage in
+//               both CTAs (one commit per CTA) and hands the accumulator to
+//               both CTAs' epilogues.
+//   warps 2..9  epilogue in each CTA: its 128 accumulator rows out of its own
+//               TMEM, the same fp32 dequantization and TMA-store path as the
+//               1-SM kernel; each warp then tells the leader (remote arrive)
+//               that its part of the accumulator is free.
+// No load is multicast: each CTA fetches its own operand halves.
+#include <mutex>
+
+#include "gemm_common.cuh"
+
+namespace dq {
+
+// BN: pair tile width (output columns); each CTA holds BN/2 rows of B.
+template <int BN>
+struct Cfg2 {
+  static constexpr int KB = 128;                        // k bytes per stage
+  static constexpr int A_BYTES = 128 * KB;              // this CTA's 128 rows of A
+  static constexpr int B_BYTES = (BN / 2) * KB;         // this CTA's half of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int OUT_BUF_BYTES = 32 * 32 * 4;     // per epilogue warp
+  static constexpr int OUT_BYTES = EPI_WARPS * OUT_BUF_BYTES;
+  static constexpr int STAGES = (224 * 1024 - OUT_BYTES) / STAGE_BYTES;
+  static constexpr int ACC_BUFS = 512 / BN >= 3 ? 3 : 2;  // accumulators of BN TMEM columns
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int K_STEPS = KB / 32;
+  static constexpr int CW = 32;
+  static constexpr int NCH = BN / CW;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_BYTES + 1024 + 512;
+  static_assert(STAGES >= 3, "stages");
+  static_assert(BN % 32 == 0 && BN <= 256 && (BN / 2) % 8 == 0, "tile width");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(Cfg2<BN>::THREADS, 1)
+    gemm2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                 const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ GemmArgs g) {
+  using C = Cfg2<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint8_t* sOut = smem + C::STAGES * C::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + C::OUT_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + C::STAGES;
+  uint64_t* accf_bar = bars + 2 * C::STAGES;
+  uint64_t* acce_bar = accf_bar + C::ACC_BUFS;
+  uint64_t* drain_bar = acce_bar + C::ACC_BUFS;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int G = gridDim.x >> 1;                // CTA pairs
+  const int pair = blockIdx.x >> 1;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(full_bar + s), 1);
+      mbar_init(smem_u32(empty_bar + s), 1);
+    }
+    for (int a = 0; a < C::ACC_BUFS; ++a) {
+      mbar_init(smem_u32(accf_bar + a), 1);
+      mbar_init(smem_u32(acce_bar + a), 2 * C::EPI_WARPS);   // one arrive per epilogue warp of both CTAs
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_c);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();            // both CTAs' barriers are initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < g.num_tiles; t += G) {
+        const int ta = t / g.b_tiles, tb = t % g.b_tiles;
+        for (int kb = 0; kb < g.kb_total; ++kb) {
+          if (!mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, g.wait, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(full_bar + stage);
+          if (leader) mbar_arrive_expect_tx(fb, 2 * C::STAGE_BYTES);
+          const uint32_t fb_leader = map_to_rank(fb, 0);
+          tma_load_2d_pair(smem_u32(sA + stage * C::A_BYTES), &tm_a, fb_leader, kb * C::KB,
+                           ta * 256 + static_cast<int>(rank) * 128);
+          tma_load_2d_pair(smem_u32(sB + stage * C::B_BYTES), &tm_b, fb_leader, kb * C::KB,
+                           tb * BN + static_cast<int>(rank) * (BN / 2));
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let loads already issued land before the CTA leaves: the leader
+        // waits on its full barriers (bounded); the follower, whose loads
+        // complete on the leader's barriers, waits a fixed 100 us.
+        if (leader) {
+          WaitCtl quick = g.wait;
+          quick.timeout_ns = quick.timeout_ns < 50000000ull ? quick.timeout_ns : 50000000ull;
+          volatile int never = 0;
+          for (long long i = 0; i < issued && i < C::STAGES; ++i) {
+            if (--stage < 0) {
+              stage = C::STAGES - 1;
+              phase ^= 1;
+            }
+            mbar_wait(smem_u32(full_bar + stage), phase, quick, &never);
+          }
+        } else {
+          const uint64_t t0 = globaltimer();
+          while (globaltimer() - t0 < 100000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(256, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < g.num_tiles; t += G) {
+        if (!mbar_wait(smem_u32(acce_bar + acc), acc_phase ^ 1, g.wait, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < g.kb_total; ++kb) {
+          if (!mbar_wait(smem_u32(full_bar + stage), phase, g.wait, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = smem_desc_kmajor<C::KB>(smem_u32(sA + stage * C::A_BYTES));
+          const uint64_t bd = smem_desc_kmajor<C::KB>(smem_u32(sB + stage * C::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < C::K_STEPS; ++k)
+            mma_i8_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          const uint32_t eb = smem_u32(empty_bar + stage);
+          mma_commit_pair(map_to_rank(eb, 0));
+          mma_commit_pair(map_to_rank(eb, 1));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        const uint32_t fb = smem_u32(accf_bar + acc);
+        mma_commit_pair(map_to_rank(fb, 0));
+        mma_commit_pair(map_to_rank(fb, 1));
+        if (++acc == C::ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      mma_commit_pair(map_to_rank(smem_u32(drain_bar), 0));
+      volatile int never = 0;
+      mbar_wait(smem_u32(drain_bar), 0, g.wait, &never);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    constexpr int GROUPS = C::EPI_WARPS / 4;
+    const int ew = warp - 2;
+    const int sp = warp & 3;
+    const int grp = ew / 4;
+    uint8_t* my_out = sOut + ew * C::OUT_BUF_BYTES;
+    int out_flip = 0;
+    auto next_buf = [&]() -> uint8_t* {
+      if (g.out_s32) {
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        return my_out;
+      }
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+      uint8_t* b = my_out + out_flip * (C::OUT_BUF_BYTES / 2);
+      out_flip ^= 1;
+      return b;
+    };
+    const int last_c = grp + ((C::NCH - 1 - grp) / GROUPS) * GROUPS;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < g.num_tiles; t += G) {
+      const int ta = t / g.b_tiles, tb = t % g.b_tiles;
+      if (!mbar_wait(smem_u32(accf_bar + acc), acc_phase, g.wait, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const int m_slab = ta * 256 + static_cast<int>(rank) * 128 + sp * 32;
+      const int m = m_slab + lane;
+      const float srow = (!g.out_s32 && m < g.M) ? __ldg(g.s_row + m) : 0.0f;
+#pragma unroll 1
+      for (int c = grp; c < C::NCH; c += GROUPS) {
+        uint32_t r[C::CW];
+        tmem_ld_32x32b_x32(tbase + c * C::CW, r);
+        tmem_ld_wait();
+        if (c == last_c) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(acce_bar + acc), 0));
+        }
+        store_row_chunk_tma(g, &tm_c, next_buf(), lane, m_slab, tb * BN + c * C::CW, r, srow);
+      }
+      if (++acc == C::ACC_BUFS) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync_all();            // no CTA leaves while its peer may still signal it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+}
+
+namespace {
+
+template <int BN>
+dq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& g,
+                      const DeviceInfo& d, cudaStream_t stream) {
+  using C = Cfg2<BN>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int max_clusters[64] = {};
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm2_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int& maxc = max_clusters[d.device & 63];
+  if (maxc == 0) {
+    cfg.gridDim = dim3(2 * (d.sm_count / 2));
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm2_kernel<BN>, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e);
+    maxc = n > 0 ? n : 1;
+  }
+  const int pairs = g.num_tiles < maxc ? g.num_tiles : maxc;
+  cfg.gridDim = dim3(2 * pairs);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm2_kernel<BN>, ta, tb, tc, g);
+  return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+// Launches gemm2_kernel with clusters of 2 CTAs, one pair per resident
+// cluster slot (persistent).  bn: pair tile width (160, 192 or 256).
+dq_status launch_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, GemmArgs g,
+                           int bn, const DeviceInfo& d, cudaStream_t stream) {
+  switch (bn) {
+    case 160: return launch_pair<160>(ta, tb, tc, g, d, stream);
+    case 192: return launch_pair<192>(ta, tb, tc, g, d, stream);
+    default: return launch_pair<256>(ta, tb, tc, g, d, stream);
+  }
+}
+
+}  // namespace dq

@@ -1,0 +1,192 @@
+// gemm_common.cuh -- pieces shared by the 1-SM and 2-SM int8 GEMM kernels:
+// launch arguments, the per-CTA tile schedule, BSR index access and the
+// dequantize / bf16 / store epilogue helpers.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace dq {
+
+enum class Kind : int { Dense = 0, Swap = 1, Bsr = 2 };
+
+struct GemmArgs {
+  int M, N, K;
+  int a_tiles, b_tiles;   // tiles along the A slot (128 rows) and the B slot (BN rows)
+  int kb_total;           // k blocks per tile (Dense / Swap)
+  int num_tiles;
+  int stream_k;           // 0: whole tiles round-robin; 1: stream-K ranges
+  long long iters_total;  // num_tiles * kb_total (stream-K)
+  const float* s_row;
+  const float* s_col;
+  const uint16_t* bias;   // bf16 bits or null
+  void* out;
+  int out_s32;
+  int32_t* ws;            // stream-K partial tiles: [tile][BN][128] int32
+  uint32_t* ws_cnt;       // stream-K arrival counters: [tile]
+  const int32_t* crow;    // Bsr
+  const int32_t* col;
+  int nnzb;
+  int nbr;                // Bsr: block rows (N / 64)
+  int idx_smem;           // Bsr: crow and col staged in shared memory (they fit)
+  WaitCtl wait;
+};
+
+
+struct Seg {
+  int tile;
+  int kb0, kb1;
+};
+
+// Enumerates the (tile, k range) segments of one CTA; every role walks the
+// same sequence.
+struct SegIter {
+  const GemmArgs* g;
+  long long it, it_end;   // stream-K
+  int next_tile;          // round-robin
+  __device__ SegIter(const GemmArgs& args) : g(&args) {
+    const long long G = gridDim.x, c = blockIdx.x;
+    if (args.stream_k) {
+      it = c * args.iters_total / G;
+      it_end = (c + 1) * args.iters_total / G;
+    }
+    next_tile = blockIdx.x;
+  }
+  __device__ bool next(Seg& s) {
+    if (g->stream_k) {
+      if (it >= it_end) return false;
+      s.tile = static_cast<int>(it / g->kb_total);
+      s.kb0 = static_cast<int>(it - static_cast<long long>(s.tile) * g->kb_total);
+      const long long left = it_end - it;
+      s.kb1 = static_cast<int>(min(static_cast<long long>(g->kb_total), s.kb0 + left));
+      it += s.kb1 - s.kb0;
+      return true;
+    }
+    if (next_tile >= g->num_tiles) return false;
+    s.tile = next_tile;
+    next_tile += gridDim.x;
+    s.kb0 = 0;
+    s.kb1 = g->kb_total;
+    return true;
+  }
+};
+
+// Stream-K: number of CTAs whose ranges touch `tile`.
+__device__ __forceinline__ int sk_contributors(const GemmArgs& g, int tile) {
+  const long long G = gridDim.x, T = g.iters_total;
+  const long long first = static_cast<long long>(tile) * g.kb_total;
+  const long long last = first + g.kb_total - 1;
+  const long long c0 = ((first + 1) * G - 1) / T;
+  const long long c1 = ((last + 1) * G - 1) / T;
+  return static_cast<int>(c1 - c0 + 1);
+}
+
+// Block range of one BSR block row, clamped to [0, nnzb].  `sidx` holds crow
+// then col in shared memory, or is null (read global memory).
+__device__ __forceinline__ void bsr_range(const GemmArgs& g, const int* sidx, int br, int& p0, int& p1) {
+  int a = sidx ? sidx[br] : __ldg(g.crow + br);
+  int b = sidx ? sidx[br + 1] : __ldg(g.crow + br + 1);
+  a = min(max(a, 0), g.nnzb);
+  b = min(max(b, a), g.nnzb);
+  p0 = a;
+  p1 = b;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Epilogue for one chunk of 32 columns of the Dense/Bsr layout: thread = row
+// `row` (0..31 inside its warp's 32-row slab), output columns n0 .. n0+31.
+// The 32x32 block is written into the warp's staging buffer with the tensor
+// map's swizzle (64 B rows for bf16, 128 B rows for int32) and stored by one
+// TMA bulk store, which also clips rows >= M and columns >= N.  Scales and
+// bias are only read for columns < N (N % 8 == 0).
+__device__ __forceinline__ void store_row_chunk_tma(const GemmArgs& g, const CUtensorMap* tm_c,
+                                                    uint8_t* buf, int lane, int m0, int n0,
+                                                    const uint32_t* r, float srow) {
+  const uint32_t base = smem_u32(buf);
+  if (g.out_s32) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t off = static_cast<uint32_t>(lane * 128 + ((j ^ (lane & 7)) << 4));
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(r[4 * j]),
+                   "r"(r[4 * j + 1]), "r"(r[4 * j + 2]), "r"(r[4 * j + 3])
+                   : "memory");
+    }
+  } else {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int n = n0 + 8 * v;
+      uint32_t w[4] = {0, 0, 0, 0};
+      if (n < g.N) {
+        const float4 c0 = __ldg(reinterpret_cast<const float4*>(g.s_col + n));
+        const float4 c1 = __ldg(reinterpret_cast<const float4*>(g.s_col + n + 4));
+        const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          f[j] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[8 * v + j])), srow), sc[j]);
+        if (g.bias) {
+          const uint4 b = __ldg(reinterpret_cast<const uint4*>(g.bias + n));
+          const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            f[2 * j] = __fadd_rn(f[2 * j], __uint_as_float(bw[j] << 16));
+            f[2 * j + 1] = __fadd_rn(f[2 * j + 1], __uint_as_float(bw[j] & 0xffff0000u));
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
+      }
+      const uint32_t off = static_cast<uint32_t>(lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4));
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(w[0]), "r"(w[1]),
+                   "r"(w[2]), "r"(w[3])
+                   : "memory");
+    }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && n0 < g.N && m0 < g.M) {   // boxes wholly past the matrix are not issued
+    tma_store_2d(tm_c, base, n0, m0);
+    bulk_commit_group();
+  }
+}
+
+// Epilogue for the Swap layout: thread = output channel n, columns are
+// tokens m0 .. m0+CW-1.
+template <int CW>
+__device__ __forceinline__ void store_col_chunk(const GemmArgs& g, int n, int m0, const uint32_t* r) {
+  if (n >= g.N) return;
+  if (g.out_s32) {
+    int32_t* o = static_cast<int32_t*>(g.out) + n;
+#pragma unroll
+    for (int j = 0; j < CW; ++j)
+      if (m0 + j < g.M) o[static_cast<int64_t>(m0 + j) * g.N] = static_cast<int>(r[j]);
+    return;
+  }
+  const float sc = __ldg(g.s_col + n);
+  const bool has_bias = g.bias != nullptr;
+  const float b = has_bias ? __uint_as_float(static_cast<uint32_t>(__ldg(g.bias + n)) << 16) : 0.0f;
+  uint16_t* o = static_cast<uint16_t*>(g.out) + n;
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    const int m = m0 + j;
+    if (m < g.M) {
+      float f = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), __ldg(g.s_row + m)), sc);
+      if (has_bias) f = __fadd_rn(f, b);
+      __nv_bfloat16 h = __float2bfloat16_rn(f);
+      o[static_cast<int64_t>(m) * g.N] = *reinterpret_cast<uint16_t*>(&h);
+    }
+  }
+}
+
+// Dense GEMM with each 256 x bn tile's MMA on a pair of SMs (gemm2sm.cu).
+// g.a_tiles / g.b_tiles count 256-row / bn-column tiles; bn is 160, 192 or 256.
+dq_status launch_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, GemmArgs g,
+                           int bn, const DeviceInfo& d, cudaStream_t stream);
+
+}  // namespace dq

@@ -48,5 +48,11 @@ inline bool aligned(const void* p, size_t a) {
 }  // namespace dq
 
 // Measurement knob, not part of the public header: 0 = automatic schedule,
-// 1 = whole tiles only, 2 = stream-K whenever a workspace allows it.
+// 1 = 1-SM kernel with whole tiles, 2 = 1-SM stream-K whenever a workspace
+// allows it, 3 = the 2-SM pair kernel for every M.
 extern "C" DQ_API void dq_debug_set_schedule(int mode);
+// Measurement knob: force the dense tile width (128, 160, 192, 256; 0 = automatic).
+extern "C" DQ_API void dq_debug_set_tile_n(int n);
+// Measurement knob: quantize kernel (0 = automatic, 1 = register-resident,
+// 2 = row-pipelined through shared memory).
+extern "C" DQ_API void dq_debug_set_quant_kernel(int mode);

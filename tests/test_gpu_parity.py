@@ -108,7 +108,9 @@ def _gemm_inputs(M, N, K, seed):
     return A, W, s_row, s_col, bias
 
 
-@pytest.mark.parametrize("schedule", [1, 2])
+# schedule: 1 = 1-SM kernel, whole tiles; 2 = 1-SM stream-K (where a split is
+# possible); 3 = the 2-SM pair kernel (any M)
+@pytest.mark.parametrize("schedule", [1, 2, 3])
 @pytest.mark.parametrize("M,N,K", GSHAPES)
 def test_dense_parity(M, N, K, schedule):
     A, W, s_row, s_col, bias = _gemm_inputs(M, N, K, 300 + M + N + K)
@@ -132,10 +134,10 @@ def test_stream_k_and_whole_tiles_agree():
         Ad, Wd = to_dev(A), to_dev(W)
         ws = torch.zeros(dq.dq_int8_linear_workspace_size(M, N, K) or 1 << 20, dtype=torch.uint8, device="cuda")
         outs = []
-        for mode in (1, 2):
+        for mode in (1, 2, 3):
             dq.dq_debug_set_schedule(mode)
             outs.append(dq.dq_int8_linear(Ad, None, Wd, None, out_dtype="s32", workspace=ws).cpu().numpy())
-        assert np.array_equal(outs[0], outs[1])
+        assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
         rows = sample_rows(M, 24)
         assert np.array_equal(outs[0][rows], oracle.gemm_s32(A[rows], W))
 
@@ -396,3 +398,22 @@ def test_quantize_weight_near_ties_fp32():
     wo, so = oracle.quantize_rows_f32(w)
     assert np.array_equal(sc.cpu().numpy().view(np.uint32), so.view(np.uint32))
     assert np.array_equal(wq.cpu().numpy(), wo)
+
+
+@pytest.mark.parametrize("tile_n", [160, 192])
+@pytest.mark.parametrize("schedule", [1, 3])
+@pytest.mark.parametrize("M,N,K", [(300, 520, 384), (513, 1032, 4096), (129, 168, 256), (2048, 4096, 512)])
+def test_dense_tile_widths(M, N, K, schedule, tile_n):
+    A, W, s_row, s_col, bias = _gemm_inputs(M, N, K, 700 + M + N)
+    dq.dq_debug_set_schedule(schedule)
+    dq.dq_debug_set_tile_n(tile_n)
+    try:
+        Ad, Wd = to_dev(A), to_dev(W)
+        acc = dq.dq_int8_linear(Ad, None, Wd, None, out_dtype="s32")
+        rows = sample_rows(M, 64)
+        want = oracle.gemm_s32(A[rows], W)
+        assert np.array_equal(acc.cpu().numpy()[rows], want)
+        out = dq.dq_int8_linear(Ad, to_dev(s_row), Wd, to_dev(s_col), bias=to_dev_bf16(bias))
+        assert_bf16_close(bf16_bits(out)[rows], oracle.epilogue_bf16(want, s_row[rows], s_col, bias))
+    finally:
+        dq.dq_debug_set_tile_n(0)
