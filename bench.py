@@ -11,10 +11,10 @@ the bf16 activations (dq_quantize_rows) and the fused i8i8->bf16 GEMM
 LLM-shaped dense linear: M=2048 tokens, K=4096, N=4096, 1% outlier channels.
 
 Timing: W warm-up steps, then EXACTLY K steps captured in one CUDA graph and
-replayed once, bracketed by a barrier and a device synchronize; the graph
-holds event-record nodes between the kernels so each kernel's average
-duration is measured live.  Inputs rotate over enough copies to exceed the
-126 MB L2 (stated in config.l2).  Multi-GPU: one process per GPU, token
+replayed once, bracketed by a barrier and a device synchronize (the value).
+Each kernel's average duration (kernels_ms, roofline) comes from a graph of K
+launches of that kernel alone on the same buffers, timed right after.
+Inputs rotate over enough copies to exceed the 126 MB L2 (config.l2).  Multi-GPU: one process per GPU, token
 batches sharded across ranks (weak scaling, no data-path collective); the
 reported time is the max over ranks.
 
@@ -37,6 +37,32 @@ sys.path.insert(0, ROOT)
 METRIC = "int8 dyn-quant linear TOPS (dense & BSR) vs INT8 peak; quant kernel HBM GB/s"
 L2_BYTES = 126 * 1024 * 1024
 INT8_PER_BF16 = 2.0   # nominal dense int8 / bf16 tensor ratio (4.5 / 2.25 PFLOP/s)
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources: a stored ncu traffic figure only applies to
+    the kernels it was measured on."""
+    import hashlib
+    d = os.path.join(ROOT, "quantized_gemm_token_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch (read + write) of `kernel` in `workload` from
+    profiles/traffic.json (written from an ncu capture), or None when absent
+    or taken on different kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            t = json.load(f)
+        e = t[workload][kernel]
+        return e["bytes_per_launch"] if e.get("source_hash") == kernel_source_hash() else None
+    except Exception:
+        return None
 
 
 def load_peaks():
@@ -183,34 +209,6 @@ class ClockSampler:
 # GPU arm
 # ----------------------------------------------------------------------------
 
-class ExtEvents:
-    """Timing events recorded as graph nodes (cudaEventRecordExternal), so
-    that kernel boundaries inside a captured CUDA graph can be timed."""
-
-    def __init__(self, n):
-        from cuda.bindings import runtime as rt
-        self.rt = rt
-        self.ev = []
-        for _ in range(n):
-            err, e = rt.cudaEventCreateWithFlags(rt.cudaEventDefault)
-            assert err == rt.cudaError_t.cudaSuccess, err
-            self.ev.append(e)
-
-    def record(self, i, stream_handle):
-        err, = self.rt.cudaEventRecordWithFlags(self.ev[i], self.rt.cudaStream_t(stream_handle),
-                                                self.rt.cudaEventRecordExternal)
-        assert err == self.rt.cudaError_t.cudaSuccess, err
-
-    def elapsed_ms(self, i, j):
-        err, ms = self.rt.cudaEventElapsedTime(self.ev[i], self.ev[j])
-        assert err == self.rt.cudaError_t.cudaSuccess, err
-        return ms
-
-    def destroy(self):
-        for e in self.ev:
-            self.rt.cudaEventDestroy(e)
-
-
 def _to_dev(torch, a):
     import numpy as np
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
@@ -219,6 +217,17 @@ def _to_dev(torch, a):
 def _to_dev_bf16(torch, bits):
     import numpy as np
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _finish(st):
+    """One step = the workload's kernels in order, each one launch."""
+    kernels = st["kernels"]
+
+    def step(c, stream):
+        for k in kernels:
+            k(c, stream)
+    st["step"], st["n_kernels"] = step, len(kernels)
+    return st
 
 
 def make_state(name, wl, dq, torch, seed):
@@ -238,13 +247,9 @@ def make_state(name, wl, dq, torch, seed):
         st["h2d"] = [("x", x.numel() * 2)]
         st["d2h"] = [("q", M * K), ("s", M * 4)]
 
-        def step(c, stream, ev=None, base=0):
-            if ev:
-                ev.record(base, stream.cuda_stream)
-            dq.dq_quantize_rows(c["x"], q, s, stream=stream)
-        st["step"], st["n_kernels"] = step, 1
+        st["kernels"] = [lambda c, stream: dq.dq_quantize_rows(c["x"], q, s, stream=stream)]
         st["names"] = ["dq_quantize_rows"]
-        return st
+        return _finish(st)
     if k == "gemm":
         A, B = _to_dev(torch, d["a"]), _to_dev(torch, d["b"])
         sr, sc = _to_dev(torch, d["s_row"]), _to_dev(torch, d["s_col"])
@@ -257,14 +262,11 @@ def make_state(name, wl, dq, torch, seed):
         st["h2d"] = [("A", M * K)]
         st["d2h"] = [("out", out.numel() * out.element_size())]
 
-        def step(c, stream, ev=None, base=0):
-            if ev:
-                ev.record(base, stream.cuda_stream)
-            dq.dq_int8_linear(c["A"], sr, c["B"], sc, out=out, out_dtype="s32" if out_s32 else "bf16",
-                              stream=stream)
-        st["step"], st["n_kernels"], st["names"] = step, 1, ["dq_int8_linear"]
+        st["kernels"] = [lambda c, stream: dq.dq_int8_linear(c["A"], sr, c["B"], sc, out=out,
+                                                             out_dtype="s32" if out_s32 else "bf16", stream=stream)]
+        st["names"] = ["dq_int8_linear"]
         st["out"] = out
-        return st
+        return _finish(st)
     # layer workloads: quantize + GEMM
     if k == "dense":
         w = _to_dev(torch, d["w"])
@@ -284,15 +286,11 @@ def make_state(name, wl, dq, torch, seed):
         st["h2d"] = [("x", M * K * 2)]
         st["d2h"] = [("out", M * N * 2)]
 
-        def step(c, stream, ev=None, base=0):
-            if ev:
-                ev.record(base, stream.cuda_stream)
-            dq.dq_quantize_rows(c["x"], q, s, stream=stream)
-            if ev:
-                ev.record(base + 1, stream.cuda_stream)
-            dq.dq_int8_linear(q, s, c["W"], sc, bias=bias, out=out, workspace=ws, stream=stream)
-        st["step"], st["n_kernels"], st["names"] = step, 2, ["dq_quantize_rows", "dq_int8_linear"]
-        return st
+        st["kernels"] = [
+            lambda c, stream: dq.dq_quantize_rows(c["x"], q, s, stream=stream),
+            lambda c, stream: dq.dq_int8_linear(q, s, c["W"], sc, bias=bias, out=out, workspace=ws, stream=stream)]
+        st["names"] = ["dq_quantize_rows", "dq_int8_linear"]
+        return _finish(st)
     if k in ("bsr", "bsr_dense"):
         w = _to_dev(torch, d["w"])
         wq, sc = dq.dq_quantize_weight(w)
@@ -312,19 +310,14 @@ def make_state(name, wl, dq, torch, seed):
         st["d2h"] = [("out", M * N * 2)]
         dense = k == "bsr_dense"
 
-        def step(c, stream, ev=None, base=0):
-            if ev:
-                ev.record(base, stream.cuda_stream)
-            dq.dq_quantize_rows(c["x"], q, s, stream=stream)
-            if ev:
-                ev.record(base + 1, stream.cuda_stream)
+        def gemm(c, stream):
             if dense:
                 dq.dq_int8_linear(q, s, wq, sc, out=out, stream=stream)
             else:
                 dq.dq_bsr_int8_linear(q, s, N, crow, col, values, sc, out=out, stream=stream)
-        st["step"], st["n_kernels"] = step, 2
+        st["kernels"] = [lambda c, stream: dq.dq_quantize_rows(c["x"], q, s, stream=stream), gemm]
         st["names"] = ["dq_quantize_rows", "dq_int8_linear" if dense else "dq_bsr_int8_linear"]
-        return st
+        return _finish(st)
     raise ValueError(k)
 
 
@@ -404,21 +397,32 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     assert dq.dq_sync_status() == dq.DQ_OK
 
-    # capture exactly K steps, with timing event nodes between kernels
-    ev = ExtEvents(nk * K + 1)
-    graph = torch.cuda.CUDAGraph()
-    cap_stream = torch.cuda.Stream()
-    cap_stream.wait_stream(stream)
-    with torch.cuda.stream(cap_stream):
-        graph.capture_begin()
-        for i in range(K):
-            step(copies[i % len(copies)], cap_stream, ev=ev, base=nk * i)
-        ev.record(nk * K, cap_stream.cuda_stream)
-        graph.capture_end()
-    stream.wait_stream(cap_stream)
-    graph.replay()            # one untimed replay (graph upload)
-    torch.cuda.synchronize()
+    def capture(launch):
+        """A CUDA graph of K launches of `launch(i, stream)`, uploaded once."""
+        graph = torch.cuda.CUDAGraph()
+        cap_stream = torch.cuda.Stream()
+        cap_stream.wait_stream(stream)
+        with torch.cuda.stream(cap_stream):
+            graph.capture_begin()
+            for i in range(K):
+                launch(i, cap_stream)
+            graph.capture_end()
+        stream.wait_stream(cap_stream)
+        graph.replay()            # one untimed replay (graph upload)
+        torch.cuda.synchronize()
+        return graph
 
+    def timed_replay(graph):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    # The timed region: one graph of exactly K steps (nothing between kernels).
+    graph = capture(lambda i, cs: step(copies[i % len(copies)], cs))
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
@@ -430,10 +434,15 @@ def run_gpu(args, rank, world, local_rank):
     barrier()
     total_ms = start.elapsed_time(end)
     assert dq.dq_sync_status() == dq.DQ_OK
-    # per-kernel durations from the event nodes
-    per_kernel = [[ev.elapsed_ms(nk * i + j, nk * i + j + 1) for i in range(K)] for j in range(nk)]
-    ev.destroy()
     del graph
+    # Per-kernel durations: right after, a graph of K launches of each kernel
+    # alone (same buffers, same input rotation), timed with events around it.
+    per_kernel_ms = []
+    for j, kern in enumerate(state["kernels"]):
+        gj = capture(lambda i, cs, kern=kern: kern(copies[i % len(copies)], cs))
+        per_kernel_ms.append(timed_replay(gj) / K)
+        del gj
+    assert dq.dq_sync_status() == dq.DQ_OK
     total_ms_max = max_over_ranks(total_ms)
 
     value = ops * world * K / (total_ms_max * 1e-3) / 1e12 if ops else None
@@ -444,7 +453,7 @@ def run_gpu(args, rank, world, local_rank):
 
     # roofline of the dominant kernel
     j = state["names"].index(dom["kernel"])
-    avg_ms = sum(per_kernel[j]) / K
+    avg_ms = per_kernel_ms[j]
     int8_peak = peaks["bf16"] * INT8_PER_BF16
     if dom["kernel"] == "dq_quantize_rows" or wl.get("out") == "s32" or wl["kind"] == "bsr":
         t_tensor = dom["ops"] / (int8_peak * 1e12) if dom["ops"] else 0.0
@@ -465,9 +474,10 @@ def run_gpu(args, rank, world, local_rank):
                     frac=round(achieved / int8_peak, 4), traffic=None,
                     peak_source=f"{peaks['src']} bf16 burst x {INT8_PER_BF16:g} (nominal int8/bf16 ratio)")
     roof["kernel"] = dom["kernel"]
+    roof["traffic"] = measured_traffic(name, dom["kernel"])
     roof["avg_launch_ms"] = round(avg_ms, 5)
     roof["algorithmic_bytes" if hbm_bound else "algorithmic_ops"] = dom["bytes"] if hbm_bound else dom["ops"]
-    kernels_ms = {n: round(sum(per_kernel[i]) / K, 5) for i, n in enumerate(state["names"])}
+    kernels_ms = {n: round(per_kernel_ms[i], 5) for i, n in enumerate(state["names"])}
 
     # end to end through the public API with host buffers
     e2e = None
@@ -480,7 +490,9 @@ def run_gpu(args, rank, world, local_rank):
                 config=dict(workload=wl["desc"], tokens_per_rank=state["d"].get("M", wl.get("M")),
                             parallelism=f"dp{world} (token rows sharded, weights replicated, no collective)",
                             l2=f"inputs rotate over {len(copies)} copies (> 2x the 126 MB L2)",
-                            timing="one CUDA graph of K steps; event-record nodes between kernels",
+                            timing="value: one CUDA graph of the K steps, events around it; "
+                                   "kernels_ms / roofline: per kernel, a graph of K launches of that "
+                                   "kernel alone on the same buffers, events around it",
                             kernels_ms=kernels_ms),
                 roofline=roof, e2e=e2e, gpu_launches=nk * K, clocks=cs.summary())
     if rank == 0 and world == 1 and not args.no_cpu_baseline and wl["kind"] in ("dense", "bsr", "quant", "gemm"):

@@ -122,6 +122,10 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
   }
+  // Everything above touched only shared memory, TMEM and the kernel
+  // parameters; with a programmatic (early) launch, wait here for the
+  // previous kernel of the stream before any global memory access.
+  griddep_wait();
   const int* idx = nullptr;      // Bsr: crow at idx[0..nbr], col at idx[nbr+1..]
   if constexpr (KIND == Kind::Bsr) {
     if (g.idx_smem) {
@@ -420,8 +424,20 @@ dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap
                                     C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err);
-  gemm_kernel<KIND, BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ta, tb, tc, args);
-  cudaError_t e = cudaGetLastError();
+  // Programmatic stream serialization: the prologue may overlap the tail of
+  // the previous kernel (e.g. the quantization that produced A); the kernel
+  // waits (griddep_wait) before its first global memory access.
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN>, ta, tb, tc, args);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 

@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(Cfg2<BN>::THREADS, 1)
   cluster_sync_all();            // both CTAs' barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  griddep_wait();                // programmatic launch: previous kernel done before global access
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -269,11 +270,13 @@ dq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
@@ -289,6 +292,7 @@ dq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
   }
   const int pairs = g.num_tiles < maxc ? g.num_tiles : maxc;
   cfg.gridDim = dim3(2 * pairs);
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemm2_kernel<BN>, ta, tb, tc, g);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }

@@ -123,24 +123,33 @@ __device__ __forceinline__ void store_row_chunk_tma(const GemmArgs& g, const CUt
       const int n = n0 + 8 * v;
       uint32_t w[4] = {0, 0, 0, 0};
       if (n < g.N) {
-        const float4 c0 = __ldg(reinterpret_cast<const float4*>(g.s_col + n));
-        const float4 c1 = __ldg(reinterpret_cast<const float4*>(g.s_col + n + 4));
-        const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        float f[8];
+        // ((float)acc * s_row) * s_col (+ bias), as pairs: each lane of a
+        // pair rounds like the scalar mul / add (RN), so the bits are those
+        // of the scalar left-to-right evaluation.
+        const ulonglong2 c0 = __ldg(reinterpret_cast<const ulonglong2*>(g.s_col + n));
+        const ulonglong2 c1 = __ldg(reinterpret_cast<const ulonglong2*>(g.s_col + n + 4));
+        const uint64_t sc2[4] = {c0.x, c0.y, c1.x, c1.y};
+        const uint64_t srow2 = pack_f2(srow, srow);
+        uint64_t f2[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          f[j] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[8 * v + j])), srow), sc[j]);
+        for (int j = 0; j < 4; ++j) {
+          const uint64_t a = pack_f2(__int2float_rn(static_cast<int>(r[8 * v + 2 * j])),
+                                     __int2float_rn(static_cast<int>(r[8 * v + 2 * j + 1])));
+          f2[j] = mul_f2(mul_f2(a, srow2), sc2[j]);
+        }
         if (g.bias) {
           const uint4 b = __ldg(reinterpret_cast<const uint4*>(g.bias + n));
           const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            f[2 * j] = __fadd_rn(f[2 * j], __uint_as_float(bw[j] << 16));
-            f[2 * j + 1] = __fadd_rn(f[2 * j + 1], __uint_as_float(bw[j] & 0xffff0000u));
-          }
+          for (int j = 0; j < 4; ++j)
+            f2[j] = add_f2(f2[j], pack_f2(__uint_as_float(bw[j] << 16), __uint_as_float(bw[j] & 0xffff0000u)));
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) w[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
+        for (int j = 0; j < 4; ++j) {
+          float lo, hi;
+          unpack_f2(f2[j], lo, hi);
+          w[j] = pack_bf16x2(lo, hi);
+        }
       }
       const uint32_t off = static_cast<uint32_t>(lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4));
       asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(w[0]), "r"(w[1]),

@@ -66,25 +66,6 @@ __device__ __forceinline__ int8_t quant_one(float v, float s) {
 constexpr float kMagic = 12582912.0f;            // 1.5 * 2^23
 constexpr float kNear = 0.49993896484375f;       // 1/2 - 2^-14
 
-__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void unpack_f2(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t fma_f2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t sub_f2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
 // Two codes (low bytes of the two t's) for the pair v; tracks max |e|.
 __device__ __forceinline__ void quant_pair(uint64_t v, uint64_t inv2, uint64_t magic2, float& emax,
                                            uint32_t& t0, uint32_t& t1) {
@@ -124,6 +105,7 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict
                                                              float* __restrict__ scales,
                                                              int tpr_log2) {
   constexpr int E = Elem<T>::kPerVec;
+  griddep_launch_dependents();     // the next kernel (e.g. the GEMM) may start its prologue
   const int tpr = 1 << tpr_log2;
   const int t = threadIdx.x & (tpr - 1);
   const int r_local = threadIdx.x >> tpr_log2;
@@ -288,6 +270,7 @@ __global__ void __launch_bounds__(QT_THREADS, 1)
                           int64_t ldq, float* __restrict__ scales, int stages, int stage_bytes, int wpr,
                           WaitCtl wait) {
   constexpr int E = Elem<T>::kPerVec;             // elements per 16-byte chunk
+  griddep_launch_dependents();     // the next kernel (e.g. the GEMM) may start its prologue
   extern __shared__ __align__(128) uint8_t qsmem[];
   __shared__ __align__(8) uint64_t full_bar[QT_RING_BYTES / 1024];
   __shared__ __align__(8) uint64_t empty_bar[QT_RING_BYTES / 1024];
