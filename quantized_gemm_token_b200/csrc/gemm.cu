@@ -77,6 +77,15 @@ struct Cfg {
   static_assert(STAGES >= 2, "stages");
 };
 
+// The stream-K finishing store, kept out of line so that this rarely taken
+// path does not add to the register pressure of the whole-tile epilogue.
+__device__ __noinline__ void store_row_chunk_tma_cold(const GemmArgs& g, const CUtensorMap* tm_c, uint8_t* buf,
+                                                      int lane, int m0, int n0, const uint32_t* r, float srow) {
+  ColScales cs;
+  if (!g.out_s32) load_col_scales(g, n0, cs);
+  store_row_chunk_tma(g, tm_c, buf, lane, m0, n0, r, srow, cs);
+}
+
 template <Kind KIND, int BN>
 __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -298,6 +307,9 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
           const int m = ta * 128 + row;
           if (!g.out_s32 && m < g.M) srow = __ldg(g.s_row + m);
         }
+        // Chunk by chunk: the TMEM load and the chunk's column-scale loads are
+        // in flight together; after reading its last chunk the warp hands
+        // the accumulator back to the MMA warp, then dequantizes and stores.
 #pragma unroll 1
         for (int c = grp; c < NCH; c += GROUPS) {
           uint32_t r[CW];
@@ -311,17 +323,22 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
           if (empty_slice) {
 #pragma unroll
             for (int j = 0; j < CW; ++j) r[j] = 0;
+          } else if constexpr (CW == 32) {
+            tmem_ld_32x32b_x32(tbase + c * CW, r);
           } else {
-            if constexpr (CW == 32) tmem_ld_32x32b_x32(tbase + c * CW, r);
-            else tmem_ld_32x32b_x16(tbase + c * CW, r);
-            tmem_ld_wait();
+            tmem_ld_32x32b_x16(tbase + c * CW, r);
           }
+          ColScales cs;
+          if constexpr (KIND != Kind::Swap) {
+            if (!g.out_s32) load_col_scales(g, tb * BN + c * CW, cs);
+          }
+          tmem_ld_wait();
           if (c == last_c) {
             tc_fence_before();
             mbar_arrive(smem_u32(acce_bar + acc));
           }
           if constexpr (KIND == Kind::Swap) store_col_chunk<CW>(g, ta * 128 + row, tb * BN + c * CW, r);
-          else store_row_chunk_tma(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, tb * BN + c * CW, r, srow);
+          else store_row_chunk_tma(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, tb * BN + c * CW, r, srow, cs);
         }
       } else {
         // Stream-K partial tile: add into the workspace (coalesced: one
@@ -365,7 +382,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
               __stcg(p, 0);
             }
             if constexpr (KIND == Kind::Swap) store_col_chunk<CW>(g, ta * 128 + row, tb * BN + c * CW, r);
-            else store_row_chunk_tma(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, tb * BN + c * CW, r, srow);
+            else store_row_chunk_tma_cold(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, tb * BN + c * CW, r, srow);
           }
           if (ep_tid == 0) g.ws_cnt[s.tile] = 0;
         }
@@ -443,9 +460,10 @@ dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap
 
 constexpr int64_t kMaxK = 133144;   // floor((2^31 - 1) / 127^2): int32 accumulation is exact
 
-// Measured on B200: the pair kernel only pays off when K is very large; for
-// K up to 8192 the 1-SM kernel is as fast or faster.
-constexpr int64_t kPairMinK = 16384;
+// Measured on B200: the pair kernel (half the operand bytes per MMA) pays off
+// from K = 8192 up (8192^3: +13 %; M=2048 N=4096 K=8192: equal); for smaller K
+// its longer prologue loses to the 1-SM kernel.
+constexpr int64_t kPairMinK = 8192;
 
 // Schedule override for measurements: 0 = automatic, 1 = 1-SM whole tiles,
 // 2 = 1-SM stream-K, 3 = pair (2-SM) kernel for every M.

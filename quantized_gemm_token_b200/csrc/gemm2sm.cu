@@ -229,17 +229,35 @@ __global__ void __launch_bounds__(Cfg2<BN>::THREADS, 1)
       const int m_slab = ta * 256 + static_cast<int>(rank) * 128 + sp * 32;
       const int m = m_slab + lane;
       const float srow = (!g.out_s32 && m < g.M) ? __ldg(g.s_row + m) : 0.0f;
+      // Chunks are read from TMEM two at a time (one wait per pair, the
+      // column scales fetched meanwhile); after the pair holding its last
+      // chunk the warp hands the accumulator back to the leader, then
+      // dequantizes and stores from registers.
+      constexpr int PER_WARP = (C::NCH + GROUPS - 1) / GROUPS;
+      constexpr int BATCH = PER_WARP < 2 ? PER_WARP : 2;
 #pragma unroll 1
-      for (int c = grp; c < C::NCH; c += GROUPS) {
-        uint32_t r[C::CW];
-        tmem_ld_32x32b_x32(tbase + c * C::CW, r);
+      for (int c0 = grp; c0 < C::NCH; c0 += BATCH * GROUPS) {
+        uint32_t r[BATCH][C::CW];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const int c = c0 + i * GROUPS;
+          if (c < C::NCH) tmem_ld_32x32b_x32(tbase + c * C::CW, r[i]);
+        }
+        ColScales cs;
+        if (!g.out_s32) load_col_scales(g, tb * BN + c0 * C::CW, cs);
         tmem_ld_wait();
-        if (c == last_c) {
+        if (c0 + (BATCH - 1) * GROUPS >= last_c) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(acce_bar + acc), 0));
         }
-        store_row_chunk_tma(g, &tm_c, next_buf(), lane, m_slab, tb * BN + c * C::CW, r, srow);
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const int c = c0 + i * GROUPS;
+          if (c >= C::NCH) break;
+          if (i > 0 && !g.out_s32) load_col_scales(g, tb * BN + c * C::CW, cs);
+          store_row_chunk_tma(g, &tm_c, next_buf(), lane, m_slab, tb * BN + c * C::CW, r[i], srow, cs);
+        }
       }
       if (++acc == C::ACC_BUFS) {
         acc = 0;

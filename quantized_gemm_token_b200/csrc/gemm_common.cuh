@@ -99,17 +99,43 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Column scales of one 32-column chunk as f32x2 pairs (s_col[n0 + 2i],
+// s_col[n0 + 2i + 1]); zero past N (N % 8 == 0, so 8-column groups are wholly
+// inside or outside).  All eight loads are issued before any is used.
+struct ColScales {
+  uint64_t sc[16];
+};
+__device__ __forceinline__ void load_col_scales(const GemmArgs& g, int n0, ColScales& p) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int n = n0 + 8 * v;
+    ulonglong2 c0 = make_ulonglong2(0ull, 0ull), c1 = c0;
+    if (n < g.N) {
+      c0 = __ldg(reinterpret_cast<const ulonglong2*>(g.s_col + n));
+      c1 = __ldg(reinterpret_cast<const ulonglong2*>(g.s_col + n + 4));
+    }
+    p.sc[4 * v] = c0.x;
+    p.sc[4 * v + 1] = c0.y;
+    p.sc[4 * v + 2] = c1.x;
+    p.sc[4 * v + 3] = c1.y;
+  }
+}
+
 // Epilogue for one chunk of 32 columns of the Dense/Bsr layout: thread = row
 // `row` (0..31 inside its warp's 32-row slab), output columns n0 .. n0+31.
 // The 32x32 block is written into the warp's staging buffer with the tensor
 // map's swizzle (64 B rows for bf16, 128 B rows for int32) and stored by one
-// TMA bulk store, which also clips rows >= M and columns >= N.  Scales and
-// bias are only read for columns < N (N % 8 == 0).
-__device__ __forceinline__ void store_row_chunk_tma(const GemmArgs& g, const CUtensorMap* tm_c,
-                                                    uint8_t* buf, int lane, int m0, int n0,
-                                                    const uint32_t* r, float srow) {
+// TMA bulk store, which also clips rows >= M and columns >= N.  `cs` holds the
+// chunk's column scales (load_col_scales); with BIAS, g.bias is read for
+// columns < N.  The output mode and the bias are template switches rather
+// than run-time tests, so the code of the modes not taken is not executed
+// predicated-off in every chunk.
+template <bool S32, bool BIAS>
+__device__ __forceinline__ void store_row_chunk_tma_t(const GemmArgs& g, const CUtensorMap* tm_c,
+                                                      uint8_t* buf, int lane, int m0, int n0,
+                                                      const uint32_t* r, float srow, const ColScales& cs) {
   const uint32_t base = smem_u32(buf);
-  if (g.out_s32) {
+  if constexpr (S32) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const uint32_t off = static_cast<uint32_t>(lane * 128 + ((j ^ (lane & 7)) << 4));
@@ -118,42 +144,43 @@ __device__ __forceinline__ void store_row_chunk_tma(const GemmArgs& g, const CUt
                    : "memory");
     }
   } else {
+    // ((float)acc * s_row) * s_col (+ bias), as pairs: each lane of a pair
+    // rounds like the scalar mul / add (RN), so the bits are those of the
+    // scalar left-to-right evaluation.  All 16 output words are formed before
+    // the shared-memory stores.
+    const uint64_t srow2 = pack_f2(srow, srow);
+    uint64_t f2[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint64_t a = pack_f2(__int2float_rn(static_cast<int>(r[2 * j])),
+                                 __int2float_rn(static_cast<int>(r[2 * j + 1])));
+      f2[j] = mul_f2(mul_f2(a, srow2), cs.sc[j]);
+    }
+    if constexpr (BIAS) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int n = n0 + 8 * v;
+        uint4 b = make_uint4(0u, 0u, 0u, 0u);
+        if (n < g.N) b = __ldg(reinterpret_cast<const uint4*>(g.bias + n));
+        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          f2[4 * v + j] =
+              add_f2(f2[4 * v + j], pack_f2(__uint_as_float(bw[j] << 16), __uint_as_float(bw[j] & 0xffff0000u)));
+      }
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      float lo, hi;
+      unpack_f2(f2[j], lo, hi);
+      w[j] = pack_bf16x2(lo, hi);
+    }
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
-      const int n = n0 + 8 * v;
-      uint32_t w[4] = {0, 0, 0, 0};
-      if (n < g.N) {
-        // ((float)acc * s_row) * s_col (+ bias), as pairs: each lane of a
-        // pair rounds like the scalar mul / add (RN), so the bits are those
-        // of the scalar left-to-right evaluation.
-        const ulonglong2 c0 = __ldg(reinterpret_cast<const ulonglong2*>(g.s_col + n));
-        const ulonglong2 c1 = __ldg(reinterpret_cast<const ulonglong2*>(g.s_col + n + 4));
-        const uint64_t sc2[4] = {c0.x, c0.y, c1.x, c1.y};
-        const uint64_t srow2 = pack_f2(srow, srow);
-        uint64_t f2[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint64_t a = pack_f2(__int2float_rn(static_cast<int>(r[8 * v + 2 * j])),
-                                     __int2float_rn(static_cast<int>(r[8 * v + 2 * j + 1])));
-          f2[j] = mul_f2(mul_f2(a, srow2), sc2[j]);
-        }
-        if (g.bias) {
-          const uint4 b = __ldg(reinterpret_cast<const uint4*>(g.bias + n));
-          const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            f2[j] = add_f2(f2[j], pack_f2(__uint_as_float(bw[j] << 16), __uint_as_float(bw[j] & 0xffff0000u)));
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float lo, hi;
-          unpack_f2(f2[j], lo, hi);
-          w[j] = pack_bf16x2(lo, hi);
-        }
-      }
       const uint32_t off = static_cast<uint32_t>(lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4));
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(w[0]), "r"(w[1]),
-                   "r"(w[2]), "r"(w[3])
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(w[4 * v]),
+                   "r"(w[4 * v + 1]), "r"(w[4 * v + 2]), "r"(w[4 * v + 3])
                    : "memory");
     }
   }
@@ -163,6 +190,14 @@ __device__ __forceinline__ void store_row_chunk_tma(const GemmArgs& g, const CUt
     tma_store_2d(tm_c, base, n0, m0);
     bulk_commit_group();
   }
+}
+
+__device__ __forceinline__ void store_row_chunk_tma(const GemmArgs& g, const CUtensorMap* tm_c, uint8_t* buf,
+                                                    int lane, int m0, int n0, const uint32_t* r, float srow,
+                                                    const ColScales& cs) {
+  if (g.out_s32) store_row_chunk_tma_t<true, false>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
+  else if (g.bias != nullptr) store_row_chunk_tma_t<false, true>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
+  else store_row_chunk_tma_t<false, false>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
 }
 
 // Epilogue for the Swap layout: thread = output channel n, columns are

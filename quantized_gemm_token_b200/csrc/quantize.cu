@@ -41,7 +41,8 @@ __device__ __forceinline__ int8_t quant_one(float v, float s) {
   return static_cast<int8_t>(r);
 }
 
-// Codes without a division, the same result as quant_one.
+// fp32 inputs (the weight path): codes without a division, the same result as
+// quant_one, with a flagged fallback to the IEEE division.
 //
 // Let inv = fp32(1 / s) and p = v * inv taken exactly (inside an FMA).  inv's
 // rounding gives |p - v/s| <= |v/s| 2^-24 < 2^-17, because |v / s| <=
@@ -60,28 +61,65 @@ __device__ __forceinline__ int8_t quant_one(float v, float s) {
 // is exact.  e = fma(v, inv, -r) is p - r (the distance to the nearest
 // integer) with one rounding (error <= 2^-25); p is treated as near a
 // half-integer when |e| >= 1/2 - 2^-14, a margin that covers that rounding.
+// That test runs as d = fma(e, e, -c) with c = 1/4 - 2^-14 (exact in fp32,
+// just below (1/2 - 2^-14)^2): d >= 0 (sign bit clear) whenever |e| >=
+// 1/2 - 2^-14, so AND-ing the sign bits of a vector's d values flags it.
 //
 // The fp32 work runs as packed pairs (sm_100 f32x2 fma/sub, each lane of the
 // pair rounded like the scalar instruction).
 constexpr float kMagic = 12582912.0f;            // 1.5 * 2^23
-constexpr float kNear = 0.49993896484375f;       // 1/2 - 2^-14
+constexpr float kNearSq = 0.24993896484375f;     // 1/4 - 2^-14
 
-// Two codes (low bytes of the two t's) for the pair v; tracks max |e|.
-__device__ __forceinline__ void quant_pair(uint64_t v, uint64_t inv2, uint64_t magic2, float& emax,
-                                           uint32_t& t0, uint32_t& t1) {
+// Two codes (low bytes of the two t's) for the pair v; `tie` keeps the AND of
+// the d sign bits (bit 31 clear once any code is near a tie), d0 / d1 the
+// two d values' bits.
+__device__ __forceinline__ void quant_pair(uint64_t v, uint64_t inv2, uint64_t magic2, uint64_t negc2,
+                                           uint32_t& tie, uint32_t& t0, uint32_t& t1, uint32_t& d0,
+                                           uint32_t& d1) {
   const uint64_t t = fma_f2(v, inv2, magic2);
   const uint64_t neg_r = sub_f2(magic2, t);          // -rint(p), exact
   const uint64_t e = fma_f2(v, inv2, neg_r);
-  float e0, e1, f0, f1;
-  unpack_f2(e, e0, e1);
-  emax = fmaxf(emax, fmaxf(fabsf(e0), fabsf(e1)));
-  unpack_f2(t, f0, f1);
-  t0 = __float_as_uint(f0);
-  t1 = __float_as_uint(f1);
+  const uint64_t d = fma_f2(e, e, negc2);
+  d0 = static_cast<uint32_t>(d);
+  d1 = static_cast<uint32_t>(d >> 32);
+  tie &= d0 & d1;
+  t0 = static_cast<uint32_t>(t);
+  t1 = static_cast<uint32_t>(t >> 32);
 }
 
 __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
   return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
+// bf16 inputs: the correctly rounded quotient without a division, by
+// Markstein's correction step (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990): q0 = fp32(v * inv), r = fma(-q0, s, v) (exact), q1 = fma(r, inv, q0)
+// = fp32(v / s); then rint(q1) by the 1.5 * 2^23 addition (ties to even, as
+// q1 is the exact fp32 quotient).  For every positive bf16 absmax and every
+// bf16 value v with |v| <= absmax, rint(q1) equals rint(fp32(v / s)) (checked
+// exhaustively against IEEE division; q1 itself differs only for quotients
+// below 1/4, where r underflows, and those round to 0 either way).
+__device__ __forceinline__ void quant_pair_bf16(uint64_t v, uint64_t inv2, uint64_t negs2, uint64_t magic2,
+                                                uint32_t& t0, uint32_t& t1) {
+  const uint64_t q0 = mul_f2(v, inv2);
+  const uint64_t r = fma_f2(q0, negs2, v);
+  const uint64_t q1 = fma_f2(r, inv2, q0);
+  const uint64_t t = add_f2(q1, magic2);
+  t0 = static_cast<uint32_t>(t);
+  t1 = static_cast<uint32_t>(t >> 32);
+}
+
+// Codes of one 16-byte vector of 8 bf16 values (w = 4 packed words) as two
+// words of int8 codes.
+__device__ __forceinline__ uint2 quant_bf16x8(const uint32_t (&w)[4], uint64_t inv2, uint64_t negs2,
+                                              uint64_t magic2) {
+  uint32_t b[8];
+#pragma unroll
+  for (int h = 0; h < 4; ++h)
+    quant_pair_bf16(pack_f2(__uint_as_float(w[h] << 16), __uint_as_float(w[h] & 0xffff0000u)), inv2, negs2,
+                    magic2, b[2 * h], b[2 * h + 1]);
+  return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
 __device__ __forceinline__ float scale_from_absmax(float a) {
@@ -93,6 +131,15 @@ __device__ __forceinline__ uint32_t pack4(int8_t a, int8_t b, int8_t c, int8_t d
          (static_cast<uint32_t>(static_cast<uint8_t>(b)) << 8) |
          (static_cast<uint32_t>(static_cast<uint8_t>(c)) << 16) |
          (static_cast<uint32_t>(static_cast<uint8_t>(d)) << 24);
+}
+
+// Exact codes (IEEE division) of one 16-byte vector of 4 fp32 values.  Out
+// of line on purpose: it runs only for a vector holding a code near a tie
+// (fp32 inputs rarely have one), and as a call the compiler cannot if-convert
+// its divisions into the common path.
+__device__ __noinline__ uint32_t quant_f32x4_exact(uint4 v, float s) {
+  return pack4(quant_one(__uint_as_float(v.x), s), quant_one(__uint_as_float(v.y), s),
+               quant_one(__uint_as_float(v.z), s), quant_one(__uint_as_float(v.w), s));
 }
 
 // Register-resident single-pass kernel.  256 threads; a row is owned by
@@ -166,40 +213,24 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict
   const float inv1 = inv;
   const uint64_t inv2 = pack_f2(inv1, inv1);
   const uint64_t magic2 = pack_f2(kMagic, kMagic);
+  const uint64_t negc2 = pack_f2(-kNearSq, -kNearSq);
+  const uint64_t negs2 = pack_f2(-s, -s);
   int8_t* qr = q + row * ldq;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int vi = t + i * tpr;
     if (vi < nv) {
       const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      float emax = 0.0f;
       if constexpr (E == 8) {
-        uint32_t b[8];
-#pragma unroll
-        for (int h = 0; h < 4; ++h)
-          quant_pair(pack_f2(__uint_as_float(w[h] << 16), __uint_as_float(w[h] & 0xffff0000u)), inv2, magic2,
-                     emax, b[2 * h], b[2 * h + 1]);
-        uint32_t out0 = pack_low_bytes(b[0], b[1], b[2], b[3]);
-        uint32_t out1 = pack_low_bytes(b[4], b[5], b[6], b[7]);
-        if (emax >= kNear) {   // rare: a code within 2^-14 of a tie, decide by IEEE division
-          float f[8];
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            f[2 * h] = __uint_as_float(w[h] << 16);
-            f[2 * h + 1] = __uint_as_float(w[h] & 0xffff0000u);
-          }
-          out0 = pack4(quant_one(f[0], s), quant_one(f[1], s), quant_one(f[2], s), quant_one(f[3], s));
-          out1 = pack4(quant_one(f[4], s), quant_one(f[5], s), quant_one(f[6], s), quant_one(f[7], s));
-        }
-        *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(vi) * 8) = make_uint2(out0, out1);
+        *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(vi) * 8) = quant_bf16x8(w, inv2, negs2, magic2);
       } else {
-        uint32_t b[4];
-        quant_pair(pack_f2(__uint_as_float(w[0]), __uint_as_float(w[1])), inv2, magic2, emax, b[0], b[1]);
-        quant_pair(pack_f2(__uint_as_float(w[2]), __uint_as_float(w[3])), inv2, magic2, emax, b[2], b[3]);
+        uint32_t tie = 0xffffffffu, b[4], dd[4];
+        quant_pair(pack_f2(__uint_as_float(w[0]), __uint_as_float(w[1])), inv2, magic2, negc2, tie, b[0], b[1],
+                   dd[0], dd[1]);
+        quant_pair(pack_f2(__uint_as_float(w[2]), __uint_as_float(w[3])), inv2, magic2, negc2, tie, b[2], b[3],
+                   dd[2], dd[3]);
         uint32_t out = pack_low_bytes(b[0], b[1], b[2], b[3]);
-        if (emax >= kNear)
-          out = pack4(quant_one(__uint_as_float(w[0]), s), quant_one(__uint_as_float(w[1]), s),
-                      quant_one(__uint_as_float(w[2]), s), quant_one(__uint_as_float(w[3]), s));
+        if (!(tie >> 31)) out = quant_f32x4_exact(v[i], s);
         *reinterpret_cast<uint32_t*>(qr + static_cast<int64_t>(vi) * 4) = out;
       }
     }
@@ -314,15 +345,14 @@ __global__ void __launch_bounds__(QT_THREADS, 1)
       }
     }
   } else {
-    // A consumer must never get more than one ring lap ahead of the rows it
-    // waits for (try_wait.parity cannot tell phase k from phase k-2), so only
-    // min(QT_CONSUMERS, stages) warps take rows, each stepping by that count.
-    // Rows go to groups of `wpr` warps (wpr = 1, 2 or 4; QT_CONSUMERS/wpr
-    // groups, at most `stages` of them, see above); the warps of a group split
-    // the row's 16-byte chunks and combine their partial maxima through
-    // shared memory under the group's named barrier.
-    const int groups_all = QT_CONSUMERS / wpr;
-    const int groups = groups_all < stages ? groups_all : stages;
+    // Rows go round-robin to the QT_CONSUMERS / wpr groups of `wpr` warps
+    // (wpr = 1, 2 or 4); the warps of a group split the row's 16-byte chunks
+    // and combine their partial maxima through shared memory under the
+    // group's named barrier.  `stages` is a multiple of the group count (the
+    // launch checks it), so all rows of one stage belong to one group: the
+    // group has consumed the stage's previous lap before it waits for the
+    // next (try_wait.parity cannot tell lap L from lap L - 2).
+    const int groups = QT_CONSUMERS / wpr;
     const int cw = warp - 1;
     const int grp = cw / wpr, wig = cw % wpr;
     const int bar_id = 1 + grp;                  // named barriers 1..groups
@@ -378,40 +408,24 @@ __global__ void __launch_bounds__(QT_THREADS, 1)
       if (lane == 0 && wig == 0) scales[row] = s;
       const uint64_t inv2 = pack_f2(inv, inv);
       const uint64_t magic2 = pack_f2(kMagic, kMagic);
+      const uint64_t negc2 = pack_f2(-kNearSq, -kNearSq);
       int8_t* qr = q + row * ldq;
+      const uint64_t negs2 = pack_f2(-s, -s);
       // pass 2: codes
 #pragma unroll 2
       for (int c = lane + 32 * wig; c < nchunks; c += cstep) {
         const uint4 v = src[c];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        float emax = 0.0f;
         if constexpr (E == 8) {
-          uint32_t b[8];
-#pragma unroll
-          for (int h = 0; h < 4; ++h)
-            quant_pair(pack_f2(__uint_as_float(w[h] << 16), __uint_as_float(w[h] & 0xffff0000u)), inv2, magic2,
-                       emax, b[2 * h], b[2 * h + 1]);
-          uint32_t out0 = pack_low_bytes(b[0], b[1], b[2], b[3]);
-          uint32_t out1 = pack_low_bytes(b[4], b[5], b[6], b[7]);
-          if (emax >= kNear) {
-            float f[8];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              f[2 * h] = __uint_as_float(w[h] << 16);
-              f[2 * h + 1] = __uint_as_float(w[h] & 0xffff0000u);
-            }
-            out0 = pack4(quant_one(f[0], s), quant_one(f[1], s), quant_one(f[2], s), quant_one(f[3], s));
-            out1 = pack4(quant_one(f[4], s), quant_one(f[5], s), quant_one(f[6], s), quant_one(f[7], s));
-          }
-          *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(c) * 8) = make_uint2(out0, out1);
+          *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(c) * 8) = quant_bf16x8(w, inv2, negs2, magic2);
         } else {
-          uint32_t b[4];
-          quant_pair(pack_f2(__uint_as_float(w[0]), __uint_as_float(w[1])), inv2, magic2, emax, b[0], b[1]);
-          quant_pair(pack_f2(__uint_as_float(w[2]), __uint_as_float(w[3])), inv2, magic2, emax, b[2], b[3]);
+          uint32_t tie = 0xffffffffu, b[4], dd[4];
+          quant_pair(pack_f2(__uint_as_float(w[0]), __uint_as_float(w[1])), inv2, magic2, negc2, tie, b[0], b[1],
+                     dd[0], dd[1]);
+          quant_pair(pack_f2(__uint_as_float(w[2]), __uint_as_float(w[3])), inv2, magic2, negc2, tie, b[2], b[3],
+                     dd[2], dd[3]);
           uint32_t out = pack_low_bytes(b[0], b[1], b[2], b[3]);
-          if (emax >= kNear)
-            out = pack4(quant_one(__uint_as_float(w[0]), s), quant_one(__uint_as_float(w[1]), s),
-                        quant_one(__uint_as_float(w[2]), s), quant_one(__uint_as_float(w[3]), s));
+          if (!(tie >> 31)) out = quant_f32x4_exact(v, s);
           *reinterpret_cast<uint32_t*>(qr + static_cast<int64_t>(c) * 4) = out;
         }
       }
@@ -448,10 +462,27 @@ dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t*
   const bool tma_ok = vec_ok && row_bytes >= 1024 && row_bytes <= QT_MAX_ROW_BYTES;
   const bool tma_pick = g_quant_kernel_override == 2 || (g_quant_kernel_override == 0 && row_bytes >= 9 * 1024);
   if (tma_ok && tma_pick) {
-    // stage = one row rounded up to 128 bytes; as many stages as the ring holds (<= 192)
+    // stage = one row rounded up to 128 bytes; at most as many stages as the
+    // ring holds (<= 192).
     const int stage_bytes = static_cast<int>((row_bytes + 127) / 128 * 128);
-    int stages = QT_RING_BYTES / stage_bytes;
-    if (stages > QT_RING_BYTES / 1024) stages = QT_RING_BYTES / 1024;
+    int max_stages = QT_RING_BYTES / stage_bytes;
+    if (max_stages > QT_RING_BYTES / 1024) max_stages = QT_RING_BYTES / 1024;
+    // Rows go round-robin to QT_CONSUMERS / wpr groups of wpr warps.  The
+    // stage count is a multiple of the group count, so a stage's rows (j,
+    // j + stages, ...) all belong to one group, which therefore has consumed
+    // the stage's previous lap before it waits for the next one: the parity
+    // wait can never see lap L - 2 as lap L.  wpr grows until at least 4
+    // stages stay loading beyond the rows being worked on (measured: 16 KB
+    // rows best with 4 warps per row).
+    int wpr = 1;
+    while (wpr < 4) {
+      const int grp = QT_CONSUMERS / wpr;
+      if ((max_stages / grp) * grp - grp >= 4) break;
+      wpr *= 2;
+    }
+    const int groups = QT_CONSUMERS / wpr;
+    const int stages = (max_stages / groups) * groups;
+    if (stages < groups) return DQ_ERR_UNSUPPORTED;    // not reachable for rows <= 16 KB
     const int smem = stages * stage_bytes;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -461,10 +492,6 @@ dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t*
     });
     if (attr_err != cudaSuccess) return cuda_fail(attr_err);
     const int64_t grid = M < d->sm_count ? M : d->sm_count;
-    // warps per row: leave at least 4 ring stages loading beyond the rows
-    // being worked on (measured best: 16 KB rows 4 warps, 10 KB rows 2)
-    int wpr = 1;
-    while (wpr < 4 && QT_CONSUMERS / wpr > stages - 4) wpr *= 2;
     WaitCtl wait{d->err_word, wait_timeout_ns()};
     quant_rows_tma_kernel<T><<<static_cast<unsigned>(grid), QT_THREADS, smem, stream>>>(
         x, M, static_cast<int>(K), ldx, q, ldq, scales, stages, stage_bytes, wpr, wait);

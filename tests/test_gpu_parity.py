@@ -61,6 +61,25 @@ def test_quantize_full_size_16384x8192():
     assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
 
 
+@pytest.mark.parametrize("kernel", [0, 2])
+@pytest.mark.parametrize("K", [512, 1280, 2560, 4608, 5120, 6144, 8192])
+def test_quantize_many_rows_per_cta(K, kernel):
+    """Every row, bit for bit, with tens of rows per CTA so that the
+    row-pipelined kernel's shared-memory ring wraps many times (1 KB .. 16 KB
+    rows; kernel 2 forces the pipelined kernel, 0 is the automatic choice)."""
+    M = 6000
+    x = synth.normal_bf16((M, K), 1.0, 300 + K)
+    dq.dq_debug_set_quant_kernel(kernel)
+    try:
+        q, s = dq.dq_quantize_rows(to_dev_bf16(x))
+        torch.cuda.synchronize()
+    finally:
+        dq.dq_debug_set_quant_kernel(0)
+    qo, so = oracle.quantize_rows_bf16(x)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
 @pytest.mark.parametrize("N,K", [(256, 256), (5120, 1280), (64, 100), (33, 4096)])
 def test_quantize_weight_parity(N, K):
     w = synth.normal_f32((N, K), 0.02, 200 + K)
@@ -261,9 +280,12 @@ def test_config_vit_h_bsr(layer):
     q, s = dq.dq_quantize_rows(to_dev_bf16(d["x"]))
     out = dq.dq_bsr_int8_linear(q, s, N, crow, col, values, sc)
     acc = dq.dq_bsr_int8_linear(q, s, N, crow, col, values, sc, out_dtype="s32")
+    # the whole activation quantization, every row
+    qo_all, so_all = oracle.quantize_rows_bf16(d["x"])
+    assert np.array_equal(q.cpu().numpy(), qo_all)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so_all.view(np.uint32))
     rows = sample_rows(M, 48)
-    qo, so = oracle.quantize_rows_bf16(d["x"][rows])
-    assert np.array_equal(q.cpu().numpy()[rows], qo)
+    qo, so = qo_all[rows], so_all[rows]
     acc_o = oracle.bsr_gemm_s32(qo, N, d["crow"], d["col"], vo)
     assert np.array_equal(acc.cpu().numpy()[rows], acc_o)
     got = bf16_bits(out)
