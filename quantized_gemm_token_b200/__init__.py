@@ -42,6 +42,7 @@ _PROTOS = {
     "dq_mma_peak_probe": (_I32, [_I32, _I32, _P]),
     "dq_debug_set_schedule": (None, [_I32]),
     "dq_debug_set_tile_n": (None, [_I32]),
+    "dq_debug_set_two_widths": (None, [_I32]),
     "dq_debug_set_quant_kernel": (None, [_I32]),
 }
 
@@ -148,6 +149,11 @@ def dq_debug_set_schedule(mode: int) -> None:
 
 def dq_debug_set_tile_n(n: int) -> None:
     lib.dq_debug_set_tile_n(int(n))
+
+
+def dq_debug_set_two_widths(on: int) -> None:
+    """Measurement knob: 0 turns off the two-width (wave-balanced) dense schedule."""
+    lib.dq_debug_set_two_widths(int(on))
 
 
 def dq_debug_set_quant_kernel(mode: int) -> None:

@@ -77,6 +77,38 @@ struct Cfg {
   static_assert(STAGES >= 2, "stages");
 };
 
+// Where a tile lies: 128-row block ta, B-slot tile tb, first output column n0
+// and the MMA width (BN, or bn2 for a Dense tile of the narrow second set).
+struct TileGeom {
+  int ta, tb, n0, width;
+  bool narrow;
+};
+template <Kind KIND, int BN>
+__device__ __forceinline__ TileGeom tile_geom(const GemmArgs& g, int tile) {
+  TileGeom t;
+  if (KIND == Kind::Dense && g.bn2 > 0 && tile >= g.t1) {
+    int j = tile - g.t1;
+    if (j < g.first_cnt) {
+      t.ta = g.mb0;
+      t.n0 = g.c_start + j * g.bn2;
+    } else {
+      j -= g.first_cnt;
+      t.ta = g.mb0 + 1 + j / g.per_row;
+      t.n0 = (j % g.per_row) * g.bn2;
+    }
+    t.tb = 0;
+    t.width = g.bn2;
+    t.narrow = true;
+  } else {
+    t.ta = tile / g.b_tiles;
+    t.tb = tile % g.b_tiles;
+    t.n0 = t.tb * BN;
+    t.width = BN;
+    t.narrow = false;
+  }
+  return t;
+}
+
 // The stream-K finishing store, kept out of line so that this rarely taken
 // path does not add to the register pressure of the whole-tile epilogue.
 __device__ __noinline__ void store_row_chunk_tma_cold(const GemmArgs& g, const CUtensorMap* tm_c, uint8_t* buf,
@@ -89,7 +121,8 @@ __device__ __noinline__ void store_row_chunk_tma_cold(const GemmArgs& g, const C
 template <Kind KIND, int BN>
 __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ GemmArgs g) {
+                const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_c,
+                const __grid_constant__ GemmArgs g) {
   using C = Cfg<KIND, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -125,6 +158,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    if (KIND == Kind::Dense && g.bn2 > 0) tma_prefetch_desc(&tm_b2);
     if constexpr (C::STAGED_OUT) tma_prefetch_desc(&tm_c);
   }
   if (warp == 1) {
@@ -159,7 +193,9 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       long long issued = 0;
       bool ok = true;
       while (ok && iter.next(s)) {
-        const int ta = s.tile / g.b_tiles, tb = s.tile % g.b_tiles;
+        const TileGeom geo = tile_geom<KIND, BN>(g, s.tile);
+        const int ta = geo.ta, tb = geo.tb;
+        const uint32_t stage_tx = C::A_BYTES + (KIND == Kind::Dense ? geo.width * C::KB : C::B_BYTES);
         for (int j = 0; ok && j < C::NSUB; ++j) {
         int k0 = s.kb0, k1 = s.kb1;
         if constexpr (KIND == Kind::Bsr) {
@@ -173,7 +209,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
             break;
           }
           const uint32_t fb = smem_u32(full_bar + stage);
-          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          mbar_arrive_expect_tx(fb, stage_tx);
           const uint32_t da = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t db = smem_u32(sB + stage * C::B_BYTES);
           if constexpr (KIND == Kind::Bsr) {
@@ -182,7 +218,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
             tma_load_2d(db, &tm_b, fb, 0, kb * 64);
           } else {
             tma_load_2d(da, &tm_a, fb, kb * C::KB, ta * 128);
-            tma_load_2d(db, &tm_b, fb, kb * C::KB, tb * BN);
+            tma_load_2d(db, geo.narrow ? &tm_b2 : &tm_b, fb, kb * C::KB, geo.n0);
           }
           ++issued;
           if (++stage == C::STAGES) {
@@ -210,7 +246,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(128, C::MMA_N);
+      constexpr uint32_t idesc_full = idesc_i8(128, C::MMA_N);
       SegIter iter(g);
       Seg s;
       int stage = 0, acc = 0;
@@ -219,6 +255,8 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       while (ok && iter.next(s)) {
         if (!mbar_wait(smem_u32(acce_bar + acc), acc_phase ^ 1, g.wait, abort_flag)) break;
         tc_fence_after();
+        const uint32_t idesc = (KIND == Kind::Dense && g.bn2 > 0 && s.tile >= g.t1)
+                                   ? idesc_i8(128, g.bn2) : idesc_full;
         for (int j = 0; ok && j < C::NSUB; ++j) {
         int k0 = s.kb0, k1 = s.kb1;
         if constexpr (KIND == Kind::Bsr) {
@@ -293,13 +331,17 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     while (iter.next(s)) {
-      const int ta = s.tile / g.b_tiles, tb = s.tile % g.b_tiles;
+      const TileGeom geo = tile_geom<KIND, BN>(g, s.tile);
+      const int ta = geo.ta, tb = geo.tb, n0 = geo.n0;
       if (!mbar_wait(smem_u32(accf_bar + acc), acc_phase, g.wait, abort_flag)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const bool whole = !g.stream_k || (s.kb0 == 0 && s.kb1 == g.kb_total);
-      // this warp's last chunk; after reading it the warp releases the accumulator
-      const int last_c = grp + ((NCH - 1 - grp) / GROUPS) * GROUPS;
+      // chunks of this tile (a narrow Dense tile has fewer; every warp still
+      // has one, as bn2 >= 64); after reading its last chunk a warp releases
+      // the accumulator
+      const int nch = KIND == Kind::Dense ? geo.width / CW : NCH;
+      const int last_c = grp + ((nch - 1 - grp) / GROUPS) * GROUPS;
 
       if (whole) {
         float srow = 0.0f;
@@ -311,7 +353,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
         // in flight together; after reading its last chunk the warp hands
         // the accumulator back to the MMA warp, then dequantizes and stores.
 #pragma unroll 1
-        for (int c = grp; c < NCH; c += GROUPS) {
+        for (int c = grp; c < nch; c += GROUPS) {
           uint32_t r[CW];
           bool empty_slice = false;     // Bsr: this chunk's block row has no block
           if constexpr (KIND == Kind::Bsr) {
@@ -330,15 +372,15 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
           }
           ColScales cs;
           if constexpr (KIND != Kind::Swap) {
-            if (!g.out_s32) load_col_scales(g, tb * BN + c * CW, cs);
+            if (!g.out_s32) load_col_scales(g, n0 + c * CW, cs);
           }
           tmem_ld_wait();
           if (c == last_c) {
             tc_fence_before();
             mbar_arrive(smem_u32(acce_bar + acc));
           }
-          if constexpr (KIND == Kind::Swap) store_col_chunk<CW>(g, ta * 128 + row, tb * BN + c * CW, r);
-          else store_row_chunk_tma(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, tb * BN + c * CW, r, srow, cs);
+          if constexpr (KIND == Kind::Swap) store_col_chunk<CW>(g, ta * 128 + row, n0 + c * CW, r);
+          else store_row_chunk_tma(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, n0 + c * CW, r, srow, cs);
         }
       } else {
         // Stream-K partial tile: add into the workspace (coalesced: one
@@ -431,8 +473,8 @@ __global__ void __launch_bounds__(256) bsr_pack_kernel(const int8_t* __restrict_
 namespace {
 
 template <Kind KIND, int BN>
-dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
-                 int grid, cudaStream_t stream) {
+dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2, const CUtensorMap& tc,
+                 const GemmArgs& args, int grid, cudaStream_t stream) {
   using C = Cfg<KIND, BN>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -454,7 +496,7 @@ dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN>, ta, tb, tc, args);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN>, ta, tb, tb2, tc, args);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 
@@ -470,6 +512,8 @@ constexpr int64_t kPairMinK = 8192;
 int g_schedule_override = 0;
 // Tile-width override for measurements (0 = automatic).
 int g_tile_n_override = 0;
+// Measurement knob: 0 turns the two-width Dense schedule off.
+int g_two_widths = 1;
 
 struct Plan {
   Kind kind;
@@ -477,7 +521,41 @@ struct Plan {
   int a_tiles, b_tiles, kb_total, num_tiles;
   bool stream_k;
   size_t ws_bytes;   // bytes needed for stream-K (0 if it never splits)
+  // Dense wave balance (bn2 > 0): the first t1 tiles (whole waves) are bn
+  // wide; the rest of the matrix goes in one last wave of bn2-wide tiles.
+  int t1, bn2, mb0, c_start, first_cnt, per_row;
 };
+
+// Whole tiles leave the SMs of a partial last wave idle (e.g. M=2048, N=4096:
+// 256 tiles of 128 x 256 on 148 SMs, 1.73 waves).  Instead the full waves keep
+// bn-wide tiles and the rest of the matrix is cut into at most `sms` tiles of
+// the narrowest width (a multiple of 32, >= 64) that fits in one wave.  Every
+// SM then does (waves - 1) wide tiles and at most one narrow one.
+void plan_two_widths(Plan& p, int64_t N, int sms) {
+  p.bn2 = 0;
+  const int T = p.num_tiles;
+  const int full = T / sms;
+  if (full < 1 || T % sms == 0 || full > 8) return;     // one partial wave, or the tail is small
+  const int t1 = full * sms;
+  const int mb0 = t1 / p.b_tiles;
+  const int c_start = (t1 % p.b_tiles) * p.bn;
+  const int rows_after = p.a_tiles - mb0 - 1;
+  for (int w = 64; w < p.bn; w += 32) {
+    const int first = static_cast<int>((N - c_start + w - 1) / w);
+    const int per_row = static_cast<int>((N + w - 1) / w);
+    const long long t2 = static_cast<long long>(first) + static_cast<long long>(rows_after) * per_row;
+    if (t2 <= sms) {
+      p.t1 = t1;
+      p.bn2 = w;
+      p.mb0 = mb0;
+      p.c_start = c_start;
+      p.first_cnt = first;
+      p.per_row = per_row;
+      p.num_tiles = t1 + static_cast<int>(t2);
+      return;
+    }
+  }
+}
 
 // Stream-K workspace: one int32 partial per tile ([BN][128], column-major so
 // that red.add of one column by a warp is one 512-byte line) plus an arrival
@@ -519,6 +597,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count) {
   const bool worth = p.kind == Kind::Swap && eff < 0.9 && iters >= 4LL * sm_count;
   p.ws_bytes = worth ? sk_workspace_bytes(p, sm_count) : 0;
   p.stream_k = worth;
+  if (p.kind == Kind::Dense && p.bn == 256 && g_tile_n_override == 0 && g_two_widths) plan_two_widths(p, N, sm_count);
   return p;
 }
 
@@ -539,6 +618,7 @@ size_t dq_int8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
 // Measurement knob (not in the public header): force a schedule.
 void dq_debug_set_schedule(int mode) { g_schedule_override = mode; }
 void dq_debug_set_tile_n(int n) { g_tile_n_override = n; }
+void dq_debug_set_two_widths(int on) { g_two_widths = on; }
 
 dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K, const int8_t* W,
                          const float* s_col, int64_t N, const void* bias_bf16, void* out,
@@ -594,17 +674,26 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   bool sk = p.stream_k && workspace != nullptr && workspace_bytes >= p.ws_bytes &&
             aligned(workspace, 16);
   if (g_schedule_override == 1) sk = false;
-  if (g_schedule_override == 2 && workspace != nullptr && aligned(workspace, 16) &&
-      workspace_bytes >= sk_workspace_bytes(p, d->sm_count))
-    sk = static_cast<long long>(p.num_tiles) * p.kb_total >= d->sm_count;
+  if (g_schedule_override == 2) {
+    p.bn2 = 0;                                    // stream-K ranges run over uniform tiles
+    p.num_tiles = p.a_tiles * p.b_tiles;
+    if (workspace != nullptr && aligned(workspace, 16) &&
+        workspace_bytes >= sk_workspace_bytes(p, d->sm_count))
+      sk = static_cast<long long>(p.num_tiles) * p.kb_total >= d->sm_count;
+  }
 
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tb2;
   const int8_t* a_src = p.kind == Kind::Swap ? W : A;
   const int8_t* b_src = p.kind == Kind::Swap ? A : W;
   const int64_t a_rows = p.kind == Kind::Swap ? N : M;
   const int64_t b_rows = p.kind == Kind::Swap ? M : N;
   if ((st = make_tmap_u8_2d(&ta, a_src, K, a_rows, K, 128, 128, 128)) != DQ_OK) return st;
   if ((st = make_tmap_u8_2d(&tb, b_src, K, b_rows, K, 128, p.bn, 128)) != DQ_OK) return st;
+  if (p.bn2 > 0) {
+    if ((st = make_tmap_u8_2d(&tb2, b_src, K, b_rows, K, 128, p.bn2, 128)) != DQ_OK) return st;
+  } else {
+    tb2 = tb;
+  }
   CUtensorMap tc;
   if ((st = make_tmap_out_2d(&tc, out, N, M, out_dtype == DQ_OUT_S32 ? 4 : 2)) != DQ_OK) return st;
   const size_t slots_bytes = static_cast<size_t>(p.num_tiles) * p.bn * 128 * 4;
@@ -619,6 +708,12 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   g.num_tiles = p.num_tiles;
   g.stream_k = sk ? 1 : 0;
   g.iters_total = static_cast<long long>(p.num_tiles) * p.kb_total;
+  g.t1 = p.t1;
+  g.bn2 = p.bn2;
+  g.mb0 = p.mb0;
+  g.c_start = p.c_start;
+  g.first_cnt = p.first_cnt;
+  g.per_row = p.per_row;
   g.s_row = s_row;
   g.s_col = s_col;
   g.bias = static_cast<const uint16_t*>(bias_bf16);
@@ -633,17 +728,17 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
 
   if (p.kind == Kind::Dense) {
     switch (p.bn) {
-      case 256: return launch<Kind::Dense, 256>(ta, tb, tc, g, grid, stream);
-      case 192: return launch<Kind::Dense, 192>(ta, tb, tc, g, grid, stream);
-      case 160: return launch<Kind::Dense, 160>(ta, tb, tc, g, grid, stream);
-      default: return launch<Kind::Dense, 128>(ta, tb, tc, g, grid, stream);
+      case 256: return launch<Kind::Dense, 256>(ta, tb, tb2, tc, g, grid, stream);
+      case 192: return launch<Kind::Dense, 192>(ta, tb, tb2, tc, g, grid, stream);
+      case 160: return launch<Kind::Dense, 160>(ta, tb, tb2, tc, g, grid, stream);
+      default: return launch<Kind::Dense, 128>(ta, tb, tb2, tc, g, grid, stream);
     }
   }
   switch (p.bn) {
-    case 16: return launch<Kind::Swap, 16>(ta, tb, tc, g, grid, stream);
-    case 32: return launch<Kind::Swap, 32>(ta, tb, tc, g, grid, stream);
-    case 64: return launch<Kind::Swap, 64>(ta, tb, tc, g, grid, stream);
-    default: return launch<Kind::Swap, 128>(ta, tb, tc, g, grid, stream);
+    case 16: return launch<Kind::Swap, 16>(ta, tb, tb, tc, g, grid, stream);
+    case 32: return launch<Kind::Swap, 32>(ta, tb, tb, tc, g, grid, stream);
+    case 64: return launch<Kind::Swap, 64>(ta, tb, tb, tc, g, grid, stream);
+    default: return launch<Kind::Swap, 128>(ta, tb, tb, tc, g, grid, stream);
   }
 }
 
@@ -701,7 +796,7 @@ dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int
   g.idx_smem = (N / 64 + 1 + nnzb) <= Cfg<Kind::Bsr, 256>::IDX_INTS ? 1 : 0;
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
   const int grid = g.num_tiles < d->sm_count ? g.num_tiles : d->sm_count;
-  return launch<Kind::Bsr, 256>(ta, tb, tc, g, grid, stream);
+  return launch<Kind::Bsr, 256>(ta, tb, tb, tc, g, grid, stream);
 }
 
 dq_status dq_bsr_pack(const int8_t* wq, int64_t N, int64_t K, const int32_t* crow, const int32_t* col,

@@ -31,6 +31,11 @@ struct GemmArgs {
   int nnzb;
   int nbr;                // Bsr: block rows (N / 64)
   int idx_smem;           // Bsr: crow and col staged in shared memory (they fit)
+  // Dense, two tile widths (bn2 > 0): tiles [0, t1) are BN wide in row-major
+  // tile order (a_tiles x b_tiles); tiles t1 .. num_tiles - 1 are bn2 wide and
+  // cover the rest of the matrix: first_cnt tiles in 128-row block mb0 from
+  // column c_start on, then per_row tiles in each later block row.
+  int t1, bn2, mb0, c_start, first_cnt, per_row;
   WaitCtl wait;
 };
 

@@ -53,6 +53,8 @@ inline bool aligned(const void* p, size_t a) {
 extern "C" DQ_API void dq_debug_set_schedule(int mode);
 // Measurement knob: force the dense tile width (128, 160, 192, 256; 0 = automatic).
 extern "C" DQ_API void dq_debug_set_tile_n(int n);
+// Measurement knob: 0 turns off the two-width (wave-balanced) dense schedule.
+extern "C" DQ_API void dq_debug_set_two_widths(int on);
 // Measurement knob: quantize kernel (0 = automatic, 1 = register-resident,
 // 2 = row-pipelined through shared memory).
 extern "C" DQ_API void dq_debug_set_quant_kernel(int mode);

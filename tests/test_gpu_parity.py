@@ -161,6 +161,35 @@ def test_stream_k_and_whole_tiles_agree():
         assert np.array_equal(outs[0][rows], oracle.gemm_s32(A[rows], W))
 
 
+# Shapes whose uniform 128 x 256 tiling leaves a partial last wave on 148 SMs,
+# so the dense schedule uses two tile widths: full waves of 256-wide tiles,
+# then one wave of narrower tiles (192 wide for 2048 x 4096; 64 wide for the
+# ragged ones, whose last narrow tile is only partly inside the matrix).
+TWO_WIDTH_SHAPES = [(2048, 4096, 512), (1300, 3464, 256), (2300, 4104, 384), (2048, 4096, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", TWO_WIDTH_SHAPES)
+def test_two_width_schedule_parity(M, N, K):
+    A, W, s_row, s_col, bias = _gemm_inputs(M, N, K, 500 + M + N)
+    Ad, Wd = to_dev(A), to_dev(W)
+    dq.dq_debug_set_schedule(1)
+    outs = {}
+    try:
+        for on in (1, 0):
+            dq.dq_debug_set_two_widths(on)
+            outs[on] = (dq.dq_int8_linear(Ad, None, Wd, None, out_dtype="s32"),
+                        dq.dq_int8_linear(Ad, to_dev(s_row), Wd, to_dev(s_col), bias=to_dev_bf16(bias)))
+    finally:
+        dq.dq_debug_set_two_widths(1)
+    # identical bits with and without the narrow second wave
+    assert torch.equal(outs[1][0], outs[0][0])
+    assert torch.equal(outs[1][1].view(torch.int16), outs[0][1].view(torch.int16))
+    rows = np.unique(np.concatenate([sample_rows(M, 40), np.arange(max(0, M - 130), M)]))
+    want = oracle.gemm_s32(A[rows], W)
+    assert np.array_equal(outs[1][0].cpu().numpy()[rows], want)
+    assert_bf16_close(bf16_bits(outs[1][1])[rows], oracle.epilogue_bf16(want, s_row[rows], s_col, bias))
+
+
 def test_identity_weight_returns_quantized_activations():
     K = 256
     x = synth.normal_bf16((300, K), 1.0, 9)
