@@ -2,8 +2,9 @@
 """Benchmark of the int8 dynamic-quantization linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload llm|tiny|large_m|large_m_s32|vit_fc1|vit_fc2|vit_fc1_dense|
-                                vit_fc2_dense|quant|small_m1|small_m16|small_m128|mma_peak]
+                    [--workload llm|tiny|large_m|large_m_s32|vit_fc1|vit_fc2|vit_fc1_20|vit_fc2_20|
+                                vit_fc1_b32|vit_fc1_b16|vit_fc1_dense|vit_fc2_dense|quant|small_m1|
+                                small_m16|small_m128|mma_peak]
 
 One step = one pass of the layer over one batch: per-token quantization of
 the bf16 activations (dq_quantize_rows) and the fused i8i8->bf16 GEMM
@@ -90,6 +91,14 @@ WORKLOADS = {
                         desc="large-M int8 GEMM M=38400 K=1024 N=4096, raw int32 out"),
     "vit_fc1": dict(kind="bsr", layer="fc1", desc="ViT-H fc1 BSR 10% of 64x64 blocks, M=65792 K=1280 N=5120"),
     "vit_fc2": dict(kind="bsr", layer="fc2", desc="ViT-H fc2 BSR 10% of 64x64 blocks, M=65792 K=5120 N=1280"),
+    "vit_fc1_20": dict(kind="bsr", layer="fc1", keep=0.2,
+                       desc="ViT-H fc1 BSR 20% of 64x64 blocks (sparsity 0.8), M=65792 K=1280 N=5120"),
+    "vit_fc2_20": dict(kind="bsr", layer="fc2", keep=0.2,
+                       desc="ViT-H fc2 BSR 20% of 64x64 blocks (sparsity 0.8), M=65792 K=5120 N=1280"),
+    "vit_fc1_b32": dict(kind="bsr", layer="fc1", bs=32,
+                        desc="ViT-H fc1 BSR 10% of 32x32 blocks, M=65792 K=1280 N=5120"),
+    "vit_fc1_b16": dict(kind="bsr", layer="fc1", bs=16,
+                        desc="ViT-H fc1 BSR 10% of 16x16 blocks, M=65792 K=1280 N=5120"),
     "vit_fc1_dense": dict(kind="bsr_dense", layer="fc1", desc="ViT-H fc1 dense int8 twin M=65792 K=1280 N=5120"),
     "vit_fc2_dense": dict(kind="bsr_dense", layer="fc2", desc="ViT-H fc2 dense int8 twin M=65792 K=5120 N=1280"),
     "quant": dict(kind="quant", M=16384, K=8192, desc="standalone per-token quantize X bf16 [16384, 8192]"),
@@ -114,7 +123,7 @@ def _synth_inputs(name, wl, seed):
     if k == "gemm":
         return synth.large_m(seed)
     if k in ("bsr", "bsr_dense"):
-        return synth.vit_h_bsr(seed, wl["layer"])
+        return synth.vit_h_bsr(seed, wl["layer"], keep=wl.get("keep", 0.10), bs=wl.get("bs", 64))
     if k == "quant":
         return synth.quant_sweep(seed)
     return {}
@@ -133,8 +142,9 @@ def step_accounting(wl, d):
     if k in ("bsr", "bsr_dense"):
         M, K, N = d["M"], d["K"], d["N"]
         nnzb = int(d["crow"][-1])
-        ops = 2.0 * M * nnzb * 64 * 64 if k == "bsr" else 2.0 * M * N * K
-        wbytes = nnzb * 4096 if k == "bsr" else N * K
+        bs = wl.get("bs", 64)
+        ops = 2.0 * M * nnzb * bs * bs if k == "bsr" else 2.0 * M * N * K
+        wbytes = nnzb * bs * bs if k == "bsr" else N * K
         return ops, dict(kernel="dq_bsr_int8_linear" if k == "bsr" else "dq_int8_linear", ops=ops,
                          bytes=M * K + wbytes + 2 * M * N + 4 * (M + N), quant_bytes=3 * M * K + 4 * M)
     if k == "quant":
@@ -296,7 +306,7 @@ def make_state(name, wl, dq, torch, seed):
         wq, sc = dq.dq_quantize_weight(w)
         del w
         crow, col = _to_dev(torch, d["crow"]), _to_dev(torch, d["col"])
-        values = dq.dq_bsr_pack(wq, crow, col)
+        values = dq.dq_bsr_pack(wq, crow, col, block=wl.get("bs", 64))
         M, K, N = d["M"], d["K"], d["N"]
         x = _to_dev_bf16(torch, d["x"])
         del d["x"]
@@ -563,13 +573,14 @@ def _oracle_sample(name, wl, d, rows):
             oracle.epilogue_bf16(acc, d["s_row"][rows], d["s_col"])
         return 2.0 * len(rows) * d["b"].shape[0] * d["b"].shape[1]
     if k == "bsr":
+        bs = wl.get("bs", 64)
         if "_vals" not in d:
             wq, sc = oracle.quantize_rows_f32(d["w"])
-            d["_vals"], d["_sc"] = oracle.bsr_pack(wq, d["crow"], d["col"]), sc
+            d["_vals"], d["_sc"] = oracle.bsr_pack(wq, d["crow"], d["col"], bs), sc
         q, s = oracle.quantize_rows_bf16(d["x"][rows])
-        acc = oracle.bsr_gemm_s32(q, d["N"], d["crow"], d["col"], d["_vals"])
+        acc = oracle.bsr_gemm_s32(q, d["N"], d["crow"], d["col"], d["_vals"], bs)
         oracle.epilogue_bf16(acc, s, d["_sc"])
-        return 2.0 * len(rows) * int(d["crow"][-1]) * 4096
+        return 2.0 * len(rows) * int(d["crow"][-1]) * bs * bs
     if k == "quant":
         oracle.quantize_rows_bf16(d["x"][rows])
         return float(len(rows) * (3 * d["x"].shape[1] + 4))
@@ -592,7 +603,7 @@ def cpu_baseline(name, wl, d, budget_s=12.0):
     if "x" not in d and wl["kind"] in ("bsr",):
         import synth
         d = dict(d)
-        d["x"] = synth.vit_h_bsr(0, wl["layer"])["x"]
+        d["x"] = synth.vit_h_bsr(0, wl["layer"], keep=wl.get("keep", 0.10), bs=wl.get("bs", 64))["x"]
     M = d["x"].shape[0] if "x" in d else d["a"].shape[0]
     chunk = _rows_per_chunk(wl, d)
     _oracle_sample(name, wl, d, np.arange(min(chunk, M)))    # prepare weights outside the clock

@@ -225,6 +225,30 @@ DQ_API dq_status dq_bsr_validate(const int32_t* crow, const int32_t* col, int64_
                           int64_t nnzb);
 
 /* ------------------------------------------------------------------------
+ * The same three calls for square blocks of 64, 32 or 16 (the BSR block
+ * size is a parameter of the pages' benchmark, --sp-linear-tile-size in the
+ * PR 821 review; PyTorch BSR tensors carry it as values' trailing shape).
+ * `block` in {64, 32, 16}; every "64" above becomes `block`: crow int32
+ * [N/block + 1], col int32 [nnzb] (0 <= col < K/block), values int8
+ * [nnzb, block, block] (row j = channel block*b + j, `block` contiguous k
+ * values).  Requirements: K % block == 0, N % block == 0, K % 16 == 0.
+ * block == 64 is exactly dq_bsr_int8_linear / dq_bsr_pack / dq_bsr_validate.
+ * Another block size returns DQ_ERR_UNSUPPORTED (DQ_ERR_INVALID_ARG from
+ * the validator).  Smaller blocks cost more per useful MAC: a 16x16 block
+ * still issues a K = 32 MMA (its other half multiplies zeros).
+ * ------------------------------------------------------------------------ */
+DQ_API dq_status dq_bsr_int8_linear_blocked(const int8_t* A, const float* s_row, int64_t M, int64_t K,
+                                            int64_t N, int64_t block, const int32_t* crow,
+                                            const int32_t* col, const int8_t* values, int64_t nnzb,
+                                            const float* s_col, const void* bias_bf16, void* out,
+                                            dq_out_dtype out_dtype, dq_stream_t stream);
+DQ_API dq_status dq_bsr_pack_blocked(const int8_t* wq, int64_t N, int64_t K, int64_t block,
+                                     const int32_t* crow, const int32_t* col, int64_t nnzb,
+                                     int8_t* values, dq_stream_t stream);
+DQ_API dq_status dq_bsr_validate_blocked(const int32_t* crow, const int32_t* col, int64_t N, int64_t K,
+                                         int64_t block, int64_t nnzb);
+
+/* ------------------------------------------------------------------------
  * Measurement helper: a kernel that only issues tcgen05.mma.kind::i8
  * (128x256x32, operands resident in shared memory, accumulator in TMEM) on
  * every SM, `iters` times per CTA, with no global-memory traffic.  Used to

@@ -39,6 +39,10 @@ _PROTOS = {
     "dq_bsr_int8_linear": (_I32, [_P, _P, _I64, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _I32, _P]),
     "dq_bsr_pack": (_I32, [_P, _I64, _I64, _P, _P, _I64, _P, _P]),
     "dq_bsr_validate": (_I32, [_P, _P, _I64, _I64, _I64]),
+    "dq_bsr_int8_linear_blocked": (_I32, [_P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _I32,
+                                          _P]),
+    "dq_bsr_pack_blocked": (_I32, [_P, _I64, _I64, _I64, _P, _P, _I64, _P, _P]),
+    "dq_bsr_validate_blocked": (_I32, [_P, _P, _I64, _I64, _I64, _I64]),
     "dq_mma_peak_probe": (_I32, [_I32, _I32, _P]),
     "dq_debug_set_schedule": (None, [_I32]),
     "dq_debug_set_tile_n": (None, [_I32]),
@@ -265,8 +269,10 @@ def dq_int8_linear_noalloc(A, s_row, W, s_col, out, bias=None, out_dtype="bf16",
 
 def dq_bsr_int8_linear(A, s_row, N, crow, col, values, s_col, bias=None, out=None, out_dtype="bf16",
                        stream=None):
-    """BSR (64x64 int8 blocks) variant of dq_int8_linear; W given as
-    crow int32 [N/64+1], col int32 [nnzb], values int8 [nnzb, 64, 64]."""
+    """BSR variant of dq_int8_linear; W given as crow int32 [N/b+1], col int32
+    [nnzb], values int8 [nnzb, b, b] with the block size b in {64, 32, 16}
+    taken from values' shape (dq_bsr_int8_linear_blocked; b = 64 is
+    dq_bsr_int8_linear)."""
     code = _out_code(out_dtype)
     _need(A, torch.int8, "A", 2)
     _contig(A, "A")
@@ -275,9 +281,9 @@ def dq_bsr_int8_linear(A, s_row, N, crow, col, values, s_col, bias=None, out=Non
     _need(col, torch.int32, "col", 1)
     _need(values, torch.int8, "values", 3)
     _contig(values, "values")
-    nnzb = values.shape[0]
-    if crow.numel() != N // 64 + 1 or col.numel() != nnzb or tuple(values.shape[1:]) != (64, 64):
-        raise ValueError("BSR arrays do not match N / nnzb")
+    nnzb, b = values.shape[0], values.shape[1]
+    if values.shape[2] != b or N % b != 0 or crow.numel() != N // b + 1 or col.numel() != nnzb:
+        raise ValueError("BSR arrays do not match N / nnzb / block size")
     if code == DQ_OUT_BF16:
         _need(s_row, torch.float32, "s_row", 1)
         _need(s_col, torch.float32, "s_col", 1)
@@ -288,27 +294,33 @@ def dq_bsr_int8_linear(A, s_row, N, crow, col, values, s_col, bias=None, out=Non
         out = torch.empty((M, N), dtype=odt, device=A.device)
     _need(out, odt, "out", 2)
     _contig(out, "out")
-    _check(lib.dq_bsr_int8_linear(_ptr(A), _ptr(s_row), M, K, N, _ptr(crow), _ptr(col),
-                                  _ptr(values) if nnzb else None, nnzb, _ptr(s_col), _ptr(bias), _ptr(out),
-                                  code, _stream(stream)), "dq_bsr_int8_linear")
+    vp = _ptr(values) if nnzb else None
+    if b == 64:
+        st = lib.dq_bsr_int8_linear(_ptr(A), _ptr(s_row), M, K, N, _ptr(crow), _ptr(col), vp, nnzb,
+                                    _ptr(s_col), _ptr(bias), _ptr(out), code, _stream(stream))
+        _check(st, "dq_bsr_int8_linear")
+    else:
+        st = lib.dq_bsr_int8_linear_blocked(_ptr(A), _ptr(s_row), M, K, N, b, _ptr(crow), _ptr(col), vp, nnzb,
+                                            _ptr(s_col), _ptr(bias), _ptr(out), code, _stream(stream))
+        _check(st, "dq_bsr_int8_linear_blocked")
     return out
 
 
-def dq_bsr_pack(wq, crow, col, values=None, stream=None):
-    """Gather the 64x64 blocks of a dense int8 weight [N, K] named by (crow, col)."""
+def dq_bsr_pack(wq, crow, col, values=None, stream=None, block: int = 64):
+    """Gather the block x block blocks of a dense int8 weight [N, K] named by (crow, col)."""
     _need(wq, torch.int8, "wq", 2)
     _contig(wq, "wq")
     N, K = wq.shape
     nnzb = col.numel()
     if values is None:
-        values = torch.empty((nnzb, 64, 64), dtype=torch.int8, device=wq.device)
-    _check(lib.dq_bsr_pack(_ptr(wq), N, K, _ptr(crow), _ptr(col), nnzb, _ptr(values) if nnzb else None,
-                           _stream(stream)), "dq_bsr_pack")
+        values = torch.empty((nnzb, block, block), dtype=torch.int8, device=wq.device)
+    _check(lib.dq_bsr_pack_blocked(_ptr(wq), N, K, block, _ptr(crow), _ptr(col), nnzb,
+                                   _ptr(values) if nnzb else None, _stream(stream)), "dq_bsr_pack_blocked")
     return values
 
 
-def dq_bsr_validate(crow, col, N: int, K: int) -> int:
-    return lib.dq_bsr_validate(_ptr(crow), _ptr(col) if col.numel() else None, N, K, col.numel())
+def dq_bsr_validate(crow, col, N: int, K: int, block: int = 64) -> int:
+    return lib.dq_bsr_validate_blocked(_ptr(crow), _ptr(col) if col.numel() else None, N, K, block, col.numel())
 
 
 def dq_mma_peak_probe(grid: int, iters: int, stream=None) -> None:

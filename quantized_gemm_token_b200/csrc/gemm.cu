@@ -18,11 +18,13 @@
 //   Dense  A slot = 128 activation rows, B slot = BN weight channels.
 //   Swap   A slot = 128 weight channels, B slot = BN (16..128) tokens: for
 //          few tokens the weight stream, not the token count, fills MMA M.
-//   Bsr    A slot = 128 activation rows x one 64-wide k slice, B slot = one
-//          nonzero 64x64 weight block; a tile spans 4 block rows (256
-//          channels) and each block accumulates into its block row's 64-column
-//          slice of the TMEM tile; the producer walks crow/col (PR 821: the
-//          kernel takes crow_indices / col_indices / values directly).
+//   Bsr    A slot = 128 activation rows x the k slice of one block column,
+//          B slot = one nonzero weight block (64x64, 32x32 or 16x16: kinds
+//          Bsr, Bsr32, Bsr16); a tile spans 256 channels (4, 8 or 16 block
+//          rows) and each block accumulates into its block row's slice of the
+//          TMEM tile; the producer walks crow/col (PR 821: the kernel takes
+//          crow_indices / col_indices / values directly).  A 16-wide block
+//          is issued as a K = 32 MMA whose other 16 k bytes read zeros.
 //
 // Schedules: whole tiles round-robin over one CTA per SM, or (when the tile
 // count would leave SMs idle) stream-K: the tile x k-block iteration space is
@@ -39,16 +41,22 @@ namespace dq {
 template <Kind KIND, int BN>
 struct Cfg {
   static constexpr int BM = 128;
-  static constexpr int KB = KIND == Kind::Bsr ? 64 : 128;     // k bytes per stage
+  static constexpr bool BSR = is_bsr(KIND);
+  static constexpr int BS = bsr_bs(KIND);                     // block size (BSR kinds)
+  // k bytes per stage: dense 128 (128-byte swizzle); 64x64 blocks 64 (64-byte
+  // swizzle); 32x32 and 16x16 blocks 32 (32-byte swizzle; a 16-wide block
+  // uses the 32-byte A slice that contains it, the other half of the MMA's K
+  // multiplying zeros, see the Bsr16 B descriptor).
+  static constexpr int KB = !BSR ? 128 : BS == 64 ? 64 : 32;
   static constexpr int A_BYTES = BM * KB;
-  // Bsr: a tile spans BN/64 block rows; each stage holds one 64x64 block
-  // that accumulates into its block row's 64-column slice of the tile.
-  static constexpr int B_ROWS = KIND == Kind::Bsr ? 64 : BN;
+  // BSR: a tile spans BN/BS block rows; each stage holds one BS x BS block
+  // that accumulates into its block row's BS-column slice of the tile.
+  static constexpr int B_ROWS = BSR ? BS : BN;
   static constexpr int MMA_N = B_ROWS;
-  static constexpr int NSUB = KIND == Kind::Bsr ? BN / 64 : 1;
-  static constexpr int B_BYTES = B_ROWS * KB;
+  static constexpr int NSUB = BSR ? BN / BS : 1;
+  static constexpr int B_BYTES = BSR ? BS * BS : B_ROWS * KB;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  // Row-layout epilogues (Dense, Bsr) stage each warp's 32x32 output block in
+  // Row-layout epilogues (Dense, BSR) stage each warp's 32x32 output block in
   // shared memory for a TMA store: 2 buffers x 4 warps x 4 KB (int32 worst case).
   // Epilogue warps: two per TMEM sub-partition when a tile has at least two
   // 32-column chunks, so one warp's latency hides behind the other's work.
@@ -56,8 +64,26 @@ struct Cfg {
   static constexpr bool STAGED_OUT = KIND != Kind::Swap;
   static constexpr int OUT_BUF_BYTES = 32 * 32 * 4;           // per epilogue warp
   static constexpr int OUT_BYTES = STAGED_OUT ? EPI_WARPS * OUT_BUF_BYTES : 0;
-  static constexpr int STAGES_RAW = (224 * 1024 - OUT_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+  // BSR: crow and col are copied to shared memory when nbr + 1 + nnzb fits
+  // (every tile and every block needs them; a global load per block would put
+  // a dependent L2 round trip in front of each TMA issue).
+  static constexpr int IDX_INTS = BSR ? 4096 : 0;
+  static constexpr int IDX_BYTES = IDX_INTS * 4;
+  // 16x16 blocks: two 256-byte zero regions, one below and one above the
+  // stage buffers, that stand in for the half of the MMA's K the block does
+  // not cover (the descriptor's leading-dimension offset must be positive).
+  static constexpr int ZERO_BYTES = KIND == Kind::Bsr16 ? 1024 : 0;
+  static constexpr int STAGE_CAP = BSR && BS < 64 ? 24 : 12;
+  static constexpr int STAGES_RAW = (224 * 1024 - OUT_BYTES - IDX_BYTES - 2 * ZERO_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > STAGE_CAP ? STAGE_CAP : STAGES_RAW;
+  // shared-memory layout (offsets from the 1024-aligned base)
+  static constexpr int OFF_ZLO = 0;
+  static constexpr int OFF_A = ZERO_BYTES;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_ZHI = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_OUT = (OFF_ZHI + ZERO_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_IDX = OFF_OUT + OUT_BYTES;
+  static constexpr int OFF_BARS = OFF_IDX + IDX_BYTES;
   static constexpr int ACC_RAW = 512 / BN;
   static constexpr int ACC_BUFS = ACC_RAW > 8 ? 8 : ACC_RAW;
   static constexpr int ACC_COLS = ACC_BUFS * BN;
@@ -65,16 +91,12 @@ struct Cfg {
                                    : ACC_COLS <= 256 ? 256 : 512;
   static constexpr int K_STEPS = KB / 32;                     // MMA K = 32 bytes
   static constexpr int CW = BN >= 32 ? 32 : 16;               // epilogue chunk (columns)
-  // Bsr: crow and col are copied to shared memory when nbr + 1 + nnzb fits
-  // (every tile and every block needs them; a global load per block would put
-  // a dependent L2 round trip in front of each TMA issue).
-  static constexpr int IDX_INTS = KIND == Kind::Bsr ? 4096 : 0;
-  static constexpr int IDX_BYTES = IDX_INTS * 4;
-  static constexpr int SMEM_BYTES =
-      STAGES * STAGE_BYTES + OUT_BYTES + IDX_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int SMEM_BYTES = OFF_BARS + 512 /*barriers*/ + 1024 /*align*/;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(STAGES >= 2, "stages");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static_assert(!BSR || BN % (BSR ? BS : 1) == 0, "tile covers whole block rows");
 };
 
 // Where a tile lies: 128-row block ta, B-slot tile tb, first output column n0
@@ -127,11 +149,11 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint8_t* sOut = smem + C::STAGES * C::STAGE_BYTES;          // 1024-aligned
-  int* sIdx = reinterpret_cast<int*>(sOut + C::OUT_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + C::OUT_BYTES + C::IDX_BYTES);
+  uint8_t* sA = smem + C::OFF_A;
+  uint8_t* sB = smem + C::OFF_B;
+  uint8_t* sOut = smem + C::OFF_OUT;                          // 1024-aligned
+  int* sIdx = reinterpret_cast<int*>(smem + C::OFF_IDX);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + C::STAGES;
   uint64_t* accf_bar = bars + 2 * C::STAGES;
@@ -169,8 +191,17 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
   // parameters; with a programmatic (early) launch, wait here for the
   // previous kernel of the stream before any global memory access.
   griddep_wait();
-  const int* idx = nullptr;      // Bsr: crow at idx[0..nbr], col at idx[nbr+1..]
-  if constexpr (KIND == Kind::Bsr) {
+  const int* idx = nullptr;      // BSR: crow at idx[0..nbr], col at idx[nbr+1..]
+  if constexpr (KIND == Kind::Bsr16) {
+    // the zero regions the 16x16-block B descriptors point at, visible to
+    // the tensor core (async proxy) before the first MMA
+    for (int i = threadIdx.x; i < C::ZERO_BYTES / 16; i += blockDim.x) {
+      reinterpret_cast<uint4*>(smem + C::OFF_ZLO)[i] = make_uint4(0u, 0u, 0u, 0u);
+      reinterpret_cast<uint4*>(smem + C::OFF_ZHI)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
+  if constexpr (C::BSR) {
     if (g.idx_smem) {
       const int nbr = g.nbr;
       for (int i = threadIdx.x; i <= nbr; i += blockDim.x) sIdx[i] = __ldg(g.crow + i);
@@ -198,7 +229,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
         const uint32_t stage_tx = C::A_BYTES + (KIND == Kind::Dense ? geo.width * C::KB : C::B_BYTES);
         for (int j = 0; ok && j < C::NSUB; ++j) {
         int k0 = s.kb0, k1 = s.kb1;
-        if constexpr (KIND == Kind::Bsr) {
+        if constexpr (C::BSR) {
           const int br = tb * C::NSUB + j;
           if (br >= g.nbr) break;
           bsr_range(g, idx, br, k0, k1);
@@ -212,10 +243,13 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
           mbar_arrive_expect_tx(fb, stage_tx);
           const uint32_t da = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t db = smem_u32(sB + stage * C::B_BYTES);
-          if constexpr (KIND == Kind::Bsr) {
+          if constexpr (C::BSR) {
+            // A: the KB-wide k slice holding block column c (for 16-wide
+            // blocks the 32-byte slice that contains it); B: block kb
             const int c = idx ? idx[g.nbr + 1 + kb] : __ldg(g.col + kb);
-            tma_load_2d(da, &tm_a, fb, c * 64, ta * 128);
-            tma_load_2d(db, &tm_b, fb, 0, kb * 64);
+            const int ax = KIND == Kind::Bsr16 ? (c >> 1) * 32 : c * C::BS;
+            tma_load_2d(da, &tm_a, fb, ax, ta * 128);
+            tma_load_2d(db, &tm_b, fb, 0, kb * C::BS);
           } else {
             tma_load_2d(da, &tm_a, fb, kb * C::KB, ta * 128);
             tma_load_2d(db, geo.narrow ? &tm_b2 : &tm_b, fb, kb * C::KB, geo.n0);
@@ -259,7 +293,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
                                    ? idesc_i8(128, g.bn2) : idesc_full;
         for (int j = 0; ok && j < C::NSUB; ++j) {
         int k0 = s.kb0, k1 = s.kb1;
-        if constexpr (KIND == Kind::Bsr) {
+        if constexpr (C::BSR) {
           const int br = (s.tile % g.b_tiles) * C::NSUB + j;
           if (br >= g.nbr) break;
           bsr_range(g, idx, br, k0, k1);
@@ -273,7 +307,17 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
           }
           tc_fence_after();
           const uint64_t ad = smem_desc_kmajor<C::KB>(smem_u32(sA + stage * C::A_BYTES));
-          const uint64_t bd = smem_desc_kmajor<C::KB>(smem_u32(sB + stage * C::B_BYTES));
+          uint64_t bd;
+          if constexpr (KIND == Kind::Bsr16) {
+            // 16 channels x 16 k of the block, rows of 16 bytes (no swizzle):
+            // the MMA's other 16 k bytes read a zero region, so the 32-byte A
+            // slice's other half contributes nothing.
+            const int c = idx ? idx[g.nbr + 1 + kb] : __ldg(g.col + kb);
+            bd = smem_desc_b16_padded(smem_u32(sB + stage * C::B_BYTES), smem_u32(smem + C::OFF_ZLO),
+                                      smem_u32(smem + C::OFF_ZHI), c & 1);
+          } else {
+            bd = smem_desc_kmajor<C::KB>(smem_u32(sB + stage * C::B_BYTES));
+          }
 #pragma unroll
           for (int k = 0; k < C::K_STEPS; ++k)
             mma_i8(d, ad + 2 * k, bd + 2 * k, idesc, (kb > k0 || k > 0) ? 1u : 0u);
@@ -355,13 +399,21 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
 #pragma unroll 1
         for (int c = grp; c < nch; c += GROUPS) {
           uint32_t r[CW];
-          bool empty_slice = false;     // Bsr: this chunk's block row has no block
-          if constexpr (KIND == Kind::Bsr) {
-            int p0, p1;
-            const int br = tb * C::NSUB + (c * CW) / 64;
-            if (br < g.nbr) bsr_range(g, idx, br, p0, p1);
-            empty_slice = br >= g.nbr || p0 == p1;
+          // BSR: block rows of this chunk without blocks (their TMEM slice
+          // was never written) read as zeros; a 32-column chunk holds one
+          // block row's columns, or two 16-wide block rows
+          bool empty_lo = false, empty_hi = false;
+          if constexpr (C::BSR) {
+            auto row_empty = [&](int br) {
+              int p0 = 0, p1 = 0;
+              if (br < g.nbr) bsr_range(g, idx, br, p0, p1);
+              return br >= g.nbr || p0 == p1;
+            };
+            const int br = tb * C::NSUB + (c * CW) / C::BS;
+            empty_lo = row_empty(br);
+            empty_hi = C::BS >= CW ? empty_lo : row_empty(br + 1);
           }
+          const bool empty_slice = empty_lo && empty_hi;
           if (empty_slice) {
 #pragma unroll
             for (int j = 0; j < CW; ++j) r[j] = 0;
@@ -375,6 +427,13 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
             if (!g.out_s32) load_col_scales(g, n0 + c * CW, cs);
           }
           tmem_ld_wait();
+          if constexpr (KIND == Kind::Bsr16) {
+            if (!empty_slice && (empty_lo || empty_hi)) {
+#pragma unroll
+              for (int j = 0; j < CW; ++j)
+                if (j < 16 ? empty_lo : empty_hi) r[j] = 0;
+            }
+          }
           if (c == last_c) {
             tc_fence_before();
             mbar_arrive(smem_u32(acce_bar + acc));
@@ -452,19 +511,23 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
 __global__ void __launch_bounds__(256) bsr_pack_kernel(const int8_t* __restrict__ wq, int64_t K,
                                                        const int32_t* __restrict__ crow,
                                                        const int32_t* __restrict__ col, int nnzb,
-                                                       int nbc, int8_t* __restrict__ values) {
+                                                       int nbc, int bs, int8_t* __restrict__ values) {
+  // one CTA per block row; a block's rows are split into 16-byte parts
   const int br = blockIdx.x;
-  int p0 = min(max(__ldg(crow + br), 0), nnzb);
-  int p1 = min(max(__ldg(crow + br + 1), p0), nnzb);
-  const int j = threadIdx.x >> 2;          // row inside the block (64 rows)
-  const int part = threadIdx.x & 3;        // 16-byte quarter of the 64-byte row
+  const int p0 = min(max(__ldg(crow + br), 0), nnzb);
+  const int p1 = min(max(__ldg(crow + br + 1), p0), nnzb);
+  const int parts = bs / 16;
   for (int p = p0; p < p1; ++p) {
     const int c = __ldg(col + p);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (c >= 0 && c < nbc)
-      v = __ldg(reinterpret_cast<const uint4*>(wq + (static_cast<int64_t>(br) * 64 + j) * K +
-                                               static_cast<int64_t>(c) * 64) + part);
-    reinterpret_cast<uint4*>(values + (static_cast<int64_t>(p) * 64 + j) * 64)[part] = v;
+    for (int t = threadIdx.x; t < bs * parts; t += blockDim.x) {
+      const int j = t / parts;             // row inside the block
+      const int part = t % parts;          // 16-byte part of the row
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (c >= 0 && c < nbc)
+        v = __ldg(reinterpret_cast<const uint4*>(wq + (static_cast<int64_t>(br) * bs + j) * K +
+                                                 static_cast<int64_t>(c) * bs) + part);
+      reinterpret_cast<uint4*>(values + (static_cast<int64_t>(p) * bs + j) * bs)[part] = v;
+    }
   }
 }
 
@@ -742,10 +805,11 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   }
 }
 
-dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K, int64_t N,
-                             const int32_t* crow, const int32_t* col, const int8_t* values,
-                             int64_t nnzb, const float* s_col, const void* bias_bf16, void* out,
-                             dq_out_dtype out_dtype, dq_stream_t stream_) {
+dq_status dq_bsr_int8_linear_blocked(const int8_t* A, const float* s_row, int64_t M, int64_t K, int64_t N,
+                                     int64_t block, const int32_t* crow, const int32_t* col,
+                                     const int8_t* values, int64_t nnzb, const float* s_col,
+                                     const void* bias_bf16, void* out, dq_out_dtype out_dtype,
+                                     dq_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (out_dtype != DQ_OUT_BF16 && out_dtype != DQ_OUT_S32) return DQ_ERR_INVALID_ARG;
   if (M < 0 || K < 1 || N < 1 || nnzb < 0) return DQ_ERR_INVALID_ARG;
@@ -753,7 +817,8 @@ dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int
   if (M > 0 && nnzb > 0 && (col == nullptr || values == nullptr)) return DQ_ERR_INVALID_ARG;
   if (M > 0 && out_dtype == DQ_OUT_BF16 && (s_row == nullptr || s_col == nullptr))
     return DQ_ERR_INVALID_ARG;
-  if (K % 64 != 0 || N % 64 != 0 || K > 133120) return DQ_ERR_UNSUPPORTED;
+  if (block != 64 && block != 32 && block != 16) return DQ_ERR_UNSUPPORTED;
+  if (K % block != 0 || N % block != 0 || K % 16 != 0 || K > 133120) return DQ_ERR_UNSUPPORTED;
   if (M > (int64_t(1) << 31) - 128 || N > (int64_t(1) << 31) - 256 || nnzb > (int64_t(1) << 24))
     return DQ_ERR_UNSUPPORTED;
   if (!aligned(A, 16) || !aligned(out, 16) || (values && !aligned(values, 16))) return DQ_ERR_UNSUPPORTED;
@@ -764,11 +829,18 @@ dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int
   if (st != DQ_OK) return st;
   if (M == 0) return DQ_OK;
 
+  // A: k slices of 64 bytes (64-wide blocks) or 32 bytes (32- and 16-wide
+  // blocks) x 128 rows, swizzled to the slice width.  B: the blocks viewed as
+  // a [nnzb * block, block] byte matrix, one block per box; 16-byte rows of
+  // 16-wide blocks are not swizzled.
+  const int kb = block == 64 ? 64 : 32;
+  const int bsw = block == 16 ? 0 : static_cast<int>(block);
+  const uint32_t ub = static_cast<uint32_t>(block);
   CUtensorMap ta, tb;
-  if ((st = make_tmap_u8_2d(&ta, A, K, M, K, 64, 128, 64)) != DQ_OK) return st;
+  if ((st = make_tmap_u8_2d(&ta, A, K, M, K, kb, 128, kb)) != DQ_OK) return st;
   // With no blocks the B map is never read; describe A again to keep it valid.
-  if (nnzb > 0) st = make_tmap_u8_2d(&tb, values, 64, static_cast<uint64_t>(nnzb) * 64, 64, 64, 64, 64);
-  else st = make_tmap_u8_2d(&tb, A, K, M, K, 64, 64, 64);
+  if (nnzb > 0) st = make_tmap_u8_2d(&tb, values, ub, static_cast<uint64_t>(nnzb) * ub, ub, ub, ub, bsw);
+  else st = make_tmap_u8_2d(&tb, A, K, M, K, ub, ub, bsw);
   if (st != DQ_OK) return st;
   CUtensorMap tc;
   if ((st = make_tmap_out_2d(&tc, out, N, M, out_dtype == DQ_OUT_S32 ? 4 : 2)) != DQ_OK) return st;
@@ -778,8 +850,9 @@ dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int
   g.N = static_cast<int>(N);
   g.K = static_cast<int>(K);
   g.a_tiles = static_cast<int>((M + 127) / 128);
-  g.nbr = static_cast<int>(N / 64);
-  g.b_tiles = (g.nbr + 3) / 4;            // tiles of 4 block rows = 256 channels
+  g.nbr = static_cast<int>(N / block);
+  const int per_tile = static_cast<int>(256 / block);     // block rows per 256-channel tile
+  g.b_tiles = (g.nbr + per_tile - 1) / per_tile;
   g.kb_total = 0;
   const int64_t tiles = static_cast<int64_t>(g.a_tiles) * g.b_tiles;
   if (tiles > 0x7fffffff) return DQ_ERR_UNSUPPORTED;
@@ -793,35 +866,51 @@ dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int
   g.crow = crow;
   g.col = col;
   g.nnzb = static_cast<int>(nnzb);
-  g.idx_smem = (N / 64 + 1 + nnzb) <= Cfg<Kind::Bsr, 256>::IDX_INTS ? 1 : 0;
+  g.idx_smem = (N / block + 1 + nnzb) <= Cfg<Kind::Bsr, 256>::IDX_INTS ? 1 : 0;
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
   const int grid = g.num_tiles < d->sm_count ? g.num_tiles : d->sm_count;
+  if (block == 32) return launch<Kind::Bsr32, 256>(ta, tb, tb, tc, g, grid, stream);
+  if (block == 16) return launch<Kind::Bsr16, 256>(ta, tb, tb, tc, g, grid, stream);
   return launch<Kind::Bsr, 256>(ta, tb, tb, tc, g, grid, stream);
 }
 
-dq_status dq_bsr_pack(const int8_t* wq, int64_t N, int64_t K, const int32_t* crow, const int32_t* col,
-                      int64_t nnzb, int8_t* values, dq_stream_t stream_) {
+dq_status dq_bsr_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K, int64_t N,
+                             const int32_t* crow, const int32_t* col, const int8_t* values,
+                             int64_t nnzb, const float* s_col, const void* bias_bf16, void* out,
+                             dq_out_dtype out_dtype, dq_stream_t stream) {
+  return dq_bsr_int8_linear_blocked(A, s_row, M, K, N, 64, crow, col, values, nnzb, s_col, bias_bf16, out,
+                                    out_dtype, stream);
+}
+
+dq_status dq_bsr_pack_blocked(const int8_t* wq, int64_t N, int64_t K, int64_t block, const int32_t* crow,
+                              const int32_t* col, int64_t nnzb, int8_t* values, dq_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (N < 1 || K < 1 || nnzb < 0 || wq == nullptr || crow == nullptr) return DQ_ERR_INVALID_ARG;
   if (nnzb > 0 && (col == nullptr || values == nullptr)) return DQ_ERR_INVALID_ARG;
-  if (K % 64 != 0 || N % 64 != 0 || nnzb > (int64_t(1) << 24)) return DQ_ERR_UNSUPPORTED;
+  if (block != 64 && block != 32 && block != 16) return DQ_ERR_UNSUPPORTED;
+  if (K % block != 0 || N % block != 0 || K % 16 != 0 || nnzb > (int64_t(1) << 24)) return DQ_ERR_UNSUPPORTED;
   if (!aligned(wq, 16) || (values && !aligned(values, 16))) return DQ_ERR_UNSUPPORTED;
   DeviceInfo* d = nullptr;
   dq_status st = current_device(&d);
   if (st != DQ_OK) return st;
   if (nnzb == 0) return DQ_OK;
-  bsr_pack_kernel<<<static_cast<unsigned>(N / 64), 256, 0, stream>>>(wq, K, crow, col,
-                                                                     static_cast<int>(nnzb),
-                                                                     static_cast<int>(K / 64), values);
+  bsr_pack_kernel<<<static_cast<unsigned>(N / block), 256, 0, stream>>>(
+      wq, K, crow, col, static_cast<int>(nnzb), static_cast<int>(K / block), static_cast<int>(block), values);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 
-dq_status dq_bsr_validate(const int32_t* crow, const int32_t* col, int64_t N, int64_t K, int64_t nnzb) {
-  if (crow == nullptr || N < 1 || K < 1 || nnzb < 0 || N % 64 != 0 || K % 64 != 0)
+dq_status dq_bsr_pack(const int8_t* wq, int64_t N, int64_t K, const int32_t* crow, const int32_t* col,
+                      int64_t nnzb, int8_t* values, dq_stream_t stream) {
+  return dq_bsr_pack_blocked(wq, N, K, 64, crow, col, nnzb, values, stream);
+}
+
+dq_status dq_bsr_validate_blocked(const int32_t* crow, const int32_t* col, int64_t N, int64_t K, int64_t block,
+                                  int64_t nnzb) {
+  if (crow == nullptr || N < 1 || K < 1 || nnzb < 0 || block < 1 || N % block != 0 || K % block != 0)
     return DQ_ERR_INVALID_ARG;
   if (nnzb > 0 && col == nullptr) return DQ_ERR_INVALID_ARG;
-  const int64_t nbr = N / 64;
+  const int64_t nbr = N / block;
   int32_t* hc = new int32_t[nbr + 1];
   int32_t* hk = nnzb > 0 ? new int32_t[nnzb] : nullptr;
   dq_status st = DQ_OK;
@@ -834,11 +923,15 @@ dq_status dq_bsr_validate(const int32_t* crow, const int32_t* col, int64_t N, in
     for (int64_t b = 0; st == DQ_OK && b < nbr; ++b)
       if (hc[b + 1] < hc[b]) st = DQ_ERR_INVALID_ARG;
     for (int64_t p = 0; st == DQ_OK && p < nnzb; ++p)
-      if (hk[p] < 0 || hk[p] >= K / 64) st = DQ_ERR_INVALID_ARG;
+      if (hk[p] < 0 || hk[p] >= K / block) st = DQ_ERR_INVALID_ARG;
   }
   delete[] hc;
   delete[] hk;
   return st;
+}
+
+dq_status dq_bsr_validate(const int32_t* crow, const int32_t* col, int64_t N, int64_t K, int64_t nnzb) {
+  return dq_bsr_validate_blocked(crow, col, N, K, 64, nnzb);
 }
 
 }  // extern "C"

@@ -10,7 +10,13 @@
 
 namespace dq {
 
-enum class Kind : int { Dense = 0, Swap = 1, Bsr = 2 };
+enum class Kind : int { Dense = 0, Swap = 1, Bsr = 2, Bsr32 = 3, Bsr16 = 4 };
+
+// Block-sparse weight kinds and their square block size (64, 32 or 16).
+__host__ __device__ constexpr bool is_bsr(Kind k) { return k == Kind::Bsr || k == Kind::Bsr32 || k == Kind::Bsr16; }
+__host__ __device__ constexpr int bsr_bs(Kind k) {
+  return k == Kind::Bsr ? 64 : k == Kind::Bsr32 ? 32 : k == Kind::Bsr16 ? 16 : 0;
+}
 
 struct GemmArgs {
   int M, N, K;
@@ -29,7 +35,7 @@ struct GemmArgs {
   const int32_t* crow;    // Bsr
   const int32_t* col;
   int nnzb;
-  int nbr;                // Bsr: block rows (N / 64)
+  int nbr;                // Bsr: block rows (N / block size)
   int idx_smem;           // Bsr: crow and col staged in shared memory (they fit)
   // Dense, two tile widths (bn2 > 0): tiles [0, t1) are BN wide in row-major
   // tile order (a_tiles x b_tiles); tiles t1 .. num_tiles - 1 are bn2 wide and

@@ -30,7 +30,8 @@ unsigned long long wait_timeout_ns();
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point.
 // 2-D, uint8 elements: dims {inner, outer}, outer stride in bytes, box
-// {box_inner, box_outer}, swizzle = 128 or 64 (bytes), zero fill out of bounds.
+// {box_inner, box_outer}, swizzle = 128, 64 or 32 (bytes; anything else: none),
+// zero fill out of bounds.
 dq_status make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                           uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer,
                           int swizzle_bytes);

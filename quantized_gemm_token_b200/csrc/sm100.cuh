@@ -207,20 +207,38 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
 }
 
 // Shared-memory matrix descriptor for a K-major operand tile whose rows are
-// `row_bytes` (128 or 64) long, stored with the matching TMA swizzle
-// (128B or 64B), rows packed contiguously so that groups of 8 rows are
-// 8*row_bytes apart.  `addr` is the shared-space byte address of the tile
-// (aligned to the swizzle repeat: 1024 B for 128B, 512 B for 64B).
+// `row_bytes` (128, 64 or 32) long, stored with the matching TMA swizzle,
+// rows packed contiguously so that groups of 8 rows are 8*row_bytes apart.
+// `addr` is the shared-space byte address of the tile (aligned to the
+// swizzle repeat: 1024 B for 128B, 512 B for 64B, 256 B for 32B).
 template <int ROW_BYTES>
 __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t addr) {
-  static_assert(ROW_BYTES == 128 || ROW_BYTES == 64, "row bytes");
-  constexpr uint64_t layout = ROW_BYTES == 128 ? 2ull : 4ull;  // SWIZZLE_128B / SWIZZLE_64B
+  static_assert(ROW_BYTES == 128 || ROW_BYTES == 64 || ROW_BYTES == 32, "row bytes");
+  // SWIZZLE_128B / SWIZZLE_64B / SWIZZLE_32B
+  constexpr uint64_t layout = ROW_BYTES == 128 ? 2ull : ROW_BYTES == 64 ? 4ull : 6ull;
   constexpr uint64_t sbo = (8ull * ROW_BYTES) >> 4;             // 8-row group stride
   return (static_cast<uint64_t>((addr & 0x3FFFFu) >> 4))        // start address
          | (1ull << 16)                                         // LBO (unused when swizzled)
          | (sbo << 32)                                          // SBO
          | (1ull << 46)                                         // descriptor version (sm_100)
          | (layout << 61);
+}
+
+// B descriptor for a 16 x 16 int8 block (16 rows of 16 bytes, no swizzle)
+// used as the 16 x 32 K-major operand of one kind::i8 MMA.  Without swizzle
+// the operand is made of 8-row x 16-byte core matrices: SBO is the step
+// between the two 8-row groups (128 B here) and LBO the step between the two
+// 16-byte k groups.  The block is k group `half` (its column's parity inside
+// the 32-byte A slice); the other k group points at 256 zero bytes: zlo
+// (below the block) when half = 1, zhi (above it) when half = 0, so LBO stays
+// positive.
+__device__ __forceinline__ uint64_t smem_desc_b16_padded(uint32_t block, uint32_t zlo, uint32_t zhi, int half) {
+  const uint32_t start = half ? zlo : block;
+  const uint32_t lbo = half ? block - zlo : zhi - block;
+  return (static_cast<uint64_t>((start & 0x3FFFFu) >> 4))
+         | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16)   // LBO: k-group step
+         | (static_cast<uint64_t>(128u >> 4) << 32)               // SBO: 8-row step
+         | (1ull << 46);                                          // version; layout 0 = no swizzle
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.

@@ -126,7 +126,8 @@ def vit_h_bsr(seed: int = 0, layer: str = "fc1", M: int = 256 * 257, keep: float
               bs: int = 64, with_x: bool = True):
     """ViT-H/14 MLP at batch 256 (257 tokens per image): fc1 K=1280 -> N=5120,
     fc2 K=5120 -> N=1280.  X bf16 ~ N(0,1); W ~ N(0,0.02) masked to a uniform
-    random 10% of its 64x64 blocks (masked-out blocks are zero); no bias."""
+    random fraction `keep` (10 % by default; the PR 821 benchmark keeps 20 %)
+    of its bs x bs blocks (masked-out blocks are zero); no bias."""
     K, N = (1280, 5120) if layer == "fc1" else (5120, 1280)
     s = seed + (0 if layer == "fc1" else 100)
     crow, col = bsr_pattern(N // bs, K // bs, keep, s + 3)

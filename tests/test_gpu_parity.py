@@ -296,9 +296,12 @@ def _bsr_gpu(d):
     return wq, sc, crow, col, values
 
 
+@pytest.mark.parametrize("keep", [0.10, 0.20])
 @pytest.mark.parametrize("layer", ["fc1", "fc2"])
-def test_config_vit_h_bsr(layer):
-    d = synth.vit_h_bsr(0, layer)
+def test_config_vit_h_bsr(layer, keep):
+    """ViT-H MLP at batch 256 with 10 % (the spec workload) and 20 % (the
+    PR 821 benchmark command's sparsity 0.8) of the 64x64 weight blocks kept."""
+    d = synth.vit_h_bsr(0, layer, keep=keep)
     M, N, K = d["M"], d["N"], d["K"]
     wq, sc, crow, col, values = _bsr_gpu(d)
     wo, sco = oracle.quantize_rows_f32(d["w"])
@@ -326,10 +329,10 @@ def test_config_vit_h_bsr(layer):
     assert _frob(d["x"][rows], d["w"], got[rows]) <= 2e-2
 
 
-def _random_bsr(N, K, keep, seed, empty_rows=(), dup=False):
-    crow, col = synth.bsr_pattern(N // 64, K // 64, keep, seed)
+def _random_bsr(N, K, keep, seed, empty_rows=(), dup=False, bs=64):
+    crow, col = synth.bsr_pattern(N // bs, K // bs, keep, seed)
     counts = np.diff(crow)
-    cols = [list(col[crow[b]:crow[b + 1]]) for b in range(N // 64)]
+    cols = [list(col[crow[b]:crow[b + 1]]) for b in range(N // bs)]
     for b in empty_rows:
         cols[b] = []
     if dup and cols[0]:
@@ -337,32 +340,57 @@ def _random_bsr(N, K, keep, seed, empty_rows=(), dup=False):
     counts = [len(c) for c in cols]
     crow = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     col = np.array([c for cs in cols for c in cs], np.int32)
-    values = synth.uniform_int8((len(col), 64, 64), -127, 127, seed + 1)
+    values = synth.uniform_int8((len(col), bs, bs), -127, 127, seed + 1)
     return crow, col, values
 
 
+@pytest.mark.parametrize("bs", [64, 32, 16])
 @pytest.mark.parametrize("case", ["empty_rows", "no_blocks", "dense", "duplicates", "ragged_m", "many_blocks"])
-def test_bsr_edge_cases(case):
-    # many_blocks: 4480 blocks, more indices than the kernel stages in shared
-    # memory, so crow/col are read from global memory
+def test_bsr_edge_cases(case, bs):
+    # many_blocks: more indices than the kernel stages in shared memory, so
+    # crow/col are read from global memory; bs: 64x64, 32x32 or 16x16 blocks
     M, N, K = {"ragged_m": (1, 256, 192), "many_blocks": (130, 6400, 4096)}.get(case, (300, 320, 256))
+    if bs < 64 and case == "many_blocks":
+        M, N, K = 130, 1600, 1024
     keep = {"dense": 1.0, "no_blocks": 0.0, "many_blocks": 0.7}.get(case, 0.3)
-    crow, col, values = _random_bsr(N, K, keep, 500, empty_rows=(1, 3) if case == "empty_rows" else (),
-                                    dup=case == "duplicates")
+    crow, col, values = _random_bsr(N, K, keep, 500 + bs, empty_rows=(1, 3) if case == "empty_rows" else (),
+                                    dup=case == "duplicates", bs=bs)
     A = synth.uniform_int8((M, K), -127, 127, 501)
     s_row = synth.uniform_f32((M,), 0.001, 0.05, 505)
     s_col = synth.uniform_f32((N,), 0.001, 0.05, 506)
     bias = synth.normal_bf16((N,), 0.1, 502)
-    vd = to_dev(values) if len(col) else torch.empty((0, 64, 64), dtype=torch.int8, device="cuda")
+    vd = to_dev(values) if len(col) else torch.empty((0, bs, bs), dtype=torch.int8, device="cuda")
     cd = to_dev(col) if len(col) else torch.empty((0,), dtype=torch.int32, device="cuda")
     acc = dq.dq_bsr_int8_linear(to_dev(A), None, N, to_dev(crow), cd, vd, None, out_dtype="s32")
-    want = oracle.bsr_gemm_s32(A, N, crow, col, values)
+    want = oracle.bsr_gemm_s32(A, N, crow, col, values, bs)
     assert np.array_equal(acc.cpu().numpy(), want)
     out = dq.dq_bsr_int8_linear(to_dev(A), to_dev(s_row), N, to_dev(crow), cd, vd, to_dev(s_col),
                                 bias=to_dev_bf16(bias))
     assert_bf16_close(bf16_bits(out), oracle.epilogue_bf16(want, s_row, s_col, bias))
     if case == "duplicates":
-        assert dq.dq_bsr_validate(to_dev(crow), cd, N, K) == dq.DQ_OK
+        assert dq.dq_bsr_validate(to_dev(crow), cd, N, K, bs) == dq.DQ_OK
+
+
+@pytest.mark.parametrize("bs", [32, 16])
+def test_bsr_small_blocks_pack_and_match_dense(bs):
+    """Weight prep with bs x bs blocks (mask, per-channel quantize, pack on the
+    GPU) equals the oracle's, and the BSR product equals the dense product on
+    the densified weight, bit for bit."""
+    d = synth.vit_h_bsr(0, "fc1", M=777, keep=0.2, bs=bs)
+    M, N, K = d["M"], d["N"], d["K"]
+    wq, sc = dq.dq_quantize_weight(to_dev(d["w"]))
+    crow, col = to_dev(d["crow"]), to_dev(d["col"])
+    values = dq.dq_bsr_pack(wq, crow, col, block=bs)
+    wo, _ = oracle.quantize_rows_f32(d["w"])
+    assert np.array_equal(values.cpu().numpy(), oracle.bsr_pack(wo, d["crow"], d["col"], bs))
+    assert dq.dq_bsr_validate(crow, col, N, K, bs) == dq.DQ_OK
+    q, s = dq.dq_quantize_rows(to_dev_bf16(d["x"]))
+    out = dq.dq_bsr_int8_linear(q, s, N, crow, col, values, sc)
+    acc = dq.dq_bsr_int8_linear(q, s, N, crow, col, values, sc, out_dtype="s32")
+    want = oracle.bsr_gemm_s32(q.cpu().numpy(), N, d["crow"], d["col"], values.cpu().numpy(), bs)
+    assert np.array_equal(acc.cpu().numpy(), want)
+    dense = dq.dq_int8_linear(q, s, wq, sc)
+    assert torch.equal(dense.view(torch.int16), out.view(torch.int16))
 
 
 def test_bsr_validate_rejects_malformed():

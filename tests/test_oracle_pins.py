@@ -247,8 +247,9 @@ def _np_densify(N, K, crow, col, values, bs):
     return W
 
 
-def test_bsr_equals_dense_on_densified_weight():
-    bs, N, K, M = 64, 5 * 64, 4 * 64, 37
+@pytest.mark.parametrize("bs", [64, 32, 16])
+def test_bsr_equals_dense_on_densified_weight(bs):
+    N, K, M = 5 * bs, 4 * bs, 37
     crow, col = synth.bsr_pattern(N // bs, K // bs, 0.3, 61)
     crow[2:] = np.maximum(crow[2:], crow[2])       # keep it canonical
     assert crow[-1] == len(col)
