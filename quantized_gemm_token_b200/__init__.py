@@ -47,6 +47,7 @@ _PROTOS = {
     "dq_debug_set_schedule": (None, [_I32]),
     "dq_debug_set_tile_n": (None, [_I32]),
     "dq_debug_set_two_widths": (None, [_I32]),
+    "dq_debug_set_bsr_panel": (None, [_I32]),
     "dq_debug_set_quant_kernel": (None, [_I32]),
 }
 
@@ -158,6 +159,11 @@ def dq_debug_set_tile_n(n: int) -> None:
 def dq_debug_set_two_widths(on: int) -> None:
     """Measurement knob: 0 turns off the two-width (wave-balanced) dense schedule."""
     lib.dq_debug_set_two_widths(int(on))
+
+
+def dq_debug_set_bsr_panel(mode: int) -> None:
+    """Measurement knob, BSR panel variant (K <= 1280): 0 never, 1 automatic, 2 always."""
+    lib.dq_debug_set_bsr_panel(int(mode))
 
 
 def dq_debug_set_quant_kernel(mode: int) -> None:

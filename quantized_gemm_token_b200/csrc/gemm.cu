@@ -38,7 +38,7 @@
 
 namespace dq {
 
-template <Kind KIND, int BN>
+template <Kind KIND, int BN, bool PANEL = false>
 struct Cfg {
   static constexpr int BM = 128;
   static constexpr bool BSR = is_bsr(KIND);
@@ -48,7 +48,13 @@ struct Cfg {
   // uses the 32-byte A slice that contains it, the other half of the MMA's K
   // multiplying zeros, see the Bsr16 B descriptor).
   static constexpr int KB = !BSR ? 128 : BS == 64 ? 64 : 32;
-  static constexpr int A_BYTES = BM * KB;
+  // BSR panel variant: the 128 x K activation panel of the current 128-row
+  // block stays in shared memory (K <= KP, chunks of 128 x 128 bytes with the
+  // 128-byte swizzle) and the stages carry weight blocks only.
+  static constexpr int KP = PANEL ? 1280 : 0;
+  static constexpr int PANEL_CHUNKS = KP / 128;
+  static constexpr int PANEL_BYTES = PANEL_CHUNKS * BM * 128;
+  static constexpr int A_BYTES = PANEL ? 0 : BM * KB;         // per stage
   // BSR: a tile spans BN/BS block rows; each stage holds one BS x BS block
   // that accumulates into its block row's BS-column slice of the tile.
   static constexpr int B_ROWS = BSR ? BS : BN;
@@ -66,22 +72,30 @@ struct Cfg {
   static constexpr int OUT_BYTES = STAGED_OUT ? EPI_WARPS * OUT_BUF_BYTES : 0;
   // BSR: crow and col are copied to shared memory when nbr + 1 + nnzb fits
   // (every tile and every block needs them; a global load per block would put
-  // a dependent L2 round trip in front of each TMA issue).
-  static constexpr int IDX_INTS = BSR ? 4096 : 0;
+  // a dependent L2 round trip in front of each TMA issue).  The panel variant
+  // has no room for them and reads them through L1.
+  static constexpr int IDX_INTS = BSR && !PANEL ? 4096 : 0;
   static constexpr int IDX_BYTES = IDX_INTS * 4;
   // 16x16 blocks: two 256-byte zero regions, one below and one above the
   // stage buffers, that stand in for the half of the MMA's K the block does
   // not cover (the descriptor's leading-dimension offset must be positive).
   static constexpr int ZERO_BYTES = KIND == Kind::Bsr16 ? 1024 : 0;
-  static constexpr int STAGE_CAP = BSR && BS < 64 ? 24 : 12;
-  static constexpr int STAGES_RAW = (224 * 1024 - OUT_BYTES - IDX_BYTES - 2 * ZERO_BYTES) / STAGE_BYTES;
+  // Panel variant: a zero weight block, used in place of a block whose
+  // column lies outside the matrix (it contributes zeros, as a load from
+  // outside the matrix does in the streaming variant).
+  static constexpr int ZB_BYTES = PANEL ? (B_BYTES > 256 ? B_BYTES : 256) : 0;
+  static constexpr int STAGE_CAP = BSR && (BS < 64 || PANEL) ? 24 : 12;
+  static constexpr int STAGES_RAW =
+      (224 * 1024 - OUT_BYTES - IDX_BYTES - 2 * ZERO_BYTES - PANEL_BYTES - ZB_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > STAGE_CAP ? STAGE_CAP : STAGES_RAW;
   // shared-memory layout (offsets from the 1024-aligned base)
   static constexpr int OFF_ZLO = 0;
-  static constexpr int OFF_A = ZERO_BYTES;
+  static constexpr int OFF_PANEL = ZERO_BYTES;
+  static constexpr int OFF_A = OFF_PANEL + PANEL_BYTES;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_ZHI = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_OUT = (OFF_ZHI + ZERO_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_ZB = (OFF_ZHI + ZERO_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_OUT = (OFF_ZB + ZB_BYTES + 1023) / 1024 * 1024;
   static constexpr int OFF_IDX = OFF_OUT + OUT_BYTES;
   static constexpr int OFF_BARS = OFF_IDX + IDX_BYTES;
   static constexpr int ACC_RAW = 512 / BN;
@@ -91,12 +105,13 @@ struct Cfg {
                                    : ACC_COLS <= 256 ? 256 : 512;
   static constexpr int K_STEPS = KB / 32;                     // MMA K = 32 bytes
   static constexpr int CW = BN >= 32 ? 32 : 16;               // epilogue chunk (columns)
-  static constexpr int SMEM_BYTES = OFF_BARS + 512 /*barriers*/ + 1024 /*align*/;
+  static constexpr int SMEM_BYTES = OFF_BARS + 1024 /*barriers, stage columns*/ + 1024 /*align*/;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(STAGES >= 2, "stages");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(!BSR || BN % (BSR ? BS : 1) == 0, "tile covers whole block rows");
+  static_assert(!PANEL || BSR, "the panel variant is for BSR weights");
 };
 
 // Where a tile lies: 128-row block ta, B-slot tile tb, first output column n0
@@ -140,12 +155,12 @@ __device__ __noinline__ void store_row_chunk_tma_cold(const GemmArgs& g, const C
   store_row_chunk_tma(g, tm_c, buf, lane, m0, n0, r, srow, cs);
 }
 
-template <Kind KIND, int BN>
-__global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
+template <Kind KIND, int BN, bool PANEL>
+__global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_c,
                 const __grid_constant__ GemmArgs g) {
-  using C = Cfg<KIND, BN>;
+  using C = Cfg<KIND, BN, PANEL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -159,9 +174,14 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
   uint64_t* accf_bar = bars + 2 * C::STAGES;
   uint64_t* acce_bar = accf_bar + C::ACC_BUFS;
   uint64_t* drain_bar = acce_bar + C::ACC_BUFS;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* panel_full = drain_bar + 1;       // panel variant: activation panel landed
+  uint64_t* panel_empty = panel_full + 1;     // panel variant: MMAs on the old panel done
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(panel_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* sk_last = const_cast<int*>(abort_flag + 1);
+  // panel variant: each stage's block column, written by the producer before
+  // it arms the stage's barrier (the MMA thread reads it after the wait)
+  int* stage_col = sk_last + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -177,6 +197,8 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       mbar_init(smem_u32(acce_bar + a), 32 * C::EPI_WARPS);
     }
     mbar_init(smem_u32(drain_bar), 1);
+    mbar_init(smem_u32(panel_full), 1);
+    mbar_init(smem_u32(panel_empty), 1);
     fence_barrier_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
@@ -192,16 +214,19 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
   // previous kernel of the stream before any global memory access.
   griddep_wait();
   const int* idx = nullptr;      // BSR: crow at idx[0..nbr], col at idx[nbr+1..]
-  if constexpr (KIND == Kind::Bsr16) {
-    // the zero regions the 16x16-block B descriptors point at, visible to
-    // the tensor core (async proxy) before the first MMA
+  if constexpr (KIND == Kind::Bsr16 || PANEL) {
+    // the zero regions the 16x16-block B descriptors and the panel variant's
+    // out-of-matrix blocks point at, visible to the tensor core (async proxy)
+    // before the first MMA
     for (int i = threadIdx.x; i < C::ZERO_BYTES / 16; i += blockDim.x) {
       reinterpret_cast<uint4*>(smem + C::OFF_ZLO)[i] = make_uint4(0u, 0u, 0u, 0u);
       reinterpret_cast<uint4*>(smem + C::OFF_ZHI)[i] = make_uint4(0u, 0u, 0u, 0u);
     }
+    for (int i = threadIdx.x; i < C::ZB_BYTES / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(smem + C::OFF_ZB)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
-  if constexpr (C::BSR) {
+  if constexpr (C::BSR && !PANEL) {
     if (g.idx_smem) {
       const int nbr = g.nbr;
       for (int i = threadIdx.x; i <= nbr; i += blockDim.x) sIdx[i] = __ldg(g.crow + i);
@@ -223,10 +248,32 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
+      int loaded_ta = -1;           // panel variant: block row whose panel is loaded
+      int panel_loads = 0;
+      const int panel_chunks = (g.K + 127) / 128;
       while (ok && iter.next(s)) {
         const TileGeom geo = tile_geom<KIND, BN>(g, s.tile);
         const int ta = geo.ta, tb = geo.tb;
         const uint32_t stage_tx = C::A_BYTES + (KIND == Kind::Dense ? geo.width * C::KB : C::B_BYTES);
+        if constexpr (PANEL) {
+          if (ta != loaded_ta) {
+            // a new 128-row block: once the MMAs on the previous panel are
+            // done, bring its 128 x K activations in (one box per 128 k bytes)
+            if (panel_loads > 0) {
+              if (!mbar_wait(smem_u32(panel_empty), static_cast<uint32_t>(panel_loads - 1) & 1u, g.wait,
+                             abort_flag)) {
+                ok = false;
+                break;
+              }
+            }
+            const uint32_t pf = smem_u32(panel_full);
+            mbar_arrive_expect_tx(pf, static_cast<uint32_t>(panel_chunks) * (C::BM * 128));
+            for (int ch = 0; ch < panel_chunks; ++ch)
+              tma_load_2d(smem_u32(smem + C::OFF_PANEL + ch * (C::BM * 128)), &tm_a, pf, ch * 128, ta * 128);
+            ++panel_loads;
+            loaded_ta = ta;
+          }
+        }
         for (int j = 0; ok && j < C::NSUB; ++j) {
         int k0 = s.kb0, k1 = s.kb1;
         if constexpr (C::BSR) {
@@ -234,16 +281,23 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
           if (br >= g.nbr) break;
           bsr_range(g, idx, br, k0, k1);
         }
+        int c_next = (PANEL && k0 < k1) ? __ldg(g.col + k0) : 0;
         for (int kb = k0; kb < k1; ++kb) {
+          const int c_cur = c_next;
+          if (PANEL && kb + 1 < k1) c_next = __ldg(g.col + kb + 1);     // one block ahead
           if (!mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, g.wait, abort_flag)) {
             ok = false;
             break;
           }
           const uint32_t fb = smem_u32(full_bar + stage);
+          if constexpr (PANEL) stage_col[stage] = c_cur;
           mbar_arrive_expect_tx(fb, stage_tx);
           const uint32_t da = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t db = smem_u32(sB + stage * C::B_BYTES);
-          if constexpr (C::BSR) {
+          if constexpr (PANEL) {
+            tma_load_2d(db, &tm_b, fb, 0, kb * C::BS);        // the block only; A is the panel
+            (void)da;
+          } else if constexpr (C::BSR) {
             // A: the KB-wide k slice holding block column c (for 16-wide
             // blocks the 32-byte slice that contains it); B: block kb
             const int c = idx ? idx[g.nbr + 1 + kb] : __ldg(g.col + kb);
@@ -275,6 +329,8 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
           }
           mbar_wait(smem_u32(full_bar + stage), phase, quick, &never);
         }
+        if (PANEL && panel_loads > 0)
+          mbar_wait(smem_u32(panel_full), static_cast<uint32_t>(panel_loads - 1) & 1u, quick, &never);
       }
     }
   } else if (warp == 1) {
@@ -286,11 +342,24 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
+      int cur_ta = -1;               // panel variant: block row of the panel in use
+      int panels = 0;
       while (ok && iter.next(s)) {
         if (!mbar_wait(smem_u32(acce_bar + acc), acc_phase ^ 1, g.wait, abort_flag)) break;
         tc_fence_after();
         const uint32_t idesc = (KIND == Kind::Dense && g.bn2 > 0 && s.tile >= g.t1)
                                    ? idesc_i8(128, g.bn2) : idesc_full;
+        if constexpr (PANEL) {
+          const int ta = s.tile / g.b_tiles;
+          if (ta != cur_ta) {
+            // hand the old panel back (once its MMAs are done), wait for the new one
+            if (panels > 0) mma_commit(smem_u32(panel_empty));
+            if (!mbar_wait(smem_u32(panel_full), static_cast<uint32_t>(panels) & 1u, g.wait, abort_flag)) break;
+            tc_fence_after();
+            ++panels;
+            cur_ta = ta;
+          }
+        }
         for (int j = 0; ok && j < C::NSUB; ++j) {
         int k0 = s.kb0, k1 = s.kb1;
         if constexpr (C::BSR) {
@@ -306,9 +375,27 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t ad = smem_desc_kmajor<C::KB>(smem_u32(sA + stage * C::A_BYTES));
-          uint64_t bd;
-          if constexpr (KIND == Kind::Bsr16) {
+          uint64_t ad, bd;
+          if constexpr (PANEL) {
+            // A: the block column's k slice inside the resident panel (a start
+            // address 32 / 64 / 96 bytes into a 128-byte swizzled row, as the
+            // k steps of the dense kernel); a column outside [0, K / BS)
+            // multiplies the zero block instead
+            const int c = stage_col[stage];
+            const bool valid = c >= 0 && c < g.K / C::BS;
+            const int kbyte = !valid ? 0 : KIND == Kind::Bsr16 ? (c >> 1) * 32 : c * C::BS;
+            ad = smem_desc_kmajor<128>(smem_u32(smem + C::OFF_PANEL + (kbyte >> 7) * (C::BM * 128))) +
+                 static_cast<uint64_t>((kbyte & 127) >> 4);
+            // (a 16-wide zero block is the low zero region itself, so that the
+            // padded descriptor's offset stays positive)
+            const uint32_t blk = valid ? smem_u32(sB + stage * C::B_BYTES)
+                                       : smem_u32(smem + (KIND == Kind::Bsr16 ? C::OFF_ZLO : C::OFF_ZB));
+            if constexpr (KIND == Kind::Bsr16)
+              bd = smem_desc_b16_padded(blk, smem_u32(smem + C::OFF_ZLO), smem_u32(smem + C::OFF_ZHI), c & 1);
+            else
+              bd = smem_desc_kmajor<C::KB>(blk);
+          } else if constexpr (KIND == Kind::Bsr16) {
+            ad = smem_desc_kmajor<C::KB>(smem_u32(sA + stage * C::A_BYTES));
             // 16 channels x 16 k of the block, rows of 16 bytes (no swizzle):
             // the MMA's other 16 k bytes read a zero region, so the 32-byte A
             // slice's other half contributes nothing.
@@ -316,6 +403,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN>::THREADS, 1)
             bd = smem_desc_b16_padded(smem_u32(sB + stage * C::B_BYTES), smem_u32(smem + C::OFF_ZLO),
                                       smem_u32(smem + C::OFF_ZHI), c & 1);
           } else {
+            ad = smem_desc_kmajor<C::KB>(smem_u32(sA + stage * C::A_BYTES));
             bd = smem_desc_kmajor<C::KB>(smem_u32(sB + stage * C::B_BYTES));
           }
 #pragma unroll
@@ -535,14 +623,14 @@ __global__ void __launch_bounds__(256) bsr_pack_kernel(const int8_t* __restrict_
 
 namespace {
 
-template <Kind KIND, int BN>
+template <Kind KIND, int BN, bool PANEL = false>
 dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2, const CUtensorMap& tc,
                  const GemmArgs& args, int grid, cudaStream_t stream) {
-  using C = Cfg<KIND, BN>;
+  using C = Cfg<KIND, BN, PANEL>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, PANEL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err);
@@ -559,7 +647,7 @@ dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN>, ta, tb, tb2, tc, args);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, PANEL>, ta, tb, tb2, tc, args);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 
@@ -577,6 +665,9 @@ int g_schedule_override = 0;
 int g_tile_n_override = 0;
 // Measurement knob: 0 turns the two-width Dense schedule off.
 int g_two_widths = 1;
+// Measurement knob: BSR panel variant 0 = never, 1 = automatic (K <= 1280 and
+// blocks smaller than 64), 2 = whenever K <= 1280.
+int g_bsr_panel = 1;
 
 struct Plan {
   Kind kind;
@@ -682,6 +773,7 @@ size_t dq_int8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
 void dq_debug_set_schedule(int mode) { g_schedule_override = mode; }
 void dq_debug_set_tile_n(int n) { g_tile_n_override = n; }
 void dq_debug_set_two_widths(int on) { g_two_widths = on; }
+void dq_debug_set_bsr_panel(int mode) { g_bsr_panel = mode; }
 
 dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K, const int8_t* W,
                          const float* s_col, int64_t N, const void* bias_bf16, void* out,
@@ -829,11 +921,21 @@ dq_status dq_bsr_int8_linear_blocked(const int8_t* A, const float* s_row, int64_
   if (st != DQ_OK) return st;
   if (M == 0) return DQ_OK;
 
-  // A: k slices of 64 bytes (64-wide blocks) or 32 bytes (32- and 16-wide
-  // blocks) x 128 rows, swizzled to the slice width.  B: the blocks viewed as
-  // a [nnzb * block, block] byte matrix, one block per box; 16-byte rows of
-  // 16-wide blocks are not swizzled.
-  const int kb = block == 64 ? 64 : 32;
+  // Panel variant (K <= 1280): each CTA keeps its 128 x K activation panel in
+  // shared memory across consecutive tiles of the same 128-row block (A read
+  // from L2 once per block row of tiles instead of once per weight block), so
+  // A is described in 128 x 128-byte boxes with the 128-byte swizzle.
+  // Streaming variant: A in k slices of 64 bytes (64-wide blocks) or 32 bytes
+  // (32- and 16-wide blocks) x 128 rows, swizzled to the slice width.  B: the
+  // blocks viewed as a [nnzb * block, block] byte matrix, one block per box;
+  // 16-byte rows of 16-wide blocks are not swizzled.
+  // Measured on B200 (ViT-H fc1, M=65792, K=1280): 32x32 blocks 627 us with
+  // the panel vs 725 streaming, 16x16 2143 vs 2514; 64x64 blocks are as fast
+  // or faster streaming (10 %: 266 vs 269 us, 20 %: 384 vs 396), where the
+  // per-block MMA issue, not the activation traffic, bounds the kernel.
+  const bool panel = K <= Cfg<Kind::Bsr, 256, true>::KP &&
+                     (g_bsr_panel == 2 || (g_bsr_panel == 1 && block < 64));
+  const int kb = panel ? 128 : block == 64 ? 64 : 32;
   const int bsw = block == 16 ? 0 : static_cast<int>(block);
   const uint32_t ub = static_cast<uint32_t>(block);
   CUtensorMap ta, tb;
@@ -866,9 +968,15 @@ dq_status dq_bsr_int8_linear_blocked(const int8_t* A, const float* s_row, int64_
   g.crow = crow;
   g.col = col;
   g.nnzb = static_cast<int>(nnzb);
-  g.idx_smem = (N / block + 1 + nnzb) <= Cfg<Kind::Bsr, 256>::IDX_INTS ? 1 : 0;
+  g.idx_smem = !panel && (N / block + 1 + nnzb) <= Cfg<Kind::Bsr, 256>::IDX_INTS ? 1 : 0;
+  g.blocked = panel ? 1 : 0;
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
   const int grid = g.num_tiles < d->sm_count ? g.num_tiles : d->sm_count;
+  if (panel) {
+    if (block == 32) return launch<Kind::Bsr32, 256, true>(ta, tb, tb, tc, g, grid, stream);
+    if (block == 16) return launch<Kind::Bsr16, 256, true>(ta, tb, tb, tc, g, grid, stream);
+    return launch<Kind::Bsr, 256, true>(ta, tb, tb, tc, g, grid, stream);
+  }
   if (block == 32) return launch<Kind::Bsr32, 256>(ta, tb, tb, tc, g, grid, stream);
   if (block == 16) return launch<Kind::Bsr16, 256>(ta, tb, tb, tc, g, grid, stream);
   return launch<Kind::Bsr, 256>(ta, tb, tb, tc, g, grid, stream);

@@ -42,6 +42,10 @@ struct GemmArgs {
   // cover the rest of the matrix: first_cnt tiles in 128-row block mb0 from
   // column c_start on, then per_row tiles in each later block row.
   int t1, bn2, mb0, c_start, first_cnt, per_row;
+  // Each CTA takes a contiguous range of tiles (row-major tile order) instead
+  // of every gridDim.x-th one: consecutive tiles then share their 128-row
+  // block (the BSR panel kernel keeps that block's activations resident).
+  int blocked;
   WaitCtl wait;
 };
 
@@ -56,14 +60,21 @@ struct Seg {
 struct SegIter {
   const GemmArgs* g;
   long long it, it_end;   // stream-K
-  int next_tile;          // round-robin
+  int next_tile;          // round-robin, or the next tile of a contiguous range
+  int end_tile;           // contiguous range (g.blocked): one past the CTA's last tile
   __device__ SegIter(const GemmArgs& args) : g(&args) {
     const long long G = gridDim.x, c = blockIdx.x;
     if (args.stream_k) {
       it = c * args.iters_total / G;
       it_end = (c + 1) * args.iters_total / G;
     }
-    next_tile = blockIdx.x;
+    if (args.blocked) {
+      next_tile = static_cast<int>(c * args.num_tiles / G);
+      end_tile = static_cast<int>((c + 1) * args.num_tiles / G);
+    } else {
+      next_tile = blockIdx.x;
+      end_tile = args.num_tiles;
+    }
   }
   __device__ bool next(Seg& s) {
     if (g->stream_k) {
@@ -75,9 +86,9 @@ struct SegIter {
       it += s.kb1 - s.kb0;
       return true;
     }
-    if (next_tile >= g->num_tiles) return false;
+    if (next_tile >= end_tile) return false;
     s.tile = next_tile;
-    next_tile += gridDim.x;
+    next_tile += g->blocked ? 1 : static_cast<int>(gridDim.x);
     s.kb0 = 0;
     s.kb1 = g->kb_total;
     return true;

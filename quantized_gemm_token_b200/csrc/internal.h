@@ -56,6 +56,9 @@ extern "C" DQ_API void dq_debug_set_schedule(int mode);
 extern "C" DQ_API void dq_debug_set_tile_n(int n);
 // Measurement knob: 0 turns off the two-width (wave-balanced) dense schedule.
 extern "C" DQ_API void dq_debug_set_two_widths(int on);
+// Measurement knob: BSR panel variant (activation panel kept in shared memory,
+// K <= 1280): 0 = never, 1 = automatic (blocks smaller than 64), 2 = always.
+extern "C" DQ_API void dq_debug_set_bsr_panel(int mode);
 // Measurement knob: quantize kernel (0 = automatic, 1 = register-resident,
 // 2 = row-pipelined through shared memory).
 extern "C" DQ_API void dq_debug_set_quant_kernel(int mode);

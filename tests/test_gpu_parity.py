@@ -371,6 +371,33 @@ def test_bsr_edge_cases(case, bs):
         assert dq.dq_bsr_validate(to_dev(crow), cd, N, K, bs) == dq.DQ_OK
 
 
+@pytest.mark.parametrize("bs", [64, 32, 16])
+@pytest.mark.parametrize("M,N,K", [(700, 512, 1216), (300, 768, 1280), (129, 256, 128)])
+def test_bsr_panel_and_streaming_variants_agree(M, N, K, bs):
+    """For K <= 1280 the BSR kernel keeps each 128-row activation panel in
+    shared memory; the streaming variant re-loads a k slice per block.  Both
+    match the oracle bit for bit (K = 1216 leaves a partial last 128-byte
+    panel chunk; an empty block row exercises the zero slices)."""
+    crow, col, values = _random_bsr(N, K, 0.3, 900 + bs + K, empty_rows=(0,), bs=bs)
+    A = synth.uniform_int8((M, K), -127, 127, 901)
+    s_row = synth.uniform_f32((M,), 0.001, 0.05, 902)
+    s_col = synth.uniform_f32((N,), 0.001, 0.05, 903)
+    Ad, cd, vd, crd = to_dev(A), to_dev(col), to_dev(values), to_dev(crow)
+    outs = {}
+    try:
+        for panel in (1, 0):
+            dq.dq_debug_set_bsr_panel(2 if panel else 0)
+            outs[panel] = (dq.dq_bsr_int8_linear(Ad, None, N, crd, cd, vd, None, out_dtype="s32"),
+                           dq.dq_bsr_int8_linear(Ad, to_dev(s_row), N, crd, cd, vd, to_dev(s_col)))
+    finally:
+        dq.dq_debug_set_bsr_panel(1)
+    want = oracle.bsr_gemm_s32(A, N, crow, col, values, bs)
+    assert np.array_equal(outs[1][0].cpu().numpy(), want)
+    assert torch.equal(outs[1][0], outs[0][0])
+    assert torch.equal(outs[1][1].view(torch.int16), outs[0][1].view(torch.int16))
+    assert_bf16_close(bf16_bits(outs[1][1]), oracle.epilogue_bf16(want, s_row, s_col))
+
+
 @pytest.mark.parametrize("bs", [32, 16])
 def test_bsr_small_blocks_pack_and_match_dense(bs):
     """Weight prep with bs x bs blocks (mask, per-channel quantize, pack on the
