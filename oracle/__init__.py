@@ -9,7 +9,8 @@ The arithmetic lives in ``dq_oracle.c`` (plain single-threaded C); this
 module only marshals numpy arrays.  bf16 tensors are carried as their uint16
 bit patterns.
 
-What each routine follows (page titles and parts):
+What each routine follows (page titles and parts; the FP8 routines follow the
+vLLM csrc/quantization commits: dynamic scales, clamp to the e4m3 range):
   * quantize_rows_bf16 / quantize_rows_f32 -- per-token (per-row) absmax int8
     dynamic quantization: "int8 dynamic quant + bsr support" (pytorch/ao PR
     821, description); absmax/127 symmetric scale: "sparse_fc supported"
@@ -54,6 +55,15 @@ def _load():
         lib.oracle_float_to_bf16.restype = ctypes.c_uint16
         lib.oracle_bf16_to_float.argtypes = [ctypes.c_uint16]
         lib.oracle_bf16_to_float.restype = ctypes.c_float
+        lib.oracle_quantize_rows_bf16_fp8.argtypes = [P, I, I, I, P, I, P]
+        lib.oracle_quantize_rows_bf16_fp8.restype = ctypes.c_int
+        lib.oracle_quantize_rows_f32_fp8.argtypes = [P, I, I, I, P, I, P]
+        lib.oracle_quantize_rows_f32_fp8.restype = ctypes.c_int
+        lib.oracle_gemm_fp8_f64.argtypes = [P, I, I, I, P, I, I, P]
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_double.restype = ctypes.c_double
+        lib.oracle_float_to_e4m3.argtypes = [ctypes.c_float]
+        lib.oracle_float_to_e4m3.restype = ctypes.c_uint8
         _lib = lib
     return _lib
 
@@ -175,3 +185,53 @@ def float_to_bf16(f: float) -> int:
 
 def bf16_to_float(h: int) -> float:
     return float(_load().oracle_bf16_to_float(int(h)))
+
+
+# ---------------------------------------------------------------- FP8 (e4m3)
+
+def e4m3_to_float64(codes) -> np.ndarray:
+    """e4m3 codes (uint8, any shape) -> their values (float64; NaN codes -> NaN)."""
+    lib = _load()
+    table = np.array([lib.oracle_e4m3_to_double(c) for c in range(256)], np.float64)
+    return table[np.asarray(codes, np.uint8)]
+
+
+def float_to_e4m3(x) -> np.ndarray:
+    """finite fp32 values -> e4m3 codes (round to nearest even, magnitudes >= 448 -> 448)."""
+    lib = _load()
+    x = np.asarray(x, np.float32)
+    return np.array([lib.oracle_float_to_e4m3(float(v)) for v in x.ravel()], np.uint8).reshape(x.shape)
+
+
+def quantize_rows_bf16_fp8(x_bits: np.ndarray):
+    """x_bits: uint16 [M, K] (bf16) -> (q e4m3 codes uint8 [M, K], scales fp32 [M]);
+    s = fp32(max(absmax, 1e-8) / 448), q = e4m3(clamp(fp32(x / s), -448, 448))."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), np.uint8)
+    s = np.empty((M,), np.float32)
+    if _load().oracle_quantize_rows_bf16_fp8(_ptr(x), M, K, K, _ptr(q), K, _ptr(s)) != 0:
+        raise MemoryError("oracle row buffer")
+    return q, s
+
+
+def quantize_rows_f32_fp8(w: np.ndarray):
+    """w: fp32 [N, K] -> (q e4m3 codes uint8 [N, K], per-row scales fp32 [N])."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    q = np.empty((N, K), np.uint8)
+    s = np.empty((N,), np.float32)
+    _load().oracle_quantize_rows_f32_fp8(_ptr(w), N, K, K, _ptr(q), K, _ptr(s))
+    return q, s
+
+
+def gemm_fp8_f64(A: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """A e4m3 [M, K], W e4m3 [N, K] (uint8 codes) -> float64 [M, N] = the exact A @ W^T."""
+    A = _c(A, np.uint8)
+    W = _c(W, np.uint8)
+    M, K = A.shape
+    N = W.shape[0]
+    assert W.shape[1] == K
+    out = np.empty((M, N), np.float64)
+    _load().oracle_gemm_fp8_f64(_ptr(A), M, K, K, _ptr(W), N, K, _ptr(out))
+    return out

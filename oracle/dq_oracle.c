@@ -40,6 +40,7 @@
 #include <fenv.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 /* bf16 is carried as its 16-bit pattern: the top half of an IEEE fp32. */
@@ -211,4 +212,99 @@ void oracle_bsr_densify(int64_t N, int64_t K, const int32_t* crow, const int32_t
             for (int64_t j = 0; j < bs; ++j)
                 for (int64_t t = 0; t < bs; ++t)
                     W[(b * bs + j) * K + col[p] * bs + t] += values[(p * bs + j) * bs + t];
+}
+
+/* ---- dynamic FP8 (e4m3) per-token quantization and product ------------- */
+/*
+ * The sibling precision of the vLLM quantization commits (csrc/quantization
+ * history: a vectorised FP8 quantize kernel; dynamic activation scales; the
+ * scaled activations clamped to +-(largest e4m3 value) so that no NaN
+ * appears), taken per token like the int8 path:
+ *     s = fp32( max(absmax, 1e-8f) / 448 ),
+ *     q = e4m3( clamp( fp32(x / s), -448, 448 ) ),
+ * the conversion rounding to nearest, ties to even mantissa.  e4m3 ("fn"
+ * variant): 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; normal
+ * values (1 + m/8) * 2^(e-7) for e = 1..15 except e = 15, m = 7 (NaN), so the
+ * largest is 448 = 1.75 * 2^8; subnormals (m/8) * 2^-6; no infinities.
+ */
+
+/* e4m3 code -> its value (exact in double). NaN codes give NaN. */
+double oracle_e4m3_to_double(uint8_t c) {
+    const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* finite fp32 -> e4m3, round to nearest, ties to even mantissa; magnitudes
+ * at or above 448 give 448 (the clamp). */
+uint8_t oracle_float_to_e4m3(float f) {
+    const uint8_t sign = signbit(f) ? 0x80 : 0x00;
+    const double a = fabs((double)f);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {                       /* subnormal range: steps of 2^-9 */
+        const double q = nearbyint(ldexp(a, 9));    /* 0 .. 8; 8 is the smallest normal */
+        return sign | (uint8_t)q;
+    }
+    int e;
+    (void)frexp(a, &e);                             /* a = fr * 2^e, fr in [0.5, 1) */
+    int ex = e - 1;                                 /* a = (1 + f) * 2^ex, ex in -6 .. 8 */
+    double mq = nearbyint((ldexp(a, -ex) - 1.0) * 8.0);   /* 0 .. 8, ties to even */
+    if (mq == 8.0) { mq = 0.0; ex += 1; }
+    int code = ((ex + 7) << 3) | (int)mq;
+    if (code > 0x7E) code = 0x7E;
+    return sign | (uint8_t)code;
+}
+
+static float quantize_one_row_fp8(const float* vals, int64_t K, uint8_t* q) {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        const float a = fabsf(vals[k]);
+        if (a > amax) amax = a;
+    }
+    const float s = fmaxf(amax, 1e-8f) / 448.0f;   /* one IEEE division */
+    for (int64_t k = 0; k < K; ++k) {
+        float v = vals[k] / s;                       /* one IEEE division */
+        if (v > 448.0f) v = 448.0f;
+        if (v < -448.0f) v = -448.0f;
+        q[k] = oracle_float_to_e4m3(v);
+    }
+    return s;
+}
+
+int oracle_quantize_rows_bf16_fp8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                  uint8_t* q, int64_t ldq, float* scales) {
+    fesetround(FE_TONEAREST);
+    float* row = (float*)malloc((size_t)K * sizeof(float));
+    if (!row) return -1;
+    for (int64_t i = 0; i < M; ++i) {
+        for (int64_t k = 0; k < K; ++k) row[k] = bf16_bits_to_float(x[i * ldx + k]);
+        scales[i] = quantize_one_row_fp8(row, K, q + i * ldq);
+    }
+    free(row);
+    return 0;
+}
+
+int oracle_quantize_rows_f32_fp8(const float* w, int64_t N, int64_t K, int64_t ldw,
+                                 uint8_t* q, int64_t ldq, float* scales) {
+    fesetround(FE_TONEAREST);
+    for (int64_t n = 0; n < N; ++n) scales[n] = quantize_one_row_fp8(w + n * ldw, K, q + n * ldq);
+    return 0;
+}
+
+/* acc[m,n] = sum_k e4m3(A[m,k]) * e4m3(W[n,k]) in double.  Every product has
+ * at most 8 significant bits and |products| lie in [2^-18, 2^17]; K <= 2^20
+ * terms keep every partial sum within 53 bits, so the double sum is exact. */
+void oracle_gemm_fp8_f64(const uint8_t* A, int64_t M, int64_t K, int64_t lda,
+                         const uint8_t* W, int64_t N, int64_t ldw, double* acc) {
+    double lut[256];
+    for (int c = 0; c < 256; ++c) lut[c] = oracle_e4m3_to_double((uint8_t)c);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double s = 0.0;
+            for (int64_t k = 0; k < K; ++k) s += lut[A[m * lda + k]] * lut[W[n * ldw + k]];
+            acc[m * N + n] = s;
+        }
 }

@@ -316,3 +316,93 @@ def test_frobenius_llm_outliers_reported_not_gated():
     wq2, sc2 = oracle.quantize_rows_f32(d2["w"])
     out2, _, _ = oracle.dynamic_linear_bf16(d2["x"], wq2, sc2)
     assert _rel_frob(d2["x"], d2["w"], out2) <= 2e-2
+
+
+# ---------------------------------------------------------------- FP8 (e4m3)
+# The sibling precision of the vLLM csrc/quantization commits (dynamic scales,
+# scaled values clamped to the e4m3 range): s = fp32(max(absmax, 1e-8)/448),
+# q = e4m3(clamp(fp32(x/s), -448, 448)), round to nearest even.
+
+def _e4m3_values_from_definition():
+    """All 256 codes decoded from the format's definition (1-4-3, bias 7,
+    e = 15 & m = 7 is NaN, exponent 0 subnormal), written independently."""
+    vals = []
+    for c in range(256):
+        sgn = -1.0 if c & 0x80 else 1.0
+        e, m = (c >> 3) & 15, c & 7
+        if e == 15 and m == 7:
+            vals.append(np.nan)
+        elif e == 0:
+            vals.append(sgn * m * 2.0 ** -9)
+        else:
+            vals.append(sgn * (8 + m) * 2.0 ** (e - 10))
+    return np.array(vals)
+
+
+def test_e4m3_decode_table():
+    got = oracle.e4m3_to_float64(np.arange(256))
+    want = _e4m3_values_from_definition()
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x38] == 1.0
+    pos = got[:0x7F]
+    assert np.all(np.diff(pos) > 0)            # codes 0 .. 0x7E increase
+
+
+def test_e4m3_rounding_is_nearest_even_by_brute_force():
+    table = _e4m3_values_from_definition()[:0x7F]          # non-negative finite values
+    rng = np.random.default_rng(5)
+    mids = (table[1:] + table[:-1]) / 2                    # every tie
+    xs = np.concatenate([rng.uniform(0, 460, 3000), rng.uniform(0, 0.03, 3000), table, mids,
+                         np.nextafter(mids.astype(np.float32), np.float32(0)),
+                         np.nextafter(mids.astype(np.float32), np.float32(1e9))]).astype(np.float32)
+    got = oracle.float_to_e4m3(xs)
+    for x, c in zip(xs.astype(np.float64), got):
+        if x >= 448.0:
+            assert c == 0x7E
+            continue
+        d = np.abs(table - x)
+        best = np.flatnonzero(d == d.min())
+        want = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        assert c == want, (x, c, want)
+    assert np.array_equal(oracle.float_to_e4m3(-xs[:500]), got[:500] | 0x80)
+
+
+def test_fp8_quantize_matches_definition_and_invariants():
+    x = synth.normal_bf16((33, 300), 1.0, 77)
+    x[0] = 0
+    q, s = oracle.quantize_rows_bf16_fp8(x)
+    xf = synth.bf16_bits_to_f32(x) if hasattr(synth, "bf16_bits_to_f32") else \
+        (x.astype(np.uint32) << 16).view(np.float32)
+    a = np.abs(xf).max(axis=1)
+    s_want = (np.maximum(a, np.float32(1e-8)) / np.float32(448)).astype(np.float32)
+    assert np.array_equal(s.view(np.uint32), s_want.view(np.uint32))
+    ratio = np.clip((xf / s_want[:, None]).astype(np.float32), -448, 448)
+    table = _e4m3_values_from_definition()
+    vals = table[q]
+    # each code is the e4m3 value nearest the IEEE quotient (ties checked above)
+    fin = table[:0x7F]
+    for i in range(1, 33):
+        for k in range(0, 300, 7):
+            r = float(abs(ratio[i, k]))
+            assert abs(abs(vals[i, k]) - r) == np.abs(fin - r).min()
+    # the absmax element maps to +-448 in every nonzero row
+    for i in range(1, 33):
+        j = int(np.argmax(np.abs(xf[i])))
+        assert q[i, j] & 0x7F == 0x7E
+    assert not q[0].any()
+
+
+def test_fp8_gemm_is_the_exact_sum():
+    rng = np.random.default_rng(8)
+    A = rng.integers(0, 256, (9, 96)).astype(np.uint8)
+    W = rng.integers(0, 256, (7, 96)).astype(np.uint8)
+    A[(A & 0x7F) == 0x7F] = 0x12                 # no NaN codes
+    W[(W & 0x7F) == 0x7F] = 0x35
+    Av, Wv = _e4m3_values_from_definition()[A], _e4m3_values_from_definition()[W]
+    want = Av @ Wv.T
+    got = oracle.gemm_fp8_f64(A, W)
+    assert np.array_equal(got, want)
+    # products of e4m3 values are exact in double: a transposed operand fails
+    assert not np.array_equal(oracle.gemm_fp8_f64(A, W[::-1]), want)
