@@ -2,7 +2,7 @@
 """Benchmark of the int8 dynamic-quantization linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload llm|tiny|large_m|large_m_s32|vit_fc1|vit_fc2|vit_fc1_20|vit_fc2_20|
+                    [--workload llm|llm_fp8|tiny|large_m|large_m_s32|vit_fc1|vit_fc2|vit_fc1_20|vit_fc2_20|
                                 vit_fc1_b32|vit_fc1_b16|vit_fc1_dense|vit_fc2_dense|quant|small_m1|
                                 small_m16|small_m128|mma_peak]
 
@@ -85,6 +85,9 @@ WORKLOADS = {
     "llm": dict(kind="dense", M=2048, K=4096, N=4096, desc="LLM-shaped dense linear M=2048 K=4096 N=4096, "
                 "1% x20 outlier channels, per-token quant + fused i8i8->bf16, no bias"),
     "tiny": dict(kind="dense", M=64, K=256, N=256, bias=True, desc="tiny dense linear M=64 K=256 N=256 + bias"),
+    "llm_fp8": dict(kind="dense_fp8", M=2048, K=4096, N=4096,
+                    desc="LLM-shaped dense linear M=2048 K=4096 N=4096, 1% x20 outlier channels, "
+                         "per-token dynamic FP8 (e4m3) quant + fused e4m3 x e4m3 -> bf16 (fp32 accumulate)"),
     "large_m": dict(kind="gemm", M=38400, K=1024, N=4096, out="bf16",
                     desc="large-M int8 GEMM M=38400 K=1024 N=4096, fused bf16 epilogue"),
     "large_m_s32": dict(kind="gemm", M=38400, K=1024, N=4096, out="s32",
@@ -112,6 +115,8 @@ WORKLOADS = {
 def _synth_inputs(name, wl, seed):
     import synth
     k = wl["kind"]
+    if k == "dense_fp8":
+        return synth.llm(seed)
     if k == "dense":
         if name == "llm":
             d = synth.llm(seed)
@@ -132,13 +137,13 @@ def _synth_inputs(name, wl, seed):
 def step_accounting(wl, d):
     """(ops per step, dominant kernel name, its algorithmic units)."""
     k = wl["kind"]
-    if k in ("dense", "gemm"):
+    if k in ("dense", "gemm", "dense_fp8"):
         M, K, N = wl["M"], wl["K"], wl["N"]
         ops = 2.0 * M * N * K
         out_b = 4 if wl.get("out") == "s32" else 2
         gemm_bytes = M * K + N * K + M * N * out_b + 4 * (M + N)
-        return ops, dict(kernel="dq_int8_linear", ops=ops, bytes=gemm_bytes,
-                         quant_bytes=(3 * M * K + 4 * M) if k == "dense" else 0)
+        return ops, dict(kernel="dq_fp8_linear" if k == "dense_fp8" else "dq_int8_linear", ops=ops,
+                         bytes=gemm_bytes, quant_bytes=(3 * M * K + 4 * M) if k != "gemm" else 0)
     if k in ("bsr", "bsr_dense"):
         M, K, N = d["M"], d["K"], d["N"]
         nnzb = int(d["crow"][-1])
@@ -278,6 +283,26 @@ def make_state(name, wl, dq, torch, seed):
         st["out"] = out
         return _finish(st)
     # layer workloads: quantize + GEMM
+    if k == "dense_fp8":
+        w = _to_dev(torch, d["w"])
+        wq, sc = dq.dq_quantize_weight_fp8(w)
+        del w
+        M, K, N = d["x"].shape[0], d["x"].shape[1], d["w"].shape[0]
+        x = _to_dev_bf16(torch, d["x"])
+        n = _ncopies(x.numel() * 2 + wq.numel())
+        st["copies"] = [dict(x=x if i == 0 else x.clone(), W=wq if i == 0 else wq.clone()) for i in range(n)]
+        q = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+        s = torch.empty((M,), dtype=torch.float32, device="cuda")
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        st.update(q=q, s=s, out=out)
+        st["h2d"] = [("x", M * K * 2)]
+        st["d2h"] = [("out", M * N * 2)]
+
+        st["kernels"] = [
+            lambda c, stream: dq.dq_quantize_rows_fp8(c["x"], q, s, stream=stream),
+            lambda c, stream: dq.dq_fp8_linear(q, s, c["W"], sc, out=out, stream=stream)]
+        st["names"] = ["dq_quantize_rows_fp8", "dq_fp8_linear"]
+        return _finish(st)
     if k == "dense":
         w = _to_dev(torch, d["w"])
         wq, sc = dq.dq_quantize_weight(w)
@@ -491,12 +516,13 @@ def run_gpu(args, rank, world, local_rank):
 
     # end to end through the public API with host buffers
     e2e = None
-    if wl["kind"] in ("dense", "bsr", "bsr_dense", "quant", "gemm"):
+    if wl["kind"] in ("dense", "bsr", "bsr_dense", "quant", "gemm", "dense_fp8"):
         e2e = run_e2e(args, wl, state, dq, torch, stream, ops, dom, world, max_over_ranks)
 
     line = dict(metric=METRIC, value=round(value, 2) if value is not None else None, unit=unit, n_gpus=world,
                 steps=K, warmup=args.warmup, ms_per_step=round(total_ms_max / K, 5), higher_is_better=True,
-                scaling="weak", vs_baseline=None, dtype="int8", data="synthetic",
+                scaling="weak", vs_baseline=None, dtype="e4m3" if wl["kind"] == "dense_fp8" else "int8",
+                data="synthetic",
                 config=dict(workload=wl["desc"], tokens_per_rank=state["d"].get("M", wl.get("M")),
                             parallelism=f"dp{world} (token rows sharded, weights replicated, no collective)",
                             l2=f"inputs rotate over {len(copies)} copies (> 2x the 126 MB L2)",

@@ -62,7 +62,8 @@ typedef enum {
 
 typedef enum {
     DQ_OUT_BF16 = 0,          /* out = bf16(acc * s_row * s_col + bias): the layer */
-    DQ_OUT_S32 = 1            /* out = acc as int32 (scales and bias ignored) */
+    DQ_OUT_S32 = 1,           /* out = acc as int32 (scales and bias ignored) */
+    DQ_OUT_F32 = 2            /* FP8 path: out = acc as fp32 (scales and bias ignored) */
 } dq_out_dtype;
 
 /* Static description of a status code. Never NULL. */
@@ -247,6 +248,39 @@ DQ_API dq_status dq_bsr_pack_blocked(const int8_t* wq, int64_t N, int64_t K, int
                                      int8_t* values, dq_stream_t stream);
 DQ_API dq_status dq_bsr_validate_blocked(const int32_t* crow, const int32_t* col, int64_t N, int64_t K,
                                          int64_t block, int64_t nnzb);
+
+/* ------------------------------------------------------------------------
+ * Dynamic FP8 (e4m3) sibling of the int8 layer (the vLLM csrc/quantization
+ * commits: dynamic activation scales, scaled values clamped to the e4m3
+ * range so that no NaN appears; applied per token here like the int8 path).
+ *
+ * dq_quantize_rows_fp8 / dq_quantize_weight_fp8: per row
+ *   s = fp32( max(absmax, 1e-8f) / 448 ),
+ *   q = e4m3( clamp( fp32(x / s), -448, 448 ) )   round to nearest even,
+ * codes are e4m3 bytes (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits; 448 the largest value), layouts and requirements as
+ * dq_quantize_rows / dq_quantize_weight.  Bit-identical to a scalar IEEE
+ * evaluation.
+ *
+ * dq_fp8_linear: acc[m, n] = sum_k e4m3(A[m, k]) * e4m3(W[n, k]) on the
+ * tensor cores (tcgen05.mma kind::f8f6f4, fp32 accumulator in TMEM), then
+ *   DQ_OUT_BF16: out = bf16((acc * s_row[m]) * s_col[n] + bias[n]) as the
+ *                int8 layer (each op rounded, left to right, no FMA);
+ *   DQ_OUT_F32:  out = acc as fp32 (scales and bias ignored).
+ * Every product of two e4m3 values is exact in fp32; the order and
+ * precision of the tensor core's fp32 sum are the hardware's, so results are
+ * not bit-reproducible by a scalar loop (the tests bound |acc - exact sum|).
+ * A and W are uint8 e4m3 codes, K-major ([M,K] and [N,K] row-major).
+ * Requirements: K % 16 == 0, N % 8 == 0 (bf16 out) or N % 4 == 0 (fp32 out),
+ * pointers 16-byte aligned; M >= 0.  DQ_OUT_S32 is rejected here.
+ * ------------------------------------------------------------------------ */
+DQ_API dq_status dq_quantize_rows_fp8(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                                      int64_t ldq, float* scales, dq_stream_t stream);
+DQ_API dq_status dq_quantize_weight_fp8(const float* w, int64_t N, int64_t K, int64_t ldw, uint8_t* wq,
+                                        int64_t ldwq, float* s_col, dq_stream_t stream);
+DQ_API dq_status dq_fp8_linear(const uint8_t* A, const float* s_row, int64_t M, int64_t K, const uint8_t* W,
+                               const float* s_col, int64_t N, const void* bias_bf16, void* out,
+                               dq_out_dtype out_dtype, dq_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Measurement helper: a kernel that only issues tcgen05.mma.kind::i8

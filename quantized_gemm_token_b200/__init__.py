@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdq.so")
 
 DQ_OK, DQ_ERR_INVALID_ARG, DQ_ERR_UNSUPPORTED, DQ_ERR_CUDA, DQ_ERR_TIMEOUT = range(5)
-DQ_OUT_BF16, DQ_OUT_S32 = 0, 1
+DQ_OUT_BF16, DQ_OUT_S32, DQ_OUT_F32 = 0, 1, 2
 
 # C prototypes: (name, restype, argtypes)
 _P, _I64, _I32, _SZ, _U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
@@ -46,6 +46,9 @@ _PROTOS = {
     "dq_mma_peak_probe": (_I32, [_I32, _I32, _P]),
     "dq_debug_set_schedule": (None, [_I32]),
     "dq_debug_set_tile_n": (None, [_I32]),
+    "dq_quantize_rows_fp8": (_I32, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
+    "dq_quantize_weight_fp8": (_I32, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
+    "dq_fp8_linear": (_I32, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P, _I32, _P]),
     "dq_debug_set_two_widths": (None, [_I32]),
     "dq_debug_set_bsr_panel": (None, [_I32]),
     "dq_debug_set_quant_kernel": (None, [_I32]),
@@ -205,6 +208,75 @@ def dq_quantize_weight(w: torch.Tensor, wq: torch.Tensor = None, s_col: torch.Te
     _check(lib.dq_quantize_weight(_ptr(w), N, K, w.stride(0), _ptr(wq), wq.stride(0), _ptr(s_col),
                                   _stream(stream)), "dq_quantize_weight")
     return wq, s_col
+
+
+def dq_quantize_rows_fp8(x: torch.Tensor, q: torch.Tensor = None, scales: torch.Tensor = None, stream=None):
+    """Per-token dynamic FP8: x bf16 [M, K] -> (q e4m3 codes uint8 [M, K], scales fp32 [M]),
+    s = max(absmax, 1e-8) / 448, q = e4m3(clamp(x / s, -448, 448))."""
+    _need(x, torch.bfloat16, "x", 2)
+    if x.stride(1) != 1:
+        raise ValueError("x: rows must be contiguous")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _need(q, torch.uint8, "q", 2)
+    _need(scales, torch.float32, "scales", 1)
+    if q.stride(1) != 1 or tuple(q.shape) != (M, K) or scales.numel() != M:
+        raise ValueError("q / scales: shape or layout mismatch")
+    _check(lib.dq_quantize_rows_fp8(_ptr(x), M, K, x.stride(0), _ptr(q), q.stride(0), _ptr(scales),
+                                    _stream(stream)), "dq_quantize_rows_fp8")
+    return q, scales
+
+
+def dq_quantize_weight_fp8(w: torch.Tensor, wq: torch.Tensor = None, s_col: torch.Tensor = None, stream=None):
+    """Per-output-channel FP8 weight: w fp32 [N, K] -> (wq e4m3 codes uint8 [N, K], s_col fp32 [N])."""
+    _need(w, torch.float32, "w", 2)
+    if w.stride(1) != 1:
+        raise ValueError("w: rows must be contiguous")
+    N, K = w.shape
+    if wq is None:
+        wq = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    if s_col is None:
+        s_col = torch.empty((N,), dtype=torch.float32, device=w.device)
+    _check(lib.dq_quantize_weight_fp8(_ptr(w), N, K, w.stride(0), _ptr(wq), wq.stride(0), _ptr(s_col),
+                                      _stream(stream)), "dq_quantize_weight_fp8")
+    return wq, s_col
+
+
+def dq_fp8_linear(A, s_row, W, s_col, bias=None, out=None, out_dtype="bf16", stream=None):
+    """FP8 sibling of dq_int8_linear: A, W e4m3 codes (uint8) [M, K], [N, K];
+    out = bf16(acc * s_row * s_col + bias), or the fp32 accumulators with out_dtype="f32"."""
+    if out_dtype in ("f32", "float32", torch.float32, DQ_OUT_F32):
+        code = DQ_OUT_F32
+    elif out_dtype in ("bf16", torch.bfloat16, DQ_OUT_BF16):
+        code = DQ_OUT_BF16
+    else:
+        raise ValueError(f"out_dtype {out_dtype!r}")
+    _need(A, torch.uint8, "A", 2)
+    _need(W, torch.uint8, "W", 2)
+    _contig(A, "A")
+    _contig(W, "W")
+    M, K = A.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("A and W disagree on K")
+    if code == DQ_OUT_BF16:
+        _need(s_row, torch.float32, "s_row", 1)
+        _need(s_col, torch.float32, "s_col", 1)
+        if s_row.numel() != M or s_col.numel() != N:
+            raise ValueError("scale length mismatch")
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias", 1)
+    odt = torch.bfloat16 if code == DQ_OUT_BF16 else torch.float32
+    if out is None:
+        out = torch.empty((M, N), dtype=odt, device=A.device)
+    _need(out, odt, "out", 2)
+    _contig(out, "out")
+    _check(lib.dq_fp8_linear(_ptr(A), _ptr(s_row), M, K, _ptr(W), _ptr(s_col), N, _ptr(bias), _ptr(out),
+                             code, _stream(stream)), "dq_fp8_linear")
+    return out
 
 
 # ---------------------------------------------------------------- linear

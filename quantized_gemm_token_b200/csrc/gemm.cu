@@ -123,7 +123,7 @@ struct TileGeom {
 template <Kind KIND, int BN>
 __device__ __forceinline__ TileGeom tile_geom(const GemmArgs& g, int tile) {
   TileGeom t;
-  if (KIND == Kind::Dense && g.bn2 > 0 && tile >= g.t1) {
+  if (is_dense_kind(KIND) && g.bn2 > 0 && tile >= g.t1) {
     int j = tile - g.t1;
     if (j < g.first_cnt) {
       t.ta = g.mb0;
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
-    if (KIND == Kind::Dense && g.bn2 > 0) tma_prefetch_desc(&tm_b2);
+    if (is_dense_kind(KIND) && g.bn2 > 0) tma_prefetch_desc(&tm_b2);
     if constexpr (C::STAGED_OUT) tma_prefetch_desc(&tm_c);
   }
   if (warp == 1) {
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
       while (ok && iter.next(s)) {
         const TileGeom geo = tile_geom<KIND, BN>(g, s.tile);
         const int ta = geo.ta, tb = geo.tb;
-        const uint32_t stage_tx = C::A_BYTES + (KIND == Kind::Dense ? geo.width * C::KB : C::B_BYTES);
+        const uint32_t stage_tx = C::A_BYTES + (is_dense_kind(KIND) ? geo.width * C::KB : C::B_BYTES);
         if constexpr (PANEL) {
           if (ta != loaded_ta) {
             // a new 128-row block: once the MMAs on the previous panel are
@@ -336,7 +336,8 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_full = idesc_i8(128, C::MMA_N);
+      constexpr bool F8 = KIND == Kind::DenseF8;
+      constexpr uint32_t idesc_full = F8 ? idesc_e4m3(128, C::MMA_N) : idesc_i8(128, C::MMA_N);
       SegIter iter(g);
       Seg s;
       int stage = 0, acc = 0;
@@ -347,8 +348,8 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
       while (ok && iter.next(s)) {
         if (!mbar_wait(smem_u32(acce_bar + acc), acc_phase ^ 1, g.wait, abort_flag)) break;
         tc_fence_after();
-        const uint32_t idesc = (KIND == Kind::Dense && g.bn2 > 0 && s.tile >= g.t1)
-                                   ? idesc_i8(128, g.bn2) : idesc_full;
+        const uint32_t idesc = (is_dense_kind(KIND) && g.bn2 > 0 && s.tile >= g.t1)
+                                   ? (F8 ? idesc_e4m3(128, g.bn2) : idesc_i8(128, g.bn2)) : idesc_full;
         if constexpr (PANEL) {
           const int ta = s.tile / g.b_tiles;
           if (ta != cur_ta) {
@@ -407,8 +408,10 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
             bd = smem_desc_kmajor<C::KB>(smem_u32(sB + stage * C::B_BYTES));
           }
 #pragma unroll
-          for (int k = 0; k < C::K_STEPS; ++k)
-            mma_i8(d, ad + 2 * k, bd + 2 * k, idesc, (kb > k0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < C::K_STEPS; ++k) {
+            if constexpr (F8) mma_f8(d, ad + 2 * k, bd + 2 * k, idesc, (kb > k0 || k > 0) ? 1u : 0u);
+            else mma_i8(d, ad + 2 * k, bd + 2 * k, idesc, (kb > k0 || k > 0) ? 1u : 0u);
+          }
           mma_commit(smem_u32(empty_bar + stage));
           if (++stage == C::STAGES) {
             stage = 0;
@@ -472,7 +475,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
       // chunks of this tile (a narrow Dense tile has fewer; every warp still
       // has one, as bn2 >= 64); after reading its last chunk a warp releases
       // the accumulator
-      const int nch = KIND == Kind::Dense ? geo.width / CW : NCH;
+      const int nch = is_dense_kind(KIND) ? geo.width / CW : NCH;
       const int last_c = grp + ((nch - 1 - grp) / GROUPS) * GROUPS;
 
       if (whole) {
@@ -527,7 +530,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
             mbar_arrive(smem_u32(acce_bar + acc));
           }
           if constexpr (KIND == Kind::Swap) store_col_chunk<CW>(g, ta * 128 + row, n0 + c * CW, r);
-          else store_row_chunk_tma(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, n0 + c * CW, r, srow, cs);
+          else store_row_chunk_tma<KIND == Kind::DenseF8>(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, n0 + c * CW, r, srow, cs);
         }
       } else {
         // Stream-K partial tile: add into the workspace (coalesced: one
@@ -895,6 +898,70 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
     case 64: return launch<Kind::Swap, 64>(ta, tb, tb, tc, g, grid, stream);
     default: return launch<Kind::Swap, 128>(ta, tb, tb, tc, g, grid, stream);
   }
+}
+
+dq_status dq_fp8_linear(const uint8_t* A, const float* s_row, int64_t M, int64_t K, const uint8_t* W,
+                        const float* s_col, int64_t N, const void* bias_bf16, void* out, dq_out_dtype out_dtype,
+                        dq_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (out_dtype != DQ_OUT_BF16 && out_dtype != DQ_OUT_F32) return DQ_ERR_INVALID_ARG;
+  if (M < 0 || K < 1 || N < 1) return DQ_ERR_INVALID_ARG;
+  if (M > 0 && (A == nullptr || W == nullptr || out == nullptr)) return DQ_ERR_INVALID_ARG;
+  if (M > 0 && out_dtype == DQ_OUT_BF16 && (s_row == nullptr || s_col == nullptr))
+    return DQ_ERR_INVALID_ARG;
+  const bool f32 = out_dtype == DQ_OUT_F32;
+  if (K % 16 != 0 || N % (f32 ? 4 : 8) != 0) return DQ_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 128 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 20))
+    return DQ_ERR_UNSUPPORTED;
+  if (!aligned(A, 16) || !aligned(W, 16) || !aligned(out, 16)) return DQ_ERR_UNSUPPORTED;
+  if (!f32 && (!aligned(s_col, 16) || (bias_bf16 && !aligned(bias_bf16, 16)))) return DQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  dq_status st = current_device(&d);
+  if (st != DQ_OK) return st;
+  if (M == 0) return DQ_OK;
+
+  // The dense arrangement (tokens on MMA M) for every M, 128 x 256 tiles
+  // (128 x 128 for N <= 128), two tile widths when the last wave is partial.
+  Plan p{};
+  p.kind = Kind::DenseF8;
+  p.bn = N <= 128 ? 128 : 256;
+  p.a_tiles = static_cast<int>((M + 127) / 128);
+  p.b_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
+  p.kb_total = static_cast<int>((K + 127) / 128);
+  p.num_tiles = p.a_tiles * p.b_tiles;
+  if (p.bn == 256 && g_two_widths) plan_two_widths(p, N, d->sm_count);
+  CUtensorMap ta, tb, tb2, tc;
+  if ((st = make_tmap_u8_2d(&ta, A, K, M, K, 128, 128, 128)) != DQ_OK) return st;
+  if ((st = make_tmap_u8_2d(&tb, W, K, N, K, 128, p.bn, 128)) != DQ_OK) return st;
+  if (p.bn2 > 0) {
+    if ((st = make_tmap_u8_2d(&tb2, W, K, N, K, 128, p.bn2, 128)) != DQ_OK) return st;
+  } else {
+    tb2 = tb;
+  }
+  if ((st = make_tmap_out_2d(&tc, out, N, M, f32 ? 4 : 2)) != DQ_OK) return st;
+  GemmArgs g{};
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.a_tiles = p.a_tiles;
+  g.b_tiles = p.b_tiles;
+  g.kb_total = p.kb_total;
+  g.num_tiles = p.num_tiles;
+  g.t1 = p.t1;
+  g.bn2 = p.bn2;
+  g.mb0 = p.mb0;
+  g.c_start = p.c_start;
+  g.first_cnt = p.first_cnt;
+  g.per_row = p.per_row;
+  g.s_row = s_row;
+  g.s_col = s_col;
+  g.bias = static_cast<const uint16_t*>(bias_bf16);
+  g.out = out;
+  g.out_s32 = f32 ? 1 : 0;                   // raw accumulator bits
+  g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
+  const int grid = p.num_tiles < d->sm_count ? p.num_tiles : d->sm_count;
+  if (p.bn == 256) return launch<Kind::DenseF8, 256>(ta, tb, tb2, tc, g, grid, stream);
+  return launch<Kind::DenseF8, 128>(ta, tb, tb2, tc, g, grid, stream);
 }
 
 dq_status dq_bsr_int8_linear_blocked(const int8_t* A, const float* s_row, int64_t M, int64_t K, int64_t N,

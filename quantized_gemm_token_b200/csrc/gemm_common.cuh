@@ -10,7 +10,11 @@
 
 namespace dq {
 
-enum class Kind : int { Dense = 0, Swap = 1, Bsr = 2, Bsr32 = 3, Bsr16 = 4 };
+enum class Kind : int { Dense = 0, Swap = 1, Bsr = 2, Bsr32 = 3, Bsr16 = 4, DenseF8 = 5 };
+
+// Dense arrangement with int8 (Dense) or e4m3 (DenseF8) operands; e4m3
+// products accumulate in fp32 (kind::f8f6f4), int8 ones in int32.
+__host__ __device__ constexpr bool is_dense_kind(Kind k) { return k == Kind::Dense || k == Kind::DenseF8; }
 
 // Block-sparse weight kinds and their square block size (64, 32 or 16).
 __host__ __device__ constexpr bool is_bsr(Kind k) { return k == Kind::Bsr || k == Kind::Bsr32 || k == Kind::Bsr16; }
@@ -152,7 +156,7 @@ __device__ __forceinline__ void load_col_scales(const GemmArgs& g, int n0, ColSc
 // columns < N.  The output mode and the bias are template switches rather
 // than run-time tests, so the code of the modes not taken is not executed
 // predicated-off in every chunk.
-template <bool S32, bool BIAS>
+template <bool S32, bool BIAS, bool F32ACC>
 __device__ __forceinline__ void store_row_chunk_tma_t(const GemmArgs& g, const CUtensorMap* tm_c,
                                                       uint8_t* buf, int lane, int m0, int n0,
                                                       const uint32_t* r, float srow, const ColScales& cs) {
@@ -174,8 +178,10 @@ __device__ __forceinline__ void store_row_chunk_tma_t(const GemmArgs& g, const C
     uint64_t f2[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const uint64_t a = pack_f2(__int2float_rn(static_cast<int>(r[2 * j])),
-                                 __int2float_rn(static_cast<int>(r[2 * j + 1])));
+      // int32 accumulators convert (round to nearest); fp32 ones are taken as they are
+      const uint64_t a = F32ACC ? pack_f2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]))
+                                : pack_f2(__int2float_rn(static_cast<int>(r[2 * j])),
+                                          __int2float_rn(static_cast<int>(r[2 * j + 1])));
       f2[j] = mul_f2(mul_f2(a, srow2), cs.sc[j]);
     }
     if constexpr (BIAS) {
@@ -214,12 +220,14 @@ __device__ __forceinline__ void store_row_chunk_tma_t(const GemmArgs& g, const C
   }
 }
 
+template <bool F32ACC = false>
 __device__ __forceinline__ void store_row_chunk_tma(const GemmArgs& g, const CUtensorMap* tm_c, uint8_t* buf,
                                                     int lane, int m0, int n0, const uint32_t* r, float srow,
                                                     const ColScales& cs) {
-  if (g.out_s32) store_row_chunk_tma_t<true, false>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
-  else if (g.bias != nullptr) store_row_chunk_tma_t<false, true>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
-  else store_row_chunk_tma_t<false, false>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
+  // raw mode stores the accumulator bits (int32, or fp32 for e4m3 operands)
+  if (g.out_s32) store_row_chunk_tma_t<true, false, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
+  else if (g.bias != nullptr) store_row_chunk_tma_t<false, true, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
+  else store_row_chunk_tma_t<false, false, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
 }
 
 // Epilogue for the Swap layout: thread = output channel n, columns are

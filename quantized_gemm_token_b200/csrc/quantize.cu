@@ -125,8 +125,47 @@ __device__ __forceinline__ uint2 quant_bf16x8(const uint32_t (&w)[4], uint64_t i
   return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
+// Output formats: int8 codes (absmax / 127) or e4m3 codes (absmax / 448, the
+// largest e4m3 value; the vLLM quantization commits' dynamic FP8 scaling with
+// the scaled values clamped to the e4m3 range).
+enum class QFmt : int { I8 = 0, E4M3 = 1 };
+
+template <QFmt F = QFmt::I8>
 __device__ __forceinline__ float scale_from_absmax(float a) {
-  return __fdiv_rn(fmaxf(a, 1e-8f), 127.0f);
+  return __fdiv_rn(fmaxf(a, 1e-8f), F == QFmt::E4M3 ? 448.0f : 127.0f);
+}
+
+// Two fp32 values -> two e4m3 codes (round to nearest even; magnitudes above
+// 448 saturate to 448, which is the clamp), lo in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// e4m3 codes of 8 bf16 values (4 packed words): the quotient by Markstein's
+// correction step as in the int8 path (for bf16 inputs and s = absmax / 448
+// its e4m3 code equals the IEEE quotient's, checked for every bf16 pair), then
+// one conversion per pair.
+__device__ __forceinline__ uint2 quant_bf16x8_e4m3(const uint32_t (&w)[4], uint64_t inv2, uint64_t negs2) {
+  uint32_t c[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const uint64_t v = pack_f2(__uint_as_float(w[h] << 16), __uint_as_float(w[h] & 0xffff0000u));
+    const uint64_t q0 = mul_f2(v, inv2);
+    const uint64_t r = fma_f2(q0, negs2, v);
+    const uint64_t q1 = fma_f2(r, inv2, q0);
+    float lo, hi;
+    unpack_f2(q1, lo, hi);
+    c[h] = e4m3x2(lo, hi);
+  }
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+// e4m3 codes of 4 fp32 values (weights, offline): the IEEE quotient itself.
+__device__ __forceinline__ uint32_t quant_f32x4_e4m3(uint4 v, float s) {
+  return e4m3x2(__fdiv_rn(__uint_as_float(v.x), s), __fdiv_rn(__uint_as_float(v.y), s)) |
+         (e4m3x2(__fdiv_rn(__uint_as_float(v.z), s), __fdiv_rn(__uint_as_float(v.w), s)) << 16);
 }
 
 __device__ __forceinline__ uint32_t pack4(int8_t a, int8_t b, int8_t c, int8_t d) {
@@ -148,7 +187,7 @@ __device__ __noinline__ uint32_t quant_f32x4_exact(uint4 v, float s) {
 // Register-resident single-pass kernel.  256 threads; a row is owned by
 // 2^tpr_log2 consecutive threads (32..256); VPT = max 16-byte vectors per
 // thread.
-template <typename T, int VPT>
+template <typename T, int VPT, QFmt F = QFmt::I8>
 __global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict__ x, int64_t M,
                                                              int64_t K, int64_t ldx,
                                                              int8_t* __restrict__ q, int64_t ldq,
@@ -209,7 +248,7 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict
     for (int w = 0; w < wpr; ++w) amax = max(amax, warp_max[w0 + w]);
   }
   if (row >= M) return;
-  const float s = scale_from_absmax(__uint_as_float(amax));
+  const float s = scale_from_absmax<F>(__uint_as_float(amax));
   const float inv = __frcp_rn(s);
   if (t == 0) scales[row] = s;
 
@@ -224,7 +263,12 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict
     const int vi = t + i * tpr;
     if (vi < nv) {
       const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      if constexpr (E == 8) {
+      if constexpr (F == QFmt::E4M3) {
+        if constexpr (E == 8)
+          *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(vi) * 8) = quant_bf16x8_e4m3(w, inv2, negs2);
+        else
+          *reinterpret_cast<uint32_t*>(qr + static_cast<int64_t>(vi) * 4) = quant_f32x4_e4m3(v[i], s);
+      } else if constexpr (E == 8) {
         *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(vi) * 8) = quant_bf16x8(w, inv2, negs2, magic2);
       } else {
         uint32_t tie = 0xffffffffu, b[4], dd[4];
@@ -253,7 +297,7 @@ __device__ __forceinline__ float load_as_float<float>(const float* p) {
 
 // Any shape, stride or alignment: one CTA of 256 threads per row, two passes
 // over the row (the second mostly from L2).
-template <typename T>
+template <typename T, QFmt F = QFmt::I8>
 __global__ void __launch_bounds__(256) quant_rows_generic_kernel(const T* __restrict__ x, int64_t M,
                                                                  int64_t K, int64_t ldx,
                                                                  int8_t* __restrict__ q,
@@ -270,10 +314,17 @@ __global__ void __launch_bounds__(256) quant_rows_generic_kernel(const T* __rest
     a = warp_max[0];
     for (int w = 1; w < 8; ++w) a = fmaxf(a, warp_max[w]);
     __syncthreads();
-    const float s = scale_from_absmax(a);
+    const float s = scale_from_absmax<F>(a);
     if (threadIdx.x == 0) scales[row] = s;
     int8_t* qr = q + row * ldq;
-    for (int64_t k = threadIdx.x; k < K; k += 256) qr[k] = quant_one(load_as_float<T>(xr + k), s);
+    for (int64_t k = threadIdx.x; k < K; k += 256) {
+      if constexpr (F == QFmt::E4M3) {
+        const float qv = __fdiv_rn(load_as_float<T>(xr + k), s);
+        qr[k] = static_cast<int8_t>(e4m3x2(qv, 0.0f) & 0xffu);
+      } else {
+        qr[k] = quant_one(load_as_float<T>(xr + k), s);
+      }
+    }
   }
 }
 
@@ -444,7 +495,7 @@ __global__ void __launch_bounds__(QT_THREADS, 1)
 // Measurement knob: 0 = automatic, 1 = register kernel, 2 = pipelined kernel.
 int g_quant_kernel_override = 0;
 
-template <typename T>
+template <typename T, QFmt F = QFmt::I8>
 dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
                           float* scales, cudaStream_t stream) {
   if (M < 0 || K < 1 || ldx < K || ldq < K) return DQ_ERR_INVALID_ARG;
@@ -465,7 +516,7 @@ dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t*
   // shape (16384 x 8192: 6.0 TB/s against 5.6-5.8 for the pipelined kernel),
   // so the pipelined kernel runs only when asked for.
   const bool tma_ok = vec_ok && row_bytes >= 1024 && row_bytes <= QT_MAX_ROW_BYTES;
-  const bool tma_pick = g_quant_kernel_override == 2;
+  const bool tma_pick = g_quant_kernel_override == 2 && F == QFmt::I8;   // int8 codes only
   if (tma_ok && tma_pick) {
     // stage = one row rounded up to 128 bytes; at most as many stages as the
     // ring holds (<= 192).
@@ -515,16 +566,16 @@ dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t*
     if (grid > 0x7fffffff) return DQ_ERR_UNSUPPORTED;
     dim3 g(static_cast<unsigned>(grid));
     if (vpt <= 1)
-      quant_rows_vec_kernel<T, 1><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+      quant_rows_vec_kernel<T, 1, F><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
     else if (vpt <= 2)
-      quant_rows_vec_kernel<T, 2><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+      quant_rows_vec_kernel<T, 2, F><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
     else if (vpt <= 4)
-      quant_rows_vec_kernel<T, 4><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+      quant_rows_vec_kernel<T, 4, F><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
     else
-      quant_rows_vec_kernel<T, 8><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+      quant_rows_vec_kernel<T, 8, F><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
   } else {
     const int64_t grid = M < int64_t(d->sm_count) * 16 ? M : int64_t(d->sm_count) * 16;
-    quant_rows_generic_kernel<T><<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, M, K, ldx, q,
+    quant_rows_generic_kernel<T, F><<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, M, K, ldx, q,
                                                                                  ldq, scales);
   }
   cudaError_t e = cudaGetLastError();
@@ -548,6 +599,19 @@ dq_status dq_quantize_weight(const float* w, int64_t N, int64_t K, int64_t ldw, 
                              int64_t ldwq, float* s_col, dq_stream_t stream) {
   return dq::launch_quantize<float>(w, N, K, ldw, wq, ldwq, s_col,
                                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+dq_status dq_quantize_rows_fp8(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                               int64_t ldq, float* scales, dq_stream_t stream) {
+  return dq::launch_quantize<uint16_t, dq::QFmt::E4M3>(static_cast<const uint16_t*>(x_bf16), M, K, ldx,
+                                                       reinterpret_cast<int8_t*>(q), ldq, scales,
+                                                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+dq_status dq_quantize_weight_fp8(const float* w, int64_t N, int64_t K, int64_t ldw, uint8_t* wq,
+                                 int64_t ldwq, float* s_col, dq_stream_t stream) {
+  return dq::launch_quantize<float, dq::QFmt::E4M3>(w, N, K, ldw, reinterpret_cast<int8_t*>(wq), ldwq, s_col,
+                                                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
