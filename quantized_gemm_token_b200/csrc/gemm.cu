@@ -662,7 +662,8 @@ constexpr int64_t kMaxK = 133144;   // floor((2^31 - 1) / 127^2): int32 accumula
 constexpr int64_t kPairMinK = 8192;
 
 // Schedule override for measurements: 0 = automatic, 1 = 1-SM whole tiles,
-// 2 = 1-SM stream-K, 3 = pair (2-SM) kernel for every M.
+// 2 = 1-SM stream-K, 3 = pair (2-SM) kernel for every M, 4 = the dense
+// (tokens on MMA M) arrangement also for M <= 128.
 int g_schedule_override = 0;
 // Tile-width override for measurements (0 = automatic).
 int g_tile_n_override = 0;
@@ -721,18 +722,32 @@ size_t sk_workspace_bytes(const Plan& p, int /*ctas*/) {
   return static_cast<size_t>(p.num_tiles) * (static_cast<size_t>(p.bn) * 128 * 4 + 4);
 }
 
+// Few tokens (M <= 128): the weight stream dominates.  With enough output
+// channels for about a wave of 128 x 224 tiles, the dense arrangement (tokens
+// on MMA M, rows past M zero-filled by TMA and clipped on store) streams the
+// weight faster than swap-AB, whose column-wise epilogue stores are
+// scattered: measured at N = 28672, K = 8192: M = 128 47 us vs 57, M = 32
+// 46.3 vs 48.9, M = 16 45.9 vs 46.7, but M = 1 54 vs 46, so from M = 17 on.
+// For fewer channels swap-AB with stream-K keeps every SM busy.
+bool small_m_dense(int64_t M, int64_t N, int sm_count) {
+  if (g_schedule_override == 4 || g_schedule_override == 5) return true;
+  return M > 16 && M <= 128 && g_schedule_override == 0 && g_tile_n_override == 0 &&
+         (N + 223) / 224 >= sm_count * 3 / 4;
+}
+
 Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count) {
   Plan p{};
-  if (M <= 128) {
+  const bool dense_small = M <= 128 && small_m_dense(M, N, sm_count);
+  if (M <= 128 && !dense_small) {
     p.kind = Kind::Swap;
     p.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
     p.a_tiles = static_cast<int>((N + 127) / 128);
     p.b_tiles = static_cast<int>((M + p.bn - 1) / p.bn);
   } else {
     p.kind = Kind::Dense;
-    p.bn = N <= 128 ? 128 : 256;
+    p.bn = N <= 128 ? 128 : dense_small ? 224 : 256;
     if (g_tile_n_override == 128 || g_tile_n_override == 160 || g_tile_n_override == 192 ||
-        g_tile_n_override == 256)
+        g_tile_n_override == 224 || g_tile_n_override == 256)
       p.bn = g_tile_n_override;
     p.a_tiles = static_cast<int>((M + 127) / 128);
     p.b_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
@@ -832,7 +847,7 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   bool sk = p.stream_k && workspace != nullptr && workspace_bytes >= p.ws_bytes &&
             aligned(workspace, 16);
   if (g_schedule_override == 1) sk = false;
-  if (g_schedule_override == 2) {
+  if (g_schedule_override == 2 || g_schedule_override == 5) {
     p.bn2 = 0;                                    // stream-K ranges run over uniform tiles
     p.num_tiles = p.a_tiles * p.b_tiles;
     if (workspace != nullptr && aligned(workspace, 16) &&
@@ -887,6 +902,7 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   if (p.kind == Kind::Dense) {
     switch (p.bn) {
       case 256: return launch<Kind::Dense, 256>(ta, tb, tb2, tc, g, grid, stream);
+      case 224: return launch<Kind::Dense, 224>(ta, tb, tb2, tc, g, grid, stream);
       case 192: return launch<Kind::Dense, 192>(ta, tb, tb2, tc, g, grid, stream);
       case 160: return launch<Kind::Dense, 160>(ta, tb, tb2, tc, g, grid, stream);
       default: return launch<Kind::Dense, 128>(ta, tb, tb2, tc, g, grid, stream);

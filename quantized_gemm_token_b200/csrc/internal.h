@@ -50,9 +50,10 @@ inline bool aligned(const void* p, size_t a) {
 
 // Measurement knob, not part of the public header: 0 = automatic schedule,
 // 1 = 1-SM kernel with whole tiles, 2 = 1-SM stream-K whenever a workspace
-// allows it, 3 = the 2-SM pair kernel for every M.
+// allows it, 3 = the 2-SM pair kernel for every M, 4 = the dense arrangement
+// also for M <= 128.
 extern "C" DQ_API void dq_debug_set_schedule(int mode);
-// Measurement knob: force the dense tile width (128, 160, 192, 256; 0 = automatic).
+// Measurement knob: force the dense tile width (128, 160, 192, 224, 256; 0 = automatic).
 extern "C" DQ_API void dq_debug_set_tile_n(int n);
 // Measurement knob: 0 turns off the two-width (wave-balanced) dense schedule.
 extern "C" DQ_API void dq_debug_set_two_widths(int on);

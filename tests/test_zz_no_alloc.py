@@ -41,9 +41,9 @@ def _call_noalloc(lib, A, s_row, W, s_col, bias, out, code):
                                       stream)
 
 
-# (M, N, K): few-token shapes whose stream-K schedule uses 1.8 MB and 14.7 MB
-# of scratch
-@pytest.mark.parametrize("M,N,K", [(16, 28672, 8192), (128, 28672, 8192)])
+# (M, N, K): few-token shapes whose (swap-AB) stream-K schedule uses 0.5 MB
+# and 8.4 MB of scratch
+@pytest.mark.parametrize("M,N,K", [(16, 8192, 8192), (128, 16384, 8192)])
 def test_noalloc_matches_workspace_entry_two_calls(M, N, K):
     import quantized_gemm_token_b200 as dq
     from gpu_util import assert_bf16_close, bf16_bits
@@ -65,9 +65,18 @@ def test_noalloc_matches_workspace_entry_two_calls(M, N, K):
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
+    """With the automatic plan no shape needs more scratch than the entry
+    point has (wide few-token shapes take the dense arrangement, which needs
+    none); forcing the swap-AB stream-K schedule on a wide one does, and the
+    call must then refuse rather than overrun the array."""
     import quantized_gemm_token_b200 as dq
-    M, N, K = 128, 66560, 256                             # stream-K here needs ~34 MB
-    assert dq.dq_int8_linear_workspace_size(M, N, K) > dq.DQ_NOALLOC_SCRATCH_BYTES
-    A, W, s_row, s_col, bias = _inputs(M, N, K, 990)
-    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    assert _call_noalloc(dq.lib, A, s_row, W, s_col, None, out, dq.DQ_OUT_BF16) == dq.DQ_ERR_UNSUPPORTED
+    M, N, K = 128, 66560, 256
+    assert dq.dq_int8_linear_workspace_size(M, N, K) == 0
+    dq.dq_debug_set_schedule(2)                           # swap-AB, stream-K: ~34 MB of scratch
+    try:
+        assert dq.dq_int8_linear_workspace_size(M, N, K) > dq.DQ_NOALLOC_SCRATCH_BYTES
+        A, W, s_row, s_col, bias = _inputs(M, N, K, 990)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        assert _call_noalloc(dq.lib, A, s_row, W, s_col, None, out, dq.DQ_OUT_BF16) == dq.DQ_ERR_UNSUPPORTED
+    finally:
+        dq.dq_debug_set_schedule(0)
