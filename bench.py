@@ -15,7 +15,10 @@ Timing: W warm-up steps, then EXACTLY K steps captured in one CUDA graph and
 replayed once, bracketed by a barrier and a device synchronize (the value).
 Each kernel's average duration (kernels_ms, roofline) comes from a graph of K
 launches of that kernel alone on the same buffers, timed right after.
-Inputs rotate over enough copies to exceed the 126 MB L2 (config.l2).  Multi-GPU: one process per GPU, token
+Inputs rotate over enough copies to exceed the 126 MB L2 (config.l2).  e2e
+repeats the K steps through the public API from pinned host memory, each
+step's host->device copy and device->host read inside the timed region,
+pipelined on three streams.  Multi-GPU: one process per GPU, token
 batches sharded across ranks (weak scaling, no data-path collective); the
 reported time is the max over ranks.
 
@@ -528,7 +531,9 @@ def run_gpu(args, rank, world, local_rank):
                             l2=f"inputs rotate over {len(copies)} copies (> 2x the 126 MB L2)",
                             timing="value: one CUDA graph of the K steps, events around it; "
                                    "kernels_ms / roofline: per kernel, a graph of K launches of that "
-                                   "kernel alone on the same buffers, events around it",
+                                   "kernel alone on the same buffers, events around it; e2e: K steps "
+                                   "through the public API, each with its pinned-host H2D copy and D2H "
+                                   "read, pipelined on three streams (copy-in / kernels / copy-out)",
                             kernels_ms=kernels_ms),
                 roofline=roof, e2e=e2e, gpu_launches=nk * K, clocks=cs.summary())
     if rank == 0 and world == 1 and not args.no_cpu_baseline and wl["kind"] in ("dense", "bsr", "quant", "gemm"):
@@ -540,41 +545,67 @@ def run_gpu(args, rank, world, local_rank):
 
 
 def run_e2e(args, wl, state, dq, torch, stream, ops, dom, world, max_over_ranks):
-    """Same metric through the public API, host (pinned) buffers: per step
-    the H2D copy of the step's activations and the D2H read of its result are
-    inside the timed region."""
-    c0 = state["copies"][0]
-    key = "x" if "x" in c0 else "A"
-    dev_in = c0[key]
-    host_in = torch.empty(dev_in.shape, dtype=dev_in.dtype, pin_memory=True)
-    host_in.copy_(dev_in)
+    """Same metric through the public API, host (pinned) buffers: every step
+    copies its activations host->device and reads its result back
+    device->host inside the timed region.  The three run as a pipeline on
+    three streams: the copy-in of step i+1 (into the other of two device
+    input buffers) overlaps step i's kernels, and step i's copy-out overlaps
+    the copy-in of step i+2; a step's kernels wait for the previous step's
+    copy-out (one device output buffer)."""
+    copies = state["copies"]
+    key = "x" if "x" in copies[0] else "A"
+    bufs = [copies[0], copies[1 % len(copies)]]
+    host_in = torch.empty(bufs[0][key].shape, dtype=bufs[0][key].dtype, pin_memory=True)
+    host_in.copy_(bufs[0][key])
     outs = [state[n] for n, _ in state["d2h"]]
     host_outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
     K = args.steps
-    st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=False)  # noqa: E731
+    in_done, comp_done = [ev(), ev()], [ev(), ev()]
+    out_done = ev()
+    state_first = {"done": False}
 
-    def one():
-        dev_in.copy_(host_in, non_blocking=True)
-        state["step"](c0, stream)
-        for o, h in zip(outs, host_outs):
-            h.copy_(o, non_blocking=True)
+    def run(n_steps, start_ev=None):
+        if start_ev is not None:
+            s_in.wait_event(start_ev)
+            s_out.wait_event(start_ev)
+        for i in range(n_steps):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[b])          # step i-2 is done with this buffer
+                bufs[b][key].copy_(host_in, non_blocking=True)
+                in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
+            if i >= 1 or state_first["done"]:
+                stream.wait_event(out_done)                # the output buffer is free again
+            state["step"](bufs[b], stream)
+            comp_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[b])
+                for o, h in zip(outs, host_outs):
+                    h.copy_(o, non_blocking=True)
+                out_done.record(s_out)
+        state_first["done"] = True
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
 
-    for _ in range(3):
-        one()
+    run(3)
     torch.cuda.synchronize()
-    st.record()
-    for _ in range(K):
-        one()
-    en.record()
+    st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st.record(stream)
+    run(K, st)
+    en.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(st.elapsed_time(en))
     h2d = sum(b for _, b in state["h2d"])
     d2h = sum(b for _, b in state["d2h"])
     if wl["kind"] == "quant":
         return dict(value=round(dom["bytes"] * world * K / (ms * 1e-3) / 1e9, 2), unit="GB/s",
-                    h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h)
+                    h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, pipelined=True)
     return dict(value=round(ops * world * K / (ms * 1e-3) / 1e12, 3), unit="TOPS",
-                h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h)
+                h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, pipelined=True)
 
 
 # ----------------------------------------------------------------------------
