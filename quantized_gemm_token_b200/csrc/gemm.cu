@@ -1,33 +1,45 @@
 // gemm.cu -- the int8 x int8 -> int32 GEMM with the dequantization epilogue
 // fused (pytorch/ao PR 821, "int8 dynamic quant + bsr support": i8i8->bf16,
-// no int32 intermediate in global memory), dense and 64x64 BSR weight.
+// no int32 intermediate in global memory), dense and block-sparse weight,
+// and its e4m3 x e4m3 -> fp32 sibling (the vLLM quantization commits'
+// dynamic FP8, applied per token).
 //
 // One persistent, warp-specialised kernel template for sm_100a:
 //   warp 0      TMA producer: streams K slices of both operands into a ring
 //               of shared-memory stages (mbarrier full/empty pairs).
-//   warp 1      MMA issuer: one thread issues tcgen05.mma.kind::i8 (M = 128)
-//               into an int32 accumulator in TMEM; tcgen05.commit releases the
-//               stage and, at the end of a tile, hands the accumulator over.
-//   warps 2..5  epilogue: tcgen05.ld the accumulator (thread = TMEM lane =
-//               output row), dequantize in fp32 (acc * s_row * s_col + bias,
-//               each op rounded to nearest even, no FMA), convert to bf16 and
-//               store.  Accumulators are multi-buffered in TMEM so the
-//               epilogue of tile i overlaps the MMAs of tile i+1.
+//   warp 1      MMA issuer: one thread issues tcgen05.mma (kind::i8, or
+//               kind::f8f6f4 for e4m3; M = 128) into an accumulator in TMEM;
+//               tcgen05.commit releases the stage and, at the end of a tile,
+//               hands the accumulator over.
+//   warps 2..9  epilogue (two warps per TMEM sub-partition, alternate
+//               32-column chunks): tcgen05.ld the accumulator (thread = TMEM
+//               lane = output row), dequantize in fp32 (acc * s_row * s_col +
+//               bias, each op rounded to nearest even, no FMA), convert to
+//               bf16, stage 32x32 blocks in shared memory and TMA-store them.
+//               Accumulators are multi-buffered in TMEM so the epilogue of
+//               tile i overlaps the MMAs of tile i+1.
 //
-// Three operand arrangements share it:
-//   Dense  A slot = 128 activation rows, B slot = BN weight channels.
-//   Swap   A slot = 128 weight channels, B slot = BN (16..128) tokens: for
-//          few tokens the weight stream, not the token count, fills MMA M.
-//   Bsr    A slot = 128 activation rows x the k slice of one block column,
-//          B slot = one nonzero weight block (64x64, 32x32 or 16x16: kinds
-//          Bsr, Bsr32, Bsr16); a tile spans 256 channels (4, 8 or 16 block
-//          rows) and each block accumulates into its block row's slice of the
-//          TMEM tile; the producer walks crow/col (PR 821: the kernel takes
-//          crow_indices / col_indices / values directly).  A 16-wide block
-//          is issued as a K = 32 MMA whose other 16 k bytes read zeros.
+// Operand arrangements sharing it:
+//   Dense    A slot = 128 activation rows, B slot = BN weight channels
+//            (DenseF8: the same with e4m3 operands).  When whole tiles leave
+//            a partial last wave, the full waves keep BN-wide tiles and the
+//            rest of the matrix goes in one wave of narrower tiles.
+//   Swap     A slot = 128 weight channels, B slot = BN (16..128) tokens: for
+//            few tokens and few channels the weight stream, not the token
+//            count, fills MMA M.
+//   Bsr*     A slot = 128 activation rows x the k slice of one block column,
+//            B slot = one nonzero weight block (64x64, 32x32 or 16x16: kinds
+//            Bsr, Bsr32, Bsr16); a tile spans 256 channels (4, 8 or 16 block
+//            rows) and each block accumulates into its block row's slice of
+//            the TMEM tile; the producer walks crow/col (PR 821: the kernel
+//            takes crow_indices / col_indices / values directly).  A 16-wide
+//            block is issued as a K = 32 MMA whose other 16 k bytes read
+//            zeros.  The panel variant keeps a 128-row block's activations in
+//            shared memory and streams only weight blocks.
 //
-// Schedules: whole tiles round-robin over one CTA per SM, or (when the tile
-// count would leave SMs idle) stream-K: the tile x k-block iteration space is
+// Schedules: whole tiles round-robin over one CTA per SM (contiguous tile
+// ranges for the BSR panel variant), or, for the swap arrangement when whole
+// tiles would leave SMs idle, stream-K: the tile x k-block iteration space is
 // cut into equal contiguous ranges, one per CTA; partial tiles meet in an
 // int32 workspace through red.add, and the last arriving CTA (an arrival
 // counter) runs the epilogue and zeroes the workspace again.  Integer adds
