@@ -43,13 +43,26 @@ L2_BYTES = 126 * 1024 * 1024
 INT8_PER_BF16 = 2.0   # nominal dense int8 / bf16 tensor ratio (4.5 / 2.25 PFLOP/s)
 
 
-def kernel_source_hash() -> str:
-    """Hash of the CUDA sources: a stored ncu traffic figure only applies to
-    the kernels it was measured on."""
+# The CUDA sources each C-ABI entry point's kernels are compiled from (with
+# the headers they include).  A stored ncu traffic figure applies only while
+# these files are unchanged.
+_GEMM_SOURCES = ("gemm.cu", "gemm2sm.cu", "gemm_common.cuh", "sm100.cuh", "host.cu", "internal.h")
+KERNEL_SOURCES = {
+    "dq_quantize_rows": ("quantize.cu", "sm100.cuh", "host.cu", "internal.h"),
+    "dq_quantize_rows_fp8": ("quantize.cu", "sm100.cuh", "host.cu", "internal.h"),
+    "dq_int8_linear": _GEMM_SOURCES,
+    "dq_bsr_int8_linear": _GEMM_SOURCES,
+    "dq_fp8_linear": _GEMM_SOURCES,
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the CUDA sources `kernel` is built from: a stored ncu traffic
+    figure only applies to the kernel it was measured on."""
     import hashlib
     d = os.path.join(ROOT, "quantized_gemm_token_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
+    for f in sorted(KERNEL_SOURCES[kernel]):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
@@ -64,7 +77,7 @@ def measured_traffic(workload: str, kernel: str):
         with open(p) as f:
             t = json.load(f)
         e = t[workload][kernel]
-        return e["bytes_per_launch"] if e.get("source_hash") == kernel_source_hash() else None
+        return e["bytes_per_launch"] if e.get("source_hash") == kernel_source_hash(kernel) else None
     except Exception:
         return None
 
