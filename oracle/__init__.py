@@ -23,6 +23,11 @@ vLLM csrc/quantization commits: dynamic scales, clamp to the e4m3 range):
     keeps accuracy).
   * bsr_gemm_s32 / bsr_pack / bsr_densify -- 64x64 BSR weight given as
     crow_indices / col_indices / values (PR 821 description; --bsr 64).
+  * hqq_pack / hqq_unpack / hqq_dequant / hqq_linear_f64 / hqq_linear_t_f64 --
+    weight-only int4 (u4 / s4) asymmetric groupwise dequantization fused into
+    a bf16 matmul, forward and transposed ("Fused HQQ Quantization Gemm",
+    pytorch/ao PR 153, description and implementation details):
+    w = bf16(bf16(q - z) * s) per group of K.
 """
 import ctypes
 import os
@@ -64,6 +69,14 @@ def _load():
         lib.oracle_e4m3_to_double.restype = ctypes.c_double
         lib.oracle_float_to_e4m3.argtypes = [ctypes.c_float]
         lib.oracle_float_to_e4m3.restype = ctypes.c_uint8
+        Ci = ctypes.c_int
+        lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
+        lib.oracle_double_to_bf16.restype = ctypes.c_uint16
+        lib.oracle_hqq_pack.argtypes = [P, I, I, P]
+        lib.oracle_hqq_unpack.argtypes = [P, I, I, Ci, P]
+        lib.oracle_hqq_dequant.argtypes = [P, P, P, I, I, I, Ci, P]
+        lib.oracle_hqq_linear_f64.argtypes = [P, P, I, I, I, P]
+        lib.oracle_hqq_linear_t_f64.argtypes = [P, P, I, I, I, P]
         _lib = lib
     return _lib
 
@@ -234,4 +247,68 @@ def gemm_fp8_f64(A: np.ndarray, W: np.ndarray) -> np.ndarray:
     assert W.shape[1] == K
     out = np.empty((M, N), np.float64)
     _load().oracle_gemm_fp8_f64(_ptr(A), M, K, K, _ptr(W), N, K, _ptr(out))
+    return out
+
+
+def double_to_bf16(v: float) -> int:
+    """float64 -> bf16 bit pattern, one rounding to nearest even."""
+    return int(_load().oracle_double_to_bf16(float(v)))
+
+
+def hqq_pack(codes: np.ndarray) -> np.ndarray:
+    """int4 codes int8 [R, C] (u4 0..15 or s4 -8..7, C even) -> packed uint8 [R, C/2]:
+    byte j = code[2j] | code[2j+1] << 4 (nibbles, two's complement for s4)."""
+    c = _c(codes, np.int8)
+    R, C = c.shape
+    assert C % 2 == 0
+    out = np.empty((R, C // 2), np.uint8)
+    _load().oracle_hqq_pack(_ptr(c), R, C, _ptr(out))
+    return out
+
+
+def hqq_unpack(packed: np.ndarray, signed: bool = False) -> np.ndarray:
+    """packed uint8 [R, C/2] -> codes int8 [R, C]."""
+    p = _c(packed, np.uint8)
+    R, H = p.shape
+    out = np.empty((R, 2 * H), np.int8)
+    _load().oracle_hqq_unpack(_ptr(p), R, 2 * H, int(signed), _ptr(out))
+    return out
+
+
+def hqq_dequant(packed, scale_bits, zero_bits, group: int, signed: bool = False) -> np.ndarray:
+    """packed uint8 [N, K/2], scale / zero bf16 bits [N, K/group] -> w bf16 bits [N, K],
+    w = bf16(bf16(q - z) * s)."""
+    p = _c(packed, np.uint8)
+    N, H = p.shape
+    K = 2 * H
+    assert K % group == 0
+    sc = _c(scale_bits, np.uint16)
+    ze = _c(zero_bits, np.uint16)
+    assert sc.shape == (N, K // group) and ze.shape == (N, K // group)
+    w = np.empty((N, K), np.uint16)
+    _load().oracle_hqq_dequant(_ptr(p), _ptr(sc), _ptr(ze), N, K, group, int(signed), _ptr(w))
+    return w
+
+
+def hqq_linear_f64(x_bits, w_bits) -> np.ndarray:
+    """x bf16 [M, K], w bf16 [N, K] -> float64 [M, N] = x @ w^T (exact products, double sums)."""
+    x = _c(x_bits, np.uint16)
+    w = _c(w_bits, np.uint16)
+    M, K = x.shape
+    N = w.shape[0]
+    assert w.shape[1] == K
+    out = np.empty((M, N), np.float64)
+    _load().oracle_hqq_linear_f64(_ptr(x), _ptr(w), M, N, K, _ptr(out))
+    return out
+
+
+def hqq_linear_t_f64(y_bits, w_bits) -> np.ndarray:
+    """y bf16 [M, N], w bf16 [N, K] -> float64 [M, K] = y @ w (the transposed product)."""
+    y = _c(y_bits, np.uint16)
+    w = _c(w_bits, np.uint16)
+    M, N = y.shape
+    K = w.shape[1]
+    assert w.shape[0] == N
+    out = np.empty((M, K), np.float64)
+    _load().oracle_hqq_linear_t_f64(_ptr(y), _ptr(w), M, N, K, _ptr(out))
     return out

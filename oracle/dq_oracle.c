@@ -31,6 +31,10 @@
  *    product (PR 821 description and the vit_h_14 --bsr 64 benchmark
  *    command), plus the pack / densify conversions between a dense int8
  *    weight and its BSR form.
+ *  - Dynamic per-token FP8 (e4m3) quantization and the exact e4m3 product
+ *    (vLLM csrc/quantization commits), and the weight-only int4 groupwise
+ *    dequantization with its bf16 product ("Fused HQQ Quantization Gemm",
+ *    pytorch/ao PR 153); their readings are stated beside each section.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fwrapv -fPIC
  * -shared (see oracle/build.py).  -ffp-contract=off forbids FMA contraction
@@ -306,5 +310,126 @@ void oracle_gemm_fp8_f64(const uint8_t* A, int64_t M, int64_t K, int64_t lda,
             double s = 0.0;
             for (int64_t k = 0; k < K; ++k) s += lut[A[m * lda + k]] * lut[W[n * ldw + k]];
             acc[m * N + n] = s;
+        }
+}
+
+/* ---- weight-only int4, asymmetric, groupwise (HQQ) ---------------------
+ *
+ * "Fused HQQ Quantization Gemm" (pytorch/ao PR 153), description and
+ * implementation details: the weight of a linear layer is held as 4-bit
+ * codes (u4: 0..15, or s4: -8..7), quantized along the in-features (K, axis 1
+ * of the [N, K] weight) in groups of `group` consecutive values, each group
+ * of each output channel with its own bf16 scale and zero point; the fused
+ * kernel upcasts the codes to bf16, shifts them by the zero point and scales
+ * them, then multiplies with the bf16 activations.  Two codes share one byte
+ * (row interleave, no other preprocessing).
+ *
+ * Readings taken where the page is silent (each one stated here):
+ *   - dequantized weight w = bf16( bf16(q - z) * s ): the zero point is
+ *     subtracted first (the usual asymmetric definition, w = (q - z) * s) and
+ *     each of the two operations rounds once to bf16, to nearest even, as a
+ *     bf16 tensor expression does;
+ *   - packing: byte j of row r holds code (r, 2j) in bits 0..3 and code
+ *     (r, 2j + 1) in bits 4..7 (s4 codes as two's-complement nibbles), the
+ *     packed rows stored [N, K/2] like the weight's own rows;
+ *   - scales and zero points are [N, K/group] (channel, group), row-major;
+ *   - the product is the plain bf16 matmul of activations and dequantized
+ *     weight: out[m, n] = sum_k x[m, k] * w[n, k] (forward), and the
+ *     transposed product out[m, k] = sum_n y[m, n] * w[n, k] used for the
+ *     input gradient in the backward pass ("handles both transposed and
+ *     non-transposed quantized weights").
+ */
+
+/* Rounds a finite double to bf16 (8 significant bits), to nearest, ties to
+ * even, in one step (no intermediate rounding to fp32); overflow gives inf. */
+static uint16_t double_to_bf16_rne(double v) {
+    if (v == 0.0) return signbit(v) ? 0x8000u : 0x0000u;
+    if (isnan(v)) return 0x7fc0u;
+    if (isinf(v)) return v > 0 ? 0x7f80u : 0xff80u;
+    int e = ilogb(v);                       /* |v| in [2^e, 2^(e+1)) */
+    if (e < -126) e = -126;                 /* subnormal bf16: fixed quantum 2^-133 */
+    const double quantum = ldexp(1.0, e - 7);
+    const double r = nearbyint(v / quantum) * quantum;   /* exact scaling by 2^k */
+    if (fabs(r) >= ldexp(1.0, 128)) return v > 0 ? 0x7f80u : 0xff80u;
+    const float f = (float)r;               /* r has <= 8 significant bits: exact */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+uint16_t oracle_double_to_bf16(double v) {
+    fesetround(FE_TONEAREST);
+    return double_to_bf16_rne(v);
+}
+
+/* codes [rows, cols] (cols even; u4 0..15 or s4 -8..7) -> packed [rows, cols/2]. */
+void oracle_hqq_pack(const int8_t* codes, int64_t rows, int64_t cols, uint8_t* packed) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < cols / 2; ++j) {
+            const uint8_t lo = (uint8_t)codes[r * cols + 2 * j] & 0x0fu;
+            const uint8_t hi = (uint8_t)codes[r * cols + 2 * j + 1] & 0x0fu;
+            packed[r * (cols / 2) + j] = (uint8_t)(lo | (hi << 4));
+        }
+}
+
+static int nibble_code(uint8_t nib, int is_signed) {
+    return (is_signed && nib >= 8) ? (int)nib - 16 : (int)nib;
+}
+
+/* packed [rows, cols/2] -> codes [rows, cols]. */
+void oracle_hqq_unpack(const uint8_t* packed, int64_t rows, int64_t cols, int is_signed, int8_t* codes) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < cols; ++k) {
+            const uint8_t b = packed[r * (cols / 2) + k / 2];
+            const uint8_t nib = (k & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 0x0fu);
+            codes[r * cols + k] = (int8_t)nibble_code(nib, is_signed);
+        }
+}
+
+/* packed codes [N, K/2], scale / zero bf16 [N, K/group] -> w bf16 [N, K]:
+ * w[n, k] = bf16( bf16(q[n, k] - z[n, g]) * s[n, g] ), g = k / group.
+ * q - z is exact in double (an integer below 16 against 8 significant bits,
+ * the bf16 inputs kept away from the far ends of the exponent range) and a
+ * product of two bf16 values has at most 16 significant bits, so each
+ * double_to_bf16_rne rounds the exact result once. */
+void oracle_hqq_dequant(const uint8_t* packed, const uint16_t* scale, const uint16_t* zero,
+                        int64_t N, int64_t K, int64_t group, int is_signed, uint16_t* w) {
+    fesetround(FE_TONEAREST);
+    const int64_t G = K / group;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            const uint8_t b = packed[n * (K / 2) + k / 2];
+            const uint8_t nib = (k & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 0x0fu);
+            const double q = (double)nibble_code(nib, is_signed);
+            const double z = (double)bf16_bits_to_float(zero[n * G + k / group]);
+            const double s = (double)bf16_bits_to_float(scale[n * G + k / group]);
+            const uint16_t t = double_to_bf16_rne(q - z);
+            w[n * K + k] = double_to_bf16_rne((double)bf16_bits_to_float(t) * s);
+        }
+}
+
+/* out[m, n] = sum_k x[m, k] * w[n, k] in double (x [M, K], w [N, K], bf16).
+ * Each product of two bf16 values is exact in double; the sum rounds in
+ * double, an error far below that of any fp32 accumulation. */
+void oracle_hqq_linear_f64(const uint16_t* x, const uint16_t* w, int64_t M, int64_t N, int64_t K,
+                           double* out) {
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double s = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                s += (double)bf16_bits_to_float(x[m * K + k]) * (double)bf16_bits_to_float(w[n * K + k]);
+            out[m * N + n] = s;
+        }
+}
+
+/* Transposed product: out[m, k] = sum_n y[m, n] * w[n, k] (y [M, N], w [N, K]). */
+void oracle_hqq_linear_t_f64(const uint16_t* y, const uint16_t* w, int64_t M, int64_t N, int64_t K,
+                             double* out) {
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                s += (double)bf16_bits_to_float(y[m * N + n]) * (double)bf16_bits_to_float(w[n * K + k]);
+            out[m * K + k] = s;
         }
 }

@@ -148,3 +148,23 @@ def small_m(seed: int = 0, M: int = 16, K: int = 8192, N: int = 28672):
     return dict(name=f"small-M dense M={M} K={K} N={N}",
                 x=normal_bf16((M, K), 1.0, seed), w=normal_f32((N, K), 0.02, seed + 1),
                 bias=None)
+
+
+def hqq(seed: int = 0, M: int = 16, N: int = 4096, K: int = 4096, group: int = 128,
+        signed: bool = False):
+    """Weight-only int4 linear, the HQQ benchmark shapes (N = K = 4096, group
+    128, M from 16 to 1024): X bf16 [M, K] ~ N(0, 1); int4 codes int8 [N, K]
+    uniform over 0..15 (u4) or -8..7 (s4); per (channel, group) bf16 scales
+    uniform in [0.002, 0.02] and bf16 zero points uniform in [6, 9] (u4) or
+    [-1.5, 1.5] (s4), non-integer like HQQ's optimised zero points.  Codes
+    are unpacked: packing is part of the method.  Sub-seeds: X = seed, codes =
+    seed+1, scales = seed+5, zero points = seed+6."""
+    lo, hi = (-8, 7) if signed else (0, 15)
+    zlo, zhi = (-1.5, 1.5) if signed else (6.0, 9.0)
+    G = K // group
+    return dict(name=f"HQQ int4 linear M={M} N={N} K={K} group={group}{' s4' if signed else ''}",
+                x=normal_bf16((M, K), 1.0, seed),
+                codes=uniform_int8((N, K), lo, hi, seed + 1),
+                scale=f32_to_bf16_bits(uniform_f32((N, G), 0.002, 0.02, seed + 5)),
+                zero=f32_to_bf16_bits(uniform_f32((N, G), zlo, zhi, seed + 6)),
+                group=group, signed=signed)
