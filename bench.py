@@ -41,6 +41,11 @@ sys.path.insert(0, ROOT)
 METRIC = "int8 dyn-quant linear TOPS (dense & BSR) vs INT8 peak; quant kernel HBM GB/s"
 L2_BYTES = 126 * 1024 * 1024
 INT8_PER_BF16 = 2.0   # nominal dense int8 / bf16 tensor ratio (4.5 / 2.25 PFLOP/s)
+METRIC_HQQ = "int4 weight-only (HQQ) linear TFLOP/s, dequant fused into the bf16 GEMM"
+# The fused int4 kernel's published times at N = K = 4096, group 128, bf16
+# ("Fused HQQ Quantization Gemm", pytorch/ao PR 153, the H100 results table,
+# Triton column): ms by token count M.  Another machine's numbers: context.
+HQQ_PAGE_H100_MS = {16: 0.1678, 32: 0.1567, 128: 0.1607, 256: 0.1515, 512: 0.1477, 1024: 0.1585}
 
 
 # The CUDA sources each C-ABI entry point's kernels are compiled from (with
@@ -121,6 +126,20 @@ WORKLOADS = {
     "vit_fc1_dense": dict(kind="bsr_dense", layer="fc1", desc="ViT-H fc1 dense int8 twin M=65792 K=1280 N=5120"),
     "vit_fc2_dense": dict(kind="bsr_dense", layer="fc2", desc="ViT-H fc2 dense int8 twin M=65792 K=5120 N=1280"),
     "quant": dict(kind="quant", M=16384, K=8192, desc="standalone per-token quantize X bf16 [16384, 8192]"),
+    "hqq_m16": dict(kind="hqq", M=16, N=4096, K=4096, group=128,
+                    desc="weight-only int4 (HQQ u4, group 128) linear M=16 N=4096 K=4096, dequant fused into a bf16 GEMM"),
+    "hqq_m32": dict(kind="hqq", M=32, N=4096, K=4096, group=128,
+                    desc="weight-only int4 (HQQ u4, group 128) linear M=32 N=4096 K=4096, dequant fused into a bf16 GEMM"),
+    "hqq_m128": dict(kind="hqq", M=128, N=4096, K=4096, group=128,
+                    desc="weight-only int4 (HQQ u4, group 128) linear M=128 N=4096 K=4096, dequant fused into a bf16 GEMM"),
+    "hqq_m256": dict(kind="hqq", M=256, N=4096, K=4096, group=128,
+                    desc="weight-only int4 (HQQ u4, group 128) linear M=256 N=4096 K=4096, dequant fused into a bf16 GEMM"),
+    "hqq_m512": dict(kind="hqq", M=512, N=4096, K=4096, group=128,
+                    desc="weight-only int4 (HQQ u4, group 128) linear M=512 N=4096 K=4096, dequant fused into a bf16 GEMM"),
+    "hqq_m1024": dict(kind="hqq", M=1024, N=4096, K=4096, group=128,
+                    desc="weight-only int4 (HQQ u4, group 128) linear M=1024 N=4096 K=4096, dequant fused into a bf16 GEMM"),
+    "hqq_t_m1024": dict(kind="hqq", M=1024, N=4096, K=4096, group=128, transposed=True,
+                        desc="transposed int4 (HQQ u4, group 128) product M=1024 N=4096 K=4096 (input gradient)"),
     "small_m1": dict(kind="dense", M=1, K=8192, N=28672, desc="small-M dense linear M=1 K=8192 N=28672"),
     "small_m16": dict(kind="dense", M=16, K=8192, N=28672, desc="small-M dense linear M=16 K=8192 N=28672"),
     "small_m128": dict(kind="dense", M=128, K=8192, N=28672, desc="small-M dense linear M=128 K=8192 N=28672"),
@@ -147,6 +166,11 @@ def _synth_inputs(name, wl, seed):
         return synth.vit_h_bsr(seed, wl["layer"], keep=wl.get("keep", 0.10), bs=wl.get("bs", 64))
     if k == "quant":
         return synth.quant_sweep(seed)
+    if k == "hqq":
+        d = synth.hqq(seed, M=wl["M"], N=wl["N"], K=wl["K"], group=wl["group"])
+        if wl.get("transposed"):
+            d["x"] = synth.normal_bf16((wl["M"], wl["N"]), 1.0, seed)
+        return d
     return {}
 
 
@@ -171,6 +195,14 @@ def step_accounting(wl, d):
     if k == "quant":
         M, K = wl["M"], wl["K"]
         return 0.0, dict(kernel="dq_quantize_rows", ops=0.0, bytes=3 * M * K + 4 * M, quant_bytes=3 * M * K + 4 * M)
+    if k == "hqq":
+        M, K, N = wl["M"], wl["K"], wl["N"]
+        ops = 2.0 * M * N * K
+        n_in, n_out = (N, K) if wl.get("transposed") else (K, N)
+        # activations + packed codes + bf16 scale and zero per group + bf16 output
+        b = 2 * M * n_in + N * K // 2 + 2 * 2 * N * (K // wl["group"]) + 2 * M * n_out
+        return ops, dict(kernel="dq_hqq_linear_t" if wl.get("transposed") else "dq_hqq_linear", ops=ops, bytes=b,
+                         quant_bytes=0)
     return 0.0, {}
 
 
@@ -341,6 +373,27 @@ def make_state(name, wl, dq, torch, seed):
             lambda c, stream: dq.dq_quantize_rows(c["x"], q, s, stream=stream),
             lambda c, stream: dq.dq_int8_linear(q, s, c["W"], sc, bias=bias, out=out, workspace=ws, stream=stream)]
         st["names"] = ["dq_quantize_rows", "dq_int8_linear"]
+        return _finish(st)
+    if k == "hqq":
+        trans = bool(wl.get("transposed"))
+        M, K, N, group = wl["M"], wl["K"], wl["N"], wl["group"]
+        packed = dq.dq_hqq_pack(_to_dev(torch, d["codes"]))
+        sc, ze = _to_dev_bf16(torch, d["scale"]), _to_dev_bf16(torch, d["zero"])
+        x = _to_dev_bf16(torch, d["x"])
+        n = _ncopies(x.numel() * 2 + packed.numel() + 2 * sc.numel() * 2)
+        st["copies"] = [dict(x=x if i == 0 else x.clone(), P=packed if i == 0 else packed.clone(),
+                             S=sc if i == 0 else sc.clone(), Z=ze if i == 0 else ze.clone()) for i in range(n)]
+        n_out = K if trans else N
+        out = torch.empty((M, n_out), dtype=torch.bfloat16, device="cuda")
+        nws = dq.dq_hqq_workspace_size(M, N, K, trans)
+        ws = torch.zeros(nws, dtype=torch.uint8, device="cuda") if nws else None
+        st.update(out=out, ws=ws)
+        st["h2d"] = [("x", x.numel() * 2)]
+        st["d2h"] = [("out", M * n_out * 2)]
+        fn = dq.dq_hqq_linear_t if trans else dq.dq_hqq_linear
+        st["kernels"] = [lambda c, stream: fn(c["x"], c["P"], c["S"], c["Z"], group, out=out, workspace=ws,
+                                             stream=stream)]
+        st["names"] = ["dq_hqq_linear_t" if trans else "dq_hqq_linear"]
         return _finish(st)
     if k in ("bsr", "bsr_dense"):
         w = _to_dev(torch, d["w"])
@@ -514,6 +567,10 @@ def run_gpu(args, rank, world, local_rank):
         hbm_bound = False
     if dom["kernel"].startswith("dq_int8_linear") and wl["kind"] == "dense" and wl["M"] <= 128:
         hbm_bound = True     # small-M: weight streaming
+    hqq = wl["kind"] == "hqq"
+    if hqq:
+        int8_peak = peaks["bf16"]      # bf16 operands on the tensor cores
+        hbm_bound = dom["bytes"] / (peaks["hbm_gbs"] * 1e9) >= dom["ops"] / (int8_peak * 1e12)
     if hbm_bound:
         achieved = dom["bytes"] / (avg_ms * 1e-3) / 1e9
         roof = dict(bound="hbm", achieved=round(achieved, 1), peak=peaks["hbm_gbs"], unit="GB/s",
@@ -524,6 +581,8 @@ def run_gpu(args, rank, world, local_rank):
         roof = dict(bound="tensor", achieved=round(achieved, 1), peak=round(int8_peak, 1), unit="TOPS",
                     frac=round(achieved / int8_peak, 4), traffic=None,
                     peak_source=f"{peaks['src']} bf16 burst x {INT8_PER_BF16:g} (nominal int8/bf16 ratio)")
+        if hqq:
+            roof.update(unit="TFLOP/s", peak_source=f"{peaks['src']} bf16 burst (cuBLAS bf16 GEMM)")
     roof["kernel"] = dom["kernel"]
     roof["traffic"] = measured_traffic(name, dom["kernel"])
     roof["avg_launch_ms"] = round(avg_ms, 5)
@@ -532,12 +591,20 @@ def run_gpu(args, rank, world, local_rank):
 
     # end to end through the public API with host buffers
     e2e = None
-    if wl["kind"] in ("dense", "bsr", "bsr_dense", "quant", "gemm", "dense_fp8"):
+    if wl["kind"] in ("dense", "bsr", "bsr_dense", "quant", "gemm", "dense_fp8", "hqq"):
         e2e = run_e2e(args, wl, state, dq, torch, stream, ops, dom, world, max_over_ranks)
 
-    line = dict(metric=METRIC, value=round(value, 2) if value is not None else None, unit=unit, n_gpus=world,
+    vs_baseline = None
+    dtype = "e4m3" if wl["kind"] == "dense_fp8" else "int8"
+    metric = METRIC
+    if hqq:
+        unit, metric, dtype = "TFLOP/s", METRIC_HQQ, "bf16 (int4 weight)"
+        page_ms = HQQ_PAGE_H100_MS.get(wl["M"]) if not wl.get("transposed") else None
+        if page_ms:
+            vs_baseline = round(value / (ops / (page_ms * 1e-3) / 1e12), 2)
+    line = dict(metric=metric, value=round(value, 2) if value is not None else None, unit=unit, n_gpus=world,
                 steps=K, warmup=args.warmup, ms_per_step=round(total_ms_max / K, 5), higher_is_better=True,
-                scaling="weak", vs_baseline=None, dtype="e4m3" if wl["kind"] == "dense_fp8" else "int8",
+                scaling="weak", vs_baseline=vs_baseline, dtype=dtype,
                 data="synthetic",
                 config=dict(workload=wl["desc"], tokens_per_rank=state["d"].get("M", wl.get("M")),
                             parallelism=f"dp{world} (token rows sharded, weights replicated, no collective)",
@@ -549,7 +616,8 @@ def run_gpu(args, rank, world, local_rank):
                                    "read, pipelined on three streams (copy-in / kernels / copy-out)",
                             kernels_ms=kernels_ms),
                 roofline=roof, e2e=e2e, gpu_launches=nk * K, clocks=cs.summary())
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and wl["kind"] in ("dense", "bsr", "quant", "gemm"):
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and wl["kind"] in ("dense", "bsr", "quant", "gemm",
+                                                                                 "hqq"):
         line["cpu_baseline"] = cpu_baseline(name, wl, state["d"], budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -617,7 +685,8 @@ def run_e2e(args, wl, state, dq, torch, stream, ops, dom, world, max_over_ranks)
     if wl["kind"] == "quant":
         return dict(value=round(dom["bytes"] * world * K / (ms * 1e-3) / 1e9, 2), unit="GB/s",
                     h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, pipelined=True)
-    return dict(value=round(ops * world * K / (ms * 1e-3) / 1e12, 3), unit="TOPS",
+    return dict(value=round(ops * world * K / (ms * 1e-3) / 1e12, 3),
+                unit="TFLOP/s" if wl["kind"] == "hqq" else "TOPS",
                 h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, pipelined=True)
 
 
@@ -654,6 +723,15 @@ def _oracle_sample(name, wl, d, rows):
     if k == "quant":
         oracle.quantize_rows_bf16(d["x"][rows])
         return float(len(rows) * (3 * d["x"].shape[1] + 4))
+    if k == "hqq":
+        if "_w" not in d:
+            d["_w"] = oracle.hqq_dequant(oracle.hqq_pack(d["codes"]), d["scale"], d["zero"], d["group"],
+                                         signed=d["signed"])
+        if wl.get("transposed"):
+            oracle.hqq_linear_t_f64(d["x"][rows], d["_w"])
+        else:
+            oracle.hqq_linear_f64(d["x"][rows], d["_w"])
+        return 2.0 * len(rows) * wl["N"] * wl["K"]
     raise ValueError(k)
 
 
@@ -686,7 +764,7 @@ def cpu_baseline(name, wl, d, budget_s=12.0):
     if wl["kind"] == "quant":
         v, unit = units / dt / 1e9, "GB/s"
     else:
-        v, unit = units / dt / 1e12, "TOPS"
+        v, unit = units / dt / 1e12, "TFLOP/s" if wl["kind"] == "hqq" else "TOPS"
     return dict(value=round(v, 6), unit=unit, cores=1, kind="oracle",
                 sample=f"first {done} of {M} rows of the same workload, {dt:.1f} s single-threaded "
                        f"(host: {os.cpu_count()} logical cores, oracle uses 1)")
@@ -716,7 +794,7 @@ def run_reference(args, rank, world):
     if wl["kind"] == "quant":
         v, unit = units / dt / 1e9, "GB/s"
     else:
-        v, unit = units / dt / 1e12, "TOPS"
+        v, unit = units / dt / 1e12, "TFLOP/s" if wl["kind"] == "hqq" else "TOPS"
     sample = f"{chunk} rows per step (of {M}), single-threaded C oracle on the host"
     line = dict(impl="reference", metric=METRIC, value=round(v, 6), unit=unit, n_gpus=world, steps=args.steps,
                 warmup=args.warmup, ms_per_step=round(1e3 * dt / args.steps, 3), higher_is_better=True,

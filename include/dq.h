@@ -1,6 +1,7 @@
 /*
  * dq.h -- C ABI of libdq: the int8 dynamic-quantization linear layer on
- * NVIDIA B200 (sm_100a), dense and 64x64 block-sparse (BSR) weight.
+ * NVIDIA B200 (sm_100a), dense and block-sparse (BSR) weight, with its
+ * dynamic FP8 sibling and the weight-only int4 (HQQ) linear.
  *
  * The layer (pytorch/ao PR 821, "int8 dynamic quant + bsr support",
  * description and review) is
@@ -281,6 +282,62 @@ DQ_API dq_status dq_quantize_weight_fp8(const float* w, int64_t N, int64_t K, in
 DQ_API dq_status dq_fp8_linear(const uint8_t* A, const float* s_row, int64_t M, int64_t K, const uint8_t* W,
                                const float* s_col, int64_t N, const void* bias_bf16, void* out,
                                dq_out_dtype out_dtype, dq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Weight-only int4 linear with the groupwise asymmetric dequantization fused
+ * into a bf16 GEMM ("Fused HQQ Quantization Gemm", pytorch/ao PR 153,
+ * description and implementation details).
+ *
+ * Weight format (shared by every call below):
+ *   codes   q[n, k], n < N output channels, k < K in-features; u4 (0..15) or,
+ *           with DQ_HQQ_S4, s4 (-8..7);
+ *   packed  uint8 [N, K/2] row-major: byte j of row n = q[n, 2j] in bits
+ *           0..3 | q[n, 2j+1] in bits 4..7 (the page's "row interleave" of
+ *           two codes per byte along K; s4 as two's-complement nibbles);
+ *   scale, zero  bf16 [N, K/group] row-major (channel, group of `group`
+ *           consecutive k);
+ *   dequantized weight w[n, k] = bf16( bf16(q - zero[n, k/group]) *
+ *           scale[n, k/group] ), each operation rounded once to nearest even.
+ *
+ * dq_hqq_pack: codes int8 [rows, cols] (cols even; values must lie in the
+ *   u4 or s4 range, only the low 4 bits are kept) -> packed [rows, cols/2].
+ * dq_hqq_dequantize: packed, scale, zero -> w bf16 [N, K] (the standalone
+ *   dequantization; bit-exact).
+ * dq_hqq_linear (forward):   out[m, n] = sum_k x[m, k] * w[n, k],
+ *   x bf16 [M, K], out bf16 [M, N].
+ * dq_hqq_linear_t (transposed, for the input gradient of the backward pass):
+ *   out[m, k] = sum_n y[m, n] * w[n, k],  y bf16 [M, N], out bf16 [M, K].
+ * Both run on the tensor cores (tcgen05.mma kind::f16, bf16 operands, fp32
+ * accumulator in TMEM); the int4 weight is dequantized in shared memory by
+ * the GEMM kernel itself and never exists as a bf16 matrix in global memory.
+ * Every bf16 x bf16 product is exact in fp32; the order of the fp32 sum is
+ * the hardware's (deterministic for a given shape and workspace), so results
+ * are compared with the exact sum within a bound, not bit for bit.
+ *
+ * Requirements: group in {32, 64, 128, 256}; K % group == 0; N % 8 == 0;
+ * M >= 0 (M == 0 launches nothing); all pointers 16-byte aligned.
+ * workspace: optional caller-owned device scratch that lets few-token calls
+ * split the contraction over more SMs (the split partial sums are added in
+ * a fixed order, so results do not depend on timing).  Its usable size is
+ * dq_hqq_workspace_size(); NULL or a smaller buffer disables splitting.  It
+ * must be ZERO-FILLED before its first use; every call leaves it zeroed again
+ * (unless a call reports DQ_ERR_TIMEOUT, after which it must be re-zeroed).
+ * Calls that may run at the same time must not share a workspace.
+ * ------------------------------------------------------------------------ */
+enum { DQ_HQQ_S4 = 1 };
+
+DQ_API dq_status dq_hqq_pack(const int8_t* codes, int64_t rows, int64_t cols, uint8_t* packed,
+                             dq_stream_t stream);
+DQ_API dq_status dq_hqq_dequantize(const uint8_t* packed, const void* scale_bf16, const void* zero_bf16,
+                                   int64_t N, int64_t K, int group, int flags, void* w_bf16,
+                                   dq_stream_t stream);
+DQ_API size_t dq_hqq_workspace_size(int64_t M, int64_t N, int64_t K, int transposed);
+DQ_API dq_status dq_hqq_linear(const void* x_bf16, int64_t M, const uint8_t* packed, const void* scale_bf16,
+                               const void* zero_bf16, int64_t N, int64_t K, int group, int flags,
+                               void* out_bf16, void* workspace, size_t workspace_bytes, dq_stream_t stream);
+DQ_API dq_status dq_hqq_linear_t(const void* y_bf16, int64_t M, const uint8_t* packed, const void* scale_bf16,
+                                 const void* zero_bf16, int64_t N, int64_t K, int group, int flags,
+                                 void* out_bf16, void* workspace, size_t workspace_bytes, dq_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Measurement helper: a kernel that only issues tcgen05.mma.kind::i8

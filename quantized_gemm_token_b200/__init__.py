@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libdq.so")
 
 DQ_OK, DQ_ERR_INVALID_ARG, DQ_ERR_UNSUPPORTED, DQ_ERR_CUDA, DQ_ERR_TIMEOUT = range(5)
 DQ_OUT_BF16, DQ_OUT_S32, DQ_OUT_F32 = 0, 1, 2
+DQ_HQQ_S4 = 1
 
 # C prototypes: (name, restype, argtypes)
 _P, _I64, _I32, _SZ, _U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
@@ -52,6 +53,11 @@ _PROTOS = {
     "dq_debug_set_two_widths": (None, [_I32]),
     "dq_debug_set_bsr_panel": (None, [_I32]),
     "dq_debug_set_quant_kernel": (None, [_I32]),
+    "dq_hqq_pack": (_I32, [_P, _I64, _I64, _P, _P]),
+    "dq_hqq_dequantize": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I32, _P, _P]),
+    "dq_hqq_workspace_size": (_SZ, [_I64, _I64, _I64, _I32]),
+    "dq_hqq_linear": (_I32, [_P, _I64, _P, _P, _P, _I64, _I64, _I32, _I32, _P, _P, _SZ, _P]),
+    "dq_hqq_linear_t": (_I32, [_P, _I64, _P, _P, _P, _I64, _I64, _I32, _I32, _P, _P, _SZ, _P]),
 }
 
 
@@ -403,6 +409,125 @@ def dq_bsr_validate(crow, col, N: int, K: int, block: int = 64) -> int:
 
 def dq_mma_peak_probe(grid: int, iters: int, stream=None) -> None:
     _check(lib.dq_mma_peak_probe(grid, iters, _stream(stream)), "dq_mma_peak_probe")
+
+
+# ---------------------------------------------------------------- int4 (HQQ)
+
+def dq_hqq_pack(codes: torch.Tensor, packed: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """int4 codes int8 [R, C] (u4 0..15 or s4 -8..7) -> packed uint8 [R, C/2]
+    (byte j = code 2j | code 2j+1 << 4)."""
+    _need(codes, torch.int8, "codes", 2)
+    _contig(codes, "codes")
+    R, C = codes.shape
+    if packed is None:
+        packed = torch.empty((R, C // 2), dtype=torch.uint8, device=codes.device)
+    _need(packed, torch.uint8, "packed", 2)
+    _contig(packed, "packed")
+    if tuple(packed.shape) != (R, C // 2):
+        raise ValueError("packed must be [R, C/2]")
+    _check(lib.dq_hqq_pack(_ptr(codes), R, C, _ptr(packed), _stream(stream)), "dq_hqq_pack")
+    return packed
+
+
+def _hqq_weights(packed, scale, zero, group):
+    _need(packed, torch.uint8, "packed", 2)
+    _need(scale, torch.bfloat16, "scale", 2)
+    _need(zero, torch.bfloat16, "zero", 2)
+    for t, n in ((packed, "packed"), (scale, "scale"), (zero, "zero")):
+        _contig(t, n)
+    N, K = packed.shape[0], packed.shape[1] * 2
+    if group <= 0 or K % group != 0:
+        raise ValueError("group must divide K")
+    if tuple(scale.shape) != (N, K // group) or tuple(zero.shape) != (N, K // group):
+        raise ValueError("scale and zero must be [N, K/group]")
+    return N, K
+
+
+def dq_hqq_dequantize(packed, scale, zero, group: int, signed: bool = False, out=None, stream=None):
+    """w bf16 [N, K] = bf16(bf16(q - zero) * scale), per group of K."""
+    N, K = _hqq_weights(packed, scale, zero, group)
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device)
+    _need(out, torch.bfloat16, "out", 2)
+    _contig(out, "out")
+    _check(lib.dq_hqq_dequantize(_ptr(packed), _ptr(scale), _ptr(zero), N, K, group,
+                                 DQ_HQQ_S4 if signed else 0, _ptr(out), _stream(stream)), "dq_hqq_dequantize")
+    return out
+
+
+def dq_hqq_workspace_size(M: int, N: int, K: int, transposed: bool = False) -> int:
+    return int(lib.dq_hqq_workspace_size(M, N, K, int(transposed)))
+
+
+def _hqq_call(fn, name, x, packed, scale, zero, group, signed, out, workspace, stream, transposed):
+    N, K = _hqq_weights(packed, scale, zero, group)
+    _need(x, torch.bfloat16, "x", 2)
+    _contig(x, "x")
+    M = x.shape[0]
+    if x.shape[1] != (N if transposed else K):
+        raise ValueError("activation width does not match the weight")
+    n_out = K if transposed else N
+    if out is None:
+        out = torch.empty((M, n_out), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out", 2)
+    _contig(out, "out")
+    if tuple(out.shape) != (M, n_out):
+        raise ValueError("out shape")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _need(workspace, torch.uint8, "workspace")
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()
+    _check(fn(_ptr(x), M, _ptr(packed), _ptr(scale), _ptr(zero), N, K, group, DQ_HQQ_S4 if signed else 0,
+              _ptr(out), ws_ptr, ws_bytes, _stream(stream)), name)
+    return out
+
+
+def dq_hqq_linear(x, packed, scale, zero, group: int, signed: bool = False, out=None, workspace=None,
+                  stream=None):
+    """out[M, N] = x[M, K] @ w^T with w the dequantized int4 weight [N, K]
+    (dequantization fused into the tensor-core GEMM).  `workspace`: optional
+    zero-filled uint8 CUDA tensor (dq_hqq_workspace_size) for few-token calls."""
+    return _hqq_call(lib.dq_hqq_linear, "dq_hqq_linear", x, packed, scale, zero, group, signed, out,
+                     workspace, stream, False)
+
+
+def dq_hqq_linear_t(y, packed, scale, zero, group: int, signed: bool = False, out=None, workspace=None,
+                    stream=None):
+    """out[M, K] = y[M, N] @ w (the transposed product, for the input gradient)."""
+    return _hqq_call(lib.dq_hqq_linear_t, "dq_hqq_linear_t", y, packed, scale, zero, group, signed, out,
+                     workspace, stream, True)
+
+
+class HqqLinear:
+    """Weight-only int4 linear: packed u4 / s4 codes with bf16 scale and zero
+    point per group of in-features.  forward(x) = x @ w^T, backward_input(g)
+    = g @ w; the workspace for few-token calls is kept per token count."""
+
+    def __init__(self, packed, scale, zero, group: int, signed: bool = False):
+        self.packed, self.scale, self.zero, self.group, self.signed = packed, scale, zero, group, signed
+        self.N, self.K = packed.shape[0], packed.shape[1] * 2
+        self._ws = {}
+
+    @classmethod
+    def from_codes(cls, codes: torch.Tensor, scale, zero, group: int, signed: bool = False):
+        return cls(dq_hqq_pack(codes), scale, zero, group, signed)
+
+    def _workspace(self, M, transposed, device):
+        key = (M, transposed)
+        if key not in self._ws:
+            n = dq_hqq_workspace_size(M, self.N, self.K, transposed)
+            self._ws[key] = torch.zeros((n,), dtype=torch.uint8, device=device) if n else None
+        return self._ws[key]
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor = None, stream=None):
+        ws = self._workspace(x.shape[0], False, x.device)
+        return dq_hqq_linear(x, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
+                             workspace=ws, stream=stream)
+
+    def backward_input(self, grad_out: torch.Tensor, out: torch.Tensor = None, stream=None):
+        ws = self._workspace(grad_out.shape[0], True, grad_out.device)
+        return dq_hqq_linear_t(grad_out, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
+                               workspace=ws, stream=stream)
 
 
 # ---------------------------------------------------------------- layer

@@ -1,0 +1,750 @@
+// hqq.cu -- weight-only int4 linear with the groupwise asymmetric
+// dequantization fused into a bf16 tensor-core GEMM ("Fused HQQ Quantization
+// Gemm", pytorch/ao PR 153: u4 / s4 codes are upcast to bf16, shifted by a
+// zero point and scaled per group of in-features, then multiplied with the
+// activations; forward and transposed products), plus the standalone
+// dequantization and the packing of codes two to a byte.
+//
+// One persistent, warp-specialised kernel for sm_100a (448 threads):
+//   warp 0       TMA producer: for each 64-deep contraction step, the packed
+//                int4 weight tile (4 KB) and the activation tile (BN tokens x
+//                64 bf16, 128B-swizzled) into a ring of NP stages.
+//   warp 1       MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in
+//                TMEM), M = 128 weight rows, N = BN tokens, K = 16 per
+//                instruction, four instructions per step.
+//   warps 2..9   dequantizers: unpack the codes, w = bf16(bf16(q - z) * s)
+//                in packed bf16x2 arithmetic, and write the 128 x 64 bf16 A
+//                operand in the 128B-swizzled K-major layout into a ring of
+//                ND stages (the bf16 weight never reaches global memory).
+//   warps 10..13 epilogue: tcgen05.ld the accumulator (TMEM lane = output
+//                channel, column = token), convert to bf16 and store.
+// The weight is the A operand (128 output channels per tile) and the tokens
+// the B operand (up to 256): the dequantization work per MMA flop is then as
+// small as a 128-row tile allows, and few-token calls need no padding to 128.
+// Few tiles: the contraction is split over S CTAs per tile; each split
+// writes an fp32 partial tile to a workspace and the last split to arrive
+// (an arrival counter per 32-channel slice) adds the S partials in split
+// order, so the result does not depend on timing.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace dq {
+namespace {
+
+constexpr int HQ_THREADS = 448;
+constexpr int HQ_DEQ_WARPS = 8;            // warps 2..9
+constexpr int HQ_EPI_WARP0 = 10;           // warps 10..13
+constexpr int HQ_BK = 64;                  // contraction elements per step (128 B of bf16)
+constexpr int HQ_A_BYTES = 128 * 128;      // dequantized weight tile: 128 rows x 128 B
+constexpr int HQ_W_BYTES = 4096;           // packed int4 tile per step
+constexpr int HQ_ND = 4;                   // dequantized-tile ring
+constexpr int HQ_MAX_NP = 16;
+constexpr int HQ_ACC_COLS = 256;           // TMEM columns per accumulator buffer
+constexpr int HQ_TMEM_COLS = 512;          // two accumulator buffers
+constexpr int HQ_SMEM_LIMIT = 227 * 1024;
+constexpr int HQ_BAR_BYTES = 1024;
+
+struct HqqArgs {
+  int M;                  // tokens
+  int n_out;              // output channels (N forward, K transposed)
+  int kc;                 // contraction length (K forward, N transposed)
+  int n_w, k_w;           // weight rows (N) and in-features (K)
+  int group, n_groups;    // group size and K / group
+  int bn;                 // tokens per tile (multiple of 16, <= 256)
+  int nt, tt;             // channel tiles (128 each), token tiles (bn each)
+  int splits;             // contraction splits per tile
+  int ks;                 // contraction steps per tile (ceil(kc / 64))
+  int units;              // nt * tt * splits
+  int np;                 // packed / activation ring stages
+  uint32_t off_x, off_w, off_bar;   // shared-memory offsets (A ring at 0)
+  const uint16_t* scale;
+  const uint16_t* zero;
+  uint16_t* out;          // bf16 [M, n_out]
+  float* ws;              // split partials: [tile][split][bn][128] fp32
+  uint32_t* cnt;          // arrival counters: [tile][4]
+  WaitCtl wait;
+};
+
+// bf16x2 arithmetic, each lane rounded once to nearest even (sm_90+ PTX).
+__device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// bf16 bit patterns of 128 + c for a code nibble c put in the low mantissa
+// bits (exact: the bf16 spacing at 128 is 1).  s4 codes are first offset by
+// 8 (nibble ^ 8 = c + 8), so the exact subtraction takes 136 instead.
+template <bool S4>
+__device__ __forceinline__ uint32_t code_bias2() {
+  return S4 ? 0x43084308u : 0x43004300u;
+}
+
+// Dequantizes the eight codes of one packed word (byte j = codes 2j, 2j+1
+// in its low / high nibble) sharing one zero point and one scale (z2, s2:
+// the bf16 pattern in both halves).  o[i] = bf16 pair (code 2i, code 2i+1).
+template <bool S4>
+__device__ __forceinline__ void dequant8(uint32_t w, uint32_t z2, uint32_t s2, uint32_t (&o)[4]) {
+  if (S4) w ^= 0x88888888u;
+  // nibbles at bit 0 and bit 16 of each shifted copy: codes (0,4) (1,5) (2,6) (3,7)
+  uint32_t d[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t p = ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+    const uint32_t q = bsub2(p, code_bias2<S4>());          // exact: the codes as bf16
+    d[i] = bmul2(bsub2(q, z2), s2);                         // bf16(bf16(q - z) * s)
+  }
+  o[0] = __byte_perm(d[0], d[1], 0x5410);   // codes 0, 1
+  o[1] = __byte_perm(d[2], d[3], 0x5410);   // codes 2, 3
+  o[2] = __byte_perm(d[0], d[1], 0x7632);   // codes 4, 5
+  o[3] = __byte_perm(d[2], d[3], 0x7632);   // codes 6, 7
+}
+
+__device__ __forceinline__ uint32_t bf16_pair_of(uint16_t v) {
+  return static_cast<uint32_t>(v) | (static_cast<uint32_t>(v) << 16);
+}
+
+// Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128B-swizzled
+// K-major tile (rows of 128 B; the chunk index is XORed with r mod 8, the
+// layout a SWIZZLE_128B tensor copy produces).
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&v)[4]) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3])
+               : "memory");
+}
+
+// Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulator,
+// both operands K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4)                                 // D format: f32
+         | (1u << 7) | (1u << 10)                  // A, B format: bf16
+         | (static_cast<uint32_t>(N >> 3) << 17)   // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Forward: 256 threads turn the packed tile (128 channel rows x 32 B = 64
+// codes) into the 128 x 64 bf16 A tile.  Thread t: row t % 128, codes
+// 32 * (t / 128) .. +31 (one group: group sizes are >= 32).
+template <bool S4>
+__device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t wtile, uint32_t atile,
+                                                 const uint8_t* wtile_ptr, int dt, int ntile, int kstep) {
+  const int r = dt & 127;
+  const int h = dt >> 7;
+  const uint4 pk = *reinterpret_cast<const uint4*>(wtile_ptr + r * 32 + h * 16);
+  const int n = ntile * 128 + r;
+  const int k = kstep * HQ_BK + h * 32;
+  uint32_t s2 = 0, z2 = 0;
+  if (n < g.n_w && k < g.k_w) {
+    const int64_t gi = static_cast<int64_t>(n) * g.n_groups + k / g.group;
+    s2 = bf16_pair_of(__ldg(g.scale + gi));
+    z2 = bf16_pair_of(__ldg(g.zero + gi));
+  }
+  const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t o[4];
+    dequant8<S4>(words[i], z2, s2, o);
+    st_shared_v4(atile + sw128_off(r, 4 * h + i), o);
+  }
+  (void)wtile;
+}
+
+// Transposed: the packed tile holds 64 contraction rows (weight rows n) x
+// 64 B (128 output channels k, two per byte); the A tile is 128 rows (k) x
+// 64 bf16 (n).  Warp w handles n = 8w .. 8w+7; lane l the byte columns l and
+// l + 32 (A rows 2l, 2l+1 and 2l+64, 2l+65): eight bytes from eight weight
+// rows give two 16-byte chunks, one per A row.
+template <bool S4>
+__device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile, const uint8_t* wtile_ptr,
+                                               int dt, int ntile, int kstep) {
+  const int nc = dt >> 5;       // n chunk (8 weight rows)
+  const int lane = dt & 31;
+  const int n0 = kstep * HQ_BK + nc * 8;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int b = lane + 32 * u;                 // byte column: k = 2b, 2b + 1 in the tile
+    const int k = ntile * 128 + 2 * b;
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // weight rows n0 + 2i and n0 + 2i + 1
+      const uint32_t b0 = wtile_ptr[(nc * 8 + 2 * i) * 64 + b];
+      const uint32_t b1 = wtile_ptr[(nc * 8 + 2 * i + 1) * 64 + b];
+      uint32_t x = b0 | (b1 << 16);
+      if (S4) x ^= 0x00880088u;
+      uint32_t s2 = 0, z2 = 0;
+      const int na = n0 + 2 * i, nb = na + 1;
+      if (k < g.k_w) {
+        const int gk = k / g.group;
+        const uint32_t sa = na < g.n_w ? __ldg(g.scale + static_cast<int64_t>(na) * g.n_groups + gk) : 0u;
+        const uint32_t sb = nb < g.n_w ? __ldg(g.scale + static_cast<int64_t>(nb) * g.n_groups + gk) : 0u;
+        const uint32_t za = na < g.n_w ? __ldg(g.zero + static_cast<int64_t>(na) * g.n_groups + gk) : 0u;
+        const uint32_t zb = nb < g.n_w ? __ldg(g.zero + static_cast<int64_t>(nb) * g.n_groups + gk) : 0u;
+        s2 = sa | (sb << 16);
+        z2 = za | (zb << 16);
+      }
+      const uint32_t pl = (x & 0x000F000Fu) | 0x43004300u;          // k = 2b: rows na, nb
+      const uint32_t ph = ((x >> 4) & 0x000F000Fu) | 0x43004300u;   // k = 2b + 1
+      lo[i] = bmul2(bsub2(bsub2(pl, code_bias2<S4>()), z2), s2);
+      hi[i] = bmul2(bsub2(bsub2(ph, code_bias2<S4>()), z2), s2);
+    }
+    st_shared_v4(atile + sw128_off(2 * b, nc), lo);
+    st_shared_v4(atile + sw128_off(2 * b + 1, nc), hi);
+  }
+}
+
+struct Unit {
+  int tile, split, ntile, ttile, k0, k1;
+};
+
+// Work unit u: tile = u / splits (channel tile major, token tile minor),
+// contraction steps [k0, k1) of split u % splits.
+__device__ __forceinline__ Unit decode_unit(const HqqArgs& g, int u) {
+  Unit t;
+  t.tile = u / g.splits;
+  t.split = u - t.tile * g.splits;
+  t.ntile = t.tile / g.tt;
+  t.ttile = t.tile - t.ntile * g.tt;
+  t.k0 = static_cast<int>(static_cast<int64_t>(t.split) * g.ks / g.splits);
+  t.k1 = static_cast<int>(static_cast<int64_t>(t.split + 1) * g.ks / g.splits);
+  return t;
+}
+
+__device__ __forceinline__ uint32_t bf16_bits(float f) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+}
+
+// Stores `width` (16 or 32) tokens of one output channel per lane as bf16:
+// lanes exchange values in pairs so that each lane writes two neighbouring
+// channels of one token (4 bytes; a warp covers 64 contiguous bytes).
+__device__ __forceinline__ void store_pairs(const HqqArgs& g, const uint32_t (&r)[32], int width, int tok0,
+                                            int ch, int lane) {
+  const bool odd = lane & 1;
+  const int ch_even = ch & ~1;
+  const bool ch_ok = ch < g.n_out;     // n_out is even: same answer for both lanes of a pair
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    if (j < width) {
+      const uint32_t h0 = bf16_bits(__uint_as_float(r[j]));
+      const uint32_t h1 = bf16_bits(__uint_as_float(r[j + 1]));
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, odd ? h0 : h1, 1);
+      const int tok = tok0 + j + (odd ? 1 : 0);
+      const uint32_t v = odd ? (recv | (h1 << 16)) : (h0 | (recv << 16));
+      if (ch_ok && tok < g.M)
+        *reinterpret_cast<uint32_t*>(g.out + static_cast<int64_t>(tok) * g.n_out + ch_even) = v;
+    }
+  }
+}
+
+template <bool TRANS, bool S4>
+__global__ void __launch_bounds__(HQ_THREADS, 1)
+    hqq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                    const HqqArgs g) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const smem = smem_raw + (base - raw);
+  const uint32_t sA = base;                 // HQ_ND dequantized tiles
+  const uint32_t sX = base + g.off_x;       // np activation tiles (bn x 128 B)
+  const uint32_t sW = base + g.off_w;       // np packed weight tiles
+  const uint8_t* const sW_ptr = smem + g.off_w;
+  uint64_t* const p_full = reinterpret_cast<uint64_t*>(smem + g.off_bar);
+  uint64_t* const p_empty = p_full + HQ_MAX_NP;
+  uint64_t* const d_full = p_empty + HQ_MAX_NP;
+  uint64_t* const d_empty = d_full + HQ_ND;
+  uint64_t* const accf = d_empty + HQ_ND;
+  uint64_t* const acce = accf + 2;
+  uint64_t* const drain = acce + 2;
+  uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < g.np; ++i) {
+      mbar_init(smem_u32(p_full + i), 1);
+      mbar_init(smem_u32(p_empty + i), 1);
+    }
+    for (int i = 0; i < HQ_ND; ++i) {
+      mbar_init(smem_u32(d_full + i), HQ_DEQ_WARPS);
+      mbar_init(smem_u32(d_empty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(accf + i), 1);
+      mbar_init(smem_u32(acce + i), 4);
+    }
+    mbar_init(smem_u32(drain), 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), HQ_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint32_t x_bytes = static_cast<uint32_t>(g.bn) * 128u;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      const uint32_t tx = x_bytes + HQ_W_BYTES;
+      for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
+        const Unit t = decode_unit(g, u);
+        for (int kk = t.k0; kk < t.k1; ++kk) {
+          if (!mbar_wait(smem_u32(p_empty + stage), phase ^ 1, g.wait, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(p_full + stage);
+          mbar_arrive_expect_tx(fb, tx);
+          tma_load_2d(sX + stage * x_bytes, &tm_x, fb, kk * 128, t.ttile * g.bn);
+          if (TRANS)
+            tma_load_2d(sW + stage * HQ_W_BYTES, &tm_w, fb, t.ntile * 64, kk * HQ_BK);
+          else
+            tma_load_2d(sW + stage * HQ_W_BYTES, &tm_w, fb, kk * 32, t.ntile * 128);
+          ++issued;
+          if (++stage == g.np) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // every copy issued lands before the CTA can exit
+      volatile int never = 0;
+      for (long long i = issued > g.np ? issued - g.np : 0; i < issued; ++i)
+        mbar_wait(smem_u32(p_full + static_cast<int>(i % g.np)), static_cast<uint32_t>((i / g.np) & 1), g.wait,
+                  &never);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, g.bn);
+      int stage = 0, dst = 0, acc = 0;
+      uint32_t phase = 0, dphase = 0, aphase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
+        const Unit t = decode_unit(g, u);
+        if (!mbar_wait(smem_u32(acce + acc), aphase ^ 1, g.wait, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * HQ_ACC_COLS);
+        for (int kk = t.k0; kk < t.k1; ++kk) {
+          if (!mbar_wait(smem_u32(d_full + dst), dphase, g.wait, abort_flag) ||
+              !mbar_wait(smem_u32(p_full + stage), phase, g.wait, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = smem_desc_kmajor<128>(sA + dst * HQ_A_BYTES);
+          const uint64_t bd = smem_desc_kmajor<128>(sX + stage * x_bytes);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)   // K = 16 bf16 = 32 bytes per instruction
+            mma_bf16(d_tmem, ad + 2 * j, bd + 2 * j, idesc, (kk > t.k0 || j > 0) ? 1u : 0u);
+          mma_commit(smem_u32(p_empty + stage));
+          mma_commit(smem_u32(d_empty + dst));
+          if (++stage == g.np) {
+            stage = 0;
+            phase ^= 1;
+          }
+          if (++dst == HQ_ND) {
+            dst = 0;
+            dphase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(accf + acc));
+        if (++acc == 2) {
+          acc = 0;
+          aphase ^= 1;
+        }
+      }
+      // every MMA issued has completed once drain flips
+      mma_commit(smem_u32(drain));
+      volatile int never = 0;
+      mbar_wait(smem_u32(drain), 0, g.wait, &never);
+    }
+  } else if (warp < HQ_EPI_WARP0) {
+    // ---------------------------------------------------------- dequantizers
+    const int dt = threadIdx.x - 64;
+    int stage = 0, dst = 0;
+    uint32_t phase = 0, dphase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
+      const Unit t = decode_unit(g, u);
+      for (int kk = t.k0; kk < t.k1; ++kk) {
+        bool w = mbar_wait(smem_u32(p_full + stage), phase, g.wait, abort_flag);
+        w = w && mbar_wait(smem_u32(d_empty + dst), dphase ^ 1, g.wait, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        const uint32_t atile = sA + dst * HQ_A_BYTES;
+        const uint8_t* wp = sW_ptr + stage * HQ_W_BYTES;
+        if (TRANS)
+          dequant_tile_t<S4>(g, atile, wp, dt, t.ntile, kk);
+        else
+          dequant_tile_fwd<S4>(g, sW + stage * HQ_W_BYTES, atile, wp, dt, t.ntile, kk);
+        fence_proxy_async_smem();     // generic-proxy writes -> visible to the MMA
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(d_full + dst));
+        if (++stage == g.np) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (++dst == HQ_ND) {
+          dst = 0;
+          dphase ^= 1;
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q = warp & 3;                 // TMEM sub-partition of this warp
+    const int row = q * 32 + lane;          // accumulator row = output channel in the tile
+    int acc = 0;
+    uint32_t aphase = 0;
+    for (int u = blockIdx.x; u < g.units; u += gridDim.x) {
+      const Unit t = decode_unit(g, u);
+      const bool w = mbar_wait(smem_u32(accf + acc), aphase, g.wait, abort_flag);
+      if (!__all_sync(0xffffffffu, w)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * HQ_ACC_COLS);
+      const int ch = t.ntile * 128 + row;
+      const int tok0 = t.ttile * g.bn;
+      float* const part =
+          g.splits > 1 ? g.ws + static_cast<int64_t>(t.tile * g.splits + t.split) * g.bn * 128 : nullptr;
+      for (int c0 = 0; c0 < g.bn; c0 += 32) {
+        const int width = min(32, g.bn - c0);
+        uint32_t r[32];
+        if (width == 32) {
+          tmem_ld_32x32b_x32(tb + c0, r);
+        } else {
+          uint32_t r16[16];
+          tmem_ld_32x32b_x16(tb + c0, r16);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) r[j] = r16[j];
+#pragma unroll
+          for (int j = 16; j < 32; ++j) r[j] = 0;
+        }
+        tmem_ld_wait();
+        if (part != nullptr) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < width) part[static_cast<int64_t>(c0 + j) * 128 + row] = __uint_as_float(r[j]);
+        } else {
+          store_pairs(g, r, width, tok0 + c0, ch, lane);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(acce + acc));
+      if (++acc == 2) {
+        acc = 0;
+        aphase ^= 1;
+      }
+      if (part != nullptr) {
+        // publish this split's slice; the last split to arrive adds all of
+        // them in split order
+        __threadfence();
+        __syncwarp();
+        uint32_t last = 0;
+        if (lane == 0)
+          last = atomicAdd(g.cnt + t.tile * 4 + q, 1u) == static_cast<uint32_t>(g.splits - 1) ? 1u : 0u;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          const float* const tile_ws = g.ws + static_cast<int64_t>(t.tile) * g.splits * g.bn * 128;
+          for (int c0 = 0; c0 < g.bn; c0 += 32) {
+            const int width = min(32, g.bn - c0);
+            uint32_t r[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              float acc_sum = 0.0f;
+              if (j < width)
+                for (int sp = 0; sp < g.splits; ++sp)
+                  acc_sum += __ldcg(tile_ws + (static_cast<int64_t>(sp) * g.bn + c0 + j) * 128 + row);
+              r[j] = __float_as_uint(acc_sum);
+            }
+            store_pairs(g, r, width, tok0 + c0, ch, lane);
+          }
+          __syncwarp();
+          if (lane == 0) g.cnt[t.tile * 4 + q] = 0u;   // the workspace is left zeroed
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, HQ_TMEM_COLS);
+}
+
+// Standalone dequantization: one thread per packed word (8 codes) -> 16 B of bf16.
+template <bool S4>
+__global__ void __launch_bounds__(256) hqq_dequant_kernel(const uint32_t* __restrict__ packed,
+                                                          const uint16_t* __restrict__ scale,
+                                                          const uint16_t* __restrict__ zero, int64_t N,
+                                                          int64_t K, int group, uint16_t* __restrict__ w) {
+  const int64_t words_per_row = K / 8;
+  const int64_t total = N * words_per_row;
+  const int64_t G = K / group;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / words_per_row;
+    const int64_t k = (i - n * words_per_row) * 8;
+    const int64_t gi = n * G + k / group;
+    uint32_t o[4];
+    dequant8<S4>(__ldg(packed + i), bf16_pair_of(__ldg(zero + gi)), bf16_pair_of(__ldg(scale + gi)), o);
+    *reinterpret_cast<uint4*>(w + n * K + k) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+__global__ void __launch_bounds__(256) hqq_pack_kernel(const int8_t* __restrict__ codes, int64_t n_bytes,
+                                                       uint8_t* __restrict__ packed) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_bytes;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t lo = static_cast<uint8_t>(codes[2 * i]) & 0x0Fu;
+    const uint32_t hi = static_cast<uint8_t>(codes[2 * i + 1]) & 0x0Fu;
+    packed[i] = static_cast<uint8_t>(lo | (hi << 4));
+  }
+}
+
+}  // namespace
+}  // namespace dq
+
+// ---------------------------------------------------------------- host side
+
+namespace dq {
+namespace {
+
+struct HqqPlan {
+  int bn, tt, nt, ks, splits, units, grid, np;
+  size_t cnt_bytes, ws_bytes, smem;
+};
+
+// Tiles: 128 output channels x bn tokens, bn = the token count split evenly
+// over ceil(M / 256) tiles and rounded up to 16.  When the tiles cannot fill
+// the SMs the contraction is split (at least 4 steps of 64 per split).
+HqqPlan plan_hqq(int64_t M, int64_t n_out, int64_t kc, int sm_count, bool allow_split) {
+  HqqPlan p{};
+  p.nt = static_cast<int>((n_out + 127) / 128);
+  p.ks = static_cast<int>((kc + HQ_BK - 1) / HQ_BK);
+  p.tt = static_cast<int>((M + 255) / 256);
+  const int64_t per = (M + p.tt - 1) / p.tt;
+  p.bn = static_cast<int>(std::max<int64_t>(16, (per + 15) / 16 * 16));
+  const int64_t tiles = static_cast<int64_t>(p.nt) * p.tt;
+  p.splits = 1;
+  if (allow_split && tiles < sm_count) {
+    int s = static_cast<int>(sm_count / tiles);
+    s = std::min(s, std::max(1, p.ks / 4));
+    p.splits = std::max(1, std::min(s, 32));
+  }
+  p.cnt_bytes = (static_cast<size_t>(tiles) * 4 * sizeof(uint32_t) + 255) / 256 * 256;
+  p.ws_bytes = p.splits > 1 ? p.cnt_bytes + static_cast<size_t>(tiles) * p.splits * p.bn * 128 * sizeof(float) : 0;
+  p.units = static_cast<int>(tiles * p.splits);
+  p.grid = std::min(p.units, sm_count);
+  const int stage = p.bn * 128 + HQ_W_BYTES;
+  const int avail = HQ_SMEM_LIMIT - 1024 - HQ_BAR_BYTES - HQ_ND * HQ_A_BYTES;
+  p.np = std::min(HQ_MAX_NP, avail / stage);
+  p.smem = 1024 + static_cast<size_t>(HQ_ND) * HQ_A_BYTES + static_cast<size_t>(p.np) * stage + HQ_BAR_BYTES;
+  return p;
+}
+
+dq_status check_weights(const uint8_t* packed, const void* scale, const void* zero, int64_t N, int64_t K,
+                        int group, int flags) {
+  if (N <= 0 || K <= 0 || (flags & ~DQ_HQQ_S4) != 0) return DQ_ERR_INVALID_ARG;
+  if (group != 32 && group != 64 && group != 128 && group != 256) return DQ_ERR_INVALID_ARG;
+  if (K % group != 0) return DQ_ERR_INVALID_ARG;
+  if (N % 8 != 0) return DQ_ERR_UNSUPPORTED;
+  if (N > (int64_t{1} << 30) || K > (int64_t{1} << 30)) return DQ_ERR_UNSUPPORTED;
+  if (packed == nullptr || scale == nullptr || zero == nullptr) return DQ_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(scale, 16) || !aligned(zero, 16)) return DQ_ERR_UNSUPPORTED;
+  return DQ_OK;
+}
+
+template <bool TRANS, bool S4>
+dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const HqqArgs& g, int grid, size_t smem,
+                     cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(hqq_gemm_kernel<TRANS, S4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    HQ_SMEM_LIMIT);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err);
+  hqq_gemm_kernel<TRANS, S4><<<grid, HQ_THREADS, smem, stream>>>(tx, tw, g);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* packed, const void* scale,
+                          const void* zero, int64_t N, int64_t K, int group, int flags, void* out,
+                          void* workspace, size_t workspace_bytes, dq_stream_t stream) {
+  dq_status st = check_weights(packed, scale, zero, N, K, group, flags);
+  if (st != DQ_OK) return st;
+  if (M < 0) return DQ_ERR_INVALID_ARG;
+  if (M > (int64_t{1} << 30)) return DQ_ERR_UNSUPPORTED;
+  if (M == 0) return DQ_OK;
+  if (x == nullptr || out == nullptr) return DQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16)) return DQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != DQ_OK) return st;
+
+  const int64_t n_out = trans ? K : N;
+  const int64_t kc = trans ? N : K;
+  HqqPlan p = plan_hqq(M, n_out, kc, d->sm_count, true);
+  if (p.splits > 1 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < p.ws_bytes))
+    p = plan_hqq(M, n_out, kc, d->sm_count, false);
+
+  CUtensorMap tx, tw;
+  // activations / output gradient: bf16 [M, kc] as bytes, 64-element k
+  // slices of bn rows, 128B-swizzled (the MMA's K-major B layout)
+  st = make_tmap_u8_2d(&tx, x, static_cast<uint64_t>(kc) * 2, static_cast<uint64_t>(M),
+                       static_cast<uint64_t>(kc) * 2, 128, static_cast<uint32_t>(p.bn), 128);
+  if (st != DQ_OK) return st;
+  // packed codes [N, K/2]: forward 128 channels x 32 B (64 k); transposed
+  // 64 weight rows x 64 B (128 output channels k)
+  st = make_tmap_u8_2d(&tw, packed, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N),
+                       static_cast<uint64_t>(K / 2), trans ? 64 : 32, trans ? 64 : 128, 0);
+  if (st != DQ_OK) return st;
+
+  HqqArgs g{};
+  g.M = static_cast<int>(M);
+  g.n_out = static_cast<int>(n_out);
+  g.kc = static_cast<int>(kc);
+  g.n_w = static_cast<int>(N);
+  g.k_w = static_cast<int>(K);
+  g.group = group;
+  g.n_groups = static_cast<int>(K / group);
+  g.bn = p.bn;
+  g.nt = p.nt;
+  g.tt = p.tt;
+  g.splits = p.splits;
+  g.ks = p.ks;
+  g.units = p.units;
+  g.np = p.np;
+  g.off_x = static_cast<uint32_t>(HQ_ND * HQ_A_BYTES);
+  g.off_w = g.off_x + static_cast<uint32_t>(p.np * p.bn * 128);
+  g.off_bar = g.off_w + static_cast<uint32_t>(p.np * HQ_W_BYTES);
+  g.scale = static_cast<const uint16_t*>(scale);
+  g.zero = static_cast<const uint16_t*>(zero);
+  g.out = static_cast<uint16_t*>(out);
+  if (p.splits > 1) {
+    g.cnt = static_cast<uint32_t*>(workspace);
+    g.ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.cnt_bytes);
+  }
+  g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
+  const bool s4 = (flags & DQ_HQQ_S4) != 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (trans) return s4 ? launch_hqq<true, true>(tx, tw, g, p.grid, p.smem, s)
+                       : launch_hqq<true, false>(tx, tw, g, p.grid, p.smem, s);
+  return s4 ? launch_hqq<false, true>(tx, tw, g, p.grid, p.smem, s)
+            : launch_hqq<false, false>(tx, tw, g, p.grid, p.smem, s);
+}
+
+int grid_for(int64_t items, int sm_count) {
+  const int64_t blocks = (items + 255) / 256;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(sm_count) * 16)));
+}
+
+}  // namespace
+}  // namespace dq
+
+using namespace dq;
+
+extern "C" {
+
+DQ_API dq_status dq_hqq_pack(const int8_t* codes, int64_t rows, int64_t cols, uint8_t* packed,
+                             dq_stream_t stream) {
+  if (rows < 0 || cols < 0 || (cols & 1) != 0) return DQ_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return DQ_OK;
+  if (codes == nullptr || packed == nullptr) return DQ_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  dq_status st = current_device(&d);
+  if (st != DQ_OK) return st;
+  const int64_t n_bytes = rows * (cols / 2);
+  hqq_pack_kernel<<<grid_for(n_bytes, d->sm_count), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      codes, n_bytes, packed);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+DQ_API dq_status dq_hqq_dequantize(const uint8_t* packed, const void* scale_bf16, const void* zero_bf16,
+                                   int64_t N, int64_t K, int group, int flags, void* w_bf16,
+                                   dq_stream_t stream) {
+  dq_status st = check_weights(packed, scale_bf16, zero_bf16, N, K, group, flags);
+  if (st != DQ_OK) return st;
+  if (w_bf16 == nullptr) return DQ_ERR_INVALID_ARG;
+  if (!aligned(w_bf16, 16)) return DQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  if ((st = current_device(&d)) != DQ_OK) return st;
+  const int64_t words = N * (K / 8);
+  const auto* pw = reinterpret_cast<const uint32_t*>(packed);
+  const auto* sc = static_cast<const uint16_t*>(scale_bf16);
+  const auto* ze = static_cast<const uint16_t*>(zero_bf16);
+  auto* w = static_cast<uint16_t*>(w_bf16);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (flags & DQ_HQQ_S4)
+    hqq_dequant_kernel<true><<<grid_for(words, d->sm_count), 256, 0, s>>>(pw, sc, ze, N, K, group, w);
+  else
+    hqq_dequant_kernel<false><<<grid_for(words, d->sm_count), 256, 0, s>>>(pw, sc, ze, N, K, group, w);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+DQ_API size_t dq_hqq_workspace_size(int64_t M, int64_t N, int64_t K, int transposed) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  DeviceInfo* d = nullptr;
+  if (current_device(&d) != DQ_OK) return 0;
+  const HqqPlan p = plan_hqq(M, transposed ? K : N, transposed ? N : K, d->sm_count, true);
+  return p.ws_bytes;
+}
+
+DQ_API dq_status dq_hqq_linear(const void* x_bf16, int64_t M, const uint8_t* packed, const void* scale_bf16,
+                               const void* zero_bf16, int64_t N, int64_t K, int group, int flags,
+                               void* out_bf16, void* workspace, size_t workspace_bytes, dq_stream_t stream) {
+  return hqq_linear_impl(false, x_bf16, M, packed, scale_bf16, zero_bf16, N, K, group, flags, out_bf16,
+                         workspace, workspace_bytes, stream);
+}
+
+DQ_API dq_status dq_hqq_linear_t(const void* y_bf16, int64_t M, const uint8_t* packed, const void* scale_bf16,
+                                 const void* zero_bf16, int64_t N, int64_t K, int group, int flags,
+                                 void* out_bf16, void* workspace, size_t workspace_bytes, dq_stream_t stream) {
+  return hqq_linear_impl(true, y_bf16, M, packed, scale_bf16, zero_bf16, N, K, group, flags, out_bf16,
+                         workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
