@@ -378,7 +378,8 @@ def make_state(name, wl, dq, torch, seed):
         trans = bool(wl.get("transposed"))
         M, K, N, group = wl["M"], wl["K"], wl["N"], wl["group"]
         packed = dq.dq_hqq_pack(_to_dev(torch, d["codes"]))
-        sc, ze = _to_dev_bf16(torch, d["scale"]), _to_dev_bf16(torch, d["zero"])
+        sc = dq.dq_hqq_group_major(_to_dev_bf16(torch, d["scale"]))
+        ze = dq.dq_hqq_group_major(_to_dev_bf16(torch, d["zero"]))
         x = _to_dev_bf16(torch, d["x"])
         n = _ncopies(x.numel() * 2 + packed.numel() + 2 * sc.numel() * 2)
         st["copies"] = [dict(x=x if i == 0 else x.clone(), P=packed if i == 0 else packed.clone(),

@@ -294,13 +294,18 @@ DQ_API dq_status dq_fp8_linear(const uint8_t* A, const float* s_row, int64_t M, 
  *   packed  uint8 [N, K/2] row-major: byte j of row n = q[n, 2j] in bits
  *           0..3 | q[n, 2j+1] in bits 4..7 (the page's "row interleave" of
  *           two codes per byte along K; s4 as two's-complement nibbles);
- *   scale, zero  bf16 [N, K/group] row-major (channel, group of `group`
- *           consecutive k);
- *   dequantized weight w[n, k] = bf16( bf16(q - zero[n, k/group]) *
- *           scale[n, k/group] ), each operation rounded once to nearest even.
+ *   scale, zero  bf16 [K/group, N] row-major, GROUP-MAJOR: element (g, n) is
+ *           channel n's value for its group g of `group` consecutive k, so
+ *           one contraction step's values for a run of channels are one
+ *           contiguous slice (dq_hqq_group_major converts the per-channel
+ *           [N, K/group] form);
+ *   dequantized weight w[n, k] = bf16( bf16(q - zero[k/group, n]) *
+ *           scale[k/group, n] ), each operation rounded once to nearest even.
  *
  * dq_hqq_pack: codes int8 [rows, cols] (cols even; values must lie in the
  *   u4 or s4 range, only the low 4 bits are kept) -> packed [rows, cols/2].
+ * dq_hqq_group_major: src bf16 [N, G] -> dst bf16 [G, N] (the per-channel
+ *   scale / zero-point layout to the group-major one; a weight-load step).
  * dq_hqq_dequantize: packed, scale, zero -> w bf16 [N, K] (the standalone
  *   dequantization; bit-exact).
  * dq_hqq_linear (forward):   out[m, n] = sum_k x[m, k] * w[n, k],
@@ -331,6 +336,8 @@ DQ_API dq_status dq_hqq_pack(const int8_t* codes, int64_t rows, int64_t cols, ui
 DQ_API dq_status dq_hqq_dequantize(const uint8_t* packed, const void* scale_bf16, const void* zero_bf16,
                                    int64_t N, int64_t K, int group, int flags, void* w_bf16,
                                    dq_stream_t stream);
+DQ_API dq_status dq_hqq_group_major(const void* src_bf16, int64_t N, int64_t G, void* dst_bf16,
+                                    dq_stream_t stream);
 DQ_API size_t dq_hqq_workspace_size(int64_t M, int64_t N, int64_t K, int transposed);
 DQ_API dq_status dq_hqq_linear(const void* x_bf16, int64_t M, const uint8_t* packed, const void* scale_bf16,
                                const void* zero_bf16, int64_t N, int64_t K, int group, int flags,

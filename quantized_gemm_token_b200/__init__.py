@@ -56,6 +56,7 @@ _PROTOS = {
     "dq_hqq_pack": (_I32, [_P, _I64, _I64, _P, _P]),
     "dq_hqq_dequantize": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I32, _P, _P]),
     "dq_hqq_workspace_size": (_SZ, [_I64, _I64, _I64, _I32]),
+    "dq_hqq_group_major": (_I32, [_P, _I64, _I64, _P, _P]),
     "dq_hqq_linear": (_I32, [_P, _I64, _P, _P, _P, _I64, _I64, _I32, _I32, _P, _P, _SZ, _P]),
     "dq_hqq_linear_t": (_I32, [_P, _I64, _P, _P, _P, _I64, _I64, _I32, _I32, _P, _P, _SZ, _P]),
 }
@@ -429,6 +430,22 @@ def dq_hqq_pack(codes: torch.Tensor, packed: torch.Tensor = None, stream=None) -
     return packed
 
 
+def dq_hqq_group_major(meta: torch.Tensor, out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """Per-channel scales or zero points bf16 [N, K/group] -> the group-major
+    [K/group, N] layout the int4 kernels read."""
+    _need(meta, torch.bfloat16, "meta", 2)
+    _contig(meta, "meta")
+    N, G = meta.shape
+    if out is None:
+        out = torch.empty((G, N), dtype=torch.bfloat16, device=meta.device)
+    _need(out, torch.bfloat16, "out", 2)
+    _contig(out, "out")
+    if tuple(out.shape) != (G, N):
+        raise ValueError("out must be [G, N]")
+    _check(lib.dq_hqq_group_major(_ptr(meta), N, G, _ptr(out), _stream(stream)), "dq_hqq_group_major")
+    return out
+
+
 def _hqq_weights(packed, scale, zero, group):
     _need(packed, torch.uint8, "packed", 2)
     _need(scale, torch.bfloat16, "scale", 2)
@@ -438,13 +455,14 @@ def _hqq_weights(packed, scale, zero, group):
     N, K = packed.shape[0], packed.shape[1] * 2
     if group <= 0 or K % group != 0:
         raise ValueError("group must divide K")
-    if tuple(scale.shape) != (N, K // group) or tuple(zero.shape) != (N, K // group):
-        raise ValueError("scale and zero must be [N, K/group]")
+    if tuple(scale.shape) != (K // group, N) or tuple(zero.shape) != (K // group, N):
+        raise ValueError("scale and zero must be group-major [K/group, N]")
     return N, K
 
 
 def dq_hqq_dequantize(packed, scale, zero, group: int, signed: bool = False, out=None, stream=None):
-    """w bf16 [N, K] = bf16(bf16(q - zero) * scale), per group of K."""
+    """w bf16 [N, K] = bf16(bf16(q - zero) * scale), per group of K (scale and
+    zero group-major [K/group, N])."""
     N, K = _hqq_weights(packed, scale, zero, group)
     if out is None:
         out = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device)
@@ -500,8 +518,9 @@ def dq_hqq_linear_t(y, packed, scale, zero, group: int, signed: bool = False, ou
 
 class HqqLinear:
     """Weight-only int4 linear: packed u4 / s4 codes with bf16 scale and zero
-    point per group of in-features.  forward(x) = x @ w^T, backward_input(g)
-    = g @ w; the workspace for few-token calls is kept per token count."""
+    point per group of in-features (held group-major, [K/group, N]).
+    forward(x) = x @ w^T, backward_input(g) = g @ w; the workspace for
+    few-token calls is kept per token count."""
 
     def __init__(self, packed, scale, zero, group: int, signed: bool = False):
         self.packed, self.scale, self.zero, self.group, self.signed = packed, scale, zero, group, signed
@@ -510,7 +529,8 @@ class HqqLinear:
 
     @classmethod
     def from_codes(cls, codes: torch.Tensor, scale, zero, group: int, signed: bool = False):
-        return cls(dq_hqq_pack(codes), scale, zero, group, signed)
+        """codes int8 [N, K]; scale, zero bf16 per channel [N, K/group]."""
+        return cls(dq_hqq_pack(codes), dq_hqq_group_major(scale), dq_hqq_group_major(zero), group, signed)
 
     def _workspace(self, M, transposed, device):
         key = (M, transposed)

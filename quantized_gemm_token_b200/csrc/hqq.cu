@@ -42,6 +42,12 @@ constexpr int HQ_EPI_WARP0 = 10;           // warps 10..13
 constexpr int HQ_BK = 64;                  // contraction elements per step (128 B of bf16)
 constexpr int HQ_A_BYTES = 128 * 128;      // dequantized weight tile: 128 rows x 128 B
 constexpr int HQ_W_BYTES = 4096;           // packed int4 tile per step
+// Per-step scale and zero-point slices, staged next to the packed tile: four
+// slots of up to 128 bf16 channel values each (one slot per 32-deep k slice
+// that starts a new group), scales at +0, zero points at +HQ_META_HALF.
+constexpr int HQ_META_SLOT = 256;
+constexpr int HQ_META_HALF = 4 * HQ_META_SLOT;
+constexpr int HQ_WM_BYTES = HQ_W_BYTES + 2 * HQ_META_HALF;   // one W ring stage
 constexpr int HQ_ND = 4;                   // dequantized-tile ring
 constexpr int HQ_MAX_NP = 16;
 constexpr int HQ_ACC_COLS = 256;           // TMEM columns per accumulator buffer
@@ -62,8 +68,8 @@ struct HqqArgs {
   int units;              // nt * tt * splits
   int np;                 // packed / activation ring stages
   uint32_t off_x, off_w, off_bar;   // shared-memory offsets (A ring at 0)
-  const uint16_t* scale;
-  const uint16_t* zero;
+  const uint16_t* scale; // bf16 [n_groups, n_w], group-major
+  const uint16_t* zero;   // bf16 [n_groups, n_w]
   uint16_t* out;          // bf16 [M, n_out]
   float* ws;              // split partials: [tile][split][bn][128] fp32
   uint32_t* cnt;          // arrival counters: [tile][4]
@@ -127,6 +133,22 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&v)[
                : "memory");
 }
 
+// 1-D bulk copy global -> shared completing `bar`'s transaction count (both
+// addresses 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// The meta slot holding the group of 32-deep k slice j: the first slice of
+// each group (groups of 32 start at every slice, groups of 64 at even ones,
+// larger groups at slice 0 of a step or tile).
+__device__ __forceinline__ int meta_slot(int j, int group) {
+  const int per = group >> 5;          // k slices per group: 1, 2, 4 or 8
+  return per >= 4 ? 0 : (j / per) * per;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulator,
 // both operands K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
@@ -148,10 +170,11 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
 
 // Forward: 256 threads turn the packed tile (128 channel rows x 32 B = 64
 // codes) into the 128 x 64 bf16 A tile.  Thread t: row t % 128, codes
-// 32 * (t / 128) .. +31 (one group: group sizes are >= 32).
+// 32 * (t / 128) .. +31 (inside one group: group sizes are >= 32); its scale
+// and zero point come from the step's staged meta slots.
 template <bool S4>
-__device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t wtile, uint32_t atile,
-                                                 const uint8_t* wtile_ptr, int dt, int ntile, int kstep) {
+__device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t atile, const uint8_t* wtile_ptr,
+                                                 int dt, int ntile, int kstep) {
   const int r = dt & 127;
   const int h = dt >> 7;
   const uint4 pk = *reinterpret_cast<const uint4*>(wtile_ptr + r * 32 + h * 16);
@@ -159,9 +182,9 @@ __device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t wtil
   const int k = kstep * HQ_BK + h * 32;
   uint32_t s2 = 0, z2 = 0;
   if (n < g.n_w && k < g.k_w) {
-    const int64_t gi = static_cast<int64_t>(n) * g.n_groups + k / g.group;
-    s2 = bf16_pair_of(__ldg(g.scale + gi));
-    z2 = bf16_pair_of(__ldg(g.zero + gi));
+    const uint8_t* meta = wtile_ptr + HQ_W_BYTES + meta_slot(h, g.group) * HQ_META_SLOT;
+    s2 = bf16_pair_of(reinterpret_cast<const uint16_t*>(meta)[r]);
+    z2 = bf16_pair_of(reinterpret_cast<const uint16_t*>(meta + HQ_META_HALF)[r]);
   }
   const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
@@ -170,24 +193,33 @@ __device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t wtil
     dequant8<S4>(words[i], z2, s2, o);
     st_shared_v4(atile + sw128_off(r, 4 * h + i), o);
   }
-  (void)wtile;
 }
 
 // Transposed: the packed tile holds 64 contraction rows (weight rows n) x
 // 64 B (128 output channels k, two per byte); the A tile is 128 rows (k) x
 // 64 bf16 (n).  Warp w handles n = 8w .. 8w+7; lane l the byte columns l and
 // l + 32 (A rows 2l, 2l+1 and 2l+64, 2l+65): eight bytes from eight weight
-// rows give two 16-byte chunks, one per A row.
+// rows give two 16-byte chunks, one per A row.  The eight rows' scales and
+// zero points are 16 contiguous bytes of a staged meta slot: the bf16 pairs
+// the packed arithmetic needs.
 template <bool S4>
 __device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile, const uint8_t* wtile_ptr,
                                                int dt, int ntile, int kstep) {
   const int nc = dt >> 5;       // n chunk (8 weight rows)
   const int lane = dt & 31;
-  const int n0 = kstep * HQ_BK + nc * 8;
+  const bool n_ok = kstep * HQ_BK + nc * 8 < g.n_w;     // n_w % 8 == 0: the chunk is all in or all out
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     const int b = lane + 32 * u;                 // byte column: k = 2b, 2b + 1 in the tile
     const int k = ntile * 128 + 2 * b;
+    uint4 s8 = make_uint4(0, 0, 0, 0), z8 = make_uint4(0, 0, 0, 0);
+    if (n_ok && k < g.k_w) {
+      const uint8_t* meta = wtile_ptr + HQ_W_BYTES + meta_slot(b >> 4, g.group) * HQ_META_SLOT + nc * 16;
+      s8 = *reinterpret_cast<const uint4*>(meta);
+      z8 = *reinterpret_cast<const uint4*>(meta + HQ_META_HALF);
+    }
+    const uint32_t sp[4] = {s8.x, s8.y, s8.z, s8.w};
+    const uint32_t zp[4] = {z8.x, z8.y, z8.z, z8.w};
     uint32_t lo[4], hi[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -196,21 +228,10 @@ __device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile,
       const uint32_t b1 = wtile_ptr[(nc * 8 + 2 * i + 1) * 64 + b];
       uint32_t x = b0 | (b1 << 16);
       if (S4) x ^= 0x00880088u;
-      uint32_t s2 = 0, z2 = 0;
-      const int na = n0 + 2 * i, nb = na + 1;
-      if (k < g.k_w) {
-        const int gk = k / g.group;
-        const uint32_t sa = na < g.n_w ? __ldg(g.scale + static_cast<int64_t>(na) * g.n_groups + gk) : 0u;
-        const uint32_t sb = nb < g.n_w ? __ldg(g.scale + static_cast<int64_t>(nb) * g.n_groups + gk) : 0u;
-        const uint32_t za = na < g.n_w ? __ldg(g.zero + static_cast<int64_t>(na) * g.n_groups + gk) : 0u;
-        const uint32_t zb = nb < g.n_w ? __ldg(g.zero + static_cast<int64_t>(nb) * g.n_groups + gk) : 0u;
-        s2 = sa | (sb << 16);
-        z2 = za | (zb << 16);
-      }
-      const uint32_t pl = (x & 0x000F000Fu) | 0x43004300u;          // k = 2b: rows na, nb
+      const uint32_t pl = (x & 0x000F000Fu) | 0x43004300u;          // k = 2b: rows 2i, 2i + 1
       const uint32_t ph = ((x >> 4) & 0x000F000Fu) | 0x43004300u;   // k = 2b + 1
-      lo[i] = bmul2(bsub2(bsub2(pl, code_bias2<S4>()), z2), s2);
-      hi[i] = bmul2(bsub2(bsub2(ph, code_bias2<S4>()), z2), s2);
+      lo[i] = bmul2(bsub2(bsub2(pl, code_bias2<S4>()), zp[i]), sp[i]);
+      hi[i] = bmul2(bsub2(bsub2(ph, code_bias2<S4>()), zp[i]), sp[i]);
     }
     st_shared_v4(atile + sw128_off(2 * b, nc), lo);
     st_shared_v4(atile + sw128_off(2 * b + 1, nc), hi);
@@ -320,21 +341,39 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
-      const uint32_t tx = x_bytes + HQ_W_BYTES;
+      const int per = g.group >> 5;          // 32-deep k slices per group
       for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
         const Unit t = decode_unit(g, u);
+        // channels of this tile's scale / zero-point rows: forward 128
+        // output channels, transposed 64 weight rows per step
         for (int kk = t.k0; kk < t.k1; ++kk) {
           if (!mbar_wait(smem_u32(p_empty + stage), phase ^ 1, g.wait, abort_flag)) {
             ok = false;
             break;
           }
+          const int c0 = TRANS ? kk * HQ_BK : t.ntile * 128;              // first weight row
+          const int cnt = min(TRANS ? HQ_BK : 128, g.n_w - c0);           // rows present (a multiple of 8)
+          const int kbase = TRANS ? t.ntile * 128 : kk * HQ_BK;            // first in-feature of the step
+          const int nslices = TRANS ? 4 : 2;
+          uint32_t meta_tx = 0;
+          for (int j = 0; j < nslices; ++j)
+            if (cnt > 0 && j % per == 0 && kbase + 32 * j < g.k_w) meta_tx += 4u * static_cast<uint32_t>(cnt);
           const uint32_t fb = smem_u32(p_full + stage);
-          mbar_arrive_expect_tx(fb, tx);
+          const uint32_t wdst = sW + stage * HQ_WM_BYTES;
+          mbar_arrive_expect_tx(fb, x_bytes + HQ_W_BYTES + meta_tx);
           tma_load_2d(sX + stage * x_bytes, &tm_x, fb, kk * 128, t.ttile * g.bn);
           if (TRANS)
-            tma_load_2d(sW + stage * HQ_W_BYTES, &tm_w, fb, t.ntile * 64, kk * HQ_BK);
+            tma_load_2d(wdst, &tm_w, fb, t.ntile * 64, kk * HQ_BK);
           else
-            tma_load_2d(sW + stage * HQ_W_BYTES, &tm_w, fb, kk * 32, t.ntile * 128);
+            tma_load_2d(wdst, &tm_w, fb, kk * 32, t.ntile * 128);
+          for (int j = 0; j < nslices; ++j) {
+            if (cnt > 0 && j % per == 0 && kbase + 32 * j < g.k_w) {
+              const int64_t off = static_cast<int64_t>((kbase + 32 * j) / g.group) * g.n_w + c0;
+              const uint32_t dst = wdst + HQ_W_BYTES + j * HQ_META_SLOT;
+              bulk_load_1d(dst, g.scale + off, 2u * cnt, fb);
+              bulk_load_1d(dst + HQ_META_HALF, g.zero + off, 2u * cnt, fb);
+            }
+          }
           ++issued;
           if (++stage == g.np) {
             stage = 0;
@@ -411,11 +450,11 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
           break;
         }
         const uint32_t atile = sA + dst * HQ_A_BYTES;
-        const uint8_t* wp = sW_ptr + stage * HQ_W_BYTES;
+        const uint8_t* wp = sW_ptr + stage * HQ_WM_BYTES;
         if (TRANS)
           dequant_tile_t<S4>(g, atile, wp, dt, t.ntile, kk);
         else
-          dequant_tile_fwd<S4>(g, sW + stage * HQ_W_BYTES, atile, wp, dt, t.ntile, kk);
+          dequant_tile_fwd<S4>(g, atile, wp, dt, t.ntile, kk);
         fence_proxy_async_smem();     // generic-proxy writes -> visible to the MMA
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(d_full + dst));
@@ -488,15 +527,21 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
           const float* const tile_ws = g.ws + static_cast<int64_t>(t.tile) * g.splits * g.bn * 128;
           for (int c0 = 0; c0 < g.bn; c0 += 32) {
             const int width = min(32, g.bn - c0);
+            // split by split (a fixed order), the chunk's loads all in flight
+            float sum[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sum[j] = 0.0f;
+            for (int sp = 0; sp < g.splits; ++sp) {
+              const float* src = tile_ws + (static_cast<int64_t>(sp) * g.bn + c0) * 128 + row;
+              float v[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = j < width ? __ldcg(src + j * 128) : 0.0f;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sum[j] += v[j];
+            }
             uint32_t r[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              float acc_sum = 0.0f;
-              if (j < width)
-                for (int sp = 0; sp < g.splits; ++sp)
-                  acc_sum += __ldcg(tile_ws + (static_cast<int64_t>(sp) * g.bn + c0 + j) * 128 + row);
-              r[j] = __float_as_uint(acc_sum);
-            }
+            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sum[j]);
             store_pairs(g, r, width, tok0 + c0, ch, lane);
           }
           __syncwarp();
@@ -512,7 +557,8 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, HQ_TMEM_COLS);
 }
 
-// Standalone dequantization: one thread per packed word (8 codes) -> 16 B of bf16.
+// Standalone dequantization: one thread per packed word (8 codes) -> 16 B of
+// bf16.  Scales and zero points group-major ([K / group, N]).
 template <bool S4>
 __global__ void __launch_bounds__(256) hqq_dequant_kernel(const uint32_t* __restrict__ packed,
                                                           const uint16_t* __restrict__ scale,
@@ -520,15 +566,31 @@ __global__ void __launch_bounds__(256) hqq_dequant_kernel(const uint32_t* __rest
                                                           int64_t K, int group, uint16_t* __restrict__ w) {
   const int64_t words_per_row = K / 8;
   const int64_t total = N * words_per_row;
-  const int64_t G = K / group;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t n = i / words_per_row;
     const int64_t k = (i - n * words_per_row) * 8;
-    const int64_t gi = n * G + k / group;
+    const int64_t gi = (k / group) * N + n;
     uint32_t o[4];
     dequant8<S4>(__ldg(packed + i), bf16_pair_of(__ldg(zero + gi)), bf16_pair_of(__ldg(scale + gi)), o);
     *reinterpret_cast<uint4*>(w + n * K + k) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// [rows, cols] -> [cols, rows] for 16-bit elements, through a 32 x 33 tile.
+__global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t* __restrict__ src, int64_t rows,
+                                                          int64_t cols, uint16_t* __restrict__ dst) {
+  __shared__ uint16_t tile[32][33];
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32, c0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;     // 32 x 8 threads
+  for (int i = ty; i < 32; i += 8) {
+    const int64_t r = r0 + i, c = c0 + tx;
+    if (r < rows && c < cols) tile[i][tx] = src[r * cols + c];
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int64_t c = c0 + i, r = r0 + tx;
+    if (r < rows && c < cols) dst[c * rows + r] = tile[tx][i];
   }
 }
 
@@ -576,7 +638,7 @@ HqqPlan plan_hqq(int64_t M, int64_t n_out, int64_t kc, int sm_count, bool allow_
   p.ws_bytes = p.splits > 1 ? p.cnt_bytes + static_cast<size_t>(tiles) * p.splits * p.bn * 128 * sizeof(float) : 0;
   p.units = static_cast<int>(tiles * p.splits);
   p.grid = std::min(p.units, sm_count);
-  const int stage = p.bn * 128 + HQ_W_BYTES;
+  const int stage = p.bn * 128 + HQ_WM_BYTES;
   const int avail = HQ_SMEM_LIMIT - 1024 - HQ_BAR_BYTES - HQ_ND * HQ_A_BYTES;
   p.np = std::min(HQ_MAX_NP, avail / stage);
   p.smem = 1024 + static_cast<size_t>(HQ_ND) * HQ_A_BYTES + static_cast<size_t>(p.np) * stage + HQ_BAR_BYTES;
@@ -658,7 +720,7 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   g.np = p.np;
   g.off_x = static_cast<uint32_t>(HQ_ND * HQ_A_BYTES);
   g.off_w = g.off_x + static_cast<uint32_t>(p.np * p.bn * 128);
-  g.off_bar = g.off_w + static_cast<uint32_t>(p.np * HQ_W_BYTES);
+  g.off_bar = g.off_w + static_cast<uint32_t>(p.np * HQ_WM_BYTES);
   g.scale = static_cast<const uint16_t*>(scale);
   g.zero = static_cast<const uint16_t*>(zero);
   g.out = static_cast<uint16_t*>(out);
@@ -721,6 +783,23 @@ DQ_API dq_status dq_hqq_dequantize(const uint8_t* packed, const void* scale_bf16
     hqq_dequant_kernel<true><<<grid_for(words, d->sm_count), 256, 0, s>>>(pw, sc, ze, N, K, group, w);
   else
     hqq_dequant_kernel<false><<<grid_for(words, d->sm_count), 256, 0, s>>>(pw, sc, ze, N, K, group, w);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+DQ_API dq_status dq_hqq_group_major(const void* src_bf16, int64_t N, int64_t G, void* dst_bf16,
+                                    dq_stream_t stream) {
+  if (N < 0 || G < 0) return DQ_ERR_INVALID_ARG;
+  if (N == 0 || G == 0) return DQ_OK;
+  if (src_bf16 == nullptr || dst_bf16 == nullptr || N > (int64_t{1} << 30) || G > (int64_t{1} << 30))
+    return DQ_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  dq_status st = current_device(&d);
+  if (st != DQ_OK) return st;
+  if ((G + 31) / 32 > 2147483647 || (N + 31) / 32 > 65535) return DQ_ERR_UNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>((N + 31) / 32));
+  transpose16_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(src_bf16), N, G, static_cast<uint16_t*>(dst_bf16));
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }

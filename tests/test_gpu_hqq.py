@@ -57,7 +57,8 @@ def _weights(d):
 
 
 def _dev_weights(d, packed):
-    return to_dev(packed), to_dev_bf16(d["scale"]), to_dev_bf16(d["zero"])
+    """Packed codes and the group-major [K/group, N] scales and zero points."""
+    return to_dev(packed), to_dev_bf16(d["scale"].T.copy()), to_dev_bf16(d["zero"].T.copy())
 
 
 def _ws(M, N, K, transposed):
@@ -73,6 +74,13 @@ def test_pack_bit_exact(R, C, signed):
     codes = synth.uniform_int8((R, C), lo, hi, 3 + C)
     p = dq.dq_hqq_pack(to_dev(codes))
     assert np.array_equal(p.cpu().numpy(), oracle.hqq_pack(codes))
+
+
+@pytest.mark.parametrize("N,G", [(1, 1), (8, 2), (4096, 32), (136, 5), (33, 70)])
+def test_group_major_bit_exact(N, G):
+    m = synth.normal_bf16((N, G), 1.0, N + G)
+    got = dq.dq_hqq_group_major(to_dev_bf16(m))
+    assert np.array_equal(bf16_bits(got), m.T)
 
 
 @pytest.mark.parametrize("N,K,group,signed", [(8, 64, 64, False), (24, 256, 32, True), (256, 4096, 128, False),
