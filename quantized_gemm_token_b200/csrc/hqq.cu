@@ -133,6 +133,53 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&v)[
                : "memory");
 }
 
+// Bounded wait on an mbarrier phase that sleeps instead of spinning: each
+// try_wait may suspend the thread (up to kSuspendNs) until the phase
+// completes, so waiting warps take no issue slots from the working ones.
+// Gives up like mbar_wait: after ctl.timeout_ns, or once *abort is raised.
+constexpr uint32_t kSuspendNs = 200000;
+__device__ __forceinline__ bool try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool hq_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl, volatile int* abort) {
+  if (try_wait_sleep(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (try_wait_sleep(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > ctl.timeout_ns) {
+      atomicOr(ctl.err, kErrTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Shared-memory loads by 32-bit shared address.
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds8(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
 // 1-D bulk copy global -> shared completing `bar`'s transaction count (both
 // addresses 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -173,18 +220,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
 // 32 * (t / 128) .. +31 (inside one group: group sizes are >= 32); its scale
 // and zero point come from the step's staged meta slots.
 template <bool S4>
-__device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t atile, const uint8_t* wtile_ptr,
-                                                 int dt, int ntile, int kstep) {
+__device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t atile, uint32_t wtile, int dt, int ntile,
+                                                 int kstep) {
   const int r = dt & 127;
   const int h = dt >> 7;
-  const uint4 pk = *reinterpret_cast<const uint4*>(wtile_ptr + r * 32 + h * 16);
+  const uint4 pk = lds128(wtile + r * 32 + h * 16);
   const int n = ntile * 128 + r;
   const int k = kstep * HQ_BK + h * 32;
   uint32_t s2 = 0, z2 = 0;
   if (n < g.n_w && k < g.k_w) {
-    const uint8_t* meta = wtile_ptr + HQ_W_BYTES + meta_slot(h, g.group) * HQ_META_SLOT;
-    s2 = bf16_pair_of(reinterpret_cast<const uint16_t*>(meta)[r]);
-    z2 = bf16_pair_of(reinterpret_cast<const uint16_t*>(meta + HQ_META_HALF)[r]);
+    const uint32_t meta = wtile + HQ_W_BYTES + meta_slot(h, g.group) * HQ_META_SLOT + 2 * r;
+    s2 = bf16_pair_of(static_cast<uint16_t>(lds16(meta)));
+    z2 = bf16_pair_of(static_cast<uint16_t>(lds16(meta + HQ_META_HALF)));
   }
   const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
@@ -203,8 +250,8 @@ __device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t atil
 // zero points are 16 contiguous bytes of a staged meta slot: the bf16 pairs
 // the packed arithmetic needs.
 template <bool S4>
-__device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile, const uint8_t* wtile_ptr,
-                                               int dt, int ntile, int kstep) {
+__device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile, uint32_t wtile, int dt, int ntile,
+                                               int kstep) {
   const int nc = dt >> 5;       // n chunk (8 weight rows)
   const int lane = dt & 31;
   const bool n_ok = kstep * HQ_BK + nc * 8 < g.n_w;     // n_w % 8 == 0: the chunk is all in or all out
@@ -214,9 +261,9 @@ __device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile,
     const int k = ntile * 128 + 2 * b;
     uint4 s8 = make_uint4(0, 0, 0, 0), z8 = make_uint4(0, 0, 0, 0);
     if (n_ok && k < g.k_w) {
-      const uint8_t* meta = wtile_ptr + HQ_W_BYTES + meta_slot(b >> 4, g.group) * HQ_META_SLOT + nc * 16;
-      s8 = *reinterpret_cast<const uint4*>(meta);
-      z8 = *reinterpret_cast<const uint4*>(meta + HQ_META_HALF);
+      const uint32_t meta = wtile + HQ_W_BYTES + meta_slot(b >> 4, g.group) * HQ_META_SLOT + nc * 16;
+      s8 = lds128(meta);
+      z8 = lds128(meta + HQ_META_HALF);
     }
     const uint32_t sp[4] = {s8.x, s8.y, s8.z, s8.w};
     const uint32_t zp[4] = {z8.x, z8.y, z8.z, z8.w};
@@ -224,8 +271,8 @@ __device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile,
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       // weight rows n0 + 2i and n0 + 2i + 1
-      const uint32_t b0 = wtile_ptr[(nc * 8 + 2 * i) * 64 + b];
-      const uint32_t b1 = wtile_ptr[(nc * 8 + 2 * i + 1) * 64 + b];
+      const uint32_t b0 = lds8(wtile + (nc * 8 + 2 * i) * 64 + b);
+      const uint32_t b1 = lds8(wtile + (nc * 8 + 2 * i + 1) * 64 + b);
       uint32_t x = b0 | (b1 << 16);
       if (S4) x ^= 0x00880088u;
       const uint32_t pl = (x & 0x000F000Fu) | 0x43004300u;          // k = 2b: rows 2i, 2i + 1
@@ -292,7 +339,6 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
   const uint32_t sA = base;                 // HQ_ND dequantized tiles
   const uint32_t sX = base + g.off_x;       // np activation tiles (bn x 128 B)
   const uint32_t sW = base + g.off_w;       // np packed weight tiles
-  const uint8_t* const sW_ptr = smem + g.off_w;
   uint64_t* const p_full = reinterpret_cast<uint64_t*>(smem + g.off_bar);
   uint64_t* const p_empty = p_full + HQ_MAX_NP;
   uint64_t* const d_full = p_empty + HQ_MAX_NP;
@@ -347,7 +393,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
         // channels of this tile's scale / zero-point rows: forward 128
         // output channels, transposed 64 weight rows per step
         for (int kk = t.k0; kk < t.k1; ++kk) {
-          if (!mbar_wait(smem_u32(p_empty + stage), phase ^ 1, g.wait, abort_flag)) {
+          if (!hq_wait(smem_u32(p_empty + stage), phase ^ 1, g.wait, abort_flag)) {
             ok = false;
             break;
           }
@@ -384,7 +430,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       // every copy issued lands before the CTA can exit
       volatile int never = 0;
       for (long long i = issued > g.np ? issued - g.np : 0; i < issued; ++i)
-        mbar_wait(smem_u32(p_full + static_cast<int>(i % g.np)), static_cast<uint32_t>((i / g.np) & 1), g.wait,
+        hq_wait(smem_u32(p_full + static_cast<int>(i % g.np)), static_cast<uint32_t>((i / g.np) & 1), g.wait,
                   &never);
     }
   } else if (warp == 1) {
@@ -396,12 +442,12 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       bool ok = true;
       for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
         const Unit t = decode_unit(g, u);
-        if (!mbar_wait(smem_u32(acce + acc), aphase ^ 1, g.wait, abort_flag)) break;
+        if (!hq_wait(smem_u32(acce + acc), aphase ^ 1, g.wait, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * HQ_ACC_COLS);
         for (int kk = t.k0; kk < t.k1; ++kk) {
-          if (!mbar_wait(smem_u32(d_full + dst), dphase, g.wait, abort_flag) ||
-              !mbar_wait(smem_u32(p_full + stage), phase, g.wait, abort_flag)) {
+          if (!hq_wait(smem_u32(d_full + dst), dphase, g.wait, abort_flag) ||
+              !hq_wait(smem_u32(p_full + stage), phase, g.wait, abort_flag)) {
             ok = false;
             break;
           }
@@ -432,7 +478,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       // every MMA issued has completed once drain flips
       mma_commit(smem_u32(drain));
       volatile int never = 0;
-      mbar_wait(smem_u32(drain), 0, g.wait, &never);
+      hq_wait(smem_u32(drain), 0, g.wait, &never);
     }
   } else if (warp < HQ_EPI_WARP0) {
     // ---------------------------------------------------------- dequantizers
@@ -443,18 +489,18 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
       const Unit t = decode_unit(g, u);
       for (int kk = t.k0; kk < t.k1; ++kk) {
-        bool w = mbar_wait(smem_u32(p_full + stage), phase, g.wait, abort_flag);
-        w = w && mbar_wait(smem_u32(d_empty + dst), dphase ^ 1, g.wait, abort_flag);
+        bool w = hq_wait(smem_u32(p_full + stage), phase, g.wait, abort_flag);
+        w = w && hq_wait(smem_u32(d_empty + dst), dphase ^ 1, g.wait, abort_flag);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
         }
         const uint32_t atile = sA + dst * HQ_A_BYTES;
-        const uint8_t* wp = sW_ptr + stage * HQ_WM_BYTES;
+        const uint32_t wt = sW + stage * HQ_WM_BYTES;
         if (TRANS)
-          dequant_tile_t<S4>(g, atile, wp, dt, t.ntile, kk);
+          dequant_tile_t<S4>(g, atile, wt, dt, t.ntile, kk);
         else
-          dequant_tile_fwd<S4>(g, atile, wp, dt, t.ntile, kk);
+          dequant_tile_fwd<S4>(g, atile, wt, dt, t.ntile, kk);
         fence_proxy_async_smem();     // generic-proxy writes -> visible to the MMA
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(d_full + dst));
@@ -476,7 +522,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     uint32_t aphase = 0;
     for (int u = blockIdx.x; u < g.units; u += gridDim.x) {
       const Unit t = decode_unit(g, u);
-      const bool w = mbar_wait(smem_u32(accf + acc), aphase, g.wait, abort_flag);
+      const bool w = hq_wait(smem_u32(accf + acc), aphase, g.wait, abort_flag);
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * HQ_ACC_COLS);
