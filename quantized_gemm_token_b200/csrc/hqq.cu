@@ -48,7 +48,6 @@ constexpr int HQ_W_BYTES = 4096;           // packed int4 tile per step
 constexpr int HQ_META_SLOT = 256;
 constexpr int HQ_META_HALF = 4 * HQ_META_SLOT;
 constexpr int HQ_WM_BYTES = HQ_W_BYTES + 2 * HQ_META_HALF;   // one W ring stage
-constexpr int HQ_ND = 4;                   // dequantized-tile ring
 constexpr int HQ_MAX_NP = 16;
 constexpr int HQ_ACC_COLS = 256;           // TMEM columns per accumulator buffer
 constexpr int HQ_TMEM_COLS = 512;          // two accumulator buffers
@@ -67,7 +66,7 @@ struct HqqArgs {
   int ks;                 // contraction steps per tile (ceil(kc / 64))
   int units;              // nt * tt * splits
   int np;                 // packed / activation ring stages
-  uint32_t off_x, off_w, off_bar;   // shared-memory offsets (A ring at 0)
+  uint32_t off_bar;       // shared-memory offset of the barriers (after the stages)
   const uint16_t* scale; // bf16 [n_groups, n_w], group-major
   const uint16_t* zero;   // bf16 [n_groups, n_w]
   uint16_t* out;          // bf16 [M, n_out]
@@ -336,30 +335,29 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* const smem = smem_raw + (base - raw);
-  const uint32_t sA = base;                 // HQ_ND dequantized tiles
-  const uint32_t sX = base + g.off_x;       // np activation tiles (bn x 128 B)
-  const uint32_t sW = base + g.off_w;       // np packed weight tiles
-  uint64_t* const p_full = reinterpret_cast<uint64_t*>(smem + g.off_bar);
-  uint64_t* const p_empty = p_full + HQ_MAX_NP;
-  uint64_t* const d_full = p_empty + HQ_MAX_NP;
-  uint64_t* const d_empty = d_full + HQ_ND;
-  uint64_t* const accf = d_empty + HQ_ND;
+  // stage s at base + s * stage_bytes: dequantized A tile (16 KB), then the
+  // activation tile (bn x 128 B), then the packed weight tile and its meta
+  const uint32_t x_bytes = static_cast<uint32_t>(g.bn) * 128u;
+  const uint32_t stage_bytes = HQ_A_BYTES + x_bytes + HQ_WM_BYTES;
+  uint64_t* const full = reinterpret_cast<uint64_t*>(smem + g.off_bar);   // TMA landed
+  uint64_t* const deq = full + HQ_MAX_NP;                                 // A tile written
+  uint64_t* const empty = deq + HQ_MAX_NP;                                // MMAs done with the stage
+  uint64_t* const accf = empty + HQ_MAX_NP;
   uint64_t* const acce = accf + 2;
   uint64_t* const drain = acce + 2;
   uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* const last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     *abort_flag = 0;
+    *last_flag = 0;
     for (int i = 0; i < g.np; ++i) {
-      mbar_init(smem_u32(p_full + i), 1);
-      mbar_init(smem_u32(p_empty + i), 1);
-    }
-    for (int i = 0; i < HQ_ND; ++i) {
-      mbar_init(smem_u32(d_full + i), HQ_DEQ_WARPS);
-      mbar_init(smem_u32(d_empty + i), 1);
+      mbar_init(smem_u32(full + i), 1);
+      mbar_init(smem_u32(deq + i), HQ_DEQ_WARPS);
+      mbar_init(smem_u32(empty + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(accf + i), 1);
@@ -378,7 +376,6 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const uint32_t x_bytes = static_cast<uint32_t>(g.bn) * 128u;
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
@@ -390,32 +387,33 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       const int per = g.group >> 5;          // 32-deep k slices per group
       for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
         const Unit t = decode_unit(g, u);
-        // channels of this tile's scale / zero-point rows: forward 128
-        // output channels, transposed 64 weight rows per step
         for (int kk = t.k0; kk < t.k1; ++kk) {
-          if (!hq_wait(smem_u32(p_empty + stage), phase ^ 1, g.wait, abort_flag)) {
+          if (!hq_wait(smem_u32(empty + stage), phase ^ 1, g.wait, abort_flag)) {
             ok = false;
             break;
           }
-          const int c0 = TRANS ? kk * HQ_BK : t.ntile * 128;              // first weight row
-          const int cnt = min(TRANS ? HQ_BK : 128, g.n_w - c0);           // rows present (a multiple of 8)
-          const int kbase = TRANS ? t.ntile * 128 : kk * HQ_BK;            // first in-feature of the step
+          // scale / zero-point rows present for this step: forward the 128
+          // output channels of the tile, transposed the step's 64 weight rows
+          const int c0 = TRANS ? kk * HQ_BK : t.ntile * 128;
+          const int cnt = min(TRANS ? HQ_BK : 128, g.n_w - c0);          // a multiple of 8
+          const int kbase = TRANS ? t.ntile * 128 : kk * HQ_BK;           // first in-feature
           const int nslices = TRANS ? 4 : 2;
           uint32_t meta_tx = 0;
           for (int j = 0; j < nslices; ++j)
             if (cnt > 0 && j % per == 0 && kbase + 32 * j < g.k_w) meta_tx += 4u * static_cast<uint32_t>(cnt);
-          const uint32_t fb = smem_u32(p_full + stage);
-          const uint32_t wdst = sW + stage * HQ_WM_BYTES;
+          const uint32_t fb = smem_u32(full + stage);
+          const uint32_t sx = base + stage * stage_bytes + HQ_A_BYTES;
+          const uint32_t sw = sx + x_bytes;
           mbar_arrive_expect_tx(fb, x_bytes + HQ_W_BYTES + meta_tx);
-          tma_load_2d(sX + stage * x_bytes, &tm_x, fb, kk * 128, t.ttile * g.bn);
+          tma_load_2d(sx, &tm_x, fb, kk * 128, t.ttile * g.bn);
           if (TRANS)
-            tma_load_2d(wdst, &tm_w, fb, t.ntile * 64, kk * HQ_BK);
+            tma_load_2d(sw, &tm_w, fb, t.ntile * 64, kk * HQ_BK);
           else
-            tma_load_2d(wdst, &tm_w, fb, kk * 32, t.ntile * 128);
+            tma_load_2d(sw, &tm_w, fb, kk * 32, t.ntile * 128);
           for (int j = 0; j < nslices; ++j) {
             if (cnt > 0 && j % per == 0 && kbase + 32 * j < g.k_w) {
               const int64_t off = static_cast<int64_t>((kbase + 32 * j) / g.group) * g.n_w + c0;
-              const uint32_t dst = wdst + HQ_W_BYTES + j * HQ_META_SLOT;
+              const uint32_t dst = sw + HQ_W_BYTES + j * HQ_META_SLOT;
               bulk_load_1d(dst, g.scale + off, 2u * cnt, fb);
               bulk_load_1d(dst + HQ_META_HALF, g.zero + off, 2u * cnt, fb);
             }
@@ -430,15 +428,15 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       // every copy issued lands before the CTA can exit
       volatile int never = 0;
       for (long long i = issued > g.np ? issued - g.np : 0; i < issued; ++i)
-        hq_wait(smem_u32(p_full + static_cast<int>(i % g.np)), static_cast<uint32_t>((i / g.np) & 1), g.wait,
-                  &never);
+        hq_wait(smem_u32(full + static_cast<int>(i % g.np)), static_cast<uint32_t>((i / g.np) & 1), g.wait,
+                &never);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, g.bn);
-      int stage = 0, dst = 0, acc = 0;
-      uint32_t phase = 0, dphase = 0, aphase = 0;
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, aphase = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
         const Unit t = decode_unit(g, u);
@@ -446,26 +444,23 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * HQ_ACC_COLS);
         for (int kk = t.k0; kk < t.k1; ++kk) {
-          if (!hq_wait(smem_u32(d_full + dst), dphase, g.wait, abort_flag) ||
-              !hq_wait(smem_u32(p_full + stage), phase, g.wait, abort_flag)) {
+          // the dequantizers waited for the copies, so deq implies full
+          if (!hq_wait(smem_u32(deq + stage), phase, g.wait, abort_flag) ||
+              !hq_wait(smem_u32(full + stage), phase, g.wait, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t ad = smem_desc_kmajor<128>(sA + dst * HQ_A_BYTES);
-          const uint64_t bd = smem_desc_kmajor<128>(sX + stage * x_bytes);
+          const uint32_t sa = base + stage * stage_bytes;
+          const uint64_t ad = smem_desc_kmajor<128>(sa);
+          const uint64_t bd = smem_desc_kmajor<128>(sa + HQ_A_BYTES);
 #pragma unroll
           for (int j = 0; j < 4; ++j)   // K = 16 bf16 = 32 bytes per instruction
             mma_bf16(d_tmem, ad + 2 * j, bd + 2 * j, idesc, (kk > t.k0 || j > 0) ? 1u : 0u);
-          mma_commit(smem_u32(p_empty + stage));
-          mma_commit(smem_u32(d_empty + dst));
+          mma_commit(smem_u32(empty + stage));
           if (++stage == g.np) {
             stage = 0;
             phase ^= 1;
-          }
-          if (++dst == HQ_ND) {
-            dst = 0;
-            dphase ^= 1;
           }
         }
         if (!ok) break;
@@ -482,35 +477,32 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     }
   } else if (warp < HQ_EPI_WARP0) {
     // ---------------------------------------------------------- dequantizers
+    // A stage's A tile is free again once its copies have landed: the
+    // producer refilled the stage only after the MMAs that read it completed.
     const int dt = threadIdx.x - 64;
-    int stage = 0, dst = 0;
-    uint32_t phase = 0, dphase = 0;
+    int stage = 0;
+    uint32_t phase = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
       const Unit t = decode_unit(g, u);
       for (int kk = t.k0; kk < t.k1; ++kk) {
-        bool w = hq_wait(smem_u32(p_full + stage), phase, g.wait, abort_flag);
-        w = w && hq_wait(smem_u32(d_empty + dst), dphase ^ 1, g.wait, abort_flag);
+        const bool w = hq_wait(smem_u32(full + stage), phase, g.wait, abort_flag);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
         }
-        const uint32_t atile = sA + dst * HQ_A_BYTES;
-        const uint32_t wt = sW + stage * HQ_WM_BYTES;
+        const uint32_t sa = base + stage * stage_bytes;
+        const uint32_t wt = sa + HQ_A_BYTES + x_bytes;
         if (TRANS)
-          dequant_tile_t<S4>(g, atile, wt, dt, t.ntile, kk);
+          dequant_tile_t<S4>(g, sa, wt, dt, t.ntile, kk);
         else
-          dequant_tile_fwd<S4>(g, atile, wt, dt, t.ntile, kk);
+          dequant_tile_fwd<S4>(g, sa, wt, dt, t.ntile, kk);
         fence_proxy_async_smem();     // generic-proxy writes -> visible to the MMA
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(d_full + dst));
+        if (lane == 0) mbar_arrive(smem_u32(deq + stage));
         if (++stage == g.np) {
           stage = 0;
           phase ^= 1;
-        }
-        if (++dst == HQ_ND) {
-          dst = 0;
-          dphase ^= 1;
         }
       }
     }
@@ -559,41 +551,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
         acc = 0;
         aphase ^= 1;
       }
-      if (part != nullptr) {
-        // publish this split's slice; the last split to arrive adds all of
-        // them in split order
-        __threadfence();
-        __syncwarp();
-        uint32_t last = 0;
-        if (lane == 0)
-          last = atomicAdd(g.cnt + t.tile * 4 + q, 1u) == static_cast<uint32_t>(g.splits - 1) ? 1u : 0u;
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          __threadfence();
-          const float* const tile_ws = g.ws + static_cast<int64_t>(t.tile) * g.splits * g.bn * 128;
-          for (int c0 = 0; c0 < g.bn; c0 += 32) {
-            const int width = min(32, g.bn - c0);
-            // split by split (a fixed order), the chunk's loads all in flight
-            float sum[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) sum[j] = 0.0f;
-            for (int sp = 0; sp < g.splits; ++sp) {
-              const float* src = tile_ws + (static_cast<int64_t>(sp) * g.bn + c0) * 128 + row;
-              float v[32];
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = j < width ? __ldcg(src + j * 128) : 0.0f;
-#pragma unroll
-              for (int j = 0; j < 32; ++j) sum[j] += v[j];
-            }
-            uint32_t r[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(sum[j]);
-            store_pairs(g, r, width, tok0 + c0, ch, lane);
-          }
-          __syncwarp();
-          if (lane == 0) g.cnt[t.tile * 4 + q] = 0u;   // the workspace is left zeroed
-        }
-      }
+      if (part != nullptr) __threadfence();     // the partial tile is published below
     }
   }
 
@@ -601,6 +559,58 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, HQ_TMEM_COLS);
+
+  // Split contraction (one unit per CTA): the last split of a tile to arrive
+  // adds the tile's partial sums in split order, with every thread of the CTA.
+  if (g.splits > 1 && blockIdx.x < g.units) {
+    const Unit t = decode_unit(g, blockIdx.x);
+    if (threadIdx.x == 0) {
+      int last = 0;
+      if (!*abort_flag) {
+        __threadfence();
+        last = atomicAdd(g.cnt + t.tile * 4, 1u) == static_cast<uint32_t>(g.splits - 1) ? 1 : 0;
+      }
+      *last_flag = last;
+    }
+    __syncthreads();
+    if (*last_flag) {
+      __threadfence();
+      const float* const tile_ws = g.ws + static_cast<int64_t>(t.tile) * g.splits * g.bn * 128;
+      const int quad = threadIdx.x & 31;                 // channels 4 * quad .. + 3
+      const int ch = t.ntile * 128 + 4 * quad;
+      constexpr int ROWS = HQ_THREADS / 32;              // token rows per pass
+      for (int tok0 = (threadIdx.x >> 5) * 4; tok0 < g.bn; tok0 += ROWS * 4) {
+        // four tokens at a time, every split's loads in flight together
+        float4 sum[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sum[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int sp = 0; sp < g.splits; ++sp) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (tok0 + i < g.bn) {
+              const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                                          tile_ws + (static_cast<int64_t>(sp) * g.bn + tok0 + i) * 128) + quad);
+              sum[i].x += v.x;
+              sum[i].y += v.y;
+              sum[i].z += v.z;
+              sum[i].w += v.w;
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = t.ttile * g.bn + tok0 + i;
+          if (tok0 + i < g.bn && m < g.M && ch < g.n_out) {
+            const uint32_t lo = bf16_bits(sum[i].x) | (bf16_bits(sum[i].y) << 16);
+            const uint32_t hi = bf16_bits(sum[i].z) | (bf16_bits(sum[i].w) << 16);
+            *reinterpret_cast<uint2*>(g.out + static_cast<int64_t>(m) * g.n_out + ch) = make_uint2(lo, hi);
+          }
+        }
+      }
+      if (threadIdx.x == 0) g.cnt[t.tile * 4] = 0u;     // the workspace is left zeroed
+    }
+  }
 }
 
 // Standalone dequantization: one thread per packed word (8 codes) -> 16 B of
@@ -684,10 +694,10 @@ HqqPlan plan_hqq(int64_t M, int64_t n_out, int64_t kc, int sm_count, bool allow_
   p.ws_bytes = p.splits > 1 ? p.cnt_bytes + static_cast<size_t>(tiles) * p.splits * p.bn * 128 * sizeof(float) : 0;
   p.units = static_cast<int>(tiles * p.splits);
   p.grid = std::min(p.units, sm_count);
-  const int stage = p.bn * 128 + HQ_WM_BYTES;
-  const int avail = HQ_SMEM_LIMIT - 1024 - HQ_BAR_BYTES - HQ_ND * HQ_A_BYTES;
+  const int stage = HQ_A_BYTES + p.bn * 128 + HQ_WM_BYTES;
+  const int avail = HQ_SMEM_LIMIT - 1024 - HQ_BAR_BYTES;
   p.np = std::min(HQ_MAX_NP, avail / stage);
-  p.smem = 1024 + static_cast<size_t>(HQ_ND) * HQ_A_BYTES + static_cast<size_t>(p.np) * stage + HQ_BAR_BYTES;
+  p.smem = 1024 + static_cast<size_t>(p.np) * stage + HQ_BAR_BYTES;
   return p;
 }
 
@@ -764,9 +774,7 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   g.ks = p.ks;
   g.units = p.units;
   g.np = p.np;
-  g.off_x = static_cast<uint32_t>(HQ_ND * HQ_A_BYTES);
-  g.off_w = g.off_x + static_cast<uint32_t>(p.np * p.bn * 128);
-  g.off_bar = g.off_w + static_cast<uint32_t>(p.np * HQ_WM_BYTES);
+  g.off_bar = static_cast<uint32_t>(p.np) * (HQ_A_BYTES + p.bn * 128 + HQ_WM_BYTES);
   g.scale = static_cast<const uint16_t*>(scale);
   g.zero = static_cast<const uint16_t*>(zero);
   g.out = static_cast<uint16_t*>(out);
