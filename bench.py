@@ -58,6 +58,8 @@ KERNEL_SOURCES = {
     "dq_int8_linear": _GEMM_SOURCES,
     "dq_bsr_int8_linear": _GEMM_SOURCES,
     "dq_fp8_linear": _GEMM_SOURCES,
+    "dq_hqq_linear": ("hqq.cu", "sm100.cuh", "host.cu", "internal.h"),
+    "dq_hqq_linear_t": ("hqq.cu", "sm100.cuh", "host.cu", "internal.h"),
 }
 
 
