@@ -336,8 +336,8 @@ void oracle_gemm_fp8_f64(const uint8_t* A, int64_t M, int64_t K, int64_t lda,
  *   - the product is the plain bf16 matmul of activations and dequantized
  *     weight: out[m, n] = sum_k x[m, k] * w[n, k] (forward), and the
  *     transposed product out[m, k] = sum_n y[m, n] * w[n, k] used for the
- *     input gradient in the backward pass ("handles both transposed and
- *     non-transposed quantized weights").
+ *     input gradient in the backward pass (the page's kernel serves both the
+ *     forward and the backward orientation of the packed weight).
  */
 
 /* Rounds a finite double to bf16 (8 significant bits), to nearest, ties to
