@@ -28,6 +28,10 @@ vLLM csrc/quantization commits: dynamic scales, clamp to the e4m3 range):
     a bf16 matmul, forward and transposed ("Fused HQQ Quantization Gemm",
     pytorch/ao PR 153, description and implementation details):
     w = bf16(bf16(q - z) * s) per group of K.
+  * s24_compress / s24_decompress -- 2:4 semi-structured sparse int8 weight
+    ("sparse_fc supported", PaddlePaddle PR 41770: 2:4-sparse FC weights
+    compressed on the device); the product is gemm_s32 on the decompressed
+    weight, then epilogue_bf16.
 """
 import ctypes
 import os
@@ -77,6 +81,9 @@ def _load():
         lib.oracle_hqq_dequant.argtypes = [P, P, P, I, I, I, Ci, P]
         lib.oracle_hqq_linear_f64.argtypes = [P, P, I, I, I, P]
         lib.oracle_hqq_linear_t_f64.argtypes = [P, P, I, I, I, P]
+        lib.oracle_s24_compress.argtypes = [P, I, I, P, P]
+        lib.oracle_s24_compress.restype = ctypes.c_int64
+        lib.oracle_s24_decompress.argtypes = [P, P, I, I, P]
         _lib = lib
     return _lib
 
@@ -312,3 +319,26 @@ def hqq_linear_t_f64(y_bits, w_bits) -> np.ndarray:
     out = np.empty((M, K), np.float64)
     _load().oracle_hqq_linear_t_f64(_ptr(y), _ptr(w), M, N, K, _ptr(out))
     return out
+
+
+def s24_compress(W: np.ndarray):
+    """Wq int8 [N, K] (K % 8 == 0) -> (values int8 [N, K/2], meta uint8 [N, K/8], groups with > 2 nonzeros)."""
+    W = _c(W, np.int8)
+    N, K = W.shape
+    assert K % 8 == 0
+    values = np.empty((N, K // 2), np.int8)
+    meta = np.zeros((N, K // 8), np.uint8)
+    bad = _load().oracle_s24_compress(_ptr(W), N, K, _ptr(values), _ptr(meta))
+    return values, meta, int(bad)
+
+
+def s24_decompress(values: np.ndarray, meta: np.ndarray) -> np.ndarray:
+    """(values [N, K/2], meta [N, K/8]) -> Wq int8 [N, K]."""
+    v = _c(values, np.int8)
+    m = _c(meta, np.uint8)
+    N, H = v.shape
+    K = 2 * H
+    assert m.shape == (N, K // 8)
+    W = np.empty((N, K), np.int8)
+    _load().oracle_s24_decompress(_ptr(v), _ptr(m), N, K, _ptr(W))
+    return W

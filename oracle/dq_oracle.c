@@ -433,3 +433,68 @@ void oracle_hqq_linear_t_f64(const uint16_t* y, const uint16_t* w, int64_t M, in
             out[m * K + k] = s;
         }
 }
+
+/* ---- 2:4 semi-structured sparse int8 weight -----------------------------
+ *
+ * "sparse_fc supported" (PaddlePaddle PR 41770, description and the
+ * SpmmPluginDynamic review): fully connected layers whose weights are
+ * already 2:4 sparse (at most two nonzeros in every group of four
+ * consecutive in-features) run through a 2:4 sparse matmul after the weight
+ * is compressed on the device; the quantized layer computes the same int8
+ * product and dequantization as the dense one.  The compressed form is this
+ * library's own (the page's comes from a closed library):
+ *   values [N, K/2] int8: group g of row n keeps two values, values[2g] and
+ *     values[2g+1], found at positions p0 < p1 (0..3) of the group;
+ *   meta [N, K/8] uint8: byte b holds group 2b in bits 0..3 and group 2b+1
+ *     in bits 4..7, each as p0 | p1 << 2.
+ *   A group with fewer than two nonzeros keeps its nonzero positions and
+ *   fills up with the lowest free positions (their values are zero).
+ * The product itself is the plain int8 GEMM of the activations with the
+ * decompressed weight (oracle_gemm_s32), then the same bf16 epilogue.
+ */
+
+/* Wq int8 [N, K] (K % 8 == 0) -> values, meta.  Returns the number of
+ * groups with more than two nonzeros (those keep their two lowest nonzero
+ * positions). */
+int64_t oracle_s24_compress(const int8_t* W, int64_t N, int64_t K, int8_t* values, uint8_t* meta) {
+    int64_t bad = 0;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < K / 4; ++g) {
+            const int8_t* grp = W + n * K + 4 * g;
+            int pos[2];
+            int cnt = 0, nz = 0;
+            for (int j = 0; j < 4; ++j)
+                if (grp[j] != 0) {
+                    ++nz;
+                    if (cnt < 2) pos[cnt++] = j;
+                }
+            if (nz > 2) ++bad;
+            for (int j = 0; j < 4 && cnt < 2; ++j) {       /* fill with the lowest free positions */
+                if (cnt == 1 && pos[0] == j) continue;
+                if (grp[j] == 0) pos[cnt++] = j;
+            }
+            if (pos[0] > pos[1]) { const int t = pos[0]; pos[0] = pos[1]; pos[1] = t; }
+            values[n * (K / 2) + 2 * g] = grp[pos[0]];
+            values[n * (K / 2) + 2 * g + 1] = grp[pos[1]];
+            const uint8_t nib = (uint8_t)(pos[0] | (pos[1] << 2));
+            uint8_t* mb = meta + n * (K / 8) + g / 2;
+            if (g % 2 == 0) *mb = (uint8_t)((*mb & 0xf0u) | nib);
+            else *mb = (uint8_t)((*mb & 0x0fu) | (nib << 4));
+        }
+    }
+    return bad;
+}
+
+/* values, meta -> Wq int8 [N, K] (zeros outside the kept positions; a
+ * group whose two positions coincide adds both values there). */
+void oracle_s24_decompress(const int8_t* values, const uint8_t* meta, int64_t N, int64_t K, int8_t* W) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < K / 4; ++g) {
+            const uint8_t mb = meta[n * (K / 8) + g / 2];
+            const uint8_t nib = (g % 2 == 0) ? (uint8_t)(mb & 0x0fu) : (uint8_t)(mb >> 4);
+            int8_t* grp = W + n * K + 4 * g;
+            for (int j = 0; j < 4; ++j) grp[j] = 0;
+            grp[nib & 3] = (int8_t)(grp[nib & 3] + values[n * (K / 2) + 2 * g]);
+            grp[(nib >> 2) & 3] = (int8_t)(grp[(nib >> 2) & 3] + values[n * (K / 2) + 2 * g + 1]);
+        }
+}

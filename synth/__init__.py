@@ -168,3 +168,22 @@ def hqq(seed: int = 0, M: int = 16, N: int = 4096, K: int = 4096, group: int = 1
                 scale=f32_to_bf16_bits(uniform_f32((N, G), 0.002, 0.02, seed + 5)),
                 zero=f32_to_bf16_bits(uniform_f32((N, G), zlo, zhi, seed + 6)),
                 group=group, signed=signed)
+
+
+def s24_mask(N: int, K: int, seed: int) -> np.ndarray:
+    """bool [N, K]: in every group of four consecutive in-features exactly
+    two kept positions, each of the six pairs equally likely."""
+    pairs = np.array([[0, 1], [0, 2], [0, 3], [1, 2], [1, 3], [2, 3]], np.int64)
+    choice = rng(seed).integers(0, 6, size=(N, K // 4))
+    mask = np.zeros((N, K // 4, 4), bool)
+    sel = pairs[choice]                                   # [N, K/4, 2]
+    np.put_along_axis(mask, sel, True, axis=2)
+    return mask.reshape(N, K)
+
+
+def s24(seed: int = 0, M: int = 2048, K: int = 4096, N: int = 4096):
+    """2:4-sparse linear: X bf16 [M, K] ~ N(0, 1); W fp32 [N, K] ~ N(0, 0.02)
+    zeroed outside a uniform 2:4 mask (seed+3)."""
+    w = normal_f32((N, K), 0.02, seed + 1)
+    w[~s24_mask(N, K, seed + 3)] = 0.0
+    return dict(name=f"2:4 sparse linear M={M} K={K} N={N}", x=normal_bf16((M, K), 1.0, seed), w=w)
