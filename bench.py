@@ -59,6 +59,7 @@ KERNEL_SOURCES = {
     "dq_bsr_int8_linear": _GEMM_SOURCES,
     "dq_fp8_linear": _GEMM_SOURCES,
     "dq_hqq_linear": ("hqq.cu", "sm100.cuh", "host.cu", "internal.h"),
+    "dq_s24_int8_linear": ("sparse24.cu", "pipeline.cuh", "sm100.cuh", "host.cu", "internal.h"),
     "dq_hqq_linear_t": ("hqq.cu", "sm100.cuh", "host.cu", "internal.h"),
 }
 
@@ -140,6 +141,10 @@ WORKLOADS = {
                     desc="weight-only int4 (HQQ u4, group 128) linear M=512 N=4096 K=4096, dequant fused into a bf16 GEMM"),
     "hqq_m1024": dict(kind="hqq", M=1024, N=4096, K=4096, group=128,
                     desc="weight-only int4 (HQQ u4, group 128) linear M=1024 N=4096 K=4096, dequant fused into a bf16 GEMM"),
+    "s24_llm": dict(kind="s24", M=2048, K=4096, N=4096,
+                    desc="2:4-sparse int8 linear M=2048 K=4096 N=4096 (per-token quant + compressed-weight GEMM, fused bf16 epilogue)"),
+    "s24_small_m16": dict(kind="s24", M=16, K=8192, N=28672,
+                          desc="2:4-sparse int8 linear M=16 K=8192 N=28672 (weight stream, compressed)"),
     "hqq_t_m1024": dict(kind="hqq", M=1024, N=4096, K=4096, group=128, transposed=True,
                         desc="transposed int4 (HQQ u4, group 128) product M=1024 N=4096 K=4096 (input gradient)"),
     "small_m1": dict(kind="dense", M=1, K=8192, N=28672, desc="small-M dense linear M=1 K=8192 N=28672"),
@@ -168,6 +173,8 @@ def _synth_inputs(name, wl, seed):
         return synth.vit_h_bsr(seed, wl["layer"], keep=wl.get("keep", 0.10), bs=wl.get("bs", 64))
     if k == "quant":
         return synth.quant_sweep(seed)
+    if k == "s24":
+        return synth.s24(seed, M=wl["M"], K=wl["K"], N=wl["N"])
     if k == "hqq":
         d = synth.hqq(seed, M=wl["M"], N=wl["N"], K=wl["K"], group=wl["group"])
         if wl.get("transposed"):
@@ -197,6 +204,11 @@ def step_accounting(wl, d):
     if k == "quant":
         M, K = wl["M"], wl["K"]
         return 0.0, dict(kernel="dq_quantize_rows", ops=0.0, bytes=3 * M * K + 4 * M, quant_bytes=3 * M * K + 4 * M)
+    if k == "s24":
+        M, K, N = wl["M"], wl["K"], wl["N"]
+        ops = 2.0 * M * N * K          # dense-equivalent work of the 2:4 product
+        gemm_bytes = M * K + N * K // 2 + N * K // 8 + 2 * M * N + 4 * (M + N)
+        return ops, dict(kernel="dq_s24_int8_linear", ops=ops, bytes=gemm_bytes, quant_bytes=3 * M * K + 4 * M)
     if k == "hqq":
         M, K, N = wl["M"], wl["K"], wl["N"]
         ops = 2.0 * M * N * K
@@ -375,6 +387,30 @@ def make_state(name, wl, dq, torch, seed):
             lambda c, stream: dq.dq_quantize_rows(c["x"], q, s, stream=stream),
             lambda c, stream: dq.dq_int8_linear(q, s, c["W"], sc, bias=bias, out=out, workspace=ws, stream=stream)]
         st["names"] = ["dq_quantize_rows", "dq_int8_linear"]
+        return _finish(st)
+    if k == "s24":
+        w = _to_dev(torch, d["w"])
+        wq, sc = dq.dq_quantize_weight(w)
+        del w
+        vals, meta = dq.dq_s24_compress(wq)
+        del wq
+        M, K, N = wl["M"], wl["K"], wl["N"]
+        x = _to_dev_bf16(torch, d["x"])
+        n = _ncopies(x.numel() * 2 + vals.numel() + meta.numel())
+        st["copies"] = [dict(x=x if i == 0 else x.clone(), V=vals if i == 0 else vals.clone(),
+                             Mt=meta if i == 0 else meta.clone()) for i in range(n)]
+        q = torch.empty((M, K), dtype=torch.int8, device="cuda")
+        s = torch.empty((M,), dtype=torch.float32, device="cuda")
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        nws = dq.dq_s24_workspace_size(M, N, K)
+        ws = torch.zeros(nws, dtype=torch.uint8, device="cuda") if nws else None
+        st.update(q=q, s=s, out=out, ws=ws)
+        st["h2d"] = [("x", M * K * 2)]
+        st["d2h"] = [("out", M * N * 2)]
+        st["kernels"] = [
+            lambda c, stream: dq.dq_quantize_rows(c["x"], q, s, stream=stream),
+            lambda c, stream: dq.dq_s24_int8_linear(q, s, c["V"], c["Mt"], sc, out=out, workspace=ws, stream=stream)]
+        st["names"] = ["dq_quantize_rows", "dq_s24_int8_linear"]
         return _finish(st)
     if k == "hqq":
         trans = bool(wl.get("transposed"))
@@ -570,6 +606,8 @@ def run_gpu(args, rank, world, local_rank):
         hbm_bound = False
     if dom["kernel"].startswith("dq_int8_linear") and wl["kind"] == "dense" and wl["M"] <= 128:
         hbm_bound = True     # small-M: weight streaming
+    if wl["kind"] == "s24":
+        hbm_bound = dom["bytes"] / (peaks["hbm_gbs"] * 1e9) >= dom["ops"] / (int8_peak * 1e12)
     hqq = wl["kind"] == "hqq"
     if hqq:
         int8_peak = peaks["bf16"]      # bf16 operands on the tensor cores
@@ -594,7 +632,7 @@ def run_gpu(args, rank, world, local_rank):
 
     # end to end through the public API with host buffers
     e2e = None
-    if wl["kind"] in ("dense", "bsr", "bsr_dense", "quant", "gemm", "dense_fp8", "hqq"):
+    if wl["kind"] in ("dense", "bsr", "bsr_dense", "quant", "gemm", "dense_fp8", "hqq", "s24"):
         e2e = run_e2e(args, wl, state, dq, torch, stream, ops, dom, world, max_over_ranks)
 
     vs_baseline = None

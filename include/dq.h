@@ -347,6 +347,42 @@ DQ_API dq_status dq_hqq_linear_t(const void* y_bf16, int64_t M, const uint8_t* p
                                  void* out_bf16, void* workspace, size_t workspace_bytes, dq_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * 2:4 semi-structured sparse int8 weight ("sparse_fc supported",
+ * PaddlePaddle PR 41770: FC weights with at most two nonzeros in every group
+ * of four consecutive in-features, compressed on the device; its review asks
+ * for the int8 product with only the dequantization fused and a 16-bit
+ * output).
+ *
+ * dq_s24_compress: wq int8 [N, K] (K % 8 == 0, row-major) ->
+ *   values int8 [N, K/2]: the two kept values of each group, in position order;
+ *   meta uint8 [N, K/8]: per group the nibble p0 | p1 << 2 (kept positions
+ *     p0 < p1), group 2b in the low nibble of byte b.
+ *   A group with fewer than two nonzeros keeps them and fills up with its
+ *   lowest free positions.  Groups with more than two nonzeros keep their two
+ *   lowest nonzero positions and are counted into *violations (device int32,
+ *   added to atomically; may be NULL).  wq 8-byte and values 4-byte aligned.
+ * dq_s24_int8_linear: out = the int8 layer of dq_int8_linear with the weight
+ *   given compressed: acc[m, n] = sum_k A[m, k] * W[n, k] (exact int32, W the
+ *   decompressed weight), then DQ_OUT_BF16: bf16((acc * s_row[m]) * s_col[n]
+ *   + bias[n]) or DQ_OUT_S32: acc.  A int8 [M, K] contiguous.  The kernel
+ *   expands the compressed weight in shared memory and multiplies on the
+ *   tensor cores (tcgen05.mma kind::i8); the weight crosses HBM compressed
+ *   (5/8 of its dense int8 bytes).  meta nibbles must have p0 < p1 (as
+ *   dq_s24_compress writes them); other nibbles give unspecified (but
+ *   in-bounds) results.  Requirements: K % 128 == 0, N % 8 == 0, M >= 0,
+ *   pointers 16-byte aligned.  workspace / workspace_bytes: as for
+ *   dq_hqq_linear (dq_s24_workspace_size; zero-filled before first use; left
+ *   zeroed; int32 partials, so results never depend on the split).
+ * ------------------------------------------------------------------------ */
+DQ_API dq_status dq_s24_compress(const int8_t* wq, int64_t N, int64_t K, int8_t* values, uint8_t* meta,
+                                 int32_t* violations, dq_stream_t stream);
+DQ_API size_t dq_s24_workspace_size(int64_t M, int64_t N, int64_t K);
+DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K, const int8_t* values,
+                                    const uint8_t* meta, const float* s_col, int64_t N, const void* bias_bf16,
+                                    void* out, dq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                    dq_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Measurement helper: a kernel that only issues tcgen05.mma.kind::i8
  * (128x256x32, operands resident in shared memory, accumulator in TMEM) on
  * every SM, `iters` times per CTA, with no global-memory traffic.  Used to

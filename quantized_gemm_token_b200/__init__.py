@@ -57,6 +57,9 @@ _PROTOS = {
     "dq_hqq_dequantize": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I32, _P, _P]),
     "dq_hqq_workspace_size": (_SZ, [_I64, _I64, _I64, _I32]),
     "dq_hqq_group_major": (_I32, [_P, _I64, _I64, _P, _P]),
+    "dq_s24_compress": (_I32, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "dq_s24_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "dq_s24_int8_linear": (_I32, [_P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _I32, _P, _SZ, _P]),
     "dq_hqq_linear": (_I32, [_P, _I64, _P, _P, _P, _I64, _I64, _I32, _I32, _P, _P, _SZ, _P]),
     "dq_hqq_linear_t": (_I32, [_P, _I64, _P, _P, _P, _I64, _I64, _I32, _I32, _P, _P, _SZ, _P]),
 }
@@ -548,6 +551,66 @@ class HqqLinear:
         ws = self._workspace(grad_out.shape[0], True, grad_out.device)
         return dq_hqq_linear_t(grad_out, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
                                workspace=ws, stream=stream)
+
+
+# ---------------------------------------------------------------- 2:4 sparse
+
+def dq_s24_compress(wq: torch.Tensor, values: torch.Tensor = None, meta: torch.Tensor = None,
+                    violations: torch.Tensor = None, stream=None):
+    """2:4-sparse int8 weight [N, K] -> (values int8 [N, K/2], meta uint8 [N, K/8]).
+    `violations` (int32 CUDA tensor of one element, optional) counts groups
+    with more than two nonzeros."""
+    _need(wq, torch.int8, "wq", 2)
+    _contig(wq, "wq")
+    N, K = wq.shape
+    if values is None:
+        values = torch.empty((N, K // 2), dtype=torch.int8, device=wq.device)
+    if meta is None:
+        meta = torch.empty((N, K // 8), dtype=torch.uint8, device=wq.device)
+    _need(values, torch.int8, "values", 2)
+    _need(meta, torch.uint8, "meta", 2)
+    if violations is not None:
+        _need(violations, torch.int32, "violations")
+    _check(lib.dq_s24_compress(_ptr(wq), N, K, _ptr(values), _ptr(meta), _ptr(violations), _stream(stream)),
+           "dq_s24_compress")
+    return values, meta
+
+
+def dq_s24_workspace_size(M: int, N: int, K: int) -> int:
+    return int(lib.dq_s24_workspace_size(M, N, K))
+
+
+def dq_s24_int8_linear(A, s_row, values, meta, s_col, bias=None, out=None, out_dtype="bf16", workspace=None,
+                       stream=None):
+    """The int8 layer with a compressed 2:4 weight: out[M, N] = bf16(acc * s_row
+    * s_col + bias), acc = A @ W^T exactly (W decompressed), or acc as int32."""
+    code = _out_code(out_dtype)
+    _need(A, torch.int8, "A", 2)
+    _need(values, torch.int8, "values", 2)
+    _need(meta, torch.uint8, "meta", 2)
+    for t, n in ((A, "A"), (values, "values"), (meta, "meta")):
+        _contig(t, n)
+    M, K = A.shape
+    N = values.shape[0]
+    if values.shape[1] * 2 != K or tuple(meta.shape) != (N, K // 8):
+        raise ValueError("values must be [N, K/2] and meta [N, K/8]")
+    if code == DQ_OUT_BF16:
+        _need(s_row, torch.float32, "s_row", 1)
+        _need(s_col, torch.float32, "s_col", 1)
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias", 1)
+    odt = torch.bfloat16 if code == DQ_OUT_BF16 else torch.int32
+    if out is None:
+        out = torch.empty((M, N), dtype=odt, device=A.device)
+    _need(out, odt, "out", 2)
+    _contig(out, "out")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _need(workspace, torch.uint8, "workspace")
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()
+    _check(lib.dq_s24_int8_linear(_ptr(A), _ptr(s_row), M, K, _ptr(values), _ptr(meta), _ptr(s_col), N, _ptr(bias),
+                                  _ptr(out), code, ws_ptr, ws_bytes, _stream(stream)), "dq_s24_int8_linear")
+    return out
 
 
 # ---------------------------------------------------------------- layer
