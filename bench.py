@@ -58,9 +58,9 @@ KERNEL_SOURCES = {
     "dq_int8_linear": _GEMM_SOURCES,
     "dq_bsr_int8_linear": _GEMM_SOURCES,
     "dq_fp8_linear": _GEMM_SOURCES,
-    "dq_hqq_linear": ("hqq.cu", "sm100.cuh", "host.cu", "internal.h"),
+    "dq_hqq_linear": ("hqq.cu", "pipeline.cuh", "sm100.cuh", "host.cu", "internal.h"),
     "dq_s24_int8_linear": ("sparse24.cu", "pipeline.cuh", "sm100.cuh", "host.cu", "internal.h"),
-    "dq_hqq_linear_t": ("hqq.cu", "sm100.cuh", "host.cu", "internal.h"),
+    "dq_hqq_linear_t": ("hqq.cu", "pipeline.cuh", "sm100.cuh", "host.cu", "internal.h"),
 }
 
 

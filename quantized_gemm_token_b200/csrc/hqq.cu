@@ -31,6 +31,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "pipeline.cuh"
 #include "sm100.cuh"
 
 namespace dq {
@@ -119,74 +120,6 @@ __device__ __forceinline__ uint32_t bf16_pair_of(uint16_t v) {
   return static_cast<uint32_t>(v) | (static_cast<uint32_t>(v) << 16);
 }
 
-// Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128B-swizzled
-// K-major tile (rows of 128 B; the chunk index is XORed with r mod 8, the
-// layout a SWIZZLE_128B tensor copy produces).
-__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
-  return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&v)[4]) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]),
-               "r"(v[3])
-               : "memory");
-}
-
-// Bounded wait on an mbarrier phase that sleeps instead of spinning: each
-// try_wait may suspend the thread (up to kSuspendNs) until the phase
-// completes, so waiting warps take no issue slots from the working ones.
-// Gives up like mbar_wait: after ctl.timeout_ns, or once *abort is raised.
-constexpr uint32_t kSuspendNs = 200000;
-__device__ __forceinline__ bool try_wait_sleep(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kSuspendNs)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool hq_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl, volatile int* abort) {
-  if (try_wait_sleep(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    if (try_wait_sleep(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer() - t0 > ctl.timeout_ns) {
-      atomicOr(ctl.err, kErrTimeout);
-      *abort = 1;
-      return false;
-    }
-  }
-}
-
-// Shared-memory loads by 32-bit shared address.
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds8(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
-}
-
-// 1-D bulk copy global -> shared completing `bar`'s transaction count (both
-// addresses 16-byte aligned, bytes a multiple of 16).
-__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-               : "memory");
-}
-
 // The meta slot holding the group of 32-deep k slice j: the first slice of
 // each group (groups of 32 start at every slice, groups of 64 at even ones,
 // larger groups at slice 0 of a step or tile).
@@ -223,21 +156,21 @@ __device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t atil
                                                  int kstep) {
   const int r = dt & 127;
   const int h = dt >> 7;
-  const uint4 pk = lds128(wtile + r * 32 + h * 16);
+  const uint4 pk = pipe::lds128(wtile + r * 32 + h * 16);
   const int n = ntile * 128 + r;
   const int k = kstep * HQ_BK + h * 32;
   uint32_t s2 = 0, z2 = 0;
   if (n < g.n_w && k < g.k_w) {
     const uint32_t meta = wtile + HQ_W_BYTES + meta_slot(h, g.group) * HQ_META_SLOT + 2 * r;
-    s2 = bf16_pair_of(static_cast<uint16_t>(lds16(meta)));
-    z2 = bf16_pair_of(static_cast<uint16_t>(lds16(meta + HQ_META_HALF)));
+    s2 = bf16_pair_of(static_cast<uint16_t>(pipe::lds16(meta)));
+    z2 = bf16_pair_of(static_cast<uint16_t>(pipe::lds16(meta + HQ_META_HALF)));
   }
   const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     uint32_t o[4];
     dequant8<S4>(words[i], z2, s2, o);
-    st_shared_v4(atile + sw128_off(r, 4 * h + i), o);
+    pipe::sts128(atile + pipe::sw128_off(r, 4 * h + i), o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -261,8 +194,8 @@ __device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile,
     uint4 s8 = make_uint4(0, 0, 0, 0), z8 = make_uint4(0, 0, 0, 0);
     if (n_ok && k < g.k_w) {
       const uint32_t meta = wtile + HQ_W_BYTES + meta_slot(b >> 4, g.group) * HQ_META_SLOT + nc * 16;
-      s8 = lds128(meta);
-      z8 = lds128(meta + HQ_META_HALF);
+      s8 = pipe::lds128(meta);
+      z8 = pipe::lds128(meta + HQ_META_HALF);
     }
     const uint32_t sp[4] = {s8.x, s8.y, s8.z, s8.w};
     const uint32_t zp[4] = {z8.x, z8.y, z8.z, z8.w};
@@ -270,8 +203,8 @@ __device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile,
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       // weight rows n0 + 2i and n0 + 2i + 1
-      const uint32_t b0 = lds8(wtile + (nc * 8 + 2 * i) * 64 + b);
-      const uint32_t b1 = lds8(wtile + (nc * 8 + 2 * i + 1) * 64 + b);
+      const uint32_t b0 = pipe::lds8(wtile + (nc * 8 + 2 * i) * 64 + b);
+      const uint32_t b1 = pipe::lds8(wtile + (nc * 8 + 2 * i + 1) * 64 + b);
       uint32_t x = b0 | (b1 << 16);
       if (S4) x ^= 0x00880088u;
       const uint32_t pl = (x & 0x000F000Fu) | 0x43004300u;          // k = 2b: rows 2i, 2i + 1
@@ -279,8 +212,8 @@ __device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile,
       lo[i] = bmul2(bsub2(bsub2(pl, code_bias2<S4>()), zp[i]), sp[i]);
       hi[i] = bmul2(bsub2(bsub2(ph, code_bias2<S4>()), zp[i]), sp[i]);
     }
-    st_shared_v4(atile + sw128_off(2 * b, nc), lo);
-    st_shared_v4(atile + sw128_off(2 * b + 1, nc), hi);
+    pipe::sts128(atile + pipe::sw128_off(2 * b, nc), lo[0], lo[1], lo[2], lo[3]);
+    pipe::sts128(atile + pipe::sw128_off(2 * b + 1, nc), hi[0], hi[1], hi[2], hi[3]);
   }
 }
 
@@ -388,7 +321,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
         const Unit t = decode_unit(g, u);
         for (int kk = t.k0; kk < t.k1; ++kk) {
-          if (!hq_wait(smem_u32(empty + stage), phase ^ 1, g.wait, abort_flag)) {
+          if (!pipe::wait(smem_u32(empty + stage), phase ^ 1, g.wait, abort_flag)) {
             ok = false;
             break;
           }
@@ -414,8 +347,8 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
             if (cnt > 0 && j % per == 0 && kbase + 32 * j < g.k_w) {
               const int64_t off = static_cast<int64_t>((kbase + 32 * j) / g.group) * g.n_w + c0;
               const uint32_t dst = sw + HQ_W_BYTES + j * HQ_META_SLOT;
-              bulk_load_1d(dst, g.scale + off, 2u * cnt, fb);
-              bulk_load_1d(dst + HQ_META_HALF, g.zero + off, 2u * cnt, fb);
+              pipe::bulk_load_1d(dst, g.scale + off, 2u * cnt, fb);
+              pipe::bulk_load_1d(dst + HQ_META_HALF, g.zero + off, 2u * cnt, fb);
             }
           }
           ++issued;
@@ -428,7 +361,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       // every copy issued lands before the CTA can exit
       volatile int never = 0;
       for (long long i = issued > g.np ? issued - g.np : 0; i < issued; ++i)
-        hq_wait(smem_u32(full + static_cast<int>(i % g.np)), static_cast<uint32_t>((i / g.np) & 1), g.wait,
+        pipe::wait(smem_u32(full + static_cast<int>(i % g.np)), static_cast<uint32_t>((i / g.np) & 1), g.wait,
                 &never);
     }
   } else if (warp == 1) {
@@ -440,13 +373,13 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       bool ok = true;
       for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
         const Unit t = decode_unit(g, u);
-        if (!hq_wait(smem_u32(acce + acc), aphase ^ 1, g.wait, abort_flag)) break;
+        if (!pipe::wait(smem_u32(acce + acc), aphase ^ 1, g.wait, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * HQ_ACC_COLS);
         for (int kk = t.k0; kk < t.k1; ++kk) {
           // the dequantizers waited for the copies, so deq implies full
-          if (!hq_wait(smem_u32(deq + stage), phase, g.wait, abort_flag) ||
-              !hq_wait(smem_u32(full + stage), phase, g.wait, abort_flag)) {
+          if (!pipe::wait(smem_u32(deq + stage), phase, g.wait, abort_flag) ||
+              !pipe::wait(smem_u32(full + stage), phase, g.wait, abort_flag)) {
             ok = false;
             break;
           }
@@ -473,7 +406,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       // every MMA issued has completed once drain flips
       mma_commit(smem_u32(drain));
       volatile int never = 0;
-      hq_wait(smem_u32(drain), 0, g.wait, &never);
+      pipe::wait(smem_u32(drain), 0, g.wait, &never);
     }
   } else if (warp < HQ_EPI_WARP0) {
     // ---------------------------------------------------------- dequantizers
@@ -486,7 +419,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
       const Unit t = decode_unit(g, u);
       for (int kk = t.k0; kk < t.k1; ++kk) {
-        const bool w = hq_wait(smem_u32(full + stage), phase, g.wait, abort_flag);
+        const bool w = pipe::wait(smem_u32(full + stage), phase, g.wait, abort_flag);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
@@ -514,7 +447,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     uint32_t aphase = 0;
     for (int u = blockIdx.x; u < g.units; u += gridDim.x) {
       const Unit t = decode_unit(g, u);
-      const bool w = hq_wait(smem_u32(accf + acc), aphase, g.wait, abort_flag);
+      const bool w = pipe::wait(smem_u32(accf + acc), aphase, g.wait, abort_flag);
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * HQ_ACC_COLS);
