@@ -324,10 +324,14 @@ DQ_API dq_status dq_fp8_linear(const uint8_t* A, const float* s_row, int64_t M, 
  * workspace: optional caller-owned device scratch that lets few-token calls
  * split the contraction over more SMs (the split partial sums are added in
  * a fixed order, so results do not depend on timing).  Its usable size is
- * dq_hqq_workspace_size(); NULL or a smaller buffer disables splitting.  It
- * must be ZERO-FILLED before its first use; every call leaves it zeroed again
- * (unless a call reports DQ_ERR_TIMEOUT, after which it must be re-zeroed).
- * Calls that may run at the same time must not share a workspace.
+ * dq_hqq_workspace_size(); NULL or a smaller buffer disables splitting.  Its
+ * first bytes hold one arrival counter per tile, the rest the split partial
+ * sums.  The counters must be zero when a call starts and every completed
+ * call leaves them zero; the partial sums are left behind.  So a workspace
+ * ZERO-FILLED once serves any number of calls of one shape (M, N, K,
+ * direction); for another shape zero it again or keep one per shape, and
+ * re-zero it after DQ_ERR_TIMEOUT.  Calls that may run at the same time must
+ * not share a workspace.
  * ------------------------------------------------------------------------ */
 enum { DQ_HQQ_S4 = 1 };
 
@@ -371,8 +375,8 @@ DQ_API dq_status dq_hqq_linear_t(const void* y_bf16, int64_t M, const uint8_t* p
  *   dq_s24_compress writes them); other nibbles give unspecified (but
  *   in-bounds) results.  Requirements: K % 128 == 0, N % 8 == 0, M >= 0,
  *   pointers 16-byte aligned.  workspace / workspace_bytes: as for
- *   dq_hqq_linear (dq_s24_workspace_size; zero-filled before first use; left
- *   zeroed; int32 partials, so results never depend on the split).
+ *   dq_hqq_linear (dq_s24_workspace_size; one zero-filled workspace per
+ *   shape; int32 partials, so results never depend on the split).
  * ------------------------------------------------------------------------ */
 DQ_API dq_status dq_s24_compress(const int8_t* wq, int64_t N, int64_t K, int8_t* values, uint8_t* meta,
                                  int32_t* violations, dq_stream_t stream);

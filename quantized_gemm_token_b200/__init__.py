@@ -507,7 +507,8 @@ def dq_hqq_linear(x, packed, scale, zero, group: int, signed: bool = False, out=
                   stream=None):
     """out[M, N] = x[M, K] @ w^T with w the dequantized int4 weight [N, K]
     (dequantization fused into the tensor-core GEMM).  `workspace`: optional
-    zero-filled uint8 CUDA tensor (dq_hqq_workspace_size) for few-token calls."""
+    uint8 CUDA tensor (dq_hqq_workspace_size) for few-token calls, zero-filled
+    once and kept for calls of this one shape."""
     return _hqq_call(lib.dq_hqq_linear, "dq_hqq_linear", x, packed, scale, zero, group, signed, out,
                      workspace, stream, False)
 
@@ -583,7 +584,8 @@ def dq_s24_workspace_size(M: int, N: int, K: int) -> int:
 def dq_s24_int8_linear(A, s_row, values, meta, s_col, bias=None, out=None, out_dtype="bf16", workspace=None,
                        stream=None):
     """The int8 layer with a compressed 2:4 weight: out[M, N] = bf16(acc * s_row
-    * s_col + bias), acc = A @ W^T exactly (W decompressed), or acc as int32."""
+    * s_col + bias), acc = A @ W^T exactly (W decompressed), or acc as int32.
+    `workspace`: as for dq_hqq_linear (dq_s24_workspace_size, one per shape)."""
     code = _out_code(out_dtype)
     _need(A, torch.int8, "A", 2)
     _need(values, torch.int8, "values", 2)
@@ -660,3 +662,39 @@ class Int8DynamicLinear:
         b = self.bsr
         return dq_bsr_int8_linear(q, s, self.N, b["crow"], b["col"], b["values"], self.s_col, self.bias,
                                   out=out, stream=stream)
+
+
+class S24Int8Linear:
+    """The int8 dynamic-quantization layer with a 2:4-sparse weight: the fp32
+    weight (already 2:4 sparse) is quantized per channel and compressed once;
+    each call quantizes the bf16 activations per token and runs the
+    compressed-weight GEMM with the fused epilogue.  Split workspaces are kept
+    per token count (a workspace serves one shape)."""
+
+    def __init__(self, values, meta, s_col, bias=None):
+        self.values, self.meta, self.s_col, self.bias = values, meta, s_col, bias
+        self.N, self.K = values.shape[0], values.shape[1] * 2
+        self._q = self._s = None
+        self._ws = {}
+
+    @classmethod
+    def from_float(cls, w: torch.Tensor, bias: torch.Tensor = None, violations: torch.Tensor = None):
+        """w: fp32 [N, K] with at most two nonzeros in every four consecutive
+        in-features (`violations`, optional int32 CUDA tensor, counts the
+        groups that have more)."""
+        wq, s_col = dq_quantize_weight(w)
+        values, meta = dq_s24_compress(wq, violations=violations)
+        return cls(values, meta, s_col, bias)
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor = None, stream=None):
+        M = x.shape[0]
+        if self._q is None or self._q.shape[0] < M:
+            self._q = torch.empty((M, self.K), dtype=torch.int8, device=x.device)
+            self._s = torch.empty((M,), dtype=torch.float32, device=x.device)
+        q, s = self._q[:M], self._s[:M]
+        dq_quantize_rows(x, q, s, stream=stream)
+        if M not in self._ws:
+            n = dq_s24_workspace_size(M, self.N, self.K)
+            self._ws[M] = torch.zeros((n,), dtype=torch.uint8, device=x.device) if n else None
+        return dq_s24_int8_linear(q, s, self.values, self.meta, self.s_col, self.bias, out=out,
+                                  workspace=self._ws[M], stream=stream)

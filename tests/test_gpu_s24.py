@@ -109,3 +109,17 @@ def test_rejections_launch_nothing():
     assert lib.dq_s24_int8_linear(P(A), None, 4, 256, P(v), P(m), None, 60, None, P(out), 1, None, 0, s) == dq.DQ_ERR_UNSUPPORTED
     assert lib.dq_s24_int8_linear(P(A), None, 4, 256, P(v), P(m), None, 64, None, P(out), 7, None, 0, s) == dq.DQ_ERR_INVALID_ARG
     assert lib.dq_s24_compress(P(A), 4, 12, P(v), P(m), None, s) == dq.DQ_ERR_INVALID_ARG
+
+
+def test_layer_class_matches_oracle():
+    """S24Int8Linear: weight quantized and compressed once, tokens quantized per call."""
+    N, K = 256, 1024
+    d = synth.s24(1, M=48, K=K, N=N)
+    bias = synth.normal_bf16((N,), 0.1, 12)
+    layer = dq.S24Int8Linear.from_float(to_dev(d["w"]), bias=to_dev_bf16(bias))
+    wo, sco = oracle.quantize_rows_f32(d["w"])
+    for M in (48, 16):                      # 16 tokens split the contraction
+        x = d["x"][:M]
+        out = layer(to_dev_bf16(x))
+        qo, so = oracle.quantize_rows_bf16(x)
+        assert_bf16_close(bf16_bits(out), oracle.linear_bf16(qo, so, wo, sco, bias))
