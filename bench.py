@@ -64,15 +64,23 @@ KERNEL_SOURCES = {
 }
 
 
+def _strip_comments(text: str) -> str:
+    """C/C++ source without its comments (string literals in these sources
+    hold no comment markers), so that a comment edit keeps the hash."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.sub(r"//[^\n]*", "", text)
+
+
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the CUDA sources `kernel` is built from: a stored ncu traffic
-    figure only applies to the kernel it was measured on."""
+    """Hash of the CUDA sources `kernel` is built from, comments removed: a
+    stored ncu traffic figure only applies to the code it was measured on."""
     import hashlib
     d = os.path.join(ROOT, "quantized_gemm_token_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(KERNEL_SOURCES[kernel]):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode() + b"\0" + fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + _strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

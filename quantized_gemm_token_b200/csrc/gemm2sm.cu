@@ -23,7 +23,7 @@
 //               TMEM, the same fp32 dequantization and TMA-store path as the
 //               1-SM kernel; each warp then tells the leader (remote arrive)
 //               that its part of the accumulator is free.
-// No load is multicast: each CTA fetches its own operand halves.
+// Every load is a plain per-CTA load: each CTA fetches its own operand halves.
 #include <mutex>
 
 #include "gemm_common.cuh"
