@@ -647,7 +647,7 @@ def run_gpu(args, rank, world, local_rank):
     dtype = "e4m3" if wl["kind"] == "dense_fp8" else "int8"
     metric = METRIC
     if hqq:
-        unit, metric, dtype = "TFLOP/s", METRIC_HQQ, "bf16 (int4 weight)"
+        unit, metric, dtype = "TFLOP/s", METRIC_HQQ, "bf16"
         page_ms = HQQ_PAGE_H100_MS.get(wl["M"]) if not wl.get("transposed") else None
         if page_ms:
             vs_baseline = round(value / (ops / (page_ms * 1e-3) / 1e12), 2)
@@ -665,8 +665,13 @@ def run_gpu(args, rank, world, local_rank):
                                    "read, pipelined on three streams (copy-in / kernels / copy-out)",
                             kernels_ms=kernels_ms),
                 roofline=roof, e2e=e2e, gpu_launches=nk * K, clocks=cs.summary())
+    if hqq:
+        line["config"]["weight"] = (f"int4 {'s4' if wl.get('signed') else 'u4'} codes, group {wl['group']}, "
+                                    "bf16 scales and zero points; dequantized in the GEMM")
+    if wl["kind"] == "s24":
+        line["config"]["weight"] = "2:4 sparse int8, compressed (two values + a position nibble per group of four)"
     if rank == 0 and world == 1 and not args.no_cpu_baseline and wl["kind"] in ("dense", "bsr", "quant", "gemm",
-                                                                                 "hqq"):
+                                                                                 "hqq", "s24"):
         line["cpu_baseline"] = cpu_baseline(name, wl, state["d"], budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -748,7 +753,7 @@ def _oracle_sample(name, wl, d, rows):
     import numpy as np
     import oracle
     k = wl["kind"]
-    if k in ("dense",):
+    if k in ("dense", "s24"):       # the 2:4 layer is the dense layer on the 2:4 weight
         if "_wq" not in d:
             d["_wq"], d["_sc"] = oracle.quantize_rows_f32(d["w"])
         x = d["x"][rows]

@@ -539,6 +539,8 @@ class HqqLinear:
     def _workspace(self, M, transposed, device):
         key = (M, transposed)
         if key not in self._ws:
+            if len(self._ws) >= 16:                 # keep the most recent shapes only
+                self._ws.pop(next(iter(self._ws)))
             n = dq_hqq_workspace_size(M, self.N, self.K, transposed)
             self._ws[key] = torch.zeros((n,), dtype=torch.uint8, device=device) if n else None
         return self._ws[key]
@@ -694,6 +696,8 @@ class S24Int8Linear:
         q, s = self._q[:M], self._s[:M]
         dq_quantize_rows(x, q, s, stream=stream)
         if M not in self._ws:
+            if len(self._ws) >= 16:                 # keep the most recent shapes only
+                self._ws.pop(next(iter(self._ws)))
             n = dq_s24_workspace_size(M, self.N, self.K)
             self._ws[M] = torch.zeros((n,), dtype=torch.uint8, device=x.device) if n else None
         return dq_s24_int8_linear(q, s, self.values, self.meta, self.s_col, self.bias, out=out,
