@@ -100,9 +100,13 @@ DQ_API dq_status dq_selftest_wait_timeout(dq_stream_t stream);
  *
  * For each row i:  a = max_k |x[i,k]|,  s[i] = fp32( max(a, 1e-8f) / 127 ),
  *                  q[i,k] = clamp( rint_half_even( fp32(x[i,k] / s[i]) ), -127, 127 ).
- * Every fp32 operation is one IEEE operation rounded to nearest even (true
- * division, no reciprocal), so results are bit-identical to a scalar IEEE
- * evaluation.  Non-finite inputs give unspecified (but in-bounds) results.
+ * Guarantee: the scales are bit-equal to the IEEE fp32 quotient
+ * max(a, 1e-8f) / 127, and every code is bit-equal to rint (half to even) of
+ * the IEEE fp32 quotient x / s, clamped, i.e. to a scalar IEEE evaluation of
+ * the formula with a true division.  (The kernels do not divide: for bf16
+ * rows they form the correctly rounded quotient from a reciprocal by one
+ * Markstein correction step, for fp32 rows they divide only near a tie.)
+ * Non-finite inputs give unspecified (but in-bounds) results.
  *
  * x: bf16 [M, K] (as 16-bit patterns), row stride ldx >= K.
  * q: int8 [M, K], row stride ldq >= K.   scales: fp32 [M].
@@ -172,14 +176,20 @@ DQ_API size_t dq_int8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
  *  - If the chosen schedule needs more scratch than DQ_NOALLOC_SCRATCH_BYTES
  *    (dq_int8_linear_workspace_size(M, N, K) > DQ_NOALLOC_SCRATCH_BYTES), the
  *    call launches nothing and returns DQ_ERR_UNSUPPORTED.
- *  - The first call on a device looks up the array's device address for that
- *    device (cudaGetSymbolAddress, with that device current); make that first
- *    call before any stream capture.
- *  - Each call clears the part of the array it uses (cudaMemsetAsync on
- *    `stream`) before the GEMM, because the array keeps the previous call's
- *    contents.  All calls on a device share the one array: two calls whose
- *    work overlaps on the GPU (different streams, no ordering between them)
- *    race on it and may produce wrong results.  Serialise them.
+ *  - The first call on a device that needs the scratch looks up the array's
+ *    device address for that device (cudaGetSymbolAddress, with that device
+ *    current), zeroes the whole array on `stream` and waits for that (it
+ *    synchronises `stream` once).  Make that first call before any stream
+ *    capture.
+ *  - The split-K kernel leaves every part of the array it used at zero when
+ *    it completes, so later calls do not clear it.  After a bounded wait ran
+ *    out (dq_sync_status returned DQ_ERR_TIMEOUT) partial sums may be left
+ *    behind; the next call then zeroes the array again, on its `stream`,
+ *    before its kernel.  All calls on a device share the one array: two
+ *    calls whose work overlaps on the GPU (different streams, no ordering
+ *    between them) race on it and may produce wrong results.  Serialise them.
+ *  - The scratch size is dq_int8_linear_workspace_size(M, N, K) under the
+ *    current measurement knobs (the same plan dq_int8_linear uses).
  *  - Everything else (requirements, results, errors) is as dq_int8_linear.
  * ------------------------------------------------------------------------ */
 #define DQ_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
@@ -385,6 +395,32 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
                                     const uint8_t* meta, const float* s_col, int64_t N, const void* bias_bf16,
                                     void* out, dq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
                                     dq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Measurement knobs.  Process-wide settings read by every later launch from
+ * any host thread (relaxed atomics); they change which schedule or kernel a
+ * call uses, never its result.  For benchmarks and tests of the alternative
+ * schedules; the defaults (all 0 except where stated) are what the library
+ * chooses by itself.  Not for concurrent use with different settings.
+ *
+ * dq_debug_set_schedule (dense int8 linear): 0 automatic; 1 the 1-SM kernel
+ *   with whole tiles; 2 the 1-SM kernel with stream-K whenever a workspace
+ *   is given; 3 the 2-SM pair kernel for every M; 4 the dense (tokens on
+ *   MMA M) arrangement also for M <= 128; 5 as 4 with stream-K.
+ * dq_debug_set_tile_n: force the dense tile width (128, 160, 192, 224, 256;
+ *   pair kernel 160, 192, 256); 0 automatic.
+ * dq_debug_set_two_widths: 1 (default) wave-balanced schedule of two tile
+ *   widths where whole tiles leave a partial last wave; 0 uniform tiles.
+ * dq_debug_set_bsr_panel: BSR activation-panel variant (K <= 1280):
+ *   0 never, 1 (default) for blocks smaller than 64, 2 always.
+ * dq_debug_set_quant_kernel: 0 automatic, 1 register-resident kernel,
+ *   2 row-pipelined (shared-memory ring) kernel for int8 codes.
+ * ------------------------------------------------------------------------ */
+DQ_API void dq_debug_set_schedule(int mode);
+DQ_API void dq_debug_set_tile_n(int n);
+DQ_API void dq_debug_set_two_widths(int on);
+DQ_API void dq_debug_set_bsr_panel(int mode);
+DQ_API void dq_debug_set_quant_kernel(int mode);
 
 /* ------------------------------------------------------------------------
  * Measurement helper: a kernel that only issues tcgen05.mma.kind::i8

@@ -124,6 +124,31 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
+def _stream_obj(stream) -> torch.cuda.Stream:
+    """The torch stream a layer call runs on (current stream when None; a raw
+    cudaStream_t handle is wrapped)."""
+    if stream is None:
+        return torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return stream
+    return torch.cuda.ExternalStream(int(stream))
+
+
+def _scratch(shape, dtype, device, stream: torch.cuda.Stream, zero: bool = False) -> torch.Tensor:
+    """Scratch a layer keeps between calls, allocated (and zero-filled) on the
+    stream its kernels run on, so that the fill is ordered before them."""
+    with torch.cuda.stream(stream):
+        return (torch.zeros if zero else torch.empty)(shape, dtype=dtype, device=device)
+
+
+def _used_on(stream: torch.cuda.Stream, *ts):
+    """Tell the caching allocator that `stream` uses the cached scratch, so a
+    later free or eviction waits for that stream's work."""
+    for t in ts:
+        if t is not None:
+            t.record_stream(stream)
+
+
 def _need(t: torch.Tensor, dtype, name: str, ndim: int = None):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name}: expected a CUDA tensor")
@@ -303,11 +328,8 @@ def dq_int8_linear_workspace_size(M: int, N: int, K: int) -> int:
     return int(lib.dq_int8_linear_workspace_size(M, N, K))
 
 
-def dq_int8_linear(A, s_row, W, s_col, bias=None, out=None, out_dtype="bf16", workspace=None, stream=None):
-    """out[M, N] = bf16(acc * s_row * s_col + bias), acc = A @ W^T exactly
-    (or acc itself as int32 with out_dtype="s32").  `workspace` is an
-    optional zero-filled uint8 CUDA tensor (see dq_int8_linear_workspace_size)."""
-    code = _out_code(out_dtype)
+def _linear_args(A, s_row, W, s_col, bias, out, code, out_required: bool):
+    """The checks of the dense int8 linear's arguments; returns (M, K, N, out)."""
     _need(A, torch.int8, "A", 2)
     _need(W, torch.int8, "W", 2)
     _contig(A, "A")
@@ -319,17 +341,33 @@ def dq_int8_linear(A, s_row, W, s_col, bias=None, out=None, out_dtype="bf16", wo
     if code == DQ_OUT_BF16:
         _need(s_row, torch.float32, "s_row", 1)
         _need(s_col, torch.float32, "s_col", 1)
+        _contig(s_row, "s_row")
+        _contig(s_col, "s_col")
         if s_row.numel() != M or s_col.numel() != N:
             raise ValueError("scale length mismatch")
     if bias is not None:
         _need(bias, torch.bfloat16, "bias", 1)
+        _contig(bias, "bias")
         if bias.numel() != N:
             raise ValueError("bias length mismatch")
     odt = torch.bfloat16 if code == DQ_OUT_BF16 else torch.int32
     if out is None:
+        if out_required:
+            raise ValueError("out: a preallocated output tensor is required")
         out = torch.empty((M, N), dtype=odt, device=A.device)
     _need(out, odt, "out", 2)
     _contig(out, "out")
+    if tuple(out.shape) != (M, N):
+        raise ValueError(f"out: expected shape {(M, N)}, got {tuple(out.shape)}")
+    return M, K, N, out
+
+
+def dq_int8_linear(A, s_row, W, s_col, bias=None, out=None, out_dtype="bf16", workspace=None, stream=None):
+    """out[M, N] = bf16(acc * s_row * s_col + bias), acc = A @ W^T exactly
+    (or acc itself as int32 with out_dtype="s32").  `workspace` is an
+    optional zero-filled uint8 CUDA tensor (see dq_int8_linear_workspace_size)."""
+    code = _out_code(out_dtype)
+    M, K, N, out = _linear_args(A, s_row, W, s_col, bias, out, code, out_required=False)
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         _need(workspace, torch.uint8, "workspace")
@@ -343,13 +381,14 @@ DQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def dq_int8_linear_noalloc(A, s_row, W, s_col, out, bias=None, out_dtype="bf16", stream=None):
-    """dq_int8_linear for callers that cannot allocate: the split-K scratch
-    comes from libdq's static 32 MiB device array (see include/dq.h), and the
-    caller passes a preallocated `out`.  Calls that overlap on the GPU race on
-    that array; the first call on a device must precede any stream capture."""
+    """dq_int8_linear for callers that cannot allocate device memory: the
+    split-K scratch comes from libdq's static 32 MiB device array and the
+    caller passes a preallocated `out` ([M, N], bf16 or int32 to match
+    out_dtype); the arguments are checked as for dq_int8_linear.  Calls that
+    overlap on the GPU race on that array; the first call on a device that
+    uses it must come before any stream capture."""
     code = _out_code(out_dtype)
-    M, K = A.shape
-    N = W.shape[0]
+    M, K, N, out = _linear_args(A, s_row, W, s_col, bias, out, code, out_required=True)
     _check(lib.dq_int8_linear_noalloc(_ptr(A), _ptr(s_row), M, K, _ptr(W), _ptr(s_col), N, _ptr(bias),
                                       _ptr(out), code, _stream(stream)), "dq_int8_linear_noalloc")
     return out
@@ -536,24 +575,30 @@ class HqqLinear:
         """codes int8 [N, K]; scale, zero bf16 per channel [N, K/group]."""
         return cls(dq_hqq_pack(codes), dq_hqq_group_major(scale), dq_hqq_group_major(zero), group, signed)
 
-    def _workspace(self, M, transposed, device):
+    def _workspace(self, M, transposed, device, st):
         key = (M, transposed)
         if key not in self._ws:
             if len(self._ws) >= 16:                 # keep the most recent shapes only
                 self._ws.pop(next(iter(self._ws)))
             n = dq_hqq_workspace_size(M, self.N, self.K, transposed)
-            self._ws[key] = torch.zeros((n,), dtype=torch.uint8, device=device) if n else None
+            self._ws[key] = _scratch((n,), torch.uint8, device, st, zero=True) if n else None
         return self._ws[key]
 
     def __call__(self, x: torch.Tensor, out: torch.Tensor = None, stream=None):
-        ws = self._workspace(x.shape[0], False, x.device)
-        return dq_hqq_linear(x, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
-                             workspace=ws, stream=stream)
+        st = _stream_obj(stream)
+        ws = self._workspace(x.shape[0], False, x.device, st)
+        y = dq_hqq_linear(x, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
+                          workspace=ws, stream=st)
+        _used_on(st, ws)
+        return y
 
     def backward_input(self, grad_out: torch.Tensor, out: torch.Tensor = None, stream=None):
-        ws = self._workspace(grad_out.shape[0], True, grad_out.device)
-        return dq_hqq_linear_t(grad_out, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
-                               workspace=ws, stream=stream)
+        st = _stream_obj(stream)
+        ws = self._workspace(grad_out.shape[0], True, grad_out.device, st)
+        y = dq_hqq_linear_t(grad_out, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
+                            workspace=ws, stream=st)
+        _used_on(st, ws)
+        return y
 
 
 # ---------------------------------------------------------------- 2:4 sparse
@@ -643,27 +688,32 @@ class Int8DynamicLinear:
         values = dq_bsr_pack(wq, crow, col)
         return cls(None, s_col, bias, dict(crow=crow, col=col, values=values, K=w_masked.shape[1]))
 
-    def _buffers(self, M, device):
+    def _buffers(self, M, device, st):
         if self._q is None or self._q.shape[0] < M:
-            self._q = torch.empty((M, self.K), dtype=torch.int8, device=device)
-            self._s = torch.empty((M,), dtype=torch.float32, device=device)
-            if self.bsr is None:
-                n = dq_int8_linear_workspace_size(M, self.N, self.K)
-                self._ws = torch.zeros((n,), dtype=torch.uint8, device=device) if n else None
+            self._q = _scratch((M, self.K), torch.int8, device, st)
+            self._s = _scratch((M,), torch.float32, device, st)
+        if self.bsr is None:
+            n = dq_int8_linear_workspace_size(M, self.N, self.K)
+            if n and (self._ws is None or self._ws.numel() < n):
+                self._ws = _scratch((n,), torch.uint8, device, st, zero=True)
         return self._q[:M], self._s[:M]
 
     def __call__(self, x: torch.Tensor, out: torch.Tensor = None, stream=None):
         M = x.shape[0]
-        q, s = self._buffers(M, x.device)
-        dq_quantize_rows(x, q, s, stream=stream)
+        st = _stream_obj(stream)
+        q, s = self._buffers(M, x.device, st)
+        dq_quantize_rows(x, q, s, stream=st)
         if self.bsr is None:
             ws = self._ws
             if ws is not None and ws.numel() < dq_int8_linear_workspace_size(M, self.N, self.K):
                 ws = None
-            return dq_int8_linear(q, s, self.wq, self.s_col, self.bias, out=out, workspace=ws, stream=stream)
-        b = self.bsr
-        return dq_bsr_int8_linear(q, s, self.N, b["crow"], b["col"], b["values"], self.s_col, self.bias,
-                                  out=out, stream=stream)
+            y = dq_int8_linear(q, s, self.wq, self.s_col, self.bias, out=out, workspace=ws, stream=st)
+        else:
+            b = self.bsr
+            y = dq_bsr_int8_linear(q, s, self.N, b["crow"], b["col"], b["values"], self.s_col, self.bias,
+                                   out=out, stream=st)
+        _used_on(st, self._q, self._s, self._ws)
+        return y
 
 
 class S24Int8Linear:
@@ -690,15 +740,18 @@ class S24Int8Linear:
 
     def __call__(self, x: torch.Tensor, out: torch.Tensor = None, stream=None):
         M = x.shape[0]
+        st = _stream_obj(stream)
         if self._q is None or self._q.shape[0] < M:
-            self._q = torch.empty((M, self.K), dtype=torch.int8, device=x.device)
-            self._s = torch.empty((M,), dtype=torch.float32, device=x.device)
+            self._q = _scratch((M, self.K), torch.int8, x.device, st)
+            self._s = _scratch((M,), torch.float32, x.device, st)
         q, s = self._q[:M], self._s[:M]
-        dq_quantize_rows(x, q, s, stream=stream)
+        dq_quantize_rows(x, q, s, stream=st)
         if M not in self._ws:
             if len(self._ws) >= 16:                 # keep the most recent shapes only
                 self._ws.pop(next(iter(self._ws)))
             n = dq_s24_workspace_size(M, self.N, self.K)
-            self._ws[M] = torch.zeros((n,), dtype=torch.uint8, device=x.device) if n else None
-        return dq_s24_int8_linear(q, s, self.values, self.meta, self.s_col, self.bias, out=out,
-                                  workspace=self._ws[M], stream=stream)
+            self._ws[M] = _scratch((n,), torch.uint8, x.device, st, zero=True) if n else None
+        y = dq_s24_int8_linear(q, s, self.values, self.meta, self.s_col, self.bias, out=out,
+                               workspace=self._ws[M], stream=st)
+        _used_on(st, self._q, self._s, self._ws[M])
+        return y

@@ -44,6 +44,7 @@
 // int32 workspace through red.add, and the last arriving CTA (an arrival
 // counter) runs the epilogue and zeroes the workspace again.  Integer adds
 // are exact and associative, so every schedule gives identical bits.
+#include <atomic>
 #include <mutex>
 
 #include "gemm_common.cuh"
@@ -97,28 +98,50 @@ struct Cfg {
   // outside the matrix does in the streaming variant).
   static constexpr int ZB_BYTES = PANEL ? (B_BYTES > 256 ? B_BYTES : 256) : 0;
   static constexpr int STAGE_CAP = BSR && (BS < 64 || PANEL) ? 24 : 12;
-  static constexpr int STAGES_RAW =
-      (224 * 1024 - OUT_BYTES - IDX_BYTES - 2 * ZERO_BYTES - PANEL_BYTES - ZB_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > STAGE_CAP ? STAGE_CAP : STAGES_RAW;
-  // shared-memory layout (offsets from the 1024-aligned base)
+  static constexpr int ACC_RAW = 512 / BN;
+  static constexpr int ACC_BUFS = ACC_RAW > 8 ? 8 : ACC_RAW;
+  // mbarriers, the TMEM address, flags and (panel variant) stage columns
+  static constexpr int BAR_BYTES = BSR ? 1024 : 512;
+  // Shared-memory layout for a given stage count and number of column-scale
+  // slots (offsets from the 1024-aligned base; the last 1024 bytes are the
+  // slack of aligning the dynamic shared-memory base).
+  static constexpr int off_b(int st) { return ZERO_BYTES + PANEL_BYTES + st * A_BYTES; }
+  static constexpr int off_out(int st) {
+    return ((((off_b(st) + st * B_BYTES + ZERO_BYTES + 1023) / 1024 * 1024) + ZB_BYTES + 1023) / 1024) * 1024;
+  }
+  static constexpr int layout_bytes(int st, int slots) {
+    return off_out(st) + OUT_BYTES + slots * kScSlotBytes + IDX_BYTES + BAR_BYTES + 1024;
+  }
+  static constexpr int pick_stages(int slots) {
+    int st = STAGE_CAP;
+    while (st > 2 && layout_bytes(st, slots) > 227 * 1024) --st;
+    return st;
+  }
+  // Row-layout epilogues stage each tile's column scales and bias in shared
+  // memory: two slots (the next tile's copy in flight while this tile is
+  // stored) where that costs no operand stage, else one.
+  static constexpr int SC_SLOTS = !STAGED_OUT ? 0 : pick_stages(2) == pick_stages(0) ? 2 : 1;
+  static constexpr int STAGES = pick_stages(SC_SLOTS);
   static constexpr int OFF_ZLO = 0;
   static constexpr int OFF_PANEL = ZERO_BYTES;
   static constexpr int OFF_A = OFF_PANEL + PANEL_BYTES;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_B = off_b(STAGES);
   static constexpr int OFF_ZHI = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_ZB = (OFF_ZHI + ZERO_BYTES + 1023) / 1024 * 1024;
-  static constexpr int OFF_OUT = (OFF_ZB + ZB_BYTES + 1023) / 1024 * 1024;
-  static constexpr int OFF_IDX = OFF_OUT + OUT_BYTES;
+  static constexpr int OFF_OUT = off_out(STAGES);
+  static constexpr int OFF_SC = OFF_OUT + OUT_BYTES;
+  static constexpr int OFF_IDX = OFF_SC + SC_SLOTS * kScSlotBytes;
   static constexpr int OFF_BARS = OFF_IDX + IDX_BYTES;
-  static constexpr int ACC_RAW = 512 / BN;
-  static constexpr int ACC_BUFS = ACC_RAW > 8 ? 8 : ACC_RAW;
   static constexpr int ACC_COLS = ACC_BUFS * BN;
   static constexpr int TMEM_COLS = ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128
                                    : ACC_COLS <= 256 ? 256 : 512;
   static constexpr int K_STEPS = KB / 32;                     // MMA K = 32 bytes
   static constexpr int CW = BN >= 32 ? 32 : 16;               // epilogue chunk (columns)
-  static constexpr int SMEM_BYTES = OFF_BARS + 1024 /*barriers, stage columns*/ + 1024 /*align*/;
+  static constexpr int SMEM_BYTES = layout_bytes(STAGES, SC_SLOTS);
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int NBARS = 2 * STAGES + 2 * ACC_BUFS + 3 + 2 * SC_SLOTS;
+  static_assert(NBARS * 8 + 16 + (PANEL ? 4 * STAGES : 0) <= BAR_BYTES, "barrier area");
+  static_assert(OFF_ZB + ZB_BYTES <= OFF_OUT, "layout");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(STAGES >= 2, "stages");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -126,45 +149,15 @@ struct Cfg {
   static_assert(!PANEL || BSR, "the panel variant is for BSR weights");
 };
 
-// Where a tile lies: 128-row block ta, B-slot tile tb, first output column n0
-// and the MMA width (BN, or bn2 for a Dense tile of the narrow second set).
-struct TileGeom {
-  int ta, tb, n0, width;
-  bool narrow;
-};
-template <Kind KIND, int BN>
-__device__ __forceinline__ TileGeom tile_geom(const GemmArgs& g, int tile) {
-  TileGeom t;
-  if (is_dense_kind(KIND) && g.bn2 > 0 && tile >= g.t1) {
-    int j = tile - g.t1;
-    if (j < g.first_cnt) {
-      t.ta = g.mb0;
-      t.n0 = g.c_start + j * g.bn2;
-    } else {
-      j -= g.first_cnt;
-      t.ta = g.mb0 + 1 + j / g.per_row;
-      t.n0 = (j % g.per_row) * g.bn2;
-    }
-    t.tb = 0;
-    t.width = g.bn2;
-    t.narrow = true;
-  } else {
-    t.ta = tile / g.b_tiles;
-    t.tb = tile % g.b_tiles;
-    t.n0 = t.tb * BN;
-    t.width = BN;
-    t.narrow = false;
-  }
-  return t;
-}
-
 // The stream-K finishing store, kept out of line so that this rarely taken
 // path does not add to the register pressure of the whole-tile epilogue.
 __device__ __noinline__ void store_row_chunk_tma_cold(const GemmArgs& g, const CUtensorMap* tm_c, uint8_t* buf,
                                                       int lane, int m0, int n0, const uint32_t* r, float srow) {
   ColScales cs;
+  uint4 bias[4];
   if (!g.out_s32) load_col_scales(g, n0, cs);
-  store_row_chunk_tma(g, tm_c, buf, lane, m0, n0, r, srow, cs);
+  if (!g.out_s32 && g.bias != nullptr) load_bias_global(g, n0, bias);
+  store_row_chunk_tma(g, tm_c, buf, lane, m0, n0, r, srow, cs, bias);
 }
 
 template <Kind KIND, int BN, bool PANEL>
@@ -188,7 +181,9 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
   uint64_t* drain_bar = acce_bar + C::ACC_BUFS;
   uint64_t* panel_full = drain_bar + 1;       // panel variant: activation panel landed
   uint64_t* panel_empty = panel_full + 1;     // panel variant: MMAs on the old panel done
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(panel_empty + 1);
+  uint64_t* sc_full = panel_empty + 1;        // row epilogues: a tile's scales landed in slot i
+  uint64_t* sc_free = sc_full + C::SC_SLOTS;   // every epilogue warp is done reading slot i
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sc_free + C::SC_SLOTS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* sk_last = const_cast<int*>(abort_flag + 1);
   // panel variant: each stage's block column, written by the producer before
@@ -211,6 +206,10 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
     mbar_init(smem_u32(drain_bar), 1);
     mbar_init(smem_u32(panel_full), 1);
     mbar_init(smem_u32(panel_empty), 1);
+    for (int i = 0; i < C::SC_SLOTS; ++i) {
+      mbar_init(smem_u32(sc_full + i), 1);
+      mbar_init(smem_u32(sc_free + i), C::EPI_WARPS);
+    }
     fence_barrier_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
@@ -264,7 +263,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
       int panel_loads = 0;
       const int panel_chunks = (g.K + 127) / 128;
       while (ok && iter.next(s)) {
-        const TileGeom geo = tile_geom<KIND, BN>(g, s.tile);
+        const TileGeom geo = tile_geom(g, s.tile, BN, is_dense_kind(KIND));
         const int ta = geo.ta, tb = geo.tb;
         const uint32_t stage_tx = C::A_BYTES + (is_dense_kind(KIND) ? geo.width * C::KB : C::B_BYTES);
         if constexpr (PANEL) {
@@ -474,13 +473,53 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
       return b;
     };
     SegIter iter(g);
+    int k = 0;               // segments started
+    const uint32_t sc_base = smem_u32(smem + C::OFF_SC);
     Seg s;
     int acc = 0;
     uint32_t acc_phase = 0;
-    while (iter.next(s)) {
-      const TileGeom geo = tile_geom<KIND, BN>(g, s.tile);
+    bool ok = true;
+    while (ok && iter.next(s)) {
+      const TileGeom geo = tile_geom(g, s.tile, BN, is_dense_kind(KIND));
       const int ta = geo.ta, tb = geo.tb, n0 = geo.n0;
+      const int slot = C::SC_SLOTS > 0 ? k % C::SC_SLOTS : 0;
+      const uint32_t sc_slot = sc_base + static_cast<uint32_t>(slot * kScSlotBytes);
+      if constexpr (C::SC_SLOTS > 0) {
+        // One thread copies each segment's scales into its slot once every
+        // epilogue warp is done with the slot's previous contents: with one
+        // slot at the start of the segment, with two one segment ahead (the
+        // copy lands while the MMAs, or the previous segment's stores, run).
+        if (ep_tid == 0) {
+          if (C::SC_SLOTS == 1 || k == 0) {
+            if (k > 0 && !mbar_wait(smem_u32(sc_free), static_cast<uint32_t>(k - 1) & 1u, g.wait, abort_flag))
+              break;
+            stage_tile_scales(g, sc_slot, n0, geo.width, smem_u32(sc_full + slot));
+          }
+          if constexpr (C::SC_SLOTS == 2) {
+            SegIter peek = iter;
+            Seg ns;
+            if (peek.next(ns)) {
+              const int k1 = k + 1, sl = k1 & 1;
+              if (k1 >= 2 &&
+                  !mbar_wait(smem_u32(sc_free + sl), static_cast<uint32_t>(k1 / 2 - 1) & 1u, g.wait, abort_flag))
+                break;
+              const TileGeom ng = tile_geom(g, ns.tile, BN, is_dense_kind(KIND));
+              stage_tile_scales(g, sc_base + static_cast<uint32_t>(sl * kScSlotBytes), ng.n0, ng.width,
+                                smem_u32(sc_full + sl));
+            }
+          }
+        }
+      }
+      float srow = 0.0f;
+      if constexpr (KIND != Kind::Swap) {
+        const int m = ta * 128 + row;
+        if (!g.out_s32 && m < g.M) srow = __ldg(g.s_row + m);
+      }
       if (!mbar_wait(smem_u32(accf_bar + acc), acc_phase, g.wait, abort_flag)) break;
+      if constexpr (C::SC_SLOTS > 0) {
+        if (!mbar_wait(smem_u32(sc_full + slot), static_cast<uint32_t>(k / C::SC_SLOTS) & 1u, g.wait, abort_flag))
+          break;
+      }
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const bool whole = !g.stream_k || (s.kb0 == 0 && s.kb1 == g.kb_total);
@@ -491,58 +530,69 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
       const int last_c = grp + ((nch - 1 - grp) / GROUPS) * GROUPS;
 
       if (whole) {
-        float srow = 0.0f;
-        if constexpr (KIND != Kind::Swap) {
-          const int m = ta * 128 + row;
-          if (!g.out_s32 && m < g.M) srow = __ldg(g.s_row + m);
-        }
-        // Chunk by chunk: the TMEM load and the chunk's column-scale loads are
-        // in flight together; after reading its last chunk the warp hands
-        // the accumulator back to the MMA warp, then dequantizes and stores.
+        // BATCH chunks per TMEM wait (row layouts: two); after the batch
+        // holding its last chunk the warp hands the accumulator back to the
+        // MMA warp, then dequantizes and stores from registers with the
+        // column scales and bias from the tile's staged slot.
+        constexpr int BATCH = C::STAGED_OUT ? 2 : 1;
 #pragma unroll 1
-        for (int c = grp; c < nch; c += GROUPS) {
-          uint32_t r[CW];
-          // BSR: block rows of this chunk without blocks (their TMEM slice
-          // was never written) read as zeros; a 32-column chunk holds one
-          // block row's columns, or two 16-wide block rows
-          bool empty_lo = false, empty_hi = false;
-          if constexpr (C::BSR) {
-            auto row_empty = [&](int br) {
-              int p0 = 0, p1 = 0;
-              if (br < g.nbr) bsr_range(g, idx, br, p0, p1);
-              return br >= g.nbr || p0 == p1;
-            };
-            const int br = tb * C::NSUB + (c * CW) / C::BS;
-            empty_lo = row_empty(br);
-            empty_hi = C::BS >= CW ? empty_lo : row_empty(br + 1);
-          }
-          const bool empty_slice = empty_lo && empty_hi;
-          if (empty_slice) {
+        for (int c0 = grp; c0 < nch; c0 += BATCH * GROUPS) {
+          uint32_t r[BATCH][CW];
+          const bool two = BATCH > 1 && c0 + GROUPS < nch;
+          // BSR: block rows of a chunk without blocks (their TMEM slice was
+          // never written) read as zeros; a 32-column chunk holds one block
+          // row's columns, or two 16-wide block rows
+          bool empty_lo[BATCH], empty_hi[BATCH];
 #pragma unroll
-            for (int j = 0; j < CW; ++j) r[j] = 0;
-          } else if constexpr (CW == 32) {
-            tmem_ld_32x32b_x32(tbase + c * CW, r);
-          } else {
-            tmem_ld_32x32b_x16(tbase + c * CW, r);
-          }
-          ColScales cs;
-          if constexpr (KIND != Kind::Swap) {
-            if (!g.out_s32) load_col_scales(g, n0 + c * CW, cs);
+          for (int i = 0; i < BATCH; ++i) {
+            empty_lo[i] = empty_hi[i] = false;
+            if (i == 1 && !two) break;
+            const int c = c0 + i * GROUPS;
+            if constexpr (C::BSR) {
+              auto row_empty = [&](int br) {
+                int p0 = 0, p1 = 0;
+                if (br < g.nbr) bsr_range(g, idx, br, p0, p1);
+                return br >= g.nbr || p0 == p1;
+              };
+              const int br = tb * C::NSUB + (c * CW) / C::BS;
+              empty_lo[i] = row_empty(br);
+              empty_hi[i] = C::BS >= CW ? empty_lo[i] : row_empty(br + 1);
+            }
+            if (empty_lo[i] && empty_hi[i]) {
+#pragma unroll
+              for (int j = 0; j < CW; ++j) r[i][j] = 0;
+            } else if constexpr (CW == 32) {
+              tmem_ld_32x32b_x32(tbase + c * CW, r[i]);
+            } else {
+              tmem_ld_32x32b_x16(tbase + c * CW, r[i]);
+            }
           }
           tmem_ld_wait();
           if constexpr (KIND == Kind::Bsr16) {
-            if (!empty_slice && (empty_lo || empty_hi)) {
 #pragma unroll
-              for (int j = 0; j < CW; ++j)
-                if (j < 16 ? empty_lo : empty_hi) r[j] = 0;
+            for (int i = 0; i < BATCH; ++i) {
+              if (!(empty_lo[i] && empty_hi[i]) && (empty_lo[i] || empty_hi[i])) {
+#pragma unroll
+                for (int j = 0; j < CW; ++j)
+                  if (j < 16 ? empty_lo[i] : empty_hi[i]) r[i][j] = 0;
+              }
             }
           }
-          if (c == last_c) {
+          if (c0 == last_c || (two && c0 + GROUPS == last_c)) {
             tc_fence_before();
             mbar_arrive(smem_u32(acce_bar + acc));
           }
-          if constexpr (KIND == Kind::Swap) store_col_chunk<CW>(g, ta * 128 + row, n0 + c * CW, r);
-          else store_row_chunk_tma<KIND == Kind::DenseF8>(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32, n0 + c * CW, r, srow, cs);
+#pragma unroll
+          for (int i = 0; i < BATCH; ++i) {
+            if (i == 1 && !two) break;
+            const int c = c0 + i * GROUPS;
+            if constexpr (KIND == Kind::Swap) {
+              store_col_chunk<CW>(g, ta * 128 + row, n0 + c * CW, r[i]);
+            } else {
+              store_row_chunk_staged<KIND == Kind::DenseF8>(g, &tm_c, next_buf(), lane, ta * 128 + sp * 32,
+                                                            n0 + c * CW, r[i], srow, sc_slot, c * CW);
+            }
+          }
         }
       } else {
         // Stream-K partial tile: add into the workspace (coalesced: one
@@ -571,11 +621,6 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
         named_bar_sync(1, EPI_THREADS);
         if (*sk_last) {
           __threadfence();
-          float srow = 0.0f;
-          if constexpr (KIND != Kind::Swap) {
-            const int m = ta * 128 + row;
-            if (!g.out_s32 && m < g.M) srow = __ldg(g.s_row + m);
-          }
 #pragma unroll 1
           for (int c = grp; c < NCH; c += GROUPS) {
             uint32_t r[CW];
@@ -591,7 +636,12 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
           if (ep_tid == 0) g.ws_cnt[s.tile] = 0;
         }
         named_bar_sync(1, EPI_THREADS);   // sk_last is reused by the next partial tile
-            }
+      }
+      if constexpr (C::SC_SLOTS > 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(sc_free + slot));
+      }
+      ++k;
       if (++acc == C::ACC_BUFS) {
         acc = 0;
         acc_phase ^= 1;
@@ -642,13 +692,8 @@ template <Kind KIND, int BN, bool PANEL = false>
 dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2, const CUtensorMap& tc,
                  const GemmArgs& args, int grid, cudaStream_t stream) {
   using C = Cfg<KIND, BN, PANEL>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel<KIND, BN, PANEL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::SMEM_BYTES);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err);
+  const dq_status st = smem_limit_once(reinterpret_cast<const void*>(&gemm_kernel<KIND, BN, PANEL>), C::SMEM_BYTES);
+  if (st != DQ_OK) return st;
   // Programmatic stream serialization: the prologue may overlap the tail of
   // the previous kernel (e.g. the quantization that produced A); the kernel
   // waits (griddep_wait) before its first global memory access.
@@ -673,20 +718,18 @@ constexpr int64_t kMaxK = 133144;   // floor((2^31 - 1) / 127^2): int32 accumula
 // its longer prologue loses to the 1-SM kernel.
 constexpr int64_t kPairMinK = 8192;
 
-// Schedule override for measurements: 0 = automatic, 1 = 1-SM whole tiles,
-// 2 = 1-SM stream-K, 3 = pair (2-SM) kernel for every M, 4 = the dense
-// (tokens on MMA M) arrangement also for M <= 128.
-int g_schedule_override = 0;
-// Tile-width override for measurements (0 = automatic).
-int g_tile_n_override = 0;
-// Measurement knob: 0 turns the two-width Dense schedule off.
-int g_two_widths = 1;
-// Measurement knob: BSR panel variant 0 = never, 1 = automatic (K <= 1280 and
-// blocks smaller than 64), 2 = whenever K <= 1280.
-int g_bsr_panel = 1;
+// The measurement knobs, read once per call.
+struct Knobs {
+  int schedule, tile_n, two_widths, bsr_panel;
+};
+Knobs knobs() {
+  return Knobs{g_schedule_override.load(std::memory_order_relaxed), g_tile_n_override.load(std::memory_order_relaxed),
+               g_two_widths.load(std::memory_order_relaxed), g_bsr_panel.load(std::memory_order_relaxed)};
+}
 
 struct Plan {
   Kind kind;
+  bool pair;         // the 2-SM pair kernel (gemm2sm.cu): 256-row tiles
   int bn;
   int a_tiles, b_tiles, kb_total, num_tiles;
   bool stream_k;
@@ -741,15 +784,32 @@ size_t sk_workspace_bytes(const Plan& p, int /*ctas*/) {
 // scattered: measured at N = 28672, K = 8192: M = 128 47 us vs 57, M = 32
 // 46.3 vs 48.9, M = 16 45.9 vs 46.7, but M = 1 54 vs 46, so from M = 17 on.
 // For fewer channels swap-AB with stream-K keeps every SM busy.
-bool small_m_dense(int64_t M, int64_t N, int sm_count) {
-  if (g_schedule_override == 4 || g_schedule_override == 5) return true;
-  return M > 16 && M <= 128 && g_schedule_override == 0 && g_tile_n_override == 0 &&
-         (N + 223) / 224 >= sm_count * 3 / 4;
+bool small_m_dense(int64_t M, int64_t N, int sm_count, const Knobs& kn) {
+  if (kn.schedule == 4 || kn.schedule == 5) return true;
+  return M > 16 && M <= 128 && kn.schedule == 0 && kn.tile_n == 0 && (N + 223) / 224 >= sm_count * 3 / 4;
 }
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count) {
+// Whether the pair kernel (256-row tiles over two SMs) takes a shape with
+// more than 128 tokens when no schedule is forced.
+bool pair_preferred(int64_t /*M*/, int64_t /*N*/, int64_t K) { return K >= kPairMinK; }
+
+// The schedule of one call: arrangement, kernel, tile widths and (swap-AB)
+// stream-K with the workspace it needs.  `slots` is the number of CTA pairs
+// that fit at once (the pair kernel's wave size), used only for the pair.
+Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count, int pair_slots_n, const Knobs& kn) {
   Plan p{};
-  const bool dense_small = M <= 128 && small_m_dense(M, N, sm_count);
+  p.kb_total = static_cast<int>((K + 127) / 128);
+  if (kn.schedule == 3 || (kn.schedule == 0 && M > 128 && pair_preferred(M, N, K))) {
+    p.kind = Kind::Dense;
+    p.pair = true;
+    p.bn = (kn.tile_n == 160 || kn.tile_n == 192) ? kn.tile_n : 256;
+    p.a_tiles = static_cast<int>((M + 255) / 256);
+    p.b_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
+    p.num_tiles = p.a_tiles * p.b_tiles;
+    if (p.bn == 256 && kn.two_widths && pair_slots_n > 0) plan_two_widths(p, N, pair_slots_n);
+    return p;
+  }
+  const bool dense_small = M <= 128 && small_m_dense(M, N, sm_count, kn);
   if (M <= 128 && !dense_small) {
     p.kind = Kind::Swap;
     p.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
@@ -758,31 +818,51 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count) {
   } else {
     p.kind = Kind::Dense;
     p.bn = N <= 128 ? 128 : dense_small ? 224 : 256;
-    if (g_tile_n_override == 128 || g_tile_n_override == 160 || g_tile_n_override == 192 ||
-        g_tile_n_override == 224 || g_tile_n_override == 256)
-      p.bn = g_tile_n_override;
+    if (kn.tile_n == 128 || kn.tile_n == 160 || kn.tile_n == 192 || kn.tile_n == 224 || kn.tile_n == 256)
+      p.bn = kn.tile_n;
     p.a_tiles = static_cast<int>((M + 127) / 128);
     p.b_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
   }
-  p.kb_total = static_cast<int>((K + 127) / 128);
   p.num_tiles = p.a_tiles * p.b_tiles;
   const long long iters = static_cast<long long>(p.num_tiles) * p.kb_total;
+  if (kn.schedule == 2 || kn.schedule == 5) {
+    // forced stream-K (measurement): ranges over uniform tiles
+    p.stream_k = iters >= sm_count;
+    p.ws_bytes = p.stream_k ? sk_workspace_bytes(p, sm_count) : 0;
+    return p;
+  }
   // Stream-K pays when whole tiles would leave a large share of the SMs idle
-  // in the last wave, and every CTA still gets a few k blocks.
+  // in the last wave, and every CTA still gets a few k blocks.  Measured on
+  // B200: for the dense arrangement splitting costs more than the idle SMs
+  // of the last wave (both with red.add partials and with per-CTA partial
+  // slots plus ready flags), so only swap-AB (few tokens, weight streaming)
+  // splits.
   const int waves = (p.num_tiles + sm_count - 1) / sm_count;
   const double eff = static_cast<double>(p.num_tiles) / (static_cast<double>(waves) * sm_count);
-  // Measured on B200: for the dense arrangement the partial-tile reduction
-  // costs more than the idle SMs it saves, so only swap-AB (few tokens,
-  // weight streaming) splits.
-  // Measured on B200: for the dense arrangement splitting costs more than the
-  // idle SMs of the last wave (both with red.add partials and with per-CTA
-  // partial slots plus ready flags), so only swap-AB (few tokens, weight
-  // streaming) splits.
   const bool worth = p.kind == Kind::Swap && eff < 0.9 && iters >= 4LL * sm_count;
   p.ws_bytes = worth ? sk_workspace_bytes(p, sm_count) : 0;
-  p.stream_k = worth;
-  if (p.kind == Kind::Dense && p.bn == 256 && g_tile_n_override == 0 && g_two_widths) plan_two_widths(p, N, sm_count);
+  p.stream_k = worth && kn.schedule != 1;
+  if (!worth) p.ws_bytes = 0;
+  if (p.kind == Kind::Dense && p.bn == 256 && kn.tile_n == 0 && kn.two_widths) plan_two_widths(p, N, sm_count);
   return p;
+}
+
+// Host-side checks of dq_int8_linear's arguments (shared with the
+// allocation-free entry point, so both refuse the same calls).
+dq_status check_linear_args(const int8_t* A, const float* s_row, int64_t M, int64_t K, const int8_t* W,
+                            const float* s_col, int64_t N, const void* bias_bf16, const void* out,
+                            dq_out_dtype out_dtype) {
+  if (out_dtype != DQ_OUT_BF16 && out_dtype != DQ_OUT_S32) return DQ_ERR_INVALID_ARG;
+  if (M < 0 || K < 1 || N < 1) return DQ_ERR_INVALID_ARG;
+  if (M > 0 && (A == nullptr || W == nullptr || out == nullptr)) return DQ_ERR_INVALID_ARG;
+  if (M > 0 && out_dtype == DQ_OUT_BF16 && (s_row == nullptr || s_col == nullptr))
+    return DQ_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > kMaxK || N % 8 != 0) return DQ_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 128 || N > (int64_t(1) << 31) - 256) return DQ_ERR_UNSUPPORTED;
+  if (!aligned(A, 16) || !aligned(W, 16) || !aligned(out, 16)) return DQ_ERR_UNSUPPORTED;
+  if (out_dtype == DQ_OUT_BF16 && (!aligned(s_col, 16) || (bias_bf16 && !aligned(bias_bf16, 16))))
+    return DQ_ERR_UNSUPPORTED;
+  return DQ_OK;
 }
 
 }  // namespace
@@ -796,76 +876,64 @@ size_t dq_int8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 1) return 0;
   DeviceInfo* d = nullptr;
   if (current_device(&d) != DQ_OK) return 0;
-  return make_plan(M, N, K, d->sm_count).ws_bytes;
+  const Plan p = make_plan(M, N, K, d->sm_count, 0, knobs());
+  return p.pair ? 0 : p.ws_bytes;
 }
-
-// Measurement knob (not in the public header): force a schedule.
-void dq_debug_set_schedule(int mode) { g_schedule_override = mode; }
-void dq_debug_set_tile_n(int n) { g_tile_n_override = n; }
-void dq_debug_set_two_widths(int on) { g_two_widths = on; }
-void dq_debug_set_bsr_panel(int mode) { g_bsr_panel = mode; }
 
 dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t K, const int8_t* W,
                          const float* s_col, int64_t N, const void* bias_bf16, void* out,
                          dq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
                          dq_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  if (out_dtype != DQ_OUT_BF16 && out_dtype != DQ_OUT_S32) return DQ_ERR_INVALID_ARG;
-  if (M < 0 || K < 1 || N < 1) return DQ_ERR_INVALID_ARG;
-  if (M > 0 && (A == nullptr || W == nullptr || out == nullptr)) return DQ_ERR_INVALID_ARG;
-  if (M > 0 && out_dtype == DQ_OUT_BF16 && (s_row == nullptr || s_col == nullptr))
-    return DQ_ERR_INVALID_ARG;
-  if (K % 16 != 0 || K > kMaxK || N % 8 != 0) return DQ_ERR_UNSUPPORTED;
-  if (M > (int64_t(1) << 31) - 128 || N > (int64_t(1) << 31) - 256) return DQ_ERR_UNSUPPORTED;
-  if (!aligned(A, 16) || !aligned(W, 16) || !aligned(out, 16)) return DQ_ERR_UNSUPPORTED;
-  if (out_dtype == DQ_OUT_BF16 && (!aligned(s_col, 16) || (bias_bf16 && !aligned(bias_bf16, 16))))
-    return DQ_ERR_UNSUPPORTED;
+  dq_status st0 = check_linear_args(A, s_row, M, K, W, s_col, N, bias_bf16, out, out_dtype);
+  if (st0 != DQ_OK) return st0;
   DeviceInfo* d = nullptr;
   dq_status st = current_device(&d);
   if (st != DQ_OK) return st;
   if (M == 0) return DQ_OK;
 
-  // Dense arrangement: each 256x256 tile runs on a pair of SMs (gemm2sm.cu)
-  // unless a 1-SM schedule is forced for measurement (1 = whole tiles,
-  // 2 = stream-K); 3 forces the pair kernel for any M.
-  if ((M > 128 && K >= kPairMinK && g_schedule_override != 1 && g_schedule_override != 2) ||
-      g_schedule_override == 3) {
-    CUtensorMap ta, tb, tc;
+  const Knobs kn = knobs();
+  int pairs = 0;
+  if (kn.schedule == 3 || (kn.schedule == 0 && M > 128 && pair_preferred(M, N, K))) {
+    if ((st = pair_slots(*d, &pairs)) != DQ_OK) return st;
+  }
+  Plan p = make_plan(M, N, K, d->sm_count, pairs, kn);
+  if (p.pair) {
+    // Each 256-row tile's MMAs run on a pair of SMs (gemm2sm.cu).
+    CUtensorMap ta, tb, tb2, tc;
     if ((st = make_tmap_u8_2d(&ta, A, K, M, K, 128, 128, 128)) != DQ_OK) return st;
-    const int bn_pair = (g_tile_n_override == 160 || g_tile_n_override == 192) ? g_tile_n_override : 256;
-    if ((st = make_tmap_u8_2d(&tb, W, K, N, K, 128, bn_pair / 2, 128)) != DQ_OK) return st;
+    if ((st = make_tmap_u8_2d(&tb, W, K, N, K, 128, p.bn / 2, 128)) != DQ_OK) return st;
+    if (p.bn2 > 0) {
+      if ((st = make_tmap_u8_2d(&tb2, W, K, N, K, 128, p.bn2 / 2, 128)) != DQ_OK) return st;
+    } else {
+      tb2 = tb;
+    }
     if ((st = make_tmap_out_2d(&tc, out, N, M, out_dtype == DQ_OUT_S32 ? 4 : 2)) != DQ_OK) return st;
     GemmArgs g{};
     g.M = static_cast<int>(M);
     g.N = static_cast<int>(N);
     g.K = static_cast<int>(K);
-    const int bn = (g_tile_n_override == 160 || g_tile_n_override == 192) ? g_tile_n_override : 256;
-    g.a_tiles = static_cast<int>((M + 255) / 256);
-    g.b_tiles = static_cast<int>((N + bn - 1) / bn);
-    g.kb_total = static_cast<int>((K + 127) / 128);
-    const int64_t tiles = static_cast<int64_t>(g.a_tiles) * g.b_tiles;
-    if (tiles > 0x7fffffff) return DQ_ERR_UNSUPPORTED;
-    g.num_tiles = static_cast<int>(tiles);
+    g.a_tiles = p.a_tiles;
+    g.b_tiles = p.b_tiles;
+    g.kb_total = p.kb_total;
+    g.num_tiles = p.num_tiles;
+    g.t1 = p.t1;
+    g.bn2 = p.bn2;
+    g.mb0 = p.mb0;
+    g.c_start = p.c_start;
+    g.first_cnt = p.first_cnt;
+    g.per_row = p.per_row;
     g.s_row = s_row;
     g.s_col = s_col;
     g.bias = static_cast<const uint16_t*>(bias_bf16);
     g.out = out;
     g.out_s32 = out_dtype == DQ_OUT_S32 ? 1 : 0;
     g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
-    return launch_pair_gemm(ta, tb, tc, g, bn, *d, stream);
+    return launch_pair_gemm(ta, tb, tb2, tc, g, p.bn, p.num_tiles < pairs ? p.num_tiles : pairs, stream);
   }
 
-  Plan p = make_plan(M, N, K, d->sm_count);
-  bool sk = p.stream_k && workspace != nullptr && workspace_bytes >= p.ws_bytes &&
-            aligned(workspace, 16);
-  if (g_schedule_override == 1) sk = false;
-  if (g_schedule_override == 2 || g_schedule_override == 5) {
-    p.bn2 = 0;                                    // stream-K ranges run over uniform tiles
-    p.num_tiles = p.a_tiles * p.b_tiles;
-    if (workspace != nullptr && aligned(workspace, 16) &&
-        workspace_bytes >= sk_workspace_bytes(p, d->sm_count))
-      sk = static_cast<long long>(p.num_tiles) * p.kb_total >= d->sm_count;
-  }
+  // stream-K only with a large enough workspace (else whole tiles, same bits)
+  const bool sk = p.stream_k && workspace != nullptr && workspace_bytes >= p.ws_bytes && aligned(workspace, 16);
 
   CUtensorMap ta, tb, tb2;
   const int8_t* a_src = p.kind == Kind::Swap ? W : A;
@@ -957,7 +1025,7 @@ dq_status dq_fp8_linear(const uint8_t* A, const float* s_row, int64_t M, int64_t
   p.b_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
   p.kb_total = static_cast<int>((K + 127) / 128);
   p.num_tiles = p.a_tiles * p.b_tiles;
-  if (p.bn == 256 && g_two_widths) plan_two_widths(p, N, d->sm_count);
+  if (p.bn == 256 && knobs().two_widths) plan_two_widths(p, N, d->sm_count);
   CUtensorMap ta, tb, tb2, tc;
   if ((st = make_tmap_u8_2d(&ta, A, K, M, K, 128, 128, 128)) != DQ_OK) return st;
   if ((st = make_tmap_u8_2d(&tb, W, K, N, K, 128, p.bn, 128)) != DQ_OK) return st;
@@ -1028,8 +1096,9 @@ dq_status dq_bsr_int8_linear_blocked(const int8_t* A, const float* s_row, int64_
   // the panel vs 725 streaming, 16x16 2143 vs 2514; 64x64 blocks are as fast
   // or faster streaming (10 %: 266 vs 269 us, 20 %: 384 vs 396), where the
   // per-block MMA issue, not the activation traffic, bounds the kernel.
+  const Knobs kn = knobs();
   const bool panel = K <= Cfg<Kind::Bsr, 256, true>::KP &&
-                     (g_bsr_panel == 2 || (g_bsr_panel == 1 && block < 64));
+                     (kn.bsr_panel == 2 || (kn.bsr_panel == 1 && block < 64));
   const int kb = panel ? 128 : block == 64 ? 64 : 32;
   const int bsw = block == 16 ? 0 : static_cast<int>(block);
   const uint32_t ub = static_cast<uint32_t>(block);
@@ -1145,6 +1214,12 @@ dq_status dq_bsr_validate(const int32_t* crow, const int32_t* col, int64_t N, in
 // memory get the stream-K workspace from this file-scope array instead.  In
 // host code `g_noalloc_scratch` names a host-side stand-in, not the device
 // array, so its device address is looked up once per device.
+//
+// The stream-K kernel leaves every partial tile and arrival counter it used
+// at zero when it completes, so the array needs zeroing only before its first
+// use on a device and after a kernel gave up a bounded wait (which can leave
+// partial sums behind): dq_sync_status reports that as DQ_ERR_TIMEOUT and
+// marks the device's array for re-zeroing by the next call.
 namespace dq {
 namespace {
 
@@ -1152,11 +1227,15 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[DQ_NOALLOC_SCRATCH_BY
 
 constexpr int kNoallocMaxDevices = 64;
 void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+std::atomic<int> g_noalloc_dirty[kNoallocMaxDevices] = {};
 std::mutex g_noalloc_mutex;
 
 // Device address of the scratch array on the current device (set-up on the
-// first call per device, with that device current).
-dq_status noalloc_scratch(void** out) {
+// first call per device, with that device current): the address lookup and
+// one zero-fill of the whole array on `stream`, which the call then waits
+// for, so that later calls on any stream find it zero.  A re-zeroing asked
+// for by dq_sync_status is queued on `stream` ahead of the call's kernel.
+dq_status noalloc_scratch(cudaStream_t stream, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -1166,31 +1245,43 @@ dq_status noalloc_scratch(void** out) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaMemsetAsync(p, 0, DQ_NOALLOC_SCRATCH_BYTES, stream)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamSynchronize(stream)) != cudaSuccess) return cuda_fail(e);
     g_noalloc_ptr[dev] = p;
+    g_noalloc_dirty[dev].store(0);
+  } else if (g_noalloc_dirty[dev].exchange(0) != 0) {
+    if ((e = cudaMemsetAsync(g_noalloc_ptr[dev], 0, DQ_NOALLOC_SCRATCH_BYTES, stream)) != cudaSuccess) {
+      g_noalloc_dirty[dev].store(1);
+      return cuda_fail(e);
+    }
   }
   *out = g_noalloc_ptr[dev];
   return DQ_OK;
 }
 
 }  // namespace
+
+void noalloc_mark_dirty(int device) {
+  if (device >= 0 && device < kNoallocMaxDevices) g_noalloc_dirty[device].store(1);
+}
+
 }  // namespace dq
 
 extern "C" dq_status dq_int8_linear_noalloc(const int8_t* A, const float* s_row, int64_t M, int64_t K,
                                             const int8_t* W, const float* s_col, int64_t N,
                                             const void* bias_bf16, void* out, dq_out_dtype out_dtype,
                                             dq_stream_t stream) {
-  if (M < 1 || K < 1 || N < 1)   // M == 0 and bad sizes: the plain entry point decides, no scratch
-    return dq_int8_linear(A, s_row, M, K, W, s_col, N, bias_bf16, out, out_dtype, nullptr, 0, stream);
+  dq_status st = check_linear_args(A, s_row, M, K, W, s_col, N, bias_bf16, out, out_dtype);
+  if (st != DQ_OK) return st;
+  if (M == 0) return dq_int8_linear(A, s_row, M, K, W, s_col, N, bias_bf16, out, out_dtype, nullptr, 0, stream);
   DeviceInfo* d = nullptr;
-  dq_status st = current_device(&d);
+  st = current_device(&d);
   if (st != DQ_OK) return st;
   const size_t need = dq_int8_linear_workspace_size(M, N, K);
   if (need > DQ_NOALLOC_SCRATCH_BYTES) return DQ_ERR_UNSUPPORTED;
   if (need == 0)
     return dq_int8_linear(A, s_row, M, K, W, s_col, N, bias_bf16, out, out_dtype, nullptr, 0, stream);
   void* scratch = nullptr;
-  if ((st = noalloc_scratch(&scratch)) != DQ_OK) return st;
-  cudaError_t e = cudaMemsetAsync(scratch, 0, need, reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e);
+  if ((st = noalloc_scratch(reinterpret_cast<cudaStream_t>(stream), &scratch)) != DQ_OK) return st;
   return dq_int8_linear(A, s_row, M, K, W, s_col, N, bias_bf16, out, out_dtype, scratch, need, stream);
 }

@@ -99,6 +99,38 @@ struct SegIter {
   }
 };
 
+// Where a tile lies: row block ta (128 rows for the 1-SM kernel, 256 for the
+// pair kernel), B-slot tile tb, first output column n0 and the MMA width (bn,
+// or g.bn2 for a Dense tile of the narrow second set).
+struct TileGeom {
+  int ta, tb, n0, width;
+  bool narrow;
+};
+__device__ __forceinline__ TileGeom tile_geom(const GemmArgs& g, int tile, int bn, bool two_widths) {
+  TileGeom t;
+  if (two_widths && g.bn2 > 0 && tile >= g.t1) {
+    int j = tile - g.t1;
+    if (j < g.first_cnt) {
+      t.ta = g.mb0;
+      t.n0 = g.c_start + j * g.bn2;
+    } else {
+      j -= g.first_cnt;
+      t.ta = g.mb0 + 1 + j / g.per_row;
+      t.n0 = (j % g.per_row) * g.bn2;
+    }
+    t.tb = 0;
+    t.width = g.bn2;
+    t.narrow = true;
+  } else {
+    t.ta = tile / g.b_tiles;
+    t.tb = tile % g.b_tiles;
+    t.n0 = t.tb * bn;
+    t.width = bn;
+    t.narrow = false;
+  }
+  return t;
+}
+
 // Stream-K: number of CTAs whose ranges touch `tile`.
 __device__ __forceinline__ int sk_contributors(const GemmArgs& g, int tile) {
   const long long G = gridDim.x, T = g.iters_total;
@@ -125,12 +157,28 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
 // Column scales of one 32-column chunk as f32x2 pairs (s_col[n0 + 2i],
 // s_col[n0 + 2i + 1]); zero past N (N % 8 == 0, so 8-column groups are wholly
 // inside or outside).  All eight loads are issued before any is used.
 struct ColScales {
   uint64_t sc[16];
 };
+// The same pairs out of a tile's staged slot (stage_tile_scales), c0 = the
+// chunk's column offset from the tile's first column.
+__device__ __forceinline__ void load_col_scales_staged(uint32_t slot, int c0, ColScales& p) {
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    const uint4 w = lds_v4(slot + static_cast<uint32_t>(c0) * 4u + 16u * v);
+    p.sc[2 * v] = (static_cast<uint64_t>(w.y) << 32) | w.x;
+    p.sc[2 * v + 1] = (static_cast<uint64_t>(w.w) << 32) | w.z;
+  }
+}
 __device__ __forceinline__ void load_col_scales(const GemmArgs& g, int n0, ColScales& p) {
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
@@ -147,6 +195,41 @@ __device__ __forceinline__ void load_col_scales(const GemmArgs& g, int n0, ColSc
   }
 }
 
+// A tile's column scales (fp32) and bias (bf16) staged in shared memory, so
+// that the epilogue reads them there instead of issuing a dependent L2 load
+// for every 32-column chunk.  One slot per tile in flight: s_col at +0 (up to
+// 256 fp32), bias at +kScBiasOff (up to 256 bf16).  One thread copies them
+// with 1-D bulk copies completing on the slot's mbarrier; columns past N are
+// not copied (their outputs are clipped by the store).
+constexpr int kScSlotBytes = 1536;
+constexpr int kScBiasOff = 1024;
+
+__device__ __forceinline__ void stage_tile_scales(const GemmArgs& g, uint32_t slot, int n0, int width,
+                                                  uint32_t bar) {
+  const int ncols = min(width, g.N - n0);          // a multiple of 8 (N % 8 == 0, n0 % 32 == 0)
+  const bool need = !g.out_s32 && ncols > 0;
+  const uint32_t sb = need ? static_cast<uint32_t>(ncols) * 4u : 0u;
+  const uint32_t bb = need && g.bias != nullptr ? static_cast<uint32_t>(ncols) * 2u : 0u;
+  mbar_arrive_expect_tx(bar, sb + bb);
+  if (sb) bulk_load_1d(slot, g.s_col + n0, sb, bar);
+  if (bb) bulk_load_1d(slot + kScBiasOff, g.bias + n0, bb, bar);
+}
+
+// Bias words of the 32-column chunk at column offset c0 (from the tile's
+// first column) out of a staged slot.
+__device__ __forceinline__ void load_bias_staged(uint32_t slot, int c0, uint4 (&b)[4]) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) b[v] = lds_v4(slot + kScBiasOff + static_cast<uint32_t>(c0) * 2u + 16u * v);
+}
+// Bias words of the chunk at output column n0 from global memory (zero past N).
+__device__ __forceinline__ void load_bias_global(const GemmArgs& g, int n0, uint4 (&b)[4]) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int n = n0 + 8 * v;
+    b[v] = n < g.N ? __ldg(reinterpret_cast<const uint4*>(g.bias + n)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 // Epilogue for one chunk of 32 columns of the Dense/Bsr layout: thread = row
 // `row` (0..31 inside its warp's 32-row slab), output columns n0 .. n0+31.
 // The 32x32 block is written into the warp's staging buffer with the tensor
@@ -159,7 +242,8 @@ __device__ __forceinline__ void load_col_scales(const GemmArgs& g, int n0, ColSc
 template <bool S32, bool BIAS, bool F32ACC>
 __device__ __forceinline__ void store_row_chunk_tma_t(const GemmArgs& g, const CUtensorMap* tm_c,
                                                       uint8_t* buf, int lane, int m0, int n0,
-                                                      const uint32_t* r, float srow, const ColScales& cs) {
+                                                      const uint32_t* r, float srow, const ColScales& cs,
+                                                      const uint4 (&bias)[4]) {
   const uint32_t base = smem_u32(buf);
   if constexpr (S32) {
 #pragma unroll
@@ -187,10 +271,7 @@ __device__ __forceinline__ void store_row_chunk_tma_t(const GemmArgs& g, const C
     if constexpr (BIAS) {
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        const int n = n0 + 8 * v;
-        uint4 b = make_uint4(0u, 0u, 0u, 0u);
-        if (n < g.N) b = __ldg(reinterpret_cast<const uint4*>(g.bias + n));
-        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+        const uint32_t bw[4] = {bias[v].x, bias[v].y, bias[v].z, bias[v].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           f2[4 * v + j] =
@@ -220,14 +301,85 @@ __device__ __forceinline__ void store_row_chunk_tma_t(const GemmArgs& g, const C
   }
 }
 
+// The same chunk epilogue with the column scales and bias read from the
+// tile's staged shared-memory slot (stage_tile_scales) as they are needed,
+// c0 = the chunk's column offset from the tile's first column: nothing is
+// held in registers beyond the 32 accumulators and the 16 packed outputs.
+template <bool S32, bool BIAS, bool F32ACC>
+__device__ __forceinline__ void store_row_chunk_staged_t(const GemmArgs& g, const CUtensorMap* tm_c, uint8_t* buf,
+                                                         int lane, int m0, int n0, const uint32_t* r, float srow,
+                                                         uint32_t slot, int c0) {
+  const uint32_t base = smem_u32(buf);
+  if constexpr (S32) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t off = static_cast<uint32_t>(lane * 128 + ((j ^ (lane & 7)) << 4));
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(r[4 * j]),
+                   "r"(r[4 * j + 1]), "r"(r[4 * j + 2]), "r"(r[4 * j + 3])
+                   : "memory");
+    }
+  } else {
+    // ((float)acc * s_row) * s_col (+ bias) as f32x2 pairs, left to right,
+    // each lane rounded like the scalar op; 8 columns per step.
+    const uint64_t srow2 = pack_f2(srow, srow);
+    const uint32_t sc_addr = slot + static_cast<uint32_t>(c0) * 4u;
+    const uint32_t b_addr = slot + kScBiasOff + static_cast<uint32_t>(c0) * 2u;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 s0 = lds_v4(sc_addr + 32u * v);
+      const uint4 s1 = lds_v4(sc_addr + 32u * v + 16u);
+      const uint64_t sc[4] = {(static_cast<uint64_t>(s0.y) << 32) | s0.x, (static_cast<uint64_t>(s0.w) << 32) | s0.z,
+                              (static_cast<uint64_t>(s1.y) << 32) | s1.x, (static_cast<uint64_t>(s1.w) << 32) | s1.z};
+      uint4 b = make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (BIAS) b = lds_v4(b_addr + 16u * v);
+      const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = 8 * v + 2 * j;
+        const uint64_t a = F32ACC ? pack_f2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]))
+                                  : pack_f2(__int2float_rn(static_cast<int>(r[e])),
+                                            __int2float_rn(static_cast<int>(r[e + 1])));
+        uint64_t f = mul_f2(mul_f2(a, srow2), sc[j]);
+        if constexpr (BIAS) f = add_f2(f, pack_f2(__uint_as_float(bw[j] << 16), __uint_as_float(bw[j] & 0xffff0000u)));
+        float lo, hi;
+        unpack_f2(f, lo, hi);
+        w[j] = pack_bf16x2(lo, hi);
+      }
+      const uint32_t off = static_cast<uint32_t>(lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4));
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                   "r"(w[3])
+                   : "memory");
+    }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && n0 < g.N && m0 < g.M) {   // boxes wholly past the matrix are not issued
+    tma_store_2d(tm_c, base, n0, m0);
+    bulk_commit_group();
+  }
+}
+
+template <bool F32ACC = false>
+__device__ __forceinline__ void store_row_chunk_staged(const GemmArgs& g, const CUtensorMap* tm_c, uint8_t* buf,
+                                                       int lane, int m0, int n0, const uint32_t* r, float srow,
+                                                       uint32_t slot, int c0) {
+  if (g.out_s32) store_row_chunk_staged_t<true, false, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, slot, c0);
+  else if (g.bias != nullptr)
+    store_row_chunk_staged_t<false, true, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, slot, c0);
+  else store_row_chunk_staged_t<false, false, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, slot, c0);
+}
+
+// `bias` holds the chunk's 32 bf16 bias values (read only when g.bias is set).
 template <bool F32ACC = false>
 __device__ __forceinline__ void store_row_chunk_tma(const GemmArgs& g, const CUtensorMap* tm_c, uint8_t* buf,
                                                     int lane, int m0, int n0, const uint32_t* r, float srow,
-                                                    const ColScales& cs) {
+                                                    const ColScales& cs, const uint4 (&bias)[4]) {
   // raw mode stores the accumulator bits (int32, or fp32 for e4m3 operands)
-  if (g.out_s32) store_row_chunk_tma_t<true, false, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
-  else if (g.bias != nullptr) store_row_chunk_tma_t<false, true, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
-  else store_row_chunk_tma_t<false, false, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, cs);
+  if (g.out_s32) store_row_chunk_tma_t<true, false, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, cs, bias);
+  else if (g.bias != nullptr)
+    store_row_chunk_tma_t<false, true, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, cs, bias);
+  else store_row_chunk_tma_t<false, false, F32ACC>(g, tm_c, buf, lane, m0, n0, r, srow, cs, bias);
 }
 
 // Epilogue for the Swap layout: thread = output channel n, columns are
@@ -259,8 +411,12 @@ __device__ __forceinline__ void store_col_chunk(const GemmArgs& g, int n, int m0
 }
 
 // Dense GEMM with each 256 x bn tile's MMA on a pair of SMs (gemm2sm.cu).
-// g.a_tiles / g.b_tiles count 256-row / bn-column tiles; bn is 160, 192 or 256.
-dq_status launch_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, GemmArgs g,
-                           int bn, const DeviceInfo& d, cudaStream_t stream);
+// g.a_tiles / g.b_tiles count 256-row / bn-column tiles; bn is 160, 192 or
+// 256; with g.bn2 > 0 the tiles from g.t1 on are bn2 wide (tm_b2's box is
+// bn2 / 2 weight rows).  `pairs` is the number of CTA pairs to launch.
+dq_status launch_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2,
+                           const CUtensorMap& tc, const GemmArgs& g, int bn, int pairs, cudaStream_t stream);
+// CTA pairs of the pair kernel that fit on the current device at once.
+dq_status pair_slots(const DeviceInfo& d, int* pairs);
 
 }  // namespace dq

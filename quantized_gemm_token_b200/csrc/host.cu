@@ -37,7 +37,54 @@ void resolve_encoder() {
     g_encode_err = cudaErrorNotSupported;
 }
 
+// Kernels whose shared-memory limit has been raised, per device.  Entries
+// are appended under the mutex and published by the release store of n, so
+// the scan needs no lock.
+struct AttrEntry {
+  const void* kernel;
+  int bytes;
+};
+constexpr int kMaxAttr = 96;
+struct DeviceAttrs {
+  std::atomic<int> n{0};
+  AttrEntry e[kMaxAttr];
+};
+DeviceAttrs g_attrs[kMaxDevices];
+std::mutex g_attr_mutex;
+
+bool attr_known(const DeviceAttrs& a, const void* kernel, int bytes) {
+  const int n = a.n.load(std::memory_order_acquire);
+  for (int i = 0; i < n; ++i)
+    if (a.e[i].kernel == kernel && a.e[i].bytes >= bytes) return true;
+  return false;
+}
+
 }  // namespace
+
+std::atomic<int> g_schedule_override{0};
+std::atomic<int> g_tile_n_override{0};
+std::atomic<int> g_two_widths{1};
+std::atomic<int> g_bsr_panel{1};
+std::atomic<int> g_quant_kernel_override{0};
+
+dq_status smem_limit_once(const void* kernel, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return DQ_ERR_UNSUPPORTED;
+  DeviceAttrs& a = g_attrs[dev];
+  if (attr_known(a, kernel, bytes)) return DQ_OK;
+  std::lock_guard<std::mutex> lock(g_attr_mutex);
+  if (attr_known(a, kernel, bytes)) return DQ_OK;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int n = a.n.load(std::memory_order_relaxed);
+  if (n < kMaxAttr) {               // a full table only costs a repeated (harmless) set
+    a.e[n] = AttrEntry{kernel, bytes};
+    a.n.store(n + 1, std::memory_order_release);
+  }
+  return DQ_OK;
+}
 
 dq_status cuda_fail(cudaError_t e) {
   t_last_cuda_error = static_cast<int>(e);
@@ -207,6 +254,12 @@ int dq_last_cuda_error(void) { return t_last_cuda_error; }
 
 int dq_version(void) { return 100; }
 
+void dq_debug_set_schedule(int mode) { g_schedule_override.store(mode, std::memory_order_relaxed); }
+void dq_debug_set_tile_n(int n) { g_tile_n_override.store(n, std::memory_order_relaxed); }
+void dq_debug_set_two_widths(int on) { g_two_widths.store(on, std::memory_order_relaxed); }
+void dq_debug_set_bsr_panel(int mode) { g_bsr_panel.store(mode, std::memory_order_relaxed); }
+void dq_debug_set_quant_kernel(int mode) { g_quant_kernel_override.store(mode, std::memory_order_relaxed); }
+
 void dq_set_wait_timeout_ns(uint64_t ns) {
   g_timeout_ns.store(ns == 0 ? 2000000000ull : static_cast<unsigned long long>(ns));
 }
@@ -224,6 +277,7 @@ dq_status dq_sync_status(dq_stream_t stream) {
     const uint32_t zero = 0;
     e = cudaMemcpyToSymbol(g_err_word, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_fail(e);
+    if (word & kErrTimeout) noalloc_mark_dirty(d->device);
   }
   return (word & kErrTimeout) ? DQ_ERR_TIMEOUT : DQ_OK;
 }
@@ -245,12 +299,7 @@ dq_status dq_mma_peak_probe(int grid, int iters, dq_stream_t stream) {
   if (iters < 1) return DQ_ERR_INVALID_ARG;
   if (grid <= 0) grid = d->sm_count;
   const int smem = (128 + 256) * 128 + 1024;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [&] {
-    attr_err = cudaFuncSetAttribute(mma_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err);
+  if ((st = smem_limit_once(reinterpret_cast<const void*>(&mma_peak_kernel), smem)) != DQ_OK) return st;
   WaitCtl ctl{d->err_word, wait_timeout_ns()};
   mma_peak_kernel<<<grid, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(iters, ctl);
   cudaError_t e = cudaGetLastError();

@@ -28,7 +28,6 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "internal.h"
 #include "pipeline.cuh"
@@ -649,13 +648,8 @@ dq_status check_weights(const uint8_t* packed, const void* scale, const void* ze
 template <bool TRANS, bool S4>
 dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const HqqArgs& g, int grid, size_t smem,
                      cudaStream_t stream) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(hqq_gemm_kernel<TRANS, S4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    HQ_SMEM_LIMIT);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err);
+  const dq_status st = smem_limit_once(reinterpret_cast<const void*>(&hqq_gemm_kernel<TRANS, S4>), HQ_SMEM_LIMIT);
+  if (st != DQ_OK) return st;
   hqq_gemm_kernel<TRANS, S4><<<grid, HQ_THREADS, smem, stream>>>(tx, tw, g);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);

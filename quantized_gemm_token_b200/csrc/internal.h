@@ -22,6 +22,17 @@ struct DeviceInfo {
 // Resolves the current device's info; DQ_ERR_UNSUPPORTED if it is not sm_100.
 dq_status current_device(DeviceInfo** out);
 
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device, once per (device, kernel): the attribute belongs to a device's
+// context, so every device the process launches on needs its own setting.
+// Thread-safe; later calls for the same pair cost a short table scan.
+dq_status smem_limit_once(const void* kernel, int bytes);
+
+// Asks dq_int8_linear_noalloc to zero its static scratch on `device` again
+// before its next use (a kernel that gave up a bounded wait may have left
+// partial sums in it).
+void noalloc_mark_dirty(int device);
+
 // Records a CUDA error for dq_last_cuda_error() and returns DQ_ERR_CUDA.
 dq_status cuda_fail(cudaError_t e);
 
@@ -48,18 +59,13 @@ inline bool aligned(const void* p, size_t a) {
 
 }  // namespace dq
 
-// Measurement knob, not part of the public header: 0 = automatic schedule,
-// 1 = 1-SM kernel with whole tiles, 2 = 1-SM stream-K whenever a workspace
-// allows it, 3 = the 2-SM pair kernel for every M, 4 = the dense arrangement
-// also for M <= 128.
-extern "C" DQ_API void dq_debug_set_schedule(int mode);
-// Measurement knob: force the dense tile width (128, 160, 192, 224, 256; 0 = automatic).
-extern "C" DQ_API void dq_debug_set_tile_n(int n);
-// Measurement knob: 0 turns off the two-width (wave-balanced) dense schedule.
-extern "C" DQ_API void dq_debug_set_two_widths(int on);
-// Measurement knob: BSR panel variant (activation panel kept in shared memory,
-// K <= 1280): 0 = never, 1 = automatic (blocks smaller than 64), 2 = always.
-extern "C" DQ_API void dq_debug_set_bsr_panel(int mode);
-// Measurement knob: quantize kernel (0 = automatic, 1 = register-resident,
-// 2 = row-pipelined through shared memory).
-extern "C" DQ_API void dq_debug_set_quant_kernel(int mode);
+// Measurement knobs (declared in include/dq.h, "measurement knobs"): read at
+// every launch, written by dq_debug_set_*; process-wide, relaxed atomics.
+#include <atomic>
+namespace dq {
+extern std::atomic<int> g_schedule_override;
+extern std::atomic<int> g_tile_n_override;
+extern std::atomic<int> g_two_widths;
+extern std::atomic<int> g_bsr_panel;
+extern std::atomic<int> g_quant_kernel_override;
+}  // namespace dq

@@ -18,8 +18,6 @@
 // shared-memory ring) is kept as an alternative for 1-16 KB rows.
 #include <cuda_bf16.h>
 
-#include <mutex>
-
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -492,9 +490,6 @@ __global__ void __launch_bounds__(QT_THREADS, 1)
   __syncthreads();      // no CTA leaves with a bulk load still landing in its ring
 }
 
-// Measurement knob: 0 = automatic, 1 = register kernel, 2 = pipelined kernel.
-int g_quant_kernel_override = 0;
-
 template <typename T, QFmt F = QFmt::I8>
 dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
                           float* scales, cudaStream_t stream) {
@@ -540,13 +535,8 @@ dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t*
     const int stages = (max_stages / groups) * groups;
     if (stages < groups) return DQ_ERR_UNSUPPORTED;    // not reachable for rows <= 16 KB
     const int smem = stages * stage_bytes;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-      attr_err = cudaFuncSetAttribute(quant_rows_tma_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      QT_RING_BYTES);
-    });
-    if (attr_err != cudaSuccess) return cuda_fail(attr_err);
+    const dq_status ast = smem_limit_once(reinterpret_cast<const void*>(&quant_rows_tma_kernel<T>), QT_RING_BYTES);
+    if (ast != DQ_OK) return ast;
     const int64_t grid = M < d->sm_count ? M : d->sm_count;
     WaitCtl wait{d->err_word, wait_timeout_ns()};
     quant_rows_tma_kernel<T><<<static_cast<unsigned>(grid), QT_THREADS, smem, stream>>>(
@@ -586,8 +576,6 @@ dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t*
 }  // namespace dq
 
 extern "C" {
-
-void dq_debug_set_quant_kernel(int mode) { dq::g_quant_kernel_override = mode; }
 
 dq_status dq_quantize_rows(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q,
                            int64_t ldq, float* scales, dq_stream_t stream) {

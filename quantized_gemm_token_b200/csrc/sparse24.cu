@@ -34,7 +34,6 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "internal.h"
 #include "pipeline.cuh"
@@ -595,12 +594,8 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
   }
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
 
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(s24_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S4_SMEM_LIMIT);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err);
+  const dq_status ast = smem_limit_once(reinterpret_cast<const void*>(&s24_gemm_kernel), S4_SMEM_LIMIT);
+  if (ast != DQ_OK) return ast;
   s24_gemm_kernel<<<p.grid, S4_THREADS, p.smem, reinterpret_cast<cudaStream_t>(stream)>>>(tq, tv, tm, g);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);

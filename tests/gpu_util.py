@@ -40,3 +40,30 @@ def sample_rows(M: int, n_random: int, seed: int = 0) -> np.ndarray:
     r = np.random.Generator(np.random.Philox(key=seed)).choice(M, size=min(M, n_random), replace=False)
     rows = np.unique(np.clip(np.concatenate([np.array(fixed), r]), 0, M - 1))
     return rows.astype(np.int64)
+
+
+def tile_rows(M: int, total: int = 1024, seed: int = 0, tile: int = 128) -> np.ndarray:
+    """Rows for full-size parity: the first and last row of every `tile`-row
+    block (so every M-tile of the 1-SM kernels and, with tile = 128, both
+    halves of every 256-row pair tile), the rows around the middle, plus
+    seeded random rows until at least `total` rows (or all M) are chosen."""
+    starts = np.arange(0, M, tile)
+    edges = np.concatenate([starts, np.minimum(starts + tile - 1, M - 1), [M // 2, M - 1]])
+    rows = np.unique(np.clip(edges, 0, M - 1))
+    if rows.size < min(total, M):
+        rng = np.random.Generator(np.random.Philox(key=seed))
+        rest = np.setdiff1d(np.arange(M), rows)
+        extra = rng.choice(rest, size=min(total, M) - rows.size, replace=False)
+        rows = np.unique(np.concatenate([rows, extra]))
+    return rows.astype(np.int64)
+
+
+def tile_cols(N: int, widths=(128, 224, 256), extra_step: int = 97) -> np.ndarray:
+    """Output channels at both edges of every tile of each width (the swap
+    arrangement's 128-channel tiles, the few-token dense arrangement's
+    224-wide tiles, the 256-wide tiles), plus a regular stride through N."""
+    cols = [np.arange(0, N, extra_step), [N - 1]]
+    for w in widths:
+        s = np.arange(0, N, w)
+        cols += [s, np.minimum(s + w - 1, N - 1)]
+    return np.unique(np.concatenate(cols)).astype(np.int64)

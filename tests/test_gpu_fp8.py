@@ -14,7 +14,7 @@ import torch
 
 import oracle
 import synth
-from gpu_util import bf16_bits, sample_rows, to_dev, to_dev_bf16
+from gpu_util import bf16_bits, sample_rows, tile_rows, to_dev, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -95,7 +95,7 @@ def test_fp8_linear_against_the_exact_sum(M, N, K):
     qd, wd = to_dev(q), to_dev(wq)
     acc = dq.dq_fp8_linear(qd, None, wd, None, out_dtype="f32").cpu().numpy().astype(np.float64)
     out = dq.dq_fp8_linear(qd, to_dev(s), wd, to_dev(sc), bias=to_dev_bf16(bias))
-    rows = sample_rows(M, 48) if M > 200 else np.arange(M)
+    rows = tile_rows(M, total=256, seed=M)
     exact = oracle.gemm_fp8_f64(q[rows], wq)
     qa = np.abs(oracle.e4m3_to_float64(q[rows]))
     wa = np.abs(oracle.e4m3_to_float64(wq))
@@ -117,9 +117,11 @@ def test_fp8_llm_shaped_layer_and_accuracy():
     q, s = dq.dq_quantize_rows_fp8(to_dev_bf16(d["x"]))
     wq, sc = dq.dq_quantize_weight_fp8(to_dev(d["w"]))
     out = dq.dq_fp8_linear(q, s, wq, sc)
-    rows = sample_rows(M, 24)
-    qo, so = oracle.quantize_rows_bf16_fp8(d["x"][rows])
-    assert np.array_equal(q.cpu().numpy()[rows], qo)
+    qo_all, so_all = oracle.quantize_rows_bf16_fp8(d["x"])
+    assert np.array_equal(q.cpu().numpy(), qo_all)            # every row's codes
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so_all.view(np.uint32))
+    rows = tile_rows(M)                         # 1024 rows, both edges of all 16 M-tiles
+    qo, so = qo_all[rows], so_all[rows]
     wo, sco = oracle.quantize_rows_f32_fp8(d["w"])
     assert np.array_equal(wq.cpu().numpy(), wo)
     exact = oracle.gemm_fp8_f64(qo, wo)

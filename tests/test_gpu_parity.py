@@ -4,7 +4,10 @@ Bit-exact for int8 codes, fp32 scales and int32 accumulators; bf16 outputs
 within 1 bf16 ulp (they are expected to be identical: both sides evaluate
 acc * s_row * s_col + bias left to right with one IEEE rounding per op).
 Sizes span several tiles with ragged tails; the five workloads run at full
-size with the oracle checked on sampled rows / channels.
+size with the oracle checked row by row on at least 1024 rows that include
+the first and last row of every 128-row M-tile (tile_rows), or, for the
+few-token workloads, on every token and the channels at both edges of every
+channel tile (tile_cols).
 """
 import numpy as np
 import pytest
@@ -12,7 +15,7 @@ import torch
 
 import oracle
 import synth
-from gpu_util import assert_bf16_close, bf16_bits, sample_rows, to_dev, to_dev_bf16
+from gpu_util import assert_bf16_close, bf16_bits, sample_rows, tile_cols, tile_rows, to_dev, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -157,22 +160,26 @@ def test_stream_k_and_whole_tiles_agree():
             dq.dq_debug_set_schedule(mode)
             outs.append(dq.dq_int8_linear(Ad, None, Wd, None, out_dtype="s32", workspace=ws).cpu().numpy())
         assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
-        rows = sample_rows(M, 24)
+        rows = tile_rows(M, total=256, seed=M)
         assert np.array_equal(outs[0][rows], oracle.gemm_s32(A[rows], W))
 
 
-# Shapes whose uniform 128 x 256 tiling leaves a partial last wave on 148 SMs,
-# so the dense schedule uses two tile widths: full waves of 256-wide tiles,
-# then one wave of narrower tiles (192 wide for 2048 x 4096; 64 wide for the
-# ragged ones, whose last narrow tile is only partly inside the matrix).
+# Shapes whose uniform tiling leaves a partial last wave, so the dense
+# schedule uses two tile widths: full waves of 256-wide tiles, then one wave of
+# narrower tiles.  1-SM kernel (schedule 1, 128 x 256 tiles on 148 SMs): 192
+# wide for 2048 x 4096, 64 wide for the ragged ones, whose last narrow tile is
+# only partly inside the matrix.  Pair kernel (schedule 3, 256 x 256 tiles on
+# the pairs that fit, 74 on a B200): 2048 x 4096 has 128 tiles (then 74 of
+# 192 wide), 1300 x 3464 84, 2300 x 4104 153.
 TWO_WIDTH_SHAPES = [(2048, 4096, 512), (1300, 3464, 256), (2300, 4104, 384), (2048, 4096, 4096)]
 
 
+@pytest.mark.parametrize("schedule", [1, 3])
 @pytest.mark.parametrize("M,N,K", TWO_WIDTH_SHAPES)
-def test_two_width_schedule_parity(M, N, K):
+def test_two_width_schedule_parity(M, N, K, schedule):
     A, W, s_row, s_col, bias = _gemm_inputs(M, N, K, 500 + M + N)
     Ad, Wd = to_dev(A), to_dev(W)
-    dq.dq_debug_set_schedule(1)
+    dq.dq_debug_set_schedule(schedule)
     outs = {}
     try:
         for on in (1, 0):
@@ -184,7 +191,7 @@ def test_two_width_schedule_parity(M, N, K):
     # identical bits with and without the narrow second wave
     assert torch.equal(outs[1][0], outs[0][0])
     assert torch.equal(outs[1][1].view(torch.int16), outs[0][1].view(torch.int16))
-    rows = np.unique(np.concatenate([sample_rows(M, 40), np.arange(max(0, M - 130), M)]))
+    rows = np.unique(np.concatenate([tile_rows(M, total=256, seed=M), np.arange(max(0, M - 130), M)]))
     want = oracle.gemm_s32(A[rows], W)
     assert np.array_equal(outs[1][0].cpu().numpy()[rows], want)
     assert_bf16_close(bf16_bits(outs[1][1])[rows], oracle.epilogue_bf16(want, s_row[rows], s_col, bias))
@@ -247,8 +254,11 @@ def test_config_llm_layer_2048x4096x4096():
     wo, sco = oracle.quantize_rows_f32(d["w"])
     assert np.array_equal(q.cpu().numpy(), qo) and np.array_equal(wq.cpu().numpy(), wo)
     assert np.array_equal(s.cpu().numpy(), so) and np.array_equal(sc.cpu().numpy(), sco)
-    rows = sample_rows(2048, 48)
-    want = oracle.linear_bf16(qo[rows], so[rows], wo, sco)
+    rows = tile_rows(2048)                      # 1024 rows, both edges of all 16 M-tiles
+    acc = dq.dq_int8_linear(q, None, wq, None, out_dtype="s32")
+    acc_o = oracle.gemm_s32(qo[rows], wo)
+    assert np.array_equal(acc.cpu().numpy()[rows], acc_o)
+    want = oracle.epilogue_bf16(acc_o, so[rows], sco)
     got = bf16_bits(out)
     assert_bf16_close(got[rows], want)
     # accuracy vs the unquantized fp32 product: reported, not gated (outliers)
@@ -261,7 +271,7 @@ def test_config_large_m_38400x1024x4096():
     A, B = to_dev(d["a"]), to_dev(d["b"])
     acc = dq.dq_int8_linear(A, None, B, None, out_dtype="s32")
     out = dq.dq_int8_linear(A, to_dev(d["s_row"]), B, to_dev(d["s_col"]))
-    rows = sample_rows(38400, 40)
+    rows = tile_rows(38400)                     # both edges of all 300 M-tiles + random rows: 1024
     want = oracle.gemm_s32(d["a"][rows], d["b"])
     assert np.array_equal(acc.cpu().numpy()[rows], want)
     assert_bf16_close(bf16_bits(out)[rows], oracle.epilogue_bf16(want, d["s_row"][rows], d["s_col"]))
@@ -278,7 +288,7 @@ def test_config_small_m(M):
     qo, so = oracle.quantize_rows_bf16(d["x"])
     assert np.array_equal(q.cpu().numpy(), qo)
     wq_np = wq.cpu().numpy()
-    ch = np.unique(np.concatenate([np.arange(0, 28672, 97), [0, 127, 128, 28543, 28671]]))
+    ch = tile_cols(28672)          # both edges of every 128-, 224- and 256-channel tile
     wo, sco = oracle.quantize_rows_f32(d["w"][ch])
     assert np.array_equal(wq_np[ch], wo)
     want = oracle.linear_bf16(qo, so, wo, sco)
@@ -316,7 +326,7 @@ def test_config_vit_h_bsr(layer, keep):
     qo_all, so_all = oracle.quantize_rows_bf16(d["x"])
     assert np.array_equal(q.cpu().numpy(), qo_all)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), so_all.view(np.uint32))
-    rows = sample_rows(M, 48)
+    rows = tile_rows(M)                         # both edges of all 514 M-tiles: 1028 rows
     qo, so = qo_all[rows], so_all[rows]
     acc_o = oracle.bsr_gemm_s32(qo, N, d["crow"], d["col"], vo)
     assert np.array_equal(acc.cpu().numpy()[rows], acc_o)
@@ -516,7 +526,7 @@ def test_dense_tile_widths(M, N, K, schedule, tile_n):
     try:
         Ad, Wd = to_dev(A), to_dev(W)
         acc = dq.dq_int8_linear(Ad, None, Wd, None, out_dtype="s32")
-        rows = sample_rows(M, 64)
+        rows = tile_rows(M, total=256, seed=M)
         want = oracle.gemm_s32(A[rows], W)
         assert np.array_equal(acc.cpu().numpy()[rows], want)
         out = dq.dq_int8_linear(Ad, to_dev(s_row), Wd, to_dev(s_col), bias=to_dev_bf16(bias))

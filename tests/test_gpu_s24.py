@@ -8,7 +8,7 @@ import torch
 
 import oracle
 import synth
-from gpu_util import assert_bf16_close, bf16_bits, sample_rows, to_dev, to_dev_bf16
+from gpu_util import assert_bf16_close, bf16_bits, tile_rows, to_dev, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -79,9 +79,10 @@ def test_linear_matches_oracle(M, N, K, use_ws):
 
 
 @pytest.mark.parametrize("M,K,N", [(2048, 4096, 4096), (16, 8192, 28672)])
-def test_layer_full_size_sampled(M, K, N):
+def test_layer_full_size(M, K, N):
     """The benchmark shapes: quantize (GPU), compress (GPU), sparse product;
-    oracle on sampled tokens."""
+    the oracle on every token (M = 16) or on 1024 tokens covering both edges
+    of every 128-row tile (M = 2048)."""
     d = synth.s24(0, M=M, K=K, N=N)
     x = to_dev_bf16(d["x"])
     q, s = dq.dq_quantize_rows(x)
@@ -91,7 +92,8 @@ def test_layer_full_size_sampled(M, K, N):
     qo, so = oracle.quantize_rows_bf16(d["x"])
     wo, sco = oracle.quantize_rows_f32(d["w"])
     assert np.array_equal(wq.cpu().numpy(), wo)
-    rows = sample_rows(M, 12)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    rows = tile_rows(M)                         # every token for M = 16; 1024 rows (all M-tile edges) for 2048
     want = oracle.linear_bf16(qo[rows], so[rows], wo, sco)
     assert_bf16_close(bf16_bits(out)[rows], want)
 

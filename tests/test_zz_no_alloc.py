@@ -41,16 +41,18 @@ def _call_noalloc(lib, A, s_row, W, s_col, bias, out, code):
                                       stream)
 
 
-# (M, N, K): few-token shapes whose (swap-AB) stream-K schedule uses 0.5 MB
-# and 8.4 MB of scratch
-@pytest.mark.parametrize("M,N,K", [(16, 8192, 8192), (128, 16384, 8192)])
-def test_noalloc_matches_workspace_entry_two_calls(M, N, K):
+# (M, N, K, uses the scratch): few-token shapes whose (swap-AB) stream-K
+# schedule uses 0.5 MB and 8.4 MB of scratch, and one whose schedule needs
+# none (the call goes straight to the plain entry point)
+@pytest.mark.parametrize("M,N,K,uses", [(16, 8192, 8192, True), (128, 16384, 8192, True), (256, 256, 256, False)])
+def test_noalloc_matches_workspace_entry_two_calls(M, N, K, uses):
     import quantized_gemm_token_b200 as dq
     from gpu_util import assert_bf16_close, bf16_bits
     lib = dq.lib
     need = dq.dq_int8_linear_workspace_size(M, N, K)
-    assert 0 < need <= dq.DQ_NOALLOC_SCRATCH_BYTES      # these shapes do use the scratch
-    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    assert need <= dq.DQ_NOALLOC_SCRATCH_BYTES
+    assert (need > 0) == uses
+    ws = torch.zeros(max(need, 16), dtype=torch.uint8, device="cuda")
     for call, seed in enumerate((900, 950)):             # two calls in a row, different data
         A, W, s_row, s_col, bias = _inputs(M, N, K, seed)
         ref32 = dq.dq_int8_linear(A, None, W, None, out_dtype="s32", workspace=ws)
@@ -80,3 +82,47 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
         assert _call_noalloc(dq.lib, A, s_row, W, s_col, None, out, dq.DQ_OUT_BF16) == dq.DQ_ERR_UNSUPPORTED
     finally:
         dq.dq_debug_set_schedule(0)
+
+
+def test_noalloc_rejects_what_the_plain_entry_rejects():
+    """Arguments the plain entry point refuses (K not a multiple of 16, a bad
+    output type, negative M) get the same status, before any launch."""
+    import quantized_gemm_token_b200 as dq
+    lib = dq.lib
+    P = ctypes.c_void_p
+    M, N, K = 16, 8192, 8200                      # K % 16 != 0
+    A, W, s_row, s_col, _ = _inputs(M, N, 8192, 991)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    stream = P(torch.cuda.current_stream().cuda_stream)
+    ptr = lambda t: P(t.data_ptr())  # noqa: E731
+    for (m, k, code) in ((M, K, dq.DQ_OUT_BF16), (M, 8192, 7), (-1, 8192, dq.DQ_OUT_BF16)):
+        args = (ptr(A), ptr(s_row), ctypes.c_int64(m), ctypes.c_int64(k), ptr(W), ptr(s_col), ctypes.c_int64(N),
+                None, ptr(out), ctypes.c_int(code))
+        plain = lib.dq_int8_linear(*args, None, ctypes.c_size_t(0), stream)
+        assert plain != dq.DQ_OK
+        assert lib.dq_int8_linear_noalloc(*args, stream) == plain
+    assert dq.dq_sync_status() == dq.DQ_OK
+
+
+def test_noalloc_python_wrapper_checks_and_matches():
+    """The binding's dq_int8_linear_noalloc checks its tensors like
+    dq_int8_linear (a wrong output type or shape raises, nothing launches)
+    and returns the same result, twice in a row."""
+    import quantized_gemm_token_b200 as dq
+    from gpu_util import assert_bf16_close, bf16_bits
+    M, N, K = 16, 8192, 8192
+    A, W, s_row, s_col, bias = _inputs(M, N, K, 993)
+    with pytest.raises(TypeError):
+        dq.dq_int8_linear_noalloc(A, s_row, W, s_col, torch.empty((M, N), dtype=torch.int32, device="cuda"))
+    with pytest.raises(ValueError):
+        dq.dq_int8_linear_noalloc(A, s_row, W, s_col, torch.empty((M, N - 8), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        dq.dq_int8_linear_noalloc(A, s_row, W[:, :K - 16].contiguous(), s_col,
+                                  torch.empty((M, N), dtype=torch.bfloat16, device="cuda"))
+    ws = torch.zeros(dq.dq_int8_linear_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
+    ref = dq.dq_int8_linear(A, s_row, W, s_col, bias=bias, workspace=ws)
+    for _ in range(2):
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        dq.dq_int8_linear_noalloc(A, s_row, W, s_col, out, bias=bias)
+        assert_bf16_close(bf16_bits(out), bf16_bits(ref))
+    assert dq.dq_sync_status() == dq.DQ_OK
