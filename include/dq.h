@@ -378,15 +378,19 @@ DQ_API dq_status dq_hqq_linear_t(const void* y_bf16, int64_t M, const uint8_t* p
  * dq_s24_int8_linear: out = the int8 layer of dq_int8_linear with the weight
  *   given compressed: acc[m, n] = sum_k A[m, k] * W[n, k] (exact int32, W the
  *   decompressed weight), then DQ_OUT_BF16: bf16((acc * s_row[m]) * s_col[n]
- *   + bias[n]) or DQ_OUT_S32: acc.  A int8 [M, K] contiguous.  The kernel
- *   expands the compressed weight in shared memory and multiplies on the
- *   tensor cores (tcgen05.mma kind::i8); the weight crosses HBM compressed
- *   (5/8 of its dense int8 bytes).  meta nibbles must have p0 < p1 (as
- *   dq_s24_compress writes them); other nibbles give unspecified (but
- *   in-bounds) results.  Requirements: K % 128 == 0, N % 8 == 0, M >= 0,
- *   pointers 16-byte aligned.  workspace / workspace_bytes: as for
- *   dq_hqq_linear (dq_s24_workspace_size; one zero-filled workspace per
- *   shape; int32 partials, so results never depend on the split).
+ *   + bias[n]) or DQ_OUT_S32: acc.  A int8 [M, K] contiguous.  The product
+ *   runs on the sparse tensor-core MMA (tcgen05.mma.sp kind::i8): the
+ *   compressed values are its A operand as they are and the metadata, copied
+ *   into tensor memory, its sparsity selectors, so only the kept half of the
+ *   weight is multiplied; the weight crosses HBM compressed (5/8 of its dense
+ *   int8 bytes).  meta nibbles must have p0 < p1 (as dq_s24_compress writes
+ *   them); other nibbles give unspecified (but in-bounds) results.
+ *   Requirements: K % 128 == 0, N % 8 == 0, M >= 0, pointers 16-byte
+ *   aligned.  workspace / workspace_bytes: as for dq_hqq_linear
+ *   (dq_s24_workspace_size; its first bytes are the split arrival counters,
+ *   eight per tile, which every completed call leaves zero; one zero-filled
+ *   workspace per shape; int32 partials, so results never depend on the
+ *   split).
  * ------------------------------------------------------------------------ */
 DQ_API dq_status dq_s24_compress(const int8_t* wq, int64_t N, int64_t K, int8_t* values, uint8_t* meta,
                                  int32_t* violations, dq_stream_t stream);

@@ -60,7 +60,7 @@ struct Cfg {
   // swizzle); 32x32 and 16x16 blocks 32 (32-byte swizzle; a 16-wide block
   // uses the 32-byte A slice that contains it, the other half of the MMA's K
   // multiplying zeros, see the Bsr16 B descriptor).
-  static constexpr int KB = !BSR ? 128 : BS == 64 ? 64 : 32;
+  static constexpr int KB = !BSR ? kDenseKB : BS == 64 ? 64 : 32;
   // BSR panel variant: the 128 x K activation panel of the current 128-row
   // block stays in shared memory (K <= KP, chunks of 128 x 128 bytes with the
   // 128-byte swizzle) and the stages carry weight blocks only.
@@ -97,11 +97,11 @@ struct Cfg {
   // column lies outside the matrix (it contributes zeros, as a load from
   // outside the matrix does in the streaming variant).
   static constexpr int ZB_BYTES = PANEL ? (B_BYTES > 256 ? B_BYTES : 256) : 0;
-  static constexpr int STAGE_CAP = BSR && (BS < 64 || PANEL) ? 24 : 12;
+  static constexpr int STAGE_CAP = (BSR && (BS < 64 || PANEL)) || (!BSR && KB < 128) ? 24 : 12;
   static constexpr int ACC_RAW = 512 / BN;
   static constexpr int ACC_BUFS = ACC_RAW > 8 ? 8 : ACC_RAW;
   // mbarriers, the TMEM address, flags and (panel variant) stage columns
-  static constexpr int BAR_BYTES = BSR ? 1024 : 512;
+  static constexpr int BAR_BYTES = BSR || STAGE_CAP > 12 ? 1024 : 512;
   // Shared-memory layout for a given stage count and number of column-scale
   // slots (offsets from the 1024-aligned base; the last 1024 bytes are the
   // slack of aligning the dynamic shared-memory base).
@@ -798,7 +798,7 @@ bool pair_preferred(int64_t /*M*/, int64_t /*N*/, int64_t K) { return K >= kPair
 // that fit at once (the pair kernel's wave size), used only for the pair.
 Plan make_plan(int64_t M, int64_t N, int64_t K, int sm_count, int pair_slots_n, const Knobs& kn) {
   Plan p{};
-  p.kb_total = static_cast<int>((K + 127) / 128);
+  p.kb_total = static_cast<int>((K + kDenseKB - 1) / kDenseKB);
   if (kn.schedule == 3 || (kn.schedule == 0 && M > 128 && pair_preferred(M, N, K))) {
     p.kind = Kind::Dense;
     p.pair = true;
@@ -901,10 +901,10 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   if (p.pair) {
     // Each 256-row tile's MMAs run on a pair of SMs (gemm2sm.cu).
     CUtensorMap ta, tb, tb2, tc;
-    if ((st = make_tmap_u8_2d(&ta, A, K, M, K, 128, 128, 128)) != DQ_OK) return st;
-    if ((st = make_tmap_u8_2d(&tb, W, K, N, K, 128, p.bn / 2, 128)) != DQ_OK) return st;
+    if ((st = make_tmap_u8_2d(&ta, A, K, M, K, kDenseKB, 128, kDenseKB)) != DQ_OK) return st;
+    if ((st = make_tmap_u8_2d(&tb, W, K, N, K, kDenseKB, p.bn / 2, kDenseKB)) != DQ_OK) return st;
     if (p.bn2 > 0) {
-      if ((st = make_tmap_u8_2d(&tb2, W, K, N, K, 128, p.bn2 / 2, 128)) != DQ_OK) return st;
+      if ((st = make_tmap_u8_2d(&tb2, W, K, N, K, kDenseKB, p.bn2 / 2, kDenseKB)) != DQ_OK) return st;
     } else {
       tb2 = tb;
     }
@@ -940,10 +940,10 @@ dq_status dq_int8_linear(const int8_t* A, const float* s_row, int64_t M, int64_t
   const int8_t* b_src = p.kind == Kind::Swap ? A : W;
   const int64_t a_rows = p.kind == Kind::Swap ? N : M;
   const int64_t b_rows = p.kind == Kind::Swap ? M : N;
-  if ((st = make_tmap_u8_2d(&ta, a_src, K, a_rows, K, 128, 128, 128)) != DQ_OK) return st;
-  if ((st = make_tmap_u8_2d(&tb, b_src, K, b_rows, K, 128, p.bn, 128)) != DQ_OK) return st;
+  if ((st = make_tmap_u8_2d(&ta, a_src, K, a_rows, K, kDenseKB, 128, kDenseKB)) != DQ_OK) return st;
+  if ((st = make_tmap_u8_2d(&tb, b_src, K, b_rows, K, kDenseKB, p.bn, kDenseKB)) != DQ_OK) return st;
   if (p.bn2 > 0) {
-    if ((st = make_tmap_u8_2d(&tb2, b_src, K, b_rows, K, 128, p.bn2, 128)) != DQ_OK) return st;
+    if ((st = make_tmap_u8_2d(&tb2, b_src, K, b_rows, K, kDenseKB, p.bn2, kDenseKB)) != DQ_OK) return st;
   } else {
     tb2 = tb;
   }
@@ -1023,14 +1023,14 @@ dq_status dq_fp8_linear(const uint8_t* A, const float* s_row, int64_t M, int64_t
   p.bn = N <= 128 ? 128 : 256;
   p.a_tiles = static_cast<int>((M + 127) / 128);
   p.b_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
-  p.kb_total = static_cast<int>((K + 127) / 128);
+  p.kb_total = static_cast<int>((K + kDenseKB - 1) / kDenseKB);
   p.num_tiles = p.a_tiles * p.b_tiles;
   if (p.bn == 256 && knobs().two_widths) plan_two_widths(p, N, d->sm_count);
   CUtensorMap ta, tb, tb2, tc;
-  if ((st = make_tmap_u8_2d(&ta, A, K, M, K, 128, 128, 128)) != DQ_OK) return st;
-  if ((st = make_tmap_u8_2d(&tb, W, K, N, K, 128, p.bn, 128)) != DQ_OK) return st;
+  if ((st = make_tmap_u8_2d(&ta, A, K, M, K, kDenseKB, 128, kDenseKB)) != DQ_OK) return st;
+  if ((st = make_tmap_u8_2d(&tb, W, K, N, K, kDenseKB, p.bn, kDenseKB)) != DQ_OK) return st;
   if (p.bn2 > 0) {
-    if ((st = make_tmap_u8_2d(&tb2, W, K, N, K, 128, p.bn2, 128)) != DQ_OK) return st;
+    if ((st = make_tmap_u8_2d(&tb2, W, K, N, K, kDenseKB, p.bn2, kDenseKB)) != DQ_OK) return st;
   } else {
     tb2 = tb;
   }

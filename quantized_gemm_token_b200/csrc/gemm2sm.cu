@@ -40,14 +40,14 @@ namespace dq {
 // BN: pair tile width (output columns); each CTA holds BN/2 rows of B.
 template <int BN>
 struct Cfg2 {
-  static constexpr int KB = 128;                        // k bytes per stage
+  static constexpr int KB = kDenseKB;                   // k bytes per stage
   static constexpr int A_BYTES = 128 * KB;              // this CTA's 128 rows of A
   static constexpr int B_BYTES = (BN / 2) * KB;         // this CTA's half of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int EPI_WARPS = 8;
   static constexpr int OUT_BUF_BYTES = 32 * 32 * 4;     // per epilogue warp
   static constexpr int OUT_BYTES = EPI_WARPS * OUT_BUF_BYTES;
-  static constexpr int BAR_BYTES = 256;                 // mbarriers, TMEM address, abort flag
+  static constexpr int BAR_BYTES = 512;                 // mbarriers, TMEM address, abort flag
   static constexpr int ALIGN_SLACK = 1024;              // the 1024-byte alignment of the base
   static constexpr int STAGES = (227 * 1024 - ALIGN_SLACK - BAR_BYTES - OUT_BYTES - kScSlotBytes) / STAGE_BYTES;
   static constexpr int ACC_BUFS = 512 / BN >= 3 ? 3 : 2;  // accumulators of BN TMEM columns

@@ -12,6 +12,11 @@ namespace dq {
 
 enum class Kind : int { Dense = 0, Swap = 1, Bsr = 2, Bsr32 = 3, Bsr16 = 4, DenseF8 = 5 };
 
+// Contraction bytes per pipeline stage of the dense arrangements (1-SM and
+// pair kernels): the K-major operand tiles are kDenseKB bytes wide, with the
+// swizzle of that width.
+constexpr int kDenseKB = 128;
+
 // Dense arrangement with int8 (Dense) or e4m3 (DenseF8) operands; e4m3
 // products accumulate in fp32 (kind::f8f6f4), int8 ones in int32.
 __host__ __device__ constexpr bool is_dense_kind(Kind k) { return k == Kind::Dense || k == Kind::DenseF8; }

@@ -193,6 +193,10 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict
                                                              int tpr_log2) {
   constexpr int E = Elem<T>::kPerVec;
   griddep_launch_dependents();     // the next kernel (e.g. the GEMM) may start its prologue
+  // Launched with programmatic stream serialization: the previous kernel of
+  // the stream (which may still read q or scales, or write x) is complete and
+  // its writes visible before this kernel touches global memory.
+  griddep_wait();
   const int tpr = 1 << tpr_log2;
   const int t = threadIdx.x & (tpr - 1);
   const int r_local = threadIdx.x >> tpr_log2;
@@ -554,15 +558,28 @@ dq_status launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t*
     const int64_t rows_per_cta = 256 / tpr;
     const int64_t grid = (M + rows_per_cta - 1) / rows_per_cta;
     if (grid > 0x7fffffff) return DQ_ERR_UNSUPPORTED;
-    dim3 g(static_cast<unsigned>(grid));
+    // Programmatic stream serialization: the launch and the CTAs' start
+    // overlap the tail of the previous kernel; the kernel waits for it
+    // (griddepcontrol.wait) before its first global memory access.
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t le;
     if (vpt <= 1)
-      quant_rows_vec_kernel<T, 1, F><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+      le = cudaLaunchKernelEx(&cfg, quant_rows_vec_kernel<T, 1, F>, x, M, K, ldx, q, ldq, scales, tpr_log2);
     else if (vpt <= 2)
-      quant_rows_vec_kernel<T, 2, F><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+      le = cudaLaunchKernelEx(&cfg, quant_rows_vec_kernel<T, 2, F>, x, M, K, ldx, q, ldq, scales, tpr_log2);
     else if (vpt <= 4)
-      quant_rows_vec_kernel<T, 4, F><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+      le = cudaLaunchKernelEx(&cfg, quant_rows_vec_kernel<T, 4, F>, x, M, K, ldx, q, ldq, scales, tpr_log2);
     else
-      quant_rows_vec_kernel<T, 8, F><<<g, 256, 0, stream>>>(x, M, K, ldx, q, ldq, scales, tpr_log2);
+      le = cudaLaunchKernelEx(&cfg, quant_rows_vec_kernel<T, 8, F>, x, M, K, ldx, q, ldq, scales, tpr_log2);
+    if (le != cudaSuccess) return cuda_fail(le);
   } else {
     const int64_t grid = M < int64_t(d->sm_count) * 16 ? M : int64_t(d->sm_count) * 16;
     quant_rows_generic_kernel<T, F><<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, M, K, ldx, q,

@@ -4,33 +4,35 @@
 // four consecutive in-features run a 2:4 sparse matmul after the weight is
 // compressed on the device; its review asks for the int8 product with only
 // the dequantization fused and a 16-bit output, which the library it used
-// could not do).  Here the product runs with the dequantization, bias and
-// bf16 conversion fused, and no int32 matrix in global memory.
+// could not do).  Here the product runs on the sparse tensor-core MMA with
+// the dequantization, bias and bf16 conversion fused, and no int32 matrix in
+// global memory.
 //
 // Compressed weight (this library's own format, written by dq_s24_compress):
 //   values [N, K/2] int8: the two kept values of each group of four, in
 //     position order;
 //   meta [N, K/8] uint8: one nibble per group, p0 | p1 << 2 (p0 < p1 the
 //     kept positions), group 2b in the low nibble of byte b.
+// This is the operand format of tcgen05.mma.sp with 8-bit operands: the
+// values are the compressed A matrix as it is, and a 128-channel x 128
+// in-feature block of the metadata (128 rows of 16 bytes) is one copy into
+// tensor memory that serves two K = 64 MMAs (8 bytes per row each).
 //
-// One persistent, warp-specialised kernel for sm_100a (448 threads):
-//   warp 0       TMA producer: per 128-deep contraction step the quantized
-//                activation tile (bn tokens x 128 B, 128B-swizzled), the
-//                step's compressed values (128 channel rows x 64 B,
-//                64B-swizzled) and metadata (128 x 16 B).
-//   warps 2..9   expanders: each group's two values go back to their
-//                positions (one byte permute per group, zeros elsewhere),
-//                written as the 128 x 128 B int8 A tile in the tensor
-//                core's 128B-swizzled K-major layout.  The weight crosses HBM
-//                compressed: 5/8 of the dense int8 bytes.
-//   warp 1       MMA issuer: tcgen05.mma kind::i8 (M = 128 weight rows, N =
-//                bn tokens, int32 accumulator in TMEM, double-buffered).
-//   warps 10..13 epilogue: out = bf16((acc * s_row) * s_col + bias), each op
-//                rounded on its own, or the raw int32; two neighbouring
-//                channels per store.
+// One persistent, warp-specialised kernel for sm_100a (320 threads):
+//   warp 0      TMA producer: per 128-deep contraction step the quantized
+//               activation tile (bn tokens x 128 B, 128B-swizzled), the
+//               step's compressed values (128 channel rows x 64 B,
+//               64B-swizzled) and metadata (128 x 16 B, unswizzled).
+//   warp 1      MMA issuer: tcgen05.cp of the step's metadata into a tensor
+//               memory slot of the stage, then two tcgen05.mma.sp kind::i8
+//               (M = 128 weight rows, N = bn tokens, logical K = 64 each,
+//               int32 accumulator in TMEM, double-buffered).
+//   warps 2..9  epilogue, two warps per TMEM sub-partition taking alternate
+//               32-token chunks: out = bf16((acc * s_row) * s_col + bias),
+//               each op rounded on its own, or the raw int32.
 // Few tiles: the contraction is split; int32 partial tiles go to a
-// workspace and the last split of a tile to arrive adds them (exact) with
-// the whole CTA before the epilogue arithmetic.
+// workspace and, per epilogue warp, the last split of a tile to arrive adds
+// them (exact, in split order) before the epilogue arithmetic.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -42,22 +44,24 @@
 namespace dq {
 namespace {
 
-constexpr int S4_THREADS = 448;
-constexpr int S4_EXP_WARPS = 8;            // warps 2..9
-constexpr int S4_EPI_WARP0 = 10;           // warps 10..13
-constexpr int S4_BK = 128;                 // in-features per step (128 B of int8)
-constexpr int S4_A_BYTES = 128 * 128;      // expanded weight tile
+constexpr int S4_THREADS = 320;
+constexpr int S4_EPI_WARPS = 8;            // warps 2..9
+constexpr int S4_BK = 128;                 // logical in-features per step (two sparse MMAs)
 constexpr int S4_V_BYTES = 128 * 64;       // compressed values per step
 constexpr int S4_M_BYTES = 128 * 16;       // metadata per step
 constexpr int S4_MAX_NP = 16;
-constexpr int S4_ACC_COLS = 256;
+constexpr int S4_MAX_BN = 224;             // tokens per tile
+constexpr int S4_ACC_COLS = 224;           // TMEM columns per accumulator buffer
+constexpr int S4_META_COL = 2 * S4_ACC_COLS;   // metadata ring: 4 TMEM columns per stage
 constexpr int S4_TMEM_COLS = 512;
 constexpr int S4_SMEM_LIMIT = 227 * 1024;
 constexpr int S4_BAR_BYTES = 1024;
+constexpr int S4_CNT_PER_TILE = 8;         // split arrival counters per tile: one per epilogue warp
+static_assert(S4_META_COL + 4 * S4_MAX_NP <= S4_TMEM_COLS, "tensor memory");
 
 struct S24Args {
   int M, N, K;
-  int bn;                 // tokens per tile (multiple of 16, <= 256)
+  int bn;                 // tokens per tile (multiple of 16, <= S4_MAX_BN)
   int nt, tt;             // channel tiles (128), token tiles (bn)
   int splits, ks, units, np;
   uint32_t off_bar;
@@ -67,7 +71,7 @@ struct S24Args {
   void* out;              // bf16 or int32 [M, N]
   int out_s32;
   int32_t* ws;            // split partials [tile][split][bn][128] int32
-  uint32_t* cnt;          // arrival counter per tile (slot tile * 4)
+  uint32_t* cnt;          // split arrival counters [tile][S4_CNT_PER_TILE]
   WaitCtl wait;
 };
 
@@ -86,39 +90,31 @@ __device__ __forceinline__ Unit decode_unit(const S24Args& g, int u) {
   return t;
 }
 
-// Four dense bytes of one group: the kept values (bytes 0, 1 of `vword` for
-// an even group, bytes 2, 3 for an odd one) at positions p0, p1, zeros
-// elsewhere.  Selector nibble 4 picks a byte of the zero operand.
-__device__ __forceinline__ uint32_t expand_group(uint32_t vword, uint32_t nib, bool odd) {
-  const uint32_t p0x4 = (nib << 2) & 0xCu;   // 4 * p0
-  const uint32_t p1x4 = nib & 0xCu;          // 4 * p1
-  const uint32_t sel = 0x4444u ^ ((odd ? 6u : 4u) << p0x4) ^ ((odd ? 7u : 5u) << p1x4);
-  return __byte_perm(vword, 0u, sel);
+// Instruction descriptor of the sparse kind::i8 MMA: the dense descriptor
+// (signed A and B, int32 accumulator, both K-major) with the sparsity flag.
+__host__ __device__ constexpr uint32_t idesc_i8_sparse(int M, int N) { return idesc_i8(M, N) | (1u << 2); }
+
+// D[tmem] (+)= A * B^T with A 2:4-compressed (128 rows x 32 B per MMA, K = 64
+// logical), its metadata at tensor-memory address `meta`; issued by one thread.
+__device__ __forceinline__ void mma_i8_sparse(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t meta,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(meta), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
-// 256 threads expand a step's 128 rows x 128 in-features: thread t takes row
-// t % 128 and in-features 64 * (t / 128) .. +63 (16 groups: 32 value bytes,
-// 8 metadata bytes).  The values tile is 64B-swizzled (16-byte chunk c of
-// row r at chunk c ^ ((r / 2) % 4)).
-__device__ __forceinline__ void expand_tile(uint32_t atile, uint32_t vtile, uint32_t mtile, int dt) {
-  const int r = dt & 127;
-  const int h = dt >> 7;
-  const int sw = (r >> 1) & 3;
-  const uint4 va = pipe::lds128(vtile + r * 64 + (((2 * h) ^ sw) << 4));
-  const uint4 vb = pipe::lds128(vtile + r * 64 + (((2 * h + 1) ^ sw) << 4));
-  const uint2 mw = pipe::lds64(mtile + r * 16 + 8 * h);
-  const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int gi = 4 * i + j;                               // group 0..15 of this thread
-      const uint32_t nib = ((gi < 8 ? mw.x : mw.y) >> (4 * (gi & 7))) & 0xFu;
-      o[j] = expand_group(vw[gi >> 1], nib, gi & 1);
-    }
-    pipe::sts128(atile + pipe::sw128_off(r, 4 * h + i), o[0], o[1], o[2], o[3]);
-  }
+// Asynchronous copy of a 128-row x 16-byte shared-memory matrix (unswizzled:
+// 8-row x 16-byte core matrices, 128 bytes apart) into 128 lanes x 4 columns
+// of tensor memory; ordered before the MMAs this thread issues after it.
+__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint32_t smem_addr) {
+  const uint64_t desc = (static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4))   // start address
+                        | (static_cast<uint64_t>(128u >> 4) << 16)              // leading byte offset
+                        | (static_cast<uint64_t>(128u >> 4) << 32)              // stride: 8-row groups
+                        | (1ull << 46);                                         // version; no swizzle
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
 __device__ __forceinline__ uint32_t bf16_bits(float f) {
@@ -165,6 +161,20 @@ __device__ __forceinline__ void store_chunk(const S24Args& g, const uint32_t (&r
   }
 }
 
+// Reads a chunk's accumulators (width 32, or 16 for a 16-token tail) from TMEM.
+__device__ __forceinline__ void load_chunk(uint32_t taddr, int width, uint32_t (&r)[32]) {
+  if (width == 32) {
+    tmem_ld_32x32b_x32(taddr, r);
+  } else {
+    uint32_t r16[16];
+    tmem_ld_32x32b_x16(taddr, r16);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) r[j] = r16[j];
+#pragma unroll
+    for (int j = 16; j < 32; ++j) r[j] = 0;
+  }
+}
+
 __global__ void __launch_bounds__(S4_THREADS, 1)
     s24_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_m, const S24Args g) {
@@ -172,33 +182,29 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* const smem = smem_raw + (base - raw);
-  // stage s at base + s * stage_bytes: expanded A tile, activation tile,
-  // compressed values, metadata
+  // stage s at base + s * stage_bytes: activation tile (bn x 128 B), compressed
+  // values (128 x 64 B), metadata (128 x 16 B); every part 1024-byte aligned
   const uint32_t q_bytes = static_cast<uint32_t>(g.bn) * 128u;
-  const uint32_t stage_bytes = S4_A_BYTES + q_bytes + S4_V_BYTES + S4_M_BYTES;
+  const uint32_t stage_bytes = q_bytes + S4_V_BYTES + S4_M_BYTES;
   uint64_t* const full = reinterpret_cast<uint64_t*>(smem + g.off_bar);
-  uint64_t* const expd = full + S4_MAX_NP;
-  uint64_t* const empty = expd + S4_MAX_NP;
+  uint64_t* const empty = full + S4_MAX_NP;
   uint64_t* const accf = empty + S4_MAX_NP;
   uint64_t* const acce = accf + 2;
   uint64_t* const drain = acce + 2;
   uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* const last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    *last_flag = 0;
     for (int i = 0; i < g.np; ++i) {
       mbar_init(smem_u32(full + i), 1);
-      mbar_init(smem_u32(expd + i), S4_EXP_WARPS);
       mbar_init(smem_u32(empty + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(accf + i), 1);
-      mbar_init(smem_u32(acce + i), 4);
+      mbar_init(smem_u32(acce + i), S4_EPI_WARPS);
     }
     mbar_init(smem_u32(drain), 1);
     fence_barrier_init();
@@ -214,6 +220,9 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // With a programmatic (early) launch, the kernel that produced A is done
+  // before any global memory is touched.
+  griddep_wait();
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
@@ -230,7 +239,7 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
             break;
           }
           const uint32_t fb = smem_u32(full + stage);
-          const uint32_t sq = base + stage * stage_bytes + S4_A_BYTES;
+          const uint32_t sq = base + stage * stage_bytes;
           const uint32_t sv = sq + q_bytes;
           mbar_arrive_expect_tx(fb, q_bytes + S4_V_BYTES + S4_M_BYTES);
           tma_load_2d(sq, &tm_q, fb, kk * S4_BK, t.ttile * g.bn);
@@ -252,7 +261,7 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_i8(128, g.bn);
+      const uint32_t idesc = idesc_i8_sparse(128, g.bn);
       int stage = 0, acc = 0;
       uint32_t phase = 0, aphase = 0;
       bool ok = true;
@@ -262,18 +271,22 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * S4_ACC_COLS);
         for (int kk = t.k0; kk < t.k1; ++kk) {
-          if (!pipe::wait(smem_u32(expd + stage), phase, g.wait, abort_flag) ||
-              !pipe::wait(smem_u32(full + stage), phase, g.wait, abort_flag)) {
+          if (!pipe::wait(smem_u32(full + stage), phase, g.wait, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = base + stage * stage_bytes;
-          const uint64_t ad = smem_desc_kmajor<128>(sa);
-          const uint64_t bd = smem_desc_kmajor<128>(sa + S4_A_BYTES);
+          const uint32_t sq = base + stage * stage_bytes;
+          const uint32_t sv = sq + q_bytes;
+          // the step's metadata into this stage's tensor-memory slot (the
+          // slot's previous MMAs completed before the stage was refilled)
+          const uint32_t meta = tmem_base + static_cast<uint32_t>(S4_META_COL + 4 * stage);
+          tmem_cp_128x128b(meta, sv + S4_V_BYTES);
+          const uint64_t ad = smem_desc_kmajor<64>(sv);
+          const uint64_t bd = smem_desc_kmajor<128>(sq);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)   // K = 32 int8 = 32 bytes per instruction
-            mma_i8(d_tmem, ad + 2 * j, bd + 2 * j, idesc, (kk > t.k0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < 2; ++j)   // logical K = 64 per MMA: 32 compressed bytes, 64 activation bytes
+            mma_i8_sparse(d_tmem, ad + 2 * j, bd + 4 * j, meta + 2 * j, idesc, (kk > t.k0 || j > 0) ? 1u : 0u);
           mma_commit(smem_u32(empty + stage));
           if (++stage == g.np) {
             stage = 0;
@@ -291,37 +304,13 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
       volatile int never = 0;
       pipe::wait(smem_u32(drain), 0, g.wait, &never);
     }
-  } else if (warp < S4_EPI_WARP0) {
-    // ---------------------------------------------------------- expanders
-    // The stage's A tile is free once its copies have landed: the producer
-    // refilled the stage only after the MMAs that read it completed.
-    const int dt = threadIdx.x - 64;
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
-      const Unit t = decode_unit(g, u);
-      for (int kk = t.k0; kk < t.k1; ++kk) {
-        const bool w = pipe::wait(smem_u32(full + stage), phase, g.wait, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
-        const uint32_t sa = base + stage * stage_bytes;
-        const uint32_t sv = sa + S4_A_BYTES + q_bytes;
-        expand_tile(sa, sv, sv + S4_V_BYTES, dt);
-        fence_proxy_async_smem();     // generic-proxy writes -> visible to the MMA
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(expd + stage));
-        if (++stage == g.np) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-    }
   } else {
     // ---------------------------------------------------------- epilogue
+    // warp w reads TMEM sub-partition w % 4 (channels 32 (w % 4) .. + 31) and
+    // takes every other 32-token chunk (grp = 0 or 1)
+    const int ew = warp - 2;
     const int q = warp & 3;
+    const int grp = ew >> 2;
     const int row = q * 32 + lane;
     int acc = 0;
     uint32_t aphase = 0;
@@ -333,38 +322,72 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S4_ACC_COLS);
       const int ch = t.ntile * 128 + row;
       const int tok0 = t.ttile * g.bn;
-      int32_t* const part =
-          g.splits > 1 ? g.ws + static_cast<int64_t>(t.tile * g.splits + t.split) * g.bn * 128 : nullptr;
-      for (int c0 = 0; c0 < g.bn; c0 += 32) {
-        const int width = min(32, g.bn - c0);
-        uint32_t r[32];
-        if (width == 32) {
-          tmem_ld_32x32b_x32(tb + c0, r);
-        } else {
-          uint32_t r16[16];
-          tmem_ld_32x32b_x16(tb + c0, r16);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) r[j] = r16[j];
-#pragma unroll
-          for (int j = 16; j < 32; ++j) r[j] = 0;
+      const int nch = (g.bn + 31) / 32;
+      if (g.splits == 1) {
+        for (int c = grp; c < nch; c += 2) {
+          const int width = min(32, g.bn - 32 * c);
+          uint32_t r[32];
+          load_chunk(tb + 32 * c, width, r);
+          tmem_ld_wait();
+          if (c + 2 >= nch) {            // this warp's last chunk: the accumulator is free
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(acce + acc));
+          }
+          store_chunk(g, r, width, tok0 + 32 * c, ch, lane);
         }
-        tmem_ld_wait();
-        if (part != nullptr) {
+        if (grp >= nch) {                 // no chunk for this warp (bn <= 32)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(acce + acc));
+        }
+      } else {
+        // Split contraction: this warp's chunks as an int32 partial tile
+        // [token][channel], then the last of the tile's splits to arrive (per
+        // warp: its own counter) adds the partials in split order and stores.
+        int32_t* const part = g.ws + (static_cast<int64_t>(t.tile) * g.splits + t.split) * g.bn * 128;
+        for (int c = grp; c < nch; c += 2) {
+          const int width = min(32, g.bn - 32 * c);
+          uint32_t r[32];
+          load_chunk(tb + 32 * c, width, r);
+          tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j < width) part[static_cast<int64_t>(c0 + j) * 128 + row] = static_cast<int32_t>(r[j]);
-        } else {
-          store_chunk(g, r, width, tok0 + c0, ch, lane);
+            if (j < width) part[static_cast<int64_t>(32 * c + j) * 128 + row] = static_cast<int32_t>(r[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(acce + acc));
+        __threadfence();
+        __syncwarp();
+        uint32_t prev = 0;
+        if (lane == 0) prev = atomicAdd(g.cnt + t.tile * S4_CNT_PER_TILE + ew, 1u);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev == static_cast<uint32_t>(g.splits - 1)) {
+          __threadfence();
+          const int32_t* const tile_ws = g.ws + static_cast<int64_t>(t.tile) * g.splits * g.bn * 128;
+          for (int c = grp; c < nch; c += 2) {
+            const int width = min(32, g.bn - 32 * c);
+            uint32_t r[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              int32_t s = 0;
+              if (j < width) {
+                for (int sp = 0; sp < g.splits; ++sp)
+                  s += __ldcg(tile_ws + (static_cast<int64_t>(sp) * g.bn + 32 * c + j) * 128 + row);
+              }
+              r[j] = static_cast<uint32_t>(s);
+            }
+            store_chunk(g, r, width, tok0 + 32 * c, ch, lane);
+          }
+          __syncwarp();
+          if (lane == 0) g.cnt[t.tile * S4_CNT_PER_TILE + ew] = 0u;    // the counters are left zeroed
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(acce + acc));
       if (++acc == 2) {
         acc = 0;
         aphase ^= 1;
       }
-      if (part != nullptr) __threadfence();     // the partial tile is published below
     }
   }
 
@@ -372,65 +395,6 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, S4_TMEM_COLS);
-
-  // Split contraction (one unit per CTA): the last split of a tile to arrive
-  // adds the int32 partials (exact, any order) and runs the epilogue
-  // arithmetic with every thread of the CTA.
-  if (g.splits > 1 && blockIdx.x < g.units) {
-    const Unit t = decode_unit(g, blockIdx.x);
-    if (threadIdx.x == 0) {
-      int last = 0;
-      if (!*abort_flag) {
-        __threadfence();
-        last = atomicAdd(g.cnt + t.tile * 4, 1u) == static_cast<uint32_t>(g.splits - 1) ? 1 : 0;
-      }
-      *last_flag = last;
-    }
-    __syncthreads();
-    if (*last_flag) {
-      __threadfence();
-      const int32_t* const tile_ws = g.ws + static_cast<int64_t>(t.tile) * g.splits * g.bn * 128;
-      const int quad = threadIdx.x & 31;                 // channels 4 * quad .. + 3
-      const int ch = t.ntile * 128 + 4 * quad;
-      const bool ch_ok = ch < g.N;                       // N % 8 == 0: all four or none
-      float sc[4] = {0.f, 0.f, 0.f, 0.f}, bs[4] = {0.f, 0.f, 0.f, 0.f};
-      const bool has_bias = g.bias != nullptr;
-      if (ch_ok && !g.out_s32) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          sc[i] = __ldg(g.s_col + ch + i);
-          if (has_bias) bs[i] = __uint_as_float(static_cast<uint32_t>(__ldg(g.bias + ch + i)) << 16);
-        }
-      }
-      constexpr int ROWS = S4_THREADS / 32;
-      for (int tok = threadIdx.x >> 5; tok < g.bn; tok += ROWS) {
-        int4 sum = make_int4(0, 0, 0, 0);
-#pragma unroll 4
-        for (int sp = 0; sp < g.splits; ++sp) {
-          const int4 v = __ldcg(reinterpret_cast<const int4*>(tile_ws + (static_cast<int64_t>(sp) * g.bn + tok) * 128) +
-                                quad);
-          sum.x += v.x;
-          sum.y += v.y;
-          sum.z += v.z;
-          sum.w += v.w;
-        }
-        const int m = t.ttile * g.bn + tok;
-        if (!ch_ok || m >= g.M) continue;
-        if (g.out_s32) {
-          *reinterpret_cast<int4*>(static_cast<int32_t*>(g.out) + static_cast<int64_t>(m) * g.N + ch) = sum;
-        } else {
-          const float sr = __ldg(g.s_row + m);
-          const uint32_t lo = bf16_bits(dequant(sum.x, sr, sc[0], has_bias, bs[0])) |
-                              (bf16_bits(dequant(sum.y, sr, sc[1], has_bias, bs[1])) << 16);
-          const uint32_t hi = bf16_bits(dequant(sum.z, sr, sc[2], has_bias, bs[2])) |
-                              (bf16_bits(dequant(sum.w, sr, sc[3], has_bias, bs[3])) << 16);
-          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(g.out) + static_cast<int64_t>(m) * g.N + ch) =
-              make_uint2(lo, hi);
-        }
-      }
-      if (threadIdx.x == 0) g.cnt[t.tile * 4] = 0u;     // the workspace is left zeroed
-    }
-  }
 }
 
 // One thread per metadata byte (two groups): compress eight weight bytes.
@@ -480,25 +444,43 @@ struct S24Plan {
   size_t cnt_bytes, ws_bytes, smem;
 };
 
+// Token tile width and contraction split: the pair (bn, splits) whose waves
+// of units over the SMs cost the least, a unit costing its steps times
+// (bn + 32) (a fixed share per step for the weight tile and the MMA issue).
+// Splits need a workspace and at least four steps per unit.
 S24Plan plan_s24(int64_t M, int64_t N, int64_t K, int sm_count, bool allow_split) {
-  S24Plan p{};
-  p.nt = static_cast<int>((N + 127) / 128);
-  p.ks = static_cast<int>(K / S4_BK);
-  p.tt = static_cast<int>((M + 255) / 256);
-  const int64_t per = (M + p.tt - 1) / p.tt;
-  p.bn = static_cast<int>(std::max<int64_t>(16, (per + 15) / 16 * 16));
-  const int64_t tiles = static_cast<int64_t>(p.nt) * p.tt;
-  p.splits = 1;
-  if (allow_split && tiles < sm_count) {
-    int s = static_cast<int>(sm_count / tiles);
-    s = std::min(s, std::max(1, p.ks / 4));
-    p.splits = std::max(1, std::min(s, 32));
+  S24Plan best{};
+  long long best_cost = -1;
+  const int nt = static_cast<int>((N + 127) / 128);
+  const int ks = static_cast<int>(K / S4_BK);
+  for (int bn = 16; bn <= S4_MAX_BN; bn += 16) {
+    if (bn > 16 && bn - 16 >= M) break;                 // wider tiles only add empty tokens
+    const int tt = static_cast<int>((M + bn - 1) / bn);
+    const long long tiles = static_cast<long long>(nt) * tt;
+    for (int s = 1; s <= (allow_split ? 8 : 1); ++s) {
+      if (s > 1 && ks / s < 4) break;
+      const long long units = tiles * s;
+      if (units > 0x7fffffffLL) continue;
+      const long long waves = (units + sm_count - 1) / sm_count;
+      const long long steps = (ks + s - 1) / s;
+      const long long cost = waves * steps * (bn + 32) + (s > 1 ? steps : 0);
+      if (best_cost < 0 || cost < best_cost) {
+        best_cost = cost;
+        best.bn = bn;
+        best.tt = tt;
+        best.splits = s;
+      }
+    }
   }
-  p.cnt_bytes = (static_cast<size_t>(tiles) * 4 * sizeof(uint32_t) + 255) / 256 * 256;
+  S24Plan& p = best;
+  p.nt = nt;
+  p.ks = ks;
+  const long long tiles = static_cast<long long>(p.nt) * p.tt;
+  p.cnt_bytes = (static_cast<size_t>(tiles) * S4_CNT_PER_TILE * sizeof(uint32_t) + 255) / 256 * 256;
   p.ws_bytes = p.splits > 1 ? p.cnt_bytes + static_cast<size_t>(tiles) * p.splits * p.bn * 128 * sizeof(int32_t) : 0;
   p.units = static_cast<int>(tiles * p.splits);
   p.grid = std::min(p.units, sm_count);
-  const int stage = S4_A_BYTES + p.bn * 128 + S4_V_BYTES + S4_M_BYTES;
+  const int stage = p.bn * 128 + S4_V_BYTES + S4_M_BYTES;
   p.np = std::min(S4_MAX_NP, (S4_SMEM_LIMIT - 1024 - S4_BAR_BYTES) / stage);
   p.smem = 1024 + static_cast<size_t>(p.np) * stage + S4_BAR_BYTES;
   return p;
@@ -582,7 +564,7 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
   g.ks = p.ks;
   g.units = p.units;
   g.np = p.np;
-  g.off_bar = static_cast<uint32_t>(p.np) * (S4_A_BYTES + p.bn * 128 + S4_V_BYTES + S4_M_BYTES);
+  g.off_bar = static_cast<uint32_t>(p.np) * (p.bn * 128 + S4_V_BYTES + S4_M_BYTES);
   g.s_row = s_row;
   g.s_col = s_col;
   g.bias = out_dtype == DQ_OUT_BF16 ? static_cast<const uint16_t*>(bias_bf16) : nullptr;
@@ -596,8 +578,19 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
 
   const dq_status ast = smem_limit_once(reinterpret_cast<const void*>(&s24_gemm_kernel), S4_SMEM_LIMIT);
   if (ast != DQ_OK) return ast;
-  s24_gemm_kernel<<<p.grid, S4_THREADS, p.smem, reinterpret_cast<cudaStream_t>(stream)>>>(tq, tv, tm, g);
-  const cudaError_t e = cudaGetLastError();
+  // Programmatic stream serialization: the prologue may overlap the tail of
+  // the quantization that produced A; the kernel waits before global access.
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(p.grid));
+  cfg.blockDim = dim3(S4_THREADS);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, s24_gemm_kernel, tq, tv, tm, g);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 

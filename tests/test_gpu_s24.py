@@ -73,9 +73,12 @@ def test_linear_matches_oracle(M, N, K, use_ws):
                                     bias=None if b is None else to_dev_bf16(b), workspace=ws)
         assert_bf16_close(bf16_bits(out), oracle.epilogue_bf16(want, s_row, s_col, b))
     if ws is not None:
-        # the arrival counters (one 16-byte slot per tile, at the start) are zero again
-        tiles = -(-N // 128) * -(-M // 256)
-        assert int(ws[:16 * tiles].count_nonzero()) == 0
+        # every completed call leaves the split arrival counters at zero: one
+        # more call with the same workspace writes every output element (a
+        # counter left behind would keep the last split from storing)
+        out = torch.full((M, N), 0x7FFFFFFF, dtype=torch.int32, device="cuda")
+        dq.dq_s24_int8_linear(Ad, None, vd, md, None, out=out, out_dtype="s32", workspace=ws)
+        assert np.array_equal(out.cpu().numpy(), want)
 
 
 @pytest.mark.parametrize("M,K,N", [(2048, 4096, 4096), (16, 8192, 28672)])
