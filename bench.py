@@ -848,6 +848,72 @@ def secondary_measurements(dq, torch, peaks, probe, n):
         e["layer_speedup_vs_dense"] = round((ms_q + ms_d) / (ms_q + ms_b), 3)
         out[f"vit_h_{layer}_bsr10_{M}x{K}x{N}"] = e
         del wq, sc, vals, x, q, s, o
+    # LLM-shaped layer with a 2:4-sparse weight (the sparse tensor-core MMA)
+    # and with dynamic FP8, against the dense int8 GEMM of the same shape;
+    # few-token 2:4 weight stream
+    for (M, K, N, tag) in ((2048, 4096, 4096, "s24_llm_2048x4096x4096"), (16, 8192, 28672, "s24_small_m16_8192x28672")):
+        w = randn((N, K), 0.02, 17 + M)
+        # a uniform 2:4 mask: one of the six position pairs per group of four
+        pairs = torch.tensor([[1, 1, 0, 0], [1, 0, 1, 0], [1, 0, 0, 1], [0, 1, 1, 0], [0, 1, 0, 1], [0, 0, 1, 1]],
+                             dtype=torch.float32, device="cuda")
+        keep = pairs[torch.randint(0, 6, (N, K // 4), generator=gen, device="cuda")]
+        w = (w.view(N, K // 4, 4) * keep).view(N, K)
+        del keep
+        wq, sc = dq.dq_quantize_weight(w)
+        del w
+        vals, meta = dq.dq_s24_compress(wq)
+        x = randn((M, K), 1.0, 18 + M).to(torch.bfloat16)
+        q, s = dq.dq_quantize_rows(x)
+        o = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        nws = dq.dq_s24_workspace_size(M, N, K)
+        ws = torch.zeros(nws, dtype=torch.uint8, device="cuda") if nws else None
+        ms_s = _graph_ms(torch, lambda i, st: dq.dq_s24_int8_linear(q, s, vals, meta, sc, out=o, workspace=ws, stream=st), n)
+        nwd = dq.dq_int8_linear_workspace_size(M, N, K)
+        wsd = torch.zeros(nwd, dtype=torch.uint8, device="cuda") if nwd else None
+        ms_d = _graph_ms(torch, lambda i, st: dq.dq_int8_linear(q, s, wq, sc, out=o, workspace=wsd, stream=st), n)
+        if M > 128:
+            e = _tensor_entry("dq_s24_int8_linear", ms_s, 2.0 * M * N * K, peaks, probe)
+            e["ops_note"] = "dense-equivalent ops (2 M N K) of the 2:4 product"
+        else:
+            e = _hbm_entry("dq_s24_int8_linear", ms_s, N * K // 2 + N * K // 8 + M * K + 2 * M * N + 4 * (M + N), peaks)
+        e["dense_int8_ms"] = round(ms_d, 5)
+        e["speedup_vs_dense_int8"] = round(ms_d / ms_s, 3)
+        out[tag] = e
+        del wq, sc, vals, meta, x, q, s, o, ws, wsd
+    M, K, N = 2048, 4096, 4096
+    wq8, sc8 = dq.dq_quantize_weight_fp8(randn((N, K), 0.02, 19))
+    q8, s8 = dq.dq_quantize_rows_fp8(randn((M, K), 1.0, 20).to(torch.bfloat16))
+    o = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ms = _graph_ms(torch, lambda i, st: dq.dq_fp8_linear(q8, s8, wq8, sc8, out=o, stream=st), n)
+    e = _tensor_entry("dq_fp8_linear", ms, 2.0 * M * N * K, peaks, probe)
+    e["peak_note"] = "e4m3 x e4m3 nominal rate = the int8 rate (bf16 x 2)"
+    out["fp8_llm_2048x4096x4096"] = e
+    del wq8, sc8, q8, s8, o
+    # weight-only int4 (HQQ) at the page's few-token and 1024-token shapes
+    N = K = 4096
+    gen.manual_seed(21)
+    codes = torch.randint(0, 16, (N, K), dtype=torch.int8, device="cuda", generator=gen)
+    packed = dq.dq_hqq_pack(codes)
+    del codes
+    scl = dq.dq_hqq_group_major((torch.rand((N, K // 128), generator=gen, device="cuda") * 0.018 + 0.002).to(torch.bfloat16))
+    zer = dq.dq_hqq_group_major((torch.rand((N, K // 128), generator=gen, device="cuda") * 3 + 6).to(torch.bfloat16))
+    for M in (16, 1024):
+        x = randn((M, K), 1.0, 22 + M).to(torch.bfloat16)
+        o = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        nws = dq.dq_hqq_workspace_size(M, N, K)
+        ws = torch.zeros(nws, dtype=torch.uint8, device="cuda") if nws else None
+        ms = _graph_ms(torch, lambda i, st: dq.dq_hqq_linear(x, packed, scl, zer, 128, out=o, workspace=ws, stream=st), n)
+        nbytes = 2 * M * K + N * K // 2 + 2 * 2 * N * (K // 128) + 2 * M * N
+        if M <= 128:
+            e = _hbm_entry("dq_hqq_linear", ms, nbytes, peaks)
+        else:
+            tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+            e = dict(kernel="dq_hqq_linear", kernel_ms=round(ms, 5), bound="tensor", achieved=round(tf, 1),
+                     unit="TFLOP/s", peak=peaks["bf16"], frac=round(tf / peaks["bf16"], 4))
+        e["page_h100_ms"] = HQQ_PAGE_H100_MS[M]
+        out[f"hqq_m{M}_4096x4096_g128"] = e
+        del x, o, ws
+    del packed, scl, zer
     torch.cuda.synchronize()
     assert dq.dq_sync_status() == dq.DQ_OK
     torch.cuda.empty_cache()

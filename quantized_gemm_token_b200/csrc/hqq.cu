@@ -308,6 +308,9 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // With a programmatic (early) launch, the previous kernel of the stream is
+  // complete before any global memory is touched.
+  griddep_wait();
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
@@ -650,8 +653,19 @@ dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const HqqArgs
                      cudaStream_t stream) {
   const dq_status st = smem_limit_once(reinterpret_cast<const void*>(&hqq_gemm_kernel<TRANS, S4>), HQ_SMEM_LIMIT);
   if (st != DQ_OK) return st;
-  hqq_gemm_kernel<TRANS, S4><<<grid, HQ_THREADS, smem, stream>>>(tx, tw, g);
-  const cudaError_t e = cudaGetLastError();
+  // Programmatic stream serialization: the prologue (barriers, tensor-memory
+  // allocation) overlaps the tail of the previous kernel of the stream.
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(HQ_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, hqq_gemm_kernel<TRANS, S4>, tx, tw, g);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 

@@ -370,13 +370,13 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
             const int width = min(32, g.bn - 32 * c);
             uint32_t r[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              int32_t s = 0;
-              if (j < width) {
-                for (int sp = 0; sp < g.splits; ++sp)
-                  s += __ldcg(tile_ws + (static_cast<int64_t>(sp) * g.bn + 32 * c + j) * 128 + row);
-              }
-              r[j] = static_cast<uint32_t>(s);
+            for (int j = 0; j < 32; ++j) r[j] = 0u;
+            // split by split, the chunk's loads all in flight together
+            for (int sp = 0; sp < g.splits; ++sp) {
+              const int32_t* src = tile_ws + (static_cast<int64_t>(sp) * g.bn + 32 * c) * 128 + row;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < width) r[j] = static_cast<uint32_t>(static_cast<int32_t>(r[j]) + __ldcg(src + j * 128));
             }
             store_chunk(g, r, width, tok0 + 32 * c, ch, lane);
           }
@@ -444,10 +444,12 @@ struct S24Plan {
   size_t cnt_bytes, ws_bytes, smem;
 };
 
-// Token tile width and contraction split: the pair (bn, splits) whose waves
-// of units over the SMs cost the least, a unit costing its steps times
-// (bn + 32) (a fixed share per step for the weight tile and the MMA issue).
-// Splits need a workspace and at least four steps per unit.
+// Token tile width: the multiple of 16 (<= S4_MAX_BN) whose whole waves of
+// tiles over the SMs cost the least, a tile costing bn + 32 per step (a fixed
+// share per step for the weight tile and the MMA issue).  The contraction is
+// split only when the tiles cannot fill the SMs (few channels and tokens), at
+// least four steps per split: each split writes and the last one reads back
+// an int32 partial tile.
 S24Plan plan_s24(int64_t M, int64_t N, int64_t K, int sm_count, bool allow_split) {
   S24Plan best{};
   long long best_cost = -1;
@@ -457,20 +459,20 @@ S24Plan plan_s24(int64_t M, int64_t N, int64_t K, int sm_count, bool allow_split
     if (bn > 16 && bn - 16 >= M) break;                 // wider tiles only add empty tokens
     const int tt = static_cast<int>((M + bn - 1) / bn);
     const long long tiles = static_cast<long long>(nt) * tt;
-    for (int s = 1; s <= (allow_split ? 8 : 1); ++s) {
-      if (s > 1 && ks / s < 4) break;
-      const long long units = tiles * s;
-      if (units > 0x7fffffffLL) continue;
-      const long long waves = (units + sm_count - 1) / sm_count;
-      const long long steps = (ks + s - 1) / s;
-      const long long cost = waves * steps * (bn + 32) + (s > 1 ? steps : 0);
-      if (best_cost < 0 || cost < best_cost) {
-        best_cost = cost;
-        best.bn = bn;
-        best.tt = tt;
-        best.splits = s;
-      }
+    const long long waves = (tiles + sm_count - 1) / sm_count;
+    const long long cost = waves * (bn + 32);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best.bn = bn;
+      best.tt = tt;
     }
+  }
+  best.splits = 1;
+  const long long tiles0 = static_cast<long long>(nt) * best.tt;
+  if (allow_split && tiles0 < sm_count) {
+    int sp = static_cast<int>(sm_count / tiles0);
+    sp = std::min(sp, std::max(1, ks / 4));
+    best.splits = std::max(1, std::min(sp, 32));
   }
   S24Plan& p = best;
   p.nt = nt;
