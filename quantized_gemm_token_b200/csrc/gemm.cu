@@ -79,6 +79,8 @@ struct Cfg {
   // shared memory for a TMA store: 2 buffers x 4 warps x 4 KB (int32 worst case).
   // Epilogue warps: two per TMEM sub-partition when a tile has at least two
   // 32-column chunks, so one warp's latency hides behind the other's work.
+  // (Measured on B200 for the epilogue-bound BSR kernel: 12 or 16 epilogue
+  // warps are slower than 8.)
   static constexpr int EPI_WARPS = BN >= 64 ? 8 : 4;
   static constexpr bool STAGED_OUT = KIND != Kind::Swap;
   static constexpr int OUT_BUF_BYTES = 32 * 32 * 4;           // per epilogue warp

@@ -50,14 +50,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// may be suspended (up to the hint, or until the phase completes) instead of
+// spinning, so waiting producer / MMA threads take no issue slots from the
+// epilogue warps of their sub-partition (measured on B200: the BSR kernel,
+// epilogue-bound, 8 % faster than with a spinning wait).
+constexpr uint32_t kWaitSuspendNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kWaitSuspendNs)
       : "memory");
   return ok != 0;
 }
