@@ -50,14 +50,15 @@ constexpr int S4_BK = 128;                 // logical in-features per step (two 
 constexpr int S4_V_BYTES = 128 * 64;       // compressed values per step
 constexpr int S4_M_BYTES = 128 * 16;       // metadata per step
 constexpr int S4_MAX_NP = 16;
-constexpr int S4_MAX_BN = 224;             // tokens per tile
-constexpr int S4_ACC_COLS = 224;           // TMEM columns per accumulator buffer
-constexpr int S4_META_COL = 2 * S4_ACC_COLS;   // metadata ring: 4 TMEM columns per stage
+constexpr int S4_MAX_BN = 240;             // tokens per tile
+// Tensor memory: two accumulators of bn columns at columns 0 and bn, then
+// the metadata ring at column 2 * bn, 4 columns per stage (so bn = 240
+// leaves room for 8 stages, bn <= 192 for all 16).
 constexpr int S4_TMEM_COLS = 512;
 constexpr int S4_SMEM_LIMIT = 227 * 1024;
 constexpr int S4_BAR_BYTES = 1024;
 constexpr int S4_CNT_PER_TILE = 8;         // split arrival counters per tile: one per epilogue warp
-static_assert(S4_META_COL + 4 * S4_MAX_NP <= S4_TMEM_COLS, "tensor memory");
+static_assert(2 * S4_MAX_BN + 4 * 8 <= S4_TMEM_COLS, "tensor memory");
 
 struct S24Args {
   int M, N, K;
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
         const Unit t = decode_unit(g, u);
         if (!pipe::wait(smem_u32(acce + acc), aphase ^ 1, g.wait, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * S4_ACC_COLS);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * g.bn);
         for (int kk = t.k0; kk < t.k1; ++kk) {
           if (!pipe::wait(smem_u32(full + stage), phase, g.wait, abort_flag)) {
             ok = false;
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
           const uint32_t sv = sq + q_bytes;
           // the step's metadata into this stage's tensor-memory slot (the
           // slot's previous MMAs completed before the stage was refilled)
-          const uint32_t meta = tmem_base + static_cast<uint32_t>(S4_META_COL + 4 * stage);
+          const uint32_t meta = tmem_base + static_cast<uint32_t>(2 * g.bn + 4 * stage);
           tmem_cp_128x128b(meta, sv + S4_V_BYTES);
           const uint64_t ad = smem_desc_kmajor<64>(sv);
           const uint64_t bd = smem_desc_kmajor<128>(sq);
@@ -319,7 +320,7 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
       const bool w = pipe::wait(smem_u32(accf + acc), aphase, g.wait, abort_flag);
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
-      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S4_ACC_COLS);
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * g.bn);
       const int ch = t.ntile * 128 + row;
       const int tok0 = t.ttile * g.bn;
       const int nch = (g.bn + 31) / 32;
@@ -483,7 +484,7 @@ S24Plan plan_s24(int64_t M, int64_t N, int64_t K, int sm_count, bool allow_split
   p.units = static_cast<int>(tiles * p.splits);
   p.grid = std::min(p.units, sm_count);
   const int stage = p.bn * 128 + S4_V_BYTES + S4_M_BYTES;
-  p.np = std::min(S4_MAX_NP, (S4_SMEM_LIMIT - 1024 - S4_BAR_BYTES) / stage);
+  p.np = std::min({S4_MAX_NP, (S4_SMEM_LIMIT - 1024 - S4_BAR_BYTES) / stage, (S4_TMEM_COLS - 2 * p.bn) / 4});
   p.smem = 1024 + static_cast<size_t>(p.np) * stage + S4_BAR_BYTES;
   return p;
 }
