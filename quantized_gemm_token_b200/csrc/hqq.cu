@@ -7,8 +7,11 @@
 //
 // One persistent, warp-specialised kernel for sm_100a (448 threads):
 //   warp 0       TMA producer: for each 64-deep contraction step, the packed
-//                int4 weight tile (4 KB) and the activation tile (BN tokens x
-//                64 bf16, 128B-swizzled) into a ring of NP stages.
+//                int4 weight tile (4 KB), the activation tile (BN tokens x
+//                64 bf16, 128B-swizzled) and the step's scale and zero-point
+//                rows (tensor copies too: 1-D bulk copies of a few hundred
+//                bytes took the issuing thread ~250 ns each) into a ring of
+//                NP stages.
 //   warp 1       MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in
 //                TMEM), M = 128 weight rows, N = BN tokens, K = 16 per
 //                instruction, four instructions per step.
@@ -67,8 +70,6 @@ struct HqqArgs {
   int units;              // nt * tt * splits
   int np;                 // packed / activation ring stages
   uint32_t off_bar;       // shared-memory offset of the barriers (after the stages)
-  const uint16_t* scale; // bf16 [n_groups, n_w], group-major
-  const uint16_t* zero;   // bf16 [n_groups, n_w]
   uint16_t* out;          // bf16 [M, n_out]
   float* ws;              // split partials: [tile][split][bn][128] fp32
   uint32_t* cnt;          // arrival counters: [tile][4]
@@ -262,6 +263,7 @@ __device__ __forceinline__ void store_pairs(const HqqArgs& g, const uint32_t (&r
 template <bool TRANS, bool S4>
 __global__ void __launch_bounds__(HQ_THREADS, 1)
     hqq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                    const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z,
                     const HqqArgs g) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -299,6 +301,8 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_s);
+    tma_prefetch_desc(&tm_z);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), HQ_TMEM_COLS);
@@ -327,15 +331,16 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
             ok = false;
             break;
           }
-          // scale / zero-point rows present for this step: forward the 128
-          // output channels of the tile, transposed the step's 64 weight rows
+          // scale / zero-point rows for this step: forward the 128 output
+          // channels of the tile, transposed the step's 64 weight rows (one
+          // box each; channels past n_w arrive as zeros)
           const int c0 = TRANS ? kk * HQ_BK : t.ntile * 128;
-          const int cnt = min(TRANS ? HQ_BK : 128, g.n_w - c0);          // a multiple of 8
+          constexpr uint32_t meta_box = TRANS ? 2 * HQ_BK : 2 * 128;       // bytes per row copy
           const int kbase = TRANS ? t.ntile * 128 : kk * HQ_BK;           // first in-feature
           const int nslices = TRANS ? 4 : 2;
           uint32_t meta_tx = 0;
           for (int j = 0; j < nslices; ++j)
-            if (cnt > 0 && j % per == 0 && kbase + 32 * j < g.k_w) meta_tx += 4u * static_cast<uint32_t>(cnt);
+            if (j % per == 0 && kbase + 32 * j < g.k_w) meta_tx += 2u * meta_box;
           const uint32_t fb = smem_u32(full + stage);
           const uint32_t sx = base + stage * stage_bytes + HQ_A_BYTES;
           const uint32_t sw = sx + x_bytes;
@@ -346,11 +351,11 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
           else
             tma_load_2d(sw, &tm_w, fb, kk * 32, t.ntile * 128);
           for (int j = 0; j < nslices; ++j) {
-            if (cnt > 0 && j % per == 0 && kbase + 32 * j < g.k_w) {
-              const int64_t off = static_cast<int64_t>((kbase + 32 * j) / g.group) * g.n_w + c0;
+            if (j % per == 0 && kbase + 32 * j < g.k_w) {
+              const int grow = (kbase + 32 * j) / g.group;
               const uint32_t dst = sw + HQ_W_BYTES + j * HQ_META_SLOT;
-              pipe::bulk_load_1d(dst, g.scale + off, 2u * cnt, fb);
-              pipe::bulk_load_1d(dst + HQ_META_HALF, g.zero + off, 2u * cnt, fb);
+              tma_load_2d(dst, &tm_s, fb, 2 * c0, grow);
+              tma_load_2d(dst + HQ_META_HALF, &tm_z, fb, 2 * c0, grow);
             }
           }
           ++issued;
@@ -649,8 +654,8 @@ dq_status check_weights(const uint8_t* packed, const void* scale, const void* ze
 }
 
 template <bool TRANS, bool S4>
-dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const HqqArgs& g, int grid, size_t smem,
-                     cudaStream_t stream) {
+dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts, const CUtensorMap& tz,
+                     const HqqArgs& g, int grid, size_t smem, cudaStream_t stream) {
   const dq_status st = smem_limit_once(reinterpret_cast<const void*>(&hqq_gemm_kernel<TRANS, S4>), HQ_SMEM_LIMIT);
   if (st != DQ_OK) return st;
   // Programmatic stream serialization: the prologue (barriers, tensor-memory
@@ -665,7 +670,7 @@ dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const HqqArgs
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, hqq_gemm_kernel<TRANS, S4>, tx, tw, g);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, hqq_gemm_kernel<TRANS, S4>, tx, tw, ts, tz, g);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 
@@ -699,6 +704,17 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   st = make_tmap_u8_2d(&tw, packed, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N),
                        static_cast<uint64_t>(K / 2), trans ? 64 : 32, trans ? 64 : 128, 0);
   if (st != DQ_OK) return st;
+  // scales and zero points, group-major [K / group, N] bf16 as bytes: one
+  // group row of the tile's channels (forward: 128) or of the step's weight
+  // rows (transposed: 64) per copy
+  CUtensorMap ts, tz;
+  const uint32_t meta_box = trans ? 2 * HQ_BK : 2 * 128;
+  st = make_tmap_u8_2d(&ts, scale, static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(K / group),
+                       static_cast<uint64_t>(N) * 2, meta_box, 1, 0);
+  if (st != DQ_OK) return st;
+  st = make_tmap_u8_2d(&tz, zero, static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(K / group),
+                       static_cast<uint64_t>(N) * 2, meta_box, 1, 0);
+  if (st != DQ_OK) return st;
 
   HqqArgs g{};
   g.M = static_cast<int>(M);
@@ -716,8 +732,6 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   g.units = p.units;
   g.np = p.np;
   g.off_bar = static_cast<uint32_t>(p.np) * (HQ_A_BYTES + p.bn * 128 + HQ_WM_BYTES);
-  g.scale = static_cast<const uint16_t*>(scale);
-  g.zero = static_cast<const uint16_t*>(zero);
   g.out = static_cast<uint16_t*>(out);
   if (p.splits > 1) {
     g.cnt = static_cast<uint32_t*>(workspace);
@@ -726,10 +740,10 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
   const bool s4 = (flags & DQ_HQQ_S4) != 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (trans) return s4 ? launch_hqq<true, true>(tx, tw, g, p.grid, p.smem, s)
-                       : launch_hqq<true, false>(tx, tw, g, p.grid, p.smem, s);
-  return s4 ? launch_hqq<false, true>(tx, tw, g, p.grid, p.smem, s)
-            : launch_hqq<false, false>(tx, tw, g, p.grid, p.smem, s);
+  if (trans) return s4 ? launch_hqq<true, true>(tx, tw, ts, tz, g, p.grid, p.smem, s)
+                       : launch_hqq<true, false>(tx, tw, ts, tz, g, p.grid, p.smem, s);
+  return s4 ? launch_hqq<false, true>(tx, tw, ts, tz, g, p.grid, p.smem, s)
+            : launch_hqq<false, false>(tx, tw, ts, tz, g, p.grid, p.smem, s);
 }
 
 int grid_for(int64_t items, int sm_count) {
