@@ -7,20 +7,25 @@
 //
 // One persistent, warp-specialised kernel for sm_100a (448 threads):
 //   warp 0       TMA producer: for each 64-deep contraction step, the packed
-//                int4 weight tile (4 KB), the activation tile (BN tokens x
-//                64 bf16, 128B-swizzled) and the step's scale and zero-point
-//                rows (tensor copies too: 1-D bulk copies of a few hundred
-//                bytes took the issuing thread ~250 ns each) into a ring of
-//                NP stages.
+//                int4 weight tile (4 KB) and the activation tile (BN tokens x
+//                64 bf16, 128B-swizzled) into a ring of NP stages.
 //   warp 1       MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in
 //                TMEM), M = 128 weight rows, N = BN tokens, K = 16 per
 //                instruction, four instructions per step.
 //   warps 2..9   dequantizers: unpack the codes, w = bf16(bf16(q - z) * s)
 //                in packed bf16x2 arithmetic, and write the 128 x 64 bf16 A
-//                operand in the 128B-swizzled K-major layout into a ring of
-//                ND stages (the bf16 weight never reaches global memory).
-//   warps 10..13 epilogue: tcgen05.ld the accumulator (TMEM lane = output
-//                channel, column = token), convert to bf16 and store.
+//                operand in the 128B-swizzled K-major layout into the stage
+//                (the bf16 weight never reaches global memory).  Each thread
+//                reads its own scales and zero points from global memory two
+//                steps ahead of use: copying them into the stages with the
+//                tiles cost the producer's copy engine about 100 ns per row
+//                copy, twice the time of an activation or weight tile.
+//   warps 10..17 epilogue, two warps per TMEM sub-partition taking
+//                alternate 32-token chunks: tcgen05.ld the accumulator (TMEM
+//                lane = output channel, column = token), convert to bf16,
+//                write the 32 tokens x 32 channels block into a staging
+//                buffer and store it with one TMA store (which clips tokens
+//                >= M and channels >= the output width).
 // The weight is the A operand (128 output channels per tile) and the tokens
 // the B operand (up to 256): the dequantization work per MMA flop is then as
 // small as a 128-row tile allows, and few-token calls need no padding to 128.
@@ -31,6 +36,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "internal.h"
 #include "pipeline.cuh"
@@ -39,18 +45,14 @@
 namespace dq {
 namespace {
 
-constexpr int HQ_THREADS = 448;
+constexpr int HQ_THREADS = 576;
 constexpr int HQ_DEQ_WARPS = 8;            // warps 2..9
-constexpr int HQ_EPI_WARP0 = 10;           // warps 10..13
+constexpr int HQ_EPI_WARP0 = 10;           // warps 10..17
+constexpr int HQ_EPI_WARPS = 8;
+constexpr int HQ_EPI_BUF = 2048;           // per epilogue warp: 32 tokens x 64 B
 constexpr int HQ_BK = 64;                  // contraction elements per step (128 B of bf16)
 constexpr int HQ_A_BYTES = 128 * 128;      // dequantized weight tile: 128 rows x 128 B
 constexpr int HQ_W_BYTES = 4096;           // packed int4 tile per step
-// Per-step scale and zero-point slices, staged next to the packed tile: four
-// slots of up to 128 bf16 channel values each (one slot per 32-deep k slice
-// that starts a new group), scales at +0, zero points at +HQ_META_HALF.
-constexpr int HQ_META_SLOT = 256;
-constexpr int HQ_META_HALF = 4 * HQ_META_SLOT;
-constexpr int HQ_WM_BYTES = HQ_W_BYTES + 2 * HQ_META_HALF;   // one W ring stage
 constexpr int HQ_MAX_NP = 16;
 constexpr int HQ_ACC_COLS = 256;           // TMEM columns per accumulator buffer
 constexpr int HQ_TMEM_COLS = 512;          // two accumulator buffers
@@ -62,14 +64,17 @@ struct HqqArgs {
   int n_out;              // output channels (N forward, K transposed)
   int kc;                 // contraction length (K forward, N transposed)
   int n_w, k_w;           // weight rows (N) and in-features (K)
-  int group, n_groups;    // group size and K / group
+  int group_log2;         // log2 of the group size (32 .. 256)
   int bn;                 // tokens per tile (multiple of 16, <= 256)
   int nt, tt;             // channel tiles (128 each), token tiles (bn each)
   int splits;             // contraction splits per tile
   int ks;                 // contraction steps per tile (ceil(kc / 64))
   int units;              // nt * tt * splits
   int np;                 // packed / activation ring stages
-  uint32_t off_bar;       // shared-memory offset of the barriers (after the stages)
+  uint32_t off_epi;       // shared-memory offset of the epilogue staging buffers (after the stages)
+  uint32_t off_bar;       // shared-memory offset of the barriers (after the staging buffers)
+  const uint16_t* scale;  // bf16 [K / group, n_w], group-major
+  const uint16_t* zero;   // bf16 [K / group, n_w]
   uint16_t* out;          // bf16 [M, n_out]
   float* ws;              // split partials: [tile][split][bn][128] fp32
   uint32_t* cnt;          // arrival counters: [tile][4]
@@ -120,14 +125,6 @@ __device__ __forceinline__ uint32_t bf16_pair_of(uint16_t v) {
   return static_cast<uint32_t>(v) | (static_cast<uint32_t>(v) << 16);
 }
 
-// The meta slot holding the group of 32-deep k slice j: the first slice of
-// each group (groups of 32 start at every slice, groups of 64 at even ones,
-// larger groups at slice 0 of a step or tile).
-__device__ __forceinline__ int meta_slot(int j, int group) {
-  const int per = group >> 5;          // k slices per group: 1, 2, 4 or 8
-  return per >= 4 ? 0 : (j / per) * per;
-}
-
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulator,
 // both operands K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
@@ -147,24 +144,73 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// A dequantizing thread's scales and zero points for one step, as loaded
+// (zero where the channel or in-feature lies outside the weight or there is
+// no step): forward one channel's s and z (bf16 bits) for its 32 codes;
+// transposed eight weight rows' values (bf16 pairs) for each of its two byte
+// columns.  The loads are predicated inline loads into the registers that
+// hold them until use: any instruction that read or selected a loaded value
+// here would wait for the load.
+struct MetaFwd {
+  uint32_t s, z;
+};
+struct MetaT {
+  uint4 s8[2], z8[2];
+};
+
+__device__ __forceinline__ void ldg_u16_or0(uint32_t& v, const uint16_t* p, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\tmov.b32 %0, 0;\n\t@q ld.global.nc.u16 %0, [%2];\n\t}"
+      : "=r"(v)
+      : "r"(static_cast<int>(pred)), "l"(p));
+}
+__device__ __forceinline__ void ldg_v4_or0(uint4& v, const uint16_t* p, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %4, 0;\n\tmov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\t"
+      "mov.b32 %3, 0;\n\t@q ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%5];\n\t}"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "r"(static_cast<int>(pred)), "l"(p));
+}
+
+// Forward: thread t handles row t % 128 and codes 32 * (t / 128) .. +31 of
+// the step, all inside one group (group sizes are >= 32).
+__device__ __forceinline__ void load_meta_fwd(const HqqArgs& g, int dt, bool valid, int ntile, int kstep,
+                                              MetaFwd& m) {
+  const int n = ntile * 128 + (dt & 127);
+  const int k = kstep * HQ_BK + (dt >> 7) * 32;
+  const bool in = valid && n < g.n_w && k < g.k_w;
+  const int64_t gi = in ? static_cast<int64_t>(k >> g.group_log2) * g.n_w + n : 0;
+  ldg_u16_or0(m.s, g.scale + gi, in);
+  ldg_u16_or0(m.z, g.zero + gi, in);
+}
+
+// Transposed: warp w of the dequantizers handles weight rows n0 = 64 *
+// kstep + 8 w .. +7 (16 contiguous bytes of a group row: n_w % 8 == 0, so
+// the eight rows are all inside or all outside), lane l the output channels
+// k = 2 b, 2 b + 1 for b = l and l + 32 (one group: groups are >= 32 wide
+// and start at even k).
+__device__ __forceinline__ void load_meta_t(const HqqArgs& g, int dt, bool valid, int ntile, int kstep, MetaT& m) {
+  const int n0 = kstep * HQ_BK + (dt >> 5) * 8;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int k = ntile * 128 + 2 * ((dt & 31) + 32 * u);
+    const bool in = valid && n0 < g.n_w && k < g.k_w;
+    const int64_t gi = in ? static_cast<int64_t>(k >> g.group_log2) * g.n_w + n0 : 0;
+    ldg_v4_or0(m.s8[u], g.scale + gi, in);
+    ldg_v4_or0(m.z8[u], g.zero + gi, in);
+  }
+}
+
 // Forward: 256 threads turn the packed tile (128 channel rows x 32 B = 64
-// codes) into the 128 x 64 bf16 A tile.  Thread t: row t % 128, codes
-// 32 * (t / 128) .. +31 (inside one group: group sizes are >= 32); its scale
-// and zero point come from the step's staged meta slots.
+// codes) into the 128 x 64 bf16 A tile (thread t: row t % 128, codes
+// 32 * (t / 128) .. +31).
 template <bool S4>
-__device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t atile, uint32_t wtile, int dt, int ntile,
-                                                 int kstep) {
+__device__ __forceinline__ void dequant_tile_fwd(uint32_t atile, uint32_t wtile, int dt, const MetaFwd& m) {
   const int r = dt & 127;
   const int h = dt >> 7;
   const uint4 pk = pipe::lds128(wtile + r * 32 + h * 16);
-  const int n = ntile * 128 + r;
-  const int k = kstep * HQ_BK + h * 32;
-  uint32_t s2 = 0, z2 = 0;
-  if (n < g.n_w && k < g.k_w) {
-    const uint32_t meta = wtile + HQ_W_BYTES + meta_slot(h, g.group) * HQ_META_SLOT + 2 * r;
-    s2 = bf16_pair_of(static_cast<uint16_t>(pipe::lds16(meta)));
-    z2 = bf16_pair_of(static_cast<uint16_t>(pipe::lds16(meta + HQ_META_HALF)));
-  }
+  const uint32_t s2 = m.s | (m.s << 16);
+  const uint32_t z2 = m.z | (m.z << 16);
   const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -179,26 +225,17 @@ __device__ __forceinline__ void dequant_tile_fwd(const HqqArgs& g, uint32_t atil
 // 64 bf16 (n).  Warp w handles n = 8w .. 8w+7; lane l the byte columns l and
 // l + 32 (A rows 2l, 2l+1 and 2l+64, 2l+65): eight bytes from eight weight
 // rows give two 16-byte chunks, one per A row.  The eight rows' scales and
-// zero points are 16 contiguous bytes of a staged meta slot: the bf16 pairs
+// zero points (16 contiguous bytes of a group row each) are the bf16 pairs
 // the packed arithmetic needs.
 template <bool S4>
-__device__ __forceinline__ void dequant_tile_t(const HqqArgs& g, uint32_t atile, uint32_t wtile, int dt, int ntile,
-                                               int kstep) {
+__device__ __forceinline__ void dequant_tile_t(uint32_t atile, uint32_t wtile, int dt, const MetaT& m) {
   const int nc = dt >> 5;       // n chunk (8 weight rows)
   const int lane = dt & 31;
-  const bool n_ok = kstep * HQ_BK + nc * 8 < g.n_w;     // n_w % 8 == 0: the chunk is all in or all out
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     const int b = lane + 32 * u;                 // byte column: k = 2b, 2b + 1 in the tile
-    const int k = ntile * 128 + 2 * b;
-    uint4 s8 = make_uint4(0, 0, 0, 0), z8 = make_uint4(0, 0, 0, 0);
-    if (n_ok && k < g.k_w) {
-      const uint32_t meta = wtile + HQ_W_BYTES + meta_slot(b >> 4, g.group) * HQ_META_SLOT + nc * 16;
-      s8 = pipe::lds128(meta);
-      z8 = pipe::lds128(meta + HQ_META_HALF);
-    }
-    const uint32_t sp[4] = {s8.x, s8.y, s8.z, s8.w};
-    const uint32_t zp[4] = {z8.x, z8.y, z8.z, z8.w};
+    const uint32_t sp[4] = {m.s8[u].x, m.s8[u].y, m.s8[u].z, m.s8[u].w};
+    const uint32_t zp[4] = {m.z8[u].x, m.z8[u].y, m.z8[u].z, m.z8[u].w};
     uint32_t lo[4], hi[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -234,28 +271,53 @@ __device__ __forceinline__ Unit decode_unit(const HqqArgs& g, int u) {
   return t;
 }
 
+// The CTA's contraction steps in order, across its units: (ntile, kk).
+struct StepIt {
+  int u, kk, k1, ntile;
+  bool valid;
+  __device__ __forceinline__ void start(const HqqArgs& g, int u0) {
+    u = u0;
+    valid = false;
+    for (; u < g.units; u += gridDim.x) {
+      const Unit t = decode_unit(g, u);
+      if (t.k0 < t.k1) {
+        kk = t.k0;
+        k1 = t.k1;
+        ntile = t.ntile;
+        valid = true;
+        return;
+      }
+    }
+  }
+  __device__ __forceinline__ void next(const HqqArgs& g) {
+    if (!valid) return;
+    if (++kk < k1) return;
+    start(g, u + gridDim.x);
+  }
+};
+
 __device__ __forceinline__ uint32_t bf16_bits(float f) {
   return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
-// Stores `width` (16 or 32) tokens of one output channel per lane as bf16:
-// lanes exchange values in pairs so that each lane writes two neighbouring
-// channels of one token (4 bytes; a warp covers 64 contiguous bytes).
-__device__ __forceinline__ void store_pairs(const HqqArgs& g, const uint32_t (&r)[32], int width, int tok0,
-                                            int ch, int lane) {
+// Writes `width` (16 or 32) tokens of one output channel per lane as bf16
+// into the staging buffer `buf` (row j = token j, 64 B = the warp's 32
+// channels): lanes exchange values in pairs so that each lane writes two
+// neighbouring channels of one token (4 bytes; rows j and j + 1 of one
+// instruction cover all 32 banks).
+__device__ __forceinline__ void stage_pairs(uint32_t buf, const uint32_t (&r)[32], int width, int lane) {
   const bool odd = lane & 1;
-  const int ch_even = ch & ~1;
-  const bool ch_ok = ch < g.n_out;     // n_out is even: same answer for both lanes of a pair
+  const uint32_t col = static_cast<uint32_t>(lane & ~1) * 2u;
+  const uint32_t sel = odd ? 0x3276u : 0x5410u;
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
     if (j < width) {
-      const uint32_t h0 = bf16_bits(__uint_as_float(r[j]));
-      const uint32_t h1 = bf16_bits(__uint_as_float(r[j + 1]));
-      const uint32_t recv = __shfl_xor_sync(0xffffffffu, odd ? h0 : h1, 1);
-      const int tok = tok0 + j + (odd ? 1 : 0);
-      const uint32_t v = odd ? (recv | (h1 << 16)) : (h0 | (recv << 16));
-      if (ch_ok && tok < g.M)
-        *reinterpret_cast<uint32_t*>(g.out + static_cast<int64_t>(tok) * g.n_out + ch_even) = v;
+      uint32_t pk;   // lo = bf16(token j), hi = bf16(token j + 1) of this lane's channel
+      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(pk) : "f"(__uint_as_float(r[j + 1])), "f"(__uint_as_float(r[j])));
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, pk, 1);
+      // even lane: (own token j, partner's token j); odd: (partner's j + 1, own j + 1)
+      const uint32_t v = __byte_perm(pk, recv, sel);
+      pipe::sts32(buf + static_cast<uint32_t>(j + (odd ? 1 : 0)) * 64u + col, v);
     }
   }
 }
@@ -263,7 +325,7 @@ __device__ __forceinline__ void store_pairs(const HqqArgs& g, const uint32_t (&r
 template <bool TRANS, bool S4>
 __global__ void __launch_bounds__(HQ_THREADS, 1)
     hqq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                    const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z,
+                    const __grid_constant__ CUtensorMap tm_c32, const __grid_constant__ CUtensorMap tm_c16,
                     const HqqArgs g) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -272,7 +334,7 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
   // stage s at base + s * stage_bytes: dequantized A tile (16 KB), then the
   // activation tile (bn x 128 B), then the packed weight tile and its meta
   const uint32_t x_bytes = static_cast<uint32_t>(g.bn) * 128u;
-  const uint32_t stage_bytes = HQ_A_BYTES + x_bytes + HQ_WM_BYTES;
+  const uint32_t stage_bytes = HQ_A_BYTES + x_bytes + HQ_W_BYTES;
   uint64_t* const full = reinterpret_cast<uint64_t*>(smem + g.off_bar);   // TMA landed
   uint64_t* const deq = full + HQ_MAX_NP;                                 // A tile written
   uint64_t* const empty = deq + HQ_MAX_NP;                                // MMAs done with the stage
@@ -295,14 +357,12 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(accf + i), 1);
-      mbar_init(smem_u32(acce + i), 4);
+      mbar_init(smem_u32(acce + i), HQ_EPI_WARPS);
     }
     mbar_init(smem_u32(drain), 1);
     fence_barrier_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
-    tma_prefetch_desc(&tm_s);
-    tma_prefetch_desc(&tm_z);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), HQ_TMEM_COLS);
@@ -323,7 +383,6 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
-      const int per = g.group >> 5;          // 32-deep k slices per group
       for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
         const Unit t = decode_unit(g, u);
         for (int kk = t.k0; kk < t.k1; ++kk) {
@@ -331,33 +390,15 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
             ok = false;
             break;
           }
-          // scale / zero-point rows for this step: forward the 128 output
-          // channels of the tile, transposed the step's 64 weight rows (one
-          // box each; channels past n_w arrive as zeros)
-          const int c0 = TRANS ? kk * HQ_BK : t.ntile * 128;
-          constexpr uint32_t meta_box = TRANS ? 2 * HQ_BK : 2 * 128;       // bytes per row copy
-          const int kbase = TRANS ? t.ntile * 128 : kk * HQ_BK;           // first in-feature
-          const int nslices = TRANS ? 4 : 2;
-          uint32_t meta_tx = 0;
-          for (int j = 0; j < nslices; ++j)
-            if (j % per == 0 && kbase + 32 * j < g.k_w) meta_tx += 2u * meta_box;
           const uint32_t fb = smem_u32(full + stage);
           const uint32_t sx = base + stage * stage_bytes + HQ_A_BYTES;
           const uint32_t sw = sx + x_bytes;
-          mbar_arrive_expect_tx(fb, x_bytes + HQ_W_BYTES + meta_tx);
+          mbar_arrive_expect_tx(fb, x_bytes + HQ_W_BYTES);
           tma_load_2d(sx, &tm_x, fb, kk * 128, t.ttile * g.bn);
           if (TRANS)
             tma_load_2d(sw, &tm_w, fb, t.ntile * 64, kk * HQ_BK);
           else
             tma_load_2d(sw, &tm_w, fb, kk * 32, t.ntile * 128);
-          for (int j = 0; j < nslices; ++j) {
-            if (j % per == 0 && kbase + 32 * j < g.k_w) {
-              const int grow = (kbase + 32 * j) / g.group;
-              const uint32_t dst = sw + HQ_W_BYTES + j * HQ_META_SLOT;
-              tma_load_2d(dst, &tm_s, fb, 2 * c0, grow);
-              tma_load_2d(dst + HQ_META_HALF, &tm_z, fb, 2 * c0, grow);
-            }
-          }
           ++issued;
           if (++stage == g.np) {
             stage = 0;
@@ -419,37 +460,61 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     // ---------------------------------------------------------- dequantizers
     // A stage's A tile is free again once its copies have landed: the
     // producer refilled the stage only after the MMAs that read it completed.
+    // Each thread's scales and zero points are loaded two steps ahead of use.
+    using Meta = typename std::conditional<TRANS, MetaT, MetaFwd>::type;
     const int dt = threadIdx.x - 64;
+    auto load_meta = [&](const StepIt& s, Meta& m) {
+      if constexpr (TRANS)
+        load_meta_t(g, dt, s.valid, s.ntile, s.kk, m);
+      else
+        load_meta_fwd(g, dt, s.valid, s.ntile, s.kk, m);
+    };
+    StepIt cur, ahead;
+    cur.start(g, blockIdx.x);
+    ahead = cur;
+    ahead.next(g);
+    ahead.next(g);
     int stage = 0;
     uint32_t phase = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; ok && u < g.units; u += gridDim.x) {
-      const Unit t = decode_unit(g, u);
-      for (int kk = t.k0; kk < t.k1; ++kk) {
-        const bool w = pipe::wait(smem_u32(full + stage), phase, g.wait, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
-        const uint32_t sa = base + stage * stage_bytes;
-        const uint32_t wt = sa + HQ_A_BYTES + x_bytes;
-        if (TRANS)
-          dequant_tile_t<S4>(g, sa, wt, dt, t.ntile, kk);
-        else
-          dequant_tile_fwd<S4>(g, sa, wt, dt, t.ntile, kk);
-        fence_proxy_async_smem();     // generic-proxy writes -> visible to the MMA
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(deq + stage));
-        if (++stage == g.np) {
-          stage = 0;
-          phase ^= 1;
-        }
+    // One step: `use` holds this step's values; the values of the step two
+    // ahead are loaded into `fill` (free since the previous step).  Three
+    // sets rotate by name, so no register is copied while its load is in
+    // flight (a copy would wait for the load).
+    auto step = [&](const Meta& use, Meta& fill) -> bool {
+      if (!cur.valid) return false;
+      load_meta(ahead, fill);
+      const bool w = pipe::wait(smem_u32(full + stage), phase, g.wait, abort_flag);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      const uint32_t sa = base + stage * stage_bytes;
+      const uint32_t wt = sa + HQ_A_BYTES + x_bytes;
+      if constexpr (TRANS)
+        dequant_tile_t<S4>(sa, wt, dt, use);
+      else
+        dequant_tile_fwd<S4>(sa, wt, dt, use);
+      fence_proxy_async_smem();     // generic-proxy writes -> visible to the MMA
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(deq + stage));
+      if (++stage == g.np) {
+        stage = 0;
+        phase ^= 1;
       }
+      cur.next(g);
+      ahead.next(g);
+      return true;
+    };
+    Meta ma, mb, mc;
+    load_meta(cur, ma);
+    StepIt one = cur;
+    one.next(g);
+    load_meta(one, mb);
+    while (step(ma, mc) && step(mb, ma) && step(mc, mb)) {
     }
   } else {
     // ---------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM sub-partition of this warp
+    const int half = (warp - HQ_EPI_WARP0) >> 2;   // chunks half, half + 2, ...
     const int row = q * 32 + lane;          // accumulator row = output channel in the tile
+    const uint32_t buf = base + g.off_epi + static_cast<uint32_t>(warp - HQ_EPI_WARP0) * HQ_EPI_BUF;
     int acc = 0;
     uint32_t aphase = 0;
     for (int u = blockIdx.x; u < g.units; u += gridDim.x) {
@@ -458,11 +523,11 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * HQ_ACC_COLS);
-      const int ch = t.ntile * 128 + row;
+      const int ch0 = t.ntile * 128 + q * 32;
       const int tok0 = t.ttile * g.bn;
       float* const part =
           g.splits > 1 ? g.ws + static_cast<int64_t>(t.tile * g.splits + t.split) * g.bn * 128 : nullptr;
-      for (int c0 = 0; c0 < g.bn; c0 += 32) {
+      for (int c0 = half * 32; c0 < g.bn; c0 += 64) {
         const int width = min(32, g.bn - c0);
         uint32_t r[32];
         if (width == 32) {
@@ -481,7 +546,15 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
           for (int j = 0; j < 32; ++j)
             if (j < width) part[static_cast<int64_t>(c0 + j) * 128 + row] = __uint_as_float(r[j]);
         } else {
-          store_pairs(g, r, width, tok0 + c0, ch, lane);
+          if (lane == 0) bulk_wait_group_read<0>();    // the previous store has read the buffer
+          __syncwarp();
+          stage_pairs(buf, r, width, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && ch0 < g.n_out && tok0 + c0 < g.M) {     // boxes wholly outside are not issued
+            tma_store_2d(width == 32 ? &tm_c32 : &tm_c16, buf, 2 * ch0, tok0 + c0);
+            bulk_commit_group();
+          }
         }
       }
       tc_fence_before();
@@ -493,6 +566,8 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       }
       if (part != nullptr) __threadfence();     // the partial tile is published below
     }
+    if (lane == 0) bulk_wait_group<0>();         // every output store complete
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -634,10 +709,10 @@ HqqPlan plan_hqq(int64_t M, int64_t n_out, int64_t kc, int sm_count, bool allow_
   p.ws_bytes = p.splits > 1 ? p.cnt_bytes + static_cast<size_t>(tiles) * p.splits * p.bn * 128 * sizeof(float) : 0;
   p.units = static_cast<int>(tiles * p.splits);
   p.grid = std::min(p.units, sm_count);
-  const int stage = HQ_A_BYTES + p.bn * 128 + HQ_WM_BYTES;
-  const int avail = HQ_SMEM_LIMIT - 1024 - HQ_BAR_BYTES;
+  const int stage = HQ_A_BYTES + p.bn * 128 + HQ_W_BYTES;
+  const int avail = HQ_SMEM_LIMIT - 1024 - HQ_EPI_WARPS * HQ_EPI_BUF - HQ_BAR_BYTES;
   p.np = std::min(HQ_MAX_NP, avail / stage);
-  p.smem = 1024 + static_cast<size_t>(p.np) * stage + HQ_BAR_BYTES;
+  p.smem = 1024 + static_cast<size_t>(p.np) * stage + HQ_EPI_WARPS * HQ_EPI_BUF + HQ_BAR_BYTES;
   return p;
 }
 
@@ -654,7 +729,7 @@ dq_status check_weights(const uint8_t* packed, const void* scale, const void* ze
 }
 
 template <bool TRANS, bool S4>
-dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts, const CUtensorMap& tz,
+dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& tc32, const CUtensorMap& tc16,
                      const HqqArgs& g, int grid, size_t smem, cudaStream_t stream) {
   const dq_status st = smem_limit_once(reinterpret_cast<const void*>(&hqq_gemm_kernel<TRANS, S4>), HQ_SMEM_LIMIT);
   if (st != DQ_OK) return st;
@@ -670,7 +745,7 @@ dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const CUtenso
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, hqq_gemm_kernel<TRANS, S4>, tx, tw, ts, tz, g);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, hqq_gemm_kernel<TRANS, S4>, tx, tw, tc32, tc16, g);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 
@@ -704,16 +779,14 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   st = make_tmap_u8_2d(&tw, packed, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N),
                        static_cast<uint64_t>(K / 2), trans ? 64 : 32, trans ? 64 : 128, 0);
   if (st != DQ_OK) return st;
-  // scales and zero points, group-major [K / group, N] bf16 as bytes: one
-  // group row of the tile's channels (forward: 128) or of the step's weight
-  // rows (transposed: 64) per copy
-  CUtensorMap ts, tz;
-  const uint32_t meta_box = trans ? 2 * HQ_BK : 2 * 128;
-  st = make_tmap_u8_2d(&ts, scale, static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(K / group),
-                       static_cast<uint64_t>(N) * 2, meta_box, 1, 0);
+
+  // output bf16 [M, n_out] as bytes: 32 channels (64 B) x 32 or 16 tokens
+  CUtensorMap tc32, tc16;
+  st = make_tmap_u8_2d(&tc32, out, static_cast<uint64_t>(n_out) * 2, static_cast<uint64_t>(M),
+                       static_cast<uint64_t>(n_out) * 2, 64, 32, 0);
   if (st != DQ_OK) return st;
-  st = make_tmap_u8_2d(&tz, zero, static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(K / group),
-                       static_cast<uint64_t>(N) * 2, meta_box, 1, 0);
+  st = make_tmap_u8_2d(&tc16, out, static_cast<uint64_t>(n_out) * 2, static_cast<uint64_t>(M),
+                       static_cast<uint64_t>(n_out) * 2, 64, 16, 0);
   if (st != DQ_OK) return st;
 
   HqqArgs g{};
@@ -722,8 +795,7 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   g.kc = static_cast<int>(kc);
   g.n_w = static_cast<int>(N);
   g.k_w = static_cast<int>(K);
-  g.group = group;
-  g.n_groups = static_cast<int>(K / group);
+  g.group_log2 = group == 32 ? 5 : group == 64 ? 6 : group == 128 ? 7 : 8;
   g.bn = p.bn;
   g.nt = p.nt;
   g.tt = p.tt;
@@ -731,7 +803,10 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   g.ks = p.ks;
   g.units = p.units;
   g.np = p.np;
-  g.off_bar = static_cast<uint32_t>(p.np) * (HQ_A_BYTES + p.bn * 128 + HQ_WM_BYTES);
+  g.off_epi = static_cast<uint32_t>(p.np) * (HQ_A_BYTES + p.bn * 128 + HQ_W_BYTES);
+  g.off_bar = g.off_epi + HQ_EPI_WARPS * HQ_EPI_BUF;
+  g.scale = static_cast<const uint16_t*>(scale);
+  g.zero = static_cast<const uint16_t*>(zero);
   g.out = static_cast<uint16_t*>(out);
   if (p.splits > 1) {
     g.cnt = static_cast<uint32_t*>(workspace);
@@ -740,10 +815,10 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
   const bool s4 = (flags & DQ_HQQ_S4) != 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (trans) return s4 ? launch_hqq<true, true>(tx, tw, ts, tz, g, p.grid, p.smem, s)
-                       : launch_hqq<true, false>(tx, tw, ts, tz, g, p.grid, p.smem, s);
-  return s4 ? launch_hqq<false, true>(tx, tw, ts, tz, g, p.grid, p.smem, s)
-            : launch_hqq<false, false>(tx, tw, ts, tz, g, p.grid, p.smem, s);
+  if (trans) return s4 ? launch_hqq<true, true>(tx, tw, tc32, tc16, g, p.grid, p.smem, s)
+                       : launch_hqq<true, false>(tx, tw, tc32, tc16, g, p.grid, p.smem, s);
+  return s4 ? launch_hqq<false, true>(tx, tw, tc32, tc16, g, p.grid, p.smem, s)
+            : launch_hqq<false, false>(tx, tw, tc32, tc16, g, p.grid, p.smem, s);
 }
 
 int grid_for(int64_t items, int sm_count) {
