@@ -12,7 +12,9 @@
 //   warp 1       MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in
 //                TMEM), M = 128 weight rows, N = BN tokens, K = 16 per
 //                instruction, four instructions per step.
-//   warps 2..9   dequantizers: unpack the codes, w = bf16(bf16(q - z) * s)
+//   warps 2..17  dequantizers, two groups of eight taking alternate steps
+//                (one group's barrier and address work overlaps the other's
+//                arithmetic): unpack the codes, w = bf16(bf16(q - z) * s)
 //                in packed bf16x2 arithmetic, and write the 128 x 64 bf16 A
 //                operand in the 128B-swizzled K-major layout into the stage
 //                (the bf16 weight never reaches global memory).  Each thread
@@ -20,12 +22,12 @@
 //                steps ahead of use: copying them into the stages with the
 //                tiles cost the producer's copy engine about 100 ns per row
 //                copy, twice the time of an activation or weight tile.
-//   warps 10..17 epilogue, two warps per TMEM sub-partition taking
-//                alternate 32-token chunks: tcgen05.ld the accumulator (TMEM
-//                lane = output channel, column = token), convert to bf16,
-//                write the 32 tokens x 32 channels block into a staging
-//                buffer and store it with one TMA store (which clips tokens
-//                >= M and channels >= the output width).
+//   warps 18..21 epilogue, one warp per TMEM sub-partition, two 32-token
+//                chunks per tensor-memory wait: tcgen05.ld the accumulator
+//                (TMEM lane = output channel, column = token), convert to
+//                bf16, write each 32 tokens x 32 channels block into a
+//                staging buffer and store it with one TMA store (which clips
+//                tokens >= M and channels >= the output width).
 // The weight is the A operand (128 output channels per tile) and the tokens
 // the B operand (up to 256): the dequantization work per MMA flop is then as
 // small as a 128-row tile allows, and few-token calls need no padding to 128.
@@ -45,11 +47,11 @@
 namespace dq {
 namespace {
 
-constexpr int HQ_THREADS = 576;
-constexpr int HQ_DEQ_WARPS = 8;            // warps 2..9
-constexpr int HQ_EPI_WARP0 = 10;           // warps 10..17
-constexpr int HQ_EPI_WARPS = 8;
-constexpr int HQ_EPI_BUF = 2048;           // per epilogue warp: 32 tokens x 64 B
+constexpr int HQ_THREADS = 704;
+constexpr int HQ_DEQ_WARPS = 8;            // per group: warps 2..9 and 10..17
+constexpr int HQ_EPI_WARP0 = 18;           // warps 18..21
+constexpr int HQ_EPI_WARPS = 4;
+constexpr int HQ_EPI_BUF = 2048;           // 32 tokens x 64 B; two per epilogue warp
 constexpr int HQ_BK = 64;                  // contraction elements per step (128 B of bf16)
 constexpr int HQ_A_BYTES = 128 * 128;      // dequantized weight tile: 128 rows x 128 B
 constexpr int HQ_W_BYTES = 4096;           // packed int4 tile per step
@@ -462,20 +464,26 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     // producer refilled the stage only after the MMAs that read it completed.
     // Each thread's scales and zero points are loaded two steps ahead of use.
     using Meta = typename std::conditional<TRANS, MetaT, MetaFwd>::type;
-    const int dt = threadIdx.x - 64;
+    const int dt = (threadIdx.x - 64) & 255;
+    const int grp = (threadIdx.x - 64) >> 8;     // group 1 takes the odd steps
     auto load_meta = [&](const StepIt& s, Meta& m) {
       if constexpr (TRANS)
         load_meta_t(g, dt, s.valid, s.ntile, s.kk, m);
       else
         load_meta_fwd(g, dt, s.valid, s.ntile, s.kk, m);
     };
+    // cur: this group's step; ahead: the group's step two of its own later
     StepIt cur, ahead;
     cur.start(g, blockIdx.x);
+    if (grp) cur.next(g);
     ahead = cur;
-    ahead.next(g);
-    ahead.next(g);
-    int stage = 0;
+    for (int i = 0; i < 4; ++i) ahead.next(g);
+    int stage = grp;
     uint32_t phase = 0;
+    if (stage >= g.np) {    // np >= 2: never, kept for clarity
+      stage -= g.np;
+      phase ^= 1;
+    }
     // One step: `use` holds this step's values; the values of the step two
     // ahead are loaded into `fill` (free since the previous step).  Three
     // sets rotate by name, so no register is copied while its load is in
@@ -494,11 +502,14 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       fence_proxy_async_smem();     // generic-proxy writes -> visible to the MMA
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(deq + stage));
-      if (++stage == g.np) {
-        stage = 0;
+      stage += 2;
+      if (stage >= g.np) {
+        stage -= g.np;
         phase ^= 1;
       }
       cur.next(g);
+      cur.next(g);
+      ahead.next(g);
       ahead.next(g);
       return true;
     };
@@ -506,15 +517,15 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     load_meta(cur, ma);
     StepIt one = cur;
     one.next(g);
+    one.next(g);
     load_meta(one, mb);
     while (step(ma, mc) && step(mb, ma) && step(mc, mb)) {
     }
   } else {
     // ---------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM sub-partition of this warp
-    const int half = (warp - HQ_EPI_WARP0) >> 2;   // chunks half, half + 2, ...
     const int row = q * 32 + lane;          // accumulator row = output channel in the tile
-    const uint32_t buf = base + g.off_epi + static_cast<uint32_t>(warp - HQ_EPI_WARP0) * HQ_EPI_BUF;
+    const uint32_t buf0 = base + g.off_epi + static_cast<uint32_t>(warp - HQ_EPI_WARP0) * 2 * HQ_EPI_BUF;
     int acc = 0;
     uint32_t aphase = 0;
     for (int u = blockIdx.x; u < g.units; u += gridDim.x) {
@@ -527,9 +538,28 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       const int tok0 = t.ttile * g.bn;
       float* const part =
           g.splits > 1 ? g.ws + static_cast<int64_t>(t.tile * g.splits + t.split) * g.bn * 128 : nullptr;
-      for (int c0 = half * 32; c0 < g.bn; c0 += 64) {
-        const int width = min(32, g.bn - c0);
-        uint32_t r[32];
+      // One 32-token chunk: the fp32 partial (split contraction) or bf16
+      // through staging buffer `b` (free once its previous store has read it:
+      // at most the other buffer's store may still be reading).
+      auto emit = [&](const uint32_t (&r)[32], int c0, int width, uint32_t b) {
+        if (part != nullptr) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < width) part[static_cast<int64_t>(c0 + j) * 128 + row] = __uint_as_float(r[j]);
+          return;
+        }
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+        stage_pairs(b, r, width, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (ch0 < g.n_out && tok0 + c0 < g.M)      // boxes wholly outside are not issued
+            tma_store_2d(width == 32 ? &tm_c32 : &tm_c16, b, 2 * ch0, tok0 + c0);
+          bulk_commit_group();                       // (an empty group keeps the count in step)
+        }
+      };
+      auto load = [&](uint32_t (&r)[32], int c0, int width) {
         if (width == 32) {
           tmem_ld_32x32b_x32(tb + c0, r);
         } else {
@@ -540,22 +570,16 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
 #pragma unroll
           for (int j = 16; j < 32; ++j) r[j] = 0;
         }
+      };
+      for (int c0 = 0; c0 < g.bn; c0 += 64) {
+        const int w0 = min(32, g.bn - c0);
+        const int w1 = min(32, g.bn - c0 - 32);     // <= 0: no second chunk
+        uint32_t r0[32], r1[32];
+        load(r0, c0, w0);
+        if (w1 > 0) load(r1, c0 + 32, w1);
         tmem_ld_wait();
-        if (part != nullptr) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < width) part[static_cast<int64_t>(c0 + j) * 128 + row] = __uint_as_float(r[j]);
-        } else {
-          if (lane == 0) bulk_wait_group_read<0>();    // the previous store has read the buffer
-          __syncwarp();
-          stage_pairs(buf, r, width, lane);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && ch0 < g.n_out && tok0 + c0 < g.M) {     // boxes wholly outside are not issued
-            tma_store_2d(width == 32 ? &tm_c32 : &tm_c16, buf, 2 * ch0, tok0 + c0);
-            bulk_commit_group();
-          }
-        }
+        emit(r0, c0, w0, buf0);
+        if (w1 > 0) emit(r1, c0 + 32, w1, buf0 + HQ_EPI_BUF);
       }
       tc_fence_before();
       __syncwarp();
@@ -710,9 +734,9 @@ HqqPlan plan_hqq(int64_t M, int64_t n_out, int64_t kc, int sm_count, bool allow_
   p.units = static_cast<int>(tiles * p.splits);
   p.grid = std::min(p.units, sm_count);
   const int stage = HQ_A_BYTES + p.bn * 128 + HQ_W_BYTES;
-  const int avail = HQ_SMEM_LIMIT - 1024 - HQ_EPI_WARPS * HQ_EPI_BUF - HQ_BAR_BYTES;
+  const int avail = HQ_SMEM_LIMIT - 1024 - 2 * HQ_EPI_WARPS * HQ_EPI_BUF - HQ_BAR_BYTES;
   p.np = std::min(HQ_MAX_NP, avail / stage);
-  p.smem = 1024 + static_cast<size_t>(p.np) * stage + HQ_EPI_WARPS * HQ_EPI_BUF + HQ_BAR_BYTES;
+  p.smem = 1024 + static_cast<size_t>(p.np) * stage + 2 * HQ_EPI_WARPS * HQ_EPI_BUF + HQ_BAR_BYTES;
   return p;
 }
 
@@ -804,7 +828,7 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   g.units = p.units;
   g.np = p.np;
   g.off_epi = static_cast<uint32_t>(p.np) * (HQ_A_BYTES + p.bn * 128 + HQ_W_BYTES);
-  g.off_bar = g.off_epi + HQ_EPI_WARPS * HQ_EPI_BUF;
+  g.off_bar = g.off_epi + 2 * HQ_EPI_WARPS * HQ_EPI_BUF;
   g.scale = static_cast<const uint16_t*>(scale);
   g.zero = static_cast<const uint16_t*>(zero);
   g.out = static_cast<uint16_t*>(out);
