@@ -331,17 +331,12 @@ DQ_API dq_status dq_fp8_linear(const uint8_t* A, const float* s_row, int64_t M, 
  *
  * Requirements: group in {32, 64, 128, 256}; K % group == 0; N % 8 == 0;
  * M >= 0 (M == 0 launches nothing); all pointers 16-byte aligned.
- * workspace: optional caller-owned device scratch that lets few-token calls
- * split the contraction over more SMs (the split partial sums are added in
- * a fixed order, so results do not depend on timing).  Its usable size is
- * dq_hqq_workspace_size(); NULL or a smaller buffer disables splitting.  Its
- * first bytes hold one arrival counter per tile, the rest the split partial
- * sums.  The counters must be zero when a call starts and every completed
- * call leaves them zero; the partial sums are left behind.  So a workspace
- * ZERO-FILLED once serves any number of calls of one shape (M, N, K,
- * direction); for another shape zero it again or keep one per shape, and
- * re-zero it after DQ_ERR_TIMEOUT.  Calls that may run at the same time must
- * not share a workspace.
+ * workspace / workspace_bytes: accepted for interface stability and not
+ * used; dq_hqq_workspace_size() returns 0.  Few-token calls split the
+ * contraction over a thread-block cluster of up to 8 CTAs per output tile,
+ * which add their partial sums through distributed shared memory in split
+ * order (results do not depend on timing, and concurrent calls share no
+ * state).
  * ------------------------------------------------------------------------ */
 enum { DQ_HQQ_S4 = 1 };
 
@@ -386,11 +381,16 @@ DQ_API dq_status dq_hqq_linear_t(const void* y_bf16, int64_t M, const uint8_t* p
  *   int8 bytes).  meta nibbles must have p0 < p1 (as dq_s24_compress writes
  *   them); other nibbles give unspecified (but in-bounds) results.
  *   Requirements: K % 128 == 0, N % 8 == 0, M >= 0, pointers 16-byte
- *   aligned.  workspace / workspace_bytes: as for dq_hqq_linear
- *   (dq_s24_workspace_size; its first bytes are the split arrival counters,
- *   eight per tile, which every completed call leaves zero; one zero-filled
- *   workspace per shape; int32 partials, so results never depend on the
- *   split).
+ *   aligned.  workspace: optional caller-owned device scratch that lets
+ *   few-token calls split the contraction over more SMs; its usable size is
+ *   dq_s24_workspace_size(), and NULL or a smaller buffer disables
+ *   splitting.  Its first bytes are the split arrival counters, eight per
+ *   tile, which must be zero when a call starts and which every completed
+ *   call leaves zero; the rest holds int32 partial sums (exact, so results
+ *   never depend on the split).  One zero-filled workspace serves any number
+ *   of calls of one shape; re-zero it for another shape or after
+ *   DQ_ERR_TIMEOUT, and do not share it between calls that may run at the
+ *   same time.
  * ------------------------------------------------------------------------ */
 DQ_API dq_status dq_s24_compress(const int8_t* wq, int64_t N, int64_t K, int8_t* values, uint8_t* meta,
                                  int32_t* violations, dq_stream_t stream);

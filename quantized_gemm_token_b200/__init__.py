@@ -545,9 +545,10 @@ def _hqq_call(fn, name, x, packed, scale, zero, group, signed, out, workspace, s
 def dq_hqq_linear(x, packed, scale, zero, group: int, signed: bool = False, out=None, workspace=None,
                   stream=None):
     """out[M, N] = x[M, K] @ w^T with w the dequantized int4 weight [N, K]
-    (dequantization fused into the tensor-core GEMM).  `workspace`: optional
-    uint8 CUDA tensor (dq_hqq_workspace_size) for few-token calls, zero-filled
-    once and kept for calls of this one shape."""
+    (dequantization fused into the tensor-core GEMM).  `workspace` is
+    accepted and unused: few-token calls split the contraction over a
+    cluster of CTAs that reduce through distributed shared memory
+    (dq_hqq_workspace_size returns 0)."""
     return _hqq_call(lib.dq_hqq_linear, "dq_hqq_linear", x, packed, scale, zero, group, signed, out,
                      workspace, stream, False)
 
@@ -562,43 +563,25 @@ def dq_hqq_linear_t(y, packed, scale, zero, group: int, signed: bool = False, ou
 class HqqLinear:
     """Weight-only int4 linear: packed u4 / s4 codes with bf16 scale and zero
     point per group of in-features (held group-major, [K/group, N]).
-    forward(x) = x @ w^T, backward_input(g) = g @ w; the workspace for
-    few-token calls is kept per token count."""
+    forward(x) = x @ w^T, backward_input(g) = g @ w.  No workspace: the
+    few-token split contraction reduces inside a cluster of CTAs."""
 
     def __init__(self, packed, scale, zero, group: int, signed: bool = False):
         self.packed, self.scale, self.zero, self.group, self.signed = packed, scale, zero, group, signed
         self.N, self.K = packed.shape[0], packed.shape[1] * 2
-        self._ws = {}
 
     @classmethod
     def from_codes(cls, codes: torch.Tensor, scale, zero, group: int, signed: bool = False):
         """codes int8 [N, K]; scale, zero bf16 per channel [N, K/group]."""
         return cls(dq_hqq_pack(codes), dq_hqq_group_major(scale), dq_hqq_group_major(zero), group, signed)
 
-    def _workspace(self, M, transposed, device, st):
-        key = (M, transposed)
-        if key not in self._ws:
-            if len(self._ws) >= 16:                 # keep the most recent shapes only
-                self._ws.pop(next(iter(self._ws)))
-            n = dq_hqq_workspace_size(M, self.N, self.K, transposed)
-            self._ws[key] = _scratch((n,), torch.uint8, device, st, zero=True) if n else None
-        return self._ws[key]
-
     def __call__(self, x: torch.Tensor, out: torch.Tensor = None, stream=None):
-        st = _stream_obj(stream)
-        ws = self._workspace(x.shape[0], False, x.device, st)
-        y = dq_hqq_linear(x, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
-                          workspace=ws, stream=st)
-        _used_on(st, ws)
-        return y
+        return dq_hqq_linear(x, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
+                             stream=stream)
 
     def backward_input(self, grad_out: torch.Tensor, out: torch.Tensor = None, stream=None):
-        st = _stream_obj(stream)
-        ws = self._workspace(grad_out.shape[0], True, grad_out.device, st)
-        y = dq_hqq_linear_t(grad_out, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
-                            workspace=ws, stream=st)
-        _used_on(st, ws)
-        return y
+        return dq_hqq_linear_t(grad_out, self.packed, self.scale, self.zero, self.group, self.signed, out=out,
+                               stream=stream)
 
 
 # ---------------------------------------------------------------- 2:4 sparse

@@ -31,13 +31,16 @@
 // The weight is the A operand (128 output channels per tile) and the tokens
 // the B operand (up to 256): the dequantization work per MMA flop is then as
 // small as a 128-row tile allows, and few-token calls need no padding to 128.
-// Few tiles: the contraction is split over S CTAs per tile; each split
-// writes an fp32 partial tile to a workspace and the last split to arrive
-// (an arrival counter per 32-channel slice) adds the S partials in split
-// order, so the result does not depend on timing.
+// Few tiles: the contraction is split over S <= 8 CTAs per tile, launched as
+// one thread-block cluster; each split leaves its fp32 partial tile in its
+// own shared memory and, after a cluster barrier, every CTA of the cluster
+// adds all S partials (read through distributed shared memory, in split
+// order, so the result does not depend on timing) for its share of the
+// tile's tokens.  No global workspace and no atomics.
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <type_traits>
 
 #include "internal.h"
@@ -78,8 +81,6 @@ struct HqqArgs {
   const uint16_t* scale;  // bf16 [K / group, n_w], group-major
   const uint16_t* zero;   // bf16 [K / group, n_w]
   uint16_t* out;          // bf16 [M, n_out]
-  float* ws;              // split partials: [tile][split][bn][128] fp32
-  uint32_t* cnt;          // arrival counters: [tile][4]
   WaitCtl wait;
 };
 
@@ -345,13 +346,11 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
   uint64_t* const drain = acce + 2;
   uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* const last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    *last_flag = 0;
     for (int i = 0; i < g.np; ++i) {
       mbar_init(smem_u32(full + i), 1);
       mbar_init(smem_u32(deq + i), HQ_DEQ_WARPS);
@@ -536,16 +535,17 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * HQ_ACC_COLS);
       const int ch0 = t.ntile * 128 + q * 32;
       const int tok0 = t.ttile * g.bn;
-      float* const part =
-          g.splits > 1 ? g.ws + static_cast<int64_t>(t.tile * g.splits + t.split) * g.bn * 128 : nullptr;
-      // One 32-token chunk: the fp32 partial (split contraction) or bf16
-      // through staging buffer `b` (free once its previous store has read it:
-      // at most the other buffer's store may still be reading).
+      // One 32-token chunk: with a split contraction the fp32 partial into
+      // this CTA's shared memory ([bn][128], at the start of the stage ring:
+      // the CTA's only unit, so every stage has been consumed once its
+      // accumulator is ready), else bf16 through staging buffer `b` (free
+      // once its previous store has read it: at most the other buffer's
+      // store may still be reading).
       auto emit = [&](const uint32_t (&r)[32], int c0, int width, uint32_t b) {
-        if (part != nullptr) {
+        if (g.splits > 1) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j < width) part[static_cast<int64_t>(c0 + j) * 128 + row] = __uint_as_float(r[j]);
+            if (j < width) pipe::sts32(base + static_cast<uint32_t>((c0 + j) * 128 + row) * 4u, r[j]);
           return;
         }
         if (lane == 0) bulk_wait_group_read<1>();
@@ -588,7 +588,6 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
         acc = 0;
         aphase ^= 1;
       }
-      if (part != nullptr) __threadfence();     // the partial tile is published below
     }
     if (lane == 0) bulk_wait_group<0>();         // every output store complete
     __syncwarp();
@@ -599,56 +598,40 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, HQ_TMEM_COLS);
 
-  // Split contraction (one unit per CTA): the last split of a tile to arrive
-  // adds the tile's partial sums in split order, with every thread of the CTA.
-  if (g.splits > 1 && blockIdx.x < g.units) {
+  // Split contraction (one unit per CTA, the tile's S splits one cluster):
+  // once every CTA of the cluster holds its partial tile, CTA r adds all S
+  // partials for tokens [r * rows, (r + 1) * rows) of the tile, four
+  // channels per thread, and stores them as bf16.  The second cluster
+  // barrier keeps every CTA's shared memory alive until its peers have read
+  // it.
+  if (g.splits > 1) {
+    cluster_sync_all();
     const Unit t = decode_unit(g, blockIdx.x);
-    if (threadIdx.x == 0) {
-      int last = 0;
-      if (!*abort_flag) {
-        __threadfence();
-        last = atomicAdd(g.cnt + t.tile * 4, 1u) == static_cast<uint32_t>(g.splits - 1) ? 1 : 0;
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int rows = (g.bn + g.splits - 1) / g.splits;
+    const int r0 = rank * rows;
+    const int r1 = min(g.bn, r0 + rows);
+    for (int i = threadIdx.x; i < (r1 - r0) * 32; i += HQ_THREADS) {
+      const int tok = r0 + (i >> 5);
+      const int quad = i & 31;                        // channels 4 * quad .. + 3 of the tile
+      const uint32_t off = base + static_cast<uint32_t>(tok * 128 + 4 * quad) * 4u;
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp = 0; sp < g.splits; ++sp) {
+        const float4 v = ld_shared_cluster_f4(map_to_rank(off, static_cast<uint32_t>(sp)));
+        sum.x += v.x;
+        sum.y += v.y;
+        sum.z += v.z;
+        sum.w += v.w;
       }
-      *last_flag = last;
-    }
-    __syncthreads();
-    if (*last_flag) {
-      __threadfence();
-      const float* const tile_ws = g.ws + static_cast<int64_t>(t.tile) * g.splits * g.bn * 128;
-      const int quad = threadIdx.x & 31;                 // channels 4 * quad .. + 3
+      const int m = t.ttile * g.bn + tok;
       const int ch = t.ntile * 128 + 4 * quad;
-      constexpr int ROWS = HQ_THREADS / 32;              // token rows per pass
-      for (int tok0 = (threadIdx.x >> 5) * 4; tok0 < g.bn; tok0 += ROWS * 4) {
-        // four tokens at a time, every split's loads in flight together
-        float4 sum[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) sum[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int sp = 0; sp < g.splits; ++sp) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            if (tok0 + i < g.bn) {
-              const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                                          tile_ws + (static_cast<int64_t>(sp) * g.bn + tok0 + i) * 128) + quad);
-              sum[i].x += v.x;
-              sum[i].y += v.y;
-              sum[i].z += v.z;
-              sum[i].w += v.w;
-            }
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int m = t.ttile * g.bn + tok0 + i;
-          if (tok0 + i < g.bn && m < g.M && ch < g.n_out) {
-            const uint32_t lo = bf16_bits(sum[i].x) | (bf16_bits(sum[i].y) << 16);
-            const uint32_t hi = bf16_bits(sum[i].z) | (bf16_bits(sum[i].w) << 16);
-            *reinterpret_cast<uint2*>(g.out + static_cast<int64_t>(m) * g.n_out + ch) = make_uint2(lo, hi);
-          }
-        }
+      if (m < g.M && ch < g.n_out) {                  // n_out % 8 == 0: the quad is all in or all out
+        const uint32_t lo = bf16_bits(sum.x) | (bf16_bits(sum.y) << 16);
+        const uint32_t hi = bf16_bits(sum.z) | (bf16_bits(sum.w) << 16);
+        *reinterpret_cast<uint2*>(g.out + static_cast<int64_t>(m) * g.n_out + ch) = make_uint2(lo, hi);
       }
-      if (threadIdx.x == 0) g.cnt[t.tile * 4] = 0u;     // the workspace is left zeroed
     }
+    cluster_sync_all();
   }
 }
 
@@ -709,12 +692,16 @@ namespace {
 
 struct HqqPlan {
   int bn, tt, nt, ks, splits, units, grid, np;
-  size_t cnt_bytes, ws_bytes, smem;
+  size_t smem;
 };
+
+constexpr int HQ_MAX_SPLITS = 8;           // portable cluster size
 
 // Tiles: 128 output channels x bn tokens, bn = the token count split evenly
 // over ceil(M / 256) tiles and rounded up to 16.  When the tiles cannot fill
-// the SMs the contraction is split (at least 4 steps of 64 per split).
+// the SMs the contraction is split over a cluster of up to 8 CTAs (at least
+// 4 steps of 64 per split; the partial tile, bn x 128 fp32, must fit in the
+// stage ring).
 HqqPlan plan_hqq(int64_t M, int64_t n_out, int64_t kc, int sm_count, bool allow_split) {
   HqqPlan p{};
   p.nt = static_cast<int>((n_out + 127) / 128);
@@ -727,16 +714,19 @@ HqqPlan plan_hqq(int64_t M, int64_t n_out, int64_t kc, int sm_count, bool allow_
   if (allow_split && tiles < sm_count) {
     int s = static_cast<int>(sm_count / tiles);
     s = std::min(s, std::max(1, p.ks / 4));
-    p.splits = std::max(1, std::min(s, 32));
+    p.splits = std::max(1, std::min(s, HQ_MAX_SPLITS));
   }
-  p.cnt_bytes = (static_cast<size_t>(tiles) * 4 * sizeof(uint32_t) + 255) / 256 * 256;
-  p.ws_bytes = p.splits > 1 ? p.cnt_bytes + static_cast<size_t>(tiles) * p.splits * p.bn * 128 * sizeof(float) : 0;
   p.units = static_cast<int>(tiles * p.splits);
   p.grid = std::min(p.units, sm_count);
   const int stage = HQ_A_BYTES + p.bn * 128 + HQ_W_BYTES;
   const int avail = HQ_SMEM_LIMIT - 1024 - 2 * HQ_EPI_WARPS * HQ_EPI_BUF - HQ_BAR_BYTES;
   p.np = std::min(HQ_MAX_NP, avail / stage);
   p.smem = 1024 + static_cast<size_t>(p.np) * stage + 2 * HQ_EPI_WARPS * HQ_EPI_BUF + HQ_BAR_BYTES;
+  if (p.splits > 1 && p.np * stage < p.bn * 128 * 4) {    // no room for the partial tile
+    p.splits = 1;
+    p.units = static_cast<int>(tiles);
+    p.grid = std::min(p.units, sm_count);
+  }
   return p;
 }
 
@@ -758,19 +748,54 @@ dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const CUtenso
   const dq_status st = smem_limit_once(reinterpret_cast<const void*>(&hqq_gemm_kernel<TRANS, S4>), HQ_SMEM_LIMIT);
   if (st != DQ_OK) return st;
   // Programmatic stream serialization: the prologue (barriers, tensor-memory
-  // allocation) overlaps the tail of the previous kernel of the stream.
+  // allocation) overlaps the tail of the previous kernel of the stream.  A
+  // split contraction runs each tile's splits as one cluster.
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(g.splits);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(HQ_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = g.splits > 1 ? 2 : 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, hqq_gemm_kernel<TRANS, S4>, tx, tw, tc32, tc16, g);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
+}
+
+std::atomic<int> g_cluster_ok[64] = {};   // per device: 0 unknown, 1 yes, 2 no
+
+// Whether a cluster of HQ_MAX_SPLITS CTAs with a full SM's shared memory
+// each can be resident on the current device (then every smaller split
+// cluster can too).  Asked once per device.
+bool split_clusters_fit(const DeviceInfo& d) {
+  int v = g_cluster_ok[d.device & 63].load(std::memory_order_relaxed);
+  if (v == 0) {
+    v = 2;
+    if (smem_limit_once(reinterpret_cast<const void*>(&hqq_gemm_kernel<false, false>), HQ_SMEM_LIMIT) == DQ_OK) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = HQ_MAX_SPLITS;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(HQ_MAX_SPLITS);
+      cfg.blockDim = dim3(HQ_THREADS);
+      cfg.dynamicSmemBytes = HQ_SMEM_LIMIT;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, hqq_gemm_kernel<false, false>, &cfg) == cudaSuccess && n >= 1) v = 1;
+      else (void)cudaGetLastError();
+    }
+    g_cluster_ok[d.device & 63].store(v, std::memory_order_relaxed);
+  }
+  return v == 1;
 }
 
 dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* packed, const void* scale,
@@ -788,9 +813,9 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
 
   const int64_t n_out = trans ? K : N;
   const int64_t kc = trans ? N : K;
-  HqqPlan p = plan_hqq(M, n_out, kc, d->sm_count, true);
-  if (p.splits > 1 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < p.ws_bytes))
-    p = plan_hqq(M, n_out, kc, d->sm_count, false);
+  (void)workspace;          // kept for the interface: the split contraction needs none
+  (void)workspace_bytes;
+  const HqqPlan p = plan_hqq(M, n_out, kc, d->sm_count, split_clusters_fit(*d));
 
   CUtensorMap tx, tw;
   // activations / output gradient: bf16 [M, kc] as bytes, 64-element k
@@ -832,10 +857,6 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   g.scale = static_cast<const uint16_t*>(scale);
   g.zero = static_cast<const uint16_t*>(zero);
   g.out = static_cast<uint16_t*>(out);
-  if (p.splits > 1) {
-    g.cnt = static_cast<uint32_t*>(workspace);
-    g.ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.cnt_bytes);
-  }
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
   const bool s4 = (flags & DQ_HQQ_S4) != 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -912,12 +933,14 @@ DQ_API dq_status dq_hqq_group_major(const void* src_bf16, int64_t N, int64_t G, 
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 
+// The split contraction reduces through distributed shared memory: no call
+// needs a workspace (the query stays for the interface).
 DQ_API size_t dq_hqq_workspace_size(int64_t M, int64_t N, int64_t K, int transposed) {
-  if (M <= 0 || N <= 0 || K <= 0) return 0;
-  DeviceInfo* d = nullptr;
-  if (current_device(&d) != DQ_OK) return 0;
-  const HqqPlan p = plan_hqq(M, transposed ? K : N, transposed ? N : K, d->sm_count, true);
-  return p.ws_bytes;
+  (void)M;
+  (void)N;
+  (void)K;
+  (void)transposed;
+  return 0;
 }
 
 DQ_API dq_status dq_hqq_linear(const void* x_bf16, int64_t M, const uint8_t* packed, const void* scale_bf16,

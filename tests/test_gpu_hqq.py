@@ -61,11 +61,6 @@ def _dev_weights(d, packed):
     return to_dev(packed), to_dev_bf16(d["scale"].T.copy()), to_dev_bf16(d["zero"].T.copy())
 
 
-def _ws(M, N, K, transposed):
-    n = dq.dq_hqq_workspace_size(M, N, K, transposed)
-    return torch.zeros((max(n, 1),), dtype=torch.uint8, device="cuda") if n else None
-
-
 # ---------------------------------------------------------------- format
 
 @pytest.mark.parametrize("R,C,signed", [(1, 2, False), (7, 40, True), (4096, 4096, False), (33, 4098, True)])
@@ -102,18 +97,18 @@ FWD = [  # M, N, K, group, signed
     (200, 384, 512, 32, False),       # 208-token tiles
     (300, 128, 256, 256, True),       # two token tiles
     (257, 136, 96, 32, False),        # K = 96: half of the last step is padding
-    (64, 1024, 2048, 128, True),
+    (64, 1024, 2048, 128, True),      # eight splits (one cluster of 8 CTAs per tile)
+    (40, 256, 2048, 64, False),       # eight splits of a 48-token tile: 6 tokens per CTA's reduction
+    (1, 128, 4096, 32, True),         # one token, one tile, eight splits
 ]
 
 
 @pytest.mark.parametrize("M,N,K,group,signed", FWD)
-@pytest.mark.parametrize("use_ws", [True, False])
-def test_linear_matches_oracle(M, N, K, group, signed, use_ws):
+def test_linear_matches_oracle(M, N, K, group, signed):
     d = synth.hqq(seed=M + N, M=M, N=N, K=K, group=group, signed=signed)
     packed, w = _weights(d)
     pk, sc, ze = _dev_weights(d, packed)
-    ws = _ws(M, N, K, False) if use_ws else None
-    out = dq.dq_hqq_linear(to_dev_bf16(d["x"]), pk, sc, ze, group, signed=signed, workspace=ws)
+    out = dq.dq_hqq_linear(to_dev_bf16(d["x"]), pk, sc, ze, group, signed=signed)
     exact = oracle.hqq_linear_f64(d["x"], w)
     bound = np.abs(_vals(d["x"])) @ np.abs(_vals(w)).T
     _assert_close(bf16_bits(out), exact, bound)
@@ -136,8 +131,7 @@ def test_one_hot_reads_dequantized_weight_exactly(signed):
     ks = np.arange(0, K, 3)
     x = np.zeros((len(ks), K), np.float32)
     x[np.arange(len(ks)), ks] = 1.0
-    out = dq.dq_hqq_linear(to_dev_bf16(synth.f32_to_bf16_bits(x)), pk, sc, ze, group, signed=signed,
-                           workspace=_ws(len(ks), N, K, False))
+    out = dq.dq_hqq_linear(to_dev_bf16(synth.f32_to_bf16_bits(x)), pk, sc, ze, group, signed=signed)
     assert np.array_equal(bf16_bits(out), w[:, ks].T)
 
 
@@ -148,7 +142,7 @@ def test_linear_full_size_every_token(M):
     d = synth.hqq(seed=M, M=M, N=N, K=K, group=128)
     packed, w = _weights(d)
     pk, sc, ze = _dev_weights(d, packed)
-    out = dq.dq_hqq_linear(to_dev_bf16(d["x"]), pk, sc, ze, 128, workspace=_ws(M, N, K, False))
+    out = dq.dq_hqq_linear(to_dev_bf16(d["x"]), pk, sc, ze, 128)
     # every token (M <= 1024)
     exact = oracle.hqq_linear_f64(d["x"], w)
     bound = np.abs(_vals(d["x"])) @ np.abs(_vals(w)).T
@@ -156,18 +150,21 @@ def test_linear_full_size_every_token(M):
 
 
 def test_split_contraction_is_deterministic():
+    """The few-token split contraction (a cluster of CTAs per tile adding
+    their partials in split order) gives identical bits on every call, and
+    needs no workspace (a caller's buffer is accepted and ignored)."""
     M, N, K = 16, 4096, 4096
+    assert dq.dq_hqq_workspace_size(M, N, K) == 0
     d = synth.hqq(seed=21, M=M, N=N, K=K, group=128)
     packed, _ = _weights(d)
     pk, sc, ze = _dev_weights(d, packed)
     x = to_dev_bf16(d["x"])
-    ws = _ws(M, N, K, False)
-    assert ws is not None
-    a = bf16_bits(dq.dq_hqq_linear(x, pk, sc, ze, 128, workspace=ws))
-    b = bf16_bits(dq.dq_hqq_linear(x, pk, sc, ze, 128, workspace=ws))
-    assert np.array_equal(a, b)
-    # the arrival counters (32 channel tiles x 4 slices, at the start) are zero again
-    assert int(ws[:32 * 4 * 4].count_nonzero()) == 0
+    junk = torch.full((1 << 20,), 0x5A, dtype=torch.uint8, device="cuda")
+    a = bf16_bits(dq.dq_hqq_linear(x, pk, sc, ze, 128))
+    b = bf16_bits(dq.dq_hqq_linear(x, pk, sc, ze, 128, workspace=junk))
+    c = bf16_bits(dq.dq_hqq_linear(x, pk, sc, ze, 128))
+    assert np.array_equal(a, b) and np.array_equal(a, c)
+    assert int((junk != 0x5A).count_nonzero()) == 0
 
 
 # ---------------------------------------------------------------- transposed
@@ -177,18 +174,17 @@ TRANS = [  # M, N, K, group, signed
     (33, 264, 320, 64, True),
     (200, 384, 512, 32, False),
     (5, 72, 192, 64, False),          # contraction 72: a ragged step; 192 outputs: a ragged tile
+    (24, 2048, 256, 64, True),        # eight splits of a 32-token tile
 ]
 
 
 @pytest.mark.parametrize("M,N,K,group,signed", TRANS)
-@pytest.mark.parametrize("use_ws", [True, False])
-def test_linear_t_matches_oracle(M, N, K, group, signed, use_ws):
+def test_linear_t_matches_oracle(M, N, K, group, signed):
     d = synth.hqq(seed=M + K, M=M, N=N, K=K, group=group, signed=signed)
     packed, w = _weights(d)
     pk, sc, ze = _dev_weights(d, packed)
     y = synth.normal_bf16((M, N), 1.0, 300 + M)
-    ws = _ws(M, N, K, True) if use_ws else None
-    out = dq.dq_hqq_linear_t(to_dev_bf16(y), pk, sc, ze, group, signed=signed, workspace=ws)
+    out = dq.dq_hqq_linear_t(to_dev_bf16(y), pk, sc, ze, group, signed=signed)
     exact = oracle.hqq_linear_t_f64(y, w)
     bound = np.abs(_vals(y)) @ np.abs(_vals(w))
     _assert_close(bf16_bits(out), exact, bound)
@@ -203,8 +199,7 @@ def test_one_hot_t_reads_dequantized_weight_exactly(signed):
     ns = np.arange(N)
     y = np.zeros((N, N), np.float32)
     y[ns, ns] = 1.0
-    out = dq.dq_hqq_linear_t(to_dev_bf16(synth.f32_to_bf16_bits(y)), pk, sc, ze, group, signed=signed,
-                             workspace=_ws(N, N, K, True))
+    out = dq.dq_hqq_linear_t(to_dev_bf16(synth.f32_to_bf16_bits(y)), pk, sc, ze, group, signed=signed)
     assert np.array_equal(bf16_bits(out), w)
 
 
@@ -214,7 +209,7 @@ def test_linear_t_full_size_every_token():
     packed, w = _weights(d)
     pk, sc, ze = _dev_weights(d, packed)
     y = synth.normal_bf16((M, N), 1.0, 78)
-    out = dq.dq_hqq_linear_t(to_dev_bf16(y), pk, sc, ze, 128, workspace=_ws(M, N, K, True))
+    out = dq.dq_hqq_linear_t(to_dev_bf16(y), pk, sc, ze, 128)
     # every token
     exact = oracle.hqq_linear_t_f64(y, w)
     bound = np.abs(_vals(y)) @ np.abs(_vals(w))
