@@ -303,26 +303,14 @@ __device__ __forceinline__ uint32_t bf16_bits(float f) {
   return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
-// Writes `width` (16 or 32) tokens of one output channel per lane as bf16
-// into the staging buffer `buf` (row j = token j, 64 B = the warp's 32
-// channels): lanes exchange values in pairs so that each lane writes two
-// neighbouring channels of one token (4 bytes; rows j and j + 1 of one
-// instruction cover all 32 banks).
+// Converts `width` (16 or 32) fp32 accumulators of one output channel per
+// lane to bf16 pairs and stages them (row j = token j of a 32 x 32 block).
 __device__ __forceinline__ void stage_pairs(uint32_t buf, const uint32_t (&r)[32], int width, int lane) {
-  const bool odd = lane & 1;
-  const uint32_t col = static_cast<uint32_t>(lane & ~1) * 2u;
-  const uint32_t sel = odd ? 0x3276u : 0x5410u;
+  uint32_t pk[16];
 #pragma unroll
-  for (int j = 0; j < 32; j += 2) {
-    if (j < width) {
-      uint32_t pk;   // lo = bf16(token j), hi = bf16(token j + 1) of this lane's channel
-      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(pk) : "f"(__uint_as_float(r[j + 1])), "f"(__uint_as_float(r[j])));
-      const uint32_t recv = __shfl_xor_sync(0xffffffffu, pk, 1);
-      // even lane: (own token j, partner's token j); odd: (partner's j + 1, own j + 1)
-      const uint32_t v = __byte_perm(pk, recv, sel);
-      pipe::sts32(buf + static_cast<uint32_t>(j + (odd ? 1 : 0)) * 64u + col, v);
-    }
-  }
+  for (int i = 0; i < 16; ++i)
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(pk[i]) : "f"(__uint_as_float(r[2 * i + 1])), "f"(__uint_as_float(r[2 * i])));
+  pipe::stage_bf16_pairs(buf, pk, width, lane);
 }
 
 template <bool TRANS, bool S4>

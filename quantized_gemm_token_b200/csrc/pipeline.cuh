@@ -72,6 +72,27 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+// Writes `width` (16 or 32) tokens of one output channel per lane, given as
+// bf16 pairs (pk[i]: token 2i in the low half, 2i + 1 in the high half),
+// into a staging buffer of 32 rows x 64 B (row j = token j; the warp's 32
+// lanes = 32 neighbouring channels) for one 2-D TMA store.  Lanes exchange
+// values in pairs so that each lane writes two neighbouring channels of one
+// token (4 bytes; rows j and j + 1 of one instruction cover all 32 banks).
+__device__ __forceinline__ void stage_bf16_pairs(uint32_t buf, const uint32_t (&pk)[16], int width, int lane) {
+  const bool odd = lane & 1;
+  const uint32_t col = static_cast<uint32_t>(lane & ~1) * 2u;
+  const uint32_t sel = odd ? 0x3276u : 0x5410u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (2 * i < width) {
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, pk[i], 1);
+      // even lane: (own token 2i, partner's token 2i); odd: (partner's 2i + 1, own 2i + 1)
+      const uint32_t v = __byte_perm(pk[i], recv, sel);
+      sts32(buf + static_cast<uint32_t>(2 * i + (odd ? 1 : 0)) * 64u + col, v);
+    }
+  }
+}
+
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128B-swizzled
 // K-major tile (rows of 128 B; the chunk index is XORed with r mod 8, as a
 // SWIZZLE_128B tensor copy lays it out).  The tile must be 1024-byte aligned.

@@ -29,7 +29,8 @@
 //               int32 accumulator in TMEM, double-buffered).
 //   warps 2..9  epilogue, two warps per TMEM sub-partition taking alternate
 //               32-token chunks: out = bf16((acc * s_row) * s_col + bias),
-//               each op rounded on its own, or the raw int32.
+//               each op rounded on its own, staged as a 32 x 32 block and
+//               written by one TMA store; or the raw int32.
 // Few tiles: the contraction is split; int32 partial tiles go to a
 // workspace and, per epilogue warp, the last split of a tile to arrive adds
 // them (exact, in split order) before the epilogue arithmetic.
@@ -58,6 +59,7 @@ constexpr int S4_TMEM_COLS = 512;
 constexpr int S4_SMEM_LIMIT = 227 * 1024;
 constexpr int S4_BAR_BYTES = 1024;
 constexpr int S4_CNT_PER_TILE = 8;         // split arrival counters per tile: one per epilogue warp
+constexpr int S4_EPI_BUF = 2048;           // bf16 staging per epilogue warp: 32 tokens x 64 B
 static_assert(2 * S4_MAX_BN + 4 * 8 <= S4_TMEM_COLS, "tensor memory");
 
 struct S24Args {
@@ -65,7 +67,8 @@ struct S24Args {
   int bn;                 // tokens per tile (multiple of 16, <= S4_MAX_BN)
   int nt, tt;             // channel tiles (128), token tiles (bn)
   int splits, ks, units, np;
-  uint32_t off_bar;
+  uint32_t off_epi;       // epilogue staging buffers (after the stages)
+  uint32_t off_bar;       // barriers (after the staging buffers)
   const float* s_row;
   const float* s_col;
   const uint16_t* bias;   // bf16 bits or null
@@ -128,10 +131,14 @@ __device__ __forceinline__ float dequant(int32_t acc, float sr, float sc, bool h
   return has_bias ? __fadd_rn(f, b) : f;
 }
 
-// Epilogue of one chunk: lane = channel ch, r[j] = int32 accumulator of token
-// tok0 + j (j < width, width 16 or 32).
+// Epilogue of one chunk: lane = channel ch (the warp's channels ch_w ..
+// ch_w + 31), r[j] = int32 accumulator of token tok0 + j (j < width, width
+// 16 or 32).  bf16 goes through the warp's staging buffer `buf` (free once
+// its previous store has read it) and one TMA store of the 32 x 32 block,
+// which clips tokens >= M and channels >= N; int32 is stored directly.
 __device__ __forceinline__ void store_chunk(const S24Args& g, const uint32_t (&r)[32], int width, int tok0, int ch,
-                                            int lane) {
+                                            int ch_w, int lane, uint32_t buf, const CUtensorMap* tm32,
+                                            const CUtensorMap* tm16) {
   const bool ch_ok = ch < g.N;
   if (g.out_s32) {
     int32_t* o = static_cast<int32_t*>(g.out);
@@ -143,22 +150,24 @@ __device__ __forceinline__ void store_chunk(const S24Args& g, const uint32_t (&r
   const float sc = ch_ok ? __ldg(g.s_col + ch) : 0.0f;
   const bool has_bias = g.bias != nullptr;
   const float b = (has_bias && ch_ok) ? __uint_as_float(static_cast<uint32_t>(__ldg(g.bias + ch)) << 16) : 0.0f;
-  const bool odd = lane & 1;
-  const int ch_even = ch & ~1;
-  uint16_t* o = static_cast<uint16_t*>(g.out);
+  uint32_t pk[16];
 #pragma unroll
-  for (int j = 0; j < 32; j += 2) {
-    if (j < width) {
-      const int m0 = tok0 + j;
-      const float sr0 = m0 < g.M ? __ldg(g.s_row + m0) : 0.0f;
-      const float sr1 = m0 + 1 < g.M ? __ldg(g.s_row + m0 + 1) : 0.0f;
-      const uint32_t h0 = bf16_bits(dequant(static_cast<int32_t>(r[j]), sr0, sc, has_bias, b));
-      const uint32_t h1 = bf16_bits(dequant(static_cast<int32_t>(r[j + 1]), sr1, sc, has_bias, b));
-      const uint32_t recv = __shfl_xor_sync(0xffffffffu, odd ? h0 : h1, 1);
-      const int tok = m0 + (odd ? 1 : 0);
-      const uint32_t v = odd ? (recv | (h1 << 16)) : (h0 | (recv << 16));
-      if (ch_ok && tok < g.M) *reinterpret_cast<uint32_t*>(o + static_cast<int64_t>(tok) * g.N + ch_even) = v;
-    }
+  for (int i = 0; i < 16; ++i) {
+    const int m0 = tok0 + 2 * i;
+    const float sr0 = m0 < g.M ? __ldg(g.s_row + m0) : 0.0f;
+    const float sr1 = m0 + 1 < g.M ? __ldg(g.s_row + m0 + 1) : 0.0f;
+    const float f0 = dequant(static_cast<int32_t>(r[2 * i]), sr0, sc, has_bias, b);
+    const float f1 = dequant(static_cast<int32_t>(r[2 * i + 1]), sr1, sc, has_bias, b);
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(pk[i]) : "f"(f1), "f"(f0));
+  }
+  if (lane == 0) bulk_wait_group_read<0>();
+  __syncwarp();
+  pipe::stage_bf16_pairs(buf, pk, width, lane);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && ch_w < g.N && tok0 < g.M) {     // boxes wholly outside are not issued
+    tma_store_2d(width == 32 ? tm32 : tm16, buf, 2 * ch_w, tok0);
+    bulk_commit_group();
   }
 }
 
@@ -178,7 +187,8 @@ __device__ __forceinline__ void load_chunk(uint32_t taddr, int width, uint32_t (
 
 __global__ void __launch_bounds__(S4_THREADS, 1)
     s24_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_m, const S24Args g) {
+                    const __grid_constant__ CUtensorMap tm_m, const __grid_constant__ CUtensorMap tm_c32,
+                    const __grid_constant__ CUtensorMap tm_c16, const S24Args g) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -313,6 +323,7 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
     const int q = warp & 3;
     const int grp = ew >> 2;
     const int row = q * 32 + lane;
+    const uint32_t buf = base + g.off_epi + static_cast<uint32_t>(ew) * S4_EPI_BUF;
     int acc = 0;
     uint32_t aphase = 0;
     for (int u = blockIdx.x; u < g.units; u += gridDim.x) {
@@ -322,6 +333,7 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * g.bn);
       const int ch = t.ntile * 128 + row;
+      const int ch_w = t.ntile * 128 + q * 32;
       const int tok0 = t.ttile * g.bn;
       const int nch = (g.bn + 31) / 32;
       if (g.splits == 1) {
@@ -335,7 +347,7 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(acce + acc));
           }
-          store_chunk(g, r, width, tok0 + 32 * c, ch, lane);
+          store_chunk(g, r, width, tok0 + 32 * c, ch, ch_w, lane, buf, &tm_c32, &tm_c16);
         }
         if (grp >= nch) {                 // no chunk for this warp (bn <= 32)
           tc_fence_before();
@@ -379,7 +391,7 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
               for (int j = 0; j < 32; ++j)
                 if (j < width) r[j] = static_cast<uint32_t>(static_cast<int32_t>(r[j]) + __ldcg(src + j * 128));
             }
-            store_chunk(g, r, width, tok0 + 32 * c, ch, lane);
+            store_chunk(g, r, width, tok0 + 32 * c, ch, ch_w, lane, buf, &tm_c32, &tm_c16);
           }
           __syncwarp();
           if (lane == 0) g.cnt[t.tile * S4_CNT_PER_TILE + ew] = 0u;    // the counters are left zeroed
@@ -390,6 +402,8 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
         aphase ^= 1;
       }
     }
+    if (lane == 0) bulk_wait_group<0>();         // every output store complete
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -484,8 +498,9 @@ S24Plan plan_s24(int64_t M, int64_t N, int64_t K, int sm_count, bool allow_split
   p.units = static_cast<int>(tiles * p.splits);
   p.grid = std::min(p.units, sm_count);
   const int stage = p.bn * 128 + S4_V_BYTES + S4_M_BYTES;
-  p.np = std::min({S4_MAX_NP, (S4_SMEM_LIMIT - 1024 - S4_BAR_BYTES) / stage, (S4_TMEM_COLS - 2 * p.bn) / 4});
-  p.smem = 1024 + static_cast<size_t>(p.np) * stage + S4_BAR_BYTES;
+  p.np = std::min({S4_MAX_NP, (S4_SMEM_LIMIT - 1024 - S4_EPI_WARPS * S4_EPI_BUF - S4_BAR_BYTES) / stage,
+                   (S4_TMEM_COLS - 2 * p.bn) / 4});
+  p.smem = 1024 + static_cast<size_t>(p.np) * stage + S4_EPI_WARPS * S4_EPI_BUF + S4_BAR_BYTES;
   return p;
 }
 
@@ -555,6 +570,14 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
   st = make_tmap_u8_2d(&tm, meta, static_cast<uint64_t>(K / 8), static_cast<uint64_t>(N),
                        static_cast<uint64_t>(K / 8), 16, 128, 0);
   if (st != DQ_OK) return st;
+  // bf16 output [M, N] as bytes: 32 channels (64 B) x 32 or 16 tokens
+  CUtensorMap tc32, tc16;
+  st = make_tmap_u8_2d(&tc32, out, static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(M),
+                       static_cast<uint64_t>(N) * 2, 64, 32, 0);
+  if (st != DQ_OK) return st;
+  st = make_tmap_u8_2d(&tc16, out, static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(M),
+                       static_cast<uint64_t>(N) * 2, 64, 16, 0);
+  if (st != DQ_OK) return st;
 
   S24Args g{};
   g.M = static_cast<int>(M);
@@ -567,7 +590,8 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
   g.ks = p.ks;
   g.units = p.units;
   g.np = p.np;
-  g.off_bar = static_cast<uint32_t>(p.np) * (p.bn * 128 + S4_V_BYTES + S4_M_BYTES);
+  g.off_epi = static_cast<uint32_t>(p.np) * (p.bn * 128 + S4_V_BYTES + S4_M_BYTES);
+  g.off_bar = g.off_epi + S4_EPI_WARPS * S4_EPI_BUF;
   g.s_row = s_row;
   g.s_col = s_col;
   g.bias = out_dtype == DQ_OUT_BF16 ? static_cast<const uint16_t*>(bias_bf16) : nullptr;
@@ -593,7 +617,7 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, s24_gemm_kernel, tq, tv, tm, g);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, s24_gemm_kernel, tq, tv, tm, tc32, tc16, g);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 
