@@ -917,7 +917,21 @@ def secondary_measurements(dq, torch, peaks, probe, n):
     torch.cuda.synchronize()
     assert dq.dq_sync_status() == dq.DQ_OK
     torch.cuda.empty_cache()
+    # DRAM bytes per launch from the ncu capture of the bench workload of the
+    # same kernel and shape (profiles/traffic.json; null when the kernel's
+    # sources changed since)
+    for tag, e in out.items():
+        wl = next((w for pre, w in SECONDARY_TRAFFIC if tag.startswith(pre)), None)
+        if wl is not None:
+            e["traffic"] = measured_traffic(wl, e["kernel"])
+            e["traffic_workload"] = wl
     return out
+
+
+SECONDARY_TRAFFIC = (("quant_", "quant"), ("small_m16_", "small_m16"), ("large_m_", "large_m"),
+                     ("vit_h_fc1_bsr10", "vit_fc1"), ("vit_h_fc2_bsr10", "vit_fc2"), ("s24_llm", "s24_llm"),
+                     ("s24_small_m16", "s24_small_m16"), ("fp8_llm", "llm_fp8"), ("hqq_m16_", "hqq_m16"),
+                     ("hqq_m1024_", "hqq_m1024"))
 
 
 def run_e2e(args, wl, state, dq, torch, stream, ops, dom, world, max_over_ranks):
