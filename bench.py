@@ -200,7 +200,8 @@ def step_accounting(wl, d):
         out_b = 4 if wl.get("out") == "s32" else 2
         gemm_bytes = M * K + N * K + M * N * out_b + 4 * (M + N)
         return ops, dict(kernel="dq_fp8_linear" if k == "dense_fp8" else "dq_int8_linear", ops=ops,
-                         bytes=gemm_bytes, quant_bytes=(3 * M * K + 4 * M) if k != "gemm" else 0)
+                         bytes=gemm_bytes, quant_bytes=(3 * M * K + 4 * M) if k != "gemm" else 0,
+                         write_bytes=M * N * out_b)
     if k in ("bsr", "bsr_dense"):
         M, K, N = d["M"], d["K"], d["N"]
         nnzb = int(d["crow"][-1])
@@ -208,10 +209,12 @@ def step_accounting(wl, d):
         ops = 2.0 * M * nnzb * bs * bs if k == "bsr" else 2.0 * M * N * K
         wbytes = nnzb * bs * bs if k == "bsr" else N * K
         return ops, dict(kernel="dq_bsr_int8_linear" if k == "bsr" else "dq_int8_linear", ops=ops,
-                         bytes=M * K + wbytes + 2 * M * N + 4 * (M + N), quant_bytes=3 * M * K + 4 * M)
+                         bytes=M * K + wbytes + 2 * M * N + 4 * (M + N), quant_bytes=3 * M * K + 4 * M,
+                         write_bytes=2 * M * N)
     if k == "quant":
         M, K = wl["M"], wl["K"]
-        return 0.0, dict(kernel="dq_quantize_rows", ops=0.0, bytes=3 * M * K + 4 * M, quant_bytes=3 * M * K + 4 * M)
+        return 0.0, dict(kernel="dq_quantize_rows", ops=0.0, bytes=3 * M * K + 4 * M, quant_bytes=3 * M * K + 4 * M,
+                         write_bytes=M * K + 4 * M)
     if k == "s24":
         M, K, N = wl["M"], wl["K"], wl["N"]
         ops = 2.0 * M * N * K          # dense-equivalent work of the 2:4 product
@@ -635,6 +638,15 @@ def run_gpu(args, rank, world, local_rank):
     probe = None
     if world == 1 and not args.no_secondary:
         probe = probe_int8_tops(dq, torch)
+    if world == 1 and (hbm_bound or not args.no_secondary):
+        peaks["write_gbs"] = probe_hbm_write_gbs(torch)
+    if hbm_bound and dom.get("write_bytes") and peaks.get("write_gbs"):
+        # floor: the output at the measured write-only rate, or all bytes at
+        # the copy rate, whichever is longer
+        floor_ms = max(dom["write_bytes"] / (peaks["write_gbs"] * 1e9), dom["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
+        roof["write_floor"] = dict(write_gbs=round(peaks["write_gbs"], 1), write_bytes=int(dom["write_bytes"]),
+                                   floor_ms=round(floor_ms, 5), frac_vs_floor=round(floor_ms / avg_ms, 4),
+                                   source="torch fill of a 1 GiB buffer, timed in this run")
     if not hbm_bound and probe is not None and not hqq:
         roof["frac_vs_probe"] = round(achieved / probe, 4)
         roof["probe_tops"] = round(probe, 1)
@@ -681,6 +693,8 @@ def run_gpu(args, rank, world, local_rank):
     if hqq:
         line["config"]["weight"] = (f"int4 {'s4' if wl.get('signed') else 'u4'} codes, group {wl['group']}, "
                                     "bf16 scales and zero points; dequantized in the GEMM")
+    if probe is not None:
+        line["probes"] = dict(int8_mma_tops=round(probe, 1), hbm_write_gbs=round(peaks["write_gbs"], 1))
     if probe is not None and name == "llm":
         line["secondary"] = secondary_measurements(dq, torch, peaks, probe, K)
         line["secondary"]["_about"] = (
@@ -754,6 +768,27 @@ def probe_int8_tops(dq, torch, iters=20000, reps=5):
     return sms * iters * 2.0 * 128 * 256 * 32 / (ms * 1e-3) / 1e12
 
 
+def probe_hbm_write_gbs(torch, nbytes=1 << 30, reps=10):
+    """Write-only HBM bandwidth: torch's fill of a 1 GiB buffer (a plain
+    vectorized store stream), timed with events.  On this part a pure write
+    stream runs well below the copy bandwidth, so kernels whose bytes are
+    mostly output are also reported against the floor it sets."""
+    x = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        x.fill_(1)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        x.fill_(1)
+    b.record()
+    torch.cuda.synchronize()
+    gbs = nbytes * reps / (a.elapsed_time(b) * 1e-3) / 1e9
+    del x
+    torch.cuda.empty_cache()
+    return gbs
+
+
 def _tensor_entry(name, ms, ops, peaks, probe):
     int8_peak = peaks["bf16"] * INT8_PER_BF16
     tops = ops / (ms * 1e-3) / 1e12
@@ -762,11 +797,18 @@ def _tensor_entry(name, ms, ops, peaks, probe):
                 frac_vs_spec=round(tops / SPEC_INT8_TOPS, 4))
 
 
-def _hbm_entry(name, ms, nbytes, peaks):
+def _hbm_entry(name, ms, nbytes, peaks, write_bytes=0):
     gbs = nbytes / (ms * 1e-3) / 1e9
-    return dict(kernel=name, kernel_ms=round(ms, 5), bound="hbm", achieved=round(gbs, 1), unit="GB/s",
-                peak=peaks["hbm_gbs"], frac=round(gbs / peaks["hbm_gbs"], 4), frac_vs_spec=round(gbs / SPEC_HBM_GBS, 4),
-                algorithmic_bytes=int(nbytes))
+    e = dict(kernel=name, kernel_ms=round(ms, 5), bound="hbm", achieved=round(gbs, 1), unit="GB/s",
+             peak=peaks["hbm_gbs"], frac=round(gbs / peaks["hbm_gbs"], 4), frac_vs_spec=round(gbs / SPEC_HBM_GBS, 4),
+             algorithmic_bytes=int(nbytes))
+    wgbs = peaks.get("write_gbs")
+    if write_bytes and wgbs:
+        # floor: the output at the measured write-only rate, or all bytes at
+        # the copy rate, whichever is longer
+        floor_ms = max(write_bytes / (wgbs * 1e9), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+        e.update(write_bytes=int(write_bytes), floor_ms=round(floor_ms, 5), frac_vs_floor=round(floor_ms / ms, 4))
+    return e
 
 
 def secondary_measurements(dq, torch, peaks, probe, n):
@@ -789,7 +831,7 @@ def secondary_measurements(dq, torch, peaks, probe, n):
     q = torch.empty((M, K), dtype=torch.int8, device="cuda")
     s = torch.empty((M,), dtype=torch.float32, device="cuda")
     ms = _graph_ms(torch, lambda i, st: dq.dq_quantize_rows(x, q, s, stream=st), n)
-    out["quant_16384x8192"] = _hbm_entry("dq_quantize_rows", ms, 3 * M * K + 4 * M, peaks)
+    out["quant_16384x8192"] = _hbm_entry("dq_quantize_rows", ms, 3 * M * K + 4 * M, peaks, M * K + 4 * M)
     del x, q, s
 
     # few-token dense linear M=16, K=8192, N=28672: the weight stream (235 MB)
@@ -841,7 +883,7 @@ def secondary_measurements(dq, torch, peaks, probe, n):
                                                                       stream=st), n)
         ms_d = _graph_ms(torch, lambda i, st: dq.dq_int8_linear(q, s, wq, sc, out=o, stream=st), n)
         nnzb = int(crow[-1])
-        e = _hbm_entry("dq_bsr_int8_linear", ms_b, M * K + nnzb * 4096 + 2 * M * N + 4 * (M + N), peaks)
+        e = _hbm_entry("dq_bsr_int8_linear", ms_b, M * K + nnzb * 4096 + 2 * M * N + 4 * (M + N), peaks, 2 * M * N)
         e["dense_twin"] = _tensor_entry("dq_int8_linear", ms_d, 2.0 * M * N * K, peaks, probe)
         e["quantize_ms"] = round(ms_q, 5)
         e["gemm_speedup_vs_dense"] = round(ms_d / ms_b, 3)
