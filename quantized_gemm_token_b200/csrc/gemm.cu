@@ -715,10 +715,15 @@ dq_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap
 
 constexpr int64_t kMaxK = 133144;   // floor((2^31 - 1) / 127^2): int32 accumulation is exact
 
-// Measured on B200: the pair kernel (half the operand bytes per MMA) pays off
-// from K = 8192 up (8192^3: +13 %; M=2048 N=4096 K=8192: equal); for smaller K
-// its longer prologue loses to the 1-SM kernel.
+// Measured on B200 (graphs of 20 launches, int8 data in [-40, 40]): with one
+// multicast commit per stage the pair kernel (two thirds of the operand bytes
+// per SM) is faster from about 1536 tokens and K = 2048 up (2048 x 4096 x
+// 4096: 25.3 against 27.2 us; 4096^3: 46.1 against 52.1; 16384 x 4096 x 2048:
+// 89 against 105), equal at 1024 tokens and at K = 1024 (38400 x 4096 x 1024:
+// 143 us both), and from K = 8192 up at any token count above 128.
 constexpr int64_t kPairMinK = 8192;
+constexpr int64_t kPairMinKManyTokens = 2048;
+constexpr int64_t kPairManyTokens = 1536;
 
 // The measurement knobs, read once per call.
 struct Knobs {
@@ -793,7 +798,9 @@ bool small_m_dense(int64_t M, int64_t N, int sm_count, const Knobs& kn) {
 
 // Whether the pair kernel (256-row tiles over two SMs) takes a shape with
 // more than 128 tokens when no schedule is forced.
-bool pair_preferred(int64_t /*M*/, int64_t /*N*/, int64_t K) { return K >= kPairMinK; }
+bool pair_preferred(int64_t M, int64_t /*N*/, int64_t K) {
+  return K >= kPairMinK || (M >= kPairManyTokens && K >= kPairMinKManyTokens);
+}
 
 // The schedule of one call: arrangement, kernel, tile widths and (swap-AB)
 // stream-K with the workspace it needs.  `slots` is the number of CTA pairs

@@ -17,7 +17,7 @@
 //               which expects the bytes of both CTAs.
 //   warp 1      MMA issuer, leader only: tcgen05.mma.cta_group::2.kind::i8
 //               (M = 256, N = tile width, K = 32); tcgen05.commit frees the
-//               stage in both CTAs (one commit per CTA) and hands the
+//               stage in both CTAs (one commit multicast to both) and hands the
 //               accumulator to both CTAs' epilogues.
 //   warps 2..9  epilogue in each CTA: at the start of a tile one thread
 //               copies the tile's column scales and bias into shared memory
@@ -201,18 +201,14 @@ __global__ void __launch_bounds__(Cfg2<BN>::THREADS, 1)
 #pragma unroll
           for (int k = 0; k < C::K_STEPS; ++k)
             mma_i8_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-          const uint32_t eb = smem_u32(empty_bar + stage);
-          mma_commit_pair(map_to_rank(eb, 0));
-          mma_commit_pair(map_to_rank(eb, 1));
+          mma_commit_pair_both(smem_u32(empty_bar + stage));    // frees the stage in both CTAs
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        const uint32_t fb = smem_u32(accf_bar + acc);
-        mma_commit_pair(map_to_rank(fb, 0));
-        mma_commit_pair(map_to_rank(fb, 1));
+        mma_commit_pair_both(smem_u32(accf_bar + acc));        // both CTAs' epilogues
         if (++acc == C::ACC_BUFS) {
           acc = 0;
           acc_phase ^= 1;
