@@ -746,9 +746,28 @@ def _graph_ms(torch, launch, n):
     a.record()
     graph.replay()
     b.record()
+    mhz = _sm_clock_mhz()       # read while the replay runs
     torch.cuda.synchronize()
     del graph
+    _LAST_CLOCK[0] = mhz
     return a.elapsed_time(b) / n
+
+
+_LAST_CLOCK = [None]
+_NVML = {}
+
+
+def _sm_clock_mhz():
+    """SM clock of the current device through NVML (None if unavailable)."""
+    try:
+        if "h" not in _NVML:
+            import pynvml
+            pynvml.nvmlInit()
+            _NVML["nv"] = pynvml
+            _NVML["h"] = pynvml.nvmlDeviceGetHandleByIndex(int(os.environ.get("LOCAL_RANK", "0")))
+        return _NVML["nv"].nvmlDeviceGetClockInfo(_NVML["h"], _NVML["nv"].NVML_CLOCK_SM)
+    except Exception:
+        return None
 
 
 def probe_int8_tops(dq, torch, iters=20000, reps=5):
@@ -794,14 +813,14 @@ def _tensor_entry(name, ms, ops, peaks, probe):
     tops = ops / (ms * 1e-3) / 1e12
     return dict(kernel=name, kernel_ms=round(ms, 5), bound="tensor", achieved=round(tops, 1), unit="TOPS",
                 peak=round(int8_peak, 1), frac=round(tops / int8_peak, 4), frac_vs_probe=round(tops / probe, 4),
-                frac_vs_spec=round(tops / SPEC_INT8_TOPS, 4))
+                frac_vs_spec=round(tops / SPEC_INT8_TOPS, 4), sm_mhz=_LAST_CLOCK[0])
 
 
 def _hbm_entry(name, ms, nbytes, peaks, write_bytes=0):
     gbs = nbytes / (ms * 1e-3) / 1e9
     e = dict(kernel=name, kernel_ms=round(ms, 5), bound="hbm", achieved=round(gbs, 1), unit="GB/s",
              peak=peaks["hbm_gbs"], frac=round(gbs / peaks["hbm_gbs"], 4), frac_vs_spec=round(gbs / SPEC_HBM_GBS, 4),
-             algorithmic_bytes=int(nbytes))
+             algorithmic_bytes=int(nbytes), sm_mhz=_LAST_CLOCK[0])
     wgbs = peaks.get("write_gbs")
     if write_bytes and wgbs:
         # floor: the output at the measured write-only rate, or all bytes at
@@ -825,6 +844,12 @@ def secondary_measurements(dq, torch, peaks, probe, n):
         gen.manual_seed(seed)
         return torch.randn(shape, generator=gen, device="cuda", dtype=torch.float32) * std
 
+    # Each workload starts after a 1 s pause, so that every one is timed from
+    # the same clock state (long runs of the large ones can leave the part
+    # under its power cap for a while); each entry records the SM clock read
+    # during its timed replay.
+    pause = lambda: time.sleep(1.0)  # noqa: E731
+    pause()
     # standalone quantize, X bf16 [16384, 8192] (268 MB read)
     M, K = 16384, 8192
     x = randn((M, K), 1.0, 11).to(torch.bfloat16)
@@ -834,6 +859,7 @@ def secondary_measurements(dq, torch, peaks, probe, n):
     out["quant_16384x8192"] = _hbm_entry("dq_quantize_rows", ms, 3 * M * K + 4 * M, peaks, M * K + 4 * M)
     del x, q, s
 
+    pause()
     # few-token dense linear M=16, K=8192, N=28672: the weight stream (235 MB)
     M, K, N = 16, 8192, 28672
     wq, sc = dq.dq_quantize_weight(randn((N, K), 0.02, 12))
@@ -846,6 +872,7 @@ def secondary_measurements(dq, torch, peaks, probe, n):
     out["small_m16_8192x28672"] = _hbm_entry("dq_int8_linear", ms, N * K + M * K + 2 * M * N + 4 * (M + N), peaks)
     del wq, sc, x, q, s, o, ws
 
+    pause()
     # large-M GEMM M=38400, K=1024, N=4096, bf16 out (A rotated over 4 copies)
     M, K, N = 38400, 1024, 4096
     gen.manual_seed(14)
@@ -862,6 +889,7 @@ def secondary_measurements(dq, torch, peaks, probe, n):
     # dense twin (the same masked weight, dense int8) and the layer with its
     # quantize
     for layer in ("fc1", "fc2"):
+        pause()
         K, N = (1280, 5120) if layer == "fc1" else (5120, 1280)
         M = 256 * 257
         crow, col = synth.bsr_pattern(N // 64, K // 64, 0.10, (0 if layer == "fc1" else 100) + 3)
@@ -881,9 +909,11 @@ def secondary_measurements(dq, torch, peaks, probe, n):
         ms_q = _graph_ms(torch, lambda i, st: dq.dq_quantize_rows(x, q, s, stream=st), n)
         ms_b = _graph_ms(torch, lambda i, st: dq.dq_bsr_int8_linear(q, s, N, crow_d, col_d, vals, sc, out=o,
                                                                       stream=st), n)
+        clk_b = _LAST_CLOCK[0]
         ms_d = _graph_ms(torch, lambda i, st: dq.dq_int8_linear(q, s, wq, sc, out=o, stream=st), n)
         nnzb = int(crow[-1])
         e = _hbm_entry("dq_bsr_int8_linear", ms_b, M * K + nnzb * 4096 + 2 * M * N + 4 * (M + N), peaks, 2 * M * N)
+        e["sm_mhz"] = clk_b
         e["dense_twin"] = _tensor_entry("dq_int8_linear", ms_d, 2.0 * M * N * K, peaks, probe)
         e["quantize_ms"] = round(ms_q, 5)
         e["gemm_speedup_vs_dense"] = round(ms_d / ms_b, 3)
@@ -894,6 +924,7 @@ def secondary_measurements(dq, torch, peaks, probe, n):
     # and with dynamic FP8, against the dense int8 GEMM of the same shape;
     # few-token 2:4 weight stream
     for (M, K, N, tag) in ((2048, 4096, 4096, "s24_llm_2048x4096x4096"), (16, 8192, 28672, "s24_small_m16_8192x28672")):
+        pause()
         w = randn((N, K), 0.02, 17 + M)
         # a uniform 2:4 mask: one of the six position pairs per group of four
         pairs = torch.tensor([[1, 1, 0, 0], [1, 0, 1, 0], [1, 0, 0, 1], [0, 1, 1, 0], [0, 1, 0, 1], [0, 0, 1, 1]],
@@ -910,6 +941,7 @@ def secondary_measurements(dq, torch, peaks, probe, n):
         nws = dq.dq_s24_workspace_size(M, N, K)
         ws = torch.zeros(nws, dtype=torch.uint8, device="cuda") if nws else None
         ms_s = _graph_ms(torch, lambda i, st: dq.dq_s24_int8_linear(q, s, vals, meta, sc, out=o, workspace=ws, stream=st), n)
+        clk_s = _LAST_CLOCK[0]
         nwd = dq.dq_int8_linear_workspace_size(M, N, K)
         wsd = torch.zeros(nwd, dtype=torch.uint8, device="cuda") if nwd else None
         ms_d = _graph_ms(torch, lambda i, st: dq.dq_int8_linear(q, s, wq, sc, out=o, workspace=wsd, stream=st), n)
@@ -918,11 +950,13 @@ def secondary_measurements(dq, torch, peaks, probe, n):
             e["ops_note"] = "dense-equivalent ops (2 M N K) of the 2:4 product"
         else:
             e = _hbm_entry("dq_s24_int8_linear", ms_s, N * K // 2 + N * K // 8 + M * K + 2 * M * N + 4 * (M + N), peaks)
+        e["sm_mhz"] = clk_s
         e["dense_int8_ms"] = round(ms_d, 5)
         e["speedup_vs_dense_int8"] = round(ms_d / ms_s, 3)
         out[tag] = e
         del wq, sc, vals, meta, x, q, s, o, ws, wsd
     M, K, N = 2048, 4096, 4096
+    pause()
     wq8, sc8 = dq.dq_quantize_weight_fp8(randn((N, K), 0.02, 19))
     q8, s8 = dq.dq_quantize_rows_fp8(randn((M, K), 1.0, 20).to(torch.bfloat16))
     o = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
@@ -940,6 +974,7 @@ def secondary_measurements(dq, torch, peaks, probe, n):
     scl = dq.dq_hqq_group_major((torch.rand((N, K // 128), generator=gen, device="cuda") * 0.018 + 0.002).to(torch.bfloat16))
     zer = dq.dq_hqq_group_major((torch.rand((N, K // 128), generator=gen, device="cuda") * 3 + 6).to(torch.bfloat16))
     for M in (16, 1024):
+        pause()
         x = randn((M, K), 1.0, 22 + M).to(torch.bfloat16)
         o = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         nws = dq.dq_hqq_workspace_size(M, N, K)

@@ -1025,8 +1025,55 @@ dq_status dq_fp8_linear(const uint8_t* A, const float* s_row, int64_t M, int64_t
   if (st != DQ_OK) return st;
   if (M == 0) return DQ_OK;
 
-  // The dense arrangement (tokens on MMA M) for every M, 128 x 256 tiles
-  // (128 x 128 for N <= 128), two tile widths when the last wave is partial.
+  // Many tokens (the int8 kernel's rule): the 2-SM pair kernel, 256 x 256
+  // tiles over two SMs, two tile widths when the last wave is partial.
+  const Knobs kn = knobs();
+  if (N > 128 && (kn.schedule == 3 || (kn.schedule == 0 && M > 128 && pair_preferred(M, N, K)))) {
+    int pairs = 0;
+    if ((st = pair_slots(*d, &pairs)) != DQ_OK) return st;
+    Plan p{};
+    p.kind = Kind::DenseF8;
+    p.pair = true;
+    p.bn = 256;
+    p.a_tiles = static_cast<int>((M + 255) / 256);
+    p.b_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
+    p.kb_total = static_cast<int>((K + kDenseKB - 1) / kDenseKB);
+    p.num_tiles = p.a_tiles * p.b_tiles;
+    if (kn.two_widths) plan_two_widths(p, N, pairs);
+    CUtensorMap ta, tb, tb2, tc;
+    if ((st = make_tmap_u8_2d(&ta, A, K, M, K, kDenseKB, 128, kDenseKB)) != DQ_OK) return st;
+    if ((st = make_tmap_u8_2d(&tb, W, K, N, K, kDenseKB, p.bn / 2, kDenseKB)) != DQ_OK) return st;
+    if (p.bn2 > 0) {
+      if ((st = make_tmap_u8_2d(&tb2, W, K, N, K, kDenseKB, p.bn2 / 2, kDenseKB)) != DQ_OK) return st;
+    } else {
+      tb2 = tb;
+    }
+    if ((st = make_tmap_out_2d(&tc, out, N, M, f32 ? 4 : 2)) != DQ_OK) return st;
+    GemmArgs g{};
+    g.M = static_cast<int>(M);
+    g.N = static_cast<int>(N);
+    g.K = static_cast<int>(K);
+    g.a_tiles = p.a_tiles;
+    g.b_tiles = p.b_tiles;
+    g.kb_total = p.kb_total;
+    g.num_tiles = p.num_tiles;
+    g.t1 = p.t1;
+    g.bn2 = p.bn2;
+    g.mb0 = p.mb0;
+    g.c_start = p.c_start;
+    g.first_cnt = p.first_cnt;
+    g.per_row = p.per_row;
+    g.s_row = s_row;
+    g.s_col = s_col;
+    g.bias = static_cast<const uint16_t*>(bias_bf16);
+    g.out = out;
+    g.out_s32 = f32 ? 1 : 0;                   // raw accumulator bits
+    g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
+    return launch_pair_gemm(ta, tb, tb2, tc, g, p.bn, p.num_tiles < pairs ? p.num_tiles : pairs, stream, true);
+  }
+
+  // The dense arrangement (tokens on MMA M), 128 x 256 tiles (128 x 128 for
+  // N <= 128), two tile widths when the last wave is partial.
   Plan p{};
   p.kind = Kind::DenseF8;
   p.bn = N <= 128 ? 128 : 256;
@@ -1034,7 +1081,7 @@ dq_status dq_fp8_linear(const uint8_t* A, const float* s_row, int64_t M, int64_t
   p.b_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
   p.kb_total = static_cast<int>((K + kDenseKB - 1) / kDenseKB);
   p.num_tiles = p.a_tiles * p.b_tiles;
-  if (p.bn == 256 && knobs().two_widths) plan_two_widths(p, N, d->sm_count);
+  if (p.bn == 256 && kn.two_widths) plan_two_widths(p, N, d->sm_count);
   CUtensorMap ta, tb, tb2, tc;
   if ((st = make_tmap_u8_2d(&ta, A, K, M, K, kDenseKB, 128, kDenseKB)) != DQ_OK) return st;
   if ((st = make_tmap_u8_2d(&tb, W, K, N, K, kDenseKB, p.bn, kDenseKB)) != DQ_OK) return st;

@@ -65,7 +65,9 @@ struct Cfg2 {
   static_assert(BN % 32 == 0 && BN <= 256 && (BN / 2) % 8 == 0, "tile width");
 };
 
-template <int BN>
+// F8: e4m3 operands (kind::f8f6f4, fp32 accumulator; the epilogue takes the
+// accumulator bits as fp32), else int8 (kind::i8, int32).
+template <int BN, bool F8>
 __global__ void __launch_bounds__(Cfg2<BN>::THREADS, 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                  const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_c,
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(Cfg2<BN>::THREADS, 1)
       bool ok = true;
       for (int t = pair; ok && t < g.num_tiles; t += G) {
         const TileGeom geo = tile_geom(g, t, BN, true);
-        const uint32_t idesc = idesc_i8(256, geo.width);
+        const uint32_t idesc = F8 ? idesc_e4m3(256, geo.width) : idesc_i8(256, geo.width);
         if (!mbar_wait(smem_u32(acce_bar + acc), acc_phase ^ 1, g.wait, abort_flag)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -200,7 +202,8 @@ __global__ void __launch_bounds__(Cfg2<BN>::THREADS, 1)
           const uint64_t bd = smem_desc_kmajor<C::KB>(smem_u32(sB + stage * C::B_BYTES));
 #pragma unroll
           for (int k = 0; k < C::K_STEPS; ++k)
-            mma_i8_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            if constexpr (F8) mma_f8_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            else mma_i8_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
           mma_commit_pair_both(smem_u32(empty_bar + stage));    // frees the stage in both CTAs
           if (++stage == C::STAGES) {
             stage = 0;
@@ -279,7 +282,7 @@ __global__ void __launch_bounds__(Cfg2<BN>::THREADS, 1)
         for (int i = 0; i < 2; ++i) {
           const int c = c0 + i * GROUPS;
           if (i == 1 && !two) break;
-          store_row_chunk_staged(g, &tm_c, next_buf(), lane, m_slab, geo.n0 + c * C::CW, r[i], srow, sc_slot,
+          store_row_chunk_staged<F8>(g, &tm_c, next_buf(), lane, m_slab, geo.n0 + c * C::CW, r[i], srow, sc_slot,
                                  c * C::CW);
         }
       }
@@ -322,16 +325,16 @@ cudaLaunchConfig_t pair_config(cudaLaunchAttribute (&attr)[2], cudaStream_t stre
   return cfg;
 }
 
-template <int BN>
+template <int BN, bool F8>
 dq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2, const CUtensorMap& tc,
                       const GemmArgs& g, int pairs, cudaStream_t stream) {
   using C = Cfg2<BN>;
-  const dq_status st = smem_limit_once(reinterpret_cast<const void*>(&gemm2_kernel<BN>), C::SMEM_BYTES);
+  const dq_status st = smem_limit_once(reinterpret_cast<const void*>(&gemm2_kernel<BN, F8>), C::SMEM_BYTES);
   if (st != DQ_OK) return st;
   cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pair_config<BN>(attr, stream);
   cfg.gridDim = dim3(2 * pairs);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm2_kernel<BN>, ta, tb, tb2, tc, g);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm2_kernel<BN, F8>, ta, tb, tb2, tc, g);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 
@@ -342,13 +345,14 @@ dq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
 dq_status pair_slots(const DeviceInfo& d, int* pairs) {
   int n = g_pair_slots[d.device & 63].load(std::memory_order_relaxed);
   if (n == 0) {
-    const dq_status st = smem_limit_once(reinterpret_cast<const void*>(&gemm2_kernel<256>), Cfg2<256>::SMEM_BYTES);
+    const dq_status st =
+        smem_limit_once(reinterpret_cast<const void*>(&gemm2_kernel<256, false>), Cfg2<256>::SMEM_BYTES);
     if (st != DQ_OK) return st;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = pair_config<256>(attr, nullptr);
     cfg.numAttrs = 1;                         // the cluster shape only
     cfg.gridDim = dim3(2 * (d.sm_count / 2));
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm2_kernel<256>, &cfg);
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm2_kernel<256, false>, &cfg);
     if (e != cudaSuccess) return cuda_fail(e);
     if (n < 1) n = 1;
     g_pair_slots[d.device & 63].store(n, std::memory_order_relaxed);
@@ -358,13 +362,15 @@ dq_status pair_slots(const DeviceInfo& d, int* pairs) {
 }
 
 // Launches gemm2_kernel with clusters of 2 CTAs, `pairs` pairs (persistent).
-// bn: pair tile width (160, 192 or 256).
+// bn: pair tile width (160, 192 or 256); f8: e4m3 operands (only with 256).
 dq_status launch_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2,
-                           const CUtensorMap& tc, const GemmArgs& g, int bn, int pairs, cudaStream_t stream) {
+                           const CUtensorMap& tc, const GemmArgs& g, int bn, int pairs, cudaStream_t stream,
+                           bool f8) {
+  if (f8) return launch_pair<256, true>(ta, tb, tb2, tc, g, pairs, stream);
   switch (bn) {
-    case 160: return launch_pair<160>(ta, tb, tb2, tc, g, pairs, stream);
-    case 192: return launch_pair<192>(ta, tb, tb2, tc, g, pairs, stream);
-    default: return launch_pair<256>(ta, tb, tb2, tc, g, pairs, stream);
+    case 160: return launch_pair<160, false>(ta, tb, tb2, tc, g, pairs, stream);
+    case 192: return launch_pair<192, false>(ta, tb, tb2, tc, g, pairs, stream);
+    default: return launch_pair<256, false>(ta, tb, tb2, tc, g, pairs, stream);
   }
 }
 

@@ -418,9 +418,11 @@ __device__ __forceinline__ void store_col_chunk(const GemmArgs& g, int n, int m0
 // Dense GEMM with each 256 x bn tile's MMA on a pair of SMs (gemm2sm.cu).
 // g.a_tiles / g.b_tiles count 256-row / bn-column tiles; bn is 160, 192 or
 // 256; with g.bn2 > 0 the tiles from g.t1 on are bn2 wide (tm_b2's box is
-// bn2 / 2 weight rows).  `pairs` is the number of CTA pairs to launch.
+// bn2 / 2 weight rows).  `pairs` is the number of CTA pairs to launch; f8:
+// e4m3 operands and an fp32 accumulator (bn 256 only).
 dq_status launch_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2,
-                           const CUtensorMap& tc, const GemmArgs& g, int bn, int pairs, cudaStream_t stream);
+                           const CUtensorMap& tc, const GemmArgs& g, int bn, int pairs, cudaStream_t stream,
+                           bool f8 = false);
 // CTA pairs of the pair kernel that fit on the current device at once.
 dq_status pair_slots(const DeviceInfo& d, int* pairs);
 
