@@ -111,6 +111,28 @@ def test_fp8_linear_against_the_exact_sum(M, N, K):
     assert np.all(np.abs(got - y) <= tol)
 
 
+@pytest.mark.parametrize("M,N,K", [(300, 520, 384), (513, 1032, 4096), (1600, 4104, 2048)])
+def test_fp8_pair_kernel_against_the_exact_sum(M, N, K):
+    """The 2-SM pair kernel with e4m3 operands (forced with schedule 3;
+    the automatic choice from 1536 tokens and K >= 2048): ragged rows,
+    columns and both tile widths, within the same bounds as the 1-SM kernel."""
+    x, w, q, s, wq, sc = _fp8_operands(M, N, K, 700 + M + N + K)
+    qd, wd = to_dev(q), to_dev(wq)
+    dq.dq_debug_set_schedule(3)
+    try:
+        acc = dq.dq_fp8_linear(qd, None, wd, None, out_dtype="f32").cpu().numpy().astype(np.float64)
+        out = dq.dq_fp8_linear(qd, to_dev(s), wd, to_dev(sc))
+    finally:
+        dq.dq_debug_set_schedule(0)
+    rows = tile_rows(M, total=256, seed=M)
+    exact = oracle.gemm_fp8_f64(q[rows], wq)
+    mag = np.abs(oracle.e4m3_to_float64(q[rows])) @ np.abs(oracle.e4m3_to_float64(wq)).T
+    assert np.all(np.abs(acc[rows] - exact) <= ACC_REL * mag + 1e-30)
+    y = exact * s[rows, None].astype(np.float64) * sc[None, :].astype(np.float64)
+    got = _bf16_to_f32(bf16_bits(out)[rows]).astype(np.float64)
+    assert np.all(np.abs(got - y) <= ACC_REL * mag * s[rows, None] * sc[None, :] + np.abs(y) * 2.0 ** -8 + 1e-30)
+
+
 def test_fp8_llm_shaped_layer_and_accuracy():
     d = synth.llm(0)
     M, K, N = d["x"].shape[0], d["x"].shape[1], d["w"].shape[0]
