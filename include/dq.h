@@ -410,7 +410,9 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
  * dq_debug_set_schedule (dense int8 linear): 0 automatic; 1 the 1-SM kernel
  *   with whole tiles; 2 the 1-SM kernel with stream-K whenever a workspace
  *   is given; 3 the 2-SM pair kernel for every M; 4 the dense (tokens on
- *   MMA M) arrangement also for M <= 128; 5 as 4 with stream-K.
+ *   MMA M) arrangement also for M <= 128; 5 as 4 with stream-K.  The FP8
+ *   and 2:4 linears read it too: 1 keeps their 1-SM kernels, 3 takes their
+ *   2-SM pair kernels (2:4: when its contraction is not split).
  * dq_debug_set_tile_n: force the dense tile width (128, 160, 192, 224, 256;
  *   pair kernel 160, 192, 256); 0 automatic.
  * dq_debug_set_two_widths: 1 (default) wave-balanced schedule of two tile

@@ -412,6 +412,239 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, S4_TMEM_COLS);
 }
 
+// ---------------------------------------------------------------- 2-SM pair
+// Many tokens: each 256-channel x bn-token tile's sparse MMAs run on a pair
+// of SMs (a cluster of two CTAs, tcgen05.mma.sp.cta_group::2, M = 256).  Each
+// CTA loads its own 128 weight rows (compressed values and metadata) and half
+// of the activation tile (bn / 2 tokens); the pair MMA reads each CTA's half
+// of the activations once for both SMs, so per SM and 128-deep step TMA
+// writes 25 KB instead of 40 KB (bn = 240) and more stages fit.  The leader
+// (rank 0) copies the step's metadata of both CTAs into their tensor memory
+// (tcgen05.cp.cta_group::2: each CTA's rows from its own shared memory) and
+// issues the MMAs; one commit multicast to both CTAs frees a stage or hands
+// over an accumulator.  No split contraction.
+
+__device__ __forceinline__ void mma_i8_sparse_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t meta,
+                                                   uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(meta), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_cp_128x128b_pair(uint32_t taddr, uint32_t smem_addr) {
+  const uint64_t desc = (static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4))
+                        | (static_cast<uint64_t>(128u >> 4) << 16)
+                        | (static_cast<uint64_t>(128u >> 4) << 32)
+                        | (1ull << 46);
+  asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+__global__ void __launch_bounds__(S4_THREADS, 1)
+    s24_gemm2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_m, const __grid_constant__ CUtensorMap tm_c32,
+                     const __grid_constant__ CUtensorMap tm_c16, const S24Args g) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const smem = smem_raw + (base - raw);
+  // stage s at base + s * stage_bytes: this CTA's half of the activation tile
+  // (bn / 2 x 128 B), its compressed values (128 x 64 B) and metadata (128 x
+  // 16 B); every part 1024-byte aligned
+  const uint32_t q_bytes = static_cast<uint32_t>(g.bn / 2) * 128u;
+  const uint32_t stage_bytes = q_bytes + S4_V_BYTES + S4_M_BYTES;
+  uint64_t* const full = reinterpret_cast<uint64_t*>(smem + g.off_bar);
+  uint64_t* const empty = full + S4_MAX_NP;
+  uint64_t* const accf = empty + S4_MAX_NP;
+  uint64_t* const acce = accf + 2;
+  uint64_t* const drain = acce + 2;
+  uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int pairs = static_cast<int>(gridDim.x >> 1);
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < g.np; ++i) {
+      mbar_init(smem_u32(full + i), 1);
+      mbar_init(smem_u32(empty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(accf + i), 1);
+      mbar_init(smem_u32(acce + i), 2 * S4_EPI_WARPS);
+    }
+    mbar_init(smem_u32(drain), 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_m);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), S4_TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();            // both CTAs' barriers are initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  griddep_wait();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int u = pair; ok && u < g.units; u += pairs) {
+        const int ntile = 2 * (u / g.tt) + rank;
+        const int ttile = u % g.tt;
+        for (int kk = 0; kk < g.ks; ++kk) {
+          if (!pipe::wait(smem_u32(empty + stage), phase ^ 1, g.wait, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(full + stage);
+          const uint32_t fb_leader = map_to_rank(fb, 0);
+          const uint32_t sq = base + stage * stage_bytes;
+          const uint32_t sv = sq + q_bytes;
+          if (leader) mbar_arrive_expect_tx(fb, 2u * stage_bytes);
+          tma_load_2d_pair(sq, &tm_q, fb_leader, kk * S4_BK, ttile * g.bn + rank * (g.bn / 2));
+          tma_load_2d_pair(sv, &tm_v, fb_leader, kk * (S4_BK / 2), ntile * 128);
+          tma_load_2d_pair(sv + S4_V_BYTES, &tm_m, fb_leader, kk * (S4_BK / 8), ntile * 128);
+          ++issued;
+          if (++stage == g.np) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies already issued land before the CTA leaves: the leader
+        // waits on its full barriers (bounded); the follower, whose copies
+        // complete on the leader's barriers, waits a fixed 100 us.
+        if (leader) {
+          WaitCtl quick = g.wait;
+          quick.timeout_ns = quick.timeout_ns < 50000000ull ? quick.timeout_ns : 50000000ull;
+          volatile int never = 0;
+          for (long long i = issued > g.np ? issued - g.np : 0; i < issued; ++i)
+            pipe::wait(smem_u32(full + static_cast<int>(i % g.np)), static_cast<uint32_t>((i / g.np) & 1), quick,
+                       &never);
+        } else {
+          const uint64_t t0 = globaltimer();
+          while (globaltimer() - t0 < 100000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer (leader)
+    if (leader && lane == 0) {
+      const uint32_t idesc = idesc_i8_sparse(256, g.bn);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, aphase = 0;
+      bool ok = true;
+      for (int u = pair; ok && u < g.units; u += pairs) {
+        if (!pipe::wait(smem_u32(acce + acc), aphase ^ 1, g.wait, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * g.bn);
+        for (int kk = 0; kk < g.ks; ++kk) {
+          if (!pipe::wait(smem_u32(full + stage), phase, g.wait, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sq = base + stage * stage_bytes;
+          const uint32_t sv = sq + q_bytes;
+          // both CTAs' metadata of the step into their tensor-memory slot of
+          // this stage (the slot's previous MMAs completed before the stage
+          // was refilled)
+          const uint32_t meta = tmem_base + static_cast<uint32_t>(2 * g.bn + 4 * stage);
+          tmem_cp_128x128b_pair(meta, sv + S4_V_BYTES);
+          const uint64_t ad = smem_desc_kmajor<64>(sv);
+          const uint64_t bd = smem_desc_kmajor<128>(sq);
+#pragma unroll
+          for (int j = 0; j < 2; ++j)   // logical K = 64 per MMA: 32 compressed bytes, 64 activation bytes
+            mma_i8_sparse_pair(d_tmem, ad + 2 * j, bd + 4 * j, meta + 2 * j, idesc, (kk > 0 || j > 0) ? 1u : 0u);
+          mma_commit_pair_both(smem_u32(empty + stage));
+          if (++stage == g.np) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair_both(smem_u32(accf + acc));
+        if (++acc == 2) {
+          acc = 0;
+          aphase ^= 1;
+        }
+      }
+      mma_commit_pair(map_to_rank(smem_u32(drain), 0));
+      volatile int never = 0;
+      pipe::wait(smem_u32(drain), 0, g.wait, &never);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue (both CTAs)
+    // This CTA's 128 channels (its TMEM lanes) x all bn tokens, as in the
+    // 1-SM kernel; each warp frees the accumulator on the leader once it has
+    // read its last chunk.
+    const int ew = warp - 2;
+    const int q = warp & 3;
+    const int grp = ew >> 2;
+    const int row = q * 32 + lane;
+    const uint32_t buf = base + g.off_epi + static_cast<uint32_t>(ew) * S4_EPI_BUF;
+    const uint32_t acce_leader = map_to_rank(smem_u32(acce), 0);
+    int acc = 0;
+    uint32_t aphase = 0;
+    for (int u = pair; u < g.units; u += pairs) {
+      const int ntile = 2 * (u / g.tt) + rank;
+      const int ttile = u % g.tt;
+      const bool w = pipe::wait(smem_u32(accf + acc), aphase, g.wait, abort_flag);
+      if (!__all_sync(0xffffffffu, w)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * g.bn);
+      const int ch = ntile * 128 + row;
+      const int ch_w = ntile * 128 + q * 32;
+      const int tok0 = ttile * g.bn;
+      const int nch = (g.bn + 31) / 32;
+      for (int c = grp; c < nch; c += 2) {
+        const int width = min(32, g.bn - 32 * c);
+        uint32_t r[32];
+        load_chunk(tb + 32 * c, width, r);
+        tmem_ld_wait();
+        if (c + 2 >= nch) {            // this warp's last chunk: the accumulator is free
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(acce_leader + static_cast<uint32_t>(acc) * 8u);
+        }
+        store_chunk(g, r, width, tok0 + 32 * c, ch, ch_w, lane, buf, &tm_c32, &tm_c16);
+      }
+      if (grp >= nch) {                 // no chunk for this warp (bn <= 32)
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acce_leader + static_cast<uint32_t>(acc) * 8u);
+      }
+      if (++acc == 2) {
+        acc = 0;
+        aphase ^= 1;
+      }
+    }
+    if (lane == 0) bulk_wait_group<0>();         // every output store complete
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync_all();            // no CTA leaves while its peer may still read its shared memory or signal it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, S4_TMEM_COLS);
+}
+
 // One thread per metadata byte (two groups): compress eight weight bytes.
 __global__ void __launch_bounds__(256) s24_compress_kernel(const int8_t* __restrict__ w, int64_t N, int64_t K,
                                                            int8_t* __restrict__ values, uint8_t* __restrict__ meta,
@@ -504,6 +737,39 @@ S24Plan plan_s24(int64_t M, int64_t N, int64_t K, int sm_count, bool allow_split
   return p;
 }
 
+// 2-SM pair tiles: 256 channels (128 per CTA) x bn tokens, bn chosen as in
+// plan_s24 over the CTA pairs; no split.  Each stage holds half the
+// activation tile, so up to 8 stages fit at bn = 240.
+S24Plan plan_s24_pair(int64_t M, int64_t N, int64_t K, int sm_count) {
+  S24Plan best{};
+  long long best_cost = -1;
+  const int pairs = std::max(1, sm_count / 2);
+  const int nt = static_cast<int>((N + 255) / 256);
+  for (int bn = 16; bn <= S4_MAX_BN; bn += 16) {
+    if (bn > 16 && bn - 16 >= M) break;
+    const int tt = static_cast<int>((M + bn - 1) / bn);
+    const long long tiles = static_cast<long long>(nt) * tt;
+    const long long waves = (tiles + pairs - 1) / pairs;
+    const long long cost = waves * (bn + 32);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best.bn = bn;
+      best.tt = tt;
+    }
+  }
+  S24Plan& p = best;
+  p.splits = 1;
+  p.nt = nt;
+  p.ks = static_cast<int>(K / S4_BK);
+  p.units = static_cast<int>(static_cast<long long>(p.nt) * p.tt);
+  p.grid = 2 * std::min(p.units, pairs);
+  const int stage = (p.bn / 2) * 128 + S4_V_BYTES + S4_M_BYTES;
+  p.np = std::min({S4_MAX_NP, (S4_SMEM_LIMIT - 1024 - S4_EPI_WARPS * S4_EPI_BUF - S4_BAR_BYTES) / stage,
+                   (S4_TMEM_COLS - 2 * p.bn) / 4});
+  p.smem = 1024 + static_cast<size_t>(p.np) * stage + S4_EPI_WARPS * S4_EPI_BUF + S4_BAR_BYTES;
+  return p;
+}
+
 int grid_for(int64_t items, int sm_count) {
   const int64_t blocks = (items + 255) / 256;
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(sm_count) * 16)));
@@ -559,10 +825,16 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
   S24Plan p = plan_s24(M, N, K, d->sm_count, true);
   if (p.splits > 1 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < p.ws_bytes))
     p = plan_s24(M, N, K, d->sm_count, false);
+  // Many tokens, no split: the 2-SM pair kernel (the dense int8 linear's rule;
+  // schedule knob 3 forces it, 1 keeps the 1-SM kernel).
+  const int sched = g_schedule_override.load(std::memory_order_relaxed);
+  const bool pair = p.splits == 1 && N > 128 &&
+                    (sched == 3 || (sched == 0 && M >= 1536 && K >= 2048));
+  if (pair) p = plan_s24_pair(M, N, K, d->sm_count);
 
   CUtensorMap tq, tv, tm;
   st = make_tmap_u8_2d(&tq, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128,
-                       static_cast<uint32_t>(p.bn), 128);
+                       static_cast<uint32_t>(pair ? p.bn / 2 : p.bn), 128);
   if (st != DQ_OK) return st;
   st = make_tmap_u8_2d(&tv, values, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N),
                        static_cast<uint64_t>(K / 2), 64, 128, 64);
@@ -590,7 +862,7 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
   g.ks = p.ks;
   g.units = p.units;
   g.np = p.np;
-  g.off_epi = static_cast<uint32_t>(p.np) * (p.bn * 128 + S4_V_BYTES + S4_M_BYTES);
+  g.off_epi = static_cast<uint32_t>(p.np) * ((pair ? p.bn / 2 : p.bn) * 128 + S4_V_BYTES + S4_M_BYTES);
   g.off_bar = g.off_epi + S4_EPI_WARPS * S4_EPI_BUF;
   g.s_row = s_row;
   g.s_col = s_col;
@@ -603,21 +875,29 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
   }
   g.wait = WaitCtl{d->err_word, wait_timeout_ns()};
 
-  const dq_status ast = smem_limit_once(reinterpret_cast<const void*>(&s24_gemm_kernel), S4_SMEM_LIMIT);
+  const void* kern = pair ? reinterpret_cast<const void*>(&s24_gemm2_kernel)
+                          : reinterpret_cast<const void*>(&s24_gemm_kernel);
+  const dq_status ast = smem_limit_once(kern, S4_SMEM_LIMIT);
   if (ast != DQ_OK) return ast;
   // Programmatic stream serialization: the prologue may overlap the tail of
   // the quantization that produced A; the kernel waits before global access.
+  // The pair kernel runs as clusters of two CTAs.
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(p.grid));
   cfg.blockDim = dim3(S4_THREADS);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, s24_gemm_kernel, tq, tv, tm, tc32, tc16, g);
+  cfg.numAttrs = pair ? 2 : 1;
+  const cudaError_t e = pair ? cudaLaunchKernelEx(&cfg, s24_gemm2_kernel, tq, tv, tm, tc32, tc16, g)
+                             : cudaLaunchKernelEx(&cfg, s24_gemm_kernel, tq, tv, tm, tc32, tc16, g);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 

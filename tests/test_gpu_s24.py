@@ -81,6 +81,31 @@ def test_linear_matches_oracle(M, N, K, use_ws):
         assert np.array_equal(out.cpu().numpy(), want)
 
 
+@pytest.mark.parametrize("M,N,K", [(300, 264, 256), (513, 1032, 1024), (1600, 4104, 2048), (40, 512, 384)])
+def test_pair_kernel_matches_oracle(M, N, K):
+    """The 2-SM pair kernel (tcgen05.mma.sp over two SMs, each CTA's
+    metadata copied into its own tensor memory), forced with schedule 3 and
+    automatic from 1536 tokens and K >= 2048: int32 bit-exact and the bf16
+    epilogue with bias, on ragged channels (a pair tile whose second half
+    lies past N), tokens and both token-tile halves."""
+    W = _random_s24(N, K, 17 + N)
+    A = synth.uniform_int8((M, K), -127, 127, 18 + M)
+    s_row = synth.uniform_f32((M,), 0.001, 0.05, 19)
+    s_col = synth.uniform_f32((N,), 0.001, 0.05, 20)
+    bias = synth.normal_bf16((N,), 0.1, 21)
+    v, m, _ = oracle.s24_compress(W)
+    vd, md, Ad = to_dev(v), to_dev(m), to_dev(A)
+    want = oracle.gemm_s32(A, oracle.s24_decompress(v, m))
+    dq.dq_debug_set_schedule(3)
+    try:
+        acc = dq.dq_s24_int8_linear(Ad, None, vd, md, None, out_dtype="s32")
+        out = dq.dq_s24_int8_linear(Ad, to_dev(s_row), vd, md, to_dev(s_col), bias=to_dev_bf16(bias))
+    finally:
+        dq.dq_debug_set_schedule(0)
+    assert np.array_equal(acc.cpu().numpy(), want)
+    assert_bf16_close(bf16_bits(out), oracle.epilogue_bf16(want, s_row, s_col, bias))
+
+
 @pytest.mark.parametrize("M,K,N", [(2048, 4096, 4096), (16, 8192, 28672)])
 def test_layer_full_size(M, K, N):
     """The benchmark shapes: quantize (GPU), compress (GPU), sparse product;
