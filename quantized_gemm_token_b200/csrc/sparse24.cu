@@ -34,6 +34,9 @@
 // Few tiles: the contraction is split; int32 partial tiles go to a
 // workspace and, per epilogue warp, the last split of a tile to arrive adds
 // them (exact, in split order) before the epilogue arithmetic.
+// Many tokens (from 1536 with K >= 2048): a 2-SM pair version of the same
+// kernel (s24_gemm2_kernel, 256-channel tiles over a cluster of two CTAs,
+// each loading its own weight rows and half of the activation tile).
 #include <cuda_bf16.h>
 
 #include <algorithm>
