@@ -986,7 +986,7 @@ def secondary_measurements(dq, torch, peaks, probe, n):
         else:
             tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
             e = dict(kernel="dq_hqq_linear", kernel_ms=round(ms, 5), bound="tensor", achieved=round(tf, 1),
-                     unit="TFLOP/s", peak=peaks["bf16"], frac=round(tf / peaks["bf16"], 4))
+                     unit="TFLOP/s", peak=peaks["bf16"], frac=round(tf / peaks["bf16"], 4), sm_mhz=_LAST_CLOCK[0])
         e["page_h100_ms"] = HQQ_PAGE_H100_MS[M]
         out[f"hqq_m{M}_4096x4096_g128"] = e
         del x, o, ws
