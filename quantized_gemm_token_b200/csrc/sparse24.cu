@@ -139,9 +139,14 @@ __device__ __forceinline__ float dequant(int32_t acc, float sr, float sc, bool h
 // 16 or 32).  bf16 goes through the warp's staging buffer `buf` (free once
 // its previous store has read it) and one TMA store of the 32 x 32 block,
 // which clips tokens >= M and channels >= N; int32 is stored directly.
-__device__ __forceinline__ void store_chunk(const S24Args& g, const uint32_t (&r)[32], int width, int tok0, int ch,
-                                            int ch_w, int lane, uint32_t buf, const CUtensorMap* tm32,
-                                            const CUtensorMap* tm16) {
+// PENDING: how many of this warp's earlier stores may still be reading their
+// staging buffers (0: one buffer per warp; 1: two buffers used in turn, and
+// every chunk commits a group, an empty one when it stores nothing, so that
+// the count stays in step with the buffers).
+template <int PENDING>
+__device__ __forceinline__ void store_chunk_t(const S24Args& g, const uint32_t (&r)[32], int width, int tok0, int ch,
+                                              int ch_w, int lane, uint32_t buf, const CUtensorMap* tm32,
+                                              const CUtensorMap* tm16) {
   const bool ch_ok = ch < g.N;
   if (g.out_s32) {
     int32_t* o = static_cast<int32_t*>(g.out);
@@ -163,15 +168,28 @@ __device__ __forceinline__ void store_chunk(const S24Args& g, const uint32_t (&r
     const float f1 = dequant(static_cast<int32_t>(r[2 * i + 1]), sr1, sc, has_bias, b);
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(pk[i]) : "f"(f1), "f"(f0));
   }
-  if (lane == 0) bulk_wait_group_read<0>();
+  if (lane == 0) bulk_wait_group_read<PENDING>();
   __syncwarp();
   pipe::stage_bf16_pairs(buf, pk, width, lane);
   fence_proxy_async_smem();
   __syncwarp();
-  if (lane == 0 && ch_w < g.N && tok0 < g.M) {     // boxes wholly outside are not issued
-    tma_store_2d(width == 32 ? tm32 : tm16, buf, 2 * ch_w, tok0);
-    bulk_commit_group();
+  if constexpr (PENDING == 0) {
+    if (lane == 0 && ch_w < g.N && tok0 < g.M) {     // boxes wholly outside are not issued
+      tma_store_2d(width == 32 ? tm32 : tm16, buf, 2 * ch_w, tok0);
+      bulk_commit_group();
+    }
+  } else {
+    if (lane == 0) {
+      if (ch_w < g.N && tok0 < g.M) tma_store_2d(width == 32 ? tm32 : tm16, buf, 2 * ch_w, tok0);
+      bulk_commit_group();
+    }
   }
+}
+
+__device__ __forceinline__ void store_chunk(const S24Args& g, const uint32_t (&r)[32], int width, int tok0, int ch,
+                                            int ch_w, int lane, uint32_t buf, const CUtensorMap* tm32,
+                                            const CUtensorMap* tm16) {
+  store_chunk_t<0>(g, r, width, tok0, ch, ch_w, lane, buf, tm32, tm16);
 }
 
 // Reads a chunk's accumulators (width 32, or 16 for a 16-token tail) from TMEM.
@@ -601,7 +619,8 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
     const int q = warp & 3;
     const int grp = ew >> 2;
     const int row = q * 32 + lane;
-    const uint32_t buf = base + g.off_epi + static_cast<uint32_t>(ew) * S4_EPI_BUF;
+    const uint32_t buf0 = base + g.off_epi + static_cast<uint32_t>(ew) * 2u * S4_EPI_BUF;   // two per warp
+    uint32_t flip = 0;
     const uint32_t acce_leader = map_to_rank(smem_u32(acce), 0);
     int acc = 0;
     uint32_t aphase = 0;
@@ -616,17 +635,28 @@ __global__ void __launch_bounds__(S4_THREADS, 1)
       const int ch_w = ntile * 128 + q * 32;
       const int tok0 = ttile * g.bn;
       const int nch = (g.bn + 31) / 32;
-      for (int c = grp; c < nch; c += 2) {
-        const int width = min(32, g.bn - 32 * c);
-        uint32_t r[32];
-        load_chunk(tb + 32 * c, width, r);
+      // two of this warp's chunks per tensor-memory wait; the staging
+      // buffers alternate, so a chunk waits only for the store before last
+      for (int c0 = grp; c0 < nch; c0 += 4) {
+        const int c1 = c0 + 2;
+        const bool two = c1 < nch;
+        const int w0 = min(32, g.bn - 32 * c0);
+        const int w1 = two ? min(32, g.bn - 32 * c1) : 0;
+        uint32_t r0[32], r1[32];
+        load_chunk(tb + 32 * c0, w0, r0);
+        if (two) load_chunk(tb + 32 * c1, w1, r1);
         tmem_ld_wait();
-        if (c + 2 >= nch) {            // this warp's last chunk: the accumulator is free
+        if (c0 + 4 >= nch) {           // the batch with this warp's last chunk: the accumulator is free
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(acce_leader + static_cast<uint32_t>(acc) * 8u);
         }
-        store_chunk(g, r, width, tok0 + 32 * c, ch, ch_w, lane, buf, &tm_c32, &tm_c16);
+        store_chunk_t<1>(g, r0, w0, tok0 + 32 * c0, ch, ch_w, lane, buf0 + flip * S4_EPI_BUF, &tm_c32, &tm_c16);
+        flip ^= 1u;
+        if (two) {
+          store_chunk_t<1>(g, r1, w1, tok0 + 32 * c1, ch, ch_w, lane, buf0 + flip * S4_EPI_BUF, &tm_c32, &tm_c16);
+          flip ^= 1u;
+        }
       }
       if (grp >= nch) {                 // no chunk for this warp (bn <= 32)
         tc_fence_before();
@@ -767,9 +797,9 @@ S24Plan plan_s24_pair(int64_t M, int64_t N, int64_t K, int sm_count) {
   p.units = static_cast<int>(static_cast<long long>(p.nt) * p.tt);
   p.grid = 2 * std::min(p.units, pairs);
   const int stage = (p.bn / 2) * 128 + S4_V_BYTES + S4_M_BYTES;
-  p.np = std::min({S4_MAX_NP, (S4_SMEM_LIMIT - 1024 - S4_EPI_WARPS * S4_EPI_BUF - S4_BAR_BYTES) / stage,
+  p.np = std::min({S4_MAX_NP, (S4_SMEM_LIMIT - 1024 - 2 * S4_EPI_WARPS * S4_EPI_BUF - S4_BAR_BYTES) / stage,
                    (S4_TMEM_COLS - 2 * p.bn) / 4});
-  p.smem = 1024 + static_cast<size_t>(p.np) * stage + S4_EPI_WARPS * S4_EPI_BUF + S4_BAR_BYTES;
+  p.smem = 1024 + static_cast<size_t>(p.np) * stage + 2 * S4_EPI_WARPS * S4_EPI_BUF + S4_BAR_BYTES;
   return p;
 }
 
@@ -866,7 +896,7 @@ DQ_API dq_status dq_s24_int8_linear(const int8_t* A, const float* s_row, int64_t
   g.units = p.units;
   g.np = p.np;
   g.off_epi = static_cast<uint32_t>(p.np) * ((pair ? p.bn / 2 : p.bn) * 128 + S4_V_BYTES + S4_M_BYTES);
-  g.off_bar = g.off_epi + S4_EPI_WARPS * S4_EPI_BUF;
+  g.off_bar = g.off_epi + (pair ? 2 : 1) * S4_EPI_WARPS * S4_EPI_BUF;   // the pair: two staging buffers per warp
   g.s_row = s_row;
   g.s_col = s_col;
   g.bias = out_dtype == DQ_OUT_BF16 ? static_cast<const uint16_t*>(bias_bf16) : nullptr;
