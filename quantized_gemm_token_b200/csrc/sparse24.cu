@@ -124,21 +124,13 @@ __device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint32_t smem_a
   asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
-__device__ __forceinline__ uint32_t bf16_bits(float f) {
-  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
-}
-
-// (acc * s_row) * s_col + bias, each operation rounded on its own.
-__device__ __forceinline__ float dequant(int32_t acc, float sr, float sc, bool has_bias, float b) {
-  float f = __fmul_rn(__fmul_rn(__int2float_rn(acc), sr), sc);
-  return has_bias ? __fadd_rn(f, b) : f;
-}
-
 // Epilogue of one chunk: lane = channel ch (the warp's channels ch_w ..
 // ch_w + 31), r[j] = int32 accumulator of token tok0 + j (j < width, width
 // 16 or 32).  bf16 goes through the warp's staging buffer `buf` (free once
 // its previous store has read it) and one TMA store of the 32 x 32 block,
 // which clips tokens >= M and channels >= N; int32 is stored directly.
+// bf16: out = bf16(((float)acc * s_row) * s_col + bias), each operation
+// rounded on its own.
 // PENDING: how many of this warp's earlier stores may still be reading their
 // staging buffers (0: one buffer per warp; 1: two buffers used in turn, and
 // every chunk commits a group, an empty one when it stores nothing, so that
@@ -158,14 +150,26 @@ __device__ __forceinline__ void store_chunk_t(const S24Args& g, const uint32_t (
   const float sc = ch_ok ? __ldg(g.s_col + ch) : 0.0f;
   const bool has_bias = g.bias != nullptr;
   const float b = (has_bias && ch_ok) ? __uint_as_float(static_cast<uint32_t>(__ldg(g.bias + ch)) << 16) : 0.0f;
+  // the chunk's 32 token scales: one load per lane (lane j: token tok0 + j),
+  // then handed out by shuffles; tokens past M get 0
+  const int mj = tok0 + lane;
+  const float sr_lane = mj < g.M ? __ldg(g.s_row + mj) : 0.0f;
+  // ((float)acc * s_row) * s_col (+ bias) for the token pair (2i, 2i + 1) as
+  // f32x2, each lane rounded like the scalar operation
+  const uint64_t sc2 = pack_f2(sc, sc);
+  const uint64_t b2 = pack_f2(b, b);
   uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const int m0 = tok0 + 2 * i;
-    const float sr0 = m0 < g.M ? __ldg(g.s_row + m0) : 0.0f;
-    const float sr1 = m0 + 1 < g.M ? __ldg(g.s_row + m0 + 1) : 0.0f;
-    const float f0 = dequant(static_cast<int32_t>(r[2 * i]), sr0, sc, has_bias, b);
-    const float f1 = dequant(static_cast<int32_t>(r[2 * i + 1]), sr1, sc, has_bias, b);
+    const float sr0 = __shfl_sync(0xffffffffu, sr_lane, 2 * i);
+    const float sr1 = __shfl_sync(0xffffffffu, sr_lane, 2 * i + 1);
+    uint64_t f = mul_f2(mul_f2(pack_f2(__int2float_rn(static_cast<int32_t>(r[2 * i])),
+                                       __int2float_rn(static_cast<int32_t>(r[2 * i + 1]))),
+                               pack_f2(sr0, sr1)),
+                        sc2);
+    if (has_bias) f = add_f2(f, b2);
+    float f0, f1;
+    unpack_f2(f, f0, f1);
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(pk[i]) : "f"(f1), "f"(f0));
   }
   if (lane == 0) bulk_wait_group_read<PENDING>();
