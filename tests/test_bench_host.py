@@ -57,3 +57,33 @@ def test_stored_traffic_points_at_profiles():
                 assert bench.measured_traffic(wl, kernel) is None
             else:
                 assert bench.measured_traffic(wl, kernel) == e["bytes_per_launch"]
+
+
+def test_write_floor_is_the_slower_of_write_and_copy():
+    """_hbm_entry's floor: the output at the measured write-only rate, or all
+    bytes at the copy rate, whichever takes longer; frac_vs_floor = floor /
+    measured time."""
+    peaks = dict(hbm_gbs=6000.0, write_gbs=4000.0)
+    # write-bound: 8 GB written of 10 GB -> 2 ms at 4 TB/s beats 10/6 ms
+    e = bench._hbm_entry("k", 4.0, 10e9, peaks, write_bytes=8e9)
+    assert abs(e["floor_ms"] - 2.0) < 1e-9 and abs(e["frac_vs_floor"] - 0.5) < 1e-9
+    # copy-bound: 1 GB written of 12 GB -> 2 ms at 6 TB/s beats 0.25 ms
+    e = bench._hbm_entry("k", 2.5, 12e9, peaks, write_bytes=1e9)
+    assert abs(e["floor_ms"] - 2.0) < 1e-9 and abs(e["frac_vs_floor"] - 0.8) < 1e-9
+    # no write bytes, or no measured write rate: no floor reported
+    assert "floor_ms" not in bench._hbm_entry("k", 1.0, 1e9, peaks)
+    assert "floor_ms" not in bench._hbm_entry("k", 1.0, 1e9, dict(hbm_gbs=6000.0), write_bytes=1e9)
+
+
+def test_output_heavy_workloads_declare_their_writes():
+    """The workloads whose bytes are mostly output carry their write bytes,
+    so their roofline reports the write floor."""
+    for name in ("quant", "large_m_s32", "vit_fc1"):
+        wl = bench.WORKLOADS[name]
+        d = {}
+        if wl["kind"] == "bsr":
+            import synth
+            crow, _ = synth.bsr_pattern(5120 // 64, 1280 // 64, 0.10, 3)
+            d = dict(M=65792, K=1280, N=5120, crow=crow)
+        _, dom = bench.step_accounting(wl, d)
+        assert 0 < dom["write_bytes"] < dom["bytes"]
