@@ -37,6 +37,10 @@
 //            zeros.  The panel variant keeps a 128-row block's activations in
 //            shared memory and streams only weight blocks.
 //
+// Many tokens (from 1536 with K >= 2048, and any K >= 8192) take the 2-SM
+// pair kernel of gemm2sm.cu instead (int8 and e4m3); the 1-SM kernel keeps
+// the rest and every BSR and swap call.
+//
 // Schedules: whole tiles round-robin over one CTA per SM (contiguous tile
 // ranges for the BSR panel variant), or, for the swap arrangement when whole
 // tiles would leave SMs idle, stream-K: the tile x k-block iteration space is
