@@ -66,10 +66,12 @@ KERNEL_SOURCES = {
 
 def _strip_comments(text: str) -> str:
     """C/C++ source without its comments (string literals in these sources
-    hold no comment markers), so that a comment edit keeps the hash."""
+    hold no comment markers) and with every run of whitespace made one space,
+    so that an edit of comments or layout keeps the hash."""
     import re
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return re.sub(r"//[^\n]*", "", text)
+    text = re.sub(r"//[^\n]*", "", text)
+    return re.sub(r"\s+", " ", text).strip()
 
 
 def kernel_source_hash(kernel: str) -> str:
