@@ -157,6 +157,10 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
 struct MetaFwd {
   uint32_t s, z;
 };
+// Forward with two 64-deep sub-tiles per step: one (s, z) per sub-tile.
+struct MetaFwd2 {
+  MetaFwd m[2];
+};
 struct MetaT {
   uint4 s8[2], z8[2];
 };
@@ -180,7 +184,7 @@ __device__ __forceinline__ void ldg_v4_or0(uint4& v, const uint16_t* p, bool pre
 __device__ __forceinline__ void load_meta_fwd(const HqqArgs& g, int dt, bool valid, int ntile, int kstep,
                                               MetaFwd& m) {
   const int n = ntile * 128 + (dt & 127);
-  const int k = kstep * HQ_BK + (dt >> 7) * 32;
+  const int k = kstep * HQ_BK + (dt >> 7) * 32;   // kstep: 64-deep sub-tile index
   const bool in = valid && n < g.n_w && k < g.k_w;
   const int64_t gi = in ? static_cast<int64_t>(k >> g.group_log2) * g.n_w + n : 0;
   ldg_u16_or0(m.s, g.scale + gi, in);
@@ -208,10 +212,11 @@ __device__ __forceinline__ void load_meta_t(const HqqArgs& g, int dt, bool valid
 // codes) into the 128 x 64 bf16 A tile (thread t: row t % 128, codes
 // 32 * (t / 128) .. +31).
 template <bool S4>
-__device__ __forceinline__ void dequant_tile_fwd(uint32_t atile, uint32_t wtile, int dt, const MetaFwd& m) {
+__device__ __forceinline__ void dequant_tile_fwd(uint32_t atile, uint32_t wtile, int dt, const MetaFwd& m,
+                                                 int wrow = 32) {
   const int r = dt & 127;
   const int h = dt >> 7;
-  const uint4 pk = pipe::lds128(wtile + r * 32 + h * 16);
+  const uint4 pk = pipe::lds128(wtile + r * wrow + h * 16);
   const uint32_t s2 = m.s | (m.s << 16);
   const uint32_t z2 = m.z | (m.z << 16);
   const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
@@ -313,7 +318,9 @@ __device__ __forceinline__ void stage_pairs(uint32_t buf, const uint32_t (&r)[32
   pipe::stage_bf16_pairs(buf, pk, width, lane);
 }
 
-template <bool TRANS, bool S4>
+// SUB: 64-deep sub-tiles per contraction step (forward, few tokens: 2, so
+// that each copy, barrier and hand-off serves 128 in-features; else 1).
+template <bool TRANS, bool S4, int SUB = 1>
 __global__ void __launch_bounds__(HQ_THREADS, 1)
     hqq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_c32, const __grid_constant__ CUtensorMap tm_c16,
@@ -322,10 +329,13 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* const smem = smem_raw + (base - raw);
-  // stage s at base + s * stage_bytes: dequantized A tile (16 KB), then the
-  // activation tile (bn x 128 B), then the packed weight tile and its meta
-  const uint32_t x_bytes = static_cast<uint32_t>(g.bn) * 128u;
-  const uint32_t stage_bytes = HQ_A_BYTES + x_bytes + HQ_W_BYTES;
+  // stage s at base + s * stage_bytes: SUB dequantized A tiles (16 KB each),
+  // then SUB activation tiles (bn x 128 B each), then the packed weight tile
+  // (128 rows x 32 SUB bytes forward)
+  static_assert(SUB == 1 || (SUB == 2 && !TRANS), "two sub-tiles per step: forward only");
+  const uint32_t x_sub = static_cast<uint32_t>(g.bn) * 128u;
+  const uint32_t x_bytes = x_sub * SUB;
+  const uint32_t stage_bytes = HQ_A_BYTES * SUB + x_bytes + HQ_W_BYTES * SUB;
   uint64_t* const full = reinterpret_cast<uint64_t*>(smem + g.off_bar);   // TMA landed
   uint64_t* const deq = full + HQ_MAX_NP;                                 // A tile written
   uint64_t* const empty = deq + HQ_MAX_NP;                                // MMAs done with the stage
@@ -380,14 +390,16 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
             break;
           }
           const uint32_t fb = smem_u32(full + stage);
-          const uint32_t sx = base + stage * stage_bytes + HQ_A_BYTES;
+          const uint32_t sx = base + stage * stage_bytes + HQ_A_BYTES * SUB;
           const uint32_t sw = sx + x_bytes;
-          mbar_arrive_expect_tx(fb, x_bytes + HQ_W_BYTES);
-          tma_load_2d(sx, &tm_x, fb, kk * 128, t.ttile * g.bn);
+          mbar_arrive_expect_tx(fb, x_bytes + HQ_W_BYTES * SUB);
+#pragma unroll
+          for (int sb = 0; sb < SUB; ++sb)
+            tma_load_2d(sx + sb * x_sub, &tm_x, fb, (kk * SUB + sb) * 128, t.ttile * g.bn);
           if (TRANS)
             tma_load_2d(sw, &tm_w, fb, t.ntile * 64, kk * HQ_BK);
           else
-            tma_load_2d(sw, &tm_w, fb, kk * 32, t.ntile * 128);
+            tma_load_2d(sw, &tm_w, fb, kk * 32 * SUB, t.ntile * 128);
           ++issued;
           if (++stage == g.np) {
             stage = 0;
@@ -422,11 +434,14 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
           }
           tc_fence_after();
           const uint32_t sa = base + stage * stage_bytes;
-          const uint64_t ad = smem_desc_kmajor<128>(sa);
-          const uint64_t bd = smem_desc_kmajor<128>(sa + HQ_A_BYTES);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)   // K = 16 bf16 = 32 bytes per instruction
-            mma_bf16(d_tmem, ad + 2 * j, bd + 2 * j, idesc, (kk > t.k0 || j > 0) ? 1u : 0u);
+          for (int sb = 0; sb < SUB; ++sb) {
+            const uint64_t ad = smem_desc_kmajor<128>(sa + sb * HQ_A_BYTES);
+            const uint64_t bd = smem_desc_kmajor<128>(sa + HQ_A_BYTES * SUB + sb * x_sub);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)   // K = 16 bf16 = 32 bytes per instruction
+              mma_bf16(d_tmem, ad + 2 * j, bd + 2 * j, idesc, (kk > t.k0 || sb > 0 || j > 0) ? 1u : 0u);
+          }
           mma_commit(smem_u32(empty + stage));
           if (++stage == g.np) {
             stage = 0;
@@ -450,14 +465,18 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
     // A stage's A tile is free again once its copies have landed: the
     // producer refilled the stage only after the MMAs that read it completed.
     // Each thread's scales and zero points are loaded two steps ahead of use.
-    using Meta = typename std::conditional<TRANS, MetaT, MetaFwd>::type;
+    using Meta = typename std::conditional<TRANS, MetaT, typename std::conditional<SUB == 2, MetaFwd2, MetaFwd>::type>::type;
     const int dt = (threadIdx.x - 64) & 255;
     const int grp = (threadIdx.x - 64) >> 8;     // group 1 takes the odd steps
     auto load_meta = [&](const StepIt& s, Meta& m) {
-      if constexpr (TRANS)
+      if constexpr (TRANS) {
         load_meta_t(g, dt, s.valid, s.ntile, s.kk, m);
-      else
+      } else if constexpr (SUB == 2) {
+        load_meta_fwd(g, dt, s.valid, s.ntile, 2 * s.kk, m.m[0]);
+        load_meta_fwd(g, dt, s.valid, s.ntile, 2 * s.kk + 1, m.m[1]);
+      } else {
         load_meta_fwd(g, dt, s.valid, s.ntile, s.kk, m);
+      }
     };
     // cur: this group's step; ahead: the group's step two of its own later
     StepIt cur, ahead;
@@ -481,11 +500,15 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
       const bool w = pipe::wait(smem_u32(full + stage), phase, g.wait, abort_flag);
       if (!__all_sync(0xffffffffu, w)) return false;
       const uint32_t sa = base + stage * stage_bytes;
-      const uint32_t wt = sa + HQ_A_BYTES + x_bytes;
-      if constexpr (TRANS)
+      const uint32_t wt = sa + HQ_A_BYTES * SUB + x_bytes;
+      if constexpr (TRANS) {
         dequant_tile_t<S4>(sa, wt, dt, use);
-      else
+      } else if constexpr (SUB == 2) {
+        dequant_tile_fwd<S4>(sa, wt, dt, use.m[0], 64);
+        dequant_tile_fwd<S4>(sa + HQ_A_BYTES, wt + 32, dt, use.m[1], 64);
+      } else {
         dequant_tile_fwd<S4>(sa, wt, dt, use);
+      }
       fence_proxy_async_smem();     // generic-proxy writes -> visible to the MMA
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(deq + stage));
@@ -690,10 +713,10 @@ constexpr int HQ_MAX_SPLITS = 8;           // portable cluster size
 // the SMs the contraction is split over a cluster of up to 8 CTAs (at least
 // 4 steps of 64 per split; the partial tile, bn x 128 fp32, must fit in the
 // stage ring).
-HqqPlan plan_hqq(int64_t M, int64_t n_out, int64_t kc, int sm_count, bool allow_split) {
+HqqPlan plan_hqq(int64_t M, int64_t n_out, int64_t kc, int sm_count, bool allow_split, int sub = 1) {
   HqqPlan p{};
   p.nt = static_cast<int>((n_out + 127) / 128);
-  p.ks = static_cast<int>((kc + HQ_BK - 1) / HQ_BK);
+  p.ks = static_cast<int>((kc + HQ_BK * sub - 1) / (HQ_BK * sub));
   p.tt = static_cast<int>((M + 255) / 256);
   const int64_t per = (M + p.tt - 1) / p.tt;
   p.bn = static_cast<int>(std::max<int64_t>(16, (per + 15) / 16 * 16));
@@ -706,7 +729,7 @@ HqqPlan plan_hqq(int64_t M, int64_t n_out, int64_t kc, int sm_count, bool allow_
   }
   p.units = static_cast<int>(tiles * p.splits);
   p.grid = std::min(p.units, sm_count);
-  const int stage = HQ_A_BYTES + p.bn * 128 + HQ_W_BYTES;
+  const int stage = (HQ_A_BYTES + p.bn * 128 + HQ_W_BYTES) * sub;
   const int avail = HQ_SMEM_LIMIT - 1024 - 2 * HQ_EPI_WARPS * HQ_EPI_BUF - HQ_BAR_BYTES;
   p.np = std::min(HQ_MAX_NP, avail / stage);
   p.smem = 1024 + static_cast<size_t>(p.np) * stage + 2 * HQ_EPI_WARPS * HQ_EPI_BUF + HQ_BAR_BYTES;
@@ -730,10 +753,11 @@ dq_status check_weights(const uint8_t* packed, const void* scale, const void* ze
   return DQ_OK;
 }
 
-template <bool TRANS, bool S4>
+template <bool TRANS, bool S4, int SUB = 1>
 dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& tc32, const CUtensorMap& tc16,
                      const HqqArgs& g, int grid, size_t smem, cudaStream_t stream) {
-  const dq_status st = smem_limit_once(reinterpret_cast<const void*>(&hqq_gemm_kernel<TRANS, S4>), HQ_SMEM_LIMIT);
+  const dq_status st =
+      smem_limit_once(reinterpret_cast<const void*>(&hqq_gemm_kernel<TRANS, S4, SUB>), HQ_SMEM_LIMIT);
   if (st != DQ_OK) return st;
   // Programmatic stream serialization: the prologue (barriers, tensor-memory
   // allocation) overlaps the tail of the previous kernel of the stream.  A
@@ -752,7 +776,7 @@ dq_status launch_hqq(const CUtensorMap& tx, const CUtensorMap& tw, const CUtenso
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = g.splits > 1 ? 2 : 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, hqq_gemm_kernel<TRANS, S4>, tx, tw, tc32, tc16, g);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, hqq_gemm_kernel<TRANS, S4, SUB>, tx, tw, tc32, tc16, g);
   return e == cudaSuccess ? DQ_OK : cuda_fail(e);
 }
 
@@ -803,7 +827,10 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   const int64_t kc = trans ? N : K;
   (void)workspace;          // kept for the interface: the split contraction needs none
   (void)workspace_bytes;
-  const HqqPlan p = plan_hqq(M, n_out, kc, d->sm_count, split_clusters_fit(*d));
+  // Few tokens (forward): 128-deep steps of two 64-deep sub-tiles, half the
+  // copies, barrier waits and hand-offs per in-feature.
+  const int sub = (!trans && M <= 64) ? 2 : 1;
+  const HqqPlan p = plan_hqq(M, n_out, kc, d->sm_count, split_clusters_fit(*d), sub);
 
   CUtensorMap tx, tw;
   // activations / output gradient: bf16 [M, kc] as bytes, 64-element k
@@ -814,7 +841,7 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   // packed codes [N, K/2]: forward 128 channels x 32 B (64 k); transposed
   // 64 weight rows x 64 B (128 output channels k)
   st = make_tmap_u8_2d(&tw, packed, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N),
-                       static_cast<uint64_t>(K / 2), trans ? 64 : 32, trans ? 64 : 128, 0);
+                       static_cast<uint64_t>(K / 2), trans ? 64 : 32 * sub, trans ? 64 : 128, 0);
   if (st != DQ_OK) return st;
 
   // output bf16 [M, n_out] as bytes: 32 channels (64 B) x 32 or 16 tokens
@@ -840,7 +867,7 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   g.ks = p.ks;
   g.units = p.units;
   g.np = p.np;
-  g.off_epi = static_cast<uint32_t>(p.np) * (HQ_A_BYTES + p.bn * 128 + HQ_W_BYTES);
+  g.off_epi = static_cast<uint32_t>(p.np) * (HQ_A_BYTES + p.bn * 128 + HQ_W_BYTES) * sub;
   g.off_bar = g.off_epi + 2 * HQ_EPI_WARPS * HQ_EPI_BUF;
   g.scale = static_cast<const uint16_t*>(scale);
   g.zero = static_cast<const uint16_t*>(zero);
@@ -850,6 +877,9 @@ dq_status hqq_linear_impl(bool trans, const void* x, int64_t M, const uint8_t* p
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (trans) return s4 ? launch_hqq<true, true>(tx, tw, tc32, tc16, g, p.grid, p.smem, s)
                        : launch_hqq<true, false>(tx, tw, tc32, tc16, g, p.grid, p.smem, s);
+  if (sub == 2)
+    return s4 ? launch_hqq<false, true, 2>(tx, tw, tc32, tc16, g, p.grid, p.smem, s)
+              : launch_hqq<false, false, 2>(tx, tw, tc32, tc16, g, p.grid, p.smem, s);
   return s4 ? launch_hqq<false, true>(tx, tw, tc32, tc16, g, p.grid, p.smem, s)
             : launch_hqq<false, false>(tx, tw, tc32, tc16, g, p.grid, p.smem, s);
 }
