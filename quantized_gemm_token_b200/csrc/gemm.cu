@@ -18,6 +18,8 @@
 //               bf16, stage 32x32 blocks in shared memory and TMA-store them.
 //               Accumulators are multi-buffered in TMEM so the epilogue of
 //               tile i overlaps the MMAs of tile i+1.
+//   last warp   streaming BSR only (warp 10): a second producer that issues the weight
+//               block copies while warp 0 issues the activation slices.
 //
 // Operand arrangements sharing it:
 //   Dense    A slot = 128 activation rows, B slot = BN weight channels
@@ -144,7 +146,13 @@ struct Cfg {
   static constexpr int K_STEPS = KB / 32;                     // MMA K = 32 bytes
   static constexpr int CW = BN >= 32 ? 32 : 16;               // epilogue chunk (columns)
   static constexpr int SMEM_BYTES = layout_bytes(STAGES, SC_SLOTS);
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  // Streaming BSR stages carry a small activation slice and a small weight
+  // block, so issuing their tensor copies bounds the K-heavy shapes (each
+  // copy holds its issuing thread a few hundred cycles): there the two copies
+  // of a stage come from two threads, warp 0 and one warp after the epilogue
+  // warps.  Every other kind issues both from warp 0.
+  static constexpr int NPROD = BSR && !PANEL ? 2 : 1;
+  static constexpr int THREADS = 32 + 32 * NPROD + 32 * EPI_WARPS;
   static constexpr int NBARS = 2 * STAGES + 2 * ACC_BUFS + 3 + 2 * SC_SLOTS;
   static_assert(NBARS * 8 + 16 + (PANEL ? 4 * STAGES : 0) <= BAR_BYTES, "barrier area");
   static_assert(OFF_ZB + ZB_BYTES <= OFF_OUT, "layout");
@@ -256,8 +264,15 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp == 0) {
+  if (warp == 0 || warp >= 2 + C::EPI_WARPS) {
     // ------------------------------------------------------------ producer
+    // Warp 0 arms each stage's barrier with the stage's bytes and issues the
+    // A copies; with two producers the other one issues the B copies (its
+    // copies may land before the barrier is armed: the transaction count
+    // then runs below zero until the arming, and the phase cannot complete
+    // before that arrival).
+    const bool a_side = warp == 0;
+    const bool b_side = C::NPROD == 1 || warp != 0;
     if (lane == 0) {
       SegIter iter(g);
       Seg s;
@@ -308,7 +323,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
           }
           const uint32_t fb = smem_u32(full_bar + stage);
           if constexpr (PANEL) stage_col[stage] = c_cur;
-          mbar_arrive_expect_tx(fb, stage_tx);
+          if (a_side) mbar_arrive_expect_tx(fb, stage_tx);
           const uint32_t da = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t db = smem_u32(sB + stage * C::B_BYTES);
           if constexpr (PANEL) {
@@ -317,10 +332,12 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
           } else if constexpr (C::BSR) {
             // A: the KB-wide k slice holding block column c (for 16-wide
             // blocks the 32-byte slice that contains it); B: block kb
-            const int c = idx ? idx[g.nbr + 1 + kb] : __ldg(g.col + kb);
-            const int ax = KIND == Kind::Bsr16 ? (c >> 1) * 32 : c * C::BS;
-            tma_load_2d(da, &tm_a, fb, ax, ta * 128);
-            tma_load_2d(db, &tm_b, fb, 0, kb * C::BS);
+            if (a_side) {
+              const int c = idx ? idx[g.nbr + 1 + kb] : __ldg(g.col + kb);
+              const int ax = KIND == Kind::Bsr16 ? (c >> 1) * 32 : c * C::BS;
+              tma_load_2d(da, &tm_a, fb, ax, ta * 128);
+            }
+            if (b_side) tma_load_2d(db, &tm_b, fb, 0, kb * C::BS);
           } else {
             tma_load_2d(da, &tm_a, fb, kb * C::KB, ta * 128);
             tma_load_2d(db, geo.narrow ? &tm_b2 : &tm_b, fb, kb * C::KB, geo.n0);
@@ -333,7 +350,13 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
         }
         }
       }
-      if (!ok) {
+      if (!ok && !a_side) {
+        // the B producer: its copies land on barriers warp 0 drains (below);
+        // a fixed 100 us covers the ones whose stage was never armed
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 100000ull) {
+        }
+      } else if (!ok) {
         // Let the (at most STAGES) most recent loads land before the CTA
         // leaves; each wait is bounded by a short limit.
         WaitCtl quick = g.wait;
@@ -448,7 +471,7 @@ __global__ void __launch_bounds__(Cfg<KIND, BN, PANEL>::THREADS, 1)
       volatile int never = 0;
       mbar_wait(smem_u32(drain_bar), 0, g.wait, &never);
     }
-  } else {
+  } else if (warp < 2 + C::EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     // EPI_WARPS warps; warp w reads TMEM sub-partition w % 4 (rows 32*(w%4) ..
     // +31) and, with EPI_WARPS == 8, the two warps of a sub-partition take
