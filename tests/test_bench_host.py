@@ -87,3 +87,17 @@ def test_output_heavy_workloads_declare_their_writes():
             d = dict(M=65792, K=1280, N=5120, crow=crow)
         _, dom = bench.step_accounting(wl, d)
         assert 0 < dom["write_bytes"] < dom["bytes"]
+
+
+def test_profile_summaries_give_their_command():
+    """Every ncu summary under profiles/ states the command that made it, with
+    the clocks left alone, and runs committed files only (bench.py)."""
+    pdir = os.path.join(ROOT, "profiles")
+    names = sorted(f for f in os.listdir(pdir) if f.endswith(".md"))
+    assert names
+    for f in names:
+        with open(os.path.join(pdir, f), encoding="utf-8") as fh:
+            text = fh.read()
+        assert "ncu " in text and "--clock-control none" in text, f
+        assert "bench.py" in text, f
+        assert "_work/" not in text, f
